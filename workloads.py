@@ -1,0 +1,176 @@
+"""Seeded synthetic inputs for the gated delta-rule prefill and decode paths.
+
+This module is shared by the tests, ``bench.py`` and ``__graft_entry__.smoke``.
+It only draws and shapes random inputs; it holds none of the recurrence's
+arithmetic.  The distributions follow the layer the pages describe:
+
+* the Qwen2.5-0.5B KDA graft ("kda-graft", section "Идея и архитектура"):
+  14 heads of dimension 64, an alpha gate initialised with bias +5 so that
+  sigmoid(5) ~ 0.993, and an fp32 recurrent state;
+* the Gated DeltaNet hybrids ("Modele hybrydowe: co Gated DeltaNet zastępuje
+  w cache KV", sections "Atencja liniowa" and "Gated DeltaNet: dodaj zanik"):
+  head dimension 128 and contexts up to 262K tokens.
+
+Every tensor is drawn in fp32 from a CPU (or CUDA) ``torch.Generator`` seeded
+per workload, normalised where stated, then cast once to the compute dtype.
+Both sides of a parity test receive exactly those bits.
+
+Layouts (token-major, packed over sequences by ``cu_seqlens``):
+  q, k     [T_tot, H, d_k]     v        [T_tot, H, d_v]
+  beta     [T_tot, H] fp32     log_a    [T_tot, H, d_k] or [T_tot, H] (scalar gate)
+  state    [N, H, d_v, d_k] fp32 (row = value channel, column = key channel)
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field, replace
+from typing import Optional
+
+import torch
+
+
+@dataclass(frozen=True)
+class PrefillWorkload:
+    name: str
+    seed: int
+    n_heads: int
+    d_k: int
+    d_v: int
+    lengths: Optional[tuple] = None      # fixed lengths; None -> drawn (varlen)
+    n_seqs: int = 1
+    len_range: Optional[tuple] = None    # inclusive uniform range for varlen
+    qkv_dtype: torch.dtype = torch.bfloat16
+    scalar_decay: bool = False
+    log_a_mu: float = 5.0                # log_a = logsigmoid(N(mu, sd))
+    log_a_sd: float = 1.0
+    log_a_clamp: Optional[tuple] = None  # (lo, hi) applied after logsigmoid
+    init_std: float = 0.0                # 0 -> zero initial state
+    snap_interval: int = 0
+    scale: float = 1.0
+
+
+@dataclass(frozen=True)
+class DecodeWorkload:
+    name: str
+    seed: int
+    batch: int
+    n_heads: int
+    d_k: int
+    d_v: int
+    steps: int
+    qkv_dtype: torch.dtype = torch.bfloat16
+    scalar_decay: bool = False
+    log_a_mu: float = 5.0
+    log_a_sd: float = 1.0
+    init_std: float = 0.1
+    scale: float = 1.0
+
+
+# The five workloads the method is measured on.  Seeds are 1000 + index.
+TINY_KDA = PrefillWorkload("tiny_kda_H2_T256_d64_f32", 1001, 2, 64, 64,
+                           lengths=(256,), qkv_dtype=torch.float32)
+GRAFT_LAYER = PrefillWorkload("graft_layer_H14_T8192_d64_bf16", 1002, 14, 64, 64,
+                              lengths=(8192,))
+DECODE = DecodeWorkload("decode_B256_H14_d64_1024steps", 1003, 256, 14, 64, 64, 1024)
+GDN_LONG = PrefillWorkload("gdn_long_H16_T65536_d128_scalar_snap4096", 1004, 16, 128, 128,
+                           lengths=(65536,), scalar_decay=True, log_a_mu=4.0,
+                           log_a_sd=1.5, snap_interval=4096)
+VARLEN = PrefillWorkload("varlen_N32_H32_d128_L1024to16384", 1005, 32, 128, 128,
+                         n_seqs=32, len_range=(1024, 16384), log_a_mu=3.0,
+                         log_a_sd=2.0, log_a_clamp=(-5.0, 0.0), init_std=0.1)
+
+PREFILL_WORKLOADS = {w.name: w for w in (TINY_KDA, GRAFT_LAYER, GDN_LONG, VARLEN)}
+
+
+def shrink(w: PrefillWorkload, **kw) -> PrefillWorkload:
+    """Same distributions, other sizes (for fast parity cases)."""
+    return replace(w, **kw)
+
+
+def _l2norm(x: torch.Tensor) -> torch.Tensor:
+    # Per (token, head) normalisation in fp32; Gaussian rows never vanish.
+    return x / x.norm(dim=-1, keepdim=True)
+
+
+def _draw_lengths(w: PrefillWorkload, gen: torch.Generator) -> list:
+    if w.lengths is not None:
+        return list(w.lengths)
+    lo, hi = w.len_range
+    return torch.randint(lo, hi + 1, (w.n_seqs,), generator=gen).tolist()
+
+
+def cu_seqlens_of(lengths) -> torch.Tensor:
+    cu = [0]
+    for n in lengths:
+        cu.append(cu[-1] + int(n))
+    return torch.tensor(cu, dtype=torch.int32)
+
+
+def make_prefill_inputs(w: PrefillWorkload, device="cpu", lengths=None,
+                        draw_device=None) -> dict:
+    """Draw one batch of prefill inputs.
+
+    ``draw_device`` selects where the random numbers are drawn ("cpu" by
+    default: bit-identical on every machine; "cuda" for multi-GB workloads).
+    The result lives on ``device``.
+    """
+    draw_device = draw_device or "cpu"
+    gen = torch.Generator(device=draw_device)
+    gen.manual_seed(w.seed)
+    if lengths is None:
+        # lengths always come from a CPU generator so they never depend on device
+        lgen = torch.Generator().manual_seed(w.seed)
+        lengths = _draw_lengths(w, lgen)
+    lengths = [int(n) for n in lengths]
+    T = sum(lengths)
+    H, dk, dv = w.n_heads, w.d_k, w.d_v
+    f32 = dict(dtype=torch.float32, device=draw_device, generator=gen)
+    q = _l2norm(torch.randn(T, H, dk, **f32)).to(w.qkv_dtype)
+    k = _l2norm(torch.randn(T, H, dk, **f32)).to(w.qkv_dtype)
+    v = torch.randn(T, H, dv, **f32).to(w.qkv_dtype)
+    beta = torch.sigmoid(torch.randn(T, H, **f32))
+    la_shape = (T, H) if w.scalar_decay else (T, H, dk)
+    log_a = torch.nn.functional.logsigmoid(w.log_a_mu + w.log_a_sd * torch.randn(la_shape, **f32))
+    if w.log_a_clamp is not None:
+        log_a = log_a.clamp(*w.log_a_clamp)
+    n = len(lengths)
+    if w.init_std > 0:
+        init = w.init_std * torch.randn(n, H, dv, dk, **f32)
+    else:
+        init = None
+    out = dict(q=q, k=k, v=v, beta=beta.contiguous(), log_a=log_a.contiguous(),
+               init_state=init, cu_seqlens=cu_seqlens_of(lengths), lengths=lengths,
+               scalar_decay=w.scalar_decay, scale=w.scale, snap_interval=w.snap_interval)
+    dev = torch.device(device)
+    for key in ("q", "k", "v", "beta", "log_a", "init_state", "cu_seqlens"):
+        if out[key] is not None:
+            out[key] = out[key].to(dev).contiguous()
+    return out
+
+
+def make_decode_inputs(w: DecodeWorkload, steps: Optional[int] = None, device="cpu",
+                       draw_device=None) -> dict:
+    """Initial state plus ``steps`` fresh single-token inputs per sequence/head.
+
+    Per-step tensors carry a leading step axis: q, k [S, B, H, d_k],
+    v [S, B, H, d_v], beta [S, B, H], log_a [S, B, H, d_k] (or [S, B, H]).
+    """
+    steps = w.steps if steps is None else steps
+    draw_device = draw_device or "cpu"
+    gen = torch.Generator(device=draw_device)
+    gen.manual_seed(w.seed)
+    B, H, dk, dv = w.batch, w.n_heads, w.d_k, w.d_v
+    f32 = dict(dtype=torch.float32, device=draw_device, generator=gen)
+    state = w.init_std * torch.randn(B, H, dv, dk, **f32)
+    q = _l2norm(torch.randn(steps, B, H, dk, **f32)).to(w.qkv_dtype)
+    k = _l2norm(torch.randn(steps, B, H, dk, **f32)).to(w.qkv_dtype)
+    v = torch.randn(steps, B, H, dv, **f32).to(w.qkv_dtype)
+    beta = torch.sigmoid(torch.randn(steps, B, H, **f32))
+    la_shape = (steps, B, H) if w.scalar_decay else (steps, B, H, dk)
+    log_a = torch.nn.functional.logsigmoid(w.log_a_mu + w.log_a_sd * torch.randn(la_shape, **f32))
+    out = dict(state=state, q=q, k=k, v=v, beta=beta, log_a=log_a,
+               scalar_decay=w.scalar_decay, scale=w.scale)
+    dev = torch.device(device)
+    for key in ("state", "q", "k", "v", "beta", "log_a"):
+        out[key] = out[key].to(dev).contiguous()
+    return out
+
