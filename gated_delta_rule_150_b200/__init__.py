@@ -1,0 +1,259 @@
+"""Gated delta-rule prefill and decode on B200 (sm_100a).
+
+A thin ctypes binding over the C ABI in ``include/gdr.h``.  Every function
+here only checks and marshals torch tensors (device pointers, sizes and the
+current CUDA stream) into one library call; all arithmetic runs in the CUDA
+kernels of ``libgdr.so``.  There is no CPU or PyTorch fallback: if the
+library is missing, every call raises.
+
+Layouts (token-major, sequences packed by ``cu_seqlens``):
+  q, k [T, H, d_k]   v, o [T, H, d_v]   beta [T, H] fp32
+  log_a [T, H, d_k] fp32 (per-channel decay) or [T, H] (scalar decay)
+  state [N, H, d_v, d_k] fp32, row = value channel, column = key channel
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+__all__ = ["prefill", "decode_step", "cumdecay", "chunk_factors", "workspace_size",
+           "snapshot_count", "prefill_status", "lib", "GdrError", "LIB_PATH"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_build", "libgdr.so")
+
+GDR_OK = 0
+_STATUS = {0: "GDR_OK", 1: "GDR_ERR_INVALID_ARG", 2: "GDR_ERR_UNSUPPORTED",
+           3: "GDR_ERR_WORKSPACE", 4: "GDR_ERR_CUDA", 5: "GDR_ERR_TIMEOUT"}
+GDR_BF16, GDR_F32 = 0, 1
+
+
+class GdrError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {_STATUS.get(status, status)}")
+
+
+class PrefillArgs(ctypes.Structure):
+    """Mirror of ``gdr_prefill_args`` (include/gdr.h)."""
+    _fields_ = [
+        ("n_seqs", ctypes.c_int), ("n_heads", ctypes.c_int), ("d_k", ctypes.c_int),
+        ("d_v", ctypes.c_int), ("total_tokens", ctypes.c_int64),
+        ("cu_seqlens", ctypes.c_void_p), ("qkv_dtype", ctypes.c_int),
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("beta", ctypes.c_void_p), ("log_a", ctypes.c_void_p), ("scalar_decay", ctypes.c_int),
+        ("scale", ctypes.c_float), ("init_state", ctypes.c_void_p), ("o", ctypes.c_void_p),
+        ("final_state", ctypes.c_void_p), ("snap_interval", ctypes.c_int),
+        ("snapshots", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
+        ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
+_LOCK = threading.Lock()
+_LIB = None
+
+
+def lib():
+    """Load libgdr.so (raises if it has not been built)."""
+    global _LIB
+    with _LOCK:
+        if _LIB is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"CUDA library not built: {LIB_PATH} is missing "
+                                   "(run python -m gated_delta_rule_150_b200.build)")
+            L = ctypes.CDLL(LIB_PATH)
+            vp, i, i64, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
+            L.gdr_status_string.restype = ctypes.c_char_p
+            L.gdr_status_string.argtypes = [i]
+            L.gdr_version.restype = i
+            L.gdr_prefill_workspace_size.restype = ctypes.c_size_t
+            L.gdr_prefill_workspace_size.argtypes = [i, i, i, i, i64, i]
+            L.gdr_snapshot_count.restype = i64
+            L.gdr_snapshot_count.argtypes = [vp, i, i]
+            L.gdr_prefill.restype = i
+            L.gdr_prefill.argtypes = [ctypes.POINTER(PrefillArgs), vp]
+            L.gdr_prefill_status.restype = i
+            L.gdr_prefill_status.argtypes = [vp, vp]
+            L.gdr_cumdecay.restype = i
+            L.gdr_cumdecay.argtypes = [i, i, i, i64, vp, vp, i, vp, vp]
+            L.gdr_chunk_factors.restype = i
+            L.gdr_chunk_factors.argtypes = [ctypes.POINTER(PrefillArgs), vp, vp, vp, vp, vp, vp, vp]
+            L.gdr_decode_step.restype = i
+            L.gdr_decode_step.argtypes = [i, i, i, i, i, vp, vp, vp, vp, vp, i, f, vp, vp, vp]
+            _LIB = L
+        return _LIB
+
+
+def _check(status: int, what: str):
+    if status != GDR_OK:
+        raise GdrError(status, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return GDR_BF16
+    if t.dtype == torch.float32:
+        return GDR_F32
+    raise TypeError(f"q/k/v must be bfloat16 or float32, got {t.dtype}")
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None:
+            if not t.is_cuda:
+                raise ValueError("all tensors must be CUDA tensors")
+            if not t.is_contiguous():
+                raise ValueError("all tensors must be contiguous")
+
+
+def _host_cu(cu_seqlens, cu_seqlens_host):
+    if cu_seqlens_host is not None:
+        return torch.as_tensor(cu_seqlens_host, dtype=torch.int32).contiguous()
+    return cu_seqlens.detach().to("cpu", torch.int32).contiguous()
+
+
+def workspace_size(n_seqs, n_heads, d_k, d_v, total_tokens, scalar_decay=False) -> int:
+    return int(lib().gdr_prefill_workspace_size(n_seqs, n_heads, d_k, d_v, total_tokens,
+                                                int(bool(scalar_decay))))
+
+
+def snapshot_count(cu_seqlens_host, snap_interval: int) -> int:
+    cu = torch.as_tensor(cu_seqlens_host, dtype=torch.int32).contiguous()
+    n = int(lib().gdr_snapshot_count(ctypes.c_void_p(cu.data_ptr()), cu.numel() - 1,
+                                     int(snap_interval)))
+    if n < 0:
+        raise GdrError(1, "gdr_snapshot_count")
+    return n
+
+
+def _prefill_args(q, k, v, beta, log_a, cu_seqlens, scalar_decay, scale, init_state,
+                  snap_interval, o, final_state, snapshots, workspace):
+    T, H, dk = q.shape
+    a = PrefillArgs()
+    a.n_seqs = cu_seqlens.numel() - 1
+    a.n_heads = H
+    a.d_k = dk
+    a.d_v = v.shape[-1]
+    a.total_tokens = T
+    a.cu_seqlens = cu_seqlens.data_ptr()
+    a.qkv_dtype = _dtype_code(q)
+    a.q, a.k, a.v = q.data_ptr(), k.data_ptr(), v.data_ptr()
+    a.beta, a.log_a = beta.data_ptr(), log_a.data_ptr()
+    a.scalar_decay = int(bool(scalar_decay))
+    a.scale = float(scale)
+    a.init_state = None if init_state is None else init_state.data_ptr()
+    a.o = None if o is None else o.data_ptr()
+    a.final_state = None if final_state is None else final_state.data_ptr()
+    a.snap_interval = int(snap_interval)
+    a.snapshots = None if snapshots is None else snapshots.data_ptr()
+    a.workspace = workspace.data_ptr()
+    a.workspace_bytes = workspace.numel()
+    return a
+
+
+def prefill(q, k, v, beta, log_a, cu_seqlens, *, scalar_decay=False, scale=1.0,
+            init_state=None, snap_interval=0, cu_seqlens_host=None, out=None,
+            final_state=None, snapshots=None, workspace=None):
+    """Chunked prefill over a packed batch.  Returns (o, final_state, snapshots).
+
+    ``cu_seqlens`` is a device int32 tensor [N+1]; its host copy (taken from
+    ``cu_seqlens_host`` when given, else read back) sizes the snapshots.
+    Output buffers and the workspace may be passed in to avoid allocation.
+    """
+    if q.dtype != k.dtype or q.dtype != v.dtype:
+        raise TypeError("q, k and v must share a dtype")
+    _need_cuda(q, k, v, beta, log_a, cu_seqlens, init_state, out, final_state, snapshots,
+               workspace)
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    n = cu_seqlens.numel() - 1
+    dev = q.device
+    if out is None:
+        out = torch.empty(T, H, dv, dtype=q.dtype, device=dev)
+    if final_state is None:
+        final_state = torch.empty(n, H, dv, dk, dtype=torch.float32, device=dev)
+    if snap_interval and snapshots is None:
+        ns = snapshot_count(_host_cu(cu_seqlens, cu_seqlens_host), snap_interval)
+        snapshots = torch.empty(max(ns, 1), H, dv, dk, dtype=torch.float32, device=dev)[:ns]
+    if workspace is None:
+        nbytes = workspace_size(n, H, dk, dv, T, scalar_decay)
+        if nbytes == 0:
+            raise GdrError(2, "gdr_prefill_workspace_size")
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    snap_arg = snapshots if (snap_interval and snapshots is not None and snapshots.numel()) else None
+    if snap_interval and snap_arg is None:
+        # no full interval in any sequence: any valid aligned pointer will do
+        snap_arg = final_state
+    a = _prefill_args(q, k, v, beta, log_a, cu_seqlens, scalar_decay, scale, init_state,
+                      snap_interval, out, final_state, snap_arg, workspace)
+    _check(lib().gdr_prefill(ctypes.byref(a), _stream(dev)), "gdr_prefill")
+    return out, final_state, snapshots
+
+
+def prefill_status(workspace) -> None:
+    """Raise if the device side of the last prefill on ``workspace`` timed out."""
+    _check(lib().gdr_prefill_status(_ptr(workspace), _stream(workspace.device)),
+           "gdr_prefill_status")
+
+
+def cumdecay(log_a, cu_seqlens, *, scalar_decay=False, d_k=None, out=None):
+    """Chunk-local cumulative log decay (the first prefill kernel on its own)."""
+    _need_cuda(log_a, cu_seqlens, out)
+    T, H = log_a.shape[0], log_a.shape[1]
+    dk = d_k if scalar_decay else log_a.shape[2]
+    if out is None:
+        out = torch.empty_like(log_a)
+    _check(lib().gdr_cumdecay(cu_seqlens.numel() - 1, H, dk, T, _ptr(cu_seqlens), _ptr(log_a),
+                              int(bool(scalar_decay)), _ptr(out), _stream(log_a.device)),
+           "gdr_cumdecay")
+    return out
+
+
+def chunk_factors(q, k, v, beta, log_a, cu_seqlens, *, scalar_decay=False, scale=1.0):
+    """Intra-chunk factors (W, U, P, Qg, Kd, gamma) per chunk slot, fp32."""
+    _need_cuda(q, k, v, beta, log_a, cu_seqlens)
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    n = cu_seqlens.numel() - 1
+    dev = q.device
+    slots = T // 64 + n
+    f = dict(W=torch.zeros(slots, H, 64, dk, device=dev), U=torch.zeros(slots, H, 64, dv, device=dev),
+             P=torch.zeros(slots, H, 64, 64, device=dev), Qg=torch.zeros(slots, H, 64, dk, device=dev),
+             Kd=torch.zeros(slots, H, 64, dk, device=dev), gamma=torch.zeros(slots, H, dk, device=dev))
+    workspace = torch.empty(workspace_size(n, H, dk, dv, T, scalar_decay), dtype=torch.uint8,
+                            device=dev)
+    a = _prefill_args(q, k, v, beta, log_a, cu_seqlens, scalar_decay, scale, None, 0, None,
+                      None, None, workspace)
+    _check(lib().gdr_chunk_factors(ctypes.byref(a), _ptr(f["W"]), _ptr(f["U"]), _ptr(f["P"]),
+                                   _ptr(f["Qg"]), _ptr(f["Kd"]), _ptr(f["gamma"]), _stream(dev)),
+           "gdr_chunk_factors")
+    return f
+
+
+def decode_step(state, q, k, v, beta, log_a, *, scalar_decay=False, scale=1.0, out=None):
+    """One decode step; ``state`` [B, H, d_v, d_k] fp32 is updated in place.
+    Returns o [B, H, d_v] fp32."""
+    if q.dtype != k.dtype or q.dtype != v.dtype:
+        raise TypeError("q, k and v must share a dtype")
+    _need_cuda(state, q, k, v, beta, log_a, out)
+    if state.dtype != torch.float32:
+        raise TypeError("state must be float32")
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    if out is None:
+        out = torch.empty(B, H, dv, dtype=torch.float32, device=q.device)
+    _check(lib().gdr_decode_step(B, H, dk, dv, _dtype_code(q), _ptr(q), _ptr(k), _ptr(v),
+                                 _ptr(beta), _ptr(log_a), int(bool(scalar_decay)), float(scale),
+                                 _ptr(state), _ptr(out), _stream(q.device)),
+           "gdr_decode_step")
+    return out

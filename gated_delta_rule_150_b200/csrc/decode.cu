@@ -1,0 +1,156 @@
+// decode.cu -- one O(1)-state decode step of the gated delta rule.
+//
+// "kda-graft", section "2. Decode: O(1) против O(L)": a decode step of the
+// KDA layer reads and writes a fixed-size state, so its cost does not depend
+// on the context length.  Per (sequence, head) and per state row j (value
+// channel), with s the row of S and a = exp(log_a):
+//     s' = s * a                      (S Diag(a); "Gated DeltaNet: dodaj zanik")
+//     p  = s' . k,  c = s' . (scale q)
+//     d  = beta (v_j - p)             ("Reguła delta: zapisz poprawkę, nie sumę")
+//     s  = s' + d k
+//     o_j = s . (scale q) = c + d (k . scale q)   (read after the update)
+// Rows are independent given (k, beta, a), so the kernel streams the state
+// once: each row is read and written exactly once with 128-bit accesses.
+//
+// Memory roofline: per head-state 2 * 4 * d_v * d_k bytes of state plus the
+// token's inputs and the output row; no reuse, so the kernel is HBM-bound.
+#include <cuda_bf16.h>
+
+#include "internal.h"
+
+namespace gdr {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kTPR = 16;                      // threads per state row
+constexpr int kRowsPerPass = kThreads / kTPR; // 16 rows at a time
+
+template <typename T>
+__device__ __forceinline__ float to_f(T x);
+template <>
+__device__ __forceinline__ float to_f<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// Four consecutive elements starting at p (16-byte aligned for fp32, 8 for bf16).
+__device__ __forceinline__ float4 load4(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
+__device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
+    const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+}
+
+__device__ __forceinline__ float sum16(float x) {
+#pragma unroll
+    for (int m = 8; m >= 1; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
+    return x;
+}
+
+// One CTA per (sequence, head).  Thread t handles row group t / 16 and the
+// float4 columns {t % 16 + 16 i}.  DK/64 float4 per thread per row.
+template <typename T, int DK, int DV, bool SCALAR>
+__global__ void __launch_bounds__(kThreads)
+decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+                   const float* __restrict__ beta, const float* __restrict__ log_a, float scale,
+                   float* __restrict__ state, float* __restrict__ o) {
+    constexpr int NV = DK / (4 * kTPR);        // float4 per thread per row: 1 or 2
+    constexpr int PASSES = DV / kRowsPerPass;  // 4 or 8
+    const int bh = blockIdx.x;
+    const int lane16 = threadIdx.x % kTPR;
+    const int rgrp = threadIdx.x / kTPR;
+
+    float4 kk[NV], qq[NV], aa[NV];
+    float kq_part = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const int c = 4 * (lane16 + kTPR * i);
+        kk[i] = load4(k + (size_t)bh * DK + c);
+        float4 qv = load4(q + (size_t)bh * DK + c);
+        qq[i] = make_float4(qv.x * scale, qv.y * scale, qv.z * scale, qv.w * scale);
+        if (SCALAR) {
+            const float a = expf(__ldg(log_a + bh));
+            aa[i] = make_float4(a, a, a, a);
+        } else {
+            const float4 la = load4(log_a + (size_t)bh * DK + c);
+            aa[i] = make_float4(expf(la.x), expf(la.y), expf(la.z), expf(la.w));
+        }
+        kq_part += kk[i].x * qq[i].x + kk[i].y * qq[i].y + kk[i].z * qq[i].z + kk[i].w * qq[i].w;
+    }
+    const float kq = sum16(kq_part);
+    const float b = __ldg(beta + bh);
+
+    float* S = state + (size_t)bh * DV * DK;
+    // Issue every load of this thread's rows first (memory-level parallelism).
+    float4 s[PASSES][NV];
+#pragma unroll
+    for (int p = 0; p < PASSES; ++p)
+#pragma unroll
+        for (int i = 0; i < NV; ++i)
+            s[p][i] = *reinterpret_cast<const float4*>(S + (size_t)(rgrp + kRowsPerPass * p) * DK +
+                                                       4 * (lane16 + kTPR * i));
+    float vv[PASSES];
+#pragma unroll
+    for (int p = 0; p < PASSES; ++p) vv[p] = to_f<T>(v[(size_t)bh * DV + rgrp + kRowsPerPass * p]);
+
+#pragma unroll
+    for (int p = 0; p < PASSES; ++p) {
+        const int row = rgrp + kRowsPerPass * p;
+        float pk = 0.f, pq = 0.f;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            float4& x = s[p][i];
+            x.x *= aa[i].x; x.y *= aa[i].y; x.z *= aa[i].z; x.w *= aa[i].w;
+            pk += x.x * kk[i].x + x.y * kk[i].y + x.z * kk[i].z + x.w * kk[i].w;
+            pq += x.x * qq[i].x + x.y * qq[i].y + x.z * qq[i].z + x.w * qq[i].w;
+        }
+        pk = sum16(pk);
+        pq = sum16(pq);
+        const float d = b * (vv[p] - pk);
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            float4& x = s[p][i];
+            x.x += d * kk[i].x; x.y += d * kk[i].y; x.z += d * kk[i].z; x.w += d * kk[i].w;
+            *reinterpret_cast<float4*>(S + (size_t)row * DK + 4 * (lane16 + kTPR * i)) = x;
+        }
+        if (lane16 == 0) o[(size_t)bh * DV + row] = pq + d * kq;
+    }
+}
+
+template <typename T, int DK, int DV>
+cudaError_t launch_typed(int B, int H, const void* q, const void* k, const void* v,
+                         const float* beta, const float* log_a, int scalar, float scale,
+                         float* state, float* o, cudaStream_t st) {
+    const dim3 grid((unsigned)(B * H));
+    if (scalar)
+        decode_step_kernel<T, DK, DV, true><<<grid, kThreads, 0, st>>>(
+            (const T*)q, (const T*)k, (const T*)v, beta, log_a, scale, state, o);
+    else
+        decode_step_kernel<T, DK, DV, false><<<grid, kThreads, 0, st>>>(
+            (const T*)q, (const T*)k, (const T*)v, beta, log_a, scale, state, o);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_dims(int B, int H, int dk, int dv, const void* q, const void* k,
+                        const void* v, const float* beta, const float* log_a, int scalar,
+                        float scale, float* state, float* o, cudaStream_t st) {
+    if (dk == 64 && dv == 64) return launch_typed<T, 64, 64>(B, H, q, k, v, beta, log_a, scalar, scale, state, o, st);
+    if (dk == 64 && dv == 128) return launch_typed<T, 64, 128>(B, H, q, k, v, beta, log_a, scalar, scale, state, o, st);
+    if (dk == 128 && dv == 64) return launch_typed<T, 128, 64>(B, H, q, k, v, beta, log_a, scalar, scale, state, o, st);
+    return launch_typed<T, 128, 128>(B, H, q, k, v, beta, log_a, scalar, scale, state, o, st);
+}
+
+}  // namespace
+
+cudaError_t launch_decode(int B, int H, int dk, int dv, gdr_dtype dt, const void* q,
+                          const void* k, const void* v, const float* beta,
+                          const float* log_a, int scalar, float scale, float* state,
+                          float* o, cudaStream_t st) {
+    if (dt == GDR_BF16)
+        return launch_dims<__nv_bfloat16>(B, H, dk, dv, q, k, v, beta, log_a, scalar, scale,
+                                          state, o, st);
+    return launch_dims<float>(B, H, dk, dv, q, k, v, beta, log_a, scalar, scale, state, o, st);
+}
+
+}  // namespace gdr

@@ -1,0 +1,185 @@
+// gdr_api.cu -- the C ABI declared in include/gdr.h: argument checks, the
+// prefill workspace layout and the kernel launches, all on the caller's
+// stream.  Nothing here allocates, frees or synchronises (except
+// gdr_prefill_status, which reads one word back by design).
+#include <cstring>
+
+#include "internal.h"
+
+namespace {
+
+using gdr::WorkspaceLayout;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+bool aligned_elem(const void* p, gdr_dtype dt) {
+    return (reinterpret_cast<uintptr_t>(p) & (dt == GDR_BF16 ? 1u : 3u)) == 0;
+}
+
+gdr_status from_cuda(cudaError_t e) { return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA; }
+
+bool supported_width(int d) { return d == 64 || d == 128; }
+
+// Shared checks of the prefill arguments that do not depend on outputs.
+gdr_status check_prefill_inputs(const gdr_prefill_args* a) {
+    if (!a) return GDR_ERR_INVALID_ARG;
+    if (a->n_seqs < 0 || a->n_heads <= 0 || a->d_k <= 0 || a->d_v <= 0 || a->total_tokens < 0)
+        return GDR_ERR_INVALID_ARG;
+    if (a->total_tokens > (int64_t)INT32_MAX) return GDR_ERR_INVALID_ARG;
+    if (a->qkv_dtype != GDR_BF16 && a->qkv_dtype != GDR_F32) return GDR_ERR_INVALID_ARG;
+    if (!supported_width(a->d_k) || a->d_v != a->d_k) return GDR_ERR_UNSUPPORTED;
+    if (!a->cu_seqlens || !aligned4(a->cu_seqlens)) return GDR_ERR_INVALID_ARG;
+    if (a->total_tokens > 0) {
+        const void* vec[] = {a->q, a->k, a->v};
+        for (const void* p : vec)
+            if (!p || !aligned16(p)) return GDR_ERR_INVALID_ARG;
+        if (!a->beta || !aligned4(a->beta)) return GDR_ERR_INVALID_ARG;
+        if (!a->log_a || !(a->scalar_decay ? aligned4(a->log_a) : aligned16(a->log_a)))
+            return GDR_ERR_INVALID_ARG;
+    }
+    if (a->snap_interval < 0 || a->snap_interval % gdr::kChunk != 0) return GDR_ERR_INVALID_ARG;
+    return GDR_OK;
+}
+
+gdr_status check_workspace(const gdr_prefill_args* a, WorkspaceLayout* lay) {
+    *lay = gdr::workspace_layout(a->n_seqs, a->n_heads, a->d_k, a->total_tokens, a->scalar_decay);
+    if (!a->workspace || (reinterpret_cast<uintptr_t>(a->workspace) & 255u) != 0)
+        return GDR_ERR_WORKSPACE;
+    if (a->workspace_bytes < lay->total) return GDR_ERR_WORKSPACE;
+    return GDR_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* gdr_status_string(gdr_status s) {
+    switch (s) {
+        case GDR_OK: return "GDR_OK";
+        case GDR_ERR_INVALID_ARG: return "GDR_ERR_INVALID_ARG";
+        case GDR_ERR_UNSUPPORTED: return "GDR_ERR_UNSUPPORTED";
+        case GDR_ERR_WORKSPACE: return "GDR_ERR_WORKSPACE";
+        case GDR_ERR_CUDA: return "GDR_ERR_CUDA";
+        case GDR_ERR_TIMEOUT: return "GDR_ERR_TIMEOUT";
+    }
+    return "GDR_ERR_UNKNOWN";
+}
+
+int gdr_version(void) { return 100; }
+
+size_t gdr_prefill_workspace_size(int n_seqs, int n_heads, int d_k, int d_v,
+                                  int64_t total_tokens, int scalar_decay) {
+    if (n_seqs < 0 || n_heads <= 0 || total_tokens < 0) return 0;
+    if (!supported_width(d_k) || d_v != d_k) return 0;
+    return gdr::workspace_layout(n_seqs, n_heads, d_k, total_tokens, scalar_decay).total;
+}
+
+int64_t gdr_snapshot_count(const int32_t* host_cu, int n_seqs, int snap_interval) {
+    if (!host_cu || n_seqs < 0 || snap_interval < 0) return -1;
+    if (snap_interval == 0) return 0;
+    int64_t total = 0;
+    for (int n = 0; n < n_seqs; ++n) {
+        const int32_t len = host_cu[n + 1] - host_cu[n];
+        if (len < 0) return -1;
+        total += len / snap_interval;
+    }
+    return total;
+}
+
+gdr_status gdr_prefill(const gdr_prefill_args* a, void* stream) {
+    gdr_status s = check_prefill_inputs(a);
+    if (s != GDR_OK) return s;
+    if (!a->final_state || !aligned16(a->final_state)) return GDR_ERR_INVALID_ARG;
+    if (a->total_tokens > 0 && (!a->o || !aligned_elem(a->o, a->qkv_dtype))) return GDR_ERR_INVALID_ARG;
+    if (a->init_state && !aligned16(a->init_state)) return GDR_ERR_INVALID_ARG;
+    if (a->snap_interval > 0 && (!a->snapshots || !aligned16(a->snapshots)))
+        return GDR_ERR_INVALID_ARG;
+    WorkspaceLayout lay;
+    s = check_workspace(a, &lay);
+    if (s != GDR_OK) return s;
+    if (a->n_seqs == 0) return GDR_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(a->workspace);
+    uint32_t* err = reinterpret_cast<uint32_t*>(ws + lay.err_off);
+    float* g = reinterpret_cast<float*>(ws + lay.g_off);
+    uint8_t* rec = ws + lay.rec_off;
+    if (cudaMemsetAsync(err, 0, sizeof(uint32_t), st) != cudaSuccess) return GDR_ERR_CUDA;
+    if (a->total_tokens > 0) {
+        s = from_cuda(gdr::launch_cumdecay(a->n_seqs, a->n_heads, a->d_k, a->total_tokens,
+                                           a->cu_seqlens, a->log_a, a->scalar_decay, g, st));
+        if (s != GDR_OK) return s;
+        s = from_cuda(gdr::launch_intra_chunk(*a, g, rec, err, st));
+        if (s != GDR_OK) return s;
+    }
+    return from_cuda(gdr::launch_state_pass(*a, rec, err, st));
+}
+
+gdr_status gdr_prefill_status(const void* workspace, void* stream) {
+    if (!workspace) return GDR_ERR_INVALID_ARG;
+    uint32_t word = 0;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return GDR_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return GDR_ERR_CUDA;
+    return word == 0 ? GDR_OK : GDR_ERR_TIMEOUT;
+}
+
+gdr_status gdr_cumdecay(int n_seqs, int n_heads, int d_k, int64_t total_tokens,
+                        const int32_t* cu_seqlens, const float* log_a, int scalar_decay,
+                        float* g, void* stream) {
+    if (n_seqs < 0 || n_heads <= 0 || total_tokens < 0 || total_tokens > (int64_t)INT32_MAX)
+        return GDR_ERR_INVALID_ARG;
+    if (!supported_width(d_k)) return GDR_ERR_UNSUPPORTED;
+    if (!cu_seqlens || !aligned4(cu_seqlens)) return GDR_ERR_INVALID_ARG;
+    if (total_tokens == 0 || n_seqs == 0) return GDR_OK;
+    if (!log_a || !g || !aligned4(log_a) || !aligned4(g)) return GDR_ERR_INVALID_ARG;
+    return from_cuda(gdr::launch_cumdecay(n_seqs, n_heads, d_k, total_tokens, cu_seqlens, log_a,
+                                          scalar_decay, g, static_cast<cudaStream_t>(stream)));
+}
+
+gdr_status gdr_chunk_factors(const gdr_prefill_args* a, float* W, float* U, float* P,
+                             float* Qg, float* Kd, float* gamma, void* stream) {
+    gdr_status s = check_prefill_inputs(a);
+    if (s != GDR_OK) return s;
+    WorkspaceLayout lay;
+    s = check_workspace(a, &lay);
+    if (s != GDR_OK) return s;
+    if (a->n_seqs == 0 || a->total_tokens == 0) return GDR_OK;
+    const void* outs[] = {W, U, P, Qg, Kd, gamma};
+    for (const void* p : outs)
+        if (!p || !aligned16(p)) return GDR_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(a->workspace);
+    uint32_t* err = reinterpret_cast<uint32_t*>(ws + lay.err_off);
+    float* g = reinterpret_cast<float*>(ws + lay.g_off);
+    uint8_t* rec = ws + lay.rec_off;
+    if (cudaMemsetAsync(err, 0, sizeof(uint32_t), st) != cudaSuccess) return GDR_ERR_CUDA;
+    s = from_cuda(gdr::launch_cumdecay(a->n_seqs, a->n_heads, a->d_k, a->total_tokens,
+                                       a->cu_seqlens, a->log_a, a->scalar_decay, g, st));
+    if (s != GDR_OK) return s;
+    s = from_cuda(gdr::launch_intra_chunk(*a, g, rec, err, st));
+    if (s != GDR_OK) return s;
+    return from_cuda(gdr::launch_unpack_records(*a, rec, W, U, P, Qg, Kd, gamma, st));
+}
+
+gdr_status gdr_decode_step(int batch, int n_heads, int d_k, int d_v, gdr_dtype qkv_dtype,
+                           const void* q, const void* k, const void* v, const float* beta,
+                           const float* log_a, int scalar_decay, float scale, float* state,
+                           float* o, void* stream) {
+    if (batch < 0 || n_heads <= 0 || d_k <= 0 || d_v <= 0) return GDR_ERR_INVALID_ARG;
+    if (qkv_dtype != GDR_BF16 && qkv_dtype != GDR_F32) return GDR_ERR_INVALID_ARG;
+    if (!supported_width(d_k) || !supported_width(d_v)) return GDR_ERR_UNSUPPORTED;
+    if ((int64_t)batch * n_heads > (int64_t)INT32_MAX) return GDR_ERR_INVALID_ARG;
+    if (batch == 0) return GDR_OK;
+    const void* vec[] = {q, k, state};
+    for (const void* p : vec)
+        if (!p || !aligned16(p)) return GDR_ERR_INVALID_ARG;
+    if (!v || !aligned_elem(v, qkv_dtype) || !beta || !aligned4(beta) || !o || !aligned4(o))
+        return GDR_ERR_INVALID_ARG;
+    if (!log_a || !(scalar_decay ? aligned4(log_a) : aligned16(log_a))) return GDR_ERR_INVALID_ARG;
+    return from_cuda(gdr::launch_decode(batch, n_heads, d_k, d_v, qkv_dtype, q, k, v, beta, log_a,
+                                        scalar_decay, scale, state, o,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,187 @@
+/*
+ * gdr.h -- C ABI of the gated delta-rule library (B200, sm_100a).
+ *
+ * The operation.  For every sequence and head, with a state S of d_v x d_k
+ * values (row = value channel, column = key channel):
+ *
+ *     S_t = S_{t-1} Diag(a_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *     o_t = S_t (scale * q_t)
+ *
+ * Sources (the pages this library implements):
+ *   - "Modele hybrydowe: co Gated DeltaNet zastępuje w cache KV" (trefon.com):
+ *       section "Atencja liniowa: stan o stałym rozmiarze" -- a fixed
+ *       d_v x d_k state per head and o_t = S_t q_t;
+ *       section "Reguła delta: zapisz poprawkę, nie sumę" -- the delta write;
+ *       section "Gated DeltaNet: dodaj zanik" -- the decay alpha_t applied to
+ *       the old state before the delta read;
+ *       section "Co stan rekurencyjny zmienia przy serwowaniu" -- point 1
+ *       (prefix snapshots), and the closing paragraph: chunked prefill, dense
+ *       products inside a chunk, sequential only from chunk to chunk.
+ *   - "kda-graft: Qwen2.5-0.5B с трансплантированным KDA" (ailist.pro):
+ *       section "Идея и архитектура" -- KDA (Kimi Delta Attention / gated
+ *       delta rule), whose decay is one gate per key channel, a_t in (0,1]^d_k;
+ *       section "Быстрый старт" -- the state is kept in fp32;
+ *       section "2. Decode: O(1) против O(L)" -- the decode step reads and
+ *       writes a state whose size does not depend on the context length.
+ *
+ * Conventions for every call below.
+ *   - Pointers marked "device" are CUDA device pointers (cudaMalloc'd or from
+ *     any allocator of the same context); "host" pointers are ordinary memory.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  All work is enqueued on it; nothing synchronises the host.
+ *   - The library never allocates, frees or synchronises.  The caller owns
+ *     every buffer, including the prefill workspace.
+ *   - Tensors are dense, row-major, in the layouts stated per argument.
+ *     q, k, v (prefill), per-channel log_a, states, snapshots and the
+ *     workspace pointers must be 16-byte aligned (the workspace 256-byte);
+ *     beta, scalar log_a, o and the decode v need only their element
+ *     alignment.
+ *   - Arguments are checked on the host before anything is launched; a failed
+ *     check returns an error status and enqueues nothing.  A launch failure
+ *     returns GDR_ERR_CUDA.
+ */
+#ifndef GDR_H_
+#define GDR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDR_OK = 0,
+    GDR_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misalignment, bad cu_seqlens */
+    GDR_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement */
+    GDR_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required */
+    GDR_ERR_CUDA = 4,          /* a CUDA launch or device query failed */
+    GDR_ERR_TIMEOUT = 5        /* a kernel gave up a bounded wait (see gdr_prefill_status) */
+} gdr_status;
+
+typedef enum {
+    GDR_BF16 = 0,              /* bfloat16 q, k, v (and o for prefill) */
+    GDR_F32 = 1                /* float32 q, k, v (and o for prefill) */
+} gdr_dtype;
+
+/* Human-readable name of a status; never NULL. */
+const char* gdr_status_string(gdr_status s);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int gdr_version(void);
+
+/* ------------------------------------------------------------------------
+ * Prefill: chunked-parallel evaluation of the recurrence over a packed batch
+ * of sequences ("Modele hybrydowe", closing paragraph of "Co stan rekurencyjny
+ * zmienia przy serwowaniu": chunks of C = 64 tokens, dense products inside a
+ * chunk, a sequential pass from chunk to chunk).  Chunks restart at every
+ * sequence start; the last chunk of a sequence may be partial.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+    int n_seqs;                 /* N >= 0 sequences packed by cu_seqlens */
+    int n_heads;                /* H >= 1 */
+    int d_k;                    /* key/query width: 64 or 128 */
+    int d_v;                    /* value width: must equal d_k in this build */
+    int64_t total_tokens;       /* T_tot = cu_seqlens[N]; host copy of the device value */
+    const int32_t* cu_seqlens;  /* device [N+1]: 0 = cu[0] <= cu[1] <= ... <= cu[N] = T_tot */
+    gdr_dtype qkv_dtype;        /* dtype of q, k, v and o */
+    const void* q;              /* device [T_tot, H, d_k] */
+    const void* k;              /* device [T_tot, H, d_k] */
+    const void* v;              /* device [T_tot, H, d_v] */
+    const float* beta;          /* device [T_tot, H], write strength in (0, 1) */
+    const float* log_a;         /* device [T_tot, H, d_k] (KDA), or [T_tot, H] when
+                                   scalar_decay != 0 (Gated DeltaNet); log a_t <= 0 */
+    int scalar_decay;           /* 0: per-key-channel decay, 1: one decay per head-token */
+    float scale;                /* multiplies q; the pages use none: pass 1.0f */
+    const float* init_state;    /* device [N, H, d_v, d_k] or NULL for zero states.
+                                   May alias final_state. */
+    void* o;                    /* device [T_tot, H, d_v], dtype qkv_dtype (output) */
+    float* final_state;         /* device [N, H, d_v, d_k] (output) */
+    int snap_interval;          /* 0: no snapshots; else a multiple of 64 */
+    float* snapshots;           /* device [gdr_snapshot_count(...), H, d_v, d_k] (output):
+                                   the state after tokens [0, m*snap_interval) of each
+                                   sequence, m = 1 .. floor(L_n / snap_interval),
+                                   sequences in order ("Co stan rekurencyjny zmienia przy
+                                   serwowaniu", point 1: a prefix is reused from the
+                                   snapshot taken at its end). */
+    void* workspace;            /* device scratch, >= gdr_prefill_workspace_size(...) bytes,
+                                   256-byte aligned; contents on entry do not matter */
+    size_t workspace_bytes;
+} gdr_prefill_args;
+
+/* Bytes of device workspace gdr_prefill needs for these sizes (0 on bad sizes). */
+size_t gdr_prefill_workspace_size(int n_seqs, int n_heads, int d_k, int d_v,
+                                  int64_t total_tokens, int scalar_decay);
+
+/* Number of snapshot slots for host-side cu_seqlens [N+1] (-1 on bad input). */
+int64_t gdr_snapshot_count(const int32_t* host_cu_seqlens, int n_seqs, int snap_interval);
+
+/*
+ * Enqueue a prefill.  Outputs: o, final_state and (if snap_interval > 0)
+ * snapshots.  Zero-length sequences are legal: their final state is their
+ * initial state.  Errors: GDR_ERR_INVALID_ARG / GDR_ERR_UNSUPPORTED /
+ * GDR_ERR_WORKSPACE before launch, GDR_ERR_CUDA on a failed launch.
+ */
+gdr_status gdr_prefill(const gdr_prefill_args* args, void* stream);
+
+/*
+ * Status the device side of the most recent gdr_prefill on this workspace
+ * recorded: GDR_OK, or GDR_ERR_TIMEOUT if a kernel abandoned a bounded wait
+ * (its outputs are then undefined).  Synchronises `stream`.
+ */
+gdr_status gdr_prefill_status(const void* workspace, void* stream);
+
+/*
+ * The chunk-local cumulative log decay on its own (the first kernel of the
+ * prefill): g[t] = sum of log_a over the tokens of t's chunk up to and
+ * including t, chunks as in gdr_prefill.  log_a and g share the layout
+ * [T_tot, H, d_k] (or [T_tot, H] when scalar_decay != 0), fp32, device.
+ */
+gdr_status gdr_cumdecay(int n_seqs, int n_heads, int d_k, int64_t total_tokens,
+                        const int32_t* cu_seqlens, const float* log_a, int scalar_decay,
+                        float* g, void* stream);
+
+/*
+ * The intra-chunk factors on their own (cumulative decay + intra-chunk
+ * kernel), unpacked to plain fp32 arrays for inspection.  With
+ * n_slots = floor(T_tot / 64) + N chunk slots, chunk j of sequence n lives in
+ * slot floor((cu[n] + 64 j) / 64) + n; unused slots are left untouched.
+ * Per slot and head (row r = token of the chunk, i = earlier token, c = key
+ * channel, e = value channel):
+ *   W  [n_slots, H, 64, d_k] = T diag(beta) (K * exp(g))
+ *   U  [n_slots, H, 64, d_v] = T diag(beta) V
+ *   P  [n_slots, H, 64, 64]  = scale * sum_c q[r,c] k[i,c] exp(g[r,c] - g[i,c]), i <= r
+ *   Qg [n_slots, H, 64, d_k] = scale * Q * exp(g)
+ *   Kd [n_slots, H, 64, d_k] = K * exp(g_last - g)
+ *   gamma [n_slots, H, d_k]  = exp(g_last)
+ * with T = (I + A)^-1, A[r,i] = beta_r sum_c k[r,c] k[i,c] exp(g[r,c] - g[i,c])
+ * for i < r, g the chunk-local cumulative log decay.  Rows past the end of a
+ * partial chunk are zero.  `workspace` as for gdr_prefill with the same
+ * arguments; q, k, v, beta, log_a, cu_seqlens, scalar_decay and scale are
+ * read from `args`, its outputs are ignored.
+ */
+gdr_status gdr_chunk_factors(const gdr_prefill_args* args, float* W, float* U, float* P,
+                             float* Qg, float* Kd, float* gamma, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Decode: one token per sequence, state updated in place ("kda-graft",
+ * section "2. Decode: O(1) против O(L)": the step streams a fixed-size fp32
+ * state, independent of the context length).
+ *   q, k   device [B, H, d_k], dtype qkv_dtype
+ *   v      device [B, H, d_v], dtype qkv_dtype
+ *   beta   device [B, H] fp32
+ *   log_a  device [B, H, d_k] fp32, or [B, H] when scalar_decay != 0
+ *   state  device [B, H, d_v, d_k] fp32, read and overwritten
+ *   o      device [B, H, d_v] fp32 (output), o = S_new (scale * q)
+ * d_k in {64, 128}; d_v in {64, 128}.  B == 0 is a no-op.
+ * ---------------------------------------------------------------------- */
+gdr_status gdr_decode_step(int batch, int n_heads, int d_k, int d_v, gdr_dtype qkv_dtype,
+                           const void* q, const void* k, const void* v, const float* beta,
+                           const float* log_a, int scalar_decay, float scale, float* state,
+                           float* o, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDR_H_ */

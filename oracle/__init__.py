@@ -208,7 +208,9 @@ def chunk_factors(q, k, v, beta, log_a, start, end, h, scalar_decay=False, scale
     g = np.cumsum(la, axis=0)
     gam = np.exp(g)
     # decay-weighted products, term by term exp(g_r - g_i) (no factoring)
-    D = np.exp(g[:, None, :] - g[None, :, :])             # [r, i, c]
+    # exp(g_r - g_i) for i <= r only (the other entries are masked out below)
+    low = np.tril(np.ones((L, L), dtype=bool))[:, :, None]
+    D = np.exp(np.where(low, g[:, None, :] - g[None, :, :], -np.inf))   # [r, i, c]
     KK = np.einsum("rc,ic,ric->ri", K, K, D)
     QK = np.einsum("rc,ic,ric->ri", Q, K, D)
     A = np.tril(b[:, None] * KK, -1)

@@ -1,0 +1,110 @@
+"""Host-side checks of the C ABI: the library loads without a GPU, exports
+every function include/gdr.h declares, rejects bad arguments before any
+launch, and sizes workspaces and snapshot buffers as documented."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import gated_delta_rule_150_b200 as gdr
+from gated_delta_rule_150_b200 import build as gdr_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    gdr_build.build()
+    return gdr.lib()
+
+
+def declared_functions():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", h)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(gdr_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert "gdr_prefill" in names and "gdr_decode_step" in names
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in include/ but not exported"
+
+
+def test_status_strings(L):
+    for s, name in gdr._STATUS.items():
+        assert L.gdr_status_string(s).decode() == name
+
+
+def _fake(n):
+    # 256-byte aligned fake device addresses: validation must fail before any use
+    return ctypes.c_void_p(0x10000 * (n + 1))
+
+
+def test_decode_rejects_bad_arguments(L):
+    ok = [_fake(i) for i in range(7)]
+    st = None
+    def call(B=2, H=2, dk=64, dv=64, dt=0, ptrs=ok):
+        return L.gdr_decode_step(B, H, dk, dv, dt, *ptrs[:5], 0, 1.0, ptrs[5], ptrs[6], st)
+    assert call(B=-1) == 1
+    assert call(dk=96) == 2
+    assert call(dv=32) == 2
+    assert call(dt=7) == 1
+    bad = list(ok); bad[2] = None
+    assert call(ptrs=bad) == 1
+    mis = list(ok); mis[0] = ctypes.c_void_p(0x10008)
+    assert call(ptrs=mis) == 1
+    assert call(B=0) == 0
+
+
+def _args(**kw):
+    a = gdr.PrefillArgs()
+    a.n_seqs, a.n_heads, a.d_k, a.d_v, a.total_tokens = 1, 2, 64, 64, 128
+    a.cu_seqlens = 0x10000
+    a.qkv_dtype = 0
+    a.q, a.k, a.v, a.beta, a.log_a = 0x20000, 0x30000, 0x40000, 0x50000, 0x60000
+    a.scale = 1.0
+    a.o, a.final_state = 0x70000, 0x80000
+    a.workspace = 0x100000
+    a.workspace_bytes = 1 << 40
+    for k_, v_ in kw.items():
+        setattr(a, k_, v_)
+    return a
+
+
+def test_prefill_rejects_bad_arguments(L):
+    pre = lambda a: L.gdr_prefill(ctypes.byref(a), None)
+    assert pre(_args(n_heads=0)) == 1
+    assert pre(_args(d_k=96, d_v=96)) == 2
+    assert pre(_args(d_v=128)) == 2
+    assert pre(_args(q=None)) == 1
+    assert pre(_args(k=0x30004)) == 1
+    assert pre(_args(snap_interval=100, snapshots=0x90000)) == 1
+    assert pre(_args(snap_interval=128, snapshots=None)) == 1
+    assert pre(_args(workspace=None)) == 3
+    assert pre(_args(workspace_bytes=16)) == 3
+    assert pre(_args(workspace=0x100080)) == 3
+    assert pre(_args(final_state=None)) == 1
+    assert pre(_args(total_tokens=-1)) == 1
+    assert pre(_args(n_seqs=0, total_tokens=0)) == 0
+
+
+def test_workspace_size_grows_with_tokens(L):
+    s1 = gdr.workspace_size(1, 14, 64, 64, 8192)
+    s2 = gdr.workspace_size(1, 14, 64, 64, 16384)
+    assert 0 < s1 < s2
+    assert gdr.workspace_size(1, 14, 96, 96, 8192) == 0
+    assert gdr.workspace_size(1, 14, 128, 128, 8192, True) < gdr.workspace_size(1, 14, 128, 128, 8192, False)
+
+
+def test_snapshot_count_matches_oracle(L):
+    import oracle
+    for lengths, iv in (([4096, 100, 8192, 0, 4095], 4096), ([64, 128, 1], 64), ([5, 7], 0)):
+        cu = torch.tensor([0] + list(torch.tensor(lengths).cumsum(0)), dtype=torch.int32)
+        assert gdr.snapshot_count(cu, iv) == oracle.snapshot_count(cu, iv)
