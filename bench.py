@@ -1,0 +1,502 @@
+#!/usr/bin/env python
+"""Throughput of the gated delta-rule hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl gdr|reference]
+
+One JSON line on rank 0.  A "step" is one chunked prefill (cumulative decay,
+intra-chunk factors, sequential state pass: three kernels) over one batch of
+the Qwen2.5-0.5B KDA-graft layer workload (1 sequence x 8192 tokens, 14 heads,
+d_k = d_v = 64, bf16 q/k/v, fp32 beta/log_a/state).  ``value`` is prefill
+tokens/s over all ranks (each rank runs its own batch: weak scaling, no
+collective on the data path).  The same run also measures:
+
+* ``decode``: the decode step on 256 sequences x 14 heads x 64 x 64 fp32 states,
+  state bytes streamed per second (four state sets rotated so that the 235 MB
+  working set exceeds the 126 MB L2);
+* ``roofline``: the step's dominant kernel, timed alone with CUDA events;
+* ``e2e``: the same prefill through the public API with pinned host buffers,
+  host<->device copies inside the timed region;
+* ``cpu_baseline``: the fp64 oracle on the host cores, same workload;
+* ``extra``: the other prefill workloads (tiny fp32, 65K-token scalar gate with
+  snapshots, 32-sequence varlen batch), a few steps each.
+
+``--impl reference`` times the fp64 CPU oracle alone (rank 0; other ranks exit).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+METRIC = "gated-delta prefill tokens/s + decode state GB/s, 1×B200 (% of roofline)"
+CHUNK = 64
+L2_BYTES = 126 * 2 ** 20
+
+
+# ---------------------------------------------------------------------------
+# algorithmic counts (per unit of work)
+# ---------------------------------------------------------------------------
+def prefill_flops_per_token_head(d_k: int, d_v: int) -> int:
+    """Causal halves counted once: K K^T, Q K^T and T (b K) (C d_k each),
+    T (b V) and P Delta (C d_v each), W S^T, Q S^T and Delta^T K (2 d_k d_v each)."""
+    return 3 * CHUNK * d_k + 2 * CHUNK * d_v + 6 * d_k * d_v
+
+
+def prefill_bytes_per_token_head(d_k: int, d_v: int, elem: int, scalar: bool) -> int:
+    """q, k, v read and o written once, plus beta and log_a (fp32)."""
+    return 2 * d_k * elem + 2 * d_v * elem + 4 + (4 if scalar else 4 * d_k)
+
+
+def prefill_state_bytes(n_seqs: int, H: int, d_k: int, d_v: int, has_init: bool, n_snap: int) -> int:
+    per = d_k * d_v * 4 * H
+    return per * n_seqs * (2 if has_init else 1) + per * n_snap
+
+
+def decode_bytes_per_head_state(d_k: int, d_v: int, elem: int, scalar: bool) -> int:
+    """state read + written (fp32), q, k, v, beta, log_a read, o (fp32) written."""
+    return 2 * 4 * d_k * d_v + (2 * d_k + d_v) * elem + 4 + (4 if scalar else 4 * d_k) + 4 * d_v
+
+
+def peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        p = json.load(open(path))
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(gpu_index)], stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self, t0: datetime.datetime, t1: datetime.datetime):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.file.flush()
+        rows = []
+        for line in open(self.file.name):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f")
+                rows.append((ts, float(parts[1]), float(parts[2]), parts[4:8]))
+            except ValueError:
+                continue
+        os.unlink(self.file.name)
+        if not rows:
+            return None
+        inside = [r for r in rows if t0 <= r[0] <= t1]
+        window = inside or sorted(rows, key=lambda r: abs((r[0] - t0).total_seconds()))[:3]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in window for i, s in enumerate(r[3]) if s.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[1] for r in window),
+                "sm_max_mhz": max(r[2] for r in window), "reasons": reasons,
+                "samples": len(window), "samples_inside_timed_region": len(inside)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (one process per GPU, torchrun)
+# ---------------------------------------------------------------------------
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def timed(fn, n, stream):
+    """Average device time (ms) of n calls of fn, CUDA events on `stream`."""
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(n):
+        fn(i)
+    end.record(stream)
+    torch.cuda.synchronize()
+    return start.elapsed_time(end) / n
+
+
+# ---------------------------------------------------------------------------
+# prefill workloads on the GPU
+# ---------------------------------------------------------------------------
+class PrefillSets:
+    """R independent input sets (rotated every step), outputs and workspaces."""
+
+    def __init__(self, gdr, w: wl.PrefillWorkload, n_sets: int, rank: int):
+        self.w = w
+        self.sets = []
+        for i in range(n_sets):
+            wi = wl.shrink(w, seed=w.seed + 7919 * i + 100003 * rank)
+            inp = wl.make_prefill_inputs(wi, device="cuda", draw_device="cuda")
+            T, H, dk = inp["q"].shape
+            dv = inp["v"].shape[-1]
+            n = len(inp["lengths"])
+            ns = gdr.snapshot_count(wl.cu_seqlens_of(inp["lengths"]), w.snap_interval) if w.snap_interval else 0
+            out = torch.empty(T, H, dv, dtype=inp["q"].dtype, device="cuda")
+            fin = torch.empty(n, H, dv, dk, device="cuda")
+            snaps = torch.empty(max(ns, 1), H, dv, dk, device="cuda") if w.snap_interval else None
+            ws = torch.empty(gdr.workspace_size(n, H, dk, dv, T, w.scalar_decay), dtype=torch.uint8,
+                             device="cuda")
+            prep = gdr.PreparedPrefill(inp["q"], inp["k"], inp["v"], inp["beta"], inp["log_a"],
+                                       inp["cu_seqlens"], out=out, final_state=fin, workspace=ws,
+                                       scalar_decay=w.scalar_decay, scale=w.scale,
+                                       init_state=inp["init_state"], snap_interval=w.snap_interval,
+                                       snapshots=snaps)
+            self.sets.append(dict(inp=inp, prep=prep, n_snap=ns, T=T, H=H, dk=dk, dv=dv, n=n))
+        s0 = self.sets[0]
+        self.T, self.H, self.dk, self.dv, self.n = s0["T"], s0["H"], s0["dk"], s0["dv"], s0["n"]
+        elem = 2 if w.qkv_dtype == torch.bfloat16 else 4
+        self.units = self.T * self.H
+        self.flops = prefill_flops_per_token_head(self.dk, self.dv) * self.units
+        self.bytes = (prefill_bytes_per_token_head(self.dk, self.dv, elem, w.scalar_decay) * self.units
+                      + prefill_state_bytes(self.n, self.H, self.dk, self.dv, w.init_std > 0,
+                                            s0["n_snap"]))
+        self.footprint = sum(sum(t.numel() * t.element_size() for t in s["prep"]._keep
+                                 if torch.is_tensor(t)) for s in self.sets)
+
+    def step(self, i, stages=(0, 2)):
+        self.sets[i % len(self.sets)]["prep"].run(stages)
+
+
+def stage_times(ps: PrefillSets, n: int, stream) -> list:
+    """Device time of each of the three prefill kernels launched alone (ms)."""
+    for i in range(len(ps.sets)):
+        ps.step(i)
+    out = []
+    for s in range(3):
+        out.append(timed(lambda i: ps.step(i, (s, s)), n, stream))
+    return out
+
+
+def roofline_obj(bytes_, flops, t_ms, pk, traffic=None):
+    gbs = bytes_ / (t_ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": round(gbs / pk["hbm_gbs"], 4), "traffic": traffic,
+            "tensor_tflops": round(flops / (t_ms * 1e-3) / 1e12, 2),
+            "tensor_frac": round(flops / (t_ms * 1e-3) / 1e12 / pk["bf16_tflops"], 4),
+            "peak_source": pk["source"]}
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """dram bytes per launch from the committed ncu summary, if it still
+    matches the kernel's current source."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        rows = json.load(open(path))
+    except Exception:
+        return None
+    for r in rows:
+        if r.get("kernel") == kernel and r.get("workload") == workload:
+            src = os.path.join(ROOT, r["source"])
+            sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+            if sha == r.get("source_sha"):
+                return r.get("dram_bytes_per_launch")
+    return None
+
+
+# ---------------------------------------------------------------------------
+# arms
+# ---------------------------------------------------------------------------
+def run_reference(args):
+    """The fp64 CPU oracle as the reference arm (rank 0 only)."""
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    w = wl.GRAFT_LAYER
+    inp = wl.make_prefill_inputs(w)
+    T, H = inp["q"].shape[0], inp["q"].shape[1]
+
+    def run(heads):
+        oracle.prefill(inp["q"][:, heads], inp["k"][:, heads], inp["v"][:, heads],
+                       inp["beta"][:, heads], inp["log_a"][:, heads], inp["cu_seqlens"])
+
+    # bounded sample: all heads if one pass takes <= 2 s, else the first few
+    t0 = time.perf_counter()
+    run(list(range(H)))
+    t_full = time.perf_counter() - t0
+    heads = list(range(H)) if t_full <= 2.0 else list(range(max(1, int(H * 2.0 / t_full))))
+    for _ in range(max(0, args.warmup - 1)):
+        run(heads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run(heads)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = T * len(heads) / H / dt          # tokens/s (token-heads/s over H)
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count()))
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "n_seqs": 1, "seq_len": T, "heads": H, "d_k": w.d_k,
+                       "d_v": w.d_v, "parallelism": "none (host cores)"},
+            "cpu_baseline": {"value": round(value, 1), "unit": "tokens/s", "cores": cores,
+                             "kind": "oracle",
+                             "sample": f"{len(heads)} of {H} heads x {T} tokens per step"},
+            "e2e": {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline_graft(budget_s: float = 12.0) -> dict:
+    import oracle
+    w = wl.GRAFT_LAYER
+    inp = wl.make_prefill_inputs(w)
+    T, H = inp["q"].shape[0], inp["q"].shape[1]
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle.prefill(inp["q"], inp["k"], inp["v"], inp["beta"], inp["log_a"], inp["cu_seqlens"])
+        n += 1
+        if time.perf_counter() - t0 > budget_s or n >= 20:
+            break
+    dt = (time.perf_counter() - t0) / n
+    return {"value": round(T / dt, 1), "unit": "tokens/s",
+            "cores": int(os.environ.get("OMP_NUM_THREADS", os.cpu_count())), "kind": "oracle",
+            "sample": f"{n} full passes of {w.name} ({T} tokens x {H} heads), fp64"}
+
+
+def run_gdr(args):
+    world, rank, local = dist_env()
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    torch.cuda.set_device(local)
+    import gated_delta_rule_150_b200 as gdr
+    gdr.lib()                                   # raises if the CUDA library is missing
+    stream = torch.cuda.current_stream()
+    pk = peaks()
+
+    # ---- main workload: graft-layer prefill, 4 rotating input sets ----------
+    ps = PrefillSets(gdr, wl.GRAFT_LAYER, 4, rank)
+    for i in range(args.warmup):
+        ps.step(i)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_wall0 = datetime.datetime.now()
+    start.record(stream)
+    for i in range(args.steps):
+        ps.step(i)
+    end.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = datetime.datetime.now()
+    barrier(world)
+    clocks = sampler.stop(t_wall0, t_wall1)
+    ms_local = start.elapsed_time(end)
+    ms_total = max_over_ranks(ms_local, world)
+    ms_step = ms_total / args.steps
+    value = world * ps.T * args.steps / (ms_total * 1e-3)
+
+    # ---- the three kernels alone -> dominant kernel roofline --------------------
+    names = ["cumdecay", "intra_chunk", "state_pass"]
+    sources = ["gated_delta_rule_150_b200/csrc/cumdecay.cu",
+               "gated_delta_rule_150_b200/csrc/intra_chunk.cu",
+               "gated_delta_rule_150_b200/csrc/state_pass.cu"]
+    st_ms = stage_times(ps, max(20, min(args.steps, 200)), stream)
+    dom = max(range(3), key=lambda s: st_ms[s])
+    roof = roofline_obj(ps.bytes, ps.flops, st_ms[dom], pk,
+                        recorded_traffic(names[dom], ps.w.name))
+    roof["kernel"] = names[dom]
+    roof["kernel_ms"] = round(st_ms[dom], 4)
+    stage_report = {names[s]: round(st_ms[s], 4) for s in range(3)}
+    path_roof = roofline_obj(ps.bytes, ps.flops, ms_step, pk)
+
+    extra = {}
+    decode = None
+    if not args.no_extra:
+        decode = bench_decode(gdr, stream, pk, args)
+        for w in (wl.TINY_KDA, wl.GDN_LONG, wl.VARLEN):
+            extra[w.name] = bench_prefill_workload(gdr, w, stream, pk, rank, args)
+    e2e = bench_e2e(gdr, stream, args)
+
+    cpu = cpu_baseline_graft() if (rank == 0 and world == 1 and not args.no_cpu) else None
+    if rank != 0:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": ps.w.name, "n_seqs": ps.n, "seq_len": ps.T, "heads": ps.H,
+                   "d_k": ps.dk, "d_v": ps.dv, "parallelism": "replicas" if world > 1 else "none",
+                   "l2": f"4 rotating input sets, {ps.footprint / 2**20:.0f} MiB > 126 MiB L2"},
+        "roofline": roof,
+        "path_roofline": path_roof,
+        "kernel_ms": stage_report,
+        "decode": decode,
+        "e2e": e2e,
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+        "extra": extra,
+        "gpu": torch.cuda.get_device_name(),
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def bench_prefill_workload(gdr, w, stream, pk, rank, args):
+    ps = PrefillSets(gdr, w, 1 if w is not wl.TINY_KDA else 4, rank)
+    n = 3 if ps.T > 100000 else 20
+    for i in range(2):
+        ps.step(i)
+    ms = timed(lambda i: ps.step(i), n, stream)
+    st = stage_times(ps, n, stream)
+    res = {"tokens_per_s": round(ps.T / (ms * 1e-3), 1), "ms_per_step": round(ms, 4),
+           "kernel_ms": {k: round(v, 4) for k, v in zip(("cumdecay", "intra_chunk", "state_pass"), st)},
+           "path_roofline": roofline_obj(ps.bytes, ps.flops, ms, pk), "tokens": ps.T,
+           "sequences": ps.n, "inputs_exceed_l2": ps.footprint > L2_BYTES}
+    del ps
+    torch.cuda.empty_cache()
+    return res
+
+
+def bench_decode(gdr, stream, pk, args):
+    """Decode step on the decode workload: 1024 steps, four rotating state sets."""
+    w = wl.DECODE
+    steps = w.steps
+    inp = wl.make_decode_inputs(w, steps=steps, device="cuda", draw_device="cuda")
+    states = [inp["state"].clone() for _ in range(4)]
+    o = torch.empty(w.batch, w.n_heads, w.d_v, device="cuda")
+
+    def step(i):
+        t = i % steps
+        gdr.decode_step(states[i % 4], inp["q"][t], inp["k"][t], inp["v"][t], inp["beta"][t],
+                        inp["log_a"][t], scalar_decay=w.scalar_decay, scale=w.scale, out=o)
+
+    for i in range(8):
+        step(i)
+    ms = timed(step, steps, stream)
+    elem = 2 if w.qkv_dtype == torch.bfloat16 else 4
+    per = decode_bytes_per_head_state(w.d_k, w.d_v, elem, w.scalar_decay)
+    units = w.batch * w.n_heads
+    gbs = per * units / (ms * 1e-3) / 1e9
+    res = {"workload": w.name, "gbs": round(gbs, 1), "ms_per_step": round(ms, 5),
+           "bytes_per_head_state": per, "head_states_per_step": units,
+           "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"],
+                        "unit": "GB/s", "frac": round(gbs / pk["hbm_gbs"], 4),
+                        "traffic": recorded_traffic("decode_step", w.name)},
+           "l2": "4 rotating state sets, 235 MB > 126 MB L2", "steps": steps}
+    del inp, states
+    torch.cuda.empty_cache()
+    return res
+
+
+def bench_e2e(gdr, stream, args):
+    """Prefill through the public API from pinned host buffers: H2D of the
+    inputs, the prefill, D2H of o and the final state, every step."""
+    w = wl.GRAFT_LAYER
+    host = wl.make_prefill_inputs(w)
+    pinned = {k: host[k].pin_memory() for k in ("q", "k", "v", "beta", "log_a", "cu_seqlens")}
+    dev = {k: torch.empty_like(v, device="cuda") for k, v in pinned.items()}
+    T, H, dk = host["q"].shape
+    dv = host["v"].shape[-1]
+    out = torch.empty(T, H, dv, dtype=host["q"].dtype, device="cuda")
+    fin = torch.empty(1, H, dv, dk, device="cuda")
+    ws = torch.empty(gdr.workspace_size(1, H, dk, dv, T), dtype=torch.uint8, device="cuda")
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    fin_h = torch.empty(fin.shape, dtype=fin.dtype).pin_memory()
+    prep = gdr.PreparedPrefill(dev["q"], dev["k"], dev["v"], dev["beta"], dev["log_a"],
+                               dev["cu_seqlens"], out=out, final_state=fin, workspace=ws)
+
+    def step(_):
+        for k_ in pinned:
+            dev[k_].copy_(pinned[k_], non_blocking=True)
+        prep.run()
+        out_h.copy_(out, non_blocking=True)
+        fin_h.copy_(fin, non_blocking=True)
+
+    for i in range(3):
+        step(i)
+    n = max(5, min(args.steps, 50))
+    ms = timed(step, n, stream)
+    h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+    d2h = out_h.numel() * out_h.element_size() + fin_h.numel() * fin_h.element_size()
+    return {"value": round(T / (ms * 1e-3), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 4), "steps": n}
+
+
+def main():
+    p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["gdr", "reference"], default="gdr")
+    p.add_argument("--no-extra", action="store_true", help="skip decode and the other workloads")
+    p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    p.add_argument("--only-decode", action="store_true",
+                   help="run only the decode measurement (for profiling)")
+    args = p.parse_args()
+    if args.warmup < 3:
+        p.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    elif args.only_decode:
+        import gated_delta_rule_150_b200 as gdr
+        gdr.lib()
+        print(json.dumps(bench_decode(gdr, torch.cuda.current_stream(), peaks(), args)), flush=True)
+    else:
+        run_gdr(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -19,7 +19,7 @@ import threading
 
 import torch
 
-__all__ = ["prefill", "decode_step", "cumdecay", "chunk_factors", "workspace_size",
+__all__ = ["PrefillArgs", "PreparedPrefill", "prefill", "decode_step", "cumdecay", "chunk_factors", "workspace_size",
            "snapshot_count", "prefill_status", "lib", "GdrError", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_build", "libgdr.so")
@@ -74,6 +74,8 @@ def lib():
             L.gdr_snapshot_count.argtypes = [vp, i, i]
             L.gdr_prefill.restype = i
             L.gdr_prefill.argtypes = [ctypes.POINTER(PrefillArgs), vp]
+            L.gdr_prefill_stages.restype = i
+            L.gdr_prefill_stages.argtypes = [ctypes.POINTER(PrefillArgs), i, i, vp]
             L.gdr_prefill_status.restype = i
             L.gdr_prefill_status.argtypes = [vp, vp]
             L.gdr_cumdecay.restype = i
@@ -163,12 +165,14 @@ def _prefill_args(q, k, v, beta, log_a, cu_seqlens, scalar_decay, scale, init_st
 
 def prefill(q, k, v, beta, log_a, cu_seqlens, *, scalar_decay=False, scale=1.0,
             init_state=None, snap_interval=0, cu_seqlens_host=None, out=None,
-            final_state=None, snapshots=None, workspace=None):
+            final_state=None, snapshots=None, workspace=None, stages=(0, 2)):
     """Chunked prefill over a packed batch.  Returns (o, final_state, snapshots).
 
     ``cu_seqlens`` is a device int32 tensor [N+1]; its host copy (taken from
     ``cu_seqlens_host`` when given, else read back) sizes the snapshots.
     Output buffers and the workspace may be passed in to avoid allocation.
+    ``stages`` = (first, last) runs only that range of the three kernels
+    (0 cumulative decay, 1 intra-chunk, 2 state pass), for timing them apart.
     """
     if q.dtype != k.dtype or q.dtype != v.dtype:
         raise TypeError("q, k and v must share a dtype")
@@ -196,8 +200,43 @@ def prefill(q, k, v, beta, log_a, cu_seqlens, *, scalar_decay=False, scale=1.0,
         snap_arg = final_state
     a = _prefill_args(q, k, v, beta, log_a, cu_seqlens, scalar_decay, scale, init_state,
                       snap_interval, out, final_state, snap_arg, workspace)
-    _check(lib().gdr_prefill(ctypes.byref(a), _stream(dev)), "gdr_prefill")
+    first, last = stages
+    if (first, last) == (0, 2):
+        _check(lib().gdr_prefill(ctypes.byref(a), _stream(dev)), "gdr_prefill")
+    else:
+        _check(lib().gdr_prefill_stages(ctypes.byref(a), int(first), int(last), _stream(dev)),
+               "gdr_prefill_stages")
     return out, final_state, snapshots
+
+
+class PreparedPrefill:
+    """A prefill whose argument block is built once and replayed.
+
+    Holds references to every tensor it points at.  ``run()`` enqueues one
+    gdr_prefill (or a stage range) on the current stream of the tensors' device.
+    """
+
+    def __init__(self, q, k, v, beta, log_a, cu_seqlens, *, out, final_state, workspace,
+                 scalar_decay=False, scale=1.0, init_state=None, snap_interval=0,
+                 snapshots=None):
+        _need_cuda(q, k, v, beta, log_a, cu_seqlens, out, final_state, workspace, init_state,
+                   snapshots)
+        self._keep = (q, k, v, beta, log_a, cu_seqlens, out, final_state, workspace,
+                      init_state, snapshots)
+        self.args = _prefill_args(q, k, v, beta, log_a, cu_seqlens, scalar_decay, scale,
+                                  init_state, snap_interval, out, final_state,
+                                  snapshots if snap_interval else None, workspace)
+        self.device = q.device
+        self.out, self.final_state, self.snapshots, self.workspace = out, final_state, snapshots, workspace
+        lib()
+
+    def run(self, stages=(0, 2), stream=None):
+        st = ctypes.c_void_p(stream.cuda_stream) if stream is not None else _stream(self.device)
+        if tuple(stages) == (0, 2):
+            _check(_LIB.gdr_prefill(ctypes.byref(self.args), st), "gdr_prefill")
+        else:
+            _check(_LIB.gdr_prefill_stages(ctypes.byref(self.args), int(stages[0]), int(stages[1]), st),
+                   "gdr_prefill_stages")
 
 
 def prefill_status(workspace) -> None:

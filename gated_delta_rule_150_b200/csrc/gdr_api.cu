@@ -86,7 +86,8 @@ int64_t gdr_snapshot_count(const int32_t* host_cu, int n_seqs, int snap_interval
     return total;
 }
 
-gdr_status gdr_prefill(const gdr_prefill_args* a, void* stream) {
+gdr_status gdr_prefill_stages(const gdr_prefill_args* a, int first, int last, void* stream) {
+    if (first < 0 || last > 2 || first > last) return GDR_ERR_INVALID_ARG;
     gdr_status s = check_prefill_inputs(a);
     if (s != GDR_OK) return s;
     if (!a->final_state || !aligned16(a->final_state)) return GDR_ERR_INVALID_ARG;
@@ -103,15 +104,25 @@ gdr_status gdr_prefill(const gdr_prefill_args* a, void* stream) {
     uint32_t* err = reinterpret_cast<uint32_t*>(ws + lay.err_off);
     float* g = reinterpret_cast<float*>(ws + lay.g_off);
     uint8_t* rec = ws + lay.rec_off;
-    if (cudaMemsetAsync(err, 0, sizeof(uint32_t), st) != cudaSuccess) return GDR_ERR_CUDA;
+    if (first == 0 && cudaMemsetAsync(err, 0, sizeof(uint32_t), st) != cudaSuccess)
+        return GDR_ERR_CUDA;
     if (a->total_tokens > 0) {
-        s = from_cuda(gdr::launch_cumdecay(a->n_seqs, a->n_heads, a->d_k, a->total_tokens,
-                                           a->cu_seqlens, a->log_a, a->scalar_decay, g, st));
-        if (s != GDR_OK) return s;
-        s = from_cuda(gdr::launch_intra_chunk(*a, g, rec, err, st));
-        if (s != GDR_OK) return s;
+        if (first <= 0 && last >= 0) {
+            s = from_cuda(gdr::launch_cumdecay(a->n_seqs, a->n_heads, a->d_k, a->total_tokens,
+                                               a->cu_seqlens, a->log_a, a->scalar_decay, g, st));
+            if (s != GDR_OK) return s;
+        }
+        if (first <= 1 && last >= 1) {
+            s = from_cuda(gdr::launch_intra_chunk(*a, g, rec, err, st));
+            if (s != GDR_OK) return s;
+        }
     }
-    return from_cuda(gdr::launch_state_pass(*a, rec, err, st));
+    if (last >= 2) return from_cuda(gdr::launch_state_pass(*a, rec, err, st));
+    return GDR_OK;
+}
+
+gdr_status gdr_prefill(const gdr_prefill_args* a, void* stream) {
+    return gdr_prefill_stages(a, 0, 2, stream);
 }
 
 gdr_status gdr_prefill_status(const void* workspace, void* stream) {

@@ -125,6 +125,17 @@ int64_t gdr_snapshot_count(const int32_t* host_cu_seqlens, int n_seqs, int snap_
 gdr_status gdr_prefill(const gdr_prefill_args* args, void* stream);
 
 /*
+ * Enqueue only stages first..last (inclusive) of a prefill: 0 = chunk-local
+ * cumulative decay, 1 = intra-chunk factors, 2 = sequential inter-chunk pass.
+ * gdr_prefill(a) is gdr_prefill_stages(a, 0, 2).  A later stage reads what the
+ * earlier stages left in the workspace, so a range starting after 0 must
+ * follow a call that ran the stages before it with the same arguments.  Used
+ * to time the kernels one by one.  Errors as for gdr_prefill, plus
+ * GDR_ERR_INVALID_ARG for a bad stage range.
+ */
+gdr_status gdr_prefill_stages(const gdr_prefill_args* args, int first, int last, void* stream);
+
+/*
  * Status the device side of the most recent gdr_prefill on this workspace
  * recorded: GDR_OK, or GDR_ERR_TIMEOUT if a kernel abandoned a bounded wait
  * (its outputs are then undefined).  Synchronises `stream`.
