@@ -136,6 +136,29 @@ gdr_status gdr_prefill(const gdr_prefill_args* args, void* stream);
 gdr_status gdr_prefill_stages(const gdr_prefill_args* args, int first, int last, void* stream);
 
 /*
+ * gdr_prefill without a caller-provided workspace, for callers that cannot
+ * allocate device memory: code running under CUDA graph capture (cudaMalloc
+ * cannot be captured), plugins whose host framework owns all allocation, and
+ * serving paths where allocating is not allowed.  The pages have no
+ * counterpart; this is a property of the library, not of the method.
+ *
+ * The workspace is a fixed GDR_STATIC_WORKSPACE_BYTES array in the library's
+ * own device memory (held by every GPU that loads the library until the
+ * process exits).  args->workspace and args->workspace_bytes are ignored; every
+ * other field means what it means for gdr_prefill, and the results are the
+ * same.  A request whose workspace (gdr_prefill_workspace_size) exceeds
+ * GDR_STATIC_WORKSPACE_BYTES returns GDR_ERR_WORKSPACE and enqueues nothing.
+ * Nothing is allocated or freed.  The first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress) with that device current;
+ * make that first call before any stream capture.  All calls share the one
+ * array: calls that may overlap on the GPU (other streams, other host threads)
+ * race and must be serialised by the caller.  gdr_prefill_status needs a
+ * workspace pointer and does not apply to this path.
+ */
+#define GDR_STATIC_WORKSPACE_BYTES (64u << 20)
+gdr_status gdr_prefill_static_workspace(const gdr_prefill_args* args, void* stream);
+
+/*
  * Status the device side of the most recent gdr_prefill on this workspace
  * recorded: GDR_OK, or GDR_ERR_TIMEOUT if a kernel abandoned a bounded wait
  * (its outputs are then undefined).  Synchronises `stream`.
