@@ -81,7 +81,7 @@ def lib():
             L.gdr_cumdecay.restype = i
             L.gdr_cumdecay.argtypes = [i, i, i, i64, vp, vp, i, vp, vp]
             L.gdr_chunk_factors.restype = i
-            L.gdr_chunk_factors.argtypes = [ctypes.POINTER(PrefillArgs), vp, vp, vp, vp, vp, vp, vp]
+            L.gdr_chunk_factors.argtypes = [ctypes.POINTER(PrefillArgs), vp, vp, vp, vp, vp, vp]
             L.gdr_decode_step.restype = i
             L.gdr_decode_step.argtypes = [i, i, i, i, i, vp, vp, vp, vp, vp, i, f, vp, vp, vp]
             _LIB = L
@@ -259,22 +259,22 @@ def cumdecay(log_a, cu_seqlens, *, scalar_decay=False, d_k=None, out=None):
 
 
 def chunk_factors(q, k, v, beta, log_a, cu_seqlens, *, scalar_decay=False, scale=1.0):
-    """Intra-chunk factors (W, U, P, Qg, Kd, gamma) per chunk slot, fp32."""
+    """Per-chunk affine map of the state (Qt, PU, BS, NC, gamma) per chunk slot, fp32."""
     _need_cuda(q, k, v, beta, log_a, cu_seqlens)
     T, H, dk = q.shape
     dv = v.shape[-1]
     n = cu_seqlens.numel() - 1
     dev = q.device
     slots = T // 64 + n
-    f = dict(W=torch.zeros(slots, H, 64, dk, device=dev), U=torch.zeros(slots, H, 64, dv, device=dev),
-             P=torch.zeros(slots, H, 64, 64, device=dev), Qg=torch.zeros(slots, H, 64, dk, device=dev),
-             Kd=torch.zeros(slots, H, 64, dk, device=dev), gamma=torch.zeros(slots, H, dk, device=dev))
+    f = dict(Qt=torch.zeros(slots, H, 64, dk, device=dev), PU=torch.zeros(slots, H, 64, dv, device=dev),
+             BS=torch.zeros(slots, H, dk, dk, device=dev), NC=torch.zeros(slots, H, dv, dk, device=dev),
+             gamma=torch.zeros(slots, H, dk, device=dev))
     workspace = torch.empty(workspace_size(n, H, dk, dv, T, scalar_decay), dtype=torch.uint8,
                             device=dev)
     a = _prefill_args(q, k, v, beta, log_a, cu_seqlens, scalar_decay, scale, None, 0, None,
                       None, None, workspace)
-    _check(lib().gdr_chunk_factors(ctypes.byref(a), _ptr(f["W"]), _ptr(f["U"]), _ptr(f["P"]),
-                                   _ptr(f["Qg"]), _ptr(f["Kd"]), _ptr(f["gamma"]), _stream(dev)),
+    _check(lib().gdr_chunk_factors(ctypes.byref(a), _ptr(f["Qt"]), _ptr(f["PU"]), _ptr(f["BS"]),
+                                   _ptr(f["NC"]), _ptr(f["gamma"]), _stream(dev)),
            "gdr_chunk_factors")
     return f
 

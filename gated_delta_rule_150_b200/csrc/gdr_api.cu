@@ -117,7 +117,7 @@ gdr_status gdr_prefill_stages(const gdr_prefill_args* a, int first, int last, vo
             if (s != GDR_OK) return s;
         }
     }
-    if (last >= 2) return from_cuda(gdr::launch_state_pass(*a, rec, err, st));
+    if (last >= 2) return from_cuda(gdr::launch_state_pass(*a, rec, lay, ws, err, st));
     return GDR_OK;
 }
 
@@ -148,15 +148,15 @@ gdr_status gdr_cumdecay(int n_seqs, int n_heads, int d_k, int64_t total_tokens,
                                           scalar_decay, g, static_cast<cudaStream_t>(stream)));
 }
 
-gdr_status gdr_chunk_factors(const gdr_prefill_args* a, float* W, float* U, float* P,
-                             float* Qg, float* Kd, float* gamma, void* stream) {
+gdr_status gdr_chunk_factors(const gdr_prefill_args* a, float* Qt, float* PU, float* BS,
+                             float* NC, float* gamma, void* stream) {
     gdr_status s = check_prefill_inputs(a);
     if (s != GDR_OK) return s;
     WorkspaceLayout lay;
     s = check_workspace(a, &lay);
     if (s != GDR_OK) return s;
     if (a->n_seqs == 0 || a->total_tokens == 0) return GDR_OK;
-    const void* outs[] = {W, U, P, Qg, Kd, gamma};
+    const void* outs[] = {Qt, PU, BS, NC, gamma};
     for (const void* p : outs)
         if (!p || !aligned16(p)) return GDR_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -170,7 +170,7 @@ gdr_status gdr_chunk_factors(const gdr_prefill_args* a, float* W, float* U, floa
     if (s != GDR_OK) return s;
     s = from_cuda(gdr::launch_intra_chunk(*a, g, rec, err, st));
     if (s != GDR_OK) return s;
-    return from_cuda(gdr::launch_unpack_records(*a, rec, W, U, P, Qg, Kd, gamma, st));
+    return from_cuda(gdr::launch_unpack_records(*a, rec, Qt, PU, BS, NC, gamma, st));
 }
 
 gdr_status gdr_decode_step(int batch, int n_heads, int d_k, int d_v, gdr_dtype qkv_dtype,

@@ -20,34 +20,65 @@ inline int64_t n_chunk_slots(int64_t total_tokens, int n_seqs) {
 }
 
 // One chunk-head record of the workspace, written by the intra-chunk kernel
-// and read whole (one bulk copy) by the state-pass kernel.  Every image is a
-// tensor-core operand tile in the K-major 128-byte-swizzle layout (sm100.cuh),
-// so the bytes land in shared memory ready to use.
+// and read by the state-pass kernel.  With S0 the chunk's start state
+// (d_v x d_k), the chunk's effect is affine in S0:
+//     S_next = S0 Diag(gamma) + S0 BS^T + NC        O = Qt S0^T + PU
+// so the sequential pass needs one product per chunk for the state.
+// Qt and BS are tensor-core operand tiles (K-major, 128-byte swizzle, see
+// sm100.cuh); PU and NC are read row by row by threads (same swizzle of their
+// 16-byte chunks, so rows read without bank conflicts).
 struct RecordLayout {
-    uint32_t W;       // [64 x D]  rows = token r, cols = key channel   (W)
-    uint32_t Qg;      // [64 x D]  rows = token r, cols = key channel   (scale q exp(g))
-    uint32_t Kt;      // [D x 64]  rows = key channel, cols = token i   (Kd transposed)
-    uint32_t Ut;      // [D x 64]  rows = value channel, cols = token i (U transposed)
-    uint32_t P;       // [64 x 64] rows = token r, cols = token i       (masked Q K^T decay)
-    uint32_t gamma;   // [D] fp32  exp(g_last)
-    uint32_t bytes;   // total, a multiple of 1024
+    uint32_t Qt;      // [64 x D]  row r: scale q_r exp(g_r) - (P W)_r        (bf16)
+    uint32_t BS;      // [D x D]   row c': -(Kd^T W)[c', :]                    (bf16)
+    uint32_t PU;      // [64 x D]  row r: (P U)_r                              (bf16)
+    uint32_t NC;      // [D x D]   row v: (U^T Kd)[v, :]                       (bf16)
+    uint32_t gamma;   // [D]       exp(g_last)                                 (fp32)
+    uint32_t bytes;   // total, a multiple of 256
 };
 
 __host__ __device__ constexpr RecordLayout record_layout(int D) {
     return RecordLayout{0u,
-                        (uint32_t)(D * 128),
-                        (uint32_t)(2 * D * 128),
-                        (uint32_t)(3 * D * 128),
-                        (uint32_t)(4 * D * 128),
-                        (uint32_t)(4 * D * 128 + 8192),
-                        (uint32_t)(4 * D * 128 + 8192 + 1024)};
+                        (uint32_t)(128 * D),
+                        (uint32_t)(128 * D + 2 * D * D),
+                        (uint32_t)(256 * D + 2 * D * D),
+                        (uint32_t)(256 * D + 4 * D * D),
+                        (uint32_t)(((256 * D + 4 * D * D + 4 * D) + 255) / 256 * 256)};
+}
+
+// Sequence segmentation of the sequential pass.  With few (sequence, head)
+// pairs the chunk-to-chunk chain leaves most SMs idle, so each sequence is cut
+// into segments of seg_chunks chunks: every segment first runs from a zero
+// state while also carrying the identity (its chunks' composed affine map
+// S_end = S_start M + N), a short fp32 chain combines the maps into each
+// segment's true start state, and every segment then replays its chunks from
+// that state to produce its outputs.  seg_chunks == 0 means one pass.
+inline int segment_chunks(int n_seqs, int H, int64_t T) {
+    if (n_seqs <= 0 || T <= 0) return 0;
+    const int64_t pairs = (int64_t)n_seqs * H;
+    const int64_t target_ctas = 2 * 148;
+    int64_t segs = (target_ctas + pairs - 1) / pairs;
+    if (segs > 32) segs = 32;
+    const int64_t avg_chunks = (T / n_seqs + kChunk - 1) / kChunk;
+    int64_t sc = (avg_chunks + segs - 1) / segs;
+    if (sc < 8) sc = 8;
+    if (segs <= 1 || sc >= avg_chunks) return 0;
+    return (int)sc;
+}
+
+// Segment slot of segment j of sequence n: floor(cu[n] / span) + j + n with
+// span = 64 seg_chunks tokens (same collision-free scheme as chunk slots).
+inline int64_t n_segment_slots(int64_t total_tokens, int n_seqs, int seg_chunks) {
+    return seg_chunks > 0 ? total_tokens / ((int64_t)kChunk * seg_chunks) + n_seqs : 0;
 }
 
 struct WorkspaceLayout {
     size_t err_off;     // uint32 error word (0 = ok)
     size_t g_off;       // fp32 cumulative log decay, same layout as log_a
     size_t rec_off;     // chunk-head records
+    size_t seg_off;     // per (segment slot, head): N, M, E, each [D x D] fp32
     int64_t n_slots;
+    int64_t n_seg_slots;
+    int seg_chunks;
     size_t rec_bytes;
     size_t total;
 };
@@ -62,7 +93,10 @@ inline WorkspaceLayout workspace_layout(int n_seqs, int H, int D, int64_t T, int
     w.rec_off = align_up(w.g_off + g_elems * sizeof(float), 1024);
     w.n_slots = n_chunk_slots(T, n_seqs);
     w.rec_bytes = record_layout(D).bytes;
-    w.total = w.rec_off + (size_t)w.n_slots * (size_t)H * w.rec_bytes;
+    w.seg_off = align_up(w.rec_off + (size_t)w.n_slots * (size_t)H * w.rec_bytes, 1024);
+    w.seg_chunks = segment_chunks(n_seqs, H, T);
+    w.n_seg_slots = n_segment_slots(T, n_seqs, w.seg_chunks);
+    w.total = w.seg_off + (size_t)w.n_seg_slots * (size_t)H * 3u * (size_t)D * D * sizeof(float);
     return w;
 }
 
@@ -74,11 +108,12 @@ cudaError_t launch_intra_chunk(const gdr_prefill_args& a, const float* g, uint8_
                                uint32_t* err, cudaStream_t st);
 
 cudaError_t launch_state_pass(const gdr_prefill_args& a, const uint8_t* records,
-                              uint32_t* err, cudaStream_t st);
+                              const WorkspaceLayout& lay, uint8_t* ws, uint32_t* err,
+                              cudaStream_t st);
 
 cudaError_t launch_unpack_records(const gdr_prefill_args& a, const uint8_t* records,
-                                  float* W, float* U, float* P, float* Qg, float* Kd,
-                                  float* gamma, cudaStream_t st);
+                                  float* Qt, float* PU, float* BS, float* NC, float* gamma,
+                                  cudaStream_t st);
 
 cudaError_t launch_decode(int B, int H, int dk, int dv, gdr_dtype dt, const void* q,
                           const void* k, const void* v, const float* beta,
@@ -88,23 +123,29 @@ cudaError_t launch_decode(int B, int H, int dk, int dv, gdr_dtype dt, const void
 // Device helper: slot -> (sequence, chunk index).  f(n) = floor(cu[n]/64) + n is
 // strictly increasing, so the owner of slot j is the largest n with f(n) <= j.
 // Returns false if the slot holds no chunk.
-__device__ __forceinline__ bool slot_to_chunk(const int32_t* __restrict__ cu, int n_seqs,
-                                              int64_t slot, int* seq, int* start, int* len) {
+__device__ __forceinline__ bool slot_to_span(const int32_t* __restrict__ cu, int n_seqs,
+                                             int64_t slot, int span, int* seq, int* start,
+                                             int* len) {
     int lo = 0, hi = n_seqs - 1, found = -1;
     while (lo <= hi) {
         const int mid = (lo + hi) >> 1;
-        const int64_t f = (int64_t)(__ldg(cu + mid) / kChunk) + mid;
+        const int64_t f = (int64_t)(__ldg(cu + mid) / span) + mid;
         if (f <= slot) { found = mid; lo = mid + 1; } else { hi = mid - 1; }
     }
     if (found < 0) return false;
     const int s0 = __ldg(cu + found), s1 = __ldg(cu + found + 1);
-    const int64_t c = slot - ((int64_t)(s0 / kChunk) + found);
-    const int64_t st = (int64_t)s0 + c * kChunk;
+    const int64_t c = slot - ((int64_t)(s0 / span) + found);
+    const int64_t st = (int64_t)s0 + c * span;
     if (st >= s1) return false;
     *seq = found;
     *start = (int)st;
-    *len = (int)((s1 - st) < kChunk ? (s1 - st) : kChunk);
+    *len = (int)((s1 - st) < span ? (s1 - st) : span);
     return true;
+}
+
+__device__ __forceinline__ bool slot_to_chunk(const int32_t* __restrict__ cu, int n_seqs,
+                                              int64_t slot, int* seq, int* start, int* len) {
+    return slot_to_span(cu, n_seqs, slot, kChunk, seq, start, len);
 }
 
 __host__ __device__ inline int64_t chunk_slot(int32_t seq_start, int seq, int chunk_idx) {

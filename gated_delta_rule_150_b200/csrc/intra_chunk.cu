@@ -11,30 +11,32 @@
 //     T      = (I + A)^-1                  (forward substitution, fp32)
 //     W      = T diag(b) (K * Gamma)       U = T diag(b) V
 //     Qg     = scale Q * Gamma             Kd = K * exp(g_last - g)
-//     gamma  = exp(g_last)
-// Nothing here depends on S0, so every (chunk, head) is independent: one CTA
-// each, all in parallel.  The sequential pass (state_pass.cu) then needs only
-// Delta = U - W S0^T, O = Qg S0^T + P Delta, S = S0 Diag(gamma) + Delta^T Kd.
+// so that Delta = U - W S0^T, O = Qg S0^T + P Delta and
+// S_next = S0 Diag(gamma) + Delta^T Kd with gamma = exp(g_last).  The chunk's
+// effect is affine in S0, and this kernel also forms the four S0-free
+// matrices of that map,
+//     Qt = Qg - P W,  PU = P U,  BS = -Kd^T W,  NC = U^T Kd,
+// so that the sequential pass (state_pass.cu) is left with
+//     S_next = S0 Diag(gamma) + S0 BS^T + NC,   O = Qt S0^T + PU,
+// one tensor-core product per chunk on its critical path.  Nothing here
+// depends on S0: one CTA per (chunk, head), all in parallel.
 //
 // Tensor cores.  A and P are decay-weighted K K^T / Q K^T products.  With a
-// per-channel decay (KDA) the weight exp(g[r,c] - g[i,c]) does not factor into
-// a bounded row term times a bounded column term over a whole chunk (g can
-// fall by hundreds over 64 tokens), so the chunk is cut into four 16-token
-// blocks, each with a reference point m_b = g at the middle of block b:
+// per-channel decay (KDA) exp(g[r,c] - g[i,c]) does not factor into a bounded
+// row term times a bounded column term over a whole chunk (g can fall by
+// hundreds over 64 tokens), so the chunk is cut into four 16-token blocks with
+// reference points m_b = g at the middle of block b:
 //     exp(g_r - g_i) = exp(g_r - m_b(r)) * exp(m_b(r) - m_b(i)) * exp(m_b(i) - g_i)
-// The outer factors are bounded by exp(half a block's decay); the middle one
-// is <= 1 and is folded into the key operand of query block b(r).  One
-// tcgen05 MMA per query block b (M = 128 rows: the 64 scaled queries stacked
-// on the 64 scaled keys, N = 16(b+1) keys, K = d_k) yields P and A together.
-// A chunk whose half-block decay exceeds exp(80) in some channel (log decay
-// below about -10 per token) would overflow fp32 in that form; it takes an
-// exact elementwise path instead.  With a scalar decay (Gated DeltaNet) the
-// weight is exp(g_r - g_i) for the whole row and is applied after one plain
-// Q K^T / K K^T MMA.  W and U come from one more MMA, W^T | U^T =
-// [diag(b)(K*Gamma) | diag(b)V]^T T^T, with T rounded to bf16.
-//
-// Outputs go to the chunk-head record of the workspace in tensor-core operand
-// layout (internal.h), ready for the state pass to load with one bulk copy.
+// The outer factors are bounded by exp(half a block's decay) and the middle
+// one is <= 1; it is folded into the key operand of query block b(r).  One
+// tcgen05 MMA per query block b (M = 128: the 64 scaled queries stacked on the
+// 64 scaled keys, N = 16(b+1) keys, K = d_k) yields P and A together.  A chunk
+// whose half-block decay exceeds exp(80) in some channel (log decay below
+// about -10 per token) would overflow fp32 in that form; it takes an exact
+// elementwise path instead.  With a scalar decay (Gated DeltaNet) the weight
+// exp(g_r - g_i) is applied after one plain Q K^T / K K^T MMA.  W and U come
+// from [W | U]^T = [diag(b)(K*Gamma) | diag(b)V]^T T^T with T rounded to
+// bf16; P [W | U], Kd^T W and U^T Kd are three more MMAs.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -45,46 +47,65 @@ namespace {
 
 constexpr int kThreads = 128;
 constexpr float kMaxFactorExp = 80.f;
-constexpr uint32_t kTmemCols = 256;
+constexpr int kLd = 68;                       // row stride (floats) of the fp32 64x64 tiles
 
 __host__ __device__ constexpr uint32_t al1024(uint32_t x) { return (x + 1023u) & ~1023u; }
 __host__ __device__ constexpr uint32_t umax(uint32_t a, uint32_t b) { return a > b ? a : b; }
 
-template <int D, bool SCALAR>
-struct IntraSmem {
-    static constexpr uint32_t XA = 0;                         // bf16 [128 x D] scaled [Q; K]
-    static constexpr uint32_t KT0 = 256 * D;                  // key tiles, 16(b+1) rows each
-    static constexpr uint32_t op_bytes = SCALAR ? 256 * D : 256 * D + 320 * D;
-    static constexpr uint32_t Pf = 0;                         // fp32 [64][65], after MMA 1
-    static constexpr uint32_t Wst = 17408;                    // bf16 W image [64 x D]
-    static constexpr uint32_t region0 = al1024(umax(op_bytes, Wst + 128 * D));
-    static constexpr uint32_t Bt = region0;                   // bf16 [2D x 64]
-    static constexpr uint32_t Tb = Bt + 256 * D;              // bf16 [64 x 64]
-    static constexpr uint32_t As = Tb + 8192;                 // fp32 [64][65]
-    static constexpr uint32_t Ts = As + 16896;                // fp32 [64][65]
-    static constexpr uint32_t Yt = Ts + 16896;                // fp32 [3][16][16]
-    static constexpr uint32_t Gl = Yt + 3072;                 // fp32 [D] g_last
-    static constexpr uint32_t Bs = Gl + 4 * D;                // fp32 [64] beta
-    static constexpr uint32_t Gs = Bs + 256;                  // fp32 [64] g (scalar decay)
-    static constexpr uint32_t bytes = Gs + 256;
-    static constexpr uint32_t dyn_bytes = bytes + 1024;
-    __host__ __device__ static constexpr uint32_t kt_off(int b) { return KT0 + 32u * D * (uint32_t)(b * (b + 1) / 2); }
+template <int D, typename InT, bool SCALAR>
+struct IntraLayout {
+    static constexpr uint32_t elem = sizeof(InT);
+    // fp32 q/k/v at d 128 do not fit next to everything else: read from global
+    static constexpr bool kStageQKV = !(elem == 4 && D == 128);
+    // region 1: staged inputs (operand phase), then Ts, Yt, WUt
+    static constexpr uint32_t sQ = 0;
+    static constexpr uint32_t sK = sQ + (kStageQKV ? 64u * D * elem : 0u);
+    static constexpr uint32_t sV = sK + (kStageQKV ? 64u * D * elem : 0u);
+    static constexpr uint32_t sG = sV + (kStageQKV ? 64u * D * elem : 0u);
+    static constexpr uint32_t in_bytes = sG + (SCALAR ? 0u : 64u * D * 4u);
+    static constexpr uint32_t Ts = 0;                         // fp32 [64][kLd]
+    static constexpr uint32_t Yt = Ts + 64u * kLd * 4u;       // fp32 [3][16][16]
+    static constexpr uint32_t WUt = al1024(Yt + 3072u);       // bf16 [2D][64]
+    static constexpr uint32_t r1 = al1024(umax(in_bytes, WUt + 256u * D));
+    // region 2: A/P operands, then As, Pt, Tb
+    static constexpr uint32_t XA = r1;                        // bf16 [128][D]
+    static constexpr uint32_t KT0 = XA + 256u * D;            // key tiles, 16(b+1) rows each
+    static constexpr uint32_t op_bytes = SCALAR ? 256u * D : 576u * D;
+    static constexpr uint32_t As = r1;                        // fp32 [64][kLd]
+    static constexpr uint32_t Pt = r1 + 64u * kLd * 4u;       // bf16 [64][64]
+    static constexpr uint32_t Tb = Pt + 8192u;                // bf16 [64][64]
+    static constexpr uint32_t r2 = al1024(umax(op_bytes, 64u * kLd * 4u + 16384u));
+    // region 3: live throughout
+    static constexpr uint32_t Bt = r1 + r2;                   // bf16 [2D][64]
+    static constexpr uint32_t Kdt = Bt + 256u * D;            // bf16 [D][64]
+    static constexpr uint32_t Qgs = Kdt + 128u * D;           // bf16 [64][D]
+    static constexpr uint32_t Gl = Qgs + 128u * D;            // fp32 [D] g_last
+    static constexpr uint32_t Bs = Gl + 4u * D;               // fp32 [64] beta
+    static constexpr uint32_t Gs = Bs + 256u;                 // fp32 [64] g (scalar decay)
+    static constexpr uint32_t bytes = Gs + 256u;
+    static constexpr uint32_t dyn_bytes = bytes + 1024u;
+    __host__ __device__ static constexpr uint32_t kt_off(int b) {
+        return KT0 + 32u * D * (uint32_t)(b * (b + 1) / 2);
+    }
+    static_assert(dyn_bytes <= 232448u, "shared memory budget");
+    static_assert((64u * kLd * 4u) % 1024u == 0u, "Pt alignment");
 };
 
+// TMEM column of query block b's A/P product (16(b+1) columns each).
 __host__ __device__ constexpr uint32_t ap_col(int b) { return (uint32_t)(8 * b * (b + 1)); }
 
 template <typename T> struct Vec8;
 template <> struct Vec8<__nv_bfloat16> {
     static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&x)[8]) {
-        const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+        const uint4 u = *reinterpret_cast<const uint4*>(p);
         float2 a = unpack_bf16(u.x), b = unpack_bf16(u.y), c = unpack_bf16(u.z), d = unpack_bf16(u.w);
         x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y; x[4] = c.x; x[5] = c.y; x[6] = d.x; x[7] = d.y;
     }
 };
 template <> struct Vec8<float> {
     static __device__ __forceinline__ void load(const float* p, float (&x)[8]) {
-        const float4 a = __ldg(reinterpret_cast<const float4*>(p));
-        const float4 b = __ldg(reinterpret_cast<const float4*>(p + 4));
+        const float4 a = *reinterpret_cast<const float4*>(p);
+        const float4 b = *reinterpret_cast<const float4*>(p + 4);
         x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
     }
 };
@@ -98,17 +119,67 @@ __device__ __forceinline__ uint4 pack8(const float (&x)[8]) {
     return u;
 }
 
+__device__ __forceinline__ float4 f4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+
+// Stage one [64 x D] row block of a token-major tensor into shared memory
+// (rows past the chunk end are zero-filled).
+template <typename T, int D>
+__device__ __forceinline__ void stage_rows(uint8_t* dst, const T* src, size_t tok_stride, int len,
+                                           int tid) {
+    constexpr int CPR = D * (int)sizeof(T) / 16;              // 16-byte chunks per row
+    for (int idx = tid; idx < 64 * CPR; idx += kThreads) {
+        const int r = idx / CPR, j = idx % CPR;
+        const int rs = r < len ? r : len - 1;
+        cp_async16(dst + (size_t)r * D * sizeof(T) + 16 * j,
+                   reinterpret_cast<const uint8_t*>(src + (size_t)rs * tok_stride) + 16 * j,
+                   r < len ? 16u : 0u);
+    }
+}
+
+// Read the A/P products of this thread's row from TMEM (per-channel decay).
+// Lanes of warp parity `par` own rows 32 par .. 32 par + 31, i.e. query
+// blocks 2 par and 2 par + 1, whose columns are loaded together.
+template <int PAR>
+__device__ __forceinline__ void load_ap_row(uint32_t taddr, int b, float (&v)[64]) {
+    constexpr int blo = 2 * PAR;
+    constexpr int wlo = 16 * (blo + 1);
+    constexpr int c0 = (int)ap_col(blo);
+    constexpr int ncol = 16 * (blo + 1) + 16 * (blo + 2);     // 48 or 112
+    float u[ncol];
+    if (PAR == 0) {
+        float* a = u;
+        tmem_ld32(taddr + 0, *reinterpret_cast<float(*)[32]>(a));
+        tmem_ld16(taddr + 32, *reinterpret_cast<float(*)[16]>(a + 32));
+    } else {
+        float* a = u;
+        tmem_ld16(taddr + 48, *reinterpret_cast<float(*)[16]>(a));
+        tmem_ld32(taddr + 64, *reinterpret_cast<float(*)[32]>(a + 16));
+        tmem_ld32(taddr + 96, *reinterpret_cast<float(*)[32]>(a + 48));
+        tmem_ld32(taddr + 128, *reinterpret_cast<float(*)[32]>(a + 80));
+    }
+    (void)c0;
+    tmem_ld_wait();
+    const bool lo = (b == blo);
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+        const float x_lo = (i < wlo) ? u[i] : 0.f;
+        const float x_hi = (wlo + i < ncol) ? u[(wlo + i < ncol) ? wlo + i : 0] : 0.f;
+        v[i] = lo ? x_lo : x_hi;
+    }
+}
+
 template <int D, typename InT, bool SCALAR>
 __global__ void __launch_bounds__(kThreads)
 intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                    const InT* __restrict__ q, const InT* __restrict__ k, const InT* __restrict__ v,
                    const float* __restrict__ beta, const float* __restrict__ g, float scale,
                    uint8_t* __restrict__ records, uint32_t* err) {
-    using L = IntraSmem<D, SCALAR>;
+    using L = IntraLayout<D, InT, SCALAR>;
     constexpr RecordLayout R = record_layout(D);
     constexpr int CG = D / 8;              // channel groups of 8
     constexpr int RG = kThreads / CG;      // row groups
     constexpr int RPT = 64 / RG;           // rows per thread: 4 (D=64) or 8 (D=128)
+    constexpr uint32_t kTmemCols = (D == 64) ? 256u : 512u;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -120,14 +191,16 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     const int h = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     uint8_t* rec = records + ((size_t)blockIdx.x * H + h) * R.bytes;
+    const size_t tok_stride = (size_t)H * D;
+    const size_t base = (size_t)start * tok_stride + (size_t)h * D;
 
     float* As = reinterpret_cast<float*>(sm + L::As);
     float* Ts = reinterpret_cast<float*>(sm + L::Ts);
-    float* Pf = reinterpret_cast<float*>(sm + L::Pf);
     float* Yt = reinterpret_cast<float*>(sm + L::Yt);
     float* Gl = reinterpret_cast<float*>(sm + L::Gl);
     float* Bs = reinterpret_cast<float*>(sm + L::Bs);
     float* Gs = reinterpret_cast<float*>(sm + L::Gs);
+    const float* sG = reinterpret_cast<const float*>(sm + L::sG);
 
     if (tid == 0) {
         mbar_init(&mma_bar, 1);
@@ -135,27 +208,39 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     }
     if (warp == 0) tmem_alloc(&tmem_slot, kTmemCols);
 
+    // ---- stage the chunk's inputs in shared memory -------------------------
+    if (L::kStageQKV) {
+        stage_rows<InT, D>(sm + L::sQ, q + base, tok_stride, len, tid);
+        stage_rows<InT, D>(sm + L::sK, k + base, tok_stride, len, tid);
+        stage_rows<InT, D>(sm + L::sV, v + base, tok_stride, len, tid);
+    }
+    if (!SCALAR) stage_rows<float, D>(sm + L::sG, g + base, tok_stride, len, tid);
+    if (tid < 64) {
+        Bs[tid] = tid < len ? __ldg(beta + (size_t)(start + tid) * H + h) : 0.f;
+        if (SCALAR) {
+            const float glast = __ldg(g + (size_t)(start + len - 1) * H + h);
+            Gs[tid] = tid < len ? __ldg(g + (size_t)(start + tid) * H + h) : glast;
+        }
+    }
+    cp_async_wait_all();
+    __syncthreads();
+
     const int cg = tid % CG, rg = tid / CG, c0 = 8 * cg;
     const int r0 = rg * RPT;
     const int jb = r0 / 16;                                   // this thread's 16-row block
-    const size_t tok_stride = (size_t)H * D;
-    const InT* qh = q + (size_t)start * tok_stride + (size_t)h * D + c0;
-    const InT* kh = k + (size_t)start * tok_stride + (size_t)h * D + c0;
-    const InT* vh = v + (size_t)start * tok_stride + (size_t)h * D + c0;
 
-    // ---- phase 1: reference points and the overflow check -------------------
-    float gl[8], mj[8];                       // g_last and m_{jb} for this thread's channels
+    // ---- reference points and the overflow check ---------------------------
+    float gl[8], mj[8];
     float ecross[4][8];                       // exp(m_b - m_jb) for b > jb (per-channel)
     bool bad = false;
     if (!SCALAR) {
-        const float* gh = g + (size_t)start * tok_stride + (size_t)h * D + c0;
-        load8f(gh + (size_t)(len - 1) * tok_stride, gl);
-        load8f(gh + (size_t)min(16 * jb + 8, len - 1) * tok_stride, mj);
+        load8f(sG + (size_t)(len - 1) * D + c0, gl);
+        load8f(sG + (size_t)min(16 * jb + 8, len - 1) * D + c0, mj);
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
             if (b > jb) {
                 float mb[8];
-                load8f(gh + (size_t)min(16 * b + 8, len - 1) * tok_stride, mb);
+                load8f(sG + (size_t)min(16 * b + 8, len - 1) * D + c0, mb);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) ecross[b][e] = expf(mb[e] - mj[e]);
             }
@@ -163,32 +248,30 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
 #pragma unroll
         for (int u = 0; u < RPT; ++u) {
             const int r = r0 + u;
-            float gr[8];
-            if (r < len) load8f(gh + (size_t)r * tok_stride, gr);
-            else {
+            if (r < len) {
+                float gr[8];
+                load8f(sG + (size_t)r * D + c0, gr);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) gr[e] = gl[e];
+                for (int e = 0; e < 8; ++e) bad |= fabsf(gr[e] - mj[e]) > kMaxFactorExp;
             }
-#pragma unroll
-            for (int e = 0; e < 8; ++e) bad |= fabsf(gr[e] - mj[e]) > kMaxFactorExp;
         }
         if (rg == 0) {
 #pragma unroll
             for (int e = 0; e < 8; ++e) Gl[c0 + e] = gl[e];
         }
     } else {
-        const float glast = __ldg(g + (size_t)(start + len - 1) * H + h);
+        const float glast = Gs[63 < len - 1 ? 63 : len - 1];
 #pragma unroll
         for (int e = 0; e < 8; ++e) gl[e] = glast;
-        if (tid < 64) Gs[tid] = tid < len ? __ldg(g + (size_t)(start + tid) * H + h) : glast;
         if (tid < D) Gl[tid] = glast;
     }
-    if (tid < 64) Bs[tid] = tid < len ? __ldg(beta + (size_t)(start + tid) * H + h) : 0.f;
     const bool bad_chunk = __syncthreads_or(bad);
 
-    // ---- phase 2: operands and the elementwise outputs ----------------------
+    // ---- operands and per-token outputs -------------------------------------
     uint8_t* XA = sm + L::XA;
     uint8_t* Bt = sm + L::Bt;
+    uint8_t* Kdt = sm + L::Kdt;
+    uint8_t* Qgs = sm + L::Qgs;
     float em[8], eld[8];        // exp(m_jb), exp(g_last - m_jb)
     if (!SCALAR) {
 #pragma unroll
@@ -201,16 +284,20 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         const bool valid = r < len;
         float qv[8], kv[8], vv[8], gr[8];
         const float br = Bs[r];
-        if (valid) {
-            Vec8<InT>::load(qh + (size_t)r * tok_stride, qv);
-            Vec8<InT>::load(kh + (size_t)r * tok_stride, kv);
-            Vec8<InT>::load(vh + (size_t)r * tok_stride, vv);
+        if (L::kStageQKV) {
+            Vec8<InT>::load(reinterpret_cast<const InT*>(sm + L::sQ) + (size_t)r * D + c0, qv);
+            Vec8<InT>::load(reinterpret_cast<const InT*>(sm + L::sK) + (size_t)r * D + c0, kv);
+            Vec8<InT>::load(reinterpret_cast<const InT*>(sm + L::sV) + (size_t)r * D + c0, vv);
+        } else if (valid) {
+            Vec8<InT>::load(q + base + (size_t)r * tok_stride + c0, qv);
+            Vec8<InT>::load(k + base + (size_t)r * tok_stride + c0, kv);
+            Vec8<InT>::load(v + base + (size_t)r * tok_stride + c0, vv);
         } else {
 #pragma unroll
             for (int e = 0; e < 8; ++e) qv[e] = kv[e] = vv[e] = 0.f;
         }
         if (!SCALAR) {
-            if (valid) load8f(g + (size_t)(start + r) * tok_stride + (size_t)h * D + c0, gr);
+            if (valid) load8f(sG + (size_t)r * D + c0, gr);
             else {
 #pragma unroll
                 for (int e = 0; e < 8; ++e) gr[e] = gl[e];
@@ -258,8 +345,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                 *reinterpret_cast<uint4*>(sm + L::kt_off(b) + sw128_chunk(16 * (b + 1), r, cg)) = pack8(kb);
             }
         }
-        // Qg image row r (global record)
-        *reinterpret_cast<uint4*>(rec + R.Qg + sw128_chunk(64, r, cg)) = pack8(qg);
+        *reinterpret_cast<uint4*>(Qgs + sw128_chunk(64, r, cg)) = pack8(qg);
         // transposed operands: collect pairs of rows per channel
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -275,7 +361,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
             }
         }
     }
-    // B1^T rows c (token columns r0..r0+RPT-1), B2^T rows D + c, Kd^T image rows c
+    // B1^T rows c, B2^T rows D + c, Kd^T rows c; token columns r0 .. r0 + RPT - 1
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
         const int c = c0 + e;
@@ -285,11 +371,11 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         if (RPT == 8) {
             *reinterpret_cast<uint4*>(Bt + o1) = make_uint4(pb1[e][0], pb1[e][1], pb1[e][2 % (RPT / 2)], pb1[e][3 % (RPT / 2)]);
             *reinterpret_cast<uint4*>(Bt + o2) = make_uint4(pb2[e][0], pb2[e][1], pb2[e][2 % (RPT / 2)], pb2[e][3 % (RPT / 2)]);
-            *reinterpret_cast<uint4*>(rec + R.Kt + o3) = make_uint4(pkd[e][0], pkd[e][1], pkd[e][2 % (RPT / 2)], pkd[e][3 % (RPT / 2)]);
+            *reinterpret_cast<uint4*>(Kdt + o3) = make_uint4(pkd[e][0], pkd[e][1], pkd[e][2 % (RPT / 2)], pkd[e][3 % (RPT / 2)]);
         } else {
             *reinterpret_cast<uint2*>(Bt + o1) = make_uint2(pb1[e][0], pb1[e][1 % (RPT / 2)]);
             *reinterpret_cast<uint2*>(Bt + o2) = make_uint2(pb2[e][0], pb2[e][1 % (RPT / 2)]);
-            *reinterpret_cast<uint2*>(rec + R.Kt + o3) = make_uint2(pkd[e][0], pkd[e][1 % (RPT / 2)]);
+            *reinterpret_cast<uint2*>(Kdt + o3) = make_uint2(pkd[e][0], pkd[e][1 % (RPT / 2)]);
         }
     }
     fence_proxy_async_smem();
@@ -299,7 +385,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     const uint32_t tmem = tmem_slot;
     const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
 
-    // ---- phase 3: decay-weighted Q K^T and K K^T on the tensor cores --------
+    // ---- decay-weighted Q K^T and K K^T on the tensor cores ------------------
     if (tid == 0) {
         const uint32_t aXA = smem_u32(XA);
         if (!SCALAR) {
@@ -323,119 +409,143 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     bool failed = !mbar_wait(&mma_bar, 0);
     tc_fence_after_sync();
 
-    // ---- phase 4: P (masked) and A (masked, times beta) into fp32 smem ------
+    // ---- P (masked, bf16 operand) and A (masked, times beta, fp32) ----------
     {
         const bool is_p = warp < 2;
         const int rr = 32 * (warp & 1) + lane;                // chunk row
-        float* dst = is_p ? Pf : As;
-        const float scl = is_p ? 1.f : Bs[rr];
-#pragma unroll 4
-        for (int i = 0; i < 64; ++i) dst[rr * 65 + i] = 0.f;
+        const int lim = is_p ? rr : rr - 1;                   // last valid key index
+        float vrow[64];
         if (!SCALAR) {
-            const int b = rr >> 4;
-            const int off = (int)ap_col(b), width = 16 * (b + 1);
-            const int lim = is_p ? rr : rr - 1;               // last valid key index
-#pragma unroll
-            for (int p = 0; p < 5; ++p) {
-                float x[32];
-                tmem_ld32(tmem + lane_base + 32 * p, x);
-                tmem_ld_wait();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int i = 32 * p + j - off;
-                    if (i >= 0 && i < width && i <= lim) dst[rr * 65 + i] = scl * x[j];
-                }
-            }
+            if ((warp & 1) == 0) load_ap_row<0>(tmem + lane_base, rr >> 4, vrow);
+            else load_ap_row<1>(tmem + lane_base, rr >> 4, vrow);
         } else {
+            tmem_ld32(tmem + lane_base, *reinterpret_cast<float(*)[32]>(vrow));
+            tmem_ld32(tmem + lane_base + 32, *reinterpret_cast<float(*)[32]>(vrow + 32));
+            tmem_ld_wait();
             const float gr = Gs[rr];
-            const int lim = is_p ? rr : rr - 1;
 #pragma unroll
-            for (int p = 0; p < 2; ++p) {
-                float x[32];
-                tmem_ld32(tmem + lane_base + 32 * p, x);
-                tmem_ld_wait();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int i = 32 * p + j;
-                    if (i <= lim) dst[rr * 65 + i] = scl * x[j] * expf(gr - Gs[i]);
-                }
-            }
+            for (int i = 0; i < 64; ++i) vrow[i] = (i <= lim) ? vrow[i] * expf(gr - Gs[i]) : 0.f;
         }
         if (!SCALAR && bad_chunk) {
             // exact path: every term with its own exp (chunks with extreme decay only)
-            const int lim = is_p ? rr : rr - 1;
-            const bool vr = rr < len;
-            for (int i = 0; i <= lim && vr; ++i) {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) {
                 float acc = 0.f;
-                for (int c = 0; c < D; ++c) {
-                    const size_t tr = (size_t)(start + rr) * tok_stride + (size_t)h * D + c;
-                    const size_t ti = (size_t)(start + i) * tok_stride + (size_t)h * D + c;
-                    const float xr = is_p ? scale * (float)q[tr] : (float)k[tr];
-                    acc += xr * (float)k[ti] * expf(g[tr] - g[ti]);
+                if (i <= lim && rr < len) {
+                    for (int c = 0; c < D; ++c) {
+                        const size_t tr = base + (size_t)rr * tok_stride + c;
+                        const size_t ti = base + (size_t)i * tok_stride + c;
+                        const float xr = is_p ? scale * (float)q[tr] : (float)k[tr];
+                        acc += xr * (float)k[ti] * expf(g[tr] - g[ti]);
+                    }
                 }
-                dst[rr * 65 + i] = scl * acc;
+                vrow[i] = acc;
+            }
+        }
+        if (is_p) {
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) {
+                float x[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) x[e] = (8 * jj + e <= lim) ? vrow[8 * jj + e] : 0.f;
+                *reinterpret_cast<uint4*>(sm + L::Pt + sw128_chunk(64, rr, jj)) = pack8(x);
+            }
+        } else {
+            const float br = Bs[rr];
+#pragma unroll
+            for (int i4 = 0; i4 < 16; ++i4) {
+                float4 x;
+                x.x = (4 * i4 + 0 <= lim) ? br * vrow[4 * i4 + 0] : 0.f;
+                x.y = (4 * i4 + 1 <= lim) ? br * vrow[4 * i4 + 1] : 0.f;
+                x.z = (4 * i4 + 2 <= lim) ? br * vrow[4 * i4 + 2] : 0.f;
+                x.w = (4 * i4 + 3 <= lim) ? br * vrow[4 * i4 + 3] : 0.f;
+                *reinterpret_cast<float4*>(As + rr * kLd + 4 * i4) = x;
             }
         }
     }
     __syncthreads();
 
-    // ---- phase 5: T = (I + A)^-1 by blocked forward substitution (fp32) ----
+    // ---- T = (I + A)^-1: 16x16 diagonal blocks, then three block levels ------
     if (tid < 64) {
-        // diagonal 16x16 blocks, one column per thread
         const int b = tid >> 4, cc = tid & 15, o = 16 * b;
         float x[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
-            float acc = (r == cc) ? 1.f : 0.f;
+            float ar[16];
 #pragma unroll
-            for (int i = 0; i < r; ++i)
-                if (i >= cc) acc -= As[(o + r) * 65 + o + i] * x[i];
-            x[r] = (r >= cc) ? acc : 0.f;
-            Ts[(o + r) * 65 + o + cc] = x[r];
-        }
-    } else {
-        // meanwhile: P image -> record (8 chunks of 8 per row)
-        for (int qd = tid - 64; qd < 512; qd += 64) {
-            const int r = qd >> 3, jj = qd & 7;
-            float x[8];
+            for (int i4 = 0; i4 < 4; ++i4) {
+                const float4 t = f4(As + (o + r) * kLd + o + 4 * i4);
+                ar[4 * i4] = t.x; ar[4 * i4 + 1] = t.y; ar[4 * i4 + 2] = t.z; ar[4 * i4 + 3] = t.w;
+            }
+            float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] = Pf[r * 65 + 8 * jj + e];
-            *reinterpret_cast<uint4*>(rec + R.P + sw128_chunk(64, r, jj)) = pack8(x);
+            for (int i = 0; i < r; ++i) {
+                if (i & 1) a1 = fmaf(ar[i], x[i], a1);
+                else a0 = fmaf(ar[i], x[i], a0);
+            }
+            x[r] = (r < cc) ? 0.f : ((r == cc) ? 1.f : -(a0 + a1));
+            Ts[(o + r) * kLd + o + cc] = x[r];
         }
     }
     __syncthreads();
 #pragma unroll
     for (int d = 1; d <= 3; ++d) {
-        // Y_bj = sum_{l=j}^{b-1} A_bl T_lj for all pairs (b, j = b - d)
-        for (int e = tid; e < (4 - d) * 256; e += kThreads) {
-            const int p = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-            const int b = d + p, j = p;
-            float acc = 0.f;
-            for (int l = j; l < b; ++l)
+        const int ntiles = (4 - d) * 32;
+        const int p = tid >> 5, t = tid & 31;
+        const int rr0 = 2 * (t >> 2), cq = t & 3;
+        const int b = d + p, j = p;
+        if (tid < ntiles) {
+            // Y_bj = sum_{l=j}^{b-1} A_bl T_lj, a 2 x 4 tile per thread
+            float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int l = j; l < b; ++l) {
 #pragma unroll
-                for (int m = 0; m < 16; ++m)
-                    acc += As[(16 * b + rr) * 65 + 16 * l + m] * Ts[(16 * l + m) * 65 + 16 * j + cc];
-            Yt[p * 256 + rr * 16 + cc] = acc;
+                for (int m4 = 0; m4 < 4; ++m4) {
+                    const float4 a0 = f4(As + (16 * b + rr0) * kLd + 16 * l + 4 * m4);
+                    const float4 a1 = f4(As + (16 * b + rr0 + 1) * kLd + 16 * l + 4 * m4);
+                    const float a0v[4] = {a0.x, a0.y, a0.z, a0.w}, a1v[4] = {a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+                    for (int qq = 0; qq < 4; ++qq) {
+                        const float4 tv = f4(Ts + (16 * l + 4 * m4 + qq) * kLd + 16 * j + 4 * cq);
+                        y0[0] = fmaf(a0v[qq], tv.x, y0[0]); y0[1] = fmaf(a0v[qq], tv.y, y0[1]);
+                        y0[2] = fmaf(a0v[qq], tv.z, y0[2]); y0[3] = fmaf(a0v[qq], tv.w, y0[3]);
+                        y1[0] = fmaf(a1v[qq], tv.x, y1[0]); y1[1] = fmaf(a1v[qq], tv.y, y1[1]);
+                        y1[2] = fmaf(a1v[qq], tv.z, y1[2]); y1[3] = fmaf(a1v[qq], tv.w, y1[3]);
+                    }
+                }
+            }
+            *reinterpret_cast<float4*>(Yt + p * 256 + rr0 * 16 + 4 * cq) = make_float4(y0[0], y0[1], y0[2], y0[3]);
+            *reinterpret_cast<float4*>(Yt + p * 256 + (rr0 + 1) * 16 + 4 * cq) = make_float4(y1[0], y1[1], y1[2], y1[3]);
         }
         __syncthreads();
-        // T_bj = -T_bb Y_bj
-        for (int e = tid; e < (4 - d) * 256; e += kThreads) {
-            const int p = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-            const int b = d + p, j = p;
-            float acc = 0.f;
+        if (tid < ntiles) {
+            // T_bj = -T_bb Y_bj (T_bb is lower triangular with zeros above)
+            float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int m = 0; m < 16; ++m)
-                if (m <= rr) acc += Ts[(16 * b + rr) * 65 + 16 * b + m] * Yt[p * 256 + m * 16 + cc];
-            Ts[(16 * b + rr) * 65 + 16 * j + cc] = -acc;
+            for (int m4 = 0; m4 < 4; ++m4) {
+                const float4 t0 = f4(Ts + (16 * b + rr0) * kLd + 16 * b + 4 * m4);
+                const float4 t1 = f4(Ts + (16 * b + rr0 + 1) * kLd + 16 * b + 4 * m4);
+                const float t0v[4] = {t0.x, t0.y, t0.z, t0.w}, t1v[4] = {t1.x, t1.y, t1.z, t1.w};
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                    const float4 yv = f4(Yt + p * 256 + (4 * m4 + qq) * 16 + 4 * cq);
+                    z0[0] = fmaf(t0v[qq], yv.x, z0[0]); z0[1] = fmaf(t0v[qq], yv.y, z0[1]);
+                    z0[2] = fmaf(t0v[qq], yv.z, z0[2]); z0[3] = fmaf(t0v[qq], yv.w, z0[3]);
+                    z1[0] = fmaf(t1v[qq], yv.x, z1[0]); z1[1] = fmaf(t1v[qq], yv.y, z1[1]);
+                    z1[2] = fmaf(t1v[qq], yv.z, z1[2]); z1[3] = fmaf(t1v[qq], yv.w, z1[3]);
+                }
+            }
+            *reinterpret_cast<float4*>(Ts + (16 * b + rr0) * kLd + 16 * j + 4 * cq) = make_float4(-z0[0], -z0[1], -z0[2], -z0[3]);
+            *reinterpret_cast<float4*>(Ts + (16 * b + rr0 + 1) * kLd + 16 * j + 4 * cq) = make_float4(-z1[0], -z1[1], -z1[2], -z1[3]);
         }
         __syncthreads();
     }
     // T -> bf16 operand tile [64 r][64 i] (zero above the diagonal)
     for (int qd = tid; qd < 512; qd += kThreads) {
         const int r = qd >> 3, jj = qd & 7;
-        float x[8];
+        const float4 ta = f4(Ts + r * kLd + 8 * jj), tb = f4(Ts + r * kLd + 8 * jj + 4);
+        float x[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
 #pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = (8 * jj + e <= r) ? Ts[r * 65 + 8 * jj + e] : 0.f;
+        for (int e = 0; e < 8; ++e) x[e] = (8 * jj + e <= r) ? x[e] : 0.f;
         *reinterpret_cast<uint4*>(sm + L::Tb + sw128_chunk(64, r, jj)) = pack8(x);
     }
     fence_proxy_async_smem();
@@ -443,7 +553,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     failed = __syncthreads_or(failed);
     tc_fence_after_sync();
 
-    // ---- phase 6: [W | U]^T = [diag(b)(K*Gamma) | diag(b)V]^T T^T ----------
+    // ---- [W | U]^T = [diag(b)(K*Gamma) | diag(b)V]^T T^T ---------------------
     if (tid == 0 && !failed) {
         const uint32_t id = idesc_bf16_f32(128, 64);
         const uint32_t aB = smem_u32(Bt), aT = smem_u32(sm + L::Tb);
@@ -458,59 +568,107 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     if (!failed && !mbar_wait(&mma_bar, 1)) failed = true;
     tc_fence_after_sync();
 
-    // ---- phase 7: W image (staged, transposed) and U^T image ----------------
+    // W^T rows c and U^T rows v -> one bf16 tile [2D][64] (row D + v for U^T)
     {
-        uint8_t* Wst = sm + L::Wst;
-        // lanes 0..D-1 hold W^T rows; U^T rows are lanes D..2D-1 (D = 64) or
-        // columns 64..127 of the same lanes (D = 128)
+        uint8_t* WUt = sm + L::WUt;
         const int lrow = 32 * warp + lane;
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
-            const bool wpart = (D == 64) ? (lrow < 64) : (part == 0);
-            const int row = (D == 64) ? (lrow & 63) : lrow;
-            if (D == 64 && part == 1) break;
-            const uint32_t col0 = (D == 64) ? 0u : 64u * part;
+        for (int part = 0; part < 2 * D / 128; ++part) {
+            const int row = (D == 64) ? lrow : (lrow + 128 * part);
 #pragma unroll
             for (int piece = 0; piece < 2; ++piece) {
                 float x[32];
-                tmem_ld32(tmem + lane_base + col0 + 32 * piece, x);
+                tmem_ld32(tmem + lane_base + 64 * part + 32 * piece, x);
                 tmem_ld_wait();
-                if (wpart) {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        *reinterpret_cast<__nv_bfloat16*>(Wst + sw128_offset(64, 32 * piece + j, row)) =
-                            __float2bfloat16_rn(x[j]);
-                } else {
+                for (int jj = 0; jj < 4; ++jj) {
+                    float y[8];
 #pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        float y[8];
+                    for (int e = 0; e < 8; ++e) y[e] = x[8 * jj + e];
+                    *reinterpret_cast<uint4*>(WUt + sw128_chunk(2 * D, row, 4 * piece + jj)) = pack8(y);
+                }
+            }
+        }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before_sync();
+    failed = __syncthreads_or(failed);
+    tc_fence_after_sync();
+
+    // ---- P [W | U], Kd^T W, U^T Kd --------------------------------------------
+    if (tid == 0 && !failed) {
+        const uint32_t aP = smem_u32(sm + L::Pt), aWU = smem_u32(sm + L::WUt), aKd = smem_u32(Kdt);
+        const uint32_t id_pwu = idesc_bf16_f32(64, 2 * D);
+        const uint32_t id_dd = idesc_bf16_f32(D, D);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) y[e] = x[8 * jj + e];
-                        *reinterpret_cast<uint4*>(rec + R.Ut + sw128_chunk(D, row, 4 * piece + jj)) = pack8(y);
-                    }
+        for (int kk = 0; kk < 4; ++kk) {
+            mma_bf16(tmem, sw128_desc(aP, 64, 0, 16 * kk), sw128_desc(aWU, 2 * D, 0, 16 * kk), id_pwu, kk > 0);
+            mma_bf16(tmem + 2 * D, sw128_desc(aKd, D, 0, 16 * kk), sw128_desc(aWU, 2 * D, 0, 16 * kk), id_dd, kk > 0);
+            mma_bf16(tmem + 3 * D, sw128_desc(aWU, 2 * D, D, 16 * kk), sw128_desc(aKd, D, 0, 16 * kk), id_dd, kk > 0);
+        }
+        mma_commit(&mma_bar);
+    }
+    if (!failed && !mbar_wait(&mma_bar, 0)) failed = true;
+    tc_fence_after_sync();
+
+    // ---- record: Qt = Qg - P W, PU, BS = -Kd^T W, NC = U^T Kd, gamma ----------
+    {
+        // rows of the M = 64 products live in lanes 16 w + l (l < 16)
+        const int r64 = 16 * warp + lane;
+        const bool act64 = lane < 16;
+#pragma unroll
+        for (int piece = 0; piece < D / 32; ++piece) {
+            float pw[32], pu[32];
+            tmem_ld32(tmem + lane_base + 32 * piece, pw);
+            tmem_ld32(tmem + lane_base + D + 32 * piece, pu);
+            tmem_ld_wait();
+            if (act64) {
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int chunk = 4 * piece + jj;
+                    float qgv[8];
+                    Vec8<__nv_bfloat16>::load(reinterpret_cast<const __nv_bfloat16*>(Qgs + sw128_chunk(64, r64, chunk)), qgv);
+                    float a[8], b[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) { a[e] = qgv[e] - pw[8 * jj + e]; b[e] = pu[8 * jj + e]; }
+                    *reinterpret_cast<uint4*>(rec + R.Qt + sw128_chunk(64, r64, chunk)) = pack8(a);
+                    *reinterpret_cast<uint4*>(rec + R.PU + sw128_chunk(64, r64, chunk)) = pack8(b);
+                }
+            }
+        }
+        const int rD = (D == 128) ? (32 * warp + lane) : r64;
+        const bool actD = (D == 128) || act64;
+#pragma unroll
+        for (int piece = 0; piece < D / 32; ++piece) {
+            float bs[32], nc[32];
+            tmem_ld32(tmem + lane_base + 2 * D + 32 * piece, bs);
+            tmem_ld32(tmem + lane_base + 3 * D + 32 * piece, nc);
+            tmem_ld_wait();
+            if (actD) {
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int chunk = 4 * piece + jj;
+                    float a[8], b[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) { a[e] = -bs[8 * jj + e]; b[e] = nc[8 * jj + e]; }
+                    *reinterpret_cast<uint4*>(rec + R.BS + sw128_chunk(D, rD, chunk)) = pack8(a);
+                    *reinterpret_cast<uint4*>(rec + R.NC + sw128_chunk(D, rD, chunk)) = pack8(b);
                 }
             }
         }
         if (tid < D) reinterpret_cast<float*>(rec + R.gamma)[tid] = expf(Gl[tid]);
     }
-    fence_proxy_async_smem();
     tc_fence_before_sync();
     __syncthreads();
-    if (tid == 0) {
-        bulk_s2g(rec + R.W, sm + L::Wst, (uint32_t)(D * 128));
-        bulk_commit_group();
-        bulk_wait_group_read0();
-        if (failed) atomicOr(err, 1u);
-    }
-    __syncthreads();
+    if (tid == 0 && failed) atomicOr(err, 1u);
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
 // Unpack records into plain fp32 arrays (inspection / tests only).
 template <int D>
 __global__ void unpack_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
-                              const uint8_t* __restrict__ records, float* W, float* U, float* P,
-                              float* Qg, float* Kd, float* gamma) {
+                              const uint8_t* __restrict__ records, float* Qt, float* PU, float* BS,
+                              float* NC, float* gamma) {
     constexpr RecordLayout R = record_layout(D);
     int seq, start, len;
     if (!slot_to_chunk(cu, n_seqs, blockIdx.x, &seq, &start, &len)) return;
@@ -521,13 +679,14 @@ __global__ void unpack_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     };
     for (int e = threadIdx.x; e < 64 * D; e += blockDim.x) {
         const int r = e / D, c = e % D;
-        W[sh * 64 * D + e] = bf(R.W + sw128_offset(64, r, c));
-        Qg[sh * 64 * D + e] = bf(R.Qg + sw128_offset(64, r, c));
-        U[sh * 64 * D + e] = bf(R.Ut + sw128_offset(D, c, r));
-        Kd[sh * 64 * D + e] = bf(R.Kt + sw128_offset(D, c, r));
+        Qt[sh * 64 * D + e] = bf(R.Qt + sw128_offset(64, r, c));
+        PU[sh * 64 * D + e] = bf(R.PU + sw128_offset(64, r, c));
     }
-    for (int e = threadIdx.x; e < 64 * 64; e += blockDim.x)
-        P[sh * 4096 + e] = bf(R.P + sw128_offset(64, e / 64, e % 64));
+    for (int e = threadIdx.x; e < D * D; e += blockDim.x) {
+        const int r = e / D, c = e % D;
+        BS[sh * D * D + e] = bf(R.BS + sw128_offset(D, r, c));
+        NC[sh * D * D + e] = bf(R.NC + sw128_offset(D, r, c));
+    }
     for (int c = threadIdx.x; c < D; c += blockDim.x)
         gamma[sh * D + c] = reinterpret_cast<const float*>(rec + R.gamma)[c];
 }
@@ -536,7 +695,7 @@ template <int D, typename InT, bool SCALAR>
 cudaError_t launch_typed(const gdr_prefill_args& a, const float* g, uint8_t* records,
                          uint32_t* err, cudaStream_t st) {
     auto kern = intra_chunk_kernel<D, InT, SCALAR>;
-    const uint32_t smem = IntraSmem<D, SCALAR>::dyn_bytes;
+    const uint32_t smem = IntraLayout<D, InT, SCALAR>::dyn_bytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)n_chunk_slots(a.total_tokens, a.n_seqs), (unsigned)a.n_heads);
@@ -565,16 +724,15 @@ cudaError_t launch_intra_chunk(const gdr_prefill_args& a, const float* g, uint8_
                                    : launch_decay<128, float>(a, g, records, err, st);
 }
 
-cudaError_t launch_unpack_records(const gdr_prefill_args& a, const uint8_t* records, float* W,
-                                  float* U, float* P, float* Qg, float* Kd, float* gamma,
-                                  cudaStream_t st) {
+cudaError_t launch_unpack_records(const gdr_prefill_args& a, const uint8_t* records, float* Qt,
+                                  float* PU, float* BS, float* NC, float* gamma, cudaStream_t st) {
     const int64_t slots = n_chunk_slots(a.total_tokens, a.n_seqs);
     if (slots == 0) return cudaSuccess;
     const dim3 grid((unsigned)slots, (unsigned)a.n_heads);
     if (a.d_k == 64)
-        unpack_kernel<64><<<grid, 256, 0, st>>>(a.cu_seqlens, a.n_seqs, a.n_heads, records, W, U, P, Qg, Kd, gamma);
+        unpack_kernel<64><<<grid, 256, 0, st>>>(a.cu_seqlens, a.n_seqs, a.n_heads, records, Qt, PU, BS, NC, gamma);
     else
-        unpack_kernel<128><<<grid, 256, 0, st>>>(a.cu_seqlens, a.n_seqs, a.n_heads, records, W, U, P, Qg, Kd, gamma);
+        unpack_kernel<128><<<grid, 256, 0, st>>>(a.cu_seqlens, a.n_seqs, a.n_heads, records, Qt, PU, BS, NC, gamma);
     return cudaGetLastError();
 }
 

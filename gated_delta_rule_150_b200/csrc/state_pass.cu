@@ -3,26 +3,28 @@
 // "Modele hybrydowe: co Gated DeltaNet zastępuje w cache KV", closing
 // paragraph of "Co stan rekurencyjny zmienia przy serwowaniu": inside a chunk
 // the updates are dense matrix products; only the step from one chunk to the
-// next is sequential.  This kernel is that sequential step.  For a chunk with
-// start state S0 (d_v x d_k, fp32) and the factors the intra-chunk kernel
-// stored (W, U, Qg, P, Kd, gamma), it computes
-//     Delta^T = U^T - S0 W^T                        (d_v x 64)
-//     O^T     = S0 Qg^T + Delta^T P^T                (d_v x 64)  -> o
-//     S_next  = S0 Diag(gamma) + Delta^T Kd          (d_v x d_k)
-// which is the token recurrence S_t = S_{t-1} Diag(a_t)(I - b_t k_t k_t^T) +
-// b_t v_t k_t^T, o_t = S_t q_t unrolled over the chunk.
+// next is sequential.  This file is that sequential step.  The intra-chunk
+// kernel has reduced each chunk to an affine map of its start state S0
+// (d_v x d_k, fp32):
+//     S_next = S0 Diag(gamma) + S0 BS^T + NC          O = Qt S0^T + PU
+// (record layout in internal.h).  Per chunk, two tcgen05 MMAs read the bf16
+// copy of S0 from shared memory:
+//     Z = S0 BS^T  (M = d_v, N = d_k, K = d_k)   -> the state, on the critical path
+//     O = Qt S0^T  (M = 64,  N = d_v, K = d_k)   -> the outputs, off it
+// The fp32 master state stays in registers for the whole run (8 warps; a
+// thread owns half of a state row); S = S * gamma + Z + NC is done in fp32.
+// The outputs of chunk k are added to PU and stored while the MMAs of chunk
+// k+1 run (O is double buffered in tensor memory).  Records arrive by bulk
+// (TMA) copies, prefetched up to kStages chunks ahead.  Snapshots of the state
+// are written at every snap_interval boundary (section "Co stan
+// rekurencyjny...", point 1: prefix reuse needs the state at that position).
 //
-// One CTA per (sequence, head) walks the sequence's chunks in order.  The fp32
-// master state stays in registers (thread = state row) for the whole
-// sequence; its bf16 copy in shared memory is the A operand of the tensor-core
-// products.  Each chunk's record arrives with one bulk (TMA) copy, prefetched
-// one chunk ahead into a second stage.  The four products run as tcgen05 MMAs
-// (bf16 in, fp32 accumulate in tensor memory):
-//     group 1:  X = S0 W^T  (M=d_v, N=64, K=d_k)   Y = S0 Qg^T (M=d_v, N=64, K=d_k)
-//     group 2:  Y += Delta^T P^T (K=64)              Z = Delta^T Kd (M=d_v, N=d_k, K=64)
-// Snapshots of the state are written at every snap_interval boundary
-// (section "Co stan rekurencyjny...", point 1: prefix reuse needs the state at
-// that position).
+// Long sequences with few heads are cut into segments (internal.h): kLocal
+// runs each segment from a zero state and from the identity at once, giving
+// the segment's affine map (N, M); combine_kernel chains the maps into each
+// segment's true start state E in fp32; kApply replays each segment from E to
+// produce its outputs, snapshots and, for the last segment, the final state.
+// kFull is the single pass over whole sequences.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -31,285 +33,448 @@
 namespace gdr {
 namespace {
 
-constexpr int kThreads = 128;
-constexpr uint32_t kTmemCols = 256;   // X: [0,64)  Y: [64,128)  Z: [128,128+D)
+constexpr int kThreads = 256;
+enum Mode { kFull = 0, kLocal = 1, kApply = 2 };
 
-template <typename T> __device__ __forceinline__ void store_out(T* p, float x);
-template <> __device__ __forceinline__ void store_out<float>(float* p, float x) { *p = x; }
-template <> __device__ __forceinline__ void store_out<__nv_bfloat16>(__nv_bfloat16* p, float x) {
-    *p = __float2bfloat16_rn(x);
-}
-
-template <int D>
-struct PassSmem {
-    static constexpr RecordLayout R = record_layout(D);
-    static constexpr uint32_t stage0 = 0;
-    static constexpr uint32_t stage1 = R.bytes;
-    static constexpr uint32_t S = 2 * R.bytes;               // bf16 [D x D] operand
-    static constexpr uint32_t Dt = S + D * D * 2;            // bf16 [D x 64] Delta^T
-    static constexpr uint32_t bytes = Dt + D * 128;
-    static constexpr uint32_t dyn_bytes = bytes + 1024;      // + alignment slack
+template <typename T> struct Out8;
+template <> struct Out8<float> {
+    static __device__ __forceinline__ void store(float* p, const float (&x)[8]) {
+        *reinterpret_cast<float4*>(p) = make_float4(x[0], x[1], x[2], x[3]);
+        *reinterpret_cast<float4*>(p + 4) = make_float4(x[4], x[5], x[6], x[7]);
+    }
+};
+template <> struct Out8<__nv_bfloat16> {
+    static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&x)[8]) {
+        uint4 u;
+        u.x = pack_bf16(x[0], x[1]); u.y = pack_bf16(x[2], x[3]);
+        u.z = pack_bf16(x[4], x[5]); u.w = pack_bf16(x[6], x[7]);
+        *reinterpret_cast<uint4*>(p) = u;
+    }
 };
 
-// Bounded drain used on the error path only: wait for the copies this CTA
-// issued, so no bulk copy lands after the CTA has exited.
-__device__ void drain_copies(uint64_t* full, const uint32_t* issued, const uint32_t* done) {
-    for (int s = 0; s < 2; ++s)
-        for (uint32_t u = done[s]; u < issued[s]; ++u) mbar_wait(&full[s], u & 1);
-}
+template <int D, int MODE>
+struct PassLayout {
+    static constexpr bool kOut = MODE != kLocal;
+    static constexpr int kStages = (D == 64) ? 3 : 2;
+    // rows of the bf16 state operand: S (and the identity-started X rows in kLocal)
+    static constexpr int kRows = (MODE == kLocal) ? 2 * D : D;
+    // tensor-core operand tiles, 1024-byte aligned
+    static constexpr uint32_t QtS = 0;                                      // kStages x [64 x D]
+    static constexpr uint32_t BSS = QtS + (kOut ? kStages * 128u * D : 0u); // kStages x [D x D]
+    static constexpr uint32_t S = BSS + kStages * 2u * D * D;               // bf16 [kRows x D]
+    // thread-read parts of the records
+    static constexpr uint32_t PUS = S + 2u * kRows * D;                     // kStages x [64 x D]
+    static constexpr uint32_t NCS = PUS + (kOut ? kStages * 128u * D : 0u); // kStages x [D x D]
+    static constexpr uint32_t GAS = NCS + kStages * 2u * D * D;             // kStages x [D] fp32
+    static constexpr uint32_t bytes = GAS + kStages * 4u * D;
+    static constexpr uint32_t dyn_bytes = bytes + 1024u;
+    static constexpr uint32_t tx_bytes = (kOut ? 256u * D : 0u) + 4u * D * D + 4u * D;
+    static_assert(dyn_bytes + 128u <= 232448u, "shared memory budget");
+};
 
-template <int D, typename OutT>
+template <int D, typename OutT, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                   const uint8_t* __restrict__ records, const float* init_state,
                   OutT* __restrict__ o, float* final_state, int snap_interval,
-                  float* __restrict__ snapshots, uint32_t* err) {
-    using L = PassSmem<D>;
+                  float* __restrict__ snapshots, int seg_chunks, float* seg_ws,
+                  uint32_t* err) {
+    using L = PassLayout<D, MODE>;
     constexpr RecordLayout R = record_layout(D);
+    constexpr int ST = L::kStages;
+    constexpr bool kOut = L::kOut;
+    // M of the state product: D rows (kLocal, D = 64: S and X stacked, 128 rows;
+    // kLocal, D = 128: two products of 128 rows)
+    constexpr int kMS = (MODE == kLocal && D == 64) ? 128 : D;
+    constexpr int kNT = (MODE == kLocal && D == 128) ? 2 : 1;      // state products
+    constexpr uint32_t kTmemCols = (D == 64) ? 256u : 512u;
+    constexpr int CW = D / 2;                                       // columns per thread
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-    __shared__ uint64_t full[2];
+    __shared__ uint64_t full[ST];
     __shared__ uint64_t mma_bar;
     __shared__ uint32_t tmem_slot;
     __shared__ int64_t snap_base_s;
-    __shared__ uint32_t issued_s[2], done_s[2];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int n = blockIdx.x / H, h = blockIdx.x % H;
-    const int row = (D == 128) ? (32 * warp + lane) : (16 * warp + lane);
-    const bool active = (D == 128) || (lane < 16);
-    const int s0 = __ldg(cu + n), s1 = __ldg(cu + n + 1);
-    const int len_seq = s1 - s0;
-    const int nchunks = (len_seq + kChunk - 1) / kChunk;
+    const int sub = warp & 3, half = warp >> 2;
+    int n, h, s0, s1, seg_start;
+    if (MODE == kFull) {
+        n = blockIdx.x / H;
+        h = blockIdx.x % H;
+        s0 = __ldg(cu + n);
+        s1 = __ldg(cu + n + 1);
+        seg_start = s0;
+    } else {
+        int len_span;
+        if (!slot_to_span(cu, n_seqs, blockIdx.x, kChunk * seg_chunks, &n, &s0, &len_span)) return;
+        h = blockIdx.y;
+        seg_start = __ldg(cu + n);
+        s1 = s0 + len_span;
+    }
+    const int chunk0 = (s0 - seg_start) / kChunk;             // absolute chunk index of chunk 0
+    const int nchunks = (s1 - s0 + kChunk - 1) / kChunk;
+    float* seg_base = seg_ws ? seg_ws + ((size_t)blockIdx.x * H + h) * 3u * D * D : nullptr;
 
-    uint8_t* stage[2] = {sm + L::stage0, sm + L::stage1};
-    uint8_t* sS = sm + L::S;
-    uint8_t* sDt = sm + L::Dt;
+    // thread -> state row (tensor-memory lane layout of the M = kMS product)
+    const int row = (kMS == 128) ? (32 * sub + lane) : (16 * sub + lane);
+    const bool active = (kMS == 128) || (lane < 16);
+    const bool is_x = (MODE == kLocal && D == 64) && row >= D;     // identity-started rows
+    const int srow = is_x ? row - D : row;                          // row within S or X
+    const int cb = half * CW;                                       // first column
+    // thread -> output row (lane layout of an M = 64 product), columns [cb, cb + CW)
+    const int orow = 16 * sub + lane;
+    const bool oactive = lane < 16;
 
     if (tid == 0) {
-        mbar_init(&full[0], 1);
-        mbar_init(&full[1], 1);
+#pragma unroll
+        for (int s = 0; s < ST; ++s) mbar_init(&full[s], 1);
         mbar_init(&mma_bar, 1);
         fence_mbar_init();
-        issued_s[0] = issued_s[1] = done_s[0] = done_s[1] = 0;
     }
     if (warp == 0) {
         tmem_alloc(&tmem_slot, kTmemCols);
-        // snapshot slot base: full intervals of all earlier sequences
         int64_t acc = 0;
-        if (snap_interval > 0)
+        if (kOut && snap_interval > 0)
             for (int m = lane; m < n; m += 32) acc += (__ldg(cu + m + 1) - __ldg(cu + m)) / snap_interval;
 #pragma unroll
         for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
         if (lane == 0) snap_base_s = acc;
     }
 
-    // Load the initial state row (fp32) and its bf16 operand copy.
-    float S[D];
-    const size_t state_off = ((size_t)n * H + h) * D * D + (size_t)row * D;
-#pragma unroll
-    for (int c = 0; c < D; c += 4) {
-        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (active && init_state) x = *reinterpret_cast<const float4*>(init_state + state_off + c);
-        S[c] = x.x; S[c + 1] = x.y; S[c + 2] = x.z; S[c + 3] = x.w;
+    // ---- initial state --------------------------------------------------------
+    // S[t][j]: tile t (0 = S, 1 = X for kLocal with two products), column cb + j
+    float S[kNT][CW];
+    const size_t state_off = ((size_t)n * H + h) * D * D;
+    const float* src = nullptr;
+    size_t src_off = state_off;
+    if (MODE == kFull) src = init_state;
+    if (MODE == kApply) {
+        if (s0 == seg_start) src = init_state;
+        else { src = seg_base + 2u * D * D; src_off = 0; }       // E: this segment's start state
     }
+#pragma unroll
+    for (int t = 0; t < kNT; ++t) {
+        const bool x_tile = (MODE == kLocal) && (t == 1 || is_x);
+#pragma unroll
+        for (int j = 0; j < CW; j += 4) {
+            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (MODE != kLocal && active && src)
+                x = *reinterpret_cast<const float4*>(src + src_off + (size_t)srow * D + cb + j);
+            if (x_tile) {
+                const int c = cb + j;
+                x = make_float4(c + 0 == srow ? 1.f : 0.f, c + 1 == srow ? 1.f : 0.f,
+                                c + 2 == srow ? 1.f : 0.f, c + 3 == srow ? 1.f : 0.f);
+            }
+            S[t][j] = x.x; S[t][j + 1] = x.y; S[t][j + 2] = x.z; S[t][j + 3] = x.w;
+        }
+    }
+    uint8_t* sS = sm + L::S;
+    auto write_operand = [&](int t, int j0) {   // bf16 copy of columns cb + j0 .. + 8
+        const int orow_t = (MODE == kLocal && D == 128) ? row + t * D : row;
+        uint4 u;
+        u.x = pack_bf16(S[t][j0 + 0], S[t][j0 + 1]);
+        u.y = pack_bf16(S[t][j0 + 2], S[t][j0 + 3]);
+        u.z = pack_bf16(S[t][j0 + 4], S[t][j0 + 5]);
+        u.w = pack_bf16(S[t][j0 + 6], S[t][j0 + 7]);
+        *reinterpret_cast<uint4*>(sS + sw128_chunk(L::kRows, orow_t, (cb + j0) / 8)) = u;
+    };
     if (active) {
 #pragma unroll
-        for (int j = 0; j < D / 8; ++j) {
-            uint4 u;
-            u.x = pack_bf16(S[8 * j + 0], S[8 * j + 1]);
-            u.y = pack_bf16(S[8 * j + 2], S[8 * j + 3]);
-            u.z = pack_bf16(S[8 * j + 4], S[8 * j + 5]);
-            u.w = pack_bf16(S[8 * j + 6], S[8 * j + 7]);
-            *reinterpret_cast<uint4*>(sS + sw128_chunk(D, row, j)) = u;
-        }
+        for (int t = 0; t < kNT; ++t)
+#pragma unroll
+            for (int j = 0; j < CW; j += 8) write_operand(t, j);
     }
     fence_proxy_async_smem();
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = tmem_slot;
-    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+    const uint32_t lane_base = (uint32_t)(32 * sub) << 16;
     const int64_t snap_base = snap_base_s;
 
-    auto record_of = [&](int k) -> const uint8_t* {
-        const int64_t slot = (int64_t)(s0 / kChunk) + k + n;
+    auto record_of = [&](int c) -> const uint8_t* {
+        const int64_t slot = (int64_t)(seg_start / kChunk) + chunk0 + c + n;
         return records + ((size_t)slot * H + h) * R.bytes;
     };
-    if (tid == 0 && nchunks > 0) {
-        mbar_arrive_expect_tx(&full[0], R.bytes);
-        bulk_g2s(stage[0], record_of(0), R.bytes, &full[0]);
-        issued_s[0] = 1;
-    }
+    auto issue_copy = [&](int c) {       // thread 0 only
+        const int s = c % ST;
+        const uint8_t* r = record_of(c);
+        mbar_arrive_expect_tx(&full[s], L::tx_bytes);
+        if (kOut) {
+            bulk_g2s(sm + L::QtS + s * 128u * D, r + R.Qt, 128u * D, &full[s]);
+            bulk_g2s(sm + L::PUS + s * 128u * D, r + R.PU, 128u * D, &full[s]);
+        }
+        bulk_g2s(sm + L::BSS + s * 2u * D * D, r + R.BS, 2u * D * D, &full[s]);
+        bulk_g2s(sm + L::NCS + s * 2u * D * D, r + R.NC, 2u * D * D, &full[s]);
+        bulk_g2s(sm + L::GAS + s * 4u * D, r + R.gamma, 4u * D, &full[s]);
+    };
+    const uint32_t id_z = idesc_bf16_f32(kMS, D);
+    const uint32_t id_o = idesc_bf16_f32(64, D);
+    const uint32_t aS = smem_u32(sS);
+    auto issue_mma = [&](int c) {        // thread 0 only; operands of chunk c are resident
+        const int s = c % ST;
+        const uint32_t aBS = smem_u32(sm + L::BSS + s * 2u * D * D);
+        tc_fence_after_sync();
+#pragma unroll
+        for (int t = 0; t < kNT; ++t)
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+                mma_bf16(tmem + (uint32_t)(t * 128), sw128_desc(aS, L::kRows, t * 128, 16 * kk),
+                         sw128_desc(aBS, D, 0, 16 * kk), id_z, kk > 0);
+        if (kOut) {
+            const uint32_t aQt = smem_u32(sm + L::QtS + s * 128u * D);
+            const uint32_t o_col = (uint32_t)D * (1 + (c & 1));
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+                mma_bf16(tmem + o_col, sw128_desc(aQt, 64, 0, 16 * kk), sw128_desc(aS, D, 0, 16 * kk),
+                         id_o, kk > 0);
+        }
+        mma_commit(&mma_bar);
+    };
 
-    uint32_t mma_phase = 0;
     bool failed = false;
-    const uint32_t id_y = idesc_bf16_f32(D, 64);
-    const uint32_t id_z = idesc_bf16_f32(D, D);
-    const uint32_t aS = smem_u32(sS), aDt = smem_u32(sDt);
+    int copies_issued = 0, copies_waited = 0, mmas_issued = 0;     // thread 0's bookkeeping
+    if (tid == 0 && nchunks > 0) {
+        for (int c = 0; c < ST && c < nchunks; ++c) issue_copy(c);
+        copies_issued = min(ST, nchunks);
+        if (!mbar_wait(&full[0], 0)) failed = true;
+        copies_waited = 1;
+        issue_mma(0);
+        mmas_issued = 1;
+    }
+    int mmas_waited = 0;
 
     for (int k = 0; k < nchunks; ++k) {
-        const int st = k & 1;
-        uint8_t* rec = stage[st];
+        const int st = k % ST;
         const int t0 = s0 + k * kChunk;
         const int len = min(kChunk, s1 - t0);
+        if (!mbar_wait(&full[st], (uint32_t)(k / ST) & 1)) failed = true;
+        if (!mbar_wait(&mma_bar, (uint32_t)k & 1)) failed = true;
+        mmas_waited = k + 1;
+        tc_fence_after_sync();
+
+        // ---- state: S = S * gamma + Z (+ NC for S rows), critical path ----------
+        const float* gam = reinterpret_cast<const float*>(sm + L::GAS + st * 4u * D);
+        const uint8_t* nc = sm + L::NCS + st * 2u * D * D;
+#pragma unroll
+        for (int t = 0; t < kNT; ++t) {
+            const bool x_tile = (MODE == kLocal) && (t == 1 || is_x);
+#pragma unroll
+            for (int p = 0; p < CW / 16; ++p) {
+                float z[16];
+                tmem_ld16(tmem + lane_base + (uint32_t)(t * 128) + cb + 16 * p, z);
+                tmem_ld_wait();
+                if (active) {
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj) {
+                        const int j = 16 * p + 8 * jj, c = cb + j;
+                        const float4 g0 = *reinterpret_cast<const float4*>(gam + c);
+                        const float4 g1 = *reinterpret_cast<const float4*>(gam + c + 4);
+                        float nv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                        if (!x_tile) {
+                            const uint4 u = *reinterpret_cast<const uint4*>(nc + sw128_chunk(D, srow, c / 8));
+                            const float2 n0 = unpack_bf16(u.x), n1 = unpack_bf16(u.y);
+                            const float2 n2 = unpack_bf16(u.z), n3 = unpack_bf16(u.w);
+                            nv[0] = n0.x; nv[1] = n0.y; nv[2] = n1.x; nv[3] = n1.y;
+                            nv[4] = n2.x; nv[5] = n2.y; nv[6] = n3.x; nv[7] = n3.y;
+                        }
+                        const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            S[t][j + e] = fmaf(S[t][j + e], gv[e], z[8 * jj + e] + nv[e]);
+                        write_operand(t, j);
+                    }
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before_sync();
+        if (__syncthreads_or(failed)) { failed = true; break; }
+        tc_fence_after_sync();
         if (tid == 0 && k + 1 < nchunks) {
-            const int ns = (k + 1) & 1;
-            fence_proxy_async_smem();
-            mbar_arrive_expect_tx(&full[ns], R.bytes);
-            bulk_g2s(stage[ns], record_of(k + 1), R.bytes, &full[ns]);
-            issued_s[ns] += 1;
+            if (!mbar_wait(&full[(k + 1) % ST], (uint32_t)((k + 1) / ST) & 1)) failed = true;
+            copies_waited = k + 2;
+            issue_mma(k + 1);
+            mmas_issued = k + 2;
         }
-        if (!mbar_wait(&full[st], (uint32_t)(k >> 1) & 1)) failed = true;
-        if (tid == 0) done_s[st] += 1;
 
-        // group 1: X = S0 W^T, Y = S0 Qg^T
-        if (tid == 0) {
-            tc_fence_after_sync();
-            const uint32_t aW = smem_u32(rec + R.W), aQ = smem_u32(rec + R.Qg);
+        if (kOut) {
+            // ---- snapshot and outputs of chunk k (overlap chunk k+1's MMAs) -------
+            const int kabs = chunk0 + k;
+            if (snap_interval > 0 && len == kChunk && ((kabs + 1) * kChunk) % snap_interval == 0 && active) {
+                const int64_t slot = snap_base + ((int64_t)(kabs + 1) * kChunk) / snap_interval - 1;
+                float* dst = snapshots + ((size_t)slot * H + h) * D * D + (size_t)srow * D + cb;
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const uint64_t da = sw128_desc(aS, D, 0, 16 * kk);
-                mma_bf16(tmem + 0, da, sw128_desc(aW, 64, 0, 16 * kk), id_y, kk > 0);
-                mma_bf16(tmem + 64, da, sw128_desc(aQ, 64, 0, 16 * kk), id_y, kk > 0);
+                for (int j = 0; j < CW; j += 4)
+                    *reinterpret_cast<float4*>(dst + j) = make_float4(S[0][j], S[0][j + 1], S[0][j + 2], S[0][j + 3]);
             }
-            mma_commit(&mma_bar);
-        }
-        if (!mbar_wait(&mma_bar, mma_phase)) failed = true;
-        mma_phase ^= 1;
-        tc_fence_after_sync();
-
-        // Delta^T row = U^T row - X row, stored as the bf16 A operand of group 2
+            const uint8_t* pu = sm + L::PUS + st * 128u * D;
+            OutT* orow_ptr = o + ((size_t)(t0 + orow) * H + h) * D + cb;
+            const uint32_t o_col = (uint32_t)D * (1 + (k & 1));
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            float x[32];
-            tmem_ld32(tmem + lane_base + 32 * half, x);
-            tmem_ld_wait();
-            if (active) {
+            for (int p = 0; p < CW / 16; ++p) {
+                float y[16];
+                tmem_ld16(tmem + lane_base + o_col + cb + 16 * p, y);
+                tmem_ld_wait();
+                if (oactive && orow < len) {
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int chunk = 4 * half + j;
-                    const uint4 u = *reinterpret_cast<const uint4*>(rec + R.Ut + sw128_chunk(D, row, chunk));
-                    const float2 u0 = unpack_bf16(u.x), u1 = unpack_bf16(u.y);
-                    const float2 u2 = unpack_bf16(u.z), u3 = unpack_bf16(u.w);
-                    uint4 d;
-                    d.x = pack_bf16(u0.x - x[8 * j + 0], u0.y - x[8 * j + 1]);
-                    d.y = pack_bf16(u1.x - x[8 * j + 2], u1.y - x[8 * j + 3]);
-                    d.z = pack_bf16(u2.x - x[8 * j + 4], u2.y - x[8 * j + 5]);
-                    d.w = pack_bf16(u3.x - x[8 * j + 6], u3.y - x[8 * j + 7]);
-                    *reinterpret_cast<uint4*>(sDt + sw128_chunk(D, row, chunk)) = d;
+                    for (int jj = 0; jj < 2; ++jj) {
+                        const int j = 16 * p + 8 * jj;
+                        const uint4 u = *reinterpret_cast<const uint4*>(pu + sw128_chunk(64, orow, (cb + j) / 8));
+                        const float2 p0 = unpack_bf16(u.x), p1 = unpack_bf16(u.y);
+                        const float2 p2 = unpack_bf16(u.z), p3 = unpack_bf16(u.w);
+                        const float x[8] = {y[8 * jj + 0] + p0.x, y[8 * jj + 1] + p0.y,
+                                            y[8 * jj + 2] + p1.x, y[8 * jj + 3] + p1.y,
+                                            y[8 * jj + 4] + p2.x, y[8 * jj + 5] + p2.y,
+                                            y[8 * jj + 6] + p3.x, y[8 * jj + 7] + p3.y};
+                        Out8<OutT>::store(orow_ptr + j, x);
+                    }
                 }
             }
         }
-        fence_proxy_async_smem();
         tc_fence_before_sync();
-        if (__syncthreads_or(failed)) break;
-
-        // group 2: Y += Delta^T P^T, Z = Delta^T Kd
-        if (tid == 0) {
-            tc_fence_after_sync();
-            const uint32_t aP = smem_u32(rec + R.P), aK = smem_u32(rec + R.Kt);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t da = sw128_desc(aDt, D, 0, 16 * kk);
-                mma_bf16(tmem + 64, da, sw128_desc(aP, 64, 0, 16 * kk), id_y, 1);
-                mma_bf16(tmem + 128, da, sw128_desc(aK, D, 0, 16 * kk), id_z, kk > 0);
-            }
-            mma_commit(&mma_bar);
+        if (__syncthreads_or(failed)) { failed = true; break; }
+        if (tid == 0 && k + ST < nchunks) {
+            issue_copy(k + ST);
+            copies_issued = k + ST + 1;
         }
-        if (!mbar_wait(&mma_bar, mma_phase)) failed = true;
-        mma_phase ^= 1;
-        tc_fence_after_sync();
-
-        // o rows of this chunk (column r of O^T = output token t0 + r)
-        OutT* orow = o + (size_t)t0 * H * D + (size_t)h * D + row;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            float y[32];
-            tmem_ld32(tmem + lane_base + 64 + 32 * half, y);
-            tmem_ld_wait();
-            if (active) {
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    if (32 * half + j < len) store_out<OutT>(orow + (size_t)(32 * half + j) * H * D, y[j]);
-            }
-        }
-        // S <- S Diag(gamma) + Z, and refresh the bf16 operand copy
-        const float* gam = reinterpret_cast<const float*>(rec + R.gamma);
-#pragma unroll
-        for (int piece = 0; piece < D / 32; ++piece) {
-            float z[32];
-            tmem_ld32(tmem + lane_base + 128 + 32 * piece, z);
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) S[32 * piece + j] = fmaf(S[32 * piece + j], gam[32 * piece + j], z[j]);
-            if (active) {
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int c = 32 * piece + 8 * j;
-                    uint4 u;
-                    u.x = pack_bf16(S[c + 0], S[c + 1]);
-                    u.y = pack_bf16(S[c + 2], S[c + 3]);
-                    u.z = pack_bf16(S[c + 4], S[c + 5]);
-                    u.w = pack_bf16(S[c + 6], S[c + 7]);
-                    *reinterpret_cast<uint4*>(sS + sw128_chunk(D, row, 4 * piece + j)) = u;
-                }
-            }
-        }
-        if (snap_interval > 0 && len == kChunk && ((k + 1) * kChunk) % snap_interval == 0 && active) {
-            const int64_t slot = snap_base + ((int64_t)(k + 1) * kChunk) / snap_interval - 1;
-            float* dst = snapshots + ((size_t)slot * H + h) * D * D + (size_t)row * D;
-#pragma unroll
-            for (int c = 0; c < D; c += 4)
-                *reinterpret_cast<float4*>(dst + c) = make_float4(S[c], S[c + 1], S[c + 2], S[c + 3]);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before_sync();
-        if (__syncthreads_or(failed)) break;
-        tc_fence_after_sync();
     }
 
     if (failed) {
-        if (tid == 0) {
-            atomicOr(err, 1u);
-            drain_copies(full, issued_s, done_s);
-        }
+        if (tid == 0) atomicOr(err, 1u);
     } else if (active) {
-        float* dst = final_state + state_off;
+        auto store_row = [&](float* dst, int t) {
 #pragma unroll
-        for (int c = 0; c < D; c += 4)
-            *reinterpret_cast<float4*>(dst + c) = make_float4(S[c], S[c + 1], S[c + 2], S[c + 3]);
+            for (int j = 0; j < CW; j += 4)
+                *reinterpret_cast<float4*>(dst + j) = make_float4(S[t][j], S[t][j + 1], S[t][j + 2], S[t][j + 3]);
+        };
+        if (MODE == kFull || (MODE == kApply && s1 == __ldg(cu + n + 1)))
+            store_row(final_state + state_off + (size_t)srow * D + cb, 0);
+        if (MODE == kLocal) {
+            // N (rows of S) then M (rows of X) of this segment's affine map
+            store_row(seg_base + (is_x ? (size_t)D * D : 0) + (size_t)srow * D + cb, 0);
+            if (kNT == 2) store_row(seg_base + (size_t)D * D + (size_t)srow * D + cb, kNT - 1);
+        }
+    }
+    // error path: no copy or MMA of this CTA may still be in flight when it
+    // exits (each of these waits is bounded too)
+    if (tid == 0 && failed) {
+        for (int c = mmas_waited; c < mmas_issued; ++c) mbar_wait(&mma_bar, (uint32_t)c & 1);
+        for (int c = copies_waited; c < copies_issued; ++c) mbar_wait(&full[c % ST], (uint32_t)(c / ST) & 1);
     }
     tc_fence_before_sync();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
-template <int D, typename OutT>
-cudaError_t launch_typed(const gdr_prefill_args& a, const uint8_t* records, uint32_t* err,
-                         cudaStream_t st) {
-    auto kern = state_pass_kernel<D, OutT>;
-    const uint32_t smem = PassSmem<D>::dyn_bytes;
+// Chains the segments' affine maps into each segment's start state:
+//     E_0 = init,   E_{s+1} = E_s M_s + N_s       (fp32, in the chain's order)
+// Rows of the state are independent, so a CTA owns 8 state rows of one
+// (sequence, head) and thread c' the output column c'.  E_s goes to the
+// workspace of segment s (its start state); the last segment's own map is not
+// needed (replaying that segment produces the final state).  An empty sequence
+// has no segment: its final state is its initial state.
+template <int D>
+__global__ void __launch_bounds__(D)
+combine_kernel(const int32_t* __restrict__ cu, int H, int seg_chunks, const float* init_state,
+               float* final_state, float* seg_ws) {
+    constexpr int RB = 8;
+    const int pair = blockIdx.x, rb = blockIdx.y;
+    const int n = pair / H, h = pair % H;
+    const int c = threadIdx.x;
+    const int s0 = __ldg(cu + n), s1 = __ldg(cu + n + 1);
+    const int span = kChunk * seg_chunks;
+    const int nseg = (s1 - s0 + span - 1) / span;
+    const size_t state_off = ((size_t)n * H + h) * D * D;
+    if (nseg == 0) {
+#pragma unroll
+        for (int j = 0; j < RB; ++j) {
+            const size_t i = state_off + (size_t)(rb * RB + j) * D + c;
+            final_state[i] = init_state ? init_state[i] : 0.f;
+        }
+        return;
+    }
+    if (nseg == 1) return;
+    const int64_t slot0 = (int64_t)(s0 / span) + n;
+    __shared__ __align__(16) float e[RB][D];
+#pragma unroll
+    for (int j = 0; j < RB; ++j)
+        e[j][c] = init_state ? init_state[state_off + (size_t)(rb * RB + j) * D + c] : 0.f;
+    __syncthreads();
+    for (int s = 0; s + 1 < nseg; ++s) {
+        const float* seg = seg_ws + ((size_t)(slot0 + s) * H + h) * 3u * D * D;
+        const float* Nm = seg;                     // N_s [v][c']
+        const float* Mm = seg + (size_t)D * D;     // M_s [k][c']
+        float acc[RB];
+#pragma unroll
+        for (int j = 0; j < RB; ++j) acc[j] = Nm[(size_t)(rb * RB + j) * D + c];
+#pragma unroll 4
+        for (int k4 = 0; k4 < D; k4 += 4) {
+            const float m0 = Mm[(size_t)(k4 + 0) * D + c], m1 = Mm[(size_t)(k4 + 1) * D + c];
+            const float m2 = Mm[(size_t)(k4 + 2) * D + c], m3 = Mm[(size_t)(k4 + 3) * D + c];
+#pragma unroll
+            for (int j = 0; j < RB; ++j) {
+                const float4 ev = *reinterpret_cast<const float4*>(&e[j][k4]);
+                acc[j] = fmaf(ev.x, m0, acc[j]);
+                acc[j] = fmaf(ev.y, m1, acc[j]);
+                acc[j] = fmaf(ev.z, m2, acc[j]);
+                acc[j] = fmaf(ev.w, m3, acc[j]);
+            }
+        }
+        __syncthreads();
+        float* E_next = seg_ws + ((size_t)(slot0 + s + 1) * H + h) * 3u * D * D + 2u * D * D;
+#pragma unroll
+        for (int j = 0; j < RB; ++j) {
+            e[j][c] = acc[j];
+            E_next[(size_t)(rb * RB + j) * D + c] = acc[j];
+        }
+        __syncthreads();
+    }
+}
+
+template <int D, typename OutT, int MODE>
+cudaError_t launch_mode(const gdr_prefill_args& a, const uint8_t* records,
+                        const WorkspaceLayout& lay, float* seg_ws, uint32_t* err, cudaStream_t st) {
+    auto kern = state_pass_kernel<D, OutT, MODE>;
+    const uint32_t smem = PassLayout<D, MODE>::dyn_bytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const unsigned grid = (unsigned)a.n_seqs * (unsigned)a.n_heads;
+    dim3 grid;
+    if (MODE == kFull) grid = dim3((unsigned)a.n_seqs * (unsigned)a.n_heads);
+    else grid = dim3((unsigned)lay.n_seg_slots, (unsigned)a.n_heads);
     kern<<<grid, kThreads, smem, st>>>(a.cu_seqlens, a.n_seqs, a.n_heads, records, a.init_state,
                                        static_cast<OutT*>(a.o), a.final_state, a.snap_interval,
-                                       a.snapshots, err);
+                                       a.snapshots, lay.seg_chunks, seg_ws, err);
     return cudaGetLastError();
+}
+
+template <int D, typename OutT>
+cudaError_t launch_typed(const gdr_prefill_args& a, const uint8_t* records,
+                         const WorkspaceLayout& lay, uint8_t* ws, uint32_t* err, cudaStream_t st) {
+    if (lay.seg_chunks <= 0) return launch_mode<D, OutT, kFull>(a, records, lay, nullptr, err, st);
+    float* seg_ws = reinterpret_cast<float*>(ws + lay.seg_off);
+    cudaError_t e = launch_mode<D, OutT, kLocal>(a, records, lay, seg_ws, err, st);
+    if (e != cudaSuccess) return e;
+    combine_kernel<D><<<dim3((unsigned)a.n_seqs * (unsigned)a.n_heads, D / 8), D, 0, st>>>(
+        a.cu_seqlens, a.n_heads, lay.seg_chunks, a.init_state, a.final_state, seg_ws);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_mode<D, OutT, kApply>(a, records, lay, seg_ws, err, st);
 }
 
 }  // namespace
 
-cudaError_t launch_state_pass(const gdr_prefill_args& a, const uint8_t* records, uint32_t* err,
+cudaError_t launch_state_pass(const gdr_prefill_args& a, const uint8_t* records,
+                              const WorkspaceLayout& lay, uint8_t* ws, uint32_t* err,
                               cudaStream_t st) {
     if ((int64_t)a.n_seqs * a.n_heads == 0) return cudaSuccess;
     if (a.d_k == 64)
-        return a.qkv_dtype == GDR_BF16 ? launch_typed<64, __nv_bfloat16>(a, records, err, st)
-                                       : launch_typed<64, float>(a, records, err, st);
-    return a.qkv_dtype == GDR_BF16 ? launch_typed<128, __nv_bfloat16>(a, records, err, st)
-                                   : launch_typed<128, float>(a, records, err, st);
+        return a.qkv_dtype == GDR_BF16 ? launch_typed<64, __nv_bfloat16>(a, records, lay, ws, err, st)
+                                       : launch_typed<64, float>(a, records, lay, ws, err, st);
+    return a.qkv_dtype == GDR_BF16 ? launch_typed<128, __nv_bfloat16>(a, records, lay, ws, err, st)
+                                   : launch_typed<128, float>(a, records, lay, ws, err, st);
 }
 
 }  // namespace gdr

@@ -179,23 +179,25 @@ gdr_status gdr_cumdecay(int n_seqs, int n_heads, int d_k, int64_t total_tokens,
  * The intra-chunk factors on their own (cumulative decay + intra-chunk
  * kernel), unpacked to plain fp32 arrays for inspection.  With
  * n_slots = floor(T_tot / 64) + N chunk slots, chunk j of sequence n lives in
- * slot floor((cu[n] + 64 j) / 64) + n; unused slots are left untouched.
- * Per slot and head (row r = token of the chunk, i = earlier token, c = key
- * channel, e = value channel):
- *   W  [n_slots, H, 64, d_k] = T diag(beta) (K * exp(g))
- *   U  [n_slots, H, 64, d_v] = T diag(beta) V
- *   P  [n_slots, H, 64, 64]  = scale * sum_c q[r,c] k[i,c] exp(g[r,c] - g[i,c]), i <= r
- *   Qg [n_slots, H, 64, d_k] = scale * Q * exp(g)
- *   Kd [n_slots, H, 64, d_k] = K * exp(g_last - g)
- *   gamma [n_slots, H, d_k]  = exp(g_last)
- * with T = (I + A)^-1, A[r,i] = beta_r sum_c k[r,c] k[i,c] exp(g[r,c] - g[i,c])
- * for i < r, g the chunk-local cumulative log decay.  Rows past the end of a
- * partial chunk are zero.  `workspace` as for gdr_prefill with the same
- * arguments; q, k, v, beta, log_a, cu_seqlens, scalar_decay and scale are
- * read from `args`, its outputs are ignored.
+ * slot floor(cu[n] / 64) + j + n; unused slots are left untouched.  For a
+ * chunk with start state S0, its effect on the state and outputs is
+ *     S_next = S0 Diag(gamma) + S0 BS^T + NC        O = Qt S0^T + PU
+ * where, with g the chunk-local cumulative log decay, Gamma = exp(g),
+ * A[r,i] = beta_r sum_c k[r,c] k[i,c] exp(g[r,c] - g[i,c]) (i < r),
+ * P[r,i] = scale sum_c q[r,c] k[i,c] exp(g[r,c] - g[i,c]) (i <= r),
+ * T = (I + A)^-1, W = T diag(beta)(K * Gamma), U = T diag(beta) V,
+ * Qg = scale Q * Gamma and Kd = K * exp(g_last - g):
+ *   Qt    [n_slots, H, 64, d_k]  = Qg - P W
+ *   PU    [n_slots, H, 64, d_v]  = P U
+ *   BS    [n_slots, H, d_k, d_k] = -Kd^T W
+ *   NC    [n_slots, H, d_v, d_k] = U^T Kd
+ *   gamma [n_slots, H, d_k]      = exp(g_last)
+ * Rows past the end of a partial chunk are zero.  `workspace` as for
+ * gdr_prefill with the same arguments; q, k, v, beta, log_a, cu_seqlens,
+ * scalar_decay and scale are read from `args`, its outputs are ignored.
  */
-gdr_status gdr_chunk_factors(const gdr_prefill_args* args, float* W, float* U, float* P,
-                             float* Qg, float* Kd, float* gamma, void* stream);
+gdr_status gdr_chunk_factors(const gdr_prefill_args* args, float* Qt, float* PU, float* BS,
+                             float* NC, float* gamma, void* stream);
 
 /* ------------------------------------------------------------------------
  * Decode: one token per sequence, state updated in place ("kda-graft",

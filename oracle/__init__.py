@@ -196,6 +196,9 @@ def chunk_factors(q, k, v, beta, log_a, start, end, h, scalar_decay=False, scale
       gamma_C = exp(g_last)
     so that, for start state S0, Delta = U - W S0^T, the outputs are
     O = Qg S0^T + P Delta and the end state is S0 Diag(gamma_C) + Delta^T Kd.
+    Substituting Delta gives the same map with S0-free matrices
+    Qt = Qg - P W, PU = P U, BS = -Kd^T W, NC = U^T Kd:
+    O = Qt S0^T + PU and S_next = S0 Diag(gamma_C) + S0 BS^T + NC.
     """
     Q = f64(q)[start:end, h]
     K = f64(k)[start:end, h]
@@ -220,12 +223,16 @@ def chunk_factors(q, k, v, beta, log_a, start, end, h, scalar_decay=False, scale
     U = Tm @ (b[:, None] * V)
     Qg = scale * Q * gam
     Kd = K * np.exp(g[-1][None, :] - g)
-    return dict(A=A, P=P, T=Tm, W=W, U=U, Qg=Qg, Kd=Kd, gamma_C=gam[-1], g=g)
+    # the chunk as an affine map of S0: S_next = S0 Diag(gamma_C) + S0 BS^T + NC,
+    # O = Qt S0^T + PU (Delta = U - W S0^T substituted)
+    return dict(A=A, P=P, T=Tm, W=W, U=U, Qg=Qg, Kd=Kd, gamma_C=gam[-1], g=g,
+                Qt=Qg - P @ W, PU=P @ U, BS=-(Kd.T @ W), NC=U.T @ Kd)
 
 
 def chunked_prefill(q, k, v, beta, log_a, cu_seqlens, scalar_decay=False, scale=1.0,
-                    init_state=None, chunk: int = 64):
-    """Prefill through the chunked form (fp64); must equal ``prefill``."""
+                    init_state=None, chunk: int = 64, affine: bool = False):
+    """Prefill through the chunked form (fp64); must equal ``prefill``.
+    ``affine`` uses the S0-free map (Qt, PU, BS, NC) instead of Delta."""
     q64, k64, v64 = f64(q), f64(k), f64(v)
     T, H, dk = q64.shape
     dv = v64.shape[2]
@@ -237,7 +244,11 @@ def chunked_prefill(q, k, v, beta, log_a, cu_seqlens, scalar_decay=False, scale=
         for h in range(H):
             f = chunk_factors(q64, k64, v64, beta, log_a, s, e, h, scalar_decay, scale)
             S0 = fin[s_idx, h]
-            Delta = f["U"] - f["W"] @ S0.T
-            o[s:e, h] = f["Qg"] @ S0.T + f["P"] @ Delta
-            fin[s_idx, h] = S0 * f["gamma_C"][None, :] + Delta.T @ f["Kd"]
+            if affine:
+                o[s:e, h] = f["Qt"] @ S0.T + f["PU"]
+                fin[s_idx, h] = S0 * f["gamma_C"][None, :] + S0 @ f["BS"].T + f["NC"]
+            else:
+                Delta = f["U"] - f["W"] @ S0.T
+                o[s:e, h] = f["Qg"] @ S0.T + f["P"] @ Delta
+                fin[s_idx, h] = S0 * f["gamma_C"][None, :] + Delta.T @ f["Kd"]
     return dict(o=o, final_state=fin)

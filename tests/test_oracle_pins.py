@@ -308,10 +308,11 @@ def test_chunk_form_matches_recurrence():
     for scalar in (False, True):
         la = -np.log1p(np.exp(-(3 + 2 * r.standard_normal((T, H) if scalar else (T, H, d)))))
         ref = oracle.prefill(q, k, v, beta, la, cu, scalar_decay=scalar, scale=0.5, init_state=S0)
-        ch = oracle.chunked_prefill(q, k, v, beta, la, cu, scalar_decay=scalar, scale=0.5,
-                                    init_state=S0)
-        np.testing.assert_allclose(ch["o"], ref["o"], rtol=0, atol=1e-10)
-        np.testing.assert_allclose(ch["final_state"], ref["final_state"], rtol=0, atol=1e-10)
+        for affine in (False, True):
+            ch = oracle.chunked_prefill(q, k, v, beta, la, cu, scalar_decay=scalar, scale=0.5,
+                                        init_state=S0, affine=affine)
+            np.testing.assert_allclose(ch["o"], ref["o"], rtol=0, atol=1e-10)
+            np.testing.assert_allclose(ch["final_state"], ref["final_state"], rtol=0, atol=1e-10)
 
 
 def test_cumdecay_restarts_per_chunk():

@@ -92,8 +92,9 @@ def test_chunk_factors(d, dtype, scalar):
                           scalar_decay=scalar, scale=w.scale)
     torch.cuda.synchronize()
     cu = inp["cu_seqlens"].tolist()
-    got = {k_: [] for k_ in ("W", "U", "Qg", "Kd", "P", "gamma")}
-    ref = {k_: [] for k_ in got}
+    names = ("Qt", "PU", "BS", "NC", "gamma")
+    got = {k_: [] for k_ in names}
+    ref = {k_: [] for k_ in names}
     for n in range(len(cu) - 1):
         for j, s in enumerate(range(cu[n], cu[n + 1], 64)):
             e = min(s + 64, cu[n + 1])
@@ -102,17 +103,17 @@ def test_chunk_factors(d, dtype, scalar):
             for h in range(2):
                 r = oracle.chunk_factors(inp["q"], inp["k"], inp["v"], inp["beta"], inp["log_a"],
                                          s, e, h, scalar, w.scale)
-                for name in ("W", "U", "Qg", "Kd"):
+                for name in ("Qt", "PU"):
                     got[name].append(f[name][slot, h, :L].cpu().double().numpy())
                     ref[name].append(r[name])
                     assert (f[name][slot, h, L:] == 0).all(), f"{name} rows past the chunk end"
-                got["P"].append(f["P"][slot, h, :L, :L].cpu().double().numpy())
-                ref["P"].append(r["P"])
-                assert (f["P"][slot, h].triu(1) == 0).all()
+                for name in ("BS", "NC"):
+                    got[name].append(f[name][slot, h].cpu().double().numpy())
+                    ref[name].append(r[name])
                 got["gamma"].append(f["gamma"][slot, h].cpu().double().numpy())
                 ref["gamma"].append(r["gamma_C"])
     # bound relative to the largest reference value of each factor over all chunks
-    for name in got:
+    for name in names:
         g_ = np.concatenate([x.ravel() for x in got[name]])
         r_ = np.concatenate([x.ravel() for x in ref[name]])
         assert_close_rel(g_, r_, 1e-5 if name == "gamma" else TOL, name)
@@ -131,10 +132,12 @@ def test_chunk_factors_extreme_decay():
     torch.cuda.synchronize()
     for slot, (s, e) in ((0, (0, 64)), (2, (64, 104))):
         ref = oracle.chunk_factors(inp["q"], inp["k"], inp["v"], inp["beta"], inp["log_a"], s, e, 0)
-        for name in ("W", "U", "Qg", "Kd"):
+        for name in ("Qt", "PU", "BS", "NC"):
             assert torch.isfinite(f[name][slot]).all()
-            assert_close_rel(f[name][slot, 0, :e - s], ref[name], TOL, name)
-        assert_close_rel(f["P"][slot, 0, :e - s, :e - s], ref["P"], TOL, "P")
+        assert_close_rel(f["Qt"][slot, 0, :e - s], ref["Qt"], TOL, "Qt")
+        assert_close_rel(f["PU"][slot, 0, :e - s], ref["PU"], TOL, "PU")
+        assert_close_rel(f["BS"][slot, 0], ref["BS"], TOL, "BS")
+        assert_close_rel(f["NC"][slot, 0], ref["NC"], TOL, "NC")
     o, fin, _ = _gpu_prefill(inp)
     _check(inp, o, fin, None, what="extreme decay")
 
@@ -167,6 +170,22 @@ def test_ragged_varlen(d, dtype, scalar, snap):
     inp = wl.make_prefill_inputs(w)
     o, fin, s = _gpu_prefill(inp)
     _check(inp, o, fin, s, what=f"ragged d{d} {dtype} scalar={scalar}")
+
+
+@pytest.mark.parametrize("d,scalar,snap", [(64, False, 256), (128, False, 128), (128, True, 0),
+                                           (64, True, 512)])
+def test_segmented_pass(d, scalar, snap):
+    """Few (sequence, head) pairs and long sequences: the sequential pass is
+    cut into segments (zero-state pass with the identity, fp32 chaining of the
+    segment maps, replay).  Ragged segment tails, an empty and a short
+    sequence, initial states and snapshots across segment boundaries."""
+    base = wl.GDN_LONG if scalar else wl.VARLEN
+    w = wl.shrink(base, n_heads=1, d_k=d, d_v=d, lengths=(2000, 0, 700, 1536, 65),
+                  init_std=0.1, snap_interval=snap, scale=0.9)
+    inp = wl.make_prefill_inputs(w)
+    import gated_delta_rule_150_b200 as gdr
+    o, fin, s = _gpu_prefill(inp)
+    _check(inp, o, fin, s, what=f"segmented d{d} scalar={scalar}")
 
 
 def test_all_empty_sequences_copy_init():
