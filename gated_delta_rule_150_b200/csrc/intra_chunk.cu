@@ -64,8 +64,8 @@ struct IntraLayout {
     static constexpr uint32_t sG = sV + (kStageQKV ? 64u * D * elem : 0u);
     static constexpr uint32_t in_bytes = sG + (SCALAR ? 0u : 64u * D * 4u);
     static constexpr uint32_t Ts = 0;                         // fp32 [64][kLd]
-    static constexpr uint32_t Yt = Ts + 64u * kLd * 4u;       // fp32 [3][16][16]
-    static constexpr uint32_t WUt = al1024(Yt + 3072u);       // bf16 [2D][64]
+    static constexpr uint32_t Yt = Ts + 64u * kLd * 4u;       // fp32 [32][32] scratch
+    static constexpr uint32_t WUt = al1024(Yt + 4096u);       // bf16 [2D][64]
     static constexpr uint32_t r1 = al1024(umax(in_bytes, WUt + 256u * D));
     // region 2: A/P operands, then As, Pt, Tb
     static constexpr uint32_t XA = r1;                        // bf16 [128][D]
@@ -120,6 +120,27 @@ __device__ __forceinline__ uint4 pack8(const float (&x)[8]) {
 }
 
 __device__ __forceinline__ float4 f4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+
+// acc[2][4] += X[xr, xr+1][xk .. xk+16) * Y[yk .. yk+16)[yc .. yc+4): one
+// 16-deep step of a 2 x 4 output tile (fp32, shared-memory operands; X has
+// row stride kLd, Y row stride LDY).
+template <int LDY>
+__device__ __forceinline__ void tile16(const float* X, int xr, int xk, const float* Y, int yk, int yc,
+                                       float (&a0)[4], float (&a1)[4]) {
+#pragma unroll
+    for (int m4 = 0; m4 < 4; ++m4) {
+        const float4 x0 = f4(X + xr * kLd + xk + 4 * m4), x1 = f4(X + (xr + 1) * kLd + xk + 4 * m4);
+        const float x0v[4] = {x0.x, x0.y, x0.z, x0.w}, x1v[4] = {x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+            const float4 yv = f4(Y + (yk + 4 * m4 + qq) * LDY + yc);
+            a0[0] = fmaf(x0v[qq], yv.x, a0[0]); a0[1] = fmaf(x0v[qq], yv.y, a0[1]);
+            a0[2] = fmaf(x0v[qq], yv.z, a0[2]); a0[3] = fmaf(x0v[qq], yv.w, a0[3]);
+            a1[0] = fmaf(x1v[qq], yv.x, a1[0]); a1[1] = fmaf(x1v[qq], yv.y, a1[1]);
+            a1[2] = fmaf(x1v[qq], yv.z, a1[2]); a1[3] = fmaf(x1v[qq], yv.w, a1[3]);
+        }
+    }
+}
 
 // Stage one [64 x D] row block of a token-major tensor into shared memory
 // (rows past the chunk end are zero-filled).
@@ -242,7 +263,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                 float mb[8];
                 load8f(sG + (size_t)min(16 * b + 8, len - 1) * D + c0, mb);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) ecross[b][e] = expf(mb[e] - mj[e]);
+                for (int e = 0; e < 8; ++e) ecross[b][e] = __expf(mb[e] - mj[e]);
             }
         }
 #pragma unroll
@@ -275,9 +296,10 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     float em[8], eld[8];        // exp(m_jb), exp(g_last - m_jb)
     if (!SCALAR) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) { em[e] = expf(mj[e]); eld[e] = expf(gl[e] - mj[e]); }
+        for (int e = 0; e < 8; ++e) { em[e] = __expf(mj[e]); eld[e] = __expf(gl[e] - mj[e]); }
     }
     uint32_t pb1[8][RPT / 2], pb2[8][RPT / 2], pkd[8][RPT / 2];   // transposed bf16 pairs
+    float p_b1[8], p_bv[8], p_kd[8];                               // even row of the pair
 #pragma unroll
     for (int u = 0; u < RPT; ++u) {
         const int r = r0 + u;
@@ -311,7 +333,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 const float d = gr[e] - mj[e];
-                const float F = expf(d), Fi = expf(-d);
+                const float F = __expf(d), Fi = __expf(-d);
                 xq[e] = scale * qv[e] * F;
                 xk[e] = kv[e] * F;
                 kk0[e] = kv[e] * Fi;
@@ -322,13 +344,13 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         } else {
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                const float G = expf(gr[e]);
+                const float G = __expf(gr[e]);
                 xq[e] = SCALAR ? scale * qv[e] : 0.f;
                 xk[e] = SCALAR ? kv[e] : 0.f;
                 kk0[e] = 0.f;
                 b1[e] = br * kv[e] * G;
                 qg[e] = scale * qv[e] * G;
-                kd[e] = kv[e] * expf(gl[e] - gr[e]);
+                kd[e] = kv[e] * __expf(gl[e] - gr[e]);
             }
         }
         // A-side operand rows r (queries) and 64 + r (keys)
@@ -346,18 +368,18 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
             }
         }
         *reinterpret_cast<uint4*>(Qgs + sw128_chunk(64, r, cg)) = pack8(qg);
-        // transposed operands: collect pairs of rows per channel
+        // transposed operands: pack pairs of rows (u-1, u) per channel
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
             const float bv = br * vv[e];
             if ((u & 1) == 0) {
-                pb1[e][u / 2] = pack_bf16(b1[e], 0.f);
-                pb2[e][u / 2] = pack_bf16(bv, 0.f);
-                pkd[e][u / 2] = pack_bf16(kd[e], 0.f);
+                p_b1[e] = b1[e];
+                p_bv[e] = bv;
+                p_kd[e] = kd[e];
             } else {
-                pb1[e][u / 2] = (pb1[e][u / 2] & 0xFFFFu) | (pack_bf16(0.f, b1[e]) & 0xFFFF0000u);
-                pb2[e][u / 2] = (pb2[e][u / 2] & 0xFFFFu) | (pack_bf16(0.f, bv) & 0xFFFF0000u);
-                pkd[e][u / 2] = (pkd[e][u / 2] & 0xFFFFu) | (pack_bf16(0.f, kd[e]) & 0xFFFF0000u);
+                pb1[e][u / 2] = pack_bf16(p_b1[e], b1[e]);
+                pb2[e][u / 2] = pack_bf16(p_bv[e], bv);
+                pkd[e][u / 2] = pack_bf16(p_kd[e], kd[e]);
             }
         }
     }
@@ -424,7 +446,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
             tmem_ld_wait();
             const float gr = Gs[rr];
 #pragma unroll
-            for (int i = 0; i < 64; ++i) vrow[i] = (i <= lim) ? vrow[i] * expf(gr - Gs[i]) : 0.f;
+            for (int i = 0; i < 64; ++i) vrow[i] = (i <= lim) ? vrow[i] * __expf(gr - Gs[i]) : 0.f;
         }
         if (!SCALAR && bad_chunk) {
             // exact path: every term with its own exp (chunks with extreme decay only)
@@ -465,7 +487,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     }
     __syncthreads();
 
-    // ---- T = (I + A)^-1: 16x16 diagonal blocks, then three block levels ------
+    // ---- T = (I + A)^-1: 16x16 diagonal blocks, then block merges -----------
     if (tid < 64) {
         const int b = tid >> 4, cc = tid & 15, o = 16 * b;
         float x[16];
@@ -488,57 +510,42 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         }
     }
     __syncthreads();
-#pragma unroll
-    for (int d = 1; d <= 3; ++d) {
-        const int ntiles = (4 - d) * 32;
-        const int p = tid >> 5, t = tid & 31;
-        const int rr0 = 2 * (t >> 2), cq = t & 3;
-        const int b = d + p, j = p;
-        if (tid < ntiles) {
-            // Y_bj = sum_{l=j}^{b-1} A_bl T_lj, a 2 x 4 tile per thread
-            float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int l = j; l < b; ++l) {
-#pragma unroll
-                for (int m4 = 0; m4 < 4; ++m4) {
-                    const float4 a0 = f4(As + (16 * b + rr0) * kLd + 16 * l + 4 * m4);
-                    const float4 a1 = f4(As + (16 * b + rr0 + 1) * kLd + 16 * l + 4 * m4);
-                    const float a0v[4] = {a0.x, a0.y, a0.z, a0.w}, a1v[4] = {a1.x, a1.y, a1.z, a1.w};
-#pragma unroll
-                    for (int qq = 0; qq < 4; ++qq) {
-                        const float4 tv = f4(Ts + (16 * l + 4 * m4 + qq) * kLd + 16 * j + 4 * cq);
-                        y0[0] = fmaf(a0v[qq], tv.x, y0[0]); y0[1] = fmaf(a0v[qq], tv.y, y0[1]);
-                        y0[2] = fmaf(a0v[qq], tv.z, y0[2]); y0[3] = fmaf(a0v[qq], tv.w, y0[3]);
-                        y1[0] = fmaf(a1v[qq], tv.x, y1[0]); y1[1] = fmaf(a1v[qq], tv.y, y1[1]);
-                        y1[2] = fmaf(a1v[qq], tv.z, y1[2]); y1[3] = fmaf(a1v[qq], tv.w, y1[3]);
-                    }
-                }
-            }
-            *reinterpret_cast<float4*>(Yt + p * 256 + rr0 * 16 + 4 * cq) = make_float4(y0[0], y0[1], y0[2], y0[3]);
-            *reinterpret_cast<float4*>(Yt + p * 256 + (rr0 + 1) * 16 + 4 * cq) = make_float4(y1[0], y1[1], y1[2], y1[3]);
-        }
-        __syncthreads();
-        if (tid < ntiles) {
-            // T_bj = -T_bb Y_bj (T_bb is lower triangular with zeros above)
-            float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int m4 = 0; m4 < 4; ++m4) {
-                const float4 t0 = f4(Ts + (16 * b + rr0) * kLd + 16 * b + 4 * m4);
-                const float4 t1 = f4(Ts + (16 * b + rr0 + 1) * kLd + 16 * b + 4 * m4);
-                const float t0v[4] = {t0.x, t0.y, t0.z, t0.w}, t1v[4] = {t1.x, t1.y, t1.z, t1.w};
-#pragma unroll
-                for (int qq = 0; qq < 4; ++qq) {
-                    const float4 yv = f4(Yt + p * 256 + (4 * m4 + qq) * 16 + 4 * cq);
-                    z0[0] = fmaf(t0v[qq], yv.x, z0[0]); z0[1] = fmaf(t0v[qq], yv.y, z0[1]);
-                    z0[2] = fmaf(t0v[qq], yv.z, z0[2]); z0[3] = fmaf(t0v[qq], yv.w, z0[3]);
-                    z1[0] = fmaf(t1v[qq], yv.x, z1[0]); z1[1] = fmaf(t1v[qq], yv.y, z1[1]);
-                    z1[2] = fmaf(t1v[qq], yv.z, z1[2]); z1[3] = fmaf(t1v[qq], yv.w, z1[3]);
-                }
-            }
-            *reinterpret_cast<float4*>(Ts + (16 * b + rr0) * kLd + 16 * j + 4 * cq) = make_float4(-z0[0], -z0[1], -z0[2], -z0[3]);
-            *reinterpret_cast<float4*>(Ts + (16 * b + rr0 + 1) * kLd + 16 * j + 4 * cq) = make_float4(-z1[0], -z1[1], -z1[2], -z1[3]);
-        }
-        __syncthreads();
+    // first-level merges inside each 32-row half: T_10 = -T_11 A_10 T_00 and
+    // T_32 = -T_33 A_32 T_22 (a 2 x 4 tile per thread, 64 threads)
+    const int t32 = tid & 31, rr0 = 2 * (t32 >> 2), c4 = 4 * (t32 & 3);
+    if (tid < 64) {
+        const int p = tid >> 5, b = 2 * p + 1, j = 2 * p;
+        float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
+        tile16<kLd>(As, 16 * b + rr0, 16 * j, Ts, 16 * j, 16 * j + c4, y0, y1);
+        *reinterpret_cast<float4*>(Yt + p * 256 + rr0 * 16 + c4) = make_float4(y0[0], y0[1], y0[2], y0[3]);
+        *reinterpret_cast<float4*>(Yt + p * 256 + (rr0 + 1) * 16 + c4) = make_float4(y1[0], y1[1], y1[2], y1[3]);
     }
+    __syncthreads();
+    if (tid < 64) {
+        const int p = tid >> 5, b = 2 * p + 1, j = 2 * p;
+        float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
+        tile16<16>(Ts, 16 * b + rr0, 16 * b, Yt + p * 256, 0, c4, z0, z1);
+        *reinterpret_cast<float4*>(Ts + (16 * b + rr0) * kLd + 16 * j + c4) = make_float4(-z0[0], -z0[1], -z0[2], -z0[3]);
+        *reinterpret_cast<float4*>(Ts + (16 * b + rr0 + 1) * kLd + 16 * j + c4) = make_float4(-z1[0], -z1[1], -z1[2], -z1[3]);
+    }
+    __syncthreads();
+    // bottom-left 32 x 32 block, blocks (b, j) with b in {2, 3}, j in {0, 1}:
+    //   Y_bj = sum_{l=j}^{1} A_bl T_lj        T_bj = -sum_{l=2}^{b} T_bl Y_lj
+    {
+        const int q = tid >> 5, b = 2 + (q >> 1), j = q & 1;
+        float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int l = j; l <= 1; ++l)
+            tile16<kLd>(As, 16 * b + rr0, 16 * l, Ts, 16 * l, 16 * j + c4, y0, y1);
+        *reinterpret_cast<float4*>(Yt + (16 * (b - 2) + rr0) * 32 + 16 * j + c4) = make_float4(y0[0], y0[1], y0[2], y0[3]);
+        *reinterpret_cast<float4*>(Yt + (16 * (b - 2) + rr0 + 1) * 32 + 16 * j + c4) = make_float4(y1[0], y1[1], y1[2], y1[3]);
+        __syncthreads();
+        float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int l = 2; l <= b; ++l)
+            tile16<32>(Ts, 16 * b + rr0, 16 * l, Yt, 16 * (l - 2), 16 * j + c4, z0, z1);
+        *reinterpret_cast<float4*>(Ts + (16 * b + rr0) * kLd + 16 * j + c4) = make_float4(-z0[0], -z0[1], -z0[2], -z0[3]);
+        *reinterpret_cast<float4*>(Ts + (16 * b + rr0 + 1) * kLd + 16 * j + c4) = make_float4(-z1[0], -z1[1], -z1[2], -z1[3]);
+    }
+    __syncthreads();
     // T -> bf16 operand tile [64 r][64 i] (zero above the diagonal)
     for (int qd = tid; qd < 512; qd += kThreads) {
         const int r = qd >> 3, jj = qd & 7;
@@ -612,6 +619,10 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     tc_fence_after_sync();
 
     // ---- record: Qt = Qg - P W, PU, BS = -Kd^T W, NC = U^T Kd, gamma ----------
+    // assembled in shared memory below Qgs (everything there is dead once the
+    // MMAs above have completed) and written with one bulk store
+    uint8_t* srec = sm;
+    static_assert(R.bytes <= L::Qgs, "record staging fits below Qgs");
     {
         // rows of the M = 64 products live in lanes 16 w + l (l < 16)
         const int r64 = 16 * warp + lane;
@@ -631,8 +642,8 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                     float a[8], b[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) { a[e] = qgv[e] - pw[8 * jj + e]; b[e] = pu[8 * jj + e]; }
-                    *reinterpret_cast<uint4*>(rec + R.Qt + sw128_chunk(64, r64, chunk)) = pack8(a);
-                    *reinterpret_cast<uint4*>(rec + R.PU + sw128_chunk(64, r64, chunk)) = pack8(b);
+                    *reinterpret_cast<uint4*>(srec + R.Qt + sw128_chunk(64, r64, chunk)) = pack8(a);
+                    *reinterpret_cast<uint4*>(srec + R.PU + sw128_chunk(64, r64, chunk)) = pack8(b);
                 }
             }
         }
@@ -651,16 +662,23 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                     float a[8], b[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) { a[e] = -bs[8 * jj + e]; b[e] = nc[8 * jj + e]; }
-                    *reinterpret_cast<uint4*>(rec + R.BS + sw128_chunk(D, rD, chunk)) = pack8(a);
-                    *reinterpret_cast<uint4*>(rec + R.NC + sw128_chunk(D, rD, chunk)) = pack8(b);
+                    *reinterpret_cast<uint4*>(srec + R.BS + sw128_chunk(D, rD, chunk)) = pack8(a);
+                    *reinterpret_cast<uint4*>(srec + R.NC + sw128_chunk(D, rD, chunk)) = pack8(b);
                 }
             }
         }
-        if (tid < D) reinterpret_cast<float*>(rec + R.gamma)[tid] = expf(Gl[tid]);
+        if (tid < D) reinterpret_cast<float*>(srec + R.gamma)[tid] = expf(Gl[tid]);
     }
+    fence_proxy_async_smem();
     tc_fence_before_sync();
     __syncthreads();
-    if (tid == 0 && failed) atomicOr(err, 1u);
+    if (tid == 0) {
+        bulk_s2g(rec, srec, R.bytes);
+        bulk_commit_group();
+        bulk_wait_group_read0();
+        if (failed) atomicOr(err, 1u);
+    }
+    __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 

@@ -251,39 +251,74 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         const int t0 = s0 + k * kChunk;
         const int len = min(kChunk, s1 - t0);
         if (!mbar_wait(&full[st], (uint32_t)(k / ST) & 1)) failed = true;
+        const float* gam = reinterpret_cast<const float*>(sm + L::GAS + st * 4u * D);
+        const uint8_t* nc = sm + L::NCS + st * 2u * D * D;
+        // gamma and this row's NC, read while the MMAs of chunk k finish
+        constexpr bool kPre = (kNT == 1);
+        float gv[kPre ? CW : 1];
+        uint32_t nvp[kPre ? CW / 2 : 1];
+        if (kPre && active) {
+#pragma unroll
+            for (int j = 0; j < CW; j += 4) {
+                const float4 g4 = *reinterpret_cast<const float4*>(gam + cb + j);
+                gv[j] = g4.x; gv[j + 1] = g4.y; gv[j + 2] = g4.z; gv[j + 3] = g4.w;
+            }
+            if (!is_x) {
+#pragma unroll
+                for (int j = 0; j < CW; j += 8) {
+                    const uint4 u = *reinterpret_cast<const uint4*>(nc + sw128_chunk(D, srow, (cb + j) / 8));
+                    nvp[j / 2] = u.x; nvp[j / 2 + 1] = u.y; nvp[j / 2 + 2] = u.z; nvp[j / 2 + 3] = u.w;
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < CW / 2; ++j) nvp[j] = 0u;
+            }
+        }
         if (!mbar_wait(&mma_bar, (uint32_t)k & 1)) failed = true;
         mmas_waited = k + 1;
         tc_fence_after_sync();
 
         // ---- state: S = S * gamma + Z (+ NC for S rows), critical path ----------
-        const float* gam = reinterpret_cast<const float*>(sm + L::GAS + st * 4u * D);
-        const uint8_t* nc = sm + L::NCS + st * 2u * D * D;
 #pragma unroll
         for (int t = 0; t < kNT; ++t) {
             const bool x_tile = (MODE == kLocal) && (t == 1 || is_x);
 #pragma unroll
-            for (int p = 0; p < CW / 16; ++p) {
-                float z[16];
-                tmem_ld16(tmem + lane_base + (uint32_t)(t * 128) + cb + 16 * p, z);
+            for (int p = 0; p < CW / 32; ++p) {
+                float z[32];
+                tmem_ld16(tmem + lane_base + (uint32_t)(t * 128) + cb + 32 * p, *reinterpret_cast<float(*)[16]>(z));
+                tmem_ld16(tmem + lane_base + (uint32_t)(t * 128) + cb + 32 * p + 16, *reinterpret_cast<float(*)[16]>(z + 16));
                 tmem_ld_wait();
                 if (active) {
 #pragma unroll
-                    for (int jj = 0; jj < 2; ++jj) {
-                        const int j = 16 * p + 8 * jj, c = cb + j;
-                        const float4 g0 = *reinterpret_cast<const float4*>(gam + c);
-                        const float4 g1 = *reinterpret_cast<const float4*>(gam + c + 4);
-                        float nv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                        if (!x_tile) {
-                            const uint4 u = *reinterpret_cast<const uint4*>(nc + sw128_chunk(D, srow, c / 8));
-                            const float2 n0 = unpack_bf16(u.x), n1 = unpack_bf16(u.y);
-                            const float2 n2 = unpack_bf16(u.z), n3 = unpack_bf16(u.w);
-                            nv[0] = n0.x; nv[1] = n0.y; nv[2] = n1.x; nv[3] = n1.y;
-                            nv[4] = n2.x; nv[5] = n2.y; nv[6] = n3.x; nv[7] = n3.y;
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const int j = 32 * p + 8 * jj, c = cb + j;
+                        float g8[8], n8[8];
+                        if (kPre) {
+#pragma unroll
+                            for (int e2 = 0; e2 < 4; ++e2) {
+                                const float2 f = unpack_bf16(nvp[(j + 2 * e2) / 2]);
+                                n8[2 * e2] = f.x; n8[2 * e2 + 1] = f.y;
+                            }
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) g8[e] = gv[j + e];
+                        } else {
+                            const float4 g0 = *reinterpret_cast<const float4*>(gam + c);
+                            const float4 g1 = *reinterpret_cast<const float4*>(gam + c + 4);
+                            g8[0] = g0.x; g8[1] = g0.y; g8[2] = g0.z; g8[3] = g0.w;
+                            g8[4] = g1.x; g8[5] = g1.y; g8[6] = g1.z; g8[7] = g1.w;
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) n8[e] = 0.f;
+                            if (!x_tile) {
+                                const uint4 u = *reinterpret_cast<const uint4*>(nc + sw128_chunk(D, srow, c / 8));
+                                const float2 n0 = unpack_bf16(u.x), n1 = unpack_bf16(u.y);
+                                const float2 n2 = unpack_bf16(u.z), n3 = unpack_bf16(u.w);
+                                n8[0] = n0.x; n8[1] = n0.y; n8[2] = n1.x; n8[3] = n1.y;
+                                n8[4] = n2.x; n8[5] = n2.y; n8[6] = n3.x; n8[7] = n3.y;
+                            }
                         }
-                        const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
 #pragma unroll
                         for (int e = 0; e < 8; ++e)
-                            S[t][j + e] = fmaf(S[t][j + e], gv[e], z[8 * jj + e] + nv[e]);
+                            S[t][j + e] = fmaf(S[t][j + e], g8[e], z[8 * jj + e] + n8[e]);
                         write_operand(t, j);
                     }
                 }
@@ -371,66 +406,103 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
 
 // Chains the segments' affine maps into each segment's start state:
 //     E_0 = init,   E_{s+1} = E_s M_s + N_s       (fp32, in the chain's order)
-// Rows of the state are independent, so a CTA owns 8 state rows of one
-// (sequence, head) and thread c' the output column c'.  E_s goes to the
-// workspace of segment s (its start state); the last segment's own map is not
-// needed (replaying that segment produces the final state).  An empty sequence
-// has no segment: its final state is its initial state.
+// Rows of the state are independent, so a CTA owns kCombineRows state rows of
+// one (sequence, head); thread (j, q) computes row j, columns 4q .. 4q+3.  Each
+// step's M_s and the CTA's rows of N_s arrive by bulk copies one step ahead
+// (two buffers).  E_s goes to the workspace of segment s (its start state); the
+// last segment's own map is not needed (replaying that segment produces the
+// final state).  An empty sequence has no segment: its final state is its
+// initial state.
+constexpr int kCombineRows = 8;
+
 template <int D>
-__global__ void __launch_bounds__(D)
+struct CombineLayout {
+    static constexpr uint32_t M0 = 0;                                   // 2 x [D x D] fp32
+    static constexpr uint32_t N0 = 2u * D * D * 4u;                     // 2 x [rows x D] fp32
+    static constexpr uint32_t E = N0 + 2u * kCombineRows * D * 4u;      // [rows x D] fp32
+    static constexpr uint32_t bytes = E + kCombineRows * D * 4u;
+    static constexpr uint32_t dyn_bytes = bytes + 128u;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kCombineRows * D / 4)
 combine_kernel(const int32_t* __restrict__ cu, int H, int seg_chunks, const float* init_state,
-               float* final_state, float* seg_ws) {
-    constexpr int RB = 8;
+               float* final_state, float* seg_ws, uint32_t* err) {
+    using L = CombineLayout<D>;
+    constexpr int RB = kCombineRows;
+    constexpr int QD = D / 4;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
+                                             ~static_cast<uintptr_t>(127));
+    __shared__ uint64_t full[2];
     const int pair = blockIdx.x, rb = blockIdx.y;
     const int n = pair / H, h = pair % H;
-    const int c = threadIdx.x;
+    const int tid = threadIdx.x, j = tid / QD, q = tid % QD;
     const int s0 = __ldg(cu + n), s1 = __ldg(cu + n + 1);
     const int span = kChunk * seg_chunks;
     const int nseg = (s1 - s0 + span - 1) / span;
     const size_t state_off = ((size_t)n * H + h) * D * D;
+    const size_t row_off = (size_t)(rb * RB + j) * D + 4 * q;
     if (nseg == 0) {
-#pragma unroll
-        for (int j = 0; j < RB; ++j) {
-            const size_t i = state_off + (size_t)(rb * RB + j) * D + c;
-            final_state[i] = init_state ? init_state[i] : 0.f;
-        }
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (init_state) x = *reinterpret_cast<const float4*>(init_state + state_off + row_off);
+        *reinterpret_cast<float4*>(final_state + state_off + row_off) = x;
         return;
     }
     if (nseg == 1) return;
     const int64_t slot0 = (int64_t)(s0 / span) + n;
-    __shared__ __align__(16) float e[RB][D];
-#pragma unroll
-    for (int j = 0; j < RB; ++j)
-        e[j][c] = init_state ? init_state[state_off + (size_t)(rb * RB + j) * D + c] : 0.f;
+    float* e = reinterpret_cast<float*>(sm + L::E);
+    auto seg_ptr = [&](int s) { return seg_ws + ((size_t)(slot0 + s) * H + h) * 3u * D * D; };
+    auto issue = [&](int s) {      // thread 0: M_s and this CTA's rows of N_s
+        const int b = s & 1;
+        mbar_arrive_expect_tx(&full[b], (uint32_t)(D * D * 4 + RB * D * 4));
+        bulk_g2s(sm + L::M0 + b * D * D * 4u, seg_ptr(s) + (size_t)D * D, D * D * 4u, &full[b]);
+        bulk_g2s(sm + L::N0 + b * RB * D * 4u, seg_ptr(s) + (size_t)rb * RB * D, RB * D * 4u, &full[b]);
+    };
+    if (tid == 0) {
+        mbar_init(&full[0], 1);
+        mbar_init(&full[1], 1);
+        fence_mbar_init();
+    }
+    {
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (init_state) x = *reinterpret_cast<const float4*>(init_state + state_off + row_off);
+        *reinterpret_cast<float4*>(e + j * D + 4 * q) = x;
+    }
     __syncthreads();
+    int issued = 0, consumed = 0;                  // thread 0's bookkeeping (steps)
+    if (tid == 0) {
+        issue(0);
+        issued = 1;
+        if (nseg > 2) { issue(1); issued = 2; }
+    }
+    bool failed = false;
     for (int s = 0; s + 1 < nseg; ++s) {
-        const float* seg = seg_ws + ((size_t)(slot0 + s) * H + h) * 3u * D * D;
-        const float* Nm = seg;                     // N_s [v][c']
-        const float* Mm = seg + (size_t)D * D;     // M_s [k][c']
-        float acc[RB];
-#pragma unroll
-        for (int j = 0; j < RB; ++j) acc[j] = Nm[(size_t)(rb * RB + j) * D + c];
-#pragma unroll 4
-        for (int k4 = 0; k4 < D; k4 += 4) {
-            const float m0 = Mm[(size_t)(k4 + 0) * D + c], m1 = Mm[(size_t)(k4 + 1) * D + c];
-            const float m2 = Mm[(size_t)(k4 + 2) * D + c], m3 = Mm[(size_t)(k4 + 3) * D + c];
-#pragma unroll
-            for (int j = 0; j < RB; ++j) {
-                const float4 ev = *reinterpret_cast<const float4*>(&e[j][k4]);
-                acc[j] = fmaf(ev.x, m0, acc[j]);
-                acc[j] = fmaf(ev.y, m1, acc[j]);
-                acc[j] = fmaf(ev.z, m2, acc[j]);
-                acc[j] = fmaf(ev.w, m3, acc[j]);
-            }
+        const int b = s & 1;
+        if (!mbar_wait(&full[b], (uint32_t)(s >> 1) & 1)) failed = true;
+        consumed = s + 1;
+        const float* Mm = reinterpret_cast<const float*>(sm + L::M0 + b * D * D * 4u);
+        const float* Nm = reinterpret_cast<const float*>(sm + L::N0 + b * RB * D * 4u);
+        float4 acc = *reinterpret_cast<const float4*>(Nm + j * D + 4 * q);
+#pragma unroll 8
+        for (int k = 0; k < D; ++k) {
+            const float ek = e[j * D + k];
+            const float4 m = *reinterpret_cast<const float4*>(Mm + k * D + 4 * q);
+            acc.x = fmaf(ek, m.x, acc.x);
+            acc.y = fmaf(ek, m.y, acc.y);
+            acc.z = fmaf(ek, m.z, acc.z);
+            acc.w = fmaf(ek, m.w, acc.w);
         }
+        if (__syncthreads_or(failed)) break;          // everyone is done with e and buffer b
+        *reinterpret_cast<float4*>(e + j * D + 4 * q) = acc;
+        *reinterpret_cast<float4*>(seg_ptr(s + 1) + 2u * D * D + row_off) = acc;
+        if (tid == 0 && s + 2 <= nseg - 2) { issue(s + 2); issued = s + 3; }
         __syncthreads();
-        float* E_next = seg_ws + ((size_t)(slot0 + s + 1) * H + h) * 3u * D * D + 2u * D * D;
-#pragma unroll
-        for (int j = 0; j < RB; ++j) {
-            e[j][c] = acc[j];
-            E_next[(size_t)(rb * RB + j) * D + c] = acc[j];
-        }
-        __syncthreads();
+    }
+    if (failed && tid == 0) {
+        atomicOr(err, 1u);
+        // let the copies already issued land before the CTA exits (bounded waits)
+        for (int c = consumed; c < issued; ++c) mbar_wait(&full[c & 1], (uint32_t)(c >> 1) & 1);
     }
 }
 
@@ -457,8 +529,13 @@ cudaError_t launch_typed(const gdr_prefill_args& a, const uint8_t* records,
     float* seg_ws = reinterpret_cast<float*>(ws + lay.seg_off);
     cudaError_t e = launch_mode<D, OutT, kLocal>(a, records, lay, seg_ws, err, st);
     if (e != cudaSuccess) return e;
-    combine_kernel<D><<<dim3((unsigned)a.n_seqs * (unsigned)a.n_heads, D / 8), D, 0, st>>>(
-        a.cu_seqlens, a.n_heads, lay.seg_chunks, a.init_state, a.final_state, seg_ws);
+    auto ck = combine_kernel<D>;
+    e = cudaFuncSetAttribute(ck, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)CombineLayout<D>::dyn_bytes);
+    if (e != cudaSuccess) return e;
+    ck<<<dim3((unsigned)a.n_seqs * (unsigned)a.n_heads, D / kCombineRows), kCombineRows * D / 4,
+         CombineLayout<D>::dyn_bytes, st>>>(a.cu_seqlens, a.n_heads, lay.seg_chunks, a.init_state,
+                                           a.final_state, seg_ws, err);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     return launch_mode<D, OutT, kApply>(a, records, lay, seg_ws, err, st);
