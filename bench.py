@@ -150,11 +150,24 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Slowest rank's value (timing is taken as the max over ranks)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(base_seed: int, set_index: int, rank: int) -> int:
+    """Seed of input set `set_index` on `rank`: every rank draws its own batch
+    (weak scaling: the units all ranks process add up)."""
+    return base_seed + 7919 * set_index + 100003 * rank
+
+
+def job_throughput(units_per_rank: int, world: int, steps: int, max_ms: float) -> float:
+    """Whole-job units per second: all ranks' units over the slowest rank's time."""
+    return world * units_per_rank * steps / (max_ms * 1e-3)
 
 
 def timed(fn, n, stream):
@@ -180,7 +193,7 @@ class PrefillSets:
         self.w = w
         self.sets = []
         for i in range(n_sets):
-            wi = wl.shrink(w, seed=w.seed + 7919 * i + 100003 * rank)
+            wi = wl.shrink(w, seed=rank_seed(w.seed, i, rank))
             inp = wl.make_prefill_inputs(wi, device="cuda", draw_device="cuda")
             T, H, dk = inp["q"].shape
             dv = inp["v"].shape[-1]
@@ -208,16 +221,19 @@ class PrefillSets:
         self.footprint = sum(sum(t.numel() * t.element_size() for t in s["prep"]._keep
                                  if torch.is_tensor(t)) for s in self.sets)
 
-    def step(self, i, stages=(0, 2)):
+    def step(self, i, stages=(0, 1)):
         self.sets[i % len(self.sets)]["prep"].run(stages)
 
 
+STAGES = ("intra_chunk", "state_pass")
+
+
 def stage_times(ps: PrefillSets, n: int, stream) -> list:
-    """Device time of each of the three prefill kernels launched alone (ms)."""
+    """Device time of each prefill stage launched alone (ms)."""
     for i in range(len(ps.sets)):
         ps.step(i)
     out = []
-    for s in range(3):
+    for s in range(len(STAGES)):
         out.append(timed(lambda i: ps.step(i, (s, s)), n, stream))
     return out
 
@@ -320,7 +336,8 @@ def run_gdr(args):
     pk = peaks()
 
     # ---- main workload: graft-layer prefill, 4 rotating input sets ----------
-    ps = PrefillSets(gdr, wl.GRAFT_LAYER, 4, rank)
+    n_sets = args.sets or (4 if args.workload != wl.VARLEN.name else 1)
+    ps = PrefillSets(gdr, wl.PREFILL_WORKLOADS[args.workload], n_sets, rank)
     for i in range(args.warmup):
         ps.step(i)
     torch.cuda.synchronize()
@@ -341,20 +358,27 @@ def run_gdr(args):
     ms_local = start.elapsed_time(end)
     ms_total = max_over_ranks(ms_local, world)
     ms_step = ms_total / args.steps
-    value = world * ps.T * args.steps / (ms_total * 1e-3)
+    value = job_throughput(ps.T, world, args.steps, ms_total)
 
-    # ---- the three kernels alone -> dominant kernel roofline --------------------
-    names = ["cumdecay", "intra_chunk", "state_pass"]
-    sources = ["gated_delta_rule_150_b200/csrc/cumdecay.cu",
-               "gated_delta_rule_150_b200/csrc/intra_chunk.cu",
-               "gated_delta_rule_150_b200/csrc/state_pass.cu"]
+    launches_per_step = gdr.kernel_count(ps.n, ps.H, ps.dk, ps.dv, ps.T, ps.w.scalar_decay)
+    # the cumulative-decay kernel on its own (inside the prefill it is fused
+    # into the intra-chunk stage)
+    la, cu0 = ps.sets[0]["inp"]["log_a"], ps.sets[0]["inp"]["cu_seqlens"]
+    g_out = torch.empty_like(la)
+    stage_report_cum = round(timed(lambda i: gdr.cumdecay(la, cu0, out=g_out, d_k=ps.dk,
+                                                          scalar_decay=ps.w.scalar_decay),
+                                   50, stream), 4)
+
+    # ---- the prefill stages alone -> dominant kernel roofline -------------------
+    names = list(STAGES)
     st_ms = stage_times(ps, max(20, min(args.steps, 200)), stream)
-    dom = max(range(3), key=lambda s: st_ms[s])
+    dom = max(range(len(names)), key=lambda s: st_ms[s])
     roof = roofline_obj(ps.bytes, ps.flops, st_ms[dom], pk,
                         recorded_traffic(names[dom], ps.w.name))
     roof["kernel"] = names[dom]
     roof["kernel_ms"] = round(st_ms[dom], 4)
-    stage_report = {names[s]: round(st_ms[s], 4) for s in range(3)}
+    stage_report = {names[s]: round(st_ms[s], 4) for s in range(len(names))}
+    stage_report["cumdecay_standalone"] = stage_report_cum
     path_roof = roofline_obj(ps.bytes, ps.flops, ms_step, pk)
 
     extra = {}
@@ -383,7 +407,7 @@ def run_gdr(args):
         "kernel_ms": stage_report,
         "decode": decode,
         "e2e": e2e,
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
         "cpu_baseline": cpu,
         "extra": extra,
@@ -402,7 +426,7 @@ def bench_prefill_workload(gdr, w, stream, pk, rank, args):
     ms = timed(lambda i: ps.step(i), n, stream)
     st = stage_times(ps, n, stream)
     res = {"tokens_per_s": round(ps.T / (ms * 1e-3), 1), "ms_per_step": round(ms, 4),
-           "kernel_ms": {k: round(v, 4) for k, v in zip(("cumdecay", "intra_chunk", "state_pass"), st)},
+           "kernel_ms": {k: round(v, 4) for k, v in zip(STAGES, st)},
            "path_roofline": roofline_obj(ps.bytes, ps.flops, ms, pk), "tokens": ps.T,
            "sequences": ps.n, "inputs_exceed_l2": ps.footprint > L2_BYTES}
     del ps
@@ -485,6 +509,10 @@ def main():
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     p.add_argument("--only-decode", action="store_true",
                    help="run only the decode measurement (for profiling)")
+    p.add_argument("--workload", default=wl.GRAFT_LAYER.name, choices=sorted(wl.PREFILL_WORKLOADS),
+                   help="prefill workload of the main line (default: the graft layer)")
+    p.add_argument("--sets", type=int, default=0,
+                   help="rotating input sets of the main line (default 4; 1 for varlen)")
     args = p.parse_args()
     if args.warmup < 3:
         p.error("--warmup must be >= 3")

@@ -19,7 +19,7 @@ import threading
 
 import torch
 
-__all__ = ["PrefillArgs", "PreparedPrefill", "prefill", "decode_step", "cumdecay", "chunk_factors", "workspace_size",
+__all__ = ["PrefillArgs", "PreparedPrefill", "prefill", "kernel_count", "decode_step", "cumdecay", "chunk_factors", "workspace_size",
            "snapshot_count", "prefill_status", "lib", "GdrError", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_build", "libgdr.so")
@@ -70,6 +70,8 @@ def lib():
             L.gdr_version.restype = i
             L.gdr_prefill_workspace_size.restype = ctypes.c_size_t
             L.gdr_prefill_workspace_size.argtypes = [i, i, i, i, i64, i]
+            L.gdr_prefill_kernel_count.restype = i
+            L.gdr_prefill_kernel_count.argtypes = [i, i, i, i, i64, i]
             L.gdr_snapshot_count.restype = i64
             L.gdr_snapshot_count.argtypes = [vp, i, i]
             L.gdr_prefill.restype = i
@@ -129,6 +131,12 @@ def workspace_size(n_seqs, n_heads, d_k, d_v, total_tokens, scalar_decay=False) 
                                                 int(bool(scalar_decay))))
 
 
+def kernel_count(n_seqs, n_heads, d_k, d_v, total_tokens, scalar_decay=False) -> int:
+    """Kernel launches one gdr_prefill enqueues for these sizes."""
+    return int(lib().gdr_prefill_kernel_count(n_seqs, n_heads, d_k, d_v, total_tokens,
+                                              int(bool(scalar_decay))))
+
+
 def snapshot_count(cu_seqlens_host, snap_interval: int) -> int:
     cu = torch.as_tensor(cu_seqlens_host, dtype=torch.int32).contiguous()
     n = int(lib().gdr_snapshot_count(ctypes.c_void_p(cu.data_ptr()), cu.numel() - 1,
@@ -165,14 +173,15 @@ def _prefill_args(q, k, v, beta, log_a, cu_seqlens, scalar_decay, scale, init_st
 
 def prefill(q, k, v, beta, log_a, cu_seqlens, *, scalar_decay=False, scale=1.0,
             init_state=None, snap_interval=0, cu_seqlens_host=None, out=None,
-            final_state=None, snapshots=None, workspace=None, stages=(0, 2)):
+            final_state=None, snapshots=None, workspace=None, stages=(0, 1)):
     """Chunked prefill over a packed batch.  Returns (o, final_state, snapshots).
 
     ``cu_seqlens`` is a device int32 tensor [N+1]; its host copy (taken from
     ``cu_seqlens_host`` when given, else read back) sizes the snapshots.
     Output buffers and the workspace may be passed in to avoid allocation.
-    ``stages`` = (first, last) runs only that range of the three kernels
-    (0 cumulative decay, 1 intra-chunk, 2 state pass), for timing them apart.
+    ``stages`` = (first, last) runs only that range of the two stages
+    (0 intra-chunk factors with the cumulative decay, 1 state pass), for
+    timing them apart.
     """
     if q.dtype != k.dtype or q.dtype != v.dtype:
         raise TypeError("q, k and v must share a dtype")
@@ -201,7 +210,7 @@ def prefill(q, k, v, beta, log_a, cu_seqlens, *, scalar_decay=False, scale=1.0,
     a = _prefill_args(q, k, v, beta, log_a, cu_seqlens, scalar_decay, scale, init_state,
                       snap_interval, out, final_state, snap_arg, workspace)
     first, last = stages
-    if (first, last) == (0, 2):
+    if (first, last) == (0, 1):
         _check(lib().gdr_prefill(ctypes.byref(a), _stream(dev)), "gdr_prefill")
     else:
         _check(lib().gdr_prefill_stages(ctypes.byref(a), int(first), int(last), _stream(dev)),
@@ -230,9 +239,9 @@ class PreparedPrefill:
         self.out, self.final_state, self.snapshots, self.workspace = out, final_state, snapshots, workspace
         lib()
 
-    def run(self, stages=(0, 2), stream=None):
+    def run(self, stages=(0, 1), stream=None):
         st = ctypes.c_void_p(stream.cuda_stream) if stream is not None else _stream(self.device)
-        if tuple(stages) == (0, 2):
+        if tuple(stages) == (0, 1):
             _check(_LIB.gdr_prefill(ctypes.byref(self.args), st), "gdr_prefill")
         else:
             _check(_LIB.gdr_prefill_stages(ctypes.byref(self.args), int(stages[0]), int(stages[1]), st),

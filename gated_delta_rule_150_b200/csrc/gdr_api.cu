@@ -74,6 +74,15 @@ size_t gdr_prefill_workspace_size(int n_seqs, int n_heads, int d_k, int d_v,
     return gdr::workspace_layout(n_seqs, n_heads, d_k, total_tokens, scalar_decay).total;
 }
 
+int gdr_prefill_kernel_count(int n_seqs, int n_heads, int d_k, int d_v, int64_t total_tokens,
+                             int scalar_decay) {
+    if (gdr_prefill_workspace_size(n_seqs, n_heads, d_k, d_v, total_tokens, scalar_decay) == 0)
+        return 0;
+    if (n_seqs == 0) return 0;
+    const int intra = total_tokens > 0 ? 1 : 0;
+    return intra + (gdr::segment_chunks(n_seqs, n_heads, total_tokens, d_k) > 0 ? 3 : 1);
+}
+
 int64_t gdr_snapshot_count(const int32_t* host_cu, int n_seqs, int snap_interval) {
     if (!host_cu || n_seqs < 0 || snap_interval < 0) return -1;
     if (snap_interval == 0) return 0;
@@ -87,7 +96,7 @@ int64_t gdr_snapshot_count(const int32_t* host_cu, int n_seqs, int snap_interval
 }
 
 gdr_status gdr_prefill_stages(const gdr_prefill_args* a, int first, int last, void* stream) {
-    if (first < 0 || last > 2 || first > last) return GDR_ERR_INVALID_ARG;
+    if (first < 0 || last > 1 || first > last) return GDR_ERR_INVALID_ARG;
     gdr_status s = check_prefill_inputs(a);
     if (s != GDR_OK) return s;
     if (!a->final_state || !aligned16(a->final_state)) return GDR_ERR_INVALID_ARG;
@@ -102,27 +111,19 @@ gdr_status gdr_prefill_stages(const gdr_prefill_args* a, int first, int last, vo
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint8_t* ws = static_cast<uint8_t*>(a->workspace);
     uint32_t* err = reinterpret_cast<uint32_t*>(ws + lay.err_off);
-    float* g = reinterpret_cast<float*>(ws + lay.g_off);
     uint8_t* rec = ws + lay.rec_off;
     if (first == 0 && cudaMemsetAsync(err, 0, sizeof(uint32_t), st) != cudaSuccess)
         return GDR_ERR_CUDA;
-    if (a->total_tokens > 0) {
-        if (first <= 0 && last >= 0) {
-            s = from_cuda(gdr::launch_cumdecay(a->n_seqs, a->n_heads, a->d_k, a->total_tokens,
-                                               a->cu_seqlens, a->log_a, a->scalar_decay, g, st));
-            if (s != GDR_OK) return s;
-        }
-        if (first <= 1 && last >= 1) {
-            s = from_cuda(gdr::launch_intra_chunk(*a, g, rec, err, st));
-            if (s != GDR_OK) return s;
-        }
+    if (first == 0 && a->total_tokens > 0) {
+        s = from_cuda(gdr::launch_intra_chunk(*a, rec, err, st));
+        if (s != GDR_OK) return s;
     }
-    if (last >= 2) return from_cuda(gdr::launch_state_pass(*a, rec, lay, ws, err, st));
+    if (last >= 1) return from_cuda(gdr::launch_state_pass(*a, rec, lay, ws, err, st));
     return GDR_OK;
 }
 
 gdr_status gdr_prefill(const gdr_prefill_args* a, void* stream) {
-    return gdr_prefill_stages(a, 0, 2, stream);
+    return gdr_prefill_stages(a, 0, 1, stream);
 }
 
 gdr_status gdr_prefill_status(const void* workspace, void* stream) {
@@ -162,13 +163,9 @@ gdr_status gdr_chunk_factors(const gdr_prefill_args* a, float* Qt, float* PU, fl
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint8_t* ws = static_cast<uint8_t*>(a->workspace);
     uint32_t* err = reinterpret_cast<uint32_t*>(ws + lay.err_off);
-    float* g = reinterpret_cast<float*>(ws + lay.g_off);
     uint8_t* rec = ws + lay.rec_off;
     if (cudaMemsetAsync(err, 0, sizeof(uint32_t), st) != cudaSuccess) return GDR_ERR_CUDA;
-    s = from_cuda(gdr::launch_cumdecay(a->n_seqs, a->n_heads, a->d_k, a->total_tokens,
-                                       a->cu_seqlens, a->log_a, a->scalar_decay, g, st));
-    if (s != GDR_OK) return s;
-    s = from_cuda(gdr::launch_intra_chunk(*a, g, rec, err, st));
+    s = from_cuda(gdr::launch_intra_chunk(*a, rec, err, st));
     if (s != GDR_OK) return s;
     return from_cuda(gdr::launch_unpack_records(*a, rec, Qt, PU, BS, NC, gamma, st));
 }

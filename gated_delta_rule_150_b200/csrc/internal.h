@@ -52,9 +52,12 @@ __host__ __device__ constexpr RecordLayout record_layout(int D) {
 // S_end = S_start M + N), a short fp32 chain combines the maps into each
 // segment's true start state, and every segment then replays its chunks from
 // that state to produce its outputs.  seg_chunks == 0 means one pass.
-inline int segment_chunks(int n_seqs, int H, int64_t T) {
+inline int segment_chunks(int n_seqs, int H, int64_t T, int D) {
     if (n_seqs <= 0 || T <= 0) return 0;
     const int64_t pairs = (int64_t)n_seqs * H;
+    // about two CTAs per SM (the state-pass kernels fit two per SM at d = 64;
+    // at d = 128 two waves of shorter segments beat one wave of longer ones)
+    (void)D;
     const int64_t target_ctas = 2 * 148;
     int64_t segs = (target_ctas + pairs - 1) / pairs;
     if (segs > 32) segs = 32;
@@ -73,7 +76,6 @@ inline int64_t n_segment_slots(int64_t total_tokens, int n_seqs, int seg_chunks)
 
 struct WorkspaceLayout {
     size_t err_off;     // uint32 error word (0 = ok)
-    size_t g_off;       // fp32 cumulative log decay, same layout as log_a
     size_t rec_off;     // chunk-head records
     size_t seg_off;     // per (segment slot, head): N, M, E, each [D x D] fp32
     int64_t n_slots;
@@ -87,14 +89,13 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 inline WorkspaceLayout workspace_layout(int n_seqs, int H, int D, int64_t T, int scalar) {
     WorkspaceLayout w{};
+    (void)scalar;
     w.err_off = 0;
-    w.g_off = 1024;
-    const size_t g_elems = (size_t)T * (size_t)H * (scalar ? 1 : (size_t)D);
-    w.rec_off = align_up(w.g_off + g_elems * sizeof(float), 1024);
+    w.rec_off = 1024;
     w.n_slots = n_chunk_slots(T, n_seqs);
     w.rec_bytes = record_layout(D).bytes;
     w.seg_off = align_up(w.rec_off + (size_t)w.n_slots * (size_t)H * w.rec_bytes, 1024);
-    w.seg_chunks = segment_chunks(n_seqs, H, T);
+    w.seg_chunks = segment_chunks(n_seqs, H, T, D);
     w.n_seg_slots = n_segment_slots(T, n_seqs, w.seg_chunks);
     w.total = w.seg_off + (size_t)w.n_seg_slots * (size_t)H * 3u * (size_t)D * D * sizeof(float);
     return w;
@@ -104,8 +105,8 @@ inline WorkspaceLayout workspace_layout(int n_seqs, int H, int D, int64_t T, int
 cudaError_t launch_cumdecay(int n_seqs, int H, int D, int64_t T, const int32_t* cu,
                             const float* log_a, int scalar, float* g, cudaStream_t st);
 
-cudaError_t launch_intra_chunk(const gdr_prefill_args& a, const float* g, uint8_t* records,
-                               uint32_t* err, cudaStream_t st);
+cudaError_t launch_intra_chunk(const gdr_prefill_args& a, uint8_t* records, uint32_t* err,
+                               cudaStream_t st);
 
 cudaError_t launch_state_pass(const gdr_prefill_args& a, const uint8_t* records,
                               const WorkspaceLayout& lay, uint8_t* ws, uint32_t* err,

@@ -45,7 +45,7 @@
 namespace gdr {
 namespace {
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
 constexpr float kMaxFactorExp = 80.f;
 constexpr int kLd = 68;                       // row stride (floats) of the fp32 64x64 tiles
 
@@ -82,7 +82,8 @@ struct IntraLayout {
     static constexpr uint32_t Gl = Qgs + 128u * D;            // fp32 [D] g_last
     static constexpr uint32_t Bs = Gl + 4u * D;               // fp32 [64] beta
     static constexpr uint32_t Gs = Bs + 256u;                 // fp32 [64] g (scalar decay)
-    static constexpr uint32_t bytes = Gs + 256u;
+    static constexpr uint32_t Ptot = Gs + 256u;               // fp32 scan partials [1024 B]
+    static constexpr uint32_t bytes = Ptot + 1024u;
     static constexpr uint32_t dyn_bytes = bytes + 1024u;
     __host__ __device__ static constexpr uint32_t kt_off(int b) {
         return KT0 + 32u * D * (uint32_t)(b * (b + 1) / 2);
@@ -190,16 +191,16 @@ __device__ __forceinline__ void load_ap_row(uint32_t taddr, int b, float (&v)[64
 }
 
 template <int D, typename InT, bool SCALAR>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, (D == 64) ? 2 : 1)
 intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                    const InT* __restrict__ q, const InT* __restrict__ k, const InT* __restrict__ v,
-                   const float* __restrict__ beta, const float* __restrict__ g, float scale,
+                   const float* __restrict__ beta, const float* __restrict__ log_a, float scale,
                    uint8_t* __restrict__ records, uint32_t* err) {
     using L = IntraLayout<D, InT, SCALAR>;
     constexpr RecordLayout R = record_layout(D);
     constexpr int CG = D / 8;              // channel groups of 8
     constexpr int RG = kThreads / CG;      // row groups
-    constexpr int RPT = 64 / RG;           // rows per thread: 4 (D=64) or 8 (D=128)
+    constexpr int RPT = 64 / RG;           // rows per thread: 2 (D=64) or 4 (D=128)
     constexpr uint32_t kTmemCols = (D == 64) ? 256u : 512u;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -221,7 +222,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     float* Gl = reinterpret_cast<float*>(sm + L::Gl);
     float* Bs = reinterpret_cast<float*>(sm + L::Bs);
     float* Gs = reinterpret_cast<float*>(sm + L::Gs);
-    const float* sG = reinterpret_cast<const float*>(sm + L::sG);
+    float* sG = reinterpret_cast<float*>(sm + L::sG);
 
     if (tid == 0) {
         mbar_init(&mma_bar, 1);
@@ -235,15 +236,48 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         stage_rows<InT, D>(sm + L::sK, k + base, tok_stride, len, tid);
         stage_rows<InT, D>(sm + L::sV, v + base, tok_stride, len, tid);
     }
-    if (!SCALAR) stage_rows<float, D>(sm + L::sG, g + base, tok_stride, len, tid);
+    if (!SCALAR) stage_rows<float, D>(sm + L::sG, log_a + base, tok_stride, len, tid);
     if (tid < 64) {
         Bs[tid] = tid < len ? __ldg(beta + (size_t)(start + tid) * H + h) : 0.f;
-        if (SCALAR) {
-            const float glast = __ldg(g + (size_t)(start + len - 1) * H + h);
-            Gs[tid] = tid < len ? __ldg(g + (size_t)(start + tid) * H + h) : glast;
-        }
+        if (SCALAR) Gs[tid] = tid < len ? __ldg(log_a + (size_t)(start + tid) * H + h) : 0.f;
     }
     cp_async_wait_all();
+    __syncthreads();
+
+    // ---- chunk-local cumulative log decay, g[r] = sum_{i <= r} log a_i -------
+    // (the same quantity gdr_cumdecay computes; padded rows add 0, so past the
+    // chunk end g stays at g_last)
+    if (!SCALAR) {
+        constexpr int P = kThreads / D, RP = 64 / P;          // row parts per channel
+        float* Ptot = reinterpret_cast<float*>(sm + L::Ptot);
+        const int c = tid % D, part = tid / D;
+        float run = 0.f;
+#pragma unroll 4
+        for (int r = part * RP; r < (part + 1) * RP; ++r) {
+            run += sG[r * D + c];
+            sG[r * D + c] = run;
+        }
+        Ptot[part * D + c] = run;
+        __syncthreads();
+        if (part > 0) {
+            float off = 0.f;
+            for (int p2 = 0; p2 < part; ++p2) off += Ptot[p2 * D + c];
+#pragma unroll 4
+            for (int r = part * RP; r < (part + 1) * RP; ++r) sG[r * D + c] += off;
+        }
+    } else if (warp == 0) {
+        const float x0 = Gs[2 * lane], x1 = Gs[2 * lane + 1];
+        const float pair = x0 + x1;
+        float incl = pair;
+#pragma unroll
+        for (int m = 1; m < 32; m <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, incl, m);
+            if (lane >= m) incl += y;
+        }
+        const float excl = incl - pair;
+        Gs[2 * lane] = excl + x0;
+        Gs[2 * lane + 1] = excl + pair;
+    }
     __syncthreads();
 
     const int cg = tid % CG, rg = tid / CG, c0 = 8 * cg;
@@ -390,14 +424,14 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         const uint32_t o1 = sw128_chunk(2 * D, c, r0 / 8) + (r0 % 8) * 2;
         const uint32_t o2 = sw128_chunk(2 * D, D + c, r0 / 8) + (r0 % 8) * 2;
         const uint32_t o3 = sw128_chunk(D, c, r0 / 8) + (r0 % 8) * 2;
-        if (RPT == 8) {
-            *reinterpret_cast<uint4*>(Bt + o1) = make_uint4(pb1[e][0], pb1[e][1], pb1[e][2 % (RPT / 2)], pb1[e][3 % (RPT / 2)]);
-            *reinterpret_cast<uint4*>(Bt + o2) = make_uint4(pb2[e][0], pb2[e][1], pb2[e][2 % (RPT / 2)], pb2[e][3 % (RPT / 2)]);
-            *reinterpret_cast<uint4*>(Kdt + o3) = make_uint4(pkd[e][0], pkd[e][1], pkd[e][2 % (RPT / 2)], pkd[e][3 % (RPT / 2)]);
+        if constexpr (RPT == 4) {
+            *reinterpret_cast<uint2*>(Bt + o1) = make_uint2(pb1[e][0], pb1[e][RPT / 2 - 1]);
+            *reinterpret_cast<uint2*>(Bt + o2) = make_uint2(pb2[e][0], pb2[e][RPT / 2 - 1]);
+            *reinterpret_cast<uint2*>(Kdt + o3) = make_uint2(pkd[e][0], pkd[e][RPT / 2 - 1]);
         } else {
-            *reinterpret_cast<uint2*>(Bt + o1) = make_uint2(pb1[e][0], pb1[e][1 % (RPT / 2)]);
-            *reinterpret_cast<uint2*>(Bt + o2) = make_uint2(pb2[e][0], pb2[e][1 % (RPT / 2)]);
-            *reinterpret_cast<uint2*>(Kdt + o3) = make_uint2(pkd[e][0], pkd[e][1 % (RPT / 2)]);
+            *reinterpret_cast<uint32_t*>(Bt + o1) = pb1[e][0];
+            *reinterpret_cast<uint32_t*>(Bt + o2) = pb2[e][0];
+            *reinterpret_cast<uint32_t*>(Kdt + o3) = pkd[e][0];
         }
     }
     fence_proxy_async_smem();
@@ -405,7 +439,8 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = tmem_slot;
-    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+    const int whalf = warp >> 2;                              // warps w and w+4 share TMEM lanes
 
     // ---- decay-weighted Q K^T and K K^T on the tensor cores ------------------
     if (tid == 0) {
@@ -432,7 +467,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     tc_fence_after_sync();
 
     // ---- P (masked, bf16 operand) and A (masked, times beta, fp32) ----------
-    {
+    if (warp < 4) {
         const bool is_p = warp < 2;
         const int rr = 32 * (warp & 1) + lane;                // chunk row
         const int lim = is_p ? rr : rr - 1;                   // last valid key index
@@ -458,7 +493,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                         const size_t tr = base + (size_t)rr * tok_stride + c;
                         const size_t ti = base + (size_t)i * tok_stride + c;
                         const float xr = is_p ? scale * (float)q[tr] : (float)k[tr];
-                        acc += xr * (float)k[ti] * expf(g[tr] - g[ti]);
+                        acc += xr * (float)k[ti] * expf(sG[rr * D + c] - sG[i * D + c]);
                     }
                 }
                 vrow[i] = acc;
@@ -532,18 +567,22 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     // bottom-left 32 x 32 block, blocks (b, j) with b in {2, 3}, j in {0, 1}:
     //   Y_bj = sum_{l=j}^{1} A_bl T_lj        T_bj = -sum_{l=2}^{b} T_bl Y_lj
     {
-        const int q = tid >> 5, b = 2 + (q >> 1), j = q & 1;
-        float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int l = j; l <= 1; ++l)
-            tile16<kLd>(As, 16 * b + rr0, 16 * l, Ts, 16 * l, 16 * j + c4, y0, y1);
-        *reinterpret_cast<float4*>(Yt + (16 * (b - 2) + rr0) * 32 + 16 * j + c4) = make_float4(y0[0], y0[1], y0[2], y0[3]);
-        *reinterpret_cast<float4*>(Yt + (16 * (b - 2) + rr0 + 1) * 32 + 16 * j + c4) = make_float4(y1[0], y1[1], y1[2], y1[3]);
+        const int q = (tid >> 5) & 3, b = 2 + (q >> 1), j = q & 1;
+        if (tid < 128) {
+            float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int l = j; l <= 1; ++l)
+                tile16<kLd>(As, 16 * b + rr0, 16 * l, Ts, 16 * l, 16 * j + c4, y0, y1);
+            *reinterpret_cast<float4*>(Yt + (16 * (b - 2) + rr0) * 32 + 16 * j + c4) = make_float4(y0[0], y0[1], y0[2], y0[3]);
+            *reinterpret_cast<float4*>(Yt + (16 * (b - 2) + rr0 + 1) * 32 + 16 * j + c4) = make_float4(y1[0], y1[1], y1[2], y1[3]);
+        }
         __syncthreads();
-        float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int l = 2; l <= b; ++l)
-            tile16<32>(Ts, 16 * b + rr0, 16 * l, Yt, 16 * (l - 2), 16 * j + c4, z0, z1);
-        *reinterpret_cast<float4*>(Ts + (16 * b + rr0) * kLd + 16 * j + c4) = make_float4(-z0[0], -z0[1], -z0[2], -z0[3]);
-        *reinterpret_cast<float4*>(Ts + (16 * b + rr0 + 1) * kLd + 16 * j + c4) = make_float4(-z1[0], -z1[1], -z1[2], -z1[3]);
+        if (tid < 128) {
+            float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int l = 2; l <= b; ++l)
+                tile16<32>(Ts, 16 * b + rr0, 16 * l, Yt, 16 * (l - 2), 16 * j + c4, z0, z1);
+            *reinterpret_cast<float4*>(Ts + (16 * b + rr0) * kLd + 16 * j + c4) = make_float4(-z0[0], -z0[1], -z0[2], -z0[3]);
+            *reinterpret_cast<float4*>(Ts + (16 * b + rr0 + 1) * kLd + 16 * j + c4) = make_float4(-z1[0], -z1[1], -z1[2], -z1[3]);
+        }
     }
     __syncthreads();
     // T -> bf16 operand tile [64 r][64 i] (zero above the diagonal)
@@ -578,12 +617,14 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     // W^T rows c and U^T rows v -> one bf16 tile [2D][64] (row D + v for U^T)
     {
         uint8_t* WUt = sm + L::WUt;
-        const int lrow = 32 * warp + lane;
+        const int lrow = 32 * (warp & 3) + lane;
 #pragma unroll
         for (int part = 0; part < 2 * D / 128; ++part) {
+            if (D == 128 && part != whalf) continue;
             const int row = (D == 64) ? lrow : (lrow + 128 * part);
 #pragma unroll
             for (int piece = 0; piece < 2; ++piece) {
+                if (D == 64 && piece != whalf) continue;
                 float x[32];
                 tmem_ld32(tmem + lane_base + 64 * part + 32 * piece, x);
                 tmem_ld_wait();
@@ -625,10 +666,11 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     static_assert(R.bytes <= L::Qgs, "record staging fits below Qgs");
     {
         // rows of the M = 64 products live in lanes 16 w + l (l < 16)
-        const int r64 = 16 * warp + lane;
+        const int r64 = 16 * (warp & 3) + lane;
         const bool act64 = lane < 16;
 #pragma unroll
         for (int piece = 0; piece < D / 32; ++piece) {
+            if ((piece & 1) != whalf) continue;
             float pw[32], pu[32];
             tmem_ld32(tmem + lane_base + 32 * piece, pw);
             tmem_ld32(tmem + lane_base + D + 32 * piece, pu);
@@ -647,10 +689,11 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                 }
             }
         }
-        const int rD = (D == 128) ? (32 * warp + lane) : r64;
+        const int rD = (D == 128) ? (32 * (warp & 3) + lane) : r64;
         const bool actD = (D == 128) || act64;
 #pragma unroll
         for (int piece = 0; piece < D / 32; ++piece) {
+            if ((piece & 1) != whalf) continue;
             float bs[32], nc[32];
             tmem_ld32(tmem + lane_base + 2 * D + 32 * piece, bs);
             tmem_ld32(tmem + lane_base + 3 * D + 32 * piece, nc);
@@ -710,36 +753,36 @@ __global__ void unpack_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
 }
 
 template <int D, typename InT, bool SCALAR>
-cudaError_t launch_typed(const gdr_prefill_args& a, const float* g, uint8_t* records,
-                         uint32_t* err, cudaStream_t st) {
+cudaError_t launch_typed(const gdr_prefill_args& a, uint8_t* records, uint32_t* err,
+                         cudaStream_t st) {
     auto kern = intra_chunk_kernel<D, InT, SCALAR>;
     const uint32_t smem = IntraLayout<D, InT, SCALAR>::dyn_bytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)n_chunk_slots(a.total_tokens, a.n_seqs), (unsigned)a.n_heads);
     kern<<<grid, kThreads, smem, st>>>(a.cu_seqlens, a.n_seqs, a.n_heads, (const InT*)a.q,
-                                       (const InT*)a.k, (const InT*)a.v, a.beta, g, a.scale,
+                                       (const InT*)a.k, (const InT*)a.v, a.beta, a.log_a, a.scale,
                                        records, err);
     return cudaGetLastError();
 }
 
 template <int D, typename InT>
-cudaError_t launch_decay(const gdr_prefill_args& a, const float* g, uint8_t* records,
-                         uint32_t* err, cudaStream_t st) {
-    return a.scalar_decay ? launch_typed<D, InT, true>(a, g, records, err, st)
-                          : launch_typed<D, InT, false>(a, g, records, err, st);
+cudaError_t launch_decay(const gdr_prefill_args& a, uint8_t* records, uint32_t* err,
+                         cudaStream_t st) {
+    return a.scalar_decay ? launch_typed<D, InT, true>(a, records, err, st)
+                          : launch_typed<D, InT, false>(a, records, err, st);
 }
 
 }  // namespace
 
-cudaError_t launch_intra_chunk(const gdr_prefill_args& a, const float* g, uint8_t* records,
-                               uint32_t* err, cudaStream_t st) {
+cudaError_t launch_intra_chunk(const gdr_prefill_args& a, uint8_t* records, uint32_t* err,
+                               cudaStream_t st) {
     if (n_chunk_slots(a.total_tokens, a.n_seqs) == 0) return cudaSuccess;
     if (a.d_k == 64)
-        return a.qkv_dtype == GDR_BF16 ? launch_decay<64, __nv_bfloat16>(a, g, records, err, st)
-                                       : launch_decay<64, float>(a, g, records, err, st);
-    return a.qkv_dtype == GDR_BF16 ? launch_decay<128, __nv_bfloat16>(a, g, records, err, st)
-                                   : launch_decay<128, float>(a, g, records, err, st);
+        return a.qkv_dtype == GDR_BF16 ? launch_decay<64, __nv_bfloat16>(a, records, err, st)
+                                       : launch_decay<64, float>(a, records, err, st);
+    return a.qkv_dtype == GDR_BF16 ? launch_decay<128, __nv_bfloat16>(a, records, err, st)
+                                   : launch_decay<128, float>(a, records, err, st);
 }
 
 cudaError_t launch_unpack_records(const gdr_prefill_args& a, const uint8_t* records, float* Qt,

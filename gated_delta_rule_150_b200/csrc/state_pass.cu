@@ -73,7 +73,7 @@ struct PassLayout {
 };
 
 template <int D, typename OutT, int MODE>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, (D == 64) ? 2 : 1)
 state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                   const uint8_t* __restrict__ records, const float* init_state,
                   OutT* __restrict__ o, float* final_state, int snap_interval,
@@ -415,11 +415,13 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
 // initial state.
 constexpr int kCombineRows = 8;
 
+constexpr int kCombineBufs = 3;
+
 template <int D>
 struct CombineLayout {
-    static constexpr uint32_t M0 = 0;                                   // 2 x [D x D] fp32
-    static constexpr uint32_t N0 = 2u * D * D * 4u;                     // 2 x [rows x D] fp32
-    static constexpr uint32_t E = N0 + 2u * kCombineRows * D * 4u;      // [rows x D] fp32
+    static constexpr uint32_t M0 = 0;                                   // bufs x [D x D] fp32
+    static constexpr uint32_t N0 = kCombineBufs * D * D * 4u;           // bufs x [rows x D] fp32
+    static constexpr uint32_t E = N0 + kCombineBufs * kCombineRows * D * 4u;   // [rows x D] fp32
     static constexpr uint32_t bytes = E + kCombineRows * D * 4u;
     static constexpr uint32_t dyn_bytes = bytes + 128u;
 };
@@ -434,7 +436,8 @@ combine_kernel(const int32_t* __restrict__ cu, int H, int seg_chunks, const floa
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
                                              ~static_cast<uintptr_t>(127));
-    __shared__ uint64_t full[2];
+    constexpr int NB = kCombineBufs;
+    __shared__ uint64_t full[NB];
     const int pair = blockIdx.x, rb = blockIdx.y;
     const int n = pair / H, h = pair % H;
     const int tid = threadIdx.x, j = tid / QD, q = tid % QD;
@@ -454,14 +457,14 @@ combine_kernel(const int32_t* __restrict__ cu, int H, int seg_chunks, const floa
     float* e = reinterpret_cast<float*>(sm + L::E);
     auto seg_ptr = [&](int s) { return seg_ws + ((size_t)(slot0 + s) * H + h) * 3u * D * D; };
     auto issue = [&](int s) {      // thread 0: M_s and this CTA's rows of N_s
-        const int b = s & 1;
+        const int b = s % NB;
         mbar_arrive_expect_tx(&full[b], (uint32_t)(D * D * 4 + RB * D * 4));
         bulk_g2s(sm + L::M0 + b * D * D * 4u, seg_ptr(s) + (size_t)D * D, D * D * 4u, &full[b]);
         bulk_g2s(sm + L::N0 + b * RB * D * 4u, seg_ptr(s) + (size_t)rb * RB * D, RB * D * 4u, &full[b]);
     };
     if (tid == 0) {
-        mbar_init(&full[0], 1);
-        mbar_init(&full[1], 1);
+#pragma unroll
+        for (int b = 0; b < NB; ++b) mbar_init(&full[b], 1);
         fence_mbar_init();
     }
     {
@@ -472,14 +475,13 @@ combine_kernel(const int32_t* __restrict__ cu, int H, int seg_chunks, const floa
     __syncthreads();
     int issued = 0, consumed = 0;                  // thread 0's bookkeeping (steps)
     if (tid == 0) {
-        issue(0);
-        issued = 1;
-        if (nseg > 2) { issue(1); issued = 2; }
+        for (int s = 0; s < NB && s <= nseg - 2; ++s) issue(s);
+        issued = min(NB, nseg - 1);
     }
     bool failed = false;
     for (int s = 0; s + 1 < nseg; ++s) {
-        const int b = s & 1;
-        if (!mbar_wait(&full[b], (uint32_t)(s >> 1) & 1)) failed = true;
+        const int b = s % NB;
+        if (!mbar_wait(&full[b], (uint32_t)(s / NB) & 1)) failed = true;
         consumed = s + 1;
         const float* Mm = reinterpret_cast<const float*>(sm + L::M0 + b * D * D * 4u);
         const float* Nm = reinterpret_cast<const float*>(sm + L::N0 + b * RB * D * 4u);
@@ -496,13 +498,13 @@ combine_kernel(const int32_t* __restrict__ cu, int H, int seg_chunks, const floa
         if (__syncthreads_or(failed)) break;          // everyone is done with e and buffer b
         *reinterpret_cast<float4*>(e + j * D + 4 * q) = acc;
         *reinterpret_cast<float4*>(seg_ptr(s + 1) + 2u * D * D + row_off) = acc;
-        if (tid == 0 && s + 2 <= nseg - 2) { issue(s + 2); issued = s + 3; }
+        if (tid == 0 && s + NB <= nseg - 2) { issue(s + NB); issued = s + NB + 1; }
         __syncthreads();
     }
     if (failed && tid == 0) {
         atomicOr(err, 1u);
         // let the copies already issued land before the CTA exits (bounded waits)
-        for (int c = consumed; c < issued; ++c) mbar_wait(&full[c & 1], (uint32_t)(c >> 1) & 1);
+        for (int c = consumed; c < issued; ++c) mbar_wait(&full[c % NB], (uint32_t)(c / NB) & 1);
     }
 }
 

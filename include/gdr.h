@@ -113,6 +113,15 @@ typedef struct {
 size_t gdr_prefill_workspace_size(int n_seqs, int n_heads, int d_k, int d_v,
                                   int64_t total_tokens, int scalar_decay);
 
+/*
+ * Number of kernel launches gdr_prefill enqueues for these sizes (0 on bad
+ * sizes): the intra-chunk kernel plus one state pass, or three (zero-state
+ * pass, chaining of segment maps, replay) when long sequences with few
+ * (sequence, head) pairs are cut into segments.
+ */
+int gdr_prefill_kernel_count(int n_seqs, int n_heads, int d_k, int d_v, int64_t total_tokens,
+                             int scalar_decay);
+
 /* Number of snapshot slots for host-side cu_seqlens [N+1] (-1 on bad input). */
 int64_t gdr_snapshot_count(const int32_t* host_cu_seqlens, int n_seqs, int snap_interval);
 
@@ -125,9 +134,10 @@ int64_t gdr_snapshot_count(const int32_t* host_cu_seqlens, int n_seqs, int snap_
 gdr_status gdr_prefill(const gdr_prefill_args* args, void* stream);
 
 /*
- * Enqueue only stages first..last (inclusive) of a prefill: 0 = chunk-local
- * cumulative decay, 1 = intra-chunk factors, 2 = sequential inter-chunk pass.
- * gdr_prefill(a) is gdr_prefill_stages(a, 0, 2).  A later stage reads what the
+ * Enqueue only stages first..last (inclusive) of a prefill: 0 = intra-chunk
+ * factors (the chunk-local cumulative decay of gdr_cumdecay is computed inside
+ * this stage, so g never goes through memory), 1 = sequential inter-chunk
+ * pass.  gdr_prefill(a) is gdr_prefill_stages(a, 0, 1).  A later stage reads what the
  * earlier stages left in the workspace, so a range starting after 0 must
  * follow a call that ran the stages before it with the same arguments.  Used
  * to time the kernels one by one.  Errors as for gdr_prefill, plus
@@ -166,9 +176,9 @@ gdr_status gdr_prefill_static_workspace(const gdr_prefill_args* args, void* stre
 gdr_status gdr_prefill_status(const void* workspace, void* stream);
 
 /*
- * The chunk-local cumulative log decay on its own (the first kernel of the
- * prefill): g[t] = sum of log_a over the tokens of t's chunk up to and
- * including t, chunks as in gdr_prefill.  log_a and g share the layout
+ * The chunk-local cumulative log decay on its own: g[t] = sum of log_a over
+ * the tokens of t's chunk up to and including t, chunks as in gdr_prefill.
+ * (gdr_prefill computes the same sums inside its intra-chunk stage.)  log_a and g share the layout
  * [T_tot, H, d_k] (or [T_tot, H] when scalar_decay != 0), fp32, device.
  */
 gdr_status gdr_cumdecay(int n_seqs, int n_heads, int d_k, int64_t total_tokens,
@@ -176,8 +186,8 @@ gdr_status gdr_cumdecay(int n_seqs, int n_heads, int d_k, int64_t total_tokens,
                         float* g, void* stream);
 
 /*
- * The intra-chunk factors on their own (cumulative decay + intra-chunk
- * kernel), unpacked to plain fp32 arrays for inspection.  With
+ * The intra-chunk factors on their own (the prefill's first stage), unpacked
+ * to plain fp32 arrays for inspection.  With
  * n_slots = floor(T_tot / 64) + N chunk slots, chunk j of sequence n lives in
  * slot floor(cu[n] / 64) + j + n; unused slots are left untouched.  For a
  * chunk with start state S0, its effect on the state and outputs is

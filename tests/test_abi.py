@@ -100,7 +100,7 @@ def test_workspace_size_grows_with_tokens(L):
     s2 = gdr.workspace_size(1, 14, 64, 64, 16384)
     assert 0 < s1 < s2
     assert gdr.workspace_size(1, 14, 96, 96, 8192) == 0
-    assert gdr.workspace_size(1, 14, 128, 128, 8192, True) < gdr.workspace_size(1, 14, 128, 128, 8192, False)
+    assert gdr.workspace_size(1, 14, 128, 128, 8192, True) <= gdr.workspace_size(1, 14, 128, 128, 8192, False)
 
 
 def test_snapshot_count_matches_oracle(L):
@@ -108,3 +108,22 @@ def test_snapshot_count_matches_oracle(L):
     for lengths, iv in (([4096, 100, 8192, 0, 4095], 4096), ([64, 128, 1], 64), ([5, 7], 0)):
         cu = torch.tensor([0] + list(torch.tensor(lengths).cumsum(0)), dtype=torch.int32)
         assert gdr.snapshot_count(cu, iv) == oracle.snapshot_count(cu, iv)
+
+
+def test_prefill_stage_range_and_kernel_count(L):
+    pre = lambda a, f, l: L.gdr_prefill_stages(ctypes.byref(a), f, l, None)
+    assert pre(_args(), -1, 1) == 1
+    assert pre(_args(), 0, 2) == 1
+    assert pre(_args(), 1, 0) == 1
+    assert pre(_args(n_seqs=0, total_tokens=0), 0, 1) == 0
+    # one intra-chunk kernel + one state pass, or + three when segmented
+    assert gdr.kernel_count(1, 14, 64, 64, 8192) == 4          # 14 long heads: segmented
+    assert gdr.kernel_count(32, 32, 128, 128, 278000) == 2     # many pairs: one pass
+    assert gdr.kernel_count(1, 2, 64, 64, 256) == 2            # short: one pass
+    assert gdr.kernel_count(1, 2, 64, 64, 0) == 1              # no tokens: state copy only
+    assert gdr.kernel_count(1, 2, 96, 96, 256) == 0            # unsupported width
+
+
+def test_static_workspace_is_declared_with_its_limit():
+    src = open(os.path.join(ROOT, "include", "gdr.h")).read()
+    assert "GDR_STATIC_WORKSPACE_BYTES" in src
