@@ -143,6 +143,18 @@ __device__ __forceinline__ void tile16(const float* X, int xr, int xk, const flo
     }
 }
 
+// Store -z (a 2 x 4 block of T at rows r, r+1, columns c .. c+3) to the fp32
+// tile Ts and to the bf16 operand tile Tb.
+__device__ __forceinline__ void store_t_tile(float* Ts, uint8_t* Tb, int r, int c,
+                                             const float (&z0)[4], const float (&z1)[4]) {
+    *reinterpret_cast<float4*>(Ts + r * kLd + c) = make_float4(-z0[0], -z0[1], -z0[2], -z0[3]);
+    *reinterpret_cast<float4*>(Ts + (r + 1) * kLd + c) = make_float4(-z1[0], -z1[1], -z1[2], -z1[3]);
+    *reinterpret_cast<uint2*>(Tb + sw128_offset(64, r, c)) =
+        make_uint2(pack_bf16(-z0[0], -z0[1]), pack_bf16(-z0[2], -z0[3]));
+    *reinterpret_cast<uint2*>(Tb + sw128_offset(64, r + 1, c)) =
+        make_uint2(pack_bf16(-z1[0], -z1[1]), pack_bf16(-z1[2], -z1[3]));
+}
+
 // Stage one [64 x D] row block of a token-major tensor into shared memory
 // (rows past the chunk end are zero-filled).
 template <typename T, int D>
@@ -246,7 +258,11 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
 
     // ---- chunk-local cumulative log decay, g[r] = sum_{i <= r} log a_i -------
     // (the same quantity gdr_cumdecay computes; padded rows add 0, so past the
-    // chunk end g stays at g_last)
+    // chunk end g stays at g_last).  The factored per-channel products below
+    // need |g_r - m_b| <= kMaxFactorExp inside each 16-row block, which holds
+    // whenever every log a >= -kMaxFactorExp / 8; a chunk with a smaller log a
+    // in some channel takes the exact path.
+    bool bad = false;
     if (!SCALAR) {
         constexpr int P = kThreads / D, RP = 64 / P;          // row parts per channel
         float* Ptot = reinterpret_cast<float*>(sm + L::Ptot);
@@ -254,7 +270,9 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         float run = 0.f;
 #pragma unroll 4
         for (int r = part * RP; r < (part + 1) * RP; ++r) {
-            run += sG[r * D + c];
+            const float la = sG[r * D + c];
+            bad |= la < -kMaxFactorExp / 8.f;
+            run += la;
             sG[r * D + c] = run;
         }
         Ptot[part * D + c] = run;
@@ -278,16 +296,15 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         Gs[2 * lane] = excl + x0;
         Gs[2 * lane + 1] = excl + pair;
     }
-    __syncthreads();
+    const bool bad_chunk = __syncthreads_or(bad);
 
     const int cg = tid % CG, rg = tid / CG, c0 = 8 * cg;
     const int r0 = rg * RPT;
     const int jb = r0 / 16;                                   // this thread's 16-row block
 
-    // ---- reference points and the overflow check ---------------------------
+    // ---- reference points: g_last, block midpoints m_b -------------------------
     float gl[8], mj[8];
     float ecross[4][8];                       // exp(m_b - m_jb) for b > jb (per-channel)
-    bool bad = false;
     if (!SCALAR) {
         load8f(sG + (size_t)(len - 1) * D + c0, gl);
         load8f(sG + (size_t)min(16 * jb + 8, len - 1) * D + c0, mj);
@@ -300,27 +317,16 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                 for (int e = 0; e < 8; ++e) ecross[b][e] = __expf(mb[e] - mj[e]);
             }
         }
-#pragma unroll
-        for (int u = 0; u < RPT; ++u) {
-            const int r = r0 + u;
-            if (r < len) {
-                float gr[8];
-                load8f(sG + (size_t)r * D + c0, gr);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) bad |= fabsf(gr[e] - mj[e]) > kMaxFactorExp;
-            }
-        }
         if (rg == 0) {
 #pragma unroll
             for (int e = 0; e < 8; ++e) Gl[c0 + e] = gl[e];
         }
     } else {
-        const float glast = Gs[63 < len - 1 ? 63 : len - 1];
+        const float glast = Gs[len - 1];
 #pragma unroll
         for (int e = 0; e < 8; ++e) gl[e] = glast;
         if (tid < D) Gl[tid] = glast;
     }
-    const bool bad_chunk = __syncthreads_or(bad);
 
     // ---- operands and per-token outputs -------------------------------------
     uint8_t* XA = sm + L::XA;
@@ -375,12 +381,23 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                 qg[e] = xq[e] * em[e];
                 kd[e] = kk0[e] * eld[e];
             }
+        } else if (SCALAR) {
+            const float G = __expf(gr[0]), Ed = __expf(gl[0] - gr[0]);   // one gate per row
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                xq[e] = scale * qv[e];
+                xk[e] = kv[e];
+                kk0[e] = 0.f;
+                b1[e] = br * kv[e] * G;
+                qg[e] = scale * qv[e] * G;
+                kd[e] = kv[e] * Ed;
+            }
         } else {
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 const float G = __expf(gr[e]);
-                xq[e] = SCALAR ? scale * qv[e] : 0.f;
-                xk[e] = SCALAR ? kv[e] : 0.f;
+                xq[e] = 0.f;
+                xk[e] = 0.f;
                 kk0[e] = 0.f;
                 b1[e] = br * kv[e] * G;
                 qg[e] = scale * qv[e] * G;
@@ -467,26 +484,33 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     tc_fence_after_sync();
 
     // ---- P (masked, bf16 operand) and A (masked, times beta, fp32) ----------
-    if (warp < 4) {
-        const bool is_p = warp < 2;
-        const int rr = 32 * (warp & 1) + lane;                // chunk row
+    // warps w and w+4 read the same rows; each writes one half of the columns
+    {
+        const int sub = warp & 3, ch = warp >> 2;
+        const bool is_p = sub < 2;
+        const int rr = 32 * (sub & 1) + lane;                 // chunk row
         const int lim = is_p ? rr : rr - 1;                   // last valid key index
-        float vrow[64];
+        const int i0 = 32 * ch;                               // first column of this half
+        float v32[32];
         if (!SCALAR) {
-            if ((warp & 1) == 0) load_ap_row<0>(tmem + lane_base, rr >> 4, vrow);
+            float vrow[64];
+            if ((sub & 1) == 0) load_ap_row<0>(tmem + lane_base, rr >> 4, vrow);
             else load_ap_row<1>(tmem + lane_base, rr >> 4, vrow);
+#pragma unroll
+            for (int il = 0; il < 32; ++il) v32[il] = ch ? vrow[32 + il] : vrow[il];
         } else {
-            tmem_ld32(tmem + lane_base, *reinterpret_cast<float(*)[32]>(vrow));
-            tmem_ld32(tmem + lane_base + 32, *reinterpret_cast<float(*)[32]>(vrow + 32));
+            tmem_ld32(tmem + lane_base + (uint32_t)i0, v32);
             tmem_ld_wait();
             const float gr = Gs[rr];
 #pragma unroll
-            for (int i = 0; i < 64; ++i) vrow[i] = (i <= lim) ? vrow[i] * __expf(gr - Gs[i]) : 0.f;
+            for (int il = 0; il < 32; ++il)
+                v32[il] = (i0 + il <= lim) ? v32[il] * __expf(gr - Gs[i0 + il]) : 0.f;
         }
         if (!SCALAR && bad_chunk) {
             // exact path: every term with its own exp (chunks with extreme decay only)
 #pragma unroll
-            for (int i = 0; i < 64; ++i) {
+            for (int il = 0; il < 32; ++il) {
+                const int i = i0 + il;
                 float acc = 0.f;
                 if (i <= lim && rr < len) {
                     for (int c = 0; c < D; ++c) {
@@ -496,33 +520,46 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                         acc += xr * (float)k[ti] * expf(sG[rr * D + c] - sG[i * D + c]);
                     }
                 }
-                vrow[i] = acc;
+                v32[il] = acc;
             }
         }
         if (is_p) {
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
+            for (int jj = 0; jj < 4; ++jj) {
                 float x[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] = (8 * jj + e <= lim) ? vrow[8 * jj + e] : 0.f;
-                *reinterpret_cast<uint4*>(sm + L::Pt + sw128_chunk(64, rr, jj)) = pack8(x);
+                for (int e = 0; e < 8; ++e) x[e] = (i0 + 8 * jj + e <= lim) ? v32[8 * jj + e] : 0.f;
+                *reinterpret_cast<uint4*>(sm + L::Pt + sw128_chunk(64, rr, 4 * ch + jj)) = pack8(x);
             }
         } else {
             const float br = Bs[rr];
 #pragma unroll
-            for (int i4 = 0; i4 < 16; ++i4) {
+            for (int i4 = 0; i4 < 8; ++i4) {
+                const int i = i0 + 4 * i4;
                 float4 x;
-                x.x = (4 * i4 + 0 <= lim) ? br * vrow[4 * i4 + 0] : 0.f;
-                x.y = (4 * i4 + 1 <= lim) ? br * vrow[4 * i4 + 1] : 0.f;
-                x.z = (4 * i4 + 2 <= lim) ? br * vrow[4 * i4 + 2] : 0.f;
-                x.w = (4 * i4 + 3 <= lim) ? br * vrow[4 * i4 + 3] : 0.f;
-                *reinterpret_cast<float4*>(As + rr * kLd + 4 * i4) = x;
+                x.x = (i + 0 <= lim) ? br * v32[4 * i4 + 0] : 0.f;
+                x.y = (i + 1 <= lim) ? br * v32[4 * i4 + 1] : 0.f;
+                x.z = (i + 2 <= lim) ? br * v32[4 * i4 + 2] : 0.f;
+                x.w = (i + 3 <= lim) ? br * v32[4 * i4 + 3] : 0.f;
+                *reinterpret_cast<float4*>(As + rr * kLd + i) = x;
             }
         }
     }
     __syncthreads();
 
     // ---- T = (I + A)^-1: 16x16 diagonal blocks, then block merges -----------
+    // Every phase writes its fp32 blocks to Ts and their bf16 copy straight into
+    // the operand tile Tb; the blocks above the diagonal of Tb are zeroed here.
+    uint8_t* Tb = sm + L::Tb;
+    if (tid >= 64) {
+        // (row, chunk) pairs of the zero blocks (b, j > b): 96 + 64 + 32
+        const int z = tid - 64;
+        int r, jj;
+        if (z < 96) { r = z / 6; jj = 2 + z % 6; }
+        else if (z < 160) { r = 16 + (z - 96) / 4; jj = 4 + (z - 96) % 4; }
+        else { r = 32 + (z - 160) / 2; jj = 6 + (z - 160) % 2; }
+        *reinterpret_cast<uint4*>(Tb + sw128_chunk(64, r, jj)) = make_uint4(0u, 0u, 0u, 0u);
+    }
     if (tid < 64) {
         const int b = tid >> 4, cc = tid & 15, o = 16 * b;
         float x[16];
@@ -542,6 +579,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
             }
             x[r] = (r < cc) ? 0.f : ((r == cc) ? 1.f : -(a0 + a1));
             Ts[(o + r) * kLd + o + cc] = x[r];
+            *reinterpret_cast<__nv_bfloat16*>(Tb + sw128_offset(64, o + r, o + cc)) = __float2bfloat16_rn(x[r]);
         }
     }
     __syncthreads();
@@ -560,8 +598,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         const int p = tid >> 5, b = 2 * p + 1, j = 2 * p;
         float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
         tile16<16>(Ts, 16 * b + rr0, 16 * b, Yt + p * 256, 0, c4, z0, z1);
-        *reinterpret_cast<float4*>(Ts + (16 * b + rr0) * kLd + 16 * j + c4) = make_float4(-z0[0], -z0[1], -z0[2], -z0[3]);
-        *reinterpret_cast<float4*>(Ts + (16 * b + rr0 + 1) * kLd + 16 * j + c4) = make_float4(-z1[0], -z1[1], -z1[2], -z1[3]);
+        store_t_tile(Ts, Tb, 16 * b + rr0, 16 * j + c4, z0, z1);
     }
     __syncthreads();
     // bottom-left 32 x 32 block, blocks (b, j) with b in {2, 3}, j in {0, 1}:
@@ -580,19 +617,8 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
             float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
             for (int l = 2; l <= b; ++l)
                 tile16<32>(Ts, 16 * b + rr0, 16 * l, Yt, 16 * (l - 2), 16 * j + c4, z0, z1);
-            *reinterpret_cast<float4*>(Ts + (16 * b + rr0) * kLd + 16 * j + c4) = make_float4(-z0[0], -z0[1], -z0[2], -z0[3]);
-            *reinterpret_cast<float4*>(Ts + (16 * b + rr0 + 1) * kLd + 16 * j + c4) = make_float4(-z1[0], -z1[1], -z1[2], -z1[3]);
+            store_t_tile(Ts, Tb, 16 * b + rr0, 16 * j + c4, z0, z1);
         }
-    }
-    __syncthreads();
-    // T -> bf16 operand tile [64 r][64 i] (zero above the diagonal)
-    for (int qd = tid; qd < 512; qd += kThreads) {
-        const int r = qd >> 3, jj = qd & 7;
-        const float4 ta = f4(Ts + r * kLd + 8 * jj), tb = f4(Ts + r * kLd + 8 * jj + 4);
-        float x[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = (8 * jj + e <= r) ? x[e] : 0.f;
-        *reinterpret_cast<uint4*>(sm + L::Tb + sw128_chunk(64, r, jj)) = pack8(x);
     }
     fence_proxy_async_smem();
     tc_fence_before_sync();
