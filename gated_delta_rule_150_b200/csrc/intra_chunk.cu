@@ -155,6 +155,25 @@ __device__ __forceinline__ void store_t_tile(float* Ts, uint8_t* Tb, int r, int 
         make_uint2(pack_bf16(-z1[0], -z1[1]), pack_bf16(-z1[2], -z1[3]));
 }
 
+// a[e] <- a[e ^ s] for e < 8, by three conditional swap stages (s < 8).
+template <int N>
+__device__ __forceinline__ void xor_permute(uint32_t (&a)[8][N], int s) {
+#pragma unroll
+    for (int bit = 1; bit < 8; bit <<= 1) {
+        const bool sw = (s & bit) != 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            if (e & bit) continue;
+#pragma unroll
+            for (int n = 0; n < N; ++n) {
+                const uint32_t x = a[e][n], y = a[e ^ bit][n];
+                a[e][n] = sw ? y : x;
+                a[e ^ bit][n] = sw ? x : y;
+            }
+        }
+    }
+}
+
 // Stage one [64 x D] row block of a token-major tensor into shared memory
 // (rows past the chunk end are zero-filled).
 template <typename T, int D>
@@ -434,10 +453,16 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
             }
         }
     }
-    // B1^T rows c, B2^T rows D + c, Kd^T rows c; token columns r0 .. r0 + RPT - 1
+    // B1^T rows c, B2^T rows D + c, Kd^T rows c; token columns r0 .. r0 + RPT - 1.
+    // Step e of lane group cg writes channel c0 + (e ^ s), s = cg mod 8, so the
+    // lanes of a warp hit 8 different swizzle positions instead of one.
+    const int s8 = cg & 7;
+    xor_permute(pb1, s8);
+    xor_permute(pb2, s8);
+    xor_permute(pkd, s8);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-        const int c = c0 + e;
+        const int c = c0 + (e ^ s8);
         const uint32_t o1 = sw128_chunk(2 * D, c, r0 / 8) + (r0 % 8) * 2;
         const uint32_t o2 = sw128_chunk(2 * D, D + c, r0 / 8) + (r0 % 8) * 2;
         const uint32_t o3 = sw128_chunk(D, c, r0 / 8) + (r0 % 8) * 2;
