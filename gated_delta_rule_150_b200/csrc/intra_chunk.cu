@@ -57,39 +57,56 @@ struct IntraLayout {
     static constexpr uint32_t elem = sizeof(InT);
     // fp32 q/k/v at d 128 do not fit next to everything else: read from global
     static constexpr bool kStageQKV = !(elem == 4 && D == 128);
-    // region 1: staged inputs (operand phase), then Ts, Yt, WUt
+    // region 1: the staged inputs of one chunk.  Free once the A/P products
+    // are read out, when it is refilled with the next chunk's inputs.
     static constexpr uint32_t sQ = 0;
     static constexpr uint32_t sK = sQ + (kStageQKV ? 64u * D * elem : 0u);
     static constexpr uint32_t sV = sK + (kStageQKV ? 64u * D * elem : 0u);
     static constexpr uint32_t sG = sV + (kStageQKV ? 64u * D * elem : 0u);
     static constexpr uint32_t in_bytes = sG + (SCALAR ? 0u : 64u * D * 4u);
-    static constexpr uint32_t Ts = 0;                         // fp32 [64][kLd]
-    static constexpr uint32_t Yt = Ts + 64u * kLd * 4u;       // fp32 [32][32] scratch
-    static constexpr uint32_t WUt = al1024(Yt + 4096u);       // bf16 [2D][64]
-    static constexpr uint32_t r1 = al1024(umax(in_bytes, WUt + 256u * D));
-    // region 2: A/P operands, then As, Pt, Tb
+    static constexpr uint32_t r1 = al1024(in_bytes);
+    // region 2: A/P operands; then As (A, overwritten by T), Pt, Tb, Yt;
+    // finally the record, staged for its bulk store (reaching into Bt, Kdt)
     static constexpr uint32_t XA = r1;                        // bf16 [128][D]
     static constexpr uint32_t KT0 = XA + 256u * D;            // key tiles, 16(b+1) rows each
     static constexpr uint32_t op_bytes = SCALAR ? 256u * D : 576u * D;
     static constexpr uint32_t As = r1;                        // fp32 [64][kLd]
-    static constexpr uint32_t Pt = r1 + 64u * kLd * 4u;       // bf16 [64][64]
+    static constexpr uint32_t Pt = As + 64u * kLd * 4u;       // bf16 [64][64]
     static constexpr uint32_t Tb = Pt + 8192u;                // bf16 [64][64]
-    static constexpr uint32_t r2 = al1024(umax(op_bytes, 64u * kLd * 4u + 16384u));
-    // region 3: live throughout
-    static constexpr uint32_t Bt = r1 + r2;                   // bf16 [2D][64]
+    static constexpr uint32_t Yt = Tb + 8192u;                // fp32 [32][32] scratch
+    static constexpr uint32_t solve_bytes = 64u * kLd * 4u + 16384u + 4096u;
+    static constexpr uint32_t Rec = r1;                       // record staging
+    static constexpr uint32_t rec_bytes = record_layout(D).bytes;
+    static constexpr uint32_t r2 = al1024(umax(umax(op_bytes, solve_bytes),
+                                               rec_bytes > 384u * D ? rec_bytes - 384u * D : 0u));
+    // region 3: live through the chunk
+    static constexpr uint32_t Bt = r1 + r2;                   // bf16 [2D][64]; then [W | U]^T
+    static constexpr uint32_t WUt = Bt;
     static constexpr uint32_t Kdt = Bt + 256u * D;            // bf16 [D][64]
     static constexpr uint32_t Qgs = Kdt + 128u * D;           // bf16 [64][D]
     static constexpr uint32_t Gl = Qgs + 128u * D;            // fp32 [D] g_last
     static constexpr uint32_t Bs = Gl + 4u * D;               // fp32 [64] beta
     static constexpr uint32_t Gs = Bs + 256u;                 // fp32 [64] g (scalar decay)
-    static constexpr uint32_t Ptot = Gs + 256u;               // fp32 scan partials [1024 B]
-    static constexpr uint32_t bytes = Ptot + 1024u;
-    static constexpr uint32_t dyn_bytes = bytes + 1024u;
+    // fp32 scan partials [1024 B], live only during the scan: in region 2
+    // past the operands and the (possibly still draining) record when it fits
+    static constexpr uint32_t free2 = umax(op_bytes, rec_bytes);
+    static constexpr bool kPtotInR2 = free2 + 1024u <= r2;
+    static constexpr uint32_t Ptot = kPtotInR2 ? r1 + free2 : Gs + 256u;
+    static constexpr uint32_t bytes = Gs + 256u + (kPtotInR2 ? 0u : 1024u);
+    // at d 128 the 512 TMEM columns of a CTA allow one CTA per SM: request
+    // enough shared memory that a second one is never scheduled
+    static constexpr uint32_t dyn_bytes = (D == 128) ? umax(bytes + 1024u, 118784u) : bytes + 1024u;
     __host__ __device__ static constexpr uint32_t kt_off(int b) {
         return KT0 + 32u * D * (uint32_t)(b * (b + 1) / 2);
     }
     static_assert(dyn_bytes <= 232448u, "shared memory budget");
     static_assert((64u * kLd * 4u) % 1024u == 0u, "Pt alignment");
+    static_assert(Rec + rec_bytes <= Qgs, "record staging stays below Qgs");
+    // TMEM is allocated once per persistent CTA: never more CTAs on an SM
+    // than its 512 columns hold (2 x 256 at d 64, 1 x 512 at d 128)
+    static_assert(3u * (dyn_bytes + 1088u) > 233472u, "at most two CTAs per SM");
+    static_assert(!(D == 64 && elem == 2) || dyn_bytes + 1088u <= 114688u, "two CTAs per SM at d 64");
+    static_assert(D != 128 || 2u * (dyn_bytes + 1088u) > 233472u, "one CTA per SM at d 128");
 };
 
 // TMEM column of query block b's A/P product (16(b+1) columns each).
@@ -144,7 +161,7 @@ __device__ __forceinline__ void tile16(const float* X, int xr, int xk, const flo
 }
 
 // Store -z (a 2 x 4 block of T at rows r, r+1, columns c .. c+3) to the fp32
-// tile Ts and to the bf16 operand tile Tb.
+// tile Ts (row stride kLd) and to the bf16 operand tile Tb.
 __device__ __forceinline__ void store_t_tile(float* Ts, uint8_t* Tb, int r, int c,
                                              const float (&z0)[4], const float (&z1)[4]) {
     *reinterpret_cast<float4*>(Ts + r * kLd + c) = make_float4(-z0[0], -z0[1], -z0[2], -z0[3]);
@@ -189,6 +206,58 @@ __device__ __forceinline__ void stage_rows(uint8_t* dst, const T* src, size_t to
     }
 }
 
+// One unit of work: chunk slot idx / H of head idx % H (idx < 0: none).
+struct Item {
+    int64_t idx;
+    int h, start, len;
+};
+
+// The first item at or after `from`, stepping by the grid size, whose chunk
+// slot holds a chunk (the slot map leaves one unused slot per sequence).
+__device__ __forceinline__ Item find_item(const int32_t* __restrict__ cu, int n_seqs, int H,
+                                          int64_t n_items, int64_t from) {
+    Item it{-1, 0, 0, 0};
+    for (int64_t i = from; i < n_items; i += gridDim.x) {
+        int seq, start, len;
+        if (slot_to_chunk(cu, n_seqs, i / H, &seq, &start, &len)) {
+            it.idx = i;
+            it.h = (int)(i % H);
+            it.start = start;
+            it.len = len;
+            break;
+        }
+    }
+    return it;
+}
+
+// Issue the copies of one item's inputs: log a, beta (and the scalar log a)
+// as cp.async group 0, q, k, v as group 1.  Rows past the chunk end are
+// zero-filled.
+template <int D, typename InT, bool SCALAR, typename L>
+__device__ __forceinline__ void issue_inputs(uint8_t* sm, const InT* __restrict__ q,
+                                             const InT* __restrict__ k, const InT* __restrict__ v,
+                                             const float* __restrict__ beta,
+                                             const float* __restrict__ log_a, int H, const Item& it,
+                                             int tid) {
+    const size_t tok_stride = (size_t)H * D;
+    const size_t base = (size_t)it.start * tok_stride + (size_t)it.h * D;
+    if (!SCALAR) stage_rows<float, D>(sm + L::sG, log_a + base, tok_stride, it.len, tid);
+    if (tid < 64) {
+        const int t = tid < it.len ? tid : it.len - 1;
+        const size_t o = (size_t)(it.start + t) * H + it.h;
+        const uint32_t n = tid < it.len ? 4u : 0u;
+        cp_async4(sm + L::Bs + 4 * tid, beta + o, n);
+        if (SCALAR) cp_async4(sm + L::Gs + 4 * tid, log_a + o, n);
+    }
+    cp_async_commit();
+    if (L::kStageQKV) {
+        stage_rows<InT, D>(sm + L::sQ, q + base, tok_stride, it.len, tid);
+        stage_rows<InT, D>(sm + L::sK, k + base, tok_stride, it.len, tid);
+        stage_rows<InT, D>(sm + L::sV, v + base, tok_stride, it.len, tid);
+    }
+    cp_async_commit();
+}
+
 // Read the A/P products of this thread's row from TMEM (per-channel decay).
 // Lanes of warp parity `par` own rows 32 par .. 32 par + 31, i.e. query
 // blocks 2 par and 2 par + 1, whose columns are loaded together.
@@ -226,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, (D == 64) ? 2 : 1)
 intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                    const InT* __restrict__ q, const InT* __restrict__ k, const InT* __restrict__ v,
                    const float* __restrict__ beta, const float* __restrict__ log_a, float scale,
-                   uint8_t* __restrict__ records, uint32_t* err) {
+                   int64_t n_items, uint8_t* __restrict__ records, uint32_t* err) {
     using L = IntraLayout<D, InT, SCALAR>;
     constexpr RecordLayout R = record_layout(D);
     constexpr int CG = D / 8;              // channel groups of 8
@@ -234,21 +303,15 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     constexpr int RPT = 64 / RG;           // rows per thread: 2 (D=64) or 4 (D=128)
     constexpr uint32_t kTmemCols = (D == 64) ? 256u : 512u;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+    uint8_t* sm = align_smem<1024>(smem_raw);
     __shared__ uint64_t mma_bar;
     __shared__ uint32_t tmem_slot;
+    __shared__ Item s_next;                 // the item after the current one
 
-    int seq, start, len;
-    if (!slot_to_chunk(cu, n_seqs, blockIdx.x, &seq, &start, &len)) return;
-    const int h = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    uint8_t* rec = records + ((size_t)blockIdx.x * H + h) * R.bytes;
     const size_t tok_stride = (size_t)H * D;
-    const size_t base = (size_t)start * tok_stride + (size_t)h * D;
 
     float* As = reinterpret_cast<float*>(sm + L::As);
-    float* Ts = reinterpret_cast<float*>(sm + L::Ts);
     float* Yt = reinterpret_cast<float*>(sm + L::Yt);
     float* Gl = reinterpret_cast<float*>(sm + L::Gl);
     float* Bs = reinterpret_cast<float*>(sm + L::Bs);
@@ -261,18 +324,28 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     }
     if (warp == 0) tmem_alloc(&tmem_slot, kTmemCols);
 
-    // ---- stage the chunk's inputs in shared memory -------------------------
-    if (L::kStageQKV) {
-        stage_rows<InT, D>(sm + L::sQ, q + base, tok_stride, len, tid);
-        stage_rows<InT, D>(sm + L::sK, k + base, tok_stride, len, tid);
-        stage_rows<InT, D>(sm + L::sV, v + base, tok_stride, len, tid);
-    }
-    if (!SCALAR) stage_rows<float, D>(sm + L::sG, log_a + base, tok_stride, len, tid);
-    if (tid < 64) {
-        Bs[tid] = tid < len ? __ldg(beta + (size_t)(start + tid) * H + h) : 0.f;
-        if (SCALAR) Gs[tid] = tid < len ? __ldg(log_a + (size_t)(start + tid) * H + h) : 0.f;
-    }
-    cp_async_wait_all();
+    // Persistent CTA: items blockIdx.x, blockIdx.x + gridDim.x, ...  The next
+    // item's inputs are staged while the current one is finished, and each
+    // record's bulk store drains while the next item starts.
+    Item cur = find_item(cu, n_seqs, H, n_items, blockIdx.x);
+    if (cur.idx >= 0) issue_inputs<D, InT, SCALAR, L>(sm, q, k, v, beta, log_a, H, cur, tid);
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = tmem_slot;
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+    const int whalf = warp >> 2;                              // warps w and w+4 share TMEM lanes
+    uint32_t phase = 0;                                       // parity of the next MMA commit
+    bool failed = false;
+
+    while (cur.idx >= 0) {
+    if (tid == 0) s_next = find_item(cu, n_seqs, H, n_items, cur.idx + gridDim.x);
+    const int h = cur.h, start = cur.start, len = cur.len;
+    uint8_t* rec = records + (size_t)cur.idx * R.bytes;       // item = slot * H + h
+    const size_t base = (size_t)start * tok_stride + (size_t)h * D;
+
+    // ---- this item's log a and beta (group 0) have landed ----------------------
+    cp_async_wait_group<1>();
     __syncthreads();
 
     // ---- chunk-local cumulative log decay, g[r] = sum_{i <= r} log a_i -------
@@ -346,6 +419,11 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         for (int e = 0; e < 8; ++e) gl[e] = glast;
         if (tid < D) Gl[tid] = glast;
     }
+    // q, k, v (group 1) have landed and the previous record's bulk store has
+    // finished reading the region the operands go to
+    cp_async_wait_group<0>();
+    if (tid == 0) bulk_wait_group_read0();
+    __syncthreads();
 
     // ---- operands and per-token outputs -------------------------------------
     uint8_t* XA = sm + L::XA;
@@ -480,9 +558,6 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
-    const uint32_t tmem = tmem_slot;
-    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-    const int whalf = warp >> 2;                              // warps w and w+4 share TMEM lanes
 
     // ---- decay-weighted Q K^T and K K^T on the tensor cores ------------------
     if (tid == 0) {
@@ -505,7 +580,8 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         }
         mma_commit(&mma_bar);
     }
-    bool failed = !mbar_wait(&mma_bar, 0);
+    failed = !mbar_wait(&mma_bar, phase);
+    phase ^= 1u;
     tc_fence_after_sync();
 
     // ---- P (masked, bf16 operand) and A (masked, times beta, fp32) ----------
@@ -572,9 +648,17 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     }
     __syncthreads();
 
+    // region 1 and beta are free: stage the next item's inputs
+    {
+        const Item nxt = s_next;
+        if (nxt.idx >= 0) issue_inputs<D, InT, SCALAR, L>(sm, q, k, v, beta, log_a, H, nxt, tid);
+    }
+
     // ---- T = (I + A)^-1: 16x16 diagonal blocks, then block merges -----------
-    // Every phase writes its fp32 blocks to Ts and their bf16 copy straight into
-    // the operand tile Tb; the blocks above the diagonal of Tb are zeroed here.
+    // T overwrites A in As block by block, each block once the phases that
+    // still read it have passed a barrier.  Every phase also writes its bf16
+    // copy straight into the operand tile Tb, whose blocks above the
+    // diagonal are zeroed here.
     uint8_t* Tb = sm + L::Tb;
     if (tid >= 64) {
         // (row, chunk) pairs of the zero blocks (b, j > b): 96 + 64 + 32
@@ -596,6 +680,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                 const float4 t = f4(As + (o + r) * kLd + o + 4 * i4);
                 ar[4 * i4] = t.x; ar[4 * i4 + 1] = t.y; ar[4 * i4 + 2] = t.z; ar[4 * i4 + 3] = t.w;
             }
+            __syncwarp();      // row r of A_bb is read by all 16 lanes before T overwrites it
             float a0 = 0.f, a1 = 0.f;
 #pragma unroll
             for (int i = 0; i < r; ++i) {
@@ -603,7 +688,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                 else a0 = fmaf(ar[i], x[i], a0);
             }
             x[r] = (r < cc) ? 0.f : ((r == cc) ? 1.f : -(a0 + a1));
-            Ts[(o + r) * kLd + o + cc] = x[r];
+            As[(o + r) * kLd + o + cc] = x[r];
             *reinterpret_cast<__nv_bfloat16*>(Tb + sw128_offset(64, o + r, o + cc)) = __float2bfloat16_rn(x[r]);
         }
     }
@@ -614,7 +699,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     if (tid < 64) {
         const int p = tid >> 5, b = 2 * p + 1, j = 2 * p;
         float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
-        tile16<kLd>(As, 16 * b + rr0, 16 * j, Ts, 16 * j, 16 * j + c4, y0, y1);
+        tile16<kLd>(As, 16 * b + rr0, 16 * j, As, 16 * j, 16 * j + c4, y0, y1);
         *reinterpret_cast<float4*>(Yt + p * 256 + rr0 * 16 + c4) = make_float4(y0[0], y0[1], y0[2], y0[3]);
         *reinterpret_cast<float4*>(Yt + p * 256 + (rr0 + 1) * 16 + c4) = make_float4(y1[0], y1[1], y1[2], y1[3]);
     }
@@ -622,8 +707,8 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     if (tid < 64) {
         const int p = tid >> 5, b = 2 * p + 1, j = 2 * p;
         float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
-        tile16<16>(Ts, 16 * b + rr0, 16 * b, Yt + p * 256, 0, c4, z0, z1);
-        store_t_tile(Ts, Tb, 16 * b + rr0, 16 * j + c4, z0, z1);
+        tile16<16>(As, 16 * b + rr0, 16 * b, Yt + p * 256, 0, c4, z0, z1);
+        store_t_tile(As, Tb, 16 * b + rr0, 16 * j + c4, z0, z1);
     }
     __syncthreads();
     // bottom-left 32 x 32 block, blocks (b, j) with b in {2, 3}, j in {0, 1}:
@@ -633,7 +718,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         if (tid < 128) {
             float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
             for (int l = j; l <= 1; ++l)
-                tile16<kLd>(As, 16 * b + rr0, 16 * l, Ts, 16 * l, 16 * j + c4, y0, y1);
+                tile16<kLd>(As, 16 * b + rr0, 16 * l, As, 16 * l, 16 * j + c4, y0, y1);
             *reinterpret_cast<float4*>(Yt + (16 * (b - 2) + rr0) * 32 + 16 * j + c4) = make_float4(y0[0], y0[1], y0[2], y0[3]);
             *reinterpret_cast<float4*>(Yt + (16 * (b - 2) + rr0 + 1) * 32 + 16 * j + c4) = make_float4(y1[0], y1[1], y1[2], y1[3]);
         }
@@ -641,8 +726,8 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         if (tid < 128) {
             float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
             for (int l = 2; l <= b; ++l)
-                tile16<32>(Ts, 16 * b + rr0, 16 * l, Yt, 16 * (l - 2), 16 * j + c4, z0, z1);
-            store_t_tile(Ts, Tb, 16 * b + rr0, 16 * j + c4, z0, z1);
+                tile16<32>(As, 16 * b + rr0, 16 * l, Yt, 16 * (l - 2), 16 * j + c4, z0, z1);
+            store_t_tile(As, Tb, 16 * b + rr0, 16 * j + c4, z0, z1);
         }
     }
     fence_proxy_async_smem();
@@ -662,7 +747,8 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                          sw128_desc(aT, 64, 0, 16 * kk), id, kk > 0);
         mma_commit(&mma_bar);
     }
-    if (!failed && !mbar_wait(&mma_bar, 1)) failed = true;
+    if (!failed && !mbar_wait(&mma_bar, phase)) failed = true;
+    phase ^= 1u;
     tc_fence_after_sync();
 
     // W^T rows c and U^T rows v -> one bf16 tile [2D][64] (row D + v for U^T)
@@ -707,14 +793,15 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         }
         mma_commit(&mma_bar);
     }
-    if (!failed && !mbar_wait(&mma_bar, 0)) failed = true;
+    if (!failed && !mbar_wait(&mma_bar, phase)) failed = true;
+    phase ^= 1u;
     tc_fence_after_sync();
 
     // ---- record: Qt = Qg - P W, PU, BS = -Kd^T W, NC = U^T Kd, gamma ----------
-    // assembled in shared memory below Qgs (everything there is dead once the
-    // MMAs above have completed) and written with one bulk store
-    uint8_t* srec = sm;
-    static_assert(R.bytes <= L::Qgs, "record staging fits below Qgs");
+    // assembled in region 2 and the dead Bt, Kdt (everything there is dead
+    // once the MMAs above have completed) and written with one bulk store,
+    // which drains while the next item starts
+    uint8_t* srec = sm + L::Rec;
     {
         // rows of the M = 64 products live in lanes 16 w + l (l < 16)
         const int r64 = 16 * (warp & 3) + lane;
@@ -763,15 +850,23 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         }
         if (tid < D) reinterpret_cast<float*>(srec + R.gamma)[tid] = expf(Gl[tid]);
     }
+    const Item nxt = s_next;                  // read before thread 0 may overwrite it
     fence_proxy_async_smem();
     tc_fence_before_sync();
-    __syncthreads();
+    failed = __syncthreads_or(failed);
+    tc_fence_after_sync();
     if (tid == 0) {
         bulk_s2g(rec, srec, R.bytes);
         bulk_commit_group();
-        bulk_wait_group_read0();
         if (failed) atomicOr(err, 1u);
     }
+    if (failed) break;                        // a timed-out MMA: stop issuing work                        // a timed-out MMA: stop issuing work
+    cur = nxt;
+    }
+
+    cp_async_wait_all();
+    if (tid == 0) bulk_wait_group0();
+    tc_fence_before_sync();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
@@ -810,10 +905,40 @@ cudaError_t launch_typed(const gdr_prefill_args& a, uint8_t* records, uint32_t* 
     const uint32_t smem = IntraLayout<D, InT, SCALAR>::dyn_bytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const dim3 grid((unsigned)n_chunk_slots(a.total_tokens, a.n_seqs), (unsigned)a.n_heads);
+    // all of the unified L1 / shared memory as shared memory, so that the
+    // occupancy below (two CTAs per SM at d 64) is what the launch gets
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    // persistent grid: every CTA that fits on the device at once, items
+    // (chunk slot, head) handed out round-robin
+    static thread_local int cached_dev = -1, resident = 0;
+    int dev = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if (dev != cached_dev) {
+        // CTAs per SM from the kernel's registers and shared memory (the
+        // occupancy calculator under-reports the two CTAs per SM that fit at
+        // d 64); at most two, which is what the TMEM columns allow
+        int sms = 0, smem_sm = 0, rsv = 0;
+        cudaFuncAttributes fa;
+        if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+        if ((e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev)) != cudaSuccess)
+            return e;
+        if ((e = cudaDeviceGetAttribute(&rsv, cudaDevAttrReservedSharedMemoryPerBlock, dev)) != cudaSuccess) return e;
+        if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess) return e;
+        const int cta_smem = ((int)(smem + fa.sharedSizeBytes) + rsv + 127) & ~127;
+        const int cta_regs = ((fa.numRegs + 7) & ~7) * kThreads;
+        int per_sm = smem_sm / cta_smem;
+        per_sm = per_sm < 65536 / cta_regs ? per_sm : 65536 / cta_regs;
+        per_sm = per_sm < 2 ? per_sm : 2;
+        resident = sms * (per_sm > 0 ? per_sm : 1);
+        cached_dev = dev;
+    }
+    const int64_t n_items = n_chunk_slots(a.total_tokens, a.n_seqs) * (int64_t)a.n_heads;
+    const unsigned grid = (unsigned)(n_items < resident ? n_items : resident);
     kern<<<grid, kThreads, smem, st>>>(a.cu_seqlens, a.n_seqs, a.n_heads, (const InT*)a.q,
                                        (const InT*)a.k, (const InT*)a.v, a.beta, a.log_a, a.scale,
-                                       records, err);
+                                       n_items, records, err);
     return cudaGetLastError();
 }
 

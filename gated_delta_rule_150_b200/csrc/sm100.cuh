@@ -13,6 +13,18 @@ namespace gdr {
 // ---------------------------------------------------------------------------
 // Generic helpers
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p);
+
+// Round a dynamic shared-memory pointer up to kAlign bytes.  The offset is
+// added to the shared array itself (not computed through an integer cast), so
+// every access derived from the result stays a shared-memory access instead of
+// a generic one.
+template <uint32_t kAlign>
+__device__ __forceinline__ uint8_t* align_smem(uint8_t* base) {
+    const uint32_t a = smem_u32(base);
+    return base + ((kAlign - (a & (kAlign - 1u))) & (kAlign - 1u));
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -99,6 +111,22 @@ __device__ __forceinline__ void bulk_wait_group0() {
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src, uint32_t src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
                  ::"r"(smem_u32(smem_dst)), "l"(gmem_src), "r"(src_bytes) : "memory");
+}
+
+// 4-byte cp.async (src_bytes 0 zero-fills the destination word).
+__device__ __forceinline__ void cp_async4(void* smem_dst, const void* gmem_src, uint32_t src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;"
+                 ::"r"(smem_u32(smem_dst)), "l"(gmem_src), "r"(src_bytes) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+// Wait until at most N of this thread's committed cp.async groups are pending.
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 __device__ __forceinline__ void cp_async_wait_all() {

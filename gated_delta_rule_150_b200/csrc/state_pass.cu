@@ -90,8 +90,7 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     constexpr uint32_t kTmemCols = (D == 64) ? 256u : 512u;
     constexpr int CW = D / 2;                                       // columns per thread
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+    uint8_t* sm = align_smem<1024>(smem_raw);
     __shared__ uint64_t full[ST];
     __shared__ uint64_t mma_bar;
     __shared__ uint32_t tmem_slot;
@@ -434,8 +433,7 @@ combine_kernel(const int32_t* __restrict__ cu, int H, int seg_chunks, const floa
     constexpr int RB = kCombineRows;
     constexpr int QD = D / 4;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
-                                             ~static_cast<uintptr_t>(127));
+    uint8_t* sm = align_smem<128>(smem_raw);
     constexpr int NB = kCombineBufs;
     __shared__ uint64_t full[NB];
     const int pair = blockIdx.x, rb = blockIdx.y;
