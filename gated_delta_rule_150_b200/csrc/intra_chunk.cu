@@ -39,6 +39,9 @@
 // bf16; P [W | U], Kd^T W and U^T Kd are three more MMAs.
 #include <cuda_bf16.h>
 
+#include <cstring>
+#include <cuda.h>      // CUtensorMap and its enums; the encoder is looked up at run time
+
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -191,21 +194,6 @@ __device__ __forceinline__ void xor_permute(uint32_t (&a)[8][N], int s) {
     }
 }
 
-// Stage one [64 x D] row block of a token-major tensor into shared memory
-// (rows past the chunk end are zero-filled).
-template <typename T, int D>
-__device__ __forceinline__ void stage_rows(uint8_t* dst, const T* src, size_t tok_stride, int len,
-                                           int tid) {
-    constexpr int CPR = D * (int)sizeof(T) / 16;              // 16-byte chunks per row
-    for (int idx = tid; idx < 64 * CPR; idx += kThreads) {
-        const int r = idx / CPR, j = idx % CPR;
-        const int rs = r < len ? r : len - 1;
-        cp_async16(dst + (size_t)r * D * sizeof(T) + 16 * j,
-                   reinterpret_cast<const uint8_t*>(src + (size_t)rs * tok_stride) + 16 * j,
-                   r < len ? 16u : 0u);
-    }
-}
-
 // One unit of work: chunk slot idx / H of head idx % H (idx < 0: none).
 struct Item {
     int64_t idx;
@@ -230,30 +218,41 @@ __device__ __forceinline__ Item find_item(const int32_t* __restrict__ cu, int n_
     return it;
 }
 
-// Issue the copies of one item's inputs: log a, beta (and the scalar log a)
-// as cp.async group 0, q, k, v as group 1.  Rows past the chunk end are
-// zero-filled.
+// Tensor maps of the token-major inputs: q, k, v and log a, each a 2-D view
+// [tokens][H * D] read in boxes of 64 tokens x D channels (rows past the
+// tensor end are zero-filled; rows past a sequence end are masked by their
+// consumers).
+struct InputMaps {
+    CUtensorMap q, k, v, g;
+};
+
+// Issue the copies of one item's inputs, from one warp: lane 0 starts the
+// tiled TMA loads of log a (completing on bar_g) and of q, k, v (on bar_qkv);
+// beta and the scalar log a go by 4-byte cp.async with zero fill.
 template <int D, typename InT, bool SCALAR, typename L>
-__device__ __forceinline__ void issue_inputs(uint8_t* sm, const InT* __restrict__ q,
-                                             const InT* __restrict__ k, const InT* __restrict__ v,
-                                             const float* __restrict__ beta,
+__device__ __forceinline__ void issue_inputs(uint8_t* sm, uint64_t* bar_g, uint64_t* bar_qkv,
+                                             const InputMaps& maps, const float* __restrict__ beta,
                                              const float* __restrict__ log_a, int H, const Item& it,
-                                             int tid) {
-    const size_t tok_stride = (size_t)H * D;
-    const size_t base = (size_t)it.start * tok_stride + (size_t)it.h * D;
-    if (!SCALAR) stage_rows<float, D>(sm + L::sG, log_a + base, tok_stride, it.len, tid);
-    if (tid < 64) {
-        const int t = tid < it.len ? tid : it.len - 1;
-        const size_t o = (size_t)(it.start + t) * H + it.h;
-        const uint32_t n = tid < it.len ? 4u : 0u;
-        cp_async4(sm + L::Bs + 4 * tid, beta + o, n);
-        if (SCALAR) cp_async4(sm + L::Gs + 4 * tid, log_a + o, n);
+                                             int lane) {
+    if (lane == 0) {
+        const int x = it.h * D;
+        if (!SCALAR) {
+            mbar_arrive_expect_tx(bar_g, 64u * D * 4u);
+            tma_load_2d(sm + L::sG, &maps.g, x, it.start, bar_g);
+        }
+        if (L::kStageQKV) {
+            mbar_arrive_expect_tx(bar_qkv, 3u * 64u * D * (uint32_t)sizeof(InT));
+            tma_load_2d(sm + L::sQ, &maps.q, x, it.start, bar_qkv);
+            tma_load_2d(sm + L::sK, &maps.k, x, it.start, bar_qkv);
+            tma_load_2d(sm + L::sV, &maps.v, x, it.start, bar_qkv);
+        }
     }
-    cp_async_commit();
-    if (L::kStageQKV) {
-        stage_rows<InT, D>(sm + L::sQ, q + base, tok_stride, it.len, tid);
-        stage_rows<InT, D>(sm + L::sK, k + base, tok_stride, it.len, tid);
-        stage_rows<InT, D>(sm + L::sV, v + base, tok_stride, it.len, tid);
+    for (int t = lane; t < 64; t += 32) {
+        const int tc = t < it.len ? t : it.len - 1;
+        const size_t o = (size_t)(it.start + tc) * H + it.h;
+        const uint32_t n = t < it.len ? 4u : 0u;
+        cp_async4(sm + L::Bs + 4 * t, beta + o, n);
+        if (SCALAR) cp_async4(sm + L::Gs + 4 * t, log_a + o, n);
     }
     cp_async_commit();
 }
@@ -295,7 +294,8 @@ __global__ void __launch_bounds__(kThreads, (D == 64) ? 2 : 1)
 intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                    const InT* __restrict__ q, const InT* __restrict__ k, const InT* __restrict__ v,
                    const float* __restrict__ beta, const float* __restrict__ log_a, float scale,
-                   int64_t n_items, uint8_t* __restrict__ records, uint32_t* err) {
+                   int64_t n_items, uint8_t* __restrict__ records, uint32_t* err,
+                   const __grid_constant__ InputMaps maps) {
     using L = IntraLayout<D, InT, SCALAR>;
     constexpr RecordLayout R = record_layout(D);
     constexpr int CG = D / 8;              // channel groups of 8
@@ -305,6 +305,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align_smem<1024>(smem_raw);
     __shared__ uint64_t mma_bar;
+    __shared__ uint64_t in_bar[2];          // inputs landed: log a, q/k/v
     __shared__ uint32_t tmem_slot;
     __shared__ Item s_next;                 // the item after the current one
 
@@ -318,8 +319,11 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     float* Gs = reinterpret_cast<float*>(sm + L::Gs);
     float* sG = reinterpret_cast<float*>(sm + L::sG);
 
+    constexpr int kLoadWarp = kThreads / 32 - 1;              // issues the input copies
     if (tid == 0) {
         mbar_init(&mma_bar, 1);
+        mbar_init(&in_bar[0], 1);
+        mbar_init(&in_bar[1], 1);
         fence_mbar_init();
     }
     if (warp == 0) tmem_alloc(&tmem_slot, kTmemCols);
@@ -328,14 +332,16 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     // item's inputs are staged while the current one is finished, and each
     // record's bulk store drains while the next item starts.
     Item cur = find_item(cu, n_seqs, H, n_items, blockIdx.x);
-    if (cur.idx >= 0) issue_inputs<D, InT, SCALAR, L>(sm, q, k, v, beta, log_a, H, cur, tid);
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
+    if (cur.idx >= 0 && warp == kLoadWarp)
+        issue_inputs<D, InT, SCALAR, L>(sm, &in_bar[0], &in_bar[1], maps, beta, log_a, H, cur, lane);
     const uint32_t tmem = tmem_slot;
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
     const int whalf = warp >> 2;                              // warps w and w+4 share TMEM lanes
     uint32_t phase = 0;                                       // parity of the next MMA commit
+    uint32_t in_phase = 0;                                    // parity of the inputs' barriers
     bool failed = false;
 
     while (cur.idx >= 0) {
@@ -344,9 +350,16 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     uint8_t* rec = records + (size_t)cur.idx * R.bytes;       // item = slot * H + h
     const size_t base = (size_t)start * tok_stride + (size_t)h * D;
 
-    // ---- this item's log a and beta (group 0) have landed ----------------------
-    cp_async_wait_group<1>();
-    __syncthreads();
+    // ---- this item's log a and beta have landed --------------------------------
+    {
+        const bool ok = SCALAR || mbar_wait(&in_bar[0], in_phase);
+        if (warp == kLoadWarp) cp_async_wait_all();
+        failed = __syncthreads_or(!ok);
+        if (failed) {
+            if (tid == 0) atomicOr(err, 1u);
+            break;
+        }
+    }
 
     // ---- chunk-local cumulative log decay, g[r] = sum_{i <= r} log a_i -------
     // (the same quantity gdr_cumdecay computes; padded rows add 0, so past the
@@ -362,7 +375,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         float run = 0.f;
 #pragma unroll 4
         for (int r = part * RP; r < (part + 1) * RP; ++r) {
-            const float la = sG[r * D + c];
+            const float la = r < len ? sG[r * D + c] : 0.f;   // rows past the end add 0
             bad |= la < -kMaxFactorExp / 8.f;
             run += la;
             sG[r * D + c] = run;
@@ -419,11 +432,18 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         for (int e = 0; e < 8; ++e) gl[e] = glast;
         if (tid < D) Gl[tid] = glast;
     }
-    // q, k, v (group 1) have landed and the previous record's bulk store has
-    // finished reading the region the operands go to
-    cp_async_wait_group<0>();
-    if (tid == 0) bulk_wait_group_read0();
-    __syncthreads();
+    // q, k, v have landed and the previous record's bulk store has finished
+    // reading the region the operands go to
+    {
+        const bool ok = !L::kStageQKV || mbar_wait(&in_bar[1], in_phase);
+        in_phase ^= 1u;
+        if (tid == 0) bulk_wait_group_read0();
+        failed = __syncthreads_or(!ok);
+        if (failed) {
+            if (tid == 0) atomicOr(err, 1u);
+            break;
+        }
+    }
 
     // ---- operands and per-token outputs -------------------------------------
     uint8_t* XA = sm + L::XA;
@@ -443,7 +463,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         const bool valid = r < len;
         float qv[8], kv[8], vv[8], gr[8];
         const float br = Bs[r];
-        if (L::kStageQKV) {
+        if (valid && L::kStageQKV) {
             Vec8<InT>::load(reinterpret_cast<const InT*>(sm + L::sQ) + (size_t)r * D + c0, qv);
             Vec8<InT>::load(reinterpret_cast<const InT*>(sm + L::sK) + (size_t)r * D + c0, kv);
             Vec8<InT>::load(reinterpret_cast<const InT*>(sm + L::sV) + (size_t)r * D + c0, vv);
@@ -649,9 +669,11 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     __syncthreads();
 
     // region 1 and beta are free: stage the next item's inputs
-    {
+    if (warp == kLoadWarp) {
         const Item nxt = s_next;
-        if (nxt.idx >= 0) issue_inputs<D, InT, SCALAR, L>(sm, q, k, v, beta, log_a, H, nxt, tid);
+        fence_proxy_async_smem();             // this item's reads of region 1 come first
+        if (nxt.idx >= 0)
+            issue_inputs<D, InT, SCALAR, L>(sm, &in_bar[0], &in_bar[1], maps, beta, log_a, H, nxt, lane);
     }
 
     // ---- T = (I + A)^-1: 16x16 diagonal blocks, then block merges -----------
@@ -898,6 +920,39 @@ __global__ void unpack_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         gamma[sh * D + c] = reinterpret_cast<const float*>(rec + R.gamma)[c];
 }
 
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// The driver's tensor-map encoder, fetched through the runtime once.
+cudaError_t tensor_map_encoder(EncodeTiledFn* fn) {
+    static EncodeTiledFn cached = nullptr;
+    if (!cached) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        const cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+        if (e != cudaSuccess) return e;
+        if (q != cudaDriverEntryPointSuccess || p == nullptr) return cudaErrorSymbolNotFound;
+        cached = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    *fn = cached;
+    return cudaSuccess;
+}
+
+// Map of a token-major [T][H][D] tensor as [T][H * D], box 64 tokens x D.
+cudaError_t token_map(EncodeTiledFn enc, CUtensorMap* m, const void* base, CUtensorMapDataType dt,
+                      uint32_t elem, int64_t T, int H, int D) {
+    const cuuint64_t dims[2] = {(cuuint64_t)H * D, (cuuint64_t)T};
+    const cuuint64_t strides[1] = {(cuuint64_t)H * D * elem};
+    const cuuint32_t box[2] = {(cuuint32_t)D, 64u};
+    const cuuint32_t estr[2] = {1u, 1u};
+    const CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 template <int D, typename InT, bool SCALAR>
 cudaError_t launch_typed(const gdr_prefill_args& a, uint8_t* records, uint32_t* err,
                          cudaStream_t st) {
@@ -935,10 +990,23 @@ cudaError_t launch_typed(const gdr_prefill_args& a, uint8_t* records, uint32_t* 
         cached_dev = dev;
     }
     const int64_t n_items = n_chunk_slots(a.total_tokens, a.n_seqs) * (int64_t)a.n_heads;
+    EncodeTiledFn enc = nullptr;
+    if ((e = tensor_map_encoder(&enc)) != cudaSuccess) return e;
+    InputMaps maps;
+    memset(&maps, 0, sizeof(maps));
+    const CUtensorMapDataType dt = sizeof(InT) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    if (IntraLayout<D, InT, SCALAR>::kStageQKV) {
+        if ((e = token_map(enc, &maps.q, a.q, dt, sizeof(InT), a.total_tokens, a.n_heads, D)) != cudaSuccess) return e;
+        if ((e = token_map(enc, &maps.k, a.k, dt, sizeof(InT), a.total_tokens, a.n_heads, D)) != cudaSuccess) return e;
+        if ((e = token_map(enc, &maps.v, a.v, dt, sizeof(InT), a.total_tokens, a.n_heads, D)) != cudaSuccess) return e;
+    }
+    if (!SCALAR &&
+        (e = token_map(enc, &maps.g, a.log_a, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.total_tokens, a.n_heads, D)) != cudaSuccess)
+        return e;
     const unsigned grid = (unsigned)(n_items < resident ? n_items : resident);
     kern<<<grid, kThreads, smem, st>>>(a.cu_seqlens, a.n_seqs, a.n_heads, (const InT*)a.q,
                                        (const InT*)a.k, (const InT*)a.v, a.beta, a.log_a, a.scale,
-                                       n_items, records, err);
+                                       n_items, records, err, maps);
     return cudaGetLastError();
 }
 
