@@ -48,7 +48,12 @@
 namespace gdr {
 namespace {
 
-constexpr int kThreads = 256;
+// Threads per CTA: 8 warps (two CTAs per SM at d 64); 16 for the scalar
+// decay at d 128 (one CTA per SM, whose phases then run twice as wide; the
+// per-channel kernel measured slower that way, its phases being bound by
+// shared memory rather than by issue).
+template <int D, bool SCALAR>
+__host__ __device__ constexpr int threads_for() { return (D == 128 && SCALAR) ? 512 : 256; }
 constexpr float kMaxFactorExp = 80.f;
 constexpr int kLd = 68;                       // row stride (floats) of the fp32 64x64 tiles
 
@@ -93,9 +98,10 @@ struct IntraLayout {
     // fp32 scan partials [1024 B], live only during the scan: in region 2
     // past the operands and the (possibly still draining) record when it fits
     static constexpr uint32_t free2 = umax(op_bytes, rec_bytes);
-    static constexpr bool kPtotInR2 = free2 + 1024u <= r2;
+    static constexpr uint32_t kPtotBytes = 4u * threads_for<D, SCALAR>();
+    static constexpr bool kPtotInR2 = free2 + kPtotBytes <= r2;
     static constexpr uint32_t Ptot = kPtotInR2 ? r1 + free2 : Gs + 256u;
-    static constexpr uint32_t bytes = Gs + 256u + (kPtotInR2 ? 0u : 1024u);
+    static constexpr uint32_t bytes = Gs + 256u + (kPtotInR2 ? 0u : kPtotBytes);
     // at d 128 the 512 TMEM columns of a CTA allow one CTA per SM: request
     // enough shared memory that a second one is never scheduled
     static constexpr uint32_t dyn_bytes = (D == 128) ? umax(bytes + 1024u, 118784u) : bytes + 1024u;
@@ -290,7 +296,7 @@ __device__ __forceinline__ void load_ap_row(uint32_t taddr, int b, float (&v)[64
 }
 
 template <int D, typename InT, bool SCALAR>
-__global__ void __launch_bounds__(kThreads, (D == 64) ? 2 : 1)
+__global__ void __launch_bounds__(threads_for<D, SCALAR>(), (D == 64) ? 2 : 1)
 intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                    const InT* __restrict__ q, const InT* __restrict__ k, const InT* __restrict__ v,
                    const float* __restrict__ beta, const float* __restrict__ log_a, float scale,
@@ -299,7 +305,9 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     using L = IntraLayout<D, InT, SCALAR>;
     constexpr RecordLayout R = record_layout(D);
     constexpr int CG = D / 8;              // channel groups of 8
-    constexpr int RG = kThreads / CG;      // row groups
+    constexpr int NT = threads_for<D, SCALAR>();
+    constexpr int NG = NT / 128;           // warp groups; warps w, w + 4, ... share TMEM lanes
+    constexpr int RG = NT / CG;            // row groups
     constexpr int RPT = 64 / RG;           // rows per thread: 2 (D=64) or 4 (D=128)
     constexpr uint32_t kTmemCols = (D == 64) ? 256u : 512u;
     extern __shared__ uint8_t smem_raw[];
@@ -307,7 +315,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     __shared__ uint64_t mma_bar;
     __shared__ uint64_t in_bar[2];          // inputs landed: log a, q/k/v
     __shared__ uint32_t tmem_slot;
-    __shared__ Item s_next;                 // the item after the current one
+    __shared__ Item s_item[2];              // the next two items, by iteration parity
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const size_t tok_stride = (size_t)H * D;
@@ -319,7 +327,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     float* Gs = reinterpret_cast<float*>(sm + L::Gs);
     float* sG = reinterpret_cast<float*>(sm + L::sG);
 
-    constexpr int kLoadWarp = kThreads / 32 - 1;              // issues the input copies
+    constexpr int kLoadWarp = NT / 32 - 1;                    // issues the input copies
     if (tid == 0) {
         mbar_init(&mma_bar, 1);
         mbar_init(&in_bar[0], 1);
@@ -332,6 +340,10 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     // item's inputs are staged while the current one is finished, and each
     // record's bulk store drains while the next item starts.
     Item cur = find_item(cu, n_seqs, H, n_items, blockIdx.x);
+    if (tid == 0) {
+        s_item[1] = cur.idx >= 0 ? find_item(cu, n_seqs, H, n_items, cur.idx + gridDim.x) : cur;
+        s_item[0] = s_item[1];
+    }
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
@@ -339,13 +351,13 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         issue_inputs<D, InT, SCALAR, L>(sm, &in_bar[0], &in_bar[1], maps, beta, log_a, H, cur, lane);
     const uint32_t tmem = tmem_slot;
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-    const int whalf = warp >> 2;                              // warps w and w+4 share TMEM lanes
+    const int wgrp = warp >> 2;                               // warp group (0 .. NG - 1)
     uint32_t phase = 0;                                       // parity of the next MMA commit
     uint32_t in_phase = 0;                                    // parity of the inputs' barriers
+    int iter = 0;                                             // item n: s_item[(n+1)&1] = item n+1
     bool failed = false;
 
     while (cur.idx >= 0) {
-    if (tid == 0) s_next = find_item(cu, n_seqs, H, n_items, cur.idx + gridDim.x);
     const int h = cur.h, start = cur.start, len = cur.len;
     uint8_t* rec = records + (size_t)cur.idx * R.bytes;       // item = slot * H + h
     const size_t base = (size_t)start * tok_stride + (size_t)h * D;
@@ -369,7 +381,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     // in some channel takes the exact path.
     bool bad = false;
     if (!SCALAR) {
-        constexpr int P = kThreads / D, RP = 64 / P;          // row parts per channel
+        constexpr int P = NT / D, RP = 64 / P;                // row parts per channel
         float* Ptot = reinterpret_cast<float*>(sm + L::Ptot);
         const int c = tid % D, part = tid / D;
         float run = 0.f;
@@ -605,32 +617,40 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     tc_fence_after_sync();
 
     // ---- P (masked, bf16 operand) and A (masked, times beta, fp32) ----------
-    // warps w and w+4 read the same rows; each writes one half of the columns
+    // the NG warps on the same TMEM lanes read the same rows; each writes
+    // 64 / NG of the columns
     {
-        const int sub = warp & 3, ch = warp >> 2;
+        constexpr int CWc = 64 / NG;                          // columns per warp group
+        const int sub = warp & 3;
         const bool is_p = sub < 2;
         const int rr = 32 * (sub & 1) + lane;                 // chunk row
         const int lim = is_p ? rr : rr - 1;                   // last valid key index
-        const int i0 = 32 * ch;                               // first column of this half
-        float v32[32];
+        const int i0 = CWc * wgrp;                            // first column of this group
+        float v32[CWc];
         if (!SCALAR) {
             float vrow[64];
             if ((sub & 1) == 0) load_ap_row<0>(tmem + lane_base, rr >> 4, vrow);
             else load_ap_row<1>(tmem + lane_base, rr >> 4, vrow);
 #pragma unroll
-            for (int il = 0; il < 32; ++il) v32[il] = ch ? vrow[32 + il] : vrow[il];
+            for (int il = 0; il < CWc; ++il) {
+                float x = vrow[il];
+#pragma unroll
+                for (int g = 1; g < NG; ++g) x = (wgrp == g) ? vrow[CWc * g + il] : x;
+                v32[il] = x;
+            }
         } else {
-            tmem_ld32(tmem + lane_base + (uint32_t)i0, v32);
+            if constexpr (CWc == 32) tmem_ld32(tmem + lane_base + (uint32_t)i0, v32);
+            else tmem_ld16(tmem + lane_base + (uint32_t)i0, v32);
             tmem_ld_wait();
             const float gr = Gs[rr];
 #pragma unroll
-            for (int il = 0; il < 32; ++il)
+            for (int il = 0; il < CWc; ++il)
                 v32[il] = (i0 + il <= lim) ? v32[il] * __expf(gr - Gs[i0 + il]) : 0.f;
         }
         if (!SCALAR && bad_chunk) {
             // exact path: every term with its own exp (chunks with extreme decay only)
 #pragma unroll
-            for (int il = 0; il < 32; ++il) {
+            for (int il = 0; il < CWc; ++il) {
                 const int i = i0 + il;
                 float acc = 0.f;
                 if (i <= lim && rr < len) {
@@ -646,16 +666,16 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         }
         if (is_p) {
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
+            for (int jj = 0; jj < CWc / 8; ++jj) {
                 float x[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) x[e] = (i0 + 8 * jj + e <= lim) ? v32[8 * jj + e] : 0.f;
-                *reinterpret_cast<uint4*>(sm + L::Pt + sw128_chunk(64, rr, 4 * ch + jj)) = pack8(x);
+                *reinterpret_cast<uint4*>(sm + L::Pt + sw128_chunk(64, rr, i0 / 8 + jj)) = pack8(x);
             }
         } else {
             const float br = Bs[rr];
 #pragma unroll
-            for (int i4 = 0; i4 < 8; ++i4) {
+            for (int i4 = 0; i4 < CWc / 4; ++i4) {
                 const int i = i0 + 4 * i4;
                 float4 x;
                 x.x = (i + 0 <= lim) ? br * v32[4 * i4 + 0] : 0.f;
@@ -669,11 +689,14 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     __syncthreads();
 
     // region 1 and beta are free: stage the next item's inputs
+    // and look up the item after it (read by every thread at this item's end)
     if (warp == kLoadWarp) {
-        const Item nxt = s_next;
+        const Item nxt = s_item[(iter + 1) & 1];
         fence_proxy_async_smem();             // this item's reads of region 1 come first
         if (nxt.idx >= 0)
             issue_inputs<D, InT, SCALAR, L>(sm, &in_bar[0], &in_bar[1], maps, beta, log_a, H, nxt, lane);
+        if (lane == 0)
+            s_item[iter & 1] = nxt.idx >= 0 ? find_item(cu, n_seqs, H, n_items, nxt.idx + gridDim.x) : nxt;
     }
 
     // ---- T = (I + A)^-1: 16x16 diagonal blocks, then block merges -----------
@@ -682,7 +705,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     // copy straight into the operand tile Tb, whose blocks above the
     // diagonal are zeroed here.
     uint8_t* Tb = sm + L::Tb;
-    if (tid >= 64) {
+    if (tid >= 64 && tid < 256) {
         // (row, chunk) pairs of the zero blocks (b, j > b): 96 + 64 + 32
         const int z = tid - 64;
         int r, jj;
@@ -777,13 +800,14 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     {
         uint8_t* WUt = sm + L::WUt;
         const int lrow = 32 * (warp & 3) + lane;
+        // (part, piece) = (128-row part, 32-column piece), dealt round-robin
+        // to the warp groups
 #pragma unroll
         for (int part = 0; part < 2 * D / 128; ++part) {
-            if (D == 128 && part != whalf) continue;
-            const int row = (D == 64) ? lrow : (lrow + 128 * part);
+            const int row = lrow + 128 * part;
 #pragma unroll
             for (int piece = 0; piece < 2; ++piece) {
-                if (D == 64 && piece != whalf) continue;
+                if ((2 * part + piece) % NG != wgrp) continue;
                 float x[32];
                 tmem_ld32(tmem + lane_base + 64 * part + 32 * piece, x);
                 tmem_ld_wait();
@@ -830,7 +854,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         const bool act64 = lane < 16;
 #pragma unroll
         for (int piece = 0; piece < D / 32; ++piece) {
-            if ((piece & 1) != whalf) continue;
+            if (piece % NG != wgrp) continue;
             float pw[32], pu[32];
             tmem_ld32(tmem + lane_base + 32 * piece, pw);
             tmem_ld32(tmem + lane_base + D + 32 * piece, pu);
@@ -853,7 +877,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         const bool actD = (D == 128) || act64;
 #pragma unroll
         for (int piece = 0; piece < D / 32; ++piece) {
-            if ((piece & 1) != whalf) continue;
+            if (piece % NG != wgrp) continue;
             float bs[32], nc[32];
             tmem_ld32(tmem + lane_base + 2 * D + 32 * piece, bs);
             tmem_ld32(tmem + lane_base + 3 * D + 32 * piece, nc);
@@ -872,7 +896,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         }
         if (tid < D) reinterpret_cast<float*>(srec + R.gamma)[tid] = expf(Gl[tid]);
     }
-    const Item nxt = s_next;                  // read before thread 0 may overwrite it
+    const Item nxt = s_item[(iter + 1) & 1];  // read before the loader may overwrite it
     fence_proxy_async_smem();
     tc_fence_before_sync();
     failed = __syncthreads_or(failed);
@@ -882,8 +906,9 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         bulk_commit_group();
         if (failed) atomicOr(err, 1u);
     }
-    if (failed) break;                        // a timed-out MMA: stop issuing work                        // a timed-out MMA: stop issuing work
+    if (failed) break;                        // a timed-out MMA: stop issuing work
     cur = nxt;
+    ++iter;
     }
 
     cp_async_wait_all();
@@ -982,7 +1007,7 @@ cudaError_t launch_typed(const gdr_prefill_args& a, uint8_t* records, uint32_t* 
         if ((e = cudaDeviceGetAttribute(&rsv, cudaDevAttrReservedSharedMemoryPerBlock, dev)) != cudaSuccess) return e;
         if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess) return e;
         const int cta_smem = ((int)(smem + fa.sharedSizeBytes) + rsv + 127) & ~127;
-        const int cta_regs = ((fa.numRegs + 7) & ~7) * kThreads;
+        const int cta_regs = ((fa.numRegs + 7) & ~7) * threads_for<D, SCALAR>();
         int per_sm = smem_sm / cta_smem;
         per_sm = per_sm < 65536 / cta_regs ? per_sm : 65536 / cta_regs;
         per_sm = per_sm < 2 ? per_sm : 2;
@@ -1004,7 +1029,7 @@ cudaError_t launch_typed(const gdr_prefill_args& a, uint8_t* records, uint32_t* 
         (e = token_map(enc, &maps.g, a.log_a, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.total_tokens, a.n_heads, D)) != cudaSuccess)
         return e;
     const unsigned grid = (unsigned)(n_items < resident ? n_items : resident);
-    kern<<<grid, kThreads, smem, st>>>(a.cu_seqlens, a.n_seqs, a.n_heads, (const InT*)a.q,
+    kern<<<grid, threads_for<D, SCALAR>(), smem, st>>>(a.cu_seqlens, a.n_seqs, a.n_heads, (const InT*)a.q,
                                        (const InT*)a.k, (const InT*)a.v, a.beta, a.log_a, a.scale,
                                        n_items, records, err, maps);
     return cudaGetLastError();
