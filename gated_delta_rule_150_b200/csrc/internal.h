@@ -27,22 +27,28 @@ inline int64_t n_chunk_slots(int64_t total_tokens, int n_seqs) {
 // Qt and BS are tensor-core operand tiles (K-major, 128-byte swizzle, see
 // sm100.cuh); PU and NC are read row by row by threads (same swizzle of their
 // 16-byte chunks, so rows read without bank conflicts).
+// The parts the state-only pass needs (BS, NC) come first and everything the
+// pass reads is one contiguous span (`used` bytes), fetched by one bulk copy:
+// a CTA's bulk copies are served one after another, so their number, not
+// their size, sets the fetch time of a small record.
 struct RecordLayout {
-    uint32_t Qt;      // [64 x D]  row r: scale q_r exp(g_r) - (P W)_r        (bf16)
     uint32_t BS;      // [D x D]   row c': -(Kd^T W)[c', :]                    (bf16)
-    uint32_t PU;      // [64 x D]  row r: (P U)_r                              (bf16)
     uint32_t NC;      // [D x D]   row v: (U^T Kd)[v, :]                       (bf16)
+    uint32_t Qt;      // [64 x D]  row r: scale q_r exp(g_r) - (P W)_r        (bf16)
+    uint32_t PU;      // [64 x D]  row r: (P U)_r                              (bf16)
     uint32_t gamma;   // [D]       exp(g_last)                                 (fp32)
-    uint32_t bytes;   // total, a multiple of 256
+    uint32_t used;    // bytes up to the end of gamma (a multiple of 16)
+    uint32_t bytes;   // slot size, a multiple of 1024 (tile alignment)
 };
 
 __host__ __device__ constexpr RecordLayout record_layout(int D) {
     return RecordLayout{0u,
-                        (uint32_t)(128 * D),
-                        (uint32_t)(128 * D + 2 * D * D),
-                        (uint32_t)(256 * D + 2 * D * D),
-                        (uint32_t)(256 * D + 4 * D * D),
-                        (uint32_t)(((256 * D + 4 * D * D + 4 * D) + 255) / 256 * 256)};
+                        (uint32_t)(2 * D * D),
+                        (uint32_t)(4 * D * D),
+                        (uint32_t)(4 * D * D + 128 * D),
+                        (uint32_t)(4 * D * D + 256 * D),
+                        (uint32_t)(4 * D * D + 256 * D + 4 * D),
+                        (uint32_t)(((4 * D * D + 256 * D + 4 * D) + 1023) / 1024 * 1024)};
 }
 
 // Sequence segmentation of the sequential pass.  With few (sequence, head)

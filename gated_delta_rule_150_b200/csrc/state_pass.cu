@@ -54,21 +54,22 @@ template <> struct Out8<__nv_bfloat16> {
 
 template <int D, int MODE>
 struct PassLayout {
+    static constexpr RecordLayout R = record_layout(D);
     static constexpr bool kOut = MODE != kLocal;
     static constexpr int kStages = (D == 64) ? 3 : 2;
     // rows of the bf16 state operand: S (and the identity-started X rows in kLocal)
     static constexpr int kRows = (MODE == kLocal) ? 2 * D : D;
-    // tensor-core operand tiles, 1024-byte aligned
-    static constexpr uint32_t QtS = 0;                                      // kStages x [64 x D]
-    static constexpr uint32_t BSS = QtS + (kOut ? kStages * 128u * D : 0u); // kStages x [D x D]
-    static constexpr uint32_t S = BSS + kStages * 2u * D * D;               // bf16 [kRows x D]
-    // thread-read parts of the records
-    static constexpr uint32_t PUS = S + 2u * kRows * D;                     // kStages x [64 x D]
-    static constexpr uint32_t NCS = PUS + (kOut ? kStages * 128u * D : 0u); // kStages x [D x D]
-    static constexpr uint32_t GAS = NCS + kStages * 2u * D * D;             // kStages x [D] fp32
-    static constexpr uint32_t bytes = GAS + kStages * 4u * D;
+    static constexpr uint32_t S = 0;                                        // bf16 [kRows x D]
+    // kStages record images, 1024-byte aligned, at the record's own offsets:
+    // the whole record with outputs (one bulk copy); BS, NC and then gamma
+    // (two copies) without
+    static constexpr uint32_t Rec0 = S + 2u * kRows * D;
+    static constexpr uint32_t kGamma = kOut ? R.gamma : 4u * D * D;         // gamma in a stage
+    static constexpr uint32_t kStride = kOut ? R.bytes : 4u * D * D + 1024u;
+    static constexpr uint32_t bytes = Rec0 + (kStages - 1) * kStride + kGamma + 4u * D;
     static constexpr uint32_t dyn_bytes = bytes + 1024u;
-    static constexpr uint32_t tx_bytes = (kOut ? 256u * D : 0u) + 4u * D * D + 4u * D;
+    static constexpr uint32_t tx_bytes = kOut ? R.used : 4u * D * D + 4u * D;
+    static_assert(kStride % 1024u == 0u && Rec0 % 1024u == 0u, "tile alignment");
     static_assert(dyn_bytes + 128u <= 232448u, "shared memory budget");
 };
 
@@ -126,11 +127,34 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     const int orow = 16 * sub + lane;
     const bool oactive = lane < 16;
 
+    auto record_of = [&](int c) -> const uint8_t* {
+        const int64_t slot = (int64_t)(seg_start / kChunk) + chunk0 + c + n;
+        return records + ((size_t)slot * H + h) * R.bytes;
+    };
+    auto stage = [&](int s) { return sm + L::Rec0 + (uint32_t)s * L::kStride; };
+    // A CTA's bulk copies are served one after another and their issue can
+    // block for a while: one copy per record, issued where thread 0 has slack.
+    auto issue_copy = [&](int c) {       // thread 0 only
+        const int s = c % ST;
+        const uint8_t* r = record_of(c);
+        mbar_arrive_expect_tx(&full[s], L::tx_bytes);
+        if (kOut) {
+            bulk_g2s(stage(s), r, R.used, &full[s]);
+        } else {
+            bulk_g2s(stage(s) + R.BS, r + R.BS, 4u * D * D, &full[s]);     // BS and NC
+            bulk_g2s(stage(s) + L::kGamma, r + R.gamma, 4u * D, &full[s]);
+        }
+    };
+
+    int copies_issued = 0;                                          // thread 0's bookkeeping
     if (tid == 0) {
 #pragma unroll
         for (int s = 0; s < ST; ++s) mbar_init(&full[s], 1);
         mbar_init(&mma_bar, 1);
         fence_mbar_init();
+        // the first records start arriving while the initial state is loaded
+        for (int c = 0; c < ST && c < nchunks; ++c) issue_copy(c);
+        copies_issued = min(ST, nchunks);
     }
     if (warp == 0) {
         tmem_alloc(&tmem_slot, kTmemCols);
@@ -193,28 +217,12 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     const uint32_t lane_base = (uint32_t)(32 * sub) << 16;
     const int64_t snap_base = snap_base_s;
 
-    auto record_of = [&](int c) -> const uint8_t* {
-        const int64_t slot = (int64_t)(seg_start / kChunk) + chunk0 + c + n;
-        return records + ((size_t)slot * H + h) * R.bytes;
-    };
-    auto issue_copy = [&](int c) {       // thread 0 only
-        const int s = c % ST;
-        const uint8_t* r = record_of(c);
-        mbar_arrive_expect_tx(&full[s], L::tx_bytes);
-        if (kOut) {
-            bulk_g2s(sm + L::QtS + s * 128u * D, r + R.Qt, 128u * D, &full[s]);
-            bulk_g2s(sm + L::PUS + s * 128u * D, r + R.PU, 128u * D, &full[s]);
-        }
-        bulk_g2s(sm + L::BSS + s * 2u * D * D, r + R.BS, 2u * D * D, &full[s]);
-        bulk_g2s(sm + L::NCS + s * 2u * D * D, r + R.NC, 2u * D * D, &full[s]);
-        bulk_g2s(sm + L::GAS + s * 4u * D, r + R.gamma, 4u * D, &full[s]);
-    };
     const uint32_t id_z = idesc_bf16_f32(kMS, D);
     const uint32_t id_o = idesc_bf16_f32(64, D);
     const uint32_t aS = smem_u32(sS);
     auto issue_mma = [&](int c) {        // thread 0 only; operands of chunk c are resident
         const int s = c % ST;
-        const uint32_t aBS = smem_u32(sm + L::BSS + s * 2u * D * D);
+        const uint32_t aBS = smem_u32(stage(s) + R.BS);
         tc_fence_after_sync();
 #pragma unroll
         for (int t = 0; t < kNT; ++t)
@@ -223,7 +231,7 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                 mma_bf16(tmem + (uint32_t)(t * 128), sw128_desc(aS, L::kRows, t * 128, 16 * kk),
                          sw128_desc(aBS, D, 0, 16 * kk), id_z, kk > 0);
         if (kOut) {
-            const uint32_t aQt = smem_u32(sm + L::QtS + s * 128u * D);
+            const uint32_t aQt = smem_u32(stage(s) + R.Qt);
             const uint32_t o_col = (uint32_t)D * (1 + (c & 1));
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk)
@@ -234,10 +242,8 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     };
 
     bool failed = false;
-    int copies_issued = 0, copies_waited = 0, mmas_issued = 0;     // thread 0's bookkeeping
+    int copies_waited = 0, mmas_issued = 0;                         // thread 0's bookkeeping
     if (tid == 0 && nchunks > 0) {
-        for (int c = 0; c < ST && c < nchunks; ++c) issue_copy(c);
-        copies_issued = min(ST, nchunks);
         if (!mbar_wait(&full[0], 0)) failed = true;
         copies_waited = 1;
         issue_mma(0);
@@ -250,8 +256,8 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         const int t0 = s0 + k * kChunk;
         const int len = min(kChunk, s1 - t0);
         if (!mbar_wait(&full[st], (uint32_t)(k / ST) & 1)) failed = true;
-        const float* gam = reinterpret_cast<const float*>(sm + L::GAS + st * 4u * D);
-        const uint8_t* nc = sm + L::NCS + st * 2u * D * D;
+        const float* gam = reinterpret_cast<const float*>(stage(st) + L::kGamma);
+        const uint8_t* nc = stage(st) + R.NC;
         // gamma and this row's NC, read while the MMAs of chunk k finish
         constexpr bool kPre = (kNT == 1);
         float gv[kPre ? CW : 1];
@@ -323,6 +329,18 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                 }
             }
         }
+        // this chunk's outputs Qt S0^T, read before the next chunk's MMAs are
+        // issued: a tensor-memory load behind running MMAs waits for them (at
+        // d 64 the registers are short, and the outputs are read after issue)
+        constexpr bool kOEarly = kOut && D == 128;
+        float ov[kOut ? CW : 1];
+        if (kOEarly) {
+            const uint32_t o_col = (uint32_t)D * (1 + (k & 1));
+#pragma unroll
+            for (int p = 0; p < CW / 16; ++p)
+                tmem_ld16(tmem + lane_base + o_col + cb + 16 * p, *reinterpret_cast<float(*)[16]>(ov + 16 * p));
+            tmem_ld_wait();
+        }
         fence_proxy_async_smem();
         tc_fence_before_sync();
         if (__syncthreads_or(failed)) { failed = true; break; }
@@ -332,6 +350,13 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
             copies_waited = k + 2;
             issue_mma(k + 1);
             mmas_issued = k + 2;
+        }
+        // with three or more stages, chunk k-1's stage (free since the last
+        // barrier, its reads fenced before it) takes record k-1+ST now, under
+        // the MMAs just issued
+        if (ST >= 3 && tid == 0 && k >= 1 && k - 1 + ST < nchunks) {
+            issue_copy(k - 1 + ST);
+            copies_issued = k + ST;
         }
 
         if (kOut) {
@@ -344,14 +369,16 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                 for (int j = 0; j < CW; j += 4)
                     *reinterpret_cast<float4*>(dst + j) = make_float4(S[0][j], S[0][j + 1], S[0][j + 2], S[0][j + 3]);
             }
-            const uint8_t* pu = sm + L::PUS + st * 128u * D;
+            const uint8_t* pu = stage(st) + R.PU;
             OutT* orow_ptr = o + ((size_t)(t0 + orow) * H + h) * D + cb;
-            const uint32_t o_col = (uint32_t)D * (1 + (k & 1));
 #pragma unroll
             for (int p = 0; p < CW / 16; ++p) {
-                float y[16];
-                tmem_ld16(tmem + lane_base + o_col + cb + 16 * p, y);
-                tmem_ld_wait();
+                const float* y = ov + 16 * p;
+                if (!kOEarly) {
+                    tmem_ld16(tmem + lane_base + (uint32_t)D * (1 + (k & 1)) + cb + 16 * p,
+                              *reinterpret_cast<float(*)[16]>(ov + 16 * p));
+                    tmem_ld_wait();
+                }
                 if (oactive && orow < len) {
 #pragma unroll
                     for (int jj = 0; jj < 2; ++jj) {
@@ -368,9 +395,10 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                 }
             }
         }
+        if (ST < 3) fence_proxy_async_smem();   // reads of this stage, then its refill
         tc_fence_before_sync();
         if (__syncthreads_or(failed)) { failed = true; break; }
-        if (tid == 0 && k + ST < nchunks) {
+        if (ST < 3 && tid == 0 && k + ST < nchunks) {
             issue_copy(k + ST);
             copies_issued = k + ST + 1;
         }
