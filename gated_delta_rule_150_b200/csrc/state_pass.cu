@@ -435,21 +435,24 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
 //     E_0 = init,   E_{s+1} = E_s M_s + N_s       (fp32, in the chain's order)
 // Rows of the state are independent, so a CTA owns kCombineRows state rows of
 // one (sequence, head); thread (j, q) computes row j, columns 4q .. 4q+3.  Each
-// step's M_s and the CTA's rows of N_s arrive by bulk copies one step ahead
-// (two buffers).  E_s goes to the workspace of segment s (its start state); the
-// last segment's own map is not needed (replaying that segment produces the
-// final state).  An empty sequence has no segment: its final state is its
-// initial state.
+// step's M_s and the CTA's rows of N_s are fetched kCombineBufs - 1 steps
+// ahead by 16-byte cp.async from every thread (a CTA's bulk copies would be
+// served one after another, one chain step each); E is double buffered, so a
+// step needs one barrier.  E_s goes to the workspace of segment s (its start
+// state); the last segment's own map is not needed (replaying that segment
+// produces the final state).  An empty sequence has no segment: its final
+// state is its initial state.
 constexpr int kCombineRows = 8;
 
 constexpr int kCombineBufs = 3;
 
 template <int D>
 struct CombineLayout {
+    static constexpr int kLdE = D + 4;                                  // padded E rows
     static constexpr uint32_t M0 = 0;                                   // bufs x [D x D] fp32
     static constexpr uint32_t N0 = kCombineBufs * D * D * 4u;           // bufs x [rows x D] fp32
-    static constexpr uint32_t E = N0 + kCombineBufs * kCombineRows * D * 4u;   // [rows x D] fp32
-    static constexpr uint32_t bytes = E + kCombineRows * D * 4u;
+    static constexpr uint32_t E = N0 + kCombineBufs * kCombineRows * D * 4u;   // 2 x [rows x kLdE]
+    static constexpr uint32_t bytes = E + 2u * kCombineRows * kLdE * 4u;
     static constexpr uint32_t dyn_bytes = bytes + 128u;
 };
 
@@ -460,10 +463,10 @@ combine_kernel(const int32_t* __restrict__ cu, int H, int seg_chunks, const floa
     using L = CombineLayout<D>;
     constexpr int RB = kCombineRows;
     constexpr int QD = D / 4;
+    constexpr int NT = RB * QD;                                         // threads
+    constexpr int NB = kCombineBufs;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align_smem<128>(smem_raw);
-    constexpr int NB = kCombineBufs;
-    __shared__ uint64_t full[NB];
     const int pair = blockIdx.x, rb = blockIdx.y;
     const int n = pair / H, h = pair % H;
     const int tid = threadIdx.x, j = tid / QD, q = tid % QD;
@@ -472,6 +475,7 @@ combine_kernel(const int32_t* __restrict__ cu, int H, int seg_chunks, const floa
     const int nseg = (s1 - s0 + span - 1) / span;
     const size_t state_off = ((size_t)n * H + h) * D * D;
     const size_t row_off = (size_t)(rb * RB + j) * D + 4 * q;
+    (void)err;
     if (nseg == 0) {
         float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
         if (init_state) x = *reinterpret_cast<const float4*>(init_state + state_off + row_off);
@@ -482,56 +486,51 @@ combine_kernel(const int32_t* __restrict__ cu, int H, int seg_chunks, const floa
     const int64_t slot0 = (int64_t)(s0 / span) + n;
     float* e = reinterpret_cast<float*>(sm + L::E);
     auto seg_ptr = [&](int s) { return seg_ws + ((size_t)(slot0 + s) * H + h) * 3u * D * D; };
-    auto issue = [&](int s) {      // thread 0: M_s and this CTA's rows of N_s
+    auto issue = [&](int s) {      // every thread: its share of M_s and of this CTA's rows of N_s
         const int b = s % NB;
-        mbar_arrive_expect_tx(&full[b], (uint32_t)(D * D * 4 + RB * D * 4));
-        bulk_g2s(sm + L::M0 + b * D * D * 4u, seg_ptr(s) + (size_t)D * D, D * D * 4u, &full[b]);
-        bulk_g2s(sm + L::N0 + b * RB * D * 4u, seg_ptr(s) + (size_t)rb * RB * D, RB * D * 4u, &full[b]);
-    };
-    if (tid == 0) {
+        const uint8_t* msrc = reinterpret_cast<const uint8_t*>(seg_ptr(s) + (size_t)D * D);
+        const uint8_t* nsrc = reinterpret_cast<const uint8_t*>(seg_ptr(s) + (size_t)rb * RB * D);
+        uint8_t* mdst = sm + L::M0 + b * D * D * 4u;
+        uint8_t* ndst = sm + L::N0 + b * RB * D * 4u;
 #pragma unroll
-        for (int b = 0; b < NB; ++b) mbar_init(&full[b], 1);
-        fence_mbar_init();
-    }
+        for (int c = tid; c < D * D / 4; c += NT) cp_async16(mdst + 16 * c, msrc + 16 * c, 16u);
+#pragma unroll
+        for (int c = tid; c < RB * D / 4; c += NT) cp_async16(ndst + 16 * c, nsrc + 16 * c, 16u);
+    };
     {
         float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
         if (init_state) x = *reinterpret_cast<const float4*>(init_state + state_off + row_off);
-        *reinterpret_cast<float4*>(e + j * D + 4 * q) = x;
+        *reinterpret_cast<float4*>(e + j * L::kLdE + 4 * q) = x;
     }
-    __syncthreads();
-    int issued = 0, consumed = 0;                  // thread 0's bookkeeping (steps)
-    if (tid == 0) {
-        for (int s = 0; s < NB && s <= nseg - 2; ++s) issue(s);
-        issued = min(NB, nseg - 1);
+    // steps 0 .. NB-2 in flight (one commit group per step, empty past the end)
+#pragma unroll
+    for (int s = 0; s < NB - 1; ++s) {
+        if (s <= nseg - 2) issue(s);
+        cp_async_commit();
     }
-    bool failed = false;
     for (int s = 0; s + 1 < nseg; ++s) {
+        cp_async_wait_group<NB - 2>();             // this thread's copies of step s
+        __syncthreads();                           // everyone's copies, E_s, buffer (s-1) free
+        if (s + NB - 1 <= nseg - 2) issue(s + NB - 1);
+        cp_async_commit();
         const int b = s % NB;
-        if (!mbar_wait(&full[b], (uint32_t)(s / NB) & 1)) failed = true;
-        consumed = s + 1;
         const float* Mm = reinterpret_cast<const float*>(sm + L::M0 + b * D * D * 4u);
         const float* Nm = reinterpret_cast<const float*>(sm + L::N0 + b * RB * D * 4u);
+        const float* ec = e + (s & 1) * RB * L::kLdE;
         float4 acc = *reinterpret_cast<const float4*>(Nm + j * D + 4 * q);
 #pragma unroll 8
         for (int k = 0; k < D; ++k) {
-            const float ek = e[j * D + k];
+            const float ek = ec[j * L::kLdE + k];
             const float4 m = *reinterpret_cast<const float4*>(Mm + k * D + 4 * q);
             acc.x = fmaf(ek, m.x, acc.x);
             acc.y = fmaf(ek, m.y, acc.y);
             acc.z = fmaf(ek, m.z, acc.z);
             acc.w = fmaf(ek, m.w, acc.w);
         }
-        if (__syncthreads_or(failed)) break;          // everyone is done with e and buffer b
-        *reinterpret_cast<float4*>(e + j * D + 4 * q) = acc;
+        *reinterpret_cast<float4*>(e + ((s + 1) & 1) * RB * L::kLdE + j * L::kLdE + 4 * q) = acc;
         *reinterpret_cast<float4*>(seg_ptr(s + 1) + 2u * D * D + row_off) = acc;
-        if (tid == 0 && s + NB <= nseg - 2) { issue(s + NB); issued = s + NB + 1; }
-        __syncthreads();
     }
-    if (failed && tid == 0) {
-        atomicOr(err, 1u);
-        // let the copies already issued land before the CTA exits (bounded waits)
-        for (int c = consumed; c < issued; ++c) mbar_wait(&full[c % NB], (uint32_t)(c / NB) & 1);
-    }
+    cp_async_wait_all();
 }
 
 template <int D, typename OutT, int MODE>
