@@ -337,7 +337,7 @@ def run_gdr(args):
 
     # ---- main workload: graft-layer prefill, 4 rotating input sets ----------
     n_sets = args.sets or (4 if args.workload != wl.VARLEN.name else 1)
-    ps = PrefillSets(gdr, wl.PREFILL_WORKLOADS[args.workload], n_sets, rank)
+    ps = PrefillSets(gdr, {**wl.PREFILL_WORKLOADS, **wl.PROFILE_CASES}[args.workload], n_sets, rank)
     for i in range(args.warmup):
         ps.step(i)
     torch.cuda.synchronize()
@@ -509,7 +509,8 @@ def main():
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     p.add_argument("--only-decode", action="store_true",
                    help="run only the decode measurement (for profiling)")
-    p.add_argument("--workload", default=wl.GRAFT_LAYER.name, choices=sorted(wl.PREFILL_WORKLOADS),
+    p.add_argument("--workload", default=wl.GRAFT_LAYER.name,
+                   choices=sorted(wl.PREFILL_WORKLOADS) + sorted(wl.PROFILE_CASES),
                    help="prefill workload of the main line (default: the graft layer)")
     p.add_argument("--sets", type=int, default=0,
                    help="rotating input sets of the main line (default 4; 1 for varlen)")

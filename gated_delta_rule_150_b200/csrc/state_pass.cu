@@ -434,7 +434,8 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
 // Chains the segments' affine maps into each segment's start state:
 //     E_0 = init,   E_{s+1} = E_s M_s + N_s       (fp32, in the chain's order)
 // Rows of the state are independent, so a CTA owns kCombineRows state rows of
-// one (sequence, head); thread (j, q) computes row j, columns 4q .. 4q+3.  Each
+// one (sequence, head); threads (j, q, kh) compute row j, columns 4q .. 4q+3,
+// over half kh of the inner dimension (the halves meet by a shuffle).  Each
 // step's M_s and the CTA's rows of N_s are fetched kCombineBufs - 1 steps
 // ahead by 16-byte cp.async from every thread (a CTA's bulk copies would be
 // served one after another, one chain step each); E is double buffered, so a
@@ -444,10 +445,13 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
 // state is its initial state.
 constexpr int kCombineRows = 8;
 
-constexpr int kCombineBufs = 3;
+// steps in flight: the chain step is short next to an L2 round trip
+template <int D>
+__host__ __device__ constexpr int combine_bufs() { return D == 64 ? 6 : 3; }
 
 template <int D>
 struct CombineLayout {
+    static constexpr int kCombineBufs = combine_bufs<D>();
     static constexpr int kLdE = D + 4;                                  // padded E rows
     static constexpr uint32_t M0 = 0;                                   // bufs x [D x D] fp32
     static constexpr uint32_t N0 = kCombineBufs * D * D * 4u;           // bufs x [rows x D] fp32
@@ -457,19 +461,21 @@ struct CombineLayout {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kCombineRows * D / 4)
+__global__ void __launch_bounds__(kCombineRows * D / 2)
 combine_kernel(const int32_t* __restrict__ cu, int H, int seg_chunks, const float* init_state,
                float* final_state, float* seg_ws, uint32_t* err) {
     using L = CombineLayout<D>;
     constexpr int RB = kCombineRows;
     constexpr int QD = D / 4;
-    constexpr int NT = RB * QD;                                         // threads
-    constexpr int NB = kCombineBufs;
+    constexpr int NT = RB * QD * 2;                                     // threads
+    constexpr int NB = L::kCombineBufs;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align_smem<128>(smem_raw);
     const int pair = blockIdx.x, rb = blockIdx.y;
     const int n = pair / H, h = pair % H;
-    const int tid = threadIdx.x, j = tid / QD, q = tid % QD;
+    // warp = (row j, 16 column groups); lane bit 4 = inner-dimension half kh
+    const int tid = threadIdx.x, lane = tid & 31, wq = tid >> 5;
+    const int j = wq / (QD / 16), q = 16 * (wq % (QD / 16)) + (lane & 15), kh = lane >> 4;
     const int s0 = __ldg(cu + n), s1 = __ldg(cu + n + 1);
     const int span = kChunk * seg_chunks;
     const int nseg = (s1 - s0 + span - 1) / span;
@@ -477,9 +483,11 @@ combine_kernel(const int32_t* __restrict__ cu, int H, int seg_chunks, const floa
     const size_t row_off = (size_t)(rb * RB + j) * D + 4 * q;
     (void)err;
     if (nseg == 0) {
-        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (init_state) x = *reinterpret_cast<const float4*>(init_state + state_off + row_off);
-        *reinterpret_cast<float4*>(final_state + state_off + row_off) = x;
+        if (kh == 0) {
+            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (init_state) x = *reinterpret_cast<const float4*>(init_state + state_off + row_off);
+            *reinterpret_cast<float4*>(final_state + state_off + row_off) = x;
+        }
         return;
     }
     if (nseg == 1) return;
@@ -497,7 +505,7 @@ combine_kernel(const int32_t* __restrict__ cu, int H, int seg_chunks, const floa
 #pragma unroll
         for (int c = tid; c < RB * D / 4; c += NT) cp_async16(ndst + 16 * c, nsrc + 16 * c, 16u);
     };
-    {
+    if (kh == 0) {
         float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
         if (init_state) x = *reinterpret_cast<const float4*>(init_state + state_off + row_off);
         *reinterpret_cast<float4*>(e + j * L::kLdE + 4 * q) = x;
@@ -517,18 +525,33 @@ combine_kernel(const int32_t* __restrict__ cu, int H, int seg_chunks, const floa
         const float* Mm = reinterpret_cast<const float*>(sm + L::M0 + b * D * D * 4u);
         const float* Nm = reinterpret_cast<const float*>(sm + L::N0 + b * RB * D * 4u);
         const float* ec = e + (s & 1) * RB * L::kLdE;
-        float4 acc = *reinterpret_cast<const float4*>(Nm + j * D + 4 * q);
-#pragma unroll 8
-        for (int k = 0; k < D; ++k) {
-            const float ek = ec[j * L::kLdE + k];
-            const float4 m = *reinterpret_cast<const float4*>(Mm + k * D + 4 * q);
-            acc.x = fmaf(ek, m.x, acc.x);
-            acc.y = fmaf(ek, m.y, acc.y);
-            acc.z = fmaf(ek, m.z, acc.z);
-            acc.w = fmaf(ek, m.w, acc.w);
+        float4 acc = kh == 0 ? *reinterpret_cast<const float4*>(Nm + j * D + 4 * q)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+        const int k0 = kh * (D / 2);
+#pragma unroll 2
+        for (int i = 0; i < D / 2; i += 4) {
+            // four inner steps per E load; the second half runs four steps
+            // rotated, so the two halves' E reads fall in different banks
+            const int k = k0 + ((i + 4 * kh) & (D / 2 - 1));
+            const float4 e4 = *reinterpret_cast<const float4*>(ec + j * L::kLdE + k);
+            const float ev[4] = {e4.x, e4.y, e4.z, e4.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float4 m = *reinterpret_cast<const float4*>(Mm + (k + u) * D + 4 * q);
+                acc.x = fmaf(ev[u], m.x, acc.x);
+                acc.y = fmaf(ev[u], m.y, acc.y);
+                acc.z = fmaf(ev[u], m.z, acc.z);
+                acc.w = fmaf(ev[u], m.w, acc.w);
+            }
         }
-        *reinterpret_cast<float4*>(e + ((s + 1) & 1) * RB * L::kLdE + j * L::kLdE + 4 * q) = acc;
-        *reinterpret_cast<float4*>(seg_ptr(s + 1) + 2u * D * D + row_off) = acc;
+        acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 16);
+        acc.y += __shfl_xor_sync(0xffffffffu, acc.y, 16);
+        acc.z += __shfl_xor_sync(0xffffffffu, acc.z, 16);
+        acc.w += __shfl_xor_sync(0xffffffffu, acc.w, 16);
+        if (kh == 0) {
+            *reinterpret_cast<float4*>(e + ((s + 1) & 1) * RB * L::kLdE + j * L::kLdE + 4 * q) = acc;
+            *reinterpret_cast<float4*>(seg_ptr(s + 1) + 2u * D * D + row_off) = acc;
+        }
     }
     cp_async_wait_all();
 }
@@ -560,7 +583,7 @@ cudaError_t launch_typed(const gdr_prefill_args& a, const uint8_t* records,
     e = cudaFuncSetAttribute(ck, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)CombineLayout<D>::dyn_bytes);
     if (e != cudaSuccess) return e;
-    ck<<<dim3((unsigned)a.n_seqs * (unsigned)a.n_heads, D / kCombineRows), kCombineRows * D / 4,
+    ck<<<dim3((unsigned)a.n_seqs * (unsigned)a.n_heads, D / kCombineRows), kCombineRows * D / 2,
          CombineLayout<D>::dyn_bytes, st>>>(a.cu_seqlens, a.n_heads, lay.seg_chunks, a.init_state,
                                            a.final_state, seg_ws, err);
     e = cudaGetLastError();

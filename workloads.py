@@ -80,6 +80,13 @@ VARLEN = PrefillWorkload("varlen_N32_H32_d128_L1024to16384", 1005, 32, 128, 128,
 
 PREFILL_WORKLOADS = {w.name: w for w in (TINY_KDA, GRAFT_LAYER, GDN_LONG, VARLEN)}
 
+# Smaller cases of the d 128 workloads (same distributions) for ncu captures,
+# which replay each captured launch many times: a few GB on the device at most.
+PROFILE_CASES = {w.name: w for w in (
+    replace(GDN_LONG, name="gdn_H16_T16384_d128_scalar", lengths=(16384,), snap_interval=0),
+    replace(VARLEN, name="varlen_N4_H32_d128_L1024to16384", n_seqs=4),
+)}
+
 
 def shrink(w: PrefillWorkload, **kw) -> PrefillWorkload:
     """Same distributions, other sizes (for fast parity cases)."""
