@@ -4,6 +4,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <utility>
 #include <cuda_runtime.h>
 
 #include "gdr.h"
@@ -58,6 +59,26 @@ __host__ __device__ constexpr RecordLayout record_layout(int D) {
 // S_end = S_start M + N), a short fp32 chain combines the maps into each
 // segment's true start state, and every segment then replays its chunks from
 // that state to produce its outputs.  seg_chunks == 0 means one pass.
+// Launch, with programmatic stream serialization when `early`: the kernel's
+// CTAs may then be scheduled while the previous kernel in the stream drains,
+// hiding the launch gap.  Every kernel launched here calls pdl_wait()
+// (sm100.cuh) before its first global memory access.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(bool early, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args&&... args) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = early ? 1 : 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 inline int segment_chunks(int n_seqs, int H, int64_t T, int D) {
     if (n_seqs <= 0 || T <= 0) return 0;
     const int64_t pairs = (int64_t)n_seqs * H;

@@ -335,6 +335,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         fence_mbar_init();
     }
     if (warp == 0) tmem_alloc(&tmem_slot, kTmemCols);
+    pdl_wait();                               // the previous kernel's memory is final
 
     // Persistent CTA: items blockIdx.x, blockIdx.x + gridDim.x, ...  The next
     // item's inputs are staged while the current one is finished, and each
@@ -911,6 +912,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     ++iter;
     }
 
+    pdl_launch_dependents();
     cp_async_wait_all();
     if (tid == 0) bulk_wait_group0();
     tc_fence_before_sync();
@@ -1029,10 +1031,9 @@ cudaError_t launch_typed(const gdr_prefill_args& a, uint8_t* records, uint32_t* 
         (e = token_map(enc, &maps.g, a.log_a, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.total_tokens, a.n_heads, D)) != cudaSuccess)
         return e;
     const unsigned grid = (unsigned)(n_items < resident ? n_items : resident);
-    kern<<<grid, threads_for<D, SCALAR>(), smem, st>>>(a.cu_seqlens, a.n_seqs, a.n_heads, (const InT*)a.q,
-                                       (const InT*)a.k, (const InT*)a.v, a.beta, a.log_a, a.scale,
-                                       n_items, records, err, maps);
-    return cudaGetLastError();
+    return launch_pdl(true, kern, dim3(grid), dim3(threads_for<D, SCALAR>()), smem, st, a.cu_seqlens,
+                      a.n_seqs, a.n_heads, (const InT*)a.q, (const InT*)a.k, (const InT*)a.v, a.beta,
+                      a.log_a, a.scale, n_items, records, err, maps);
 }
 
 template <int D, typename InT>

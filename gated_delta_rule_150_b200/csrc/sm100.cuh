@@ -151,6 +151,20 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while the previous kernel in the stream finishes;
+// pdl_wait() blocks until that kernel has completed and its memory is
+// visible (a no-op for an ordinary launch), so nothing before it may touch
+// global memory.  pdl_launch_dependents() lets the next kernel start once
+// every CTA of this one has called it or exited.
+__device__ __forceinline__ void pdl_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------
 // Tensor memory (TMEM)
 // ---------------------------------------------------------------------------

@@ -99,6 +99,7 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int sub = warp & 3, half = warp >> 2;
+    pdl_wait();                               // the previous kernel's memory is final
     int n, h, s0, s1, seg_start;
     if (MODE == kFull) {
         n = blockIdx.x / H;
@@ -404,6 +405,7 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         }
     }
 
+    pdl_launch_dependents();
     if (failed) {
         if (tid == 0) atomicOr(err, 1u);
     } else if (active) {
@@ -471,6 +473,7 @@ combine_kernel(const int32_t* __restrict__ cu, int H, int seg_chunks, const floa
     constexpr int NB = L::kCombineBufs;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align_smem<128>(smem_raw);
+    pdl_wait();                               // the previous kernel's memory is final
     const int pair = blockIdx.x, rb = blockIdx.y;
     const int n = pair / H, h = pair % H;
     // warp = (row j, 16 column groups); lane bit 4 = inner-dimension half kh
@@ -553,6 +556,7 @@ combine_kernel(const int32_t* __restrict__ cu, int H, int seg_chunks, const floa
             *reinterpret_cast<float4*>(seg_ptr(s + 1) + 2u * D * D + row_off) = acc;
         }
     }
+    pdl_launch_dependents();
     cp_async_wait_all();
 }
 
@@ -566,10 +570,11 @@ cudaError_t launch_mode(const gdr_prefill_args& a, const uint8_t* records,
     dim3 grid;
     if (MODE == kFull) grid = dim3((unsigned)a.n_seqs * (unsigned)a.n_heads);
     else grid = dim3((unsigned)lay.n_seg_slots, (unsigned)a.n_heads);
-    kern<<<grid, kThreads, smem, st>>>(a.cu_seqlens, a.n_seqs, a.n_heads, records, a.init_state,
-                                       static_cast<OutT*>(a.o), a.final_state, a.snap_interval,
-                                       a.snapshots, lay.seg_chunks, seg_ws, err);
-    return cudaGetLastError();
+    // early launch for the single pass only: the segmented kernels measured
+    // slower with it
+    return launch_pdl(MODE == kFull, kern, grid, dim3(kThreads), smem, st, a.cu_seqlens, a.n_seqs, a.n_heads,
+                      records, a.init_state, static_cast<OutT*>(a.o), a.final_state,
+                      a.snap_interval, a.snapshots, lay.seg_chunks, seg_ws, err);
 }
 
 template <int D, typename OutT>
@@ -583,10 +588,9 @@ cudaError_t launch_typed(const gdr_prefill_args& a, const uint8_t* records,
     e = cudaFuncSetAttribute(ck, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)CombineLayout<D>::dyn_bytes);
     if (e != cudaSuccess) return e;
-    ck<<<dim3((unsigned)a.n_seqs * (unsigned)a.n_heads, D / kCombineRows), kCombineRows * D / 2,
-         CombineLayout<D>::dyn_bytes, st>>>(a.cu_seqlens, a.n_heads, lay.seg_chunks, a.init_state,
-                                           a.final_state, seg_ws, err);
-    e = cudaGetLastError();
+    e = launch_pdl(false, ck, dim3((unsigned)a.n_seqs * (unsigned)a.n_heads, D / kCombineRows),
+                   dim3(kCombineRows * D / 2), CombineLayout<D>::dyn_bytes, st, a.cu_seqlens,
+                   a.n_heads, lay.seg_chunks, a.init_state, a.final_state, seg_ws, err);
     if (e != cudaSuccess) return e;
     return launch_mode<D, OutT, kApply>(a, records, lay, seg_ws, err, st);
 }
