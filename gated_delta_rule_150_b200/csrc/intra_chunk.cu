@@ -716,24 +716,21 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         *reinterpret_cast<uint4*>(Tb + sw128_chunk(64, r, jj)) = make_uint4(0u, 0u, 0u, 0u);
     }
     if (tid < 64) {
+        // column cc of T_bb, right-looking: once x_j is known it is folded
+        // into every later row's running sum, so each step waits on one FMA
         const int b = tid >> 4, cc = tid & 15, o = 16 * b;
-        float x[16];
+        float x[16], acc[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) acc[r] = 0.f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            x[j] = (j < cc) ? 0.f : ((j == cc) ? 1.f : -acc[j]);
+#pragma unroll
+            for (int r = j + 1; r < 16; ++r) acc[r] = fmaf(As[(o + r) * kLd + o + j], x[j], acc[r]);
+        }
+        __syncwarp();          // every lane has read A_bb before T_bb overwrites it
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
-            float ar[16];
-#pragma unroll
-            for (int i4 = 0; i4 < 4; ++i4) {
-                const float4 t = f4(As + (o + r) * kLd + o + 4 * i4);
-                ar[4 * i4] = t.x; ar[4 * i4 + 1] = t.y; ar[4 * i4 + 2] = t.z; ar[4 * i4 + 3] = t.w;
-            }
-            __syncwarp();      // row r of A_bb is read by all 16 lanes before T overwrites it
-            float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-            for (int i = 0; i < r; ++i) {
-                if (i & 1) a1 = fmaf(ar[i], x[i], a1);
-                else a0 = fmaf(ar[i], x[i], a0);
-            }
-            x[r] = (r < cc) ? 0.f : ((r == cc) ? 1.f : -(a0 + a1));
             As[(o + r) * kLd + o + cc] = x[r];
             *reinterpret_cast<__nv_bfloat16*>(Tb + sw128_offset(64, o + r, o + cc)) = __float2bfloat16_rn(x[r]);
         }

@@ -260,7 +260,8 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         const float* gam = reinterpret_cast<const float*>(stage(st) + L::kGamma);
         const uint8_t* nc = stage(st) + R.NC;
         // gamma and this row's NC, read while the MMAs of chunk k finish
-        constexpr bool kPre = (kNT == 1);
+        // (at d 64 with outputs the registers go to the early output read)
+        constexpr bool kPre = (kNT == 1) && !(kOut && D == 64);
         float gv[kPre ? CW : 1];
         uint32_t nvp[kPre ? CW / 2 : 1];
         if (kPre && active) {
@@ -331,9 +332,8 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
             }
         }
         // this chunk's outputs Qt S0^T, read before the next chunk's MMAs are
-        // issued: a tensor-memory load behind running MMAs waits for them (at
-        // d 64 the registers are short, and the outputs are read after issue)
-        constexpr bool kOEarly = kOut && D == 128;
+        // issued: a tensor-memory load behind running MMAs waits for them
+        constexpr bool kOEarly = kOut;
         float ov[kOut ? CW : 1];
         if (kOEarly) {
             const uint32_t o_col = (uint32_t)D * (1 + (k & 1));
