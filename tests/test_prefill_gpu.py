@@ -229,6 +229,24 @@ def test_split_prefill_equals_one_shot():
     assert rel_err(torch.cat([o1, o2]), o_full.cpu().double().numpy()) < TOL
 
 
+def test_chained_prefills_consume_previous_outputs():
+    """Two prefills back to back on one stream, no host sync between: the
+    second reads the first's o (as q and v) and final state (as its initial
+    state), the way stacked layers would.  Its kernels may be scheduled while
+    the first one drains, so this checks that they wait for its results."""
+    gdr = _gdr()
+    w = wl.shrink(wl.GRAFT_LAYER, n_heads=4, lengths=(700, 300))
+    inp = wl.make_prefill_inputs(w)
+    d = _to(inp, "cuda")
+    o1, f1, _ = gdr.prefill(d["q"], d["k"], d["v"], d["beta"], d["log_a"], d["cu_seqlens"])
+    o2, f2, _ = gdr.prefill(o1, d["k"], o1, d["beta"], d["log_a"], d["cu_seqlens"], init_state=f1)
+    torch.cuda.synchronize()
+    ref = oracle.prefill(o1.cpu(), inp["k"], o1.cpu(), inp["beta"], inp["log_a"], inp["cu_seqlens"],
+                         init_state=f1.cpu())
+    assert_close_rel(o2, ref["o"], TOL, "chained o")
+    assert_close_rel(f2, ref["final_state"], TOL, "chained final")
+
+
 def test_decode_steps_continue_prefill():
     """Decode steps after a prefill equal a longer prefill (same recurrence)."""
     gdr = _gdr()
