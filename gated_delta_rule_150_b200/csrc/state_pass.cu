@@ -436,16 +436,20 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
 // Chains the segments' affine maps into each segment's start state:
 //     E_0 = init,   E_{s+1} = E_s M_s + N_s       (fp32, in the chain's order)
 // Rows of the state are independent, so a CTA owns kCombineRows state rows of
-// one (sequence, head); threads (j, q, kh) compute row j, columns 4q .. 4q+3,
-// over half kh of the inner dimension (the halves meet by a shuffle).  Each
-// step's M_s and the CTA's rows of N_s are fetched kCombineBufs - 1 steps
-// ahead by 16-byte cp.async from every thread (a CTA's bulk copies would be
-// served one after another, one chain step each); E is double buffered, so a
-// step needs one barrier.  E_s goes to the workspace of segment s (its start
-// state); the last segment's own map is not needed (replaying that segment
-// produces the final state).  An empty sequence has no segment: its final
-// state is its initial state.
+// one (sequence, head).  Warp w owns the column slab [w D/8, (w+1) D/8) for
+// all of the CTA's rows, so each step reads M_s from shared memory once per
+// CTA: lane (j = lane % 8, kq = lane / 8) sums row j over the inner indices
+// k = 4i + kq, and the four partial sums meet by shuffles.  Each step's M_s
+// (rows padded so the four k of one load fall in different banks) and the
+// CTA's rows of N_s are fetched kCombineBufs - 1 steps ahead by 16-byte
+// cp.async from every thread (a CTA's bulk copies would be served one after
+// another, one chain step each); E is double buffered, so a step needs one
+// barrier.  E_s goes to the workspace of segment s (its start state); the
+// last segment's own map is not needed (replaying that segment produces the
+// final state).  An empty sequence has no segment: its final state is its
+// initial state.
 constexpr int kCombineRows = 8;
+constexpr int kCombineThreads = 256;
 
 // steps in flight: the chain step is short next to an L2 round trip
 template <int D>
@@ -454,42 +458,47 @@ __host__ __device__ constexpr int combine_bufs() { return D == 64 ? 6 : 3; }
 template <int D>
 struct CombineLayout {
     static constexpr int kCombineBufs = combine_bufs<D>();
+    static constexpr int kLdM = D + 4;                                  // padded M rows
     static constexpr int kLdE = D + 4;                                  // padded E rows
-    static constexpr uint32_t M0 = 0;                                   // bufs x [D x D] fp32
-    static constexpr uint32_t N0 = kCombineBufs * D * D * 4u;           // bufs x [rows x D] fp32
+    static constexpr uint32_t M0 = 0;                                   // bufs x [D x kLdM] fp32
+    static constexpr uint32_t N0 = kCombineBufs * D * kLdM * 4u;        // bufs x [rows x D] fp32
     static constexpr uint32_t E = N0 + kCombineBufs * kCombineRows * D * 4u;   // 2 x [rows x kLdE]
     static constexpr uint32_t bytes = E + 2u * kCombineRows * kLdE * 4u;
     static constexpr uint32_t dyn_bytes = bytes + 128u;
+    static_assert(dyn_bytes <= 232448u, "shared memory budget");
 };
 
 template <int D>
-__global__ void __launch_bounds__(kCombineRows * D / 2)
+__global__ void __launch_bounds__(kCombineThreads)
 combine_kernel(const int32_t* __restrict__ cu, int H, int seg_chunks, const float* init_state,
                float* final_state, float* seg_ws, uint32_t* err) {
     using L = CombineLayout<D>;
     constexpr int RB = kCombineRows;
-    constexpr int QD = D / 4;
-    constexpr int NT = RB * QD * 2;                                     // threads
+    constexpr int NT = kCombineThreads;
     constexpr int NB = L::kCombineBufs;
+    constexpr int CW = D / 8;                                           // columns per warp
+    static_assert(RB == 8 && NT == 256, "8 rows x 4 inner-index phases per warp, 8 warps");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align_smem<128>(smem_raw);
     pdl_wait();                               // the previous kernel's memory is final
     const int pair = blockIdx.x, rb = blockIdx.y;
     const int n = pair / H, h = pair % H;
-    // warp = (row j, 16 column groups); lane bit 4 = inner-dimension half kh
-    const int tid = threadIdx.x, lane = tid & 31, wq = tid >> 5;
-    const int j = wq / (QD / 16), q = 16 * (wq % (QD / 16)) + (lane & 15), kh = lane >> 4;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int j = lane & 7, kq = lane >> 3, c0 = CW * warp;
     const int s0 = __ldg(cu + n), s1 = __ldg(cu + n + 1);
     const int span = kChunk * seg_chunks;
     const int nseg = (s1 - s0 + span - 1) / span;
     const size_t state_off = ((size_t)n * H + h) * D * D;
-    const size_t row_off = (size_t)(rb * RB + j) * D + 4 * q;
+    const size_t row_off = (size_t)(rb * RB + j) * D + c0;              // this lane's row, slab start
     (void)err;
     if (nseg == 0) {
-        if (kh == 0) {
-            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (init_state) x = *reinterpret_cast<const float4*>(init_state + state_off + row_off);
-            *reinterpret_cast<float4*>(final_state + state_off + row_off) = x;
+        if (kq == 0) {
+#pragma unroll
+            for (int c = 0; c < CW; c += 4) {
+                float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (init_state) x = *reinterpret_cast<const float4*>(init_state + state_off + row_off + c);
+                *reinterpret_cast<float4*>(final_state + state_off + row_off + c) = x;
+            }
         }
         return;
     }
@@ -501,17 +510,17 @@ combine_kernel(const int32_t* __restrict__ cu, int H, int seg_chunks, const floa
         const int b = s % NB;
         const uint8_t* msrc = reinterpret_cast<const uint8_t*>(seg_ptr(s) + (size_t)D * D);
         const uint8_t* nsrc = reinterpret_cast<const uint8_t*>(seg_ptr(s) + (size_t)rb * RB * D);
-        uint8_t* mdst = sm + L::M0 + b * D * D * 4u;
+        float* mdst = reinterpret_cast<float*>(sm + L::M0 + b * D * L::kLdM * 4u);
         uint8_t* ndst = sm + L::N0 + b * RB * D * 4u;
 #pragma unroll
-        for (int c = tid; c < D * D / 4; c += NT) cp_async16(mdst + 16 * c, msrc + 16 * c, 16u);
+        for (int c = tid; c < D * D / 4; c += NT)
+            cp_async16(mdst + (c / (D / 4)) * L::kLdM + 4 * (c % (D / 4)), msrc + 16 * c, 16u);
 #pragma unroll
         for (int c = tid; c < RB * D / 4; c += NT) cp_async16(ndst + 16 * c, nsrc + 16 * c, 16u);
     };
-    if (kh == 0) {
-        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (init_state) x = *reinterpret_cast<const float4*>(init_state + state_off + row_off);
-        *reinterpret_cast<float4*>(e + j * L::kLdE + 4 * q) = x;
+    for (int c = tid; c < RB * D; c += NT) {
+        const int r = c / D, col = c % D;
+        e[r * L::kLdE + col] = init_state ? init_state[state_off + (size_t)(rb * RB + r) * D + col] : 0.f;
     }
     // steps 0 .. NB-2 in flight (one commit group per step, empty past the end)
 #pragma unroll
@@ -525,35 +534,42 @@ combine_kernel(const int32_t* __restrict__ cu, int H, int seg_chunks, const floa
         if (s + NB - 1 <= nseg - 2) issue(s + NB - 1);
         cp_async_commit();
         const int b = s % NB;
-        const float* Mm = reinterpret_cast<const float*>(sm + L::M0 + b * D * D * 4u);
+        const float* Mm = reinterpret_cast<const float*>(sm + L::M0 + b * D * L::kLdM * 4u);
         const float* Nm = reinterpret_cast<const float*>(sm + L::N0 + b * RB * D * 4u);
-        const float* ec = e + (s & 1) * RB * L::kLdE;
-        float4 acc = kh == 0 ? *reinterpret_cast<const float4*>(Nm + j * D + 4 * q)
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
-        const int k0 = kh * (D / 2);
-#pragma unroll 2
-        for (int i = 0; i < D / 2; i += 4) {
-            // four inner steps per E load; the second half runs four steps
-            // rotated, so the two halves' E reads fall in different banks
-            const int k = k0 + ((i + 4 * kh) & (D / 2 - 1));
-            const float4 e4 = *reinterpret_cast<const float4*>(ec + j * L::kLdE + k);
-            const float ev[4] = {e4.x, e4.y, e4.z, e4.w};
+        const float* ec = e + (s & 1) * RB * L::kLdE + j * L::kLdE;
+        float acc[CW];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const float4 m = *reinterpret_cast<const float4*>(Mm + (k + u) * D + 4 * q);
-                acc.x = fmaf(ev[u], m.x, acc.x);
-                acc.y = fmaf(ev[u], m.y, acc.y);
-                acc.z = fmaf(ev[u], m.z, acc.z);
-                acc.w = fmaf(ev[u], m.w, acc.w);
+        for (int c = 0; c < CW; ++c) acc[c] = 0.f;
+#pragma unroll 4
+        for (int i = 0; i < D / 4; ++i) {
+            const int k = 4 * i + kq;
+            const float ek = ec[k];
+            const float* mrow = Mm + k * L::kLdM + c0;
+#pragma unroll
+            for (int c = 0; c < CW; c += 4) {
+                const float4 m = *reinterpret_cast<const float4*>(mrow + c);
+                acc[c] = fmaf(ek, m.x, acc[c]);
+                acc[c + 1] = fmaf(ek, m.y, acc[c + 1]);
+                acc[c + 2] = fmaf(ek, m.z, acc[c + 2]);
+                acc[c + 3] = fmaf(ek, m.w, acc[c + 3]);
             }
         }
-        acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 16);
-        acc.y += __shfl_xor_sync(0xffffffffu, acc.y, 16);
-        acc.z += __shfl_xor_sync(0xffffffffu, acc.z, 16);
-        acc.w += __shfl_xor_sync(0xffffffffu, acc.w, 16);
-        if (kh == 0) {
-            *reinterpret_cast<float4*>(e + ((s + 1) & 1) * RB * L::kLdE + j * L::kLdE + 4 * q) = acc;
-            *reinterpret_cast<float4*>(seg_ptr(s + 1) + 2u * D * D + row_off) = acc;
+#pragma unroll
+        for (int c = 0; c < CW; ++c) {
+            acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], 8);
+            acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], 16);
+        }
+        if (kq == 0) {
+            float* en = e + ((s + 1) & 1) * RB * L::kLdE + j * L::kLdE + c0;
+            float* eg = seg_ptr(s + 1) + 2u * D * D + row_off;
+#pragma unroll
+            for (int c = 0; c < CW; c += 4) {
+                const float4 nv = *reinterpret_cast<const float4*>(Nm + j * D + c0 + c);
+                const float4 x = make_float4(acc[c] + nv.x, acc[c + 1] + nv.y, acc[c + 2] + nv.z,
+                                             acc[c + 3] + nv.w);
+                *reinterpret_cast<float4*>(en + c) = x;
+                *reinterpret_cast<float4*>(eg + c) = x;
+            }
         }
     }
     pdl_launch_dependents();
@@ -589,7 +605,7 @@ cudaError_t launch_typed(const gdr_prefill_args& a, const uint8_t* records,
                              (int)CombineLayout<D>::dyn_bytes);
     if (e != cudaSuccess) return e;
     e = launch_pdl(false, ck, dim3((unsigned)a.n_seqs * (unsigned)a.n_heads, D / kCombineRows),
-                   dim3(kCombineRows * D / 2), CombineLayout<D>::dyn_bytes, st, a.cu_seqlens,
+                   dim3(kCombineThreads), CombineLayout<D>::dyn_bytes, st, a.cu_seqlens,
                    a.n_heads, lay.seg_chunks, a.init_state, a.final_state, seg_ws, err);
     if (e != cudaSuccess) return e;
     return launch_mode<D, OutT, kApply>(a, records, lay, seg_ws, err, st);
