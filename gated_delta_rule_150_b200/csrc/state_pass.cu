@@ -439,7 +439,7 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
 // one (sequence, head).  Warp w owns the column slab [w D/8, (w+1) D/8) for
 // all of the CTA's rows, so each step reads M_s from shared memory once per
 // CTA: lane (j = lane % 8, kq = lane / 8) sums row j over the inner indices
-// k = 4i + kq, and the four partial sums meet by shuffles.  Each step's M_s
+// k = 4i + kq, and the four partial sums meet by a shuffle reduce-scatter.  Each step's M_s
 // (rows padded so the four k of one load fall in different banks) and the
 // CTA's rows of N_s are fetched kCombineBufs - 1 steps ahead by 16-byte
 // cp.async from every thread (a CTA's bulk copies would be served one after
@@ -540,35 +540,55 @@ combine_kernel(const int32_t* __restrict__ cu, int H, int seg_chunks, const floa
         float acc[CW];
 #pragma unroll
         for (int c = 0; c < CW; ++c) acc[c] = 0.f;
-#pragma unroll 4
-        for (int i = 0; i < D / 4; ++i) {
-            const int k = 4 * i + kq;
-            const float ek = ec[k];
-            const float* mrow = Mm + k * L::kLdM + c0;
+        // inner indices in groups of 16: the loads of a group are issued
+        // before its FMAs
 #pragma unroll
-            for (int c = 0; c < CW; c += 4) {
-                const float4 m = *reinterpret_cast<const float4*>(mrow + c);
-                acc[c] = fmaf(ek, m.x, acc[c]);
-                acc[c + 1] = fmaf(ek, m.y, acc[c + 1]);
-                acc[c + 2] = fmaf(ek, m.z, acc[c + 2]);
-                acc[c + 3] = fmaf(ek, m.w, acc[c + 3]);
+        for (int i0 = 0; i0 < D / 4; i0 += 16) {
+            float ek[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) ek[i] = ec[4 * (i0 + i) + kq];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float* mrow = Mm + (4 * (i0 + i) + kq) * L::kLdM + c0;
+#pragma unroll
+                for (int c = 0; c < CW; c += 4) {
+                    const float4 m = *reinterpret_cast<const float4*>(mrow + c);
+                    acc[c] = fmaf(ek[i], m.x, acc[c]);
+                    acc[c + 1] = fmaf(ek[i], m.y, acc[c + 1]);
+                    acc[c + 2] = fmaf(ek[i], m.z, acc[c + 2]);
+                    acc[c + 3] = fmaf(ek[i], m.w, acc[c + 3]);
+                }
             }
         }
+        // reduce-scatter over the four inner-index phases: after two shuffle
+        // rounds lane kq holds the full sums of columns c0 + kq * CW/4 ...
+        constexpr int CH = CW / 2, CQ = CW / 4;
+        const bool hi16 = (kq & 2) != 0, hi8 = (kq & 1) != 0;
+        float h[CH];
 #pragma unroll
-        for (int c = 0; c < CW; ++c) {
-            acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], 8);
-            acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], 16);
+        for (int c = 0; c < CH; ++c) {
+            const float send = hi16 ? acc[c] : acc[CH + c];
+            const float keep = hi16 ? acc[CH + c] : acc[c];
+            h[c] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
         }
-        if (kq == 0) {
-            float* en = e + ((s + 1) & 1) * RB * L::kLdE + j * L::kLdE + c0;
-            float* eg = seg_ptr(s + 1) + 2u * D * D + row_off;
+        float qv[CQ];
 #pragma unroll
-            for (int c = 0; c < CW; c += 4) {
-                const float4 nv = *reinterpret_cast<const float4*>(Nm + j * D + c0 + c);
-                const float4 x = make_float4(acc[c] + nv.x, acc[c + 1] + nv.y, acc[c + 2] + nv.z,
-                                             acc[c + 3] + nv.w);
-                *reinterpret_cast<float4*>(en + c) = x;
-                *reinterpret_cast<float4*>(eg + c) = x;
+        for (int c = 0; c < CQ; ++c) {
+            const float send = hi8 ? h[c] : h[CQ + c];
+            const float keep = hi8 ? h[CQ + c] : h[c];
+            qv[c] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+        }
+        {
+            const int cq = c0 + (hi16 ? CH : 0) + (hi8 ? CQ : 0);     // this lane's columns
+            float* en = e + ((s + 1) & 1) * RB * L::kLdE + j * L::kLdE + cq;
+            float* eg = seg_ptr(s + 1) + 2u * D * D + (size_t)(rb * RB + j) * D + cq;
+            const float* nr = Nm + j * D + cq;
+#pragma unroll
+            for (int c = 0; c < CQ; c += 2) {
+                const float2 nv = *reinterpret_cast<const float2*>(nr + c);
+                const float2 x = make_float2(qv[c] + nv.x, qv[c + 1] + nv.y);
+                *reinterpret_cast<float2*>(en + c) = x;
+                *reinterpret_cast<float2*>(eg + c) = x;
             }
         }
     }
