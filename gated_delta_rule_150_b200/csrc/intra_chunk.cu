@@ -200,6 +200,54 @@ __device__ __forceinline__ void xor_permute(uint32_t (&a)[8][N], int s) {
     }
 }
 
+// Barrier among the first `count` threads of the CTA (named barrier `id`).
+__device__ __forceinline__ void named_bar(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ void solve_bar() { named_bar(1, 128); }
+
+// OR of `pred` over the `count` threads that reach named barrier `id`.
+__device__ __forceinline__ bool bar_or(int id, int count, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r) : "r"((uint32_t)pred), "r"(id), "r"(count) : "memory");
+    return r != 0;
+}
+
+// Chunk-local cumulative log decay of one chunk in place (sG: [64 x D] fp32),
+// by NS threads (t = 0 .. NS-1): 128 / D row parts per channel, the parts
+// joined by a shuffle.  Rows past len add 0.  Returns whether this thread saw
+// a log a below -kMaxFactorExp / 8.
+template <int D, int NS>
+__device__ __forceinline__ bool scan_channels(float* sG, int len, int t) {
+    static_assert(NS == 128 && (D == 64 || D == 128), "two parts of 32 rows (d 64) or one of 64");
+    constexpr int P = NS / D, RP = 64 / P;
+    // D = 64: channel c = 16 (t / 32) + (t % 32) / 2, part = t % 2; D = 128: c = t
+    const int c = (P == 1) ? t : 16 * (t >> 5) + ((t & 31) >> 1);
+    const int part = (P == 1) ? 0 : (t & 1);
+    bool bad = false;
+    float run = 0.f;
+#pragma unroll 4
+    for (int r = part * RP; r < (part + 1) * RP; ++r) {
+        const float la = r < len ? sG[r * D + c] : 0.f;
+        bad |= la < -kMaxFactorExp / 8.f;
+        run += la;
+        sG[r * D + c] = run;
+    }
+    if (P == 2) {
+        const float tot0 = __shfl_xor_sync(0xffffffffu, run, 1);    // part 0's total
+        if (part == 1) {
+#pragma unroll 4
+            for (int r = RP; r < 64; ++r) sG[r * D + c] += tot0;
+        }
+    }
+    return bad;
+}
+
 // One unit of work: chunk slot idx / H of head idx % H (idx < 0: none).
 struct Item {
     int64_t idx;
@@ -316,6 +364,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     __shared__ uint64_t in_bar[2];          // inputs landed: log a, q/k/v
     __shared__ uint32_t tmem_slot;
     __shared__ Item s_item[2];              // the next two items, by iteration parity
+    __shared__ int s_bad_next;              // the scanned next item has a log a < -10
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const size_t tok_stride = (size_t)H * D;
@@ -356,6 +405,10 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     uint32_t phase = 0;                                       // parity of the next MMA commit
     uint32_t in_phase = 0;                                    // parity of the inputs' barriers
     int iter = 0;                                             // item n: s_item[(n+1)&1] = item n+1
+    // per-channel decay at 8 warps: the next item's scan runs on warps 4-7
+    // while warps 0-3 do the triangular solve
+    constexpr bool kEarlyScan = !SCALAR && NT == 256;
+    bool pre_scanned = false;                                 // this item's g is already in sG
     bool failed = false;
 
     while (cur.idx >= 0) {
@@ -381,6 +434,10 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     // whenever every log a >= -kMaxFactorExp / 8; a chunk with a smaller log a
     // in some channel takes the exact path.
     bool bad = false;
+    bool bad_chunk;
+    if (kEarlyScan && pre_scanned) {
+        bad_chunk = s_bad_next != 0;          // scanned during the previous item's solve
+    } else {
     if (!SCALAR) {
         constexpr int P = NT / D, RP = 64 / P;                // row parts per channel
         float* Ptot = reinterpret_cast<float*>(sm + L::Ptot);
@@ -414,7 +471,8 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         Gs[2 * lane] = excl + x0;
         Gs[2 * lane + 1] = excl + pair;
     }
-    const bool bad_chunk = __syncthreads_or(bad);
+    bad_chunk = __syncthreads_or(bad);
+    }
 
     const int cg = tid % CG, rg = tid / CG, c0 = 8 * cg;
     const int r0 = rg * RPT;
@@ -705,73 +763,89 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     // still read it have passed a barrier.  Every phase also writes its bf16
     // copy straight into the operand tile Tb, whose blocks above the
     // diagonal are zeroed here.
+    // Warps 0-3 solve (named barrier 1); warps 4-7 meanwhile scan the next
+    // item's log a, which the loader warp has just requested.
     uint8_t* Tb = sm + L::Tb;
-    if (tid >= 64 && tid < 256) {
-        // (row, chunk) pairs of the zero blocks (b, j > b): 96 + 64 + 32
-        const int z = tid - 64;
-        int r, jj;
-        if (z < 96) { r = z / 6; jj = 2 + z % 6; }
-        else if (z < 160) { r = 16 + (z - 96) / 4; jj = 4 + (z - 96) % 4; }
-        else { r = 32 + (z - 160) / 2; jj = 6 + (z - 160) % 2; }
-        *reinterpret_cast<uint4*>(Tb + sw128_chunk(64, r, jj)) = make_uint4(0u, 0u, 0u, 0u);
-    }
-    if (tid < 64) {
-        // column cc of T_bb, right-looking: once x_j is known it is folded
-        // into every later row's running sum, so each step waits on one FMA
-        const int b = tid >> 4, cc = tid & 15, o = 16 * b;
-        float x[16], acc[16];
+    if (tid < 128) {
+        if (tid >= 64) {
+            // (row, chunk) pairs of the zero blocks (b, j > b): 96 + 64 + 32
 #pragma unroll
-        for (int r = 0; r < 16; ++r) acc[r] = 0.f;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            x[j] = (j < cc) ? 0.f : ((j == cc) ? 1.f : -acc[j]);
-#pragma unroll
-            for (int r = j + 1; r < 16; ++r) acc[r] = fmaf(As[(o + r) * kLd + o + j], x[j], acc[r]);
+            for (int z = tid - 64; z < 192; z += 64) {
+                int r, jj;
+                if (z < 96) { r = z / 6; jj = 2 + z % 6; }
+                else if (z < 160) { r = 16 + (z - 96) / 4; jj = 4 + (z - 96) % 4; }
+                else { r = 32 + (z - 160) / 2; jj = 6 + (z - 160) % 2; }
+                *reinterpret_cast<uint4*>(Tb + sw128_chunk(64, r, jj)) = make_uint4(0u, 0u, 0u, 0u);
+            }
         }
-        __syncwarp();          // every lane has read A_bb before T_bb overwrites it
+        if (tid < 64) {
+            // column cc of T_bb, right-looking: once x_j is known it is folded
+            // into every later row's running sum, so each step waits on one FMA
+            const int b = tid >> 4, cc = tid & 15, o = 16 * b;
+            float x[16], acc[16];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            As[(o + r) * kLd + o + cc] = x[r];
-            *reinterpret_cast<__nv_bfloat16*>(Tb + sw128_offset(64, o + r, o + cc)) = __float2bfloat16_rn(x[r]);
+            for (int r = 0; r < 16; ++r) acc[r] = 0.f;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                x[j] = (j < cc) ? 0.f : ((j == cc) ? 1.f : -acc[j]);
+#pragma unroll
+                for (int r = j + 1; r < 16; ++r) acc[r] = fmaf(As[(o + r) * kLd + o + j], x[j], acc[r]);
+            }
+            __syncwarp();          // every lane has read A_bb before T_bb overwrites it
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                As[(o + r) * kLd + o + cc] = x[r];
+                *reinterpret_cast<__nv_bfloat16*>(Tb + sw128_offset(64, o + r, o + cc)) = __float2bfloat16_rn(x[r]);
+            }
         }
-    }
-    __syncthreads();
-    // first-level merges inside each 32-row half: T_10 = -T_11 A_10 T_00 and
-    // T_32 = -T_33 A_32 T_22 (a 2 x 4 tile per thread, 64 threads)
-    const int t32 = tid & 31, rr0 = 2 * (t32 >> 2), c4 = 4 * (t32 & 3);
-    if (tid < 64) {
-        const int p = tid >> 5, b = 2 * p + 1, j = 2 * p;
-        float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
-        tile16<kLd>(As, 16 * b + rr0, 16 * j, As, 16 * j, 16 * j + c4, y0, y1);
-        *reinterpret_cast<float4*>(Yt + p * 256 + rr0 * 16 + c4) = make_float4(y0[0], y0[1], y0[2], y0[3]);
-        *reinterpret_cast<float4*>(Yt + p * 256 + (rr0 + 1) * 16 + c4) = make_float4(y1[0], y1[1], y1[2], y1[3]);
-    }
-    __syncthreads();
-    if (tid < 64) {
-        const int p = tid >> 5, b = 2 * p + 1, j = 2 * p;
-        float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
-        tile16<16>(As, 16 * b + rr0, 16 * b, Yt + p * 256, 0, c4, z0, z1);
-        store_t_tile(As, Tb, 16 * b + rr0, 16 * j + c4, z0, z1);
-    }
-    __syncthreads();
-    // bottom-left 32 x 32 block, blocks (b, j) with b in {2, 3}, j in {0, 1}:
-    //   Y_bj = sum_{l=j}^{1} A_bl T_lj        T_bj = -sum_{l=2}^{b} T_bl Y_lj
-    {
-        const int q = (tid >> 5) & 3, b = 2 + (q >> 1), j = q & 1;
-        if (tid < 128) {
+        solve_bar();
+        // first-level merges inside each 32-row half: T_10 = -T_11 A_10 T_00 and
+        // T_32 = -T_33 A_32 T_22 (a 2 x 4 tile per thread, 64 threads)
+        const int t32 = tid & 31, rr0 = 2 * (t32 >> 2), c4 = 4 * (t32 & 3);
+        if (tid < 64) {
+            const int p = tid >> 5, b = 2 * p + 1, j = 2 * p;
             float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int l = j; l <= 1; ++l)
-                tile16<kLd>(As, 16 * b + rr0, 16 * l, As, 16 * l, 16 * j + c4, y0, y1);
-            *reinterpret_cast<float4*>(Yt + (16 * (b - 2) + rr0) * 32 + 16 * j + c4) = make_float4(y0[0], y0[1], y0[2], y0[3]);
-            *reinterpret_cast<float4*>(Yt + (16 * (b - 2) + rr0 + 1) * 32 + 16 * j + c4) = make_float4(y1[0], y1[1], y1[2], y1[3]);
+            tile16<kLd>(As, 16 * b + rr0, 16 * j, As, 16 * j, 16 * j + c4, y0, y1);
+            *reinterpret_cast<float4*>(Yt + p * 256 + rr0 * 16 + c4) = make_float4(y0[0], y0[1], y0[2], y0[3]);
+            *reinterpret_cast<float4*>(Yt + p * 256 + (rr0 + 1) * 16 + c4) = make_float4(y1[0], y1[1], y1[2], y1[3]);
         }
-        __syncthreads();
-        if (tid < 128) {
+        solve_bar();
+        if (tid < 64) {
+            const int p = tid >> 5, b = 2 * p + 1, j = 2 * p;
             float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int l = 2; l <= b; ++l)
-                tile16<32>(As, 16 * b + rr0, 16 * l, Yt, 16 * (l - 2), 16 * j + c4, z0, z1);
+            tile16<16>(As, 16 * b + rr0, 16 * b, Yt + p * 256, 0, c4, z0, z1);
             store_t_tile(As, Tb, 16 * b + rr0, 16 * j + c4, z0, z1);
         }
+        solve_bar();
+        // bottom-left 32 x 32 block, blocks (b, j) with b in {2, 3}, j in {0, 1}:
+        //   Y_bj = sum_{l=j}^{1} A_bl T_lj        T_bj = -sum_{l=2}^{b} T_bl Y_lj
+        {
+            const int q = (tid >> 5) & 3, b = 2 + (q >> 1), j = q & 1;
+            if (tid < 128) {
+                float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int l = j; l <= 1; ++l)
+                    tile16<kLd>(As, 16 * b + rr0, 16 * l, As, 16 * l, 16 * j + c4, y0, y1);
+                *reinterpret_cast<float4*>(Yt + (16 * (b - 2) + rr0) * 32 + 16 * j + c4) = make_float4(y0[0], y0[1], y0[2], y0[3]);
+                *reinterpret_cast<float4*>(Yt + (16 * (b - 2) + rr0 + 1) * 32 + 16 * j + c4) = make_float4(y1[0], y1[1], y1[2], y1[3]);
+            }
+            solve_bar();
+            if (tid < 128) {
+                float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int l = 2; l <= b; ++l)
+                    tile16<32>(As, 16 * b + rr0, 16 * l, Yt, 16 * (l - 2), 16 * j + c4, z0, z1);
+                store_t_tile(As, Tb, 16 * b + rr0, 16 * j + c4, z0, z1);
+            }
+        }
+    } else if (kEarlyScan && tid < 256) {
+        // the next item's chunk-local cumulative decay (see the item start)
+        const Item nx = s_item[(iter + 1) & 1];
+        bool nbad = false;
+        if (nx.idx >= 0) {
+            if (!mbar_wait(&in_bar[0], in_phase)) failed = true;
+            nbad = scan_channels<D, 128>(sG, nx.len, tid - 128);
+        }
+        nbad = bar_or(2, 128, nbad);
+        if (tid == 128) s_bad_next = nbad ? 1 : 0;
     }
     fence_proxy_async_smem();
     tc_fence_before_sync();
@@ -907,6 +981,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     if (failed) break;                        // a timed-out MMA: stop issuing work
     cur = nxt;
     ++iter;
+    pre_scanned = kEarlyScan;
     }
 
     pdl_launch_dependents();
