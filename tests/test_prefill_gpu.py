@@ -142,6 +142,20 @@ def test_chunk_factors_extreme_decay():
     _check(inp, o, fin, None, what="extreme decay")
 
 
+@pytest.mark.parametrize("d,heads,chunks", [(64, 8, 150), (128, 4, 100)])
+def test_extreme_decay_many_items_per_cta(d, heads, chunks):
+    """More chunk-heads than CTAs, so each persistent CTA runs several, with
+    every third chunk carrying a log decay of -30 in a few channels: the
+    exact path and the flag carried from one item's scan to the next."""
+    w = wl.shrink(wl.VARLEN, n_heads=heads, d_k=d, d_v=d, lengths=(64 * chunks,), init_std=0.1,
+                  snap_interval=0)
+    inp = wl.make_prefill_inputs(w)
+    for c in range(0, chunks, 3):
+        inp["log_a"][64 * c + 10: 64 * c + 20, :, 3:7] = -30.0
+    o, fin, _ = _gpu_prefill(inp)
+    _check(inp, o, fin, None, what=f"extreme decay d{d}")
+
+
 # ---------------------------------------------------------------------------
 # whole prefill
 # ---------------------------------------------------------------------------
