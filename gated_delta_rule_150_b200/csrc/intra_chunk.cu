@@ -917,34 +917,13 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
 
     // ---- record: Qt = Qg - P W, PU, BS = -Kd^T W, NC = U^T Kd, gamma ----------
     // assembled in region 2 and the dead Bt, Kdt (everything there is dead
-    // once the MMAs above have completed) and written with one bulk store,
-    // which drains while the next item starts
+    // once the MMAs above have completed) and written with two bulk stores,
+    // the second of which drains while the next item starts
     uint8_t* srec = sm + L::Rec;
+    // rows of the M = 64 products live in lanes 16 w + l (l < 16)
+    const int r64 = 16 * (warp & 3) + lane;
+    const bool act64 = lane < 16;
     {
-        // rows of the M = 64 products live in lanes 16 w + l (l < 16)
-        const int r64 = 16 * (warp & 3) + lane;
-        const bool act64 = lane < 16;
-#pragma unroll
-        for (int piece = 0; piece < D / 32; ++piece) {
-            if (piece % NG != wgrp) continue;
-            float pw[32], pu[32];
-            tmem_ld32(tmem + lane_base + 32 * piece, pw);
-            tmem_ld32(tmem + lane_base + D + 32 * piece, pu);
-            tmem_ld_wait();
-            if (act64) {
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    const int chunk = 4 * piece + jj;
-                    float qgv[8];
-                    Vec8<__nv_bfloat16>::load(reinterpret_cast<const __nv_bfloat16*>(Qgs + sw128_chunk(64, r64, chunk)), qgv);
-                    float a[8], b[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) { a[e] = qgv[e] - pw[8 * jj + e]; b[e] = pu[8 * jj + e]; }
-                    *reinterpret_cast<uint4*>(srec + R.Qt + sw128_chunk(64, r64, chunk)) = pack8(a);
-                    *reinterpret_cast<uint4*>(srec + R.PU + sw128_chunk(64, r64, chunk)) = pack8(b);
-                }
-            }
-        }
         const int rD = (D == 128) ? (32 * (warp & 3) + lane) : r64;
         const bool actD = (D == 128) || act64;
 #pragma unroll
@@ -966,6 +945,37 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                 }
             }
         }
+    }
+    // BS and NC (the larger part) go out first; their bulk store drains while
+    // Qt, PU and gamma are assembled
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+        bulk_s2g(rec + R.BS, srec + R.BS, 4u * D * D);
+        bulk_commit_group();
+    }
+    {
+#pragma unroll
+        for (int piece = 0; piece < D / 32; ++piece) {
+            if (piece % NG != wgrp) continue;
+            float pw[32], pu[32];
+            tmem_ld32(tmem + lane_base + 32 * piece, pw);
+            tmem_ld32(tmem + lane_base + D + 32 * piece, pu);
+            tmem_ld_wait();
+            if (act64) {
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int chunk = 4 * piece + jj;
+                    float qgv[8];
+                    Vec8<__nv_bfloat16>::load(reinterpret_cast<const __nv_bfloat16*>(Qgs + sw128_chunk(64, r64, chunk)), qgv);
+                    float a[8], b[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) { a[e] = qgv[e] - pw[8 * jj + e]; b[e] = pu[8 * jj + e]; }
+                    *reinterpret_cast<uint4*>(srec + R.Qt + sw128_chunk(64, r64, chunk)) = pack8(a);
+                    *reinterpret_cast<uint4*>(srec + R.PU + sw128_chunk(64, r64, chunk)) = pack8(b);
+                }
+            }
+        }
         if (tid < D) reinterpret_cast<float*>(srec + R.gamma)[tid] = expf(Gl[tid]);
     }
     const Item nxt = s_item[(iter + 1) & 1];  // read before the loader may overwrite it
@@ -974,7 +984,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     failed = __syncthreads_or(failed);
     tc_fence_after_sync();
     if (tid == 0) {
-        bulk_s2g(rec, srec, R.bytes);
+        bulk_s2g(rec + R.Qt, srec + R.Qt, R.bytes - 4u * D * D);
         bulk_commit_group();
         if (failed) atomicOr(err, 1u);
     }
