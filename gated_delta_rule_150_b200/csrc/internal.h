@@ -79,6 +79,13 @@ cudaError_t launch_pdl(bool early, void (*kern)(KArgs...), dim3 grid, dim3 block
     return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
+// Records small enough to stay in L2 (126 MB) between the two stages are
+// written and first read with an evict-last hint (and the inputs read with
+// evict-first); larger sets use the default cache policy.
+inline bool records_fit_l2(int64_t n_slots, int H, int D) {
+    return (double)n_slots * H * record_layout(D).bytes <= 96.0 * 1024 * 1024;
+}
+
 inline int segment_chunks(int n_seqs, int H, int64_t T, int D) {
     if (n_seqs <= 0 || T <= 0) return 0;
     const int64_t pairs = (int64_t)n_seqs * H;

@@ -287,18 +287,23 @@ template <int D, typename InT, bool SCALAR, typename L>
 __device__ __forceinline__ void issue_inputs(uint8_t* sm, uint64_t* bar_g, uint64_t* bar_qkv,
                                              const InputMaps& maps, const float* __restrict__ beta,
                                              const float* __restrict__ log_a, int H, const Item& it,
-                                             int lane) {
+                                             int lane, bool hint) {
     if (lane == 0) {
         const int x = it.h * D;
+        const uint64_t pol = l2_policy_evict_first();             // inputs are read once
         if (!SCALAR) {
             mbar_arrive_expect_tx(bar_g, 64u * D * 4u);
-            tma_load_2d(sm + L::sG, &maps.g, x, it.start, bar_g);
+            if (hint) tma_load_2d_hint(sm + L::sG, &maps.g, x, it.start, bar_g, pol);
+            else tma_load_2d(sm + L::sG, &maps.g, x, it.start, bar_g);
         }
         if (L::kStageQKV) {
             mbar_arrive_expect_tx(bar_qkv, 3u * 64u * D * (uint32_t)sizeof(InT));
-            tma_load_2d(sm + L::sQ, &maps.q, x, it.start, bar_qkv);
-            tma_load_2d(sm + L::sK, &maps.k, x, it.start, bar_qkv);
-            tma_load_2d(sm + L::sV, &maps.v, x, it.start, bar_qkv);
+            if (hint) tma_load_2d_hint(sm + L::sQ, &maps.q, x, it.start, bar_qkv, pol);
+            else tma_load_2d(sm + L::sQ, &maps.q, x, it.start, bar_qkv);
+            if (hint) tma_load_2d_hint(sm + L::sK, &maps.k, x, it.start, bar_qkv, pol);
+            else tma_load_2d(sm + L::sK, &maps.k, x, it.start, bar_qkv);
+            if (hint) tma_load_2d_hint(sm + L::sV, &maps.v, x, it.start, bar_qkv, pol);
+            else tma_load_2d(sm + L::sV, &maps.v, x, it.start, bar_qkv);
         }
     }
     for (int t = lane; t < 64; t += 32) {
@@ -349,7 +354,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                    const InT* __restrict__ q, const InT* __restrict__ k, const InT* __restrict__ v,
                    const float* __restrict__ beta, const float* __restrict__ log_a, float scale,
                    int64_t n_items, uint8_t* __restrict__ records, uint32_t* err,
-                   const __grid_constant__ InputMaps maps) {
+                   const __grid_constant__ InputMaps maps, int keep_records) {
     using L = IntraLayout<D, InT, SCALAR>;
     constexpr RecordLayout R = record_layout(D);
     constexpr int CG = D / 8;              // channel groups of 8
@@ -398,7 +403,8 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     __syncthreads();
     tc_fence_after_sync();
     if (cur.idx >= 0 && warp == kLoadWarp)
-        issue_inputs<D, InT, SCALAR, L>(sm, &in_bar[0], &in_bar[1], maps, beta, log_a, H, cur, lane);
+        issue_inputs<D, InT, SCALAR, L>(sm, &in_bar[0], &in_bar[1], maps, beta, log_a, H, cur, lane,
+                                        keep_records != 0);
     const uint32_t tmem = tmem_slot;
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
     const int wgrp = warp >> 2;                               // warp group (0 .. NG - 1)
@@ -753,7 +759,8 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         const Item nxt = s_item[(iter + 1) & 1];
         fence_proxy_async_smem();             // this item's reads of region 1 come first
         if (nxt.idx >= 0)
-            issue_inputs<D, InT, SCALAR, L>(sm, &in_bar[0], &in_bar[1], maps, beta, log_a, H, nxt, lane);
+            issue_inputs<D, InT, SCALAR, L>(sm, &in_bar[0], &in_bar[1], maps, beta, log_a, H, nxt, lane,
+                                            keep_records != 0);
         if (lane == 0)
             s_item[iter & 1] = nxt.idx >= 0 ? find_item(cu, n_seqs, H, n_items, nxt.idx + gridDim.x) : nxt;
     }
@@ -951,7 +958,8 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {
-        bulk_s2g(rec + R.BS, srec + R.BS, 4u * D * D);
+        if (keep_records) bulk_s2g_hint(rec + R.BS, srec + R.BS, 4u * D * D, l2_policy_evict_last());
+        else bulk_s2g(rec + R.BS, srec + R.BS, 4u * D * D);
         bulk_commit_group();
     }
     {
@@ -984,7 +992,8 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     failed = __syncthreads_or(failed);
     tc_fence_after_sync();
     if (tid == 0) {
-        bulk_s2g(rec + R.Qt, srec + R.Qt, R.bytes - 4u * D * D);
+        if (keep_records) bulk_s2g_hint(rec + R.Qt, srec + R.Qt, R.bytes - 4u * D * D, l2_policy_evict_last());
+        else bulk_s2g(rec + R.Qt, srec + R.Qt, R.bytes - 4u * D * D);
         bulk_commit_group();
         if (failed) atomicOr(err, 1u);
     }
@@ -1115,7 +1124,8 @@ cudaError_t launch_typed(const gdr_prefill_args& a, uint8_t* records, uint32_t* 
     const unsigned grid = (unsigned)(n_items < resident ? n_items : resident);
     return launch_pdl(true, kern, dim3(grid), dim3(threads_for<D, SCALAR>()), smem, st, a.cu_seqlens,
                       a.n_seqs, a.n_heads, (const InT*)a.q, (const InT*)a.k, (const InT*)a.v, a.beta,
-                      a.log_a, a.scale, n_items, records, err, maps);
+                      a.log_a, a.scale, n_items, records, err, maps,
+                      records_fit_l2(n_chunk_slots(a.total_tokens, a.n_seqs), a.n_heads, D) ? 1 : 0);
 }
 
 template <int D, typename InT>

@@ -79,7 +79,7 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                   const uint8_t* __restrict__ records, const float* init_state,
                   OutT* __restrict__ o, float* final_state, int snap_interval,
                   float* __restrict__ snapshots, int seg_chunks, float* seg_ws,
-                  uint32_t* err) {
+                  uint32_t* err, int keep_records) {
     using L = PassLayout<D, MODE>;
     constexpr RecordLayout R = record_layout(D);
     constexpr int ST = L::kStages;
@@ -139,7 +139,17 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         const int s = c % ST;
         const uint8_t* r = record_of(c);
         mbar_arrive_expect_tx(&full[s], L::tx_bytes);
-        if (kOut) {
+        if (keep_records) {
+            // a record set that fits in L2: the state-only pass leaves it there
+            // for the replay, the passes with outputs read it for the last time
+            const uint64_t pol = (MODE == kLocal) ? l2_policy_evict_last() : l2_policy_evict_first();
+            if (kOut) {
+                bulk_g2s_hint(stage(s), r, R.used, &full[s], pol);
+            } else {
+                bulk_g2s_hint(stage(s) + R.BS, r + R.BS, 4u * D * D, &full[s], pol);   // BS and NC
+                bulk_g2s_hint(stage(s) + L::kGamma, r + R.gamma, 4u * D, &full[s], pol);
+            }
+        } else if (kOut) {
             bulk_g2s(stage(s), r, R.used, &full[s]);
         } else {
             bulk_g2s(stage(s) + R.BS, r + R.BS, 4u * D * D, &full[s]);     // BS and NC
@@ -610,7 +620,8 @@ cudaError_t launch_mode(const gdr_prefill_args& a, const uint8_t* records,
     // slower with it
     return launch_pdl(MODE == kFull, kern, grid, dim3(kThreads), smem, st, a.cu_seqlens, a.n_seqs, a.n_heads,
                       records, a.init_state, static_cast<OutT*>(a.o), a.final_state,
-                      a.snap_interval, a.snapshots, lay.seg_chunks, seg_ws, err);
+                      a.snap_interval, a.snapshots, lay.seg_chunks, seg_ws, err,
+                      records_fit_l2(lay.n_slots, a.n_heads, D) ? 1 : 0);
 }
 
 template <int D, typename OutT>
