@@ -19,7 +19,15 @@
 // so that the sequential pass (state_pass.cu) is left with
 //     S_next = S0 Diag(gamma) + S0 BS^T + NC,   O = Qt S0^T + PU,
 // one tensor-core product per chunk on its critical path.  Nothing here
-// depends on S0: one CTA per (chunk, head), all in parallel.
+// depends on S0: every (chunk, head) item is independent.
+//
+// Structure.  A persistent kernel: as many CTAs as fit (two per SM at d 64,
+// one at d 128) take the items round-robin.  A loader warp requests the next
+// item's q, k, v and log a by 2-D TMA while the current item is finished;
+// the chunk-local cumulative decay (the standalone cumdecay kernel's
+// quantity) is summed in shared memory, for per-channel decay by warps 4-7
+// during the previous item's triangular solve; the record leaves by two bulk
+// stores that drain behind the next item's first phases.
 //
 // Tensor cores.  A and P are decay-weighted K K^T / Q K^T products.  With a
 // per-channel decay (KDA) exp(g[r,c] - g[i,c]) does not factor into a bounded

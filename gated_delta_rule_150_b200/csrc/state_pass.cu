@@ -13,9 +13,11 @@
 //     O = Qt S0^T  (M = 64,  N = d_v, K = d_k)   -> the outputs, off it
 // The fp32 master state stays in registers for the whole run (8 warps; a
 // thread owns half of a state row); S = S * gamma + Z + NC is done in fp32.
-// The outputs of chunk k are added to PU and stored while the MMAs of chunk
-// k+1 run (O is double buffered in tensor memory).  Records arrive by bulk
-// (TMA) copies, prefetched up to kStages chunks ahead.  Snapshots of the state
+// The outputs of chunk k are read from tensor memory before chunk k+1's MMAs
+// are issued, then added to PU and stored while those run.  Each record
+// arrives by one bulk (TMA) copy, prefetched up to kStages chunks ahead, and
+// the next kernel may be launched early (programmatic dependent launch, the
+// single pass only).  Snapshots of the state
 // are written at every snap_interval boundary (section "Co stan
 // rekurencyjny...", point 1: prefix reuse needs the state at that position).
 //
