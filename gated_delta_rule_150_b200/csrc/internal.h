@@ -52,13 +52,6 @@ __host__ __device__ constexpr RecordLayout record_layout(int D) {
                         (uint32_t)(((4 * D * D + 256 * D + 4 * D) + 1023) / 1024 * 1024)};
 }
 
-// Sequence segmentation of the sequential pass.  With few (sequence, head)
-// pairs the chunk-to-chunk chain leaves most SMs idle, so each sequence is cut
-// into segments of seg_chunks chunks: every segment first runs from a zero
-// state while also carrying the identity (its chunks' composed affine map
-// S_end = S_start M + N), a short fp32 chain combines the maps into each
-// segment's true start state, and every segment then replays its chunks from
-// that state to produce its outputs.  seg_chunks == 0 means one pass.
 // Launch, with programmatic stream serialization when `early`: the kernel's
 // CTAs may then be scheduled while the previous kernel in the stream drains,
 // hiding the launch gap.  Every kernel launched here calls pdl_wait()
@@ -86,6 +79,13 @@ inline bool records_fit_l2(int64_t n_slots, int H, int D) {
     return (double)n_slots * H * record_layout(D).bytes <= 96.0 * 1024 * 1024;
 }
 
+// Sequence segmentation of the sequential pass.  With few (sequence, head)
+// pairs the chunk-to-chunk chain leaves most SMs idle, so each sequence is cut
+// into segments of seg_chunks chunks: every segment first runs from a zero
+// state while also carrying the identity (its chunks' composed affine map
+// S_end = S_start M + N), a short fp32 chain combines the maps into each
+// segment's true start state, and every segment then replays its chunks from
+// that state to produce its outputs.  seg_chunks == 0 means one pass.
 inline int segment_chunks(int n_seqs, int H, int64_t T, int D) {
     if (n_seqs <= 0 || T <= 0) return 0;
     const int64_t pairs = (int64_t)n_seqs * H;
@@ -97,7 +97,7 @@ inline int segment_chunks(int n_seqs, int H, int64_t T, int D) {
     if (segs > 32) segs = 32;
     const int64_t avg_chunks = (T / n_seqs + kChunk - 1) / kChunk;
     int64_t sc = (avg_chunks + segs - 1) / segs;
-    if (sc < 8) sc = 8;
+    if (sc < 7) sc = 7;
     if (segs <= 1 || sc >= avg_chunks) return 0;
     return (int)sc;
 }
