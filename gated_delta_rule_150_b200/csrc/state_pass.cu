@@ -408,12 +408,18 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                 }
             }
         }
-        if (ST < 3) fence_proxy_async_smem();   // reads of this stage, then its refill
-        tc_fence_before_sync();
-        if (__syncthreads_or(failed)) { failed = true; break; }
-        if (ST < 3 && tid == 0 && k + ST < nchunks) {
-            issue_copy(k + ST);
-            copies_issued = k + ST + 1;
+        // With two stages this chunk's stage is refilled now, once every
+        // thread has read its PU.  With three or more the refill comes after
+        // the next chunk's first barrier, which orders those reads already,
+        // and no second barrier is needed.
+        if (ST < 3) {
+            fence_proxy_async_smem();         // reads of this stage, then its refill
+            tc_fence_before_sync();
+            if (__syncthreads_or(failed)) { failed = true; break; }
+            if (tid == 0 && k + ST < nchunks) {
+                issue_copy(k + ST);
+                copies_issued = k + ST + 1;
+            }
         }
     }
 
