@@ -39,6 +39,10 @@
  *   - Arguments are checked on the host before anything is launched; a failed
  *     check returns an error status and enqueues nothing.  A launch failure
  *     returns GDR_ERR_CUDA.
+ *   - Stream order holds as for ordinary launches.  Some prefill kernels are
+ *     launched with programmatic stream serialization, so their CTAs may be
+ *     scheduled while the previous kernel on the stream finishes; they touch
+ *     no global memory before that kernel has completed.
  */
 #ifndef GDR_H_
 #define GDR_H_
