@@ -89,7 +89,7 @@ __device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, u
         ::"r"(smem_u32(smem_dst)), "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
 }
 
-// One tiled 2-D TMA load (no multicast) of the box at element coordinates
+// One tiled 2-D TMA load (this CTA only) of the box at element coordinates
 // (x, y) of the tensor map into shared memory, counted on an mbarrier.  x times
 // the element size must be a multiple of 16 bytes.
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* tensor_map, int x, int y,
