@@ -9,6 +9,9 @@ Contents
 --------
 * ``prefill`` / ``decode_step``: the token-by-token recurrence in plain C
   (``gdr_oracle.c``, fp64, OpenMP over (sequence, head)), wrapped with ctypes.
+* ``decode_draft`` / ``decode_accept``: speculative decoding with rollback --
+  K draft tokens that keep the state after each token, then the state of the
+  accepted prefix (same C file).
 * ``cumdecay``: chunk-local inclusive prefix sums of log a (numpy, fp64).
 * ``chunk_factors`` / ``chunked_prefill``: the chunked form of the same
   recurrence written from its definition (numpy, fp64).  It is used to check
@@ -70,6 +73,14 @@ def _load(mutant: int = 0):
             lib.gdr_oracle_decode_step.argtypes = [
                 ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                 _dp, _dp, _dp, _dp, _dp, ctypes.c_int, ctypes.c_double, _dp, _dp]
+            lib.gdr_oracle_decode_draft.restype = ctypes.c_int
+            lib.gdr_oracle_decode_draft.argtypes = [
+                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                _dp, _dp, _dp, _dp, _dp, ctypes.c_int, ctypes.c_double, _dp, _dp, _dp]
+            lib.gdr_oracle_decode_accept.restype = ctypes.c_int
+            lib.gdr_oracle_decode_accept.argtypes = [
+                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                _ip, _dp, _dp]
             lib.gdr_oracle_snapshot_count.restype = ctypes.c_int64
             lib.gdr_oracle_snapshot_count.argtypes = [ctypes.c_int, _ip, ctypes.c_int]
             _LIBS[mutant] = lib
@@ -152,6 +163,48 @@ def decode_step(state, q, k, v, beta, log_a, scalar_decay=False, scale=1.0,
     if rc != 0:
         raise ValueError("oracle decode rejected its arguments")
     return S, o
+
+
+def decode_draft(state, q, k, v, beta, log_a, scalar_decay=False, scale=1.0,
+                 mutant: int = 0):
+    """K draft tokens per sequence for speculative decoding (fp64).
+
+    "Modele hybrydowe ...", section "Co stan rekurencyjny zmienia przy
+    serwowaniu", point 2: the recurrent state absorbs draft tokens, so a
+    rejected draft can only be undone from a state kept before it.  Runs the
+    token update K times from ``state`` [B, H, dv, dk] (not modified) on
+    q, k [B, K, H, dk], v [B, K, H, dv], beta [B, K, H], log_a [B, K, H, dk]
+    (or [B, K, H]).  Returns (o [B, K, H, dv], token_states [B, K, H, dv, dk]),
+    token_states[b, t] being the state after token t.
+    """
+    S = f64(state)
+    q, k, v, beta, log_a = (f64(x) for x in (q, k, v, beta, log_a))
+    B, K, H, dk = q.shape
+    dv = v.shape[3]
+    o = np.zeros((B, K, H, dv))
+    ts = np.zeros((B, K, H, dv, dk))
+    rc = _load(mutant).gdr_oracle_decode_draft(
+        B, K, H, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(log_a),
+        int(bool(scalar_decay)), float(scale), _ptr(S), _ptr(o), _ptr(ts))
+    if rc != 0:
+        raise ValueError("oracle draft decode rejected its arguments")
+    return o, ts
+
+
+def decode_accept(state, token_states, n_accept, mutant: int = 0) -> np.ndarray:
+    """Rollback after verification (same passage as ``decode_draft``): the
+    state of sequence b becomes token_states[b, n - 1] for n = n_accept[b] in
+    1 .. K and stays ``state[b]`` for n = 0 (n clamped to [0, K]).  Returns
+    the new state; the input is not modified."""
+    S = f64(state).copy()
+    ts = f64(token_states)
+    n = _i32(n_accept)
+    B, K, H, dv, dk = ts.shape
+    rc = _load(mutant).gdr_oracle_decode_accept(B, K, H, dk, dv, n.ctypes.data_as(_ip),
+                                                _ptr(ts), _ptr(S))
+    if rc != 0:
+        raise ValueError("oracle decode accept rejected its arguments")
+    return S
 
 
 # ---------------------------------------------------------------------------

@@ -35,12 +35,20 @@
  *   - section "Co stan rekurencyjny zmienia przy serwowaniu", point 1: a prefix
  *     can only be reused from a snapshot of the state taken at that position,
  *     so the state after every full snap_interval tokens of a sequence is
- *     copied out.
+ *     copied out;
+ *   - the same section, point 2: speculative decoding needs a real rollback,
+ *     because the state has already absorbed the rejected draft tokens, so a
+ *     draft of K tokens keeps the state after each of them and accepting n of
+ *     them restores the state kept after token n.
  *
  * Layouts (row-major, token-major, sequences packed by cu_seqlens):
  *   q, k [T, H, dk]  v [T, H, dv]  beta [T, H]  log_a [T, H, dk] or [T, H]
  *   o [T, H, dv]  init_state / final_state [N, H, dv, dk]
  *   snapshots [sum_n floor(L_n / snap_interval), H, dv, dk], sequence-major.
+ *
+ * Draft decode: q, k [B, K, H, dk]  v [B, K, H, dv]  beta [B, K, H]
+ *   log_a [B, K, H, dk] or [B, K, H]  o [B, K, H, dv]
+ *   token_states [B, K, H, dv, dk]: the state after token t of sequence b.
  *
  * GDR_ORACLE_MUTANT (compile-time, default 0) plants one deliberate mistake;
  * it exists only so that the pin tests can show that each plausible mistake
@@ -234,6 +242,73 @@ int gdr_oracle_decode_step(int B, int H, int dk, int dv, const double* q, const 
                     o + (size_t)pair * dv, tmp);
         free(a);
         free(tmp);
+    }
+    return 0;
+}
+
+/*
+ * Draft decode for speculative decoding: K tokens per sequence from `state`
+ * (not modified), keeping the state after every token in token_states.
+ * Each token is the same update as above.
+ */
+int gdr_oracle_decode_draft(int B, int K, int H, int dk, int dv, const double* q,
+                            const double* k, const double* v, const double* beta,
+                            const double* log_a, int scalar_decay, double scale,
+                            const double* state, double* o, double* token_states)
+{
+    int pair;
+    if (B < 0 || K < 0 || H <= 0 || dk <= 0 || dv <= 0) return -1;
+#pragma omp parallel for schedule(static)
+    for (pair = 0; pair < B * H; ++pair) {
+        int b = pair / H, h = pair % H, t, c;
+        size_t sz = (size_t)dv * (size_t)dk;
+        double* S = (double*)malloc(sizeof(double) * sz);
+        double* a = (double*)malloc(sizeof(double) * (size_t)dk);
+        double* tmp = (double*)malloc(sizeof(double) * (size_t)dv);
+        memcpy(S, state + (size_t)pair * sz, sizeof(double) * sz);
+        for (t = 0; t < K; ++t) {
+            size_t th = ((size_t)b * K + t) * H + h;     /* token t of sequence b, head h */
+            for (c = 0; c < dk; ++c)
+                a[c] = exp(scalar_decay ? log_a[th] : log_a[th * dk + c]);
+#if GDR_ORACLE_MUTANT == 11
+            /* mutant: keeps the state from before the token */
+            memcpy(token_states + th * sz, S, sizeof(double) * sz);
+#endif
+            oracle_step(dk, dv, S, q + th * dk, k + th * dk, v + th * dv, beta[th], a, scale,
+                        o + th * dv, tmp);
+#if GDR_ORACLE_MUTANT != 11
+            memcpy(token_states + th * sz, S, sizeof(double) * sz);
+#endif
+        }
+        free(S);
+        free(a);
+        free(tmp);
+    }
+    return 0;
+}
+
+/*
+ * Accept n_accept[b] of the K draft tokens of sequence b: its state becomes
+ * the state kept after token n (n = 1 .. K) and stays as it is for n = 0.
+ * n_accept is clamped to [0, K].
+ */
+int gdr_oracle_decode_accept(int B, int K, int H, int dk, int dv, const int32_t* n_accept,
+                             const double* token_states, double* state)
+{
+    int b, h;
+    size_t sz = (size_t)dv * (size_t)dk;
+    if (B < 0 || K < 0 || H <= 0 || dk <= 0 || dv <= 0) return -1;
+    for (b = 0; b < B; ++b) {
+        int n = n_accept[b] < 0 ? 0 : (n_accept[b] > K ? K : n_accept[b]);
+#if GDR_ORACLE_MUTANT == 12
+        int pick = n < K ? n : K - 1;                /* mutant: one token too far */
+#else
+        int pick = n - 1;
+#endif
+        if (n == 0) continue;
+        for (h = 0; h < H; ++h)
+            memcpy(state + ((size_t)b * H + h) * sz,
+                   token_states + (((size_t)b * K + pick) * H + h) * sz, sizeof(double) * sz);
     }
     return 0;
 }

@@ -4,7 +4,7 @@ None of these re-types the oracle's own loop: each compares it with an
 independent statement of the result (a closed form, a reduction to a simpler
 rule, a dense product of transition matrices, a printed worked example, or an
 invariance that any correct implementation must satisfy).  The last test
-plants each of ten plausible mistakes in the oracle (compile-time mutants of
+plants each of twelve plausible mistakes in the oracle (compile-time mutants of
 the C source) and checks that at least one pin rejects every one of them.
 """
 import json
@@ -255,9 +255,79 @@ def pin_scalar_is_broadcast(mutant=0):
     np.testing.assert_array_equal(a["final_state"], b["final_state"])
 
 
+def _draft_inputs(r, B, K, H, dk, dv, scalar=False):
+    q = r.standard_normal((B, K, H, dk))
+    k = _unit(r.standard_normal((B, K, H, dk)))
+    v = r.standard_normal((B, K, H, dv))
+    beta = r.random((B, K, H))
+    la = -0.4 * r.random((B, K, H) if scalar else (B, K, H, dk))
+    S = r.standard_normal((B, H, dv, dk))
+    return q, k, v, beta, la, S
+
+
+def pin_draft_keeps_every_state(mutant=0):
+    """Modele hybrydowe, "Co stan rekurencyjny zmienia przy serwowaniu",
+    point 2: a draft of K tokens keeps the state after each token.  Draft
+    sequence b must equal a prefill of its K tokens from state[b] with a
+    snapshot after every token (the snapshot rule is pinned on its own above):
+    the kept states are those snapshots and the outputs are the prefill's."""
+    r = _rng(12)
+    B, K, H, dk, dv = 3, 5, 2, 4, 3
+    for scalar in (False, True):
+        q, k, v, beta, la, S = _draft_inputs(r, B, K, H, dk, dv, scalar)
+        o, ts = oracle.decode_draft(S, q, k, v, beta, la, scalar_decay=scalar, scale=0.5,
+                                    mutant=mutant)
+        assert o.shape == (B, K, H, dv) and ts.shape == (B, K, H, dv, dk)
+        for b in range(B):
+            ref = oracle.prefill(q[b], k[b], v[b], beta[b], la[b], [0, K], scalar_decay=scalar,
+                                 scale=0.5, init_state=S[b:b + 1], snap_interval=1,
+                                 mutant=mutant)
+            np.testing.assert_allclose(ts[b], ref["snapshots"], rtol=1e-12, atol=1e-12)
+            np.testing.assert_allclose(o[b], ref["o"], rtol=1e-12, atol=1e-12)
+
+
+def pin_draft_frozen(mutant=0):
+    """With beta = 0 every draft token only decays the state (as in
+    pin_frozen_state): kept state t = S Diag(exp(sum_{i<=t} log a_i)) and
+    o_t = (kept state t) (scale q_t), in closed form."""
+    r = _rng(13)
+    B, K, H, dk, dv = 2, 4, 3, 5, 4
+    q, k, v, beta, la, S = _draft_inputs(r, B, K, H, dk, dv)
+    beta[:] = 0.0
+    o, ts = oracle.decode_draft(S, q, k, v, beta, la, scale=2.0, mutant=mutant)
+    G = np.cumsum(la, axis=1)                                  # [B, K, H, dk]
+    ts_ref = S[:, None] * np.exp(G)[:, :, :, None, :]          # [B, K, H, dv, dk]
+    np.testing.assert_allclose(ts, ts_ref, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(o, np.einsum("bthjc,bthc->bthj", ts_ref, 2.0 * q),
+                               rtol=1e-12, atol=1e-12)
+
+
+def pin_rollback(mutant=0):
+    """Same passage: accepting n of the K draft tokens leaves exactly the
+    state that n single decode steps give (decode steps are pinned against
+    prefill above); n = 0 gives back the state before the draft bitwise;
+    n outside [0, K] is clamped."""
+    r = _rng(14)
+    B, K, H, d = 6, 4, 2, 4
+    q, k, v, beta, la, S = _draft_inputs(r, B, K, H, d, d)
+    _, ts = oracle.decode_draft(S, q, k, v, beta, la, mutant=mutant)
+    n_acc = np.array([0, 1, 2, K, K + 3, -2], dtype=np.int32)
+    out = oracle.decode_accept(S, ts, n_acc, mutant=mutant)
+    for b in range(B):
+        n = min(max(int(n_acc[b]), 0), K)
+        ref = S[b:b + 1].copy()
+        for t in range(n):
+            ref, _ = oracle.decode_step(ref, q[b:b + 1, t], k[b:b + 1, t], v[b:b + 1, t],
+                                        beta[b:b + 1, t], la[b:b + 1, t], mutant=mutant)
+        if n == 0:
+            np.testing.assert_array_equal(out[b], S[b])
+        else:
+            np.testing.assert_allclose(out[b], ref[0], rtol=1e-12, atol=1e-12)
+
+
 PINS = [pin_exact_retrieval, pin_frozen_state, pin_linear_attention, pin_brute_force,
         pin_snapshots, pin_split_and_varlen, pin_decay_magnitude, pin_decode_equals_prefill,
-        pin_scalar_is_broadcast]
+        pin_scalar_is_broadcast, pin_draft_keeps_every_state, pin_draft_frozen, pin_rollback]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda p: p.__name__)
@@ -331,15 +401,16 @@ def test_cumdecay_restarts_per_chunk():
         np.testing.assert_allclose(np.exp(g[t]), np.prod(np.exp(la[s:t + 1]), axis=0), rtol=1e-12)
 
 
-MUTANTS = list(range(1, 11))
+MUTANTS = list(range(1, 13))
 
 
 @pytest.mark.parametrize("mutant", MUTANTS)
 def test_every_planted_mistake_is_caught(mutant):
     """Each compile-time mutant of the C oracle (wrong read order, decay on
     the wrong axis, sign, dropped beta, q/k swap, decay after the update,
-    snapshot off by one, wrong head's gate, transposed state) must fail at
-    least one pin."""
+    snapshot off by one, wrong head's gate, transposed state, draft keeping
+    the state from before each token, rollback one token too far) must fail
+    at least one pin."""
     caught = []
     for pin in PINS:
         try:
