@@ -13,6 +13,9 @@ collective on the data path).  The same run also measures:
 * ``decode``: the decode step on 256 sequences x 14 heads x 64 x 64 fp32 states,
   state bytes streamed per second (four state sets rotated so that the 235 MB
   working set exceeds the 126 MB L2);
+* ``spec_decode``: speculative decoding on the same sequences: a draft of 4
+  tokens that keeps the state after each token, then the accept (rollback)
+  step, each timed alone and as one verify cycle;
 * ``roofline``: the step's dominant kernel, timed alone with CUDA events;
 * ``e2e``: the same prefill through the public API with pinned host buffers,
   host<->device copies inside the timed region;
@@ -70,6 +73,13 @@ def prefill_state_bytes(n_seqs: int, H: int, d_k: int, d_v: int, has_init: bool,
 def decode_bytes_per_head_state(d_k: int, d_v: int, elem: int, scalar: bool) -> int:
     """state read + written (fp32), q, k, v, beta, log_a read, o (fp32) written."""
     return 2 * 4 * d_k * d_v + (2 * d_k + d_v) * elem + 4 + (4 if scalar else 4 * d_k) + 4 * d_v
+
+
+def draft_bytes_per_head_state(d_k: int, d_v: int, elem: int, scalar: bool, K: int) -> int:
+    """state read once (fp32); per draft token the kept state written (fp32),
+    q, k, v, beta, log_a read and o (fp32) written."""
+    tok = (2 * d_k + d_v) * elem + 4 + (4 if scalar else 4 * d_k) + 4 * d_v
+    return 4 * d_k * d_v + K * (4 * d_k * d_v + tok)
 
 
 def peaks() -> dict:
@@ -383,8 +393,10 @@ def run_gdr(args):
 
     extra = {}
     decode = None
+    spec = None
     if not args.no_extra:
         decode = bench_decode(gdr, stream, pk, args)
+        spec = bench_spec_decode(gdr, stream, pk, args)
         for w in (wl.TINY_KDA, wl.GDN_LONG, wl.VARLEN):
             extra[w.name] = bench_prefill_workload(gdr, w, stream, pk, rank, args)
     e2e = bench_e2e(gdr, stream, args)
@@ -406,6 +418,7 @@ def run_gdr(args):
         "path_roofline": path_roof,
         "kernel_ms": stage_report,
         "decode": decode,
+        "spec_decode": spec,
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
@@ -465,6 +478,64 @@ def bench_decode(gdr, stream, pk, args):
     return res
 
 
+def bench_spec_decode(gdr, stream, pk, args):
+    """Draft (K kept states) and accept on the draft workload, four rotating
+    state sets; the kept states (235 MB per draft) exceed L2 on their own."""
+    w = wl.SPEC_DRAFT
+    d = w.decode
+    K, B, H = w.draft_tokens, d.batch, d.n_heads
+    inp = wl.make_draft_inputs(w, device="cuda", draw_device="cuda")
+    states = [inp["state"].clone() for _ in range(4)]
+    o = torch.empty(B, K, H, d.d_v, device="cuda")
+    ts = torch.empty(B, K, H, d.d_v, d.d_k, device="cuda")
+
+    def draft(i):
+        r = i % w.rounds
+        gdr.decode_draft(states[i % 4], inp["q"][r], inp["k"][r], inp["v"][r], inp["beta"][r],
+                         inp["log_a"][r], scalar_decay=d.scalar_decay, scale=d.scale, out=o,
+                         token_states=ts)
+
+    def accept(i):
+        gdr.decode_accept(states[i % 4], ts, inp["n_accept"][i % w.rounds])
+
+    def cycle(i):
+        draft(i)
+        accept(i)
+
+    for i in range(8):
+        cycle(i)
+    n = 256
+    ms_d = timed(draft, n, stream)
+    ms_a = timed(accept, n, stream)
+    ms_c = timed(cycle, n, stream)
+    elem = 2 if d.qkv_dtype == torch.bfloat16 else 4
+    units = B * H
+    per = draft_bytes_per_head_state(d.d_k, d.d_v, elem, d.scalar_decay, K)
+    gbs_d = per * units / (ms_d * 1e-3) / 1e9
+    # accept: n_accept read per sequence; a state copied (read + write) per
+    # head of every sequence that accepted at least one token
+    acc_frac = float((inp["n_accept"] > 0).float().mean())
+    acc_bytes = 4 * B + acc_frac * units * 8 * d.d_k * d.d_v
+    gbs_a = acc_bytes / (ms_a * 1e-3) / 1e9
+    accepted = float(inp["n_accept"].float().mean()) * B
+    res = {"workload": w.name, "draft_tokens": K,
+           "draft": {"ms": round(ms_d, 5), "gbs": round(gbs_d, 1),
+                     "bytes_per_head_state": per,
+                     "roofline": {"bound": "hbm", "achieved": round(gbs_d, 1),
+                                  "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                  "frac": round(gbs_d / pk["hbm_gbs"], 4),
+                                  "traffic": recorded_traffic("decode_draft", w.name)}},
+           "accept": {"ms": round(ms_a, 5), "gbs": round(gbs_a, 1),
+                      "accepting_fraction": round(acc_frac, 4)},
+           "cycle_ms": round(ms_c, 5),
+           "accepted_tokens_per_s": round(accepted / (ms_c * 1e-3), 1),
+           "l2": "4 rotating state sets; kept states 235 MB per draft > 126 MB L2",
+           "cycles": n}
+    del inp, states, ts
+    torch.cuda.empty_cache()
+    return res
+
+
 def bench_e2e(gdr, stream, args):
     """Prefill through the public API from pinned host buffers: H2D of the
     inputs, the prefill, D2H of o and the final state, every step."""
@@ -509,6 +580,8 @@ def main():
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     p.add_argument("--only-decode", action="store_true",
                    help="run only the decode measurement (for profiling)")
+    p.add_argument("--only-spec", action="store_true",
+                   help="run only the speculative-decoding measurement (for profiling)")
     p.add_argument("--workload", default=wl.GRAFT_LAYER.name,
                    choices=sorted(wl.PREFILL_WORKLOADS) + sorted(wl.PROFILE_CASES),
                    help="prefill workload of the main line (default: the graft layer)")
@@ -523,6 +596,11 @@ def main():
         import gated_delta_rule_150_b200 as gdr
         gdr.lib()
         print(json.dumps(bench_decode(gdr, torch.cuda.current_stream(), peaks(), args)), flush=True)
+    elif args.only_spec:
+        import gated_delta_rule_150_b200 as gdr
+        gdr.lib()
+        print(json.dumps(bench_spec_decode(gdr, torch.cuda.current_stream(), peaks(), args)),
+              flush=True)
     else:
         run_gdr(args)
 

@@ -19,7 +19,8 @@ import threading
 
 import torch
 
-__all__ = ["PrefillArgs", "PreparedPrefill", "prefill", "kernel_count", "decode_step", "cumdecay", "chunk_factors", "workspace_size",
+__all__ = ["PrefillArgs", "PreparedPrefill", "prefill", "kernel_count", "decode_step",
+           "decode_draft", "decode_accept", "cumdecay", "chunk_factors", "workspace_size",
            "snapshot_count", "prefill_status", "lib", "GdrError", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_build", "libgdr.so")
@@ -86,6 +87,11 @@ def lib():
             L.gdr_chunk_factors.argtypes = [ctypes.POINTER(PrefillArgs), vp, vp, vp, vp, vp, vp]
             L.gdr_decode_step.restype = i
             L.gdr_decode_step.argtypes = [i, i, i, i, i, vp, vp, vp, vp, vp, i, f, vp, vp, vp]
+            L.gdr_decode_draft.restype = i
+            L.gdr_decode_draft.argtypes = [i, i, i, i, i, i, vp, vp, vp, vp, vp, i, f, vp, vp,
+                                           vp, vp]
+            L.gdr_decode_accept.restype = i
+            L.gdr_decode_accept.argtypes = [i, i, i, i, i, vp, vp, vp, vp]
             _LIB = L
         return _LIB
 
@@ -305,3 +311,49 @@ def decode_step(state, q, k, v, beta, log_a, *, scalar_decay=False, scale=1.0, o
                                  _ptr(state), _ptr(out), _stream(q.device)),
            "gdr_decode_step")
     return out
+
+
+def decode_draft(state, q, k, v, beta, log_a, *, scalar_decay=False, scale=1.0, out=None,
+                 token_states=None):
+    """K draft tokens per sequence for speculative decoding.
+
+    ``state`` [B, H, d_v, d_k] fp32 is read, not modified.  q, k [B, K, H, d_k],
+    v [B, K, H, d_v], beta [B, K, H], log_a [B, K, H, d_k] (or [B, K, H]).
+    Returns (o [B, K, H, d_v] fp32, token_states [B, K, H, d_v, d_k] fp32),
+    token_states[b, t] being the state after token t of sequence b.
+    """
+    if q.dtype != k.dtype or q.dtype != v.dtype:
+        raise TypeError("q, k and v must share a dtype")
+    _need_cuda(state, q, k, v, beta, log_a, out, token_states)
+    if state.dtype != torch.float32:
+        raise TypeError("state must be float32")
+    B, K, H, dk = q.shape
+    dv = v.shape[-1]
+    if tuple(state.shape) != (B, H, dv, dk):
+        raise ValueError(f"state must be [B, H, d_v, d_k] = {(B, H, dv, dk)}")
+    if out is None:
+        out = torch.empty(B, K, H, dv, dtype=torch.float32, device=q.device)
+    if token_states is None:
+        token_states = torch.empty(B, K, H, dv, dk, dtype=torch.float32, device=q.device)
+    _check(lib().gdr_decode_draft(B, K, H, dk, dv, _dtype_code(q), _ptr(q), _ptr(k), _ptr(v),
+                                  _ptr(beta), _ptr(log_a), int(bool(scalar_decay)), float(scale),
+                                  _ptr(state), _ptr(out), _ptr(token_states), _stream(q.device)),
+           "gdr_decode_draft")
+    return out, token_states
+
+
+def decode_accept(state, token_states, n_accept):
+    """Rollback after verification, in place: ``state[b]`` becomes
+    ``token_states[b, n - 1]`` for n = n_accept[b] in 1 .. K and is left as it
+    is for n = 0 (n clamped to [0, K]).  ``n_accept`` is a device int32 [B]."""
+    _need_cuda(state, token_states, n_accept)
+    if n_accept.dtype != torch.int32:
+        raise TypeError("n_accept must be int32")
+    B, K, H, dv, dk = token_states.shape
+    if tuple(state.shape) != (B, H, dv, dk) or n_accept.numel() != B:
+        raise ValueError("state must be [B, H, d_v, d_k] and n_accept [B] for token_states "
+                         "[B, K, H, d_v, d_k]")
+    _check(lib().gdr_decode_accept(B, K, H, dk, dv, _ptr(n_accept), _ptr(token_states),
+                                   _ptr(state), _stream(state.device)),
+           "gdr_decode_accept")
+    return state

@@ -190,4 +190,41 @@ gdr_status gdr_decode_step(int batch, int n_heads, int d_k, int d_v, gdr_dtype q
                                         static_cast<cudaStream_t>(stream)));
 }
 
+gdr_status gdr_decode_draft(int batch, int n_tokens, int n_heads, int d_k, int d_v,
+                            gdr_dtype qkv_dtype, const void* q, const void* k, const void* v,
+                            const float* beta, const float* log_a, int scalar_decay, float scale,
+                            const float* state, float* o, float* token_states, void* stream) {
+    if (batch < 0 || n_tokens < 0 || n_heads <= 0 || d_k <= 0 || d_v <= 0)
+        return GDR_ERR_INVALID_ARG;
+    if (qkv_dtype != GDR_BF16 && qkv_dtype != GDR_F32) return GDR_ERR_INVALID_ARG;
+    if (!supported_width(d_k) || !supported_width(d_v)) return GDR_ERR_UNSUPPORTED;
+    if ((int64_t)batch * n_heads > (int64_t)INT32_MAX) return GDR_ERR_INVALID_ARG;
+    if (batch == 0 || n_tokens == 0) return GDR_OK;
+    const void* vec[] = {q, k, state, token_states};
+    for (const void* p : vec)
+        if (!p || !aligned16(p)) return GDR_ERR_INVALID_ARG;
+    if (!v || !aligned_elem(v, qkv_dtype) || !beta || !aligned4(beta) || !o || !aligned4(o))
+        return GDR_ERR_INVALID_ARG;
+    if (!log_a || !(scalar_decay ? aligned4(log_a) : aligned16(log_a))) return GDR_ERR_INVALID_ARG;
+    return from_cuda(gdr::launch_decode_draft(batch, n_tokens, n_heads, d_k, d_v, qkv_dtype, q, k,
+                                              v, beta, log_a, scalar_decay, scale, state, o,
+                                              token_states, static_cast<cudaStream_t>(stream)));
+}
+
+gdr_status gdr_decode_accept(int batch, int n_tokens, int n_heads, int d_k, int d_v,
+                             const int32_t* n_accept, const float* token_states, float* state,
+                             void* stream) {
+    if (batch < 0 || n_tokens < 0 || n_heads <= 0 || d_k <= 0 || d_v <= 0)
+        return GDR_ERR_INVALID_ARG;
+    if (!supported_width(d_k) || !supported_width(d_v)) return GDR_ERR_UNSUPPORTED;
+    if ((int64_t)batch * n_heads > (int64_t)INT32_MAX) return GDR_ERR_INVALID_ARG;
+    if (batch == 0 || n_tokens == 0) return GDR_OK;
+    if (!n_accept || !aligned4(n_accept)) return GDR_ERR_INVALID_ARG;
+    if (!token_states || !aligned16(token_states) || !state || !aligned16(state))
+        return GDR_ERR_INVALID_ARG;
+    return from_cuda(gdr::launch_decode_accept(batch, n_tokens, n_heads, d_k, d_v, n_accept,
+                                               token_states, state,
+                                               static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -155,6 +155,14 @@ cudaError_t launch_decode(int B, int H, int dk, int dv, gdr_dtype dt, const void
                           const float* log_a, int scalar, float scale, float* state,
                           float* o, cudaStream_t st);
 
+cudaError_t launch_decode_draft(int B, int K, int H, int dk, int dv, gdr_dtype dt, const void* q,
+                                const void* k, const void* v, const float* beta,
+                                const float* log_a, int scalar, float scale, const float* state,
+                                float* o, float* token_states, cudaStream_t st);
+
+cudaError_t launch_decode_accept(int B, int K, int H, int dk, int dv, const int32_t* n_accept,
+                                 const float* token_states, float* state, cudaStream_t st);
+
 // Device helper: slot -> (sequence, chunk index).  f(n) = floor(cu[n]/64) + n is
 // strictly increasing, so the owner of slot j is the largest n with f(n) <= j.
 // Returns false if the slot holds no chunk.

@@ -1,0 +1,239 @@
+// spec_decode.cu -- draft decode with per-token state retention, and rollback.
+//
+// "Modele hybrydowe: co Gated DeltaNet zastępuje w cache KV", section "Co stan
+// rekurencyjny zmienia przy serwowaniu", point 2: a KV cache drops the
+// entries of rejected draft tokens, but a recurrent state has already
+// absorbed them, so speculative decoding needs the state from before the
+// rejected tokens back.  The draft kernel runs K decode tokens per sequence
+// from a read-only state and stores the state after every token; the accept
+// kernel then copies, per sequence, the state after its last accepted token
+// into the live state (or leaves it alone when nothing was accepted).
+//
+// Each token is the decode update of the KDA step ("kda-graft", section
+// "2. Decode: O(1) против O(L)"), per state row j (value channel):
+//     s' = s * a,  p = s' . k,  c = s' . (scale q),  d = beta (v_j - p)
+//     s  = s' + d k,  o_j = c + d (k . scale q)
+// The state rows stay in registers across the K tokens: the kernel reads the
+// state once and writes it K times, so it is HBM-bound on
+// (1 + K) * 4 d_v d_k bytes per head-state plus the tokens' inputs.
+#include <cuda_bf16.h>
+
+#include "internal.h"
+
+namespace gdr {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kTPR = 16;                      // threads per state row
+constexpr int kRowsPerPass = kThreads / kTPR; // 16 rows at a time
+
+template <typename T>
+__device__ __forceinline__ float to_f(T x);
+template <>
+__device__ __forceinline__ float to_f<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+__device__ __forceinline__ float4 load4(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
+__device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
+    const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+}
+
+__device__ __forceinline__ float sum16(float x) {
+#pragma unroll
+    for (int m = 8; m >= 1; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
+    return x;
+}
+
+// One token's inputs as seen by one thread: its float4 columns of k, q and
+// log a, the v entries of its rows, and beta.
+template <typename T, int DK, int DV, bool SCALAR>
+struct TokenIn {
+    static constexpr int NV = DK / (4 * kTPR);
+    static constexpr int PASSES = DV / kRowsPerPass;
+    float4 k[NV], q[NV], la[NV];
+    float v[PASSES];
+    float beta;
+
+    __device__ __forceinline__ void load(const T* __restrict__ q_, const T* __restrict__ k_,
+                                         const T* __restrict__ v_, const float* __restrict__ beta_,
+                                         const float* __restrict__ log_a_, size_t tok, int lane16,
+                                         int rgrp) {
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            const int c = 4 * (lane16 + kTPR * i);
+            k[i] = load4(k_ + tok * DK + c);
+            q[i] = load4(q_ + tok * DK + c);
+            if (SCALAR) {
+                const float x = __ldg(log_a_ + tok);
+                la[i] = make_float4(x, x, x, x);
+            } else {
+                la[i] = load4(log_a_ + tok * DK + c);
+            }
+        }
+#pragma unroll
+        for (int p = 0; p < PASSES; ++p) v[p] = to_f<T>(v_[tok * DV + rgrp + kRowsPerPass * p]);
+        beta = __ldg(beta_ + tok);
+    }
+};
+
+// One CTA per (sequence b, head h).  Thread t owns rows t / 16 + 16 p and the
+// float4 columns {t % 16 + 16 i} of the state for all K tokens.  Token t of
+// sequence b is input row (b K + t) H + h of q, k, v, beta, log a, o and
+// token_states; the next token's inputs are loaded while this one computes.
+template <typename T, int DK, int DV, bool SCALAR>
+__global__ void __launch_bounds__(kThreads)
+decode_draft_kernel(int H, int K, const T* __restrict__ q, const T* __restrict__ k,
+                    const T* __restrict__ v, const float* __restrict__ beta,
+                    const float* __restrict__ log_a, float scale, const float* __restrict__ state,
+                    float* __restrict__ o, float* __restrict__ token_states) {
+    using Tok = TokenIn<T, DK, DV, SCALAR>;
+    constexpr int NV = Tok::NV;
+    constexpr int PASSES = Tok::PASSES;
+    const int bh = blockIdx.x;
+    const int b = bh / H;
+    const int h = bh - b * H;
+    const int lane16 = threadIdx.x % kTPR;
+    const int rgrp = threadIdx.x / kTPR;
+
+    const size_t tok0 = (size_t)b * K * H + h;
+    Tok nxt;
+    nxt.load(q, k, v, beta, log_a, tok0, lane16, rgrp);
+
+    const float* S0 = state + (size_t)bh * DV * DK;
+    float4 s[PASSES][NV];
+#pragma unroll
+    for (int p = 0; p < PASSES; ++p)
+#pragma unroll
+        for (int i = 0; i < NV; ++i)
+            s[p][i] = __ldg(reinterpret_cast<const float4*>(
+                S0 + (size_t)(rgrp + kRowsPerPass * p) * DK + 4 * (lane16 + kTPR * i)));
+
+#pragma unroll 1
+    for (int t = 0; t < K; ++t) {
+        const Tok cur = nxt;
+        const size_t tok = tok0 + (size_t)t * H;
+        if (t + 1 < K) nxt.load(q, k, v, beta, log_a, tok + H, lane16, rgrp);
+
+        float4 aa[NV], qq[NV];
+        float kq_part = 0.f;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            aa[i] = make_float4(expf(cur.la[i].x), expf(cur.la[i].y), expf(cur.la[i].z),
+                                expf(cur.la[i].w));
+            qq[i] = make_float4(cur.q[i].x * scale, cur.q[i].y * scale, cur.q[i].z * scale,
+                                cur.q[i].w * scale);
+            kq_part += cur.k[i].x * qq[i].x + cur.k[i].y * qq[i].y + cur.k[i].z * qq[i].z +
+                       cur.k[i].w * qq[i].w;
+        }
+        const float kq = sum16(kq_part);
+
+        float* St = token_states + tok * DV * DK;
+#pragma unroll
+        for (int p = 0; p < PASSES; ++p) {
+            const int row = rgrp + kRowsPerPass * p;
+            float pk = 0.f, pq = 0.f;
+#pragma unroll
+            for (int i = 0; i < NV; ++i) {
+                float4& x = s[p][i];
+                x.x *= aa[i].x; x.y *= aa[i].y; x.z *= aa[i].z; x.w *= aa[i].w;
+                pk += x.x * cur.k[i].x + x.y * cur.k[i].y + x.z * cur.k[i].z + x.w * cur.k[i].w;
+                pq += x.x * qq[i].x + x.y * qq[i].y + x.z * qq[i].z + x.w * qq[i].w;
+            }
+            pk = sum16(pk);
+            pq = sum16(pq);
+            const float d = cur.beta * (cur.v[p] - pk);
+#pragma unroll
+            for (int i = 0; i < NV; ++i) {
+                float4& x = s[p][i];
+                x.x += d * cur.k[i].x; x.y += d * cur.k[i].y;
+                x.z += d * cur.k[i].z; x.w += d * cur.k[i].w;
+                // kept states are written once and mostly never read again
+                __stcs(reinterpret_cast<float4*>(St + (size_t)row * DK + 4 * (lane16 + kTPR * i)), x);
+            }
+            if (lane16 == 0) o[tok * DV + row] = pq + d * kq;
+        }
+    }
+}
+
+// One CTA per (sequence b, head h): state[b, h] = token_states[b, n - 1, h]
+// with n = n_accept[b] clamped to [0, K]; nothing happens for n = 0.
+__global__ void __launch_bounds__(kThreads)
+decode_accept_kernel(int H, int K, int n4, const int32_t* __restrict__ n_accept,
+                     const float* __restrict__ token_states, float* __restrict__ state) {
+    const int bh = blockIdx.x;
+    const int b = bh / H;
+    const int h = bh - b * H;
+    int n = __ldg(n_accept + b);
+    n = n < 0 ? 0 : (n > K ? K : n);
+    if (n == 0) return;
+    const float4* src = reinterpret_cast<const float4*>(token_states) +
+                        (((size_t)b * K + (n - 1)) * H + h) * (size_t)n4;
+    float4* dst = reinterpret_cast<float4*>(state) + (size_t)bh * n4;
+    constexpr int kUnroll = 4;
+    for (int base = threadIdx.x; base < n4; base += kThreads * kUnroll) {
+        float4 x[kUnroll];
+#pragma unroll
+        for (int j = 0; j < kUnroll; ++j) {
+            const int i = base + j * kThreads;
+            if (i < n4) x[j] = __ldcs(src + i);
+        }
+#pragma unroll
+        for (int j = 0; j < kUnroll; ++j) {
+            const int i = base + j * kThreads;
+            if (i < n4) dst[i] = x[j];
+        }
+    }
+}
+
+template <typename T, int DK, int DV>
+cudaError_t draft_typed(int B, int K, int H, const void* q, const void* k, const void* v,
+                        const float* beta, const float* log_a, int scalar, float scale,
+                        const float* state, float* o, float* ts, cudaStream_t st) {
+    const dim3 grid((unsigned)(B * H));
+    if (scalar)
+        decode_draft_kernel<T, DK, DV, true><<<grid, kThreads, 0, st>>>(
+            H, K, (const T*)q, (const T*)k, (const T*)v, beta, log_a, scale, state, o, ts);
+    else
+        decode_draft_kernel<T, DK, DV, false><<<grid, kThreads, 0, st>>>(
+            H, K, (const T*)q, (const T*)k, (const T*)v, beta, log_a, scale, state, o, ts);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t draft_dims(int B, int K, int H, int dk, int dv, const void* q, const void* k,
+                       const void* v, const float* beta, const float* log_a, int scalar,
+                       float scale, const float* state, float* o, float* ts, cudaStream_t st) {
+    if (dk == 64 && dv == 64)
+        return draft_typed<T, 64, 64>(B, K, H, q, k, v, beta, log_a, scalar, scale, state, o, ts, st);
+    if (dk == 64 && dv == 128)
+        return draft_typed<T, 64, 128>(B, K, H, q, k, v, beta, log_a, scalar, scale, state, o, ts, st);
+    if (dk == 128 && dv == 64)
+        return draft_typed<T, 128, 64>(B, K, H, q, k, v, beta, log_a, scalar, scale, state, o, ts, st);
+    return draft_typed<T, 128, 128>(B, K, H, q, k, v, beta, log_a, scalar, scale, state, o, ts, st);
+}
+
+}  // namespace
+
+cudaError_t launch_decode_draft(int B, int K, int H, int dk, int dv, gdr_dtype dt, const void* q,
+                                const void* k, const void* v, const float* beta,
+                                const float* log_a, int scalar, float scale, const float* state,
+                                float* o, float* token_states, cudaStream_t st) {
+    if (dt == GDR_BF16)
+        return draft_dims<__nv_bfloat16>(B, K, H, dk, dv, q, k, v, beta, log_a, scalar, scale,
+                                         state, o, token_states, st);
+    return draft_dims<float>(B, K, H, dk, dv, q, k, v, beta, log_a, scalar, scale, state, o,
+                             token_states, st);
+}
+
+cudaError_t launch_decode_accept(int B, int K, int H, int dk, int dv, const int32_t* n_accept,
+                                 const float* token_states, float* state, cudaStream_t st) {
+    decode_accept_kernel<<<(unsigned)(B * H), kThreads, 0, st>>>(H, K, dk * dv / 4, n_accept,
+                                                                 token_states, state);
+    return cudaGetLastError();
+}
+
+}  // namespace gdr

@@ -230,6 +230,52 @@ gdr_status gdr_decode_step(int batch, int n_heads, int d_k, int d_v, gdr_dtype q
                            const float* log_a, int scalar_decay, float scale, float* state,
                            float* o, void* stream);
 
+/* ------------------------------------------------------------------------
+ * Speculative decoding with rollback ("Modele hybrydowe", section "Co stan
+ * rekurencyjny zmienia przy serwowaniu", point 2: a KV cache drops rejected
+ * draft tokens, but the recurrent state has already absorbed them, so the
+ * engine needs the state from before them back).  A draft runs K tokens per
+ * sequence from a state it does not modify and keeps the state after every
+ * token; after verification, gdr_decode_accept makes each sequence's state
+ * the one kept after its last accepted token.  Each token is the decode step
+ * above.
+ * ---------------------------------------------------------------------- */
+
+/*
+ * Draft: n_tokens = K >= 0 tokens per sequence.  Token t of sequence b is
+ * row (b K + t) of the [B K, ...] arrays below (sequence-major, then token):
+ *   q, k          device [B, K, H, d_k], dtype qkv_dtype
+ *   v             device [B, K, H, d_v], dtype qkv_dtype
+ *   beta          device [B, K, H] fp32
+ *   log_a         device [B, K, H, d_k] fp32, or [B, K, H] when scalar_decay != 0
+ *   state         device [B, H, d_v, d_k] fp32, read only
+ *   o             device [B, K, H, d_v] fp32 (output): o of token t, read from
+ *                 the state after token t
+ *   token_states  device [B, K, H, d_v, d_k] fp32 (output): the state after
+ *                 token t of sequence b; must not overlap `state`
+ * d_k, d_v in {64, 128}.  B == 0 or K == 0 is a no-op.  Errors as for
+ * gdr_decode_step.
+ */
+gdr_status gdr_decode_draft(int batch, int n_tokens, int n_heads, int d_k, int d_v,
+                            gdr_dtype qkv_dtype, const void* q, const void* k, const void* v,
+                            const float* beta, const float* log_a, int scalar_decay, float scale,
+                            const float* state, float* o, float* token_states, void* stream);
+
+/*
+ * Accept (rollback): for every sequence b, with n = n_accept[b] clamped to
+ * [0, K], state[b] = token_states[b, n - 1] if n >= 1; for n == 0 state[b] is
+ * left as it was (every draft token rejected).
+ *   n_accept      device [B] int32 (read on the device, so it may be written
+ *                 by an earlier kernel on the stream)
+ *   token_states  device [B, K, H, d_v, d_k] fp32, from gdr_decode_draft
+ *   state         device [B, H, d_v, d_k] fp32, overwritten where n >= 1;
+ *                 must not overlap token_states
+ * B == 0 or K == 0 is a no-op.
+ */
+gdr_status gdr_decode_accept(int batch, int n_tokens, int n_heads, int d_k, int d_v,
+                             const int32_t* n_accept, const float* token_states, float* state,
+                             void* stream);
+
 #ifdef __cplusplus
 }
 #endif

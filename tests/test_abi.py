@@ -63,6 +63,30 @@ def test_decode_rejects_bad_arguments(L):
     assert call(B=0) == 0
 
 
+def test_draft_and_accept_reject_bad_arguments(L):
+    ok = [_fake(i) for i in range(8)]
+    def draft(B=2, K=4, H=2, dk=64, dv=64, dt=0, ptrs=ok):
+        return L.gdr_decode_draft(B, K, H, dk, dv, dt, *ptrs[:5], 0, 1.0, *ptrs[5:8], None)
+    assert draft(B=-1) == 1
+    assert draft(K=-1) == 1
+    assert draft(dk=96) == 2
+    assert draft(dt=3) == 1
+    for i in range(8):
+        bad = list(ok); bad[i] = None
+        assert draft(ptrs=bad) == 1, f"null pointer {i}"
+    mis = list(ok); mis[7] = ctypes.c_void_p(0x10008)     # token_states not 16-byte aligned
+    assert draft(ptrs=mis) == 1
+    assert draft(B=0) == 0 and draft(K=0) == 0
+    def accept(B=2, K=4, H=2, dk=64, dv=64, n=ok[0], ts=ok[1], st=ok[2]):
+        return L.gdr_decode_accept(B, K, H, dk, dv, n, ts, st, None)
+    assert accept(B=-1) == 1
+    assert accept(dv=48) == 2
+    assert accept(n=None) == 1
+    assert accept(ts=ctypes.c_void_p(0x10004)) == 1
+    assert accept(st=None) == 1
+    assert accept(K=0) == 0 and accept(B=0) == 0
+
+
 def _args(**kw):
     a = gdr.PrefillArgs()
     a.n_seqs, a.n_heads, a.d_k, a.d_v, a.total_tokens = 1, 2, 64, 64, 128

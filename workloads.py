@@ -80,6 +80,21 @@ VARLEN = PrefillWorkload("varlen_N32_H32_d128_L1024to16384", 1005, 32, 128, 128,
 
 PREFILL_WORKLOADS = {w.name: w for w in (TINY_KDA, GRAFT_LAYER, GDN_LONG, VARLEN)}
 
+
+@dataclass(frozen=True)
+class DraftWorkload:
+    """Speculative decoding on the decode workload's sequences: each round
+    drafts K tokens per sequence from the live state, then accepts a number
+    of them drawn uniformly from 0 .. K."""
+    name: str
+    seed: int
+    decode: DecodeWorkload      # sizes and distributions of state and tokens
+    draft_tokens: int
+    rounds: int
+
+
+SPEC_DRAFT = DraftWorkload("spec_draft_B256_H14_d64_K4", 1006, DECODE, 4, 16)
+
 # Smaller cases of the d 128 workloads (same distributions) for ncu captures,
 # which replay each captured launch many times: a few GB on the device at most.
 PROFILE_CASES = {w.name: w for w in (
@@ -181,3 +196,35 @@ def make_decode_inputs(w: DecodeWorkload, steps: Optional[int] = None, device="c
         out[key] = out[key].to(dev).contiguous()
     return out
 
+
+
+def make_draft_inputs(w: DraftWorkload, rounds: Optional[int] = None, device="cpu",
+                      draw_device=None) -> dict:
+    """Initial state plus ``rounds`` drafts of K tokens per sequence, drawn
+    like the decode workload's tokens, and the accepted count per round and
+    sequence.  q, k [R, B, K, H, d_k], v [R, B, K, H, d_v], beta [R, B, K, H],
+    log_a [R, B, K, H, d_k] (or [R, B, K, H]), n_accept [R, B] int32 in 0 .. K.
+    """
+    d = w.decode
+    R = w.rounds if rounds is None else rounds
+    K = w.draft_tokens
+    draw_device = draw_device or "cpu"
+    gen = torch.Generator(device=draw_device)
+    gen.manual_seed(w.seed)
+    B, H, dk, dv = d.batch, d.n_heads, d.d_k, d.d_v
+    f32 = dict(dtype=torch.float32, device=draw_device, generator=gen)
+    state = d.init_std * torch.randn(B, H, dv, dk, **f32)
+    q = _l2norm(torch.randn(R, B, K, H, dk, **f32)).to(d.qkv_dtype)
+    k = _l2norm(torch.randn(R, B, K, H, dk, **f32)).to(d.qkv_dtype)
+    v = torch.randn(R, B, K, H, dv, **f32).to(d.qkv_dtype)
+    beta = torch.sigmoid(torch.randn(R, B, K, H, **f32))
+    la_shape = (R, B, K, H) if d.scalar_decay else (R, B, K, H, dk)
+    log_a = torch.nn.functional.logsigmoid(d.log_a_mu + d.log_a_sd * torch.randn(la_shape, **f32))
+    n_accept = torch.randint(0, K + 1, (R, B), generator=gen, device=draw_device,
+                             dtype=torch.int32)
+    out = dict(state=state, q=q, k=k, v=v, beta=beta, log_a=log_a, n_accept=n_accept,
+               scalar_decay=d.scalar_decay, scale=d.scale)
+    dev = torch.device(device)
+    for key in ("state", "q", "k", "v", "beta", "log_a", "n_accept"):
+        out[key] = out[key].to(dev).contiguous()
+    return out
