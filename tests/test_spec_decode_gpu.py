@@ -124,8 +124,8 @@ def test_draft_of_one_token_matches_the_decode_step():
     o2, ts = gdr.decode_draft(d["state"], d["q"][0][:, None], d["k"][0][:, None],
                               d["v"][0][:, None], d["beta"][0][:, None], d["log_a"][0][:, None])
     torch.cuda.synchronize()
-    assert_close_rel(o2[:, 0], o1, 1e-6, "o")
-    assert_close_rel(ts[:, 0], S1, 1e-6, "state")
+    assert_close_rel(o2[:, 0], o1.double().cpu().numpy(), 1e-6, "o")
+    assert_close_rel(ts[:, 0], S1.double().cpu().numpy(), 1e-6, "state")
 
 
 def test_empty_draft_and_accept_are_noops():
