@@ -198,7 +198,8 @@ gdr_status gdr_decode_draft(int batch, int n_tokens, int n_heads, int d_k, int d
         return GDR_ERR_INVALID_ARG;
     if (qkv_dtype != GDR_BF16 && qkv_dtype != GDR_F32) return GDR_ERR_INVALID_ARG;
     if (!supported_width(d_k) || !supported_width(d_v)) return GDR_ERR_UNSUPPORTED;
-    if ((int64_t)batch * n_heads > (int64_t)INT32_MAX) return GDR_ERR_INVALID_ARG;
+    // the draft kernel runs up to four CTAs per (sequence, head)
+    if ((int64_t)batch * n_heads > (int64_t)INT32_MAX / 4) return GDR_ERR_INVALID_ARG;
     if (batch == 0 || n_tokens == 0) return GDR_OK;
     const void* vec[] = {q, k, state, token_states};
     for (const void* p : vec)

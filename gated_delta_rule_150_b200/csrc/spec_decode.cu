@@ -49,11 +49,11 @@ __device__ __forceinline__ float sum16(float x) {
 }
 
 // One token's inputs as seen by one thread: its float4 columns of k, q and
-// log a, the v entries of its rows, and beta.
-template <typename T, int DK, int DV, bool SCALAR>
+// log a, the v entries of its rows (PASSES rows from row0, 16 apart),
+// and beta.
+template <typename T, int DK, int DV, int PASSES, bool SCALAR>
 struct TokenIn {
     static constexpr int NV = DK / (4 * kTPR);
-    static constexpr int PASSES = DV / kRowsPerPass;
     float4 k[NV], q[NV], la[NV];
     float v[PASSES];
     float beta;
@@ -61,7 +61,7 @@ struct TokenIn {
     __device__ __forceinline__ void load(const T* __restrict__ q_, const T* __restrict__ k_,
                                          const T* __restrict__ v_, const float* __restrict__ beta_,
                                          const float* __restrict__ log_a_, size_t tok, int lane16,
-                                         int rgrp) {
+                                         int row0) {
 #pragma unroll
         for (int i = 0; i < NV; ++i) {
             const int c = 4 * (lane16 + kTPR * i);
@@ -75,33 +75,43 @@ struct TokenIn {
             }
         }
 #pragma unroll
-        for (int p = 0; p < PASSES; ++p) v[p] = to_f<T>(v_[tok * DV + rgrp + kRowsPerPass * p]);
+        for (int p = 0; p < PASSES; ++p) v[p] = to_f<T>(v_[tok * DV + row0 + kRowsPerPass * p]);
         beta = __ldg(beta_ + tok);
     }
 };
 
-// One CTA per (sequence b, head h).  Thread t owns rows t / 16 + 16 p and the
-// float4 columns {t % 16 + 16 i} of the state for all K tokens.  Token t of
-// sequence b is input row (b K + t) H + h of q, k, v, beta, log a, o and
-// token_states; the next token's inputs are loaded while this one computes.
-template <typename T, int DK, int DV, bool SCALAR>
-__global__ void __launch_bounds__(kThreads)
+// RS CTAs per (sequence b, head h), CTA part j owning the state rows
+// [j DV / RS, (j + 1) DV / RS) (rows are independent given the token).  Thread
+// t owns rows row0 + t / 16 + 16 p and the float4 columns {t % 16 + 16 i} of
+// the state for all K tokens.  Token t of sequence b is input row
+// (b K + t) H + h of q, k, v, beta, log a, o and token_states; the next
+// token's inputs are loaded while this one computes.
+// At d 64 the kernel is capped at 64 registers so that four CTAs fit on an SM
+// (7 % faster on B200 than three CTAs at 78 registers, despite a 24-byte
+// spill in the bf16 per-channel case); wider states keep their registers.
+template <int DK, int DV>
+constexpr int draft_min_ctas() { return (DK == 64 && DV == 64) ? 4 : 1; }
+
+template <typename T, int DK, int DV, bool SCALAR, int RS>
+__global__ void __launch_bounds__(kThreads, draft_min_ctas<DK, DV>())
 decode_draft_kernel(int H, int K, const T* __restrict__ q, const T* __restrict__ k,
                     const T* __restrict__ v, const float* __restrict__ beta,
                     const float* __restrict__ log_a, float scale, const float* __restrict__ state,
                     float* __restrict__ o, float* __restrict__ token_states) {
-    using Tok = TokenIn<T, DK, DV, SCALAR>;
+    constexpr int PASSES = DV / (RS * kRowsPerPass);
+    static_assert(PASSES >= 1 && PASSES * RS * kRowsPerPass == DV, "row split");
+    using Tok = TokenIn<T, DK, DV, PASSES, SCALAR>;
     constexpr int NV = Tok::NV;
-    constexpr int PASSES = Tok::PASSES;
-    const int bh = blockIdx.x;
+    const int bh = blockIdx.x / RS;
+    const int part = blockIdx.x - bh * RS;
     const int b = bh / H;
     const int h = bh - b * H;
     const int lane16 = threadIdx.x % kTPR;
-    const int rgrp = threadIdx.x / kTPR;
+    const int row0 = part * (DV / RS) + threadIdx.x / kTPR;
 
     const size_t tok0 = (size_t)b * K * H + h;
     Tok nxt;
-    nxt.load(q, k, v, beta, log_a, tok0, lane16, rgrp);
+    nxt.load(q, k, v, beta, log_a, tok0, lane16, row0);
 
     const float* S0 = state + (size_t)bh * DV * DK;
     float4 s[PASSES][NV];
@@ -110,13 +120,13 @@ decode_draft_kernel(int H, int K, const T* __restrict__ q, const T* __restrict__
 #pragma unroll
         for (int i = 0; i < NV; ++i)
             s[p][i] = __ldg(reinterpret_cast<const float4*>(
-                S0 + (size_t)(rgrp + kRowsPerPass * p) * DK + 4 * (lane16 + kTPR * i)));
+                S0 + (size_t)(row0 + kRowsPerPass * p) * DK + 4 * (lane16 + kTPR * i)));
 
 #pragma unroll 1
     for (int t = 0; t < K; ++t) {
         const Tok cur = nxt;
         const size_t tok = tok0 + (size_t)t * H;
-        if (t + 1 < K) nxt.load(q, k, v, beta, log_a, tok + H, lane16, rgrp);
+        if (t + 1 < K) nxt.load(q, k, v, beta, log_a, tok + H, lane16, row0);
 
         float4 aa[NV], qq[NV];
         float kq_part = 0.f;
@@ -134,7 +144,7 @@ decode_draft_kernel(int H, int K, const T* __restrict__ q, const T* __restrict__
         float* St = token_states + tok * DV * DK;
 #pragma unroll
         for (int p = 0; p < PASSES; ++p) {
-            const int row = rgrp + kRowsPerPass * p;
+            const int row = row0 + kRowsPerPass * p;
             float pk = 0.f, pq = 0.f;
 #pragma unroll
             for (int i = 0; i < NV; ++i) {
@@ -189,16 +199,21 @@ decode_accept_kernel(int H, int K, int n4, const int32_t* __restrict__ n_accept,
     }
 }
 
+// CTAs per head-state of the draft kernel (splitting the rows over 2 or 4
+// CTAs measured 8 % and 47 % slower at d 64: each CTA repeats the token's
+// inputs and k . q).
+constexpr int kRowSplit = 1;
+
 template <typename T, int DK, int DV>
 cudaError_t draft_typed(int B, int K, int H, const void* q, const void* k, const void* v,
                         const float* beta, const float* log_a, int scalar, float scale,
                         const float* state, float* o, float* ts, cudaStream_t st) {
-    const dim3 grid((unsigned)(B * H));
+    const dim3 grid((unsigned)((int64_t)B * H * kRowSplit));
     if (scalar)
-        decode_draft_kernel<T, DK, DV, true><<<grid, kThreads, 0, st>>>(
+        decode_draft_kernel<T, DK, DV, true, kRowSplit><<<grid, kThreads, 0, st>>>(
             H, K, (const T*)q, (const T*)k, (const T*)v, beta, log_a, scale, state, o, ts);
     else
-        decode_draft_kernel<T, DK, DV, false><<<grid, kThreads, 0, st>>>(
+        decode_draft_kernel<T, DK, DV, false, kRowSplit><<<grid, kThreads, 0, st>>>(
             H, K, (const T*)q, (const T*)k, (const T*)v, beta, log_a, scale, state, o, ts);
     return cudaGetLastError();
 }
