@@ -13,6 +13,9 @@ Contents
   K draft tokens that keep the state after each token, then the state of the
   accepted prefix (same C file).
 * ``cumdecay``: chunk-local inclusive prefix sums of log a (numpy, fp64).
+* ``preprocess``: the mixer's input activations from raw projections -- the
+  causal depthwise conv of width 4 on q, k, v, L2 norm of q and k, beta as a
+  sigmoid and log a as a log-sigmoid of the biased gate (numpy, fp64).
 * ``chunk_factors`` / ``chunked_prefill``: the chunked form of the same
   recurrence written from its definition (numpy, fp64).  It is used to check
   the intermediate results of the intra-chunk kernel; it is itself pinned by
@@ -305,3 +308,70 @@ def chunked_prefill(q, k, v, beta, log_a, cu_seqlens, scalar_decay=False, scale=
                 o[s:e, h] = f["Qg"] @ S0.T + f["P"] @ Delta
                 fin[s_idx, h] = S0 * f["gamma_C"][None, :] + Delta.T @ f["Kd"]
     return dict(o=o, final_state=fin)
+
+
+# ---------------------------------------------------------------------------
+# Input activations (numpy, fp64).
+#
+# "kda-graft: Qwen2.5-0.5B с трансплантированным KDA", section "Идея и
+# архитектура": the graft adds a width-4 convolution (initialised as an
+# identity tap), the alpha gate with bias +5 (sigma(5) ~ 0.993), the write
+# strength beta, an output gate and an RMSNorm around the q/k/v projections.
+# The page gives no formulas; the readings taken are stated per function.
+# ---------------------------------------------------------------------------
+
+def _conv4(x, w, cu):
+    """Causal depthwise conv of width 4 per sequence: for token t of a
+    sequence starting at s, y[t, h, c] = sum_{j=0..3} w[h*d + c, j] x[t-3+j, h, c]
+    over the taps with t-3+j >= s (zero history at every sequence start; tap 3
+    is the current token, so w = [0, 0, 0, 1] is the identity)."""
+    T, H, d = x.shape
+    W = w.reshape(H, d, 4)
+    y = np.zeros_like(x)
+    for n in range(len(cu) - 1):
+        s, e = int(cu[n]), int(cu[n + 1])
+        for t in range(s, e):
+            for j in range(4):
+                tt = t - 3 + j
+                if tt >= s:
+                    y[t] += W[:, :, j] * x[tt]
+    return y
+
+
+def _l2norm(y):
+    """y / max(||y||_2, 1e-12) per (token, head)."""
+    nrm = np.sqrt(np.sum(y * y, axis=-1, keepdims=True))
+    return y / np.maximum(nrm, 1e-12)
+
+
+def sigmoid(z):
+    """1 / (1 + exp(-z)), written with exp(-|z|) so that it never overflows."""
+    e = np.exp(-np.abs(z))
+    return np.where(z >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
+
+
+def log_sigmoid(z):
+    """log(1 / (1 + exp(-z))) = min(z, 0) - log1p(exp(-|z|)) (no overflow)."""
+    return np.minimum(z, 0.0) - np.log1p(np.exp(-np.abs(z)))
+
+
+def preprocess(xq, xk, xv, conv_q, conv_k, conv_v, beta_raw, a_raw, a_bias, cu_seqlens,
+               scalar_decay=False) -> dict:
+    """Inputs of the recurrence from raw per-head projections (fp64).
+
+    q = L2norm(conv4(xq)), k = L2norm(conv4(xk)), v = conv4(xv),
+    beta = sigmoid(beta_raw), log a = log_sigmoid(a_raw + a_bias).
+    Readings: no activation after the conv (the page names none); q and k
+    are L2-normalised per (token, head) after the conv; the bias is per
+    (head, key channel), or per head with a scalar gate.  Shapes: xq, xk
+    [T, H, d_k], xv [T, H, d_v], conv_* [H * d, 4], beta_raw [T, H], a_raw
+    [T, H, d_k] with a_bias [H, d_k] (or [T, H] with [H]).
+    """
+    cu = _i32(cu_seqlens)
+    xq, xk, xv = f64(xq), f64(xk), f64(xv)
+    q = _l2norm(_conv4(xq, f64(conv_q), cu))
+    k = _l2norm(_conv4(xk, f64(conv_k), cu))
+    v = _conv4(xv, f64(conv_v), cu)
+    beta = sigmoid(f64(beta_raw))
+    z = f64(a_raw) + f64(a_bias)[None]
+    return dict(q=q, k=k, v=v, beta=beta, log_a=log_sigmoid(z))
