@@ -16,6 +16,9 @@ collective on the data path).  The same run also measures:
 * ``spec_decode``: speculative decoding on the same sequences: a draft of 4
   tokens that keeps the state after each token, then the accept (rollback)
   step, each timed alone and as one verify cycle;
+* ``preprocess``: the input activations (conv-4, L2 norm of q and k, beta and
+  log-decay gates) from raw projections of the graft layer's shape, alone and
+  followed by the prefill;
 * ``roofline``: the step's dominant kernel, timed alone with CUDA events;
 * ``e2e``: the same prefill through the public API with pinned host buffers,
   host<->device copies inside the timed region;
@@ -80,6 +83,12 @@ def draft_bytes_per_head_state(d_k: int, d_v: int, elem: int, scalar: bool, K: i
     q, k, v, beta, log_a read and o (fp32) written."""
     tok = (2 * d_k + d_v) * elem + 4 + (4 if scalar else 4 * d_k) + 4 * d_v
     return 4 * d_k * d_v + K * (4 * d_k * d_v + tok)
+
+
+def preprocess_bytes_per_token_head(d: int, elem: int, scalar: bool) -> int:
+    """raw x_q, x_k, x_v, beta_raw and a_raw read; q, k, v, beta and log a
+    written (conv taps and biases are per head, not per token)."""
+    return 2 * (3 * d * elem + 4 + (4 if scalar else 4 * d))
 
 
 def peaks() -> dict:
@@ -394,9 +403,11 @@ def run_gdr(args):
     extra = {}
     decode = None
     spec = None
+    pre = None
     if not args.no_extra:
         decode = bench_decode(gdr, stream, pk, args)
         spec = bench_spec_decode(gdr, stream, pk, args)
+        pre = bench_preprocess(gdr, stream, pk, args)
         for w in (wl.TINY_KDA, wl.GDN_LONG, wl.VARLEN):
             extra[w.name] = bench_prefill_workload(gdr, w, stream, pk, rank, args)
     e2e = bench_e2e(gdr, stream, args)
@@ -419,6 +430,7 @@ def run_gdr(args):
         "kernel_ms": stage_report,
         "decode": decode,
         "spec_decode": spec,
+        "preprocess": pre,
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
@@ -536,6 +548,57 @@ def bench_spec_decode(gdr, stream, pk, args):
     return res
 
 
+def bench_preprocess(gdr, stream, pk, args):
+    """Input activations on the graft layer's shape, four rotating input and
+    output sets (4 x 148 MB > L2); then the same followed by the prefill."""
+    w = wl.PREPROCESS
+    names = ("xq", "xk", "xv", "conv_q", "conv_k", "conv_v", "beta_raw", "a_raw", "a_bias",
+             "cu_seqlens")
+    sets = []
+    for i in range(4):
+        inp = wl.make_preprocess_inputs(wl.shrink(w, seed=w.seed + 10 * i), device="cuda",
+                                        draw_device="cuda")
+        T, H, d = inp["xq"].shape
+        act = {n: torch.empty(T, H, d, dtype=inp["xq"].dtype, device="cuda") for n in ("q", "k", "v")}
+        act["beta"] = torch.empty(T, H, device="cuda")
+        act["log_a"] = torch.empty(inp["a_raw"].shape, device="cuda")
+        ws = torch.empty(gdr.workspace_size(1, H, d, d, T), dtype=torch.uint8, device="cuda")
+        prep = gdr.PreparedPrefill(act["q"], act["k"], act["v"], act["beta"], act["log_a"],
+                                   inp["cu_seqlens"], out=torch.empty_like(act["v"]),
+                                   final_state=torch.empty(1, H, d, d, device="cuda"),
+                                   workspace=ws)
+        sets.append((inp, act, prep))
+
+    def pre(i):
+        inp, act, _ = sets[i % 4]
+        gdr.preprocess(*(inp[n] for n in names), out=act)
+
+    def layer(i):
+        pre(i)
+        sets[i % 4][2].run()
+
+    for i in range(8):
+        layer(i)
+    n = 200
+    ms_p = timed(pre, n, stream)
+    ms_l = timed(layer, n, stream)
+    T, H, d = sets[0][0]["xq"].shape
+    elem = 2 if w.qkv_dtype == torch.bfloat16 else 4
+    per = preprocess_bytes_per_token_head(d, elem, w.scalar_decay)
+    gbs = per * T * H / (ms_p * 1e-3) / 1e9
+    res = {"workload": w.name, "ms": round(ms_p, 5), "gbs": round(gbs, 1),
+           "bytes_per_token_head": per,
+           "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"],
+                        "unit": "GB/s", "frac": round(gbs / pk["hbm_gbs"], 4),
+                        "traffic": recorded_traffic("preprocess", w.name)},
+           "with_prefill": {"ms_per_step": round(ms_l, 5),
+                            "tokens_per_s": round(T / (ms_l * 1e-3), 1)},
+           "l2": "4 rotating input and output sets, 4 x 148 MB > 126 MB L2", "steps": n}
+    del sets
+    torch.cuda.empty_cache()
+    return res
+
+
 def bench_e2e(gdr, stream, args):
     """Prefill through the public API from pinned host buffers: H2D of the
     inputs, the prefill, D2H of o and the final state, every step."""
@@ -582,6 +645,8 @@ def main():
                    help="run only the decode measurement (for profiling)")
     p.add_argument("--only-spec", action="store_true",
                    help="run only the speculative-decoding measurement (for profiling)")
+    p.add_argument("--only-preprocess", action="store_true",
+                   help="run only the input-activation measurement (for profiling)")
     p.add_argument("--workload", default=wl.GRAFT_LAYER.name,
                    choices=sorted(wl.PREFILL_WORKLOADS) + sorted(wl.PROFILE_CASES),
                    help="prefill workload of the main line (default: the graft layer)")
@@ -596,6 +661,11 @@ def main():
         import gated_delta_rule_150_b200 as gdr
         gdr.lib()
         print(json.dumps(bench_decode(gdr, torch.cuda.current_stream(), peaks(), args)), flush=True)
+    elif args.only_preprocess:
+        import gated_delta_rule_150_b200 as gdr
+        gdr.lib()
+        print(json.dumps(bench_preprocess(gdr, torch.cuda.current_stream(), peaks(), args)),
+              flush=True)
     elif args.only_spec:
         import gated_delta_rule_150_b200 as gdr
         gdr.lib()

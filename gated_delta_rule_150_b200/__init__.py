@@ -20,7 +20,7 @@ import threading
 import torch
 
 __all__ = ["PrefillArgs", "PreparedPrefill", "prefill", "kernel_count", "decode_step",
-           "decode_draft", "decode_accept", "cumdecay", "chunk_factors", "workspace_size",
+           "decode_draft", "decode_accept", "PreprocessArgs", "preprocess", "cumdecay", "chunk_factors", "workspace_size",
            "snapshot_count", "prefill_status", "lib", "GdrError", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_build", "libgdr.so")
@@ -49,6 +49,20 @@ class PrefillArgs(ctypes.Structure):
         ("final_state", ctypes.c_void_p), ("snap_interval", ctypes.c_int),
         ("snapshots", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
         ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
+class PreprocessArgs(ctypes.Structure):
+    """Mirror of ``gdr_preprocess_args`` (include/gdr.h)."""
+    _fields_ = [
+        ("n_seqs", ctypes.c_int), ("n_heads", ctypes.c_int), ("d", ctypes.c_int),
+        ("total_tokens", ctypes.c_int64), ("cu_seqlens", ctypes.c_void_p),
+        ("io_dtype", ctypes.c_int), ("xq", ctypes.c_void_p), ("xk", ctypes.c_void_p),
+        ("xv", ctypes.c_void_p), ("conv_q", ctypes.c_void_p), ("conv_k", ctypes.c_void_p),
+        ("conv_v", ctypes.c_void_p), ("beta_raw", ctypes.c_void_p), ("a_raw", ctypes.c_void_p),
+        ("a_bias", ctypes.c_void_p), ("scalar_decay", ctypes.c_int), ("q", ctypes.c_void_p),
+        ("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("beta", ctypes.c_void_p),
+        ("log_a", ctypes.c_void_p),
     ]
 
 
@@ -87,6 +101,8 @@ def lib():
             L.gdr_chunk_factors.argtypes = [ctypes.POINTER(PrefillArgs), vp, vp, vp, vp, vp, vp]
             L.gdr_decode_step.restype = i
             L.gdr_decode_step.argtypes = [i, i, i, i, i, vp, vp, vp, vp, vp, i, f, vp, vp, vp]
+            L.gdr_preprocess.restype = i
+            L.gdr_preprocess.argtypes = [ctypes.POINTER(PreprocessArgs), vp]
             L.gdr_decode_draft.restype = i
             L.gdr_decode_draft.argtypes = [i, i, i, i, i, i, vp, vp, vp, vp, vp, i, f, vp, vp,
                                            vp, vp]
@@ -357,3 +373,45 @@ def decode_accept(state, token_states, n_accept):
                                    _ptr(state), _stream(state.device)),
            "gdr_decode_accept")
     return state
+
+
+def preprocess(xq, xk, xv, conv_q, conv_k, conv_v, beta_raw, a_raw, a_bias, cu_seqlens, *,
+               scalar_decay=False, out=None):
+    """The recurrence's inputs from raw per-head projections, in one kernel.
+
+    xq, xk, xv [T, H, d] (bf16 or fp32), conv_* [H * d, 4] fp32 taps (tap 3 =
+    current token), beta_raw [T, H], a_raw [T, H, d] with a_bias [H, d] (or
+    [T, H] with [H] for a scalar gate).  Returns dict(q, k, v, beta, log_a) in
+    the layouts ``prefill`` takes: q = L2norm(conv(xq)), k = L2norm(conv(xk)),
+    v = conv(xv), beta = sigmoid(beta_raw), log_a = log_sigmoid(a_raw + a_bias).
+    ``out`` may hold preallocated outputs under the same keys.
+    """
+    if xq.dtype != xk.dtype or xq.dtype != xv.dtype:
+        raise TypeError("xq, xk and xv must share a dtype")
+    T, H, d = xq.shape
+    dev = xq.device
+    out = dict(out or {})
+    for name in ("q", "k", "v"):
+        if out.get(name) is None:
+            out[name] = torch.empty(T, H, d, dtype=xq.dtype, device=dev)
+    if out.get("beta") is None:
+        out["beta"] = torch.empty(T, H, device=dev)
+    if out.get("log_a") is None:
+        out["log_a"] = torch.empty(a_raw.shape, device=dev)
+    _need_cuda(xq, xk, xv, conv_q, conv_k, conv_v, beta_raw, a_raw, a_bias, cu_seqlens,
+               *out.values())
+    for t in (conv_q, conv_k, conv_v, beta_raw, a_raw, a_bias):
+        if t.dtype != torch.float32:
+            raise TypeError("conv taps, beta_raw, a_raw and a_bias must be float32")
+    a = PreprocessArgs()
+    a.n_seqs, a.n_heads, a.d, a.total_tokens = cu_seqlens.numel() - 1, H, d, T
+    a.cu_seqlens = cu_seqlens.data_ptr()
+    a.io_dtype = _dtype_code(xq)
+    a.xq, a.xk, a.xv = xq.data_ptr(), xk.data_ptr(), xv.data_ptr()
+    a.conv_q, a.conv_k, a.conv_v = conv_q.data_ptr(), conv_k.data_ptr(), conv_v.data_ptr()
+    a.beta_raw, a.a_raw, a.a_bias = beta_raw.data_ptr(), a_raw.data_ptr(), a_bias.data_ptr()
+    a.scalar_decay = int(bool(scalar_decay))
+    a.q, a.k, a.v = out["q"].data_ptr(), out["k"].data_ptr(), out["v"].data_ptr()
+    a.beta, a.log_a = out["beta"].data_ptr(), out["log_a"].data_ptr()
+    _check(lib().gdr_preprocess(ctypes.byref(a), _stream(dev)), "gdr_preprocess")
+    return out

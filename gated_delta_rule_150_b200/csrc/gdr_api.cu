@@ -190,6 +190,26 @@ gdr_status gdr_decode_step(int batch, int n_heads, int d_k, int d_v, gdr_dtype q
                                         static_cast<cudaStream_t>(stream)));
 }
 
+gdr_status gdr_preprocess(const gdr_preprocess_args* a, void* stream) {
+    if (!a) return GDR_ERR_INVALID_ARG;
+    if (a->n_seqs < 0 || a->n_heads <= 0 || a->d <= 0 || a->total_tokens < 0 ||
+        a->total_tokens > (int64_t)INT32_MAX)
+        return GDR_ERR_INVALID_ARG;
+    if (a->io_dtype != GDR_BF16 && a->io_dtype != GDR_F32) return GDR_ERR_INVALID_ARG;
+    if (!supported_width(a->d)) return GDR_ERR_UNSUPPORTED;
+    if (a->total_tokens == 0) return GDR_OK;
+    if (a->n_seqs == 0 || !a->cu_seqlens || !aligned4(a->cu_seqlens)) return GDR_ERR_INVALID_ARG;
+    const void* v16[] = {a->xq, a->xk, a->xv, a->conv_q, a->conv_k, a->conv_v, a->q, a->k, a->v};
+    for (const void* p : v16)
+        if (!p || !aligned16(p)) return GDR_ERR_INVALID_ARG;
+    const void* gate[] = {a->a_raw, a->a_bias, a->log_a};
+    for (const void* p : gate)
+        if (!p || !(a->scalar_decay ? aligned4(p) : aligned16(p))) return GDR_ERR_INVALID_ARG;
+    if (!a->beta_raw || !aligned4(a->beta_raw) || !a->beta || !aligned4(a->beta))
+        return GDR_ERR_INVALID_ARG;
+    return from_cuda(gdr::launch_preprocess(*a, static_cast<cudaStream_t>(stream)));
+}
+
 gdr_status gdr_decode_draft(int batch, int n_tokens, int n_heads, int d_k, int d_v,
                             gdr_dtype qkv_dtype, const void* q, const void* k, const void* v,
                             const float* beta, const float* log_a, int scalar_decay, float scale,

@@ -155,6 +155,8 @@ cudaError_t launch_decode(int B, int H, int dk, int dv, gdr_dtype dt, const void
                           const float* log_a, int scalar, float scale, float* state,
                           float* o, cudaStream_t st);
 
+cudaError_t launch_preprocess(const gdr_preprocess_args& a, cudaStream_t st);
+
 cudaError_t launch_decode_draft(int B, int K, int H, int dk, int dv, gdr_dtype dt, const void* q,
                                 const void* k, const void* v, const float* beta,
                                 const float* log_a, int scalar, float scale, const float* state,

@@ -231,6 +231,53 @@ gdr_status gdr_decode_step(int batch, int n_heads, int d_k, int d_v, gdr_dtype q
                            float* o, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Input activations: the recurrence's q, k, v, beta and log a from raw
+ * per-head projections in one pass ("kda-graft", section "Идея и
+ * архитектура": the graft adds a width-4 convolution initialised as an
+ * identity tap, the alpha gate with bias +5 and the write strength beta).
+ * For token t of a sequence starting at s, head h, channel c:
+ *     conv(x)[t] = sum_{j=0..3, t-3+j >= s} w[h d + c][j] x[t-3+j]
+ *     q = conv(x_q) / max(||conv(x_q)||, 1e-12)   (norm over the head's d channels)
+ *     k = conv(x_k) / max(||conv(x_k)||, 1e-12)
+ *     v = conv(x_v)
+ *     beta = sigmoid(beta_raw),  log_a = log_sigmoid(a_raw + a_bias)
+ * The conv restarts from zero history at every sequence start; tap 3 is the
+ * current token.  The outputs are gdr_prefill's inputs, in its layouts.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+    int n_seqs;                 /* N >= 0 sequences packed by cu_seqlens */
+    int n_heads;                /* H >= 1 */
+    int d;                      /* d_k = d_v: 64 or 128 */
+    int64_t total_tokens;       /* T_tot = cu_seqlens[N] (host copy) */
+    const int32_t* cu_seqlens;  /* device [N+1], as for gdr_prefill */
+    gdr_dtype io_dtype;         /* dtype of x_q, x_k, x_v and of q, k, v */
+    const void* xq;             /* device [T_tot, H, d] raw projections */
+    const void* xk;             /* device [T_tot, H, d] */
+    const void* xv;             /* device [T_tot, H, d] */
+    const float* conv_q;        /* device [H d, 4] fp32 taps per channel (row h d + c) */
+    const float* conv_k;        /* device [H d, 4] */
+    const float* conv_v;        /* device [H d, 4] */
+    const float* beta_raw;      /* device [T_tot, H] */
+    const float* a_raw;         /* device [T_tot, H, d], or [T_tot, H] if scalar_decay */
+    const float* a_bias;        /* device [H, d], or [H] if scalar_decay */
+    int scalar_decay;           /* 0: per-key-channel gate, 1: one gate per head-token */
+    void* q;                    /* device [T_tot, H, d], io_dtype (output) */
+    void* k;                    /* device [T_tot, H, d], io_dtype (output) */
+    void* v;                    /* device [T_tot, H, d], io_dtype (output) */
+    float* beta;                /* device [T_tot, H] (output) */
+    float* log_a;               /* device [T_tot, H, d] or [T_tot, H] (output) */
+} gdr_preprocess_args;
+
+/*
+ * Enqueue the input activations.  Outputs must not overlap the inputs.
+ * Errors: GDR_ERR_INVALID_ARG (null or misaligned pointer -- xq, xk, xv, the
+ * conv taps, q, k, v and, with a per-channel gate, a_raw, a_bias and log_a
+ * need 16-byte alignment -- or bad sizes), GDR_ERR_UNSUPPORTED (d not 64 or
+ * 128), GDR_ERR_CUDA on a failed launch.  T_tot == 0 is a no-op.
+ */
+gdr_status gdr_preprocess(const gdr_preprocess_args* args, void* stream);
+
+/* ------------------------------------------------------------------------
  * Speculative decoding with rollback ("Modele hybrydowe", section "Co stan
  * rekurencyjny zmienia przy serwowaniu", point 2: a KV cache drops rejected
  * draft tokens, but the recurrent state has already absorbed them, so the

@@ -87,6 +87,34 @@ def test_draft_and_accept_reject_bad_arguments(L):
     assert accept(K=0) == 0 and accept(B=0) == 0
 
 
+def _pre_args(**kw):
+    a = gdr.PreprocessArgs()
+    a.n_seqs, a.n_heads, a.d, a.total_tokens = 1, 2, 64, 128
+    a.cu_seqlens = 0x10000
+    a.io_dtype = 0
+    names = ("xq", "xk", "xv", "conv_q", "conv_k", "conv_v", "beta_raw", "a_raw", "a_bias",
+             "q", "k", "v", "beta", "log_a")
+    for i, n in enumerate(names):
+        setattr(a, n, 0x100000 * (i + 1))
+    for k_, v_ in kw.items():
+        setattr(a, k_, v_)
+    return a
+
+
+def test_preprocess_rejects_bad_arguments(L):
+    pre = lambda a: L.gdr_preprocess(ctypes.byref(a), None)
+    assert pre(_pre_args(n_heads=0)) == 1
+    assert pre(_pre_args(d=96)) == 2
+    assert pre(_pre_args(io_dtype=5)) == 1
+    assert pre(_pre_args(total_tokens=-1)) == 1
+    for n in ("xq", "conv_k", "beta_raw", "a_bias", "v", "log_a", "cu_seqlens"):
+        assert pre(_pre_args(**{n: None})) == 1, n
+    assert pre(_pre_args(xk=0x200008)) == 1                     # not 16-byte aligned
+    assert pre(_pre_args(log_a=0x200004)) == 1                  # per-channel gate: 16 bytes
+    assert pre(_pre_args(total_tokens=0)) == 0
+    assert pre(_pre_args(total_tokens=0, xq=None)) == 0         # nothing to do, nothing read
+
+
 def _args(**kw):
     a = gdr.PrefillArgs()
     a.n_seqs, a.n_heads, a.d_k, a.d_v, a.total_tokens = 1, 2, 64, 64, 128

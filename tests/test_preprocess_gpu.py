@@ -1,0 +1,99 @@
+"""Input activations (conv-4, L2 norm, gates) on the GPU against the fp64
+oracle.
+
+Tolerances, per element, with M = max |ref| of the tensor: q, k, v within
+2^-8 |ref| + 1e-5 M when they are bf16 (one bf16 rounding of an fp32 result)
+and 1e-6 |ref| + 1e-5 M when fp32 (fp32 conv sums); beta and log a (fp32)
+within 2e-6 |ref| + 2e-6 (fp32 rounding of the biased gate, expf / log1pf)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+
+def _gdr():
+    import gated_delta_rule_150_b200 as gdr
+    gdr.lib()
+    return gdr
+
+
+ARGS = ("xq", "xk", "xv", "conv_q", "conv_k", "conv_v", "beta_raw", "a_raw", "a_bias",
+        "cu_seqlens")
+
+
+def _check(out, ref, bf16):
+    for name in ("q", "k", "v"):
+        x = out[name].double().cpu().numpy()
+        r = ref[name]
+        M = np.abs(r).max() if r.size else 0.0
+        rel = 2.0 ** -8 if bf16 else 1e-6
+        bad = np.abs(x - r) > rel * np.abs(r) + 1e-5 * M
+        assert not bad.any(), f"{name}: {bad.sum()} elements out of bound, max err {np.abs(x - r).max():.3e}"
+    for name in ("beta", "log_a"):
+        x = out[name].double().cpu().numpy()
+        r = ref[name]
+        bad = np.abs(x - r) > 2e-6 * np.abs(r) + 2e-6
+        assert not bad.any(), f"{name}: max err {np.abs(x - r).max():.3e}"
+
+
+def _run(w, lengths=None):
+    gdr = _gdr()
+    inp = wl.make_preprocess_inputs(w, lengths=lengths)
+    d = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in inp.items()}
+    out = gdr.preprocess(*(d[a] for a in ARGS), scalar_decay=w.scalar_decay)
+    torch.cuda.synchronize()
+    ref = oracle.preprocess(*(inp[a] for a in ARGS), scalar_decay=w.scalar_decay)
+    _check(out, ref, w.qkv_dtype == torch.bfloat16)
+    return inp, out
+
+
+def test_preprocess_graft_layer_full():
+    """The graft layer's shape (8192 tokens x 14 heads x 64, bf16), every
+    output element checked."""
+    _run(wl.PREPROCESS)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("scalar", [False, True])
+def test_preprocess_ragged(d, dtype, scalar):
+    """Sequences shorter than the conv (1, 2, 3 tokens), an empty one, one
+    across a warp's worth of units, several heads."""
+    w = wl.shrink(wl.PREPROCESS, n_heads=3, d_k=d, d_v=d, qkv_dtype=dtype, scalar_decay=scalar,
+                  seed=1107)
+    _run(w, lengths=[1, 2, 3, 0, 70, 5])
+
+
+def test_preprocess_feeds_prefill():
+    """The activations go straight into the prefill: the chain matches the
+    oracle's prefill of the oracle's activations (cast to the kernel's
+    dtype) within the prefill tolerance 2e-2 max |ref|."""
+    gdr = _gdr()
+    w = wl.shrink(wl.PREPROCESS, n_heads=2, seed=1108)
+    lengths = [200, 77]
+    inp = wl.make_preprocess_inputs(w, lengths=lengths)
+    d = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in inp.items()}
+    act = gdr.preprocess(*(d[a] for a in ARGS))
+    o, fin, _ = gdr.prefill(act["q"], act["k"], act["v"], act["beta"], act["log_a"],
+                            d["cu_seqlens"])
+    torch.cuda.synchronize()
+    ref_act = oracle.preprocess(*(inp[a] for a in ARGS))
+    cast = {n: torch.from_numpy(ref_act[n]).to(torch.bfloat16) for n in ("q", "k", "v")}
+    ref = oracle.prefill(cast["q"], cast["k"], cast["v"], ref_act["beta"], ref_act["log_a"],
+                         inp["cu_seqlens"])
+    for name, x, r in (("o", o, ref["o"]), ("final_state", fin, ref["final_state"])):
+        err = np.abs(x.double().cpu().numpy() - r).max() / np.abs(r).max()
+        assert err <= 2e-2, f"{name}: {err:.3e}"
+
+
+def test_preprocess_no_tokens_is_noop():
+    gdr = _gdr()
+    w = wl.shrink(wl.PREPROCESS, n_heads=2, seed=1109)
+    inp = wl.make_preprocess_inputs(w, lengths=[0, 0])
+    d = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in inp.items()}
+    out = gdr.preprocess(*(d[a] for a in ARGS))
+    assert out["q"].shape == (0, 2, 64)

@@ -95,6 +95,11 @@ class DraftWorkload:
 
 SPEC_DRAFT = DraftWorkload("spec_draft_B256_H14_d64_K4", 1006, DECODE, 4, 16)
 
+# Raw projections of the graft layer's shape for the input activations: the
+# gates come out distributed as the graft layer's (beta = sigmoid(N(0, 1)),
+# log a = logsigmoid(5 + N(0, 1)) with the page's bias +5).
+PREPROCESS = replace(GRAFT_LAYER, name="preprocess_graft_layer_H14_T8192_d64_bf16", seed=1007)
+
 # Smaller cases of the d 128 workloads (same distributions) for ncu captures,
 # which replay each captured launch many times: a few GB on the device at most.
 PROFILE_CASES = {w.name: w for w in (
@@ -226,5 +231,40 @@ def make_draft_inputs(w: DraftWorkload, rounds: Optional[int] = None, device="cp
                scalar_decay=d.scalar_decay, scale=d.scale)
     dev = torch.device(device)
     for key in ("state", "q", "k", "v", "beta", "log_a", "n_accept"):
+        out[key] = out[key].to(dev).contiguous()
+    return out
+
+
+def make_preprocess_inputs(w: PrefillWorkload, device="cpu", lengths=None, draw_device=None,
+                           conv_noise: float = 0.1, gate_bias: float = 5.0) -> dict:
+    """Raw per-head projections and parameters for the input activations.
+
+    xq, xk, xv ~ N(0, 1) [T, H, d] (cast to the workload's dtype); conv taps
+    [H d, 4] = the identity tap [0, 0, 0, 1] plus N(0, conv_noise); beta_raw ~
+    N(0, 1) [T, H]; a_raw ~ N(0, 1) [T, H, d] (or [T, H]) with a bias of
+    ``gate_bias`` per (head, channel) (or per head).
+    """
+    draw_device = draw_device or "cpu"
+    gen = torch.Generator(device=draw_device)
+    gen.manual_seed(w.seed)
+    if lengths is None:
+        lgen = torch.Generator().manual_seed(w.seed)
+        lengths = _draw_lengths(w, lgen)
+    lengths = [int(n) for n in lengths]
+    T = sum(lengths)
+    H, d = w.n_heads, w.d_k
+    f32 = dict(dtype=torch.float32, device=draw_device, generator=gen)
+    x = [torch.randn(T, H, d, **f32).to(w.qkv_dtype) for _ in range(3)]
+    ident = torch.tensor([0.0, 0.0, 0.0, 1.0], device=draw_device)
+    conv = [ident + conv_noise * torch.randn(H * d, 4, **f32) for _ in range(3)]
+    beta_raw = torch.randn(T, H, **f32)
+    a_raw = torch.randn((T, H) if w.scalar_decay else (T, H, d), **f32)
+    a_bias = torch.full((H,) if w.scalar_decay else (H, d), gate_bias, device=draw_device)
+    out = dict(xq=x[0], xk=x[1], xv=x[2], conv_q=conv[0], conv_k=conv[1], conv_v=conv[2],
+               beta_raw=beta_raw, a_raw=a_raw, a_bias=a_bias, cu_seqlens=cu_seqlens_of(lengths),
+               lengths=lengths, scalar_decay=w.scalar_decay)
+    dev = torch.device(device)
+    for key in ("xq", "xk", "xv", "conv_q", "conv_k", "conv_v", "beta_raw", "a_raw", "a_bias",
+                "cu_seqlens"):
         out[key] = out[key].to(dev).contiguous()
     return out
