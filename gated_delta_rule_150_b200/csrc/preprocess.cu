@@ -14,7 +14,9 @@
 // contiguous rows of [T, H, D].  Each thread reads its channels of the
 // current token and up to three earlier ones of the same sequence (the
 // earlier rows were just read by neighbouring warps and come from L1/L2, so
-// HBM sees each row about once).  The L2 norms are half-warp or quarter-warp
+// HBM sees each row about once).  The tap loads are unconditional (a tap
+// before the sequence start reads the current row and is then skipped), so
+// all twelve are in flight together instead of one after another.  The L2 norms are half-warp or quarter-warp
 // shuffle sums.  HBM-bound: read x_q, x_k, x_v, beta_raw, a_raw; write q, k,
 // v, beta, log a.
 #include <cuda_bf16.h>
@@ -70,11 +72,45 @@ __device__ __forceinline__ int64_t seq_start(const int32_t* __restrict__ cu, int
     return __ldg(cu + found);
 }
 
+// Eight consecutive raw values of x_q / x_k / x_v, held as loaded (16 bytes
+// of bf16 or 32 bytes of fp32) until the conv uses them.
+template <typename T>
+struct Raw8;
+template <>
+struct Raw8<__nv_bfloat16> {
+    uint4 u;
+    __device__ __forceinline__ void load(const __nv_bfloat16* p) {
+        u = __ldg(reinterpret_cast<const uint4*>(p));
+    }
+    __device__ __forceinline__ void to_f32(float* x) const {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+            x[2 * i] = f.x;
+            x[2 * i + 1] = f.y;
+        }
+    }
+};
+template <>
+struct Raw8<float> {
+    float4 a, b;
+    __device__ __forceinline__ void load(const float* p) {
+        a = __ldg(reinterpret_cast<const float4*>(p));
+        b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    }
+    __device__ __forceinline__ void to_f32(float* x) const {
+        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+        x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+    }
+};
+
 // y[0..7] = sum over the taps j = 0..3 with t - 3 + j >= s of
-// w[c][j] * x[t - 3 + j][c], c = c0 .. c0 + 7 (w row-major [H D, 4]).
+// w[c][j] * x[t - 3 + j][c], c = c0 .. c0 + 7 (w row-major [H D, 4]); r[j]
+// holds tap j's values (any row when the tap is before the sequence start).
 template <typename T, int D>
-__device__ __forceinline__ void conv4(const T* __restrict__ x, const float* __restrict__ w,
-                                      int64_t t, int64_t s, int H, int h, int c0, float* y) {
+__device__ __forceinline__ void conv4(const Raw8<T> (&r)[4], const float* __restrict__ w,
+                                      int64_t t, int64_t s, int h, int c0, float* y) {
     float wt[8][4];
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
@@ -85,12 +121,11 @@ __device__ __forceinline__ void conv4(const T* __restrict__ x, const float* __re
     for (int e = 0; e < 8; ++e) y[e] = 0.f;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        const int64_t tt = t - 3 + j;
-        if (tt >= s) {
-            float xv[8];
-            load8(x + ((size_t)tt * H + h) * D + c0, xv);
+        if (t - 3 + j >= s) {
+            float x[8];
+            r[j].to_f32(x);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) y[e] = fmaf(wt[e][j], xv[e], y[e]);
+            for (int e = 0; e < 8; ++e) y[e] = fmaf(wt[e][j], x[e], y[e]);
         }
     }
 }
@@ -125,9 +160,11 @@ __device__ __forceinline__ float sigmoid(float z) {
 }
 
 // Grid-stride over (token, head) units, warp-uniform: every lane of a warp
-// runs the same iterations, lanes past the end only join the shuffles.
+// runs the same iterations; lanes past the end work on the last unit (so
+// every address is valid), join the shuffles and store nothing.  All global
+// loads of an iteration are issued before any of them is used.
 template <typename T, int D, bool SCALAR>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
 preprocess_kernel(int n_seqs, int H, int64_t units, const int32_t* __restrict__ cu,
                   const T* __restrict__ xq, const T* __restrict__ xk, const T* __restrict__ xv,
                   const float* __restrict__ wq, const float* __restrict__ wk,
@@ -143,38 +180,53 @@ preprocess_kernel(int n_seqs, int H, int64_t units, const int32_t* __restrict__ 
     const int64_t warp = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / 32;
     const int64_t n_warps = (int64_t)gridDim.x * kThreads / 32;
     for (int64_t base = warp * kUnitsPerWarp; base < units; base += n_warps * kUnitsPerWarp) {
-        const int64_t u = base + lane / G;
-        const bool valid = u < units;
-        const int64_t t = valid ? u / H : 0;
-        const int h = valid ? (int)(u - t * H) : 0;
-        const int64_t s = valid ? seq_start(cu, n_seqs, t) : 0;
-        float yq[8], yk[8], yv[8];
-        if (valid) {
-            conv4<T, D>(xq, wq, t, s, H, h, c0, yq);
-            conv4<T, D>(xk, wk, t, s, H, h, c0, yk);
-            conv4<T, D>(xv, wv, t, s, H, h, c0, yv);
-        } else {
+        const int64_t u0 = base + lane / G;
+        const bool valid = u0 < units;
+        const int64_t u = valid ? u0 : units - 1;
+        const int64_t t = u / H;
+        const int h = (int)(u - t * H);
+        const int64_t s = seq_start(cu, n_seqs, t);
+
+        Raw8<T> rq[4], rk[4], rv[4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) yq[e] = yk[e] = yv[e] = 0.f;
+        for (int j = 0; j < 4; ++j) {
+            const int64_t tt = (t - 3 + j >= s) ? t - 3 + j : t;   // a valid row either way
+            const size_t off = ((size_t)tt * H + h) * D + c0;
+            rq[j].load(xq + off);
+            rk[j].load(xk + off);
+            rv[j].load(xv + off);
         }
+        const size_t row = (size_t)u * D + c0;
+        float z[8];
+        if (SCALAR) {
+            z[0] = __ldg(a_raw + u) + __ldg(a_bias + h);
+        } else {
+            float bz[8];
+            load8(a_raw + row, z);
+            load8(a_bias + (size_t)h * D + c0, bz);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) z[e] += bz[e];
+        }
+        const float br = __ldg(beta_raw + u);
+
+        float yq[8], yk[8], yv[8];
+        conv4<T, D>(rq, wq, t, s, h, c0, yq);
+        conv4<T, D>(rk, wk, t, s, h, c0, yk);
+        conv4<T, D>(rv, wv, t, s, h, c0, yv);
         l2_normalise<G>(yq);
         l2_normalise<G>(yk);
         if (!valid) continue;
-        const size_t row = (size_t)u * D + c0;
         store8(q + row, yq);
         store8(k + row, yk);
         store8(v + row, yv);
         if (SCALAR) {
-            if (sub == 0) log_a[u] = log_sigmoid(__ldg(a_raw + u) + __ldg(a_bias + h));
+            if (sub == 0) log_a[u] = log_sigmoid(z[0]);
         } else {
-            float z[8], bz[8];
-            load8(a_raw + row, z);
-            load8(a_bias + (size_t)h * D + c0, bz);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) z[e] = log_sigmoid(z[e] + bz[e]);
+            for (int e = 0; e < 8; ++e) z[e] = log_sigmoid(z[e]);
             store8(log_a + row, z);
         }
-        if (sub == 0) beta[u] = sigmoid(__ldg(beta_raw + u));
+        if (sub == 0) beta[u] = sigmoid(br);
     }
 }
 
