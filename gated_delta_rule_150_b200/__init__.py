@@ -142,6 +142,66 @@ def _need_cuda(*ts):
                 raise ValueError("all tensors must be contiguous")
 
 
+def _expect(t, shape, dtype, name):
+    """Raise unless ``t`` (when given) has exactly ``shape`` and ``dtype``.
+
+    The C ABI receives bare pointers and sizes, so a tensor of the wrong shape
+    would be read or written past its end by the kernels; every binding
+    checks its tensors' shapes here, on the host, before anything else."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _expect_dim(t, dim, name):
+    if t.dim() != dim:
+        raise ValueError(f"{name} must have {dim} dimensions, got shape {tuple(t.shape)}")
+
+
+def _check_cu(cu_seqlens, total_tokens, cu_host=None):
+    """cu_seqlens: int32, one dimension, N + 1 >= 1 entries; the host copy,
+    when there is one, must start at 0, never decrease and end at T."""
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or cu_seqlens.numel() < 1:
+        raise ValueError("cu_seqlens must be a 1-D int32 tensor with N + 1 >= 1 entries")
+    if cu_host is not None:
+        c = torch.as_tensor(cu_host, dtype=torch.int64).reshape(-1)
+        if c.numel() != cu_seqlens.numel():
+            raise ValueError("cu_seqlens_host and cu_seqlens differ in length")
+        if int(c[0]) != 0 or int(c[-1]) != total_tokens or bool((c[1:] < c[:-1]).any()):
+            raise ValueError("cu_seqlens must start at 0, never decrease and end at the "
+                             "number of tokens")
+
+
+def _check_prefill_shapes(q, k, v, beta, log_a, cu_seqlens, scalar_decay, init_state=None,
+                          out=None, final_state=None, snapshots=None, cu_host=None,
+                          snap_interval=0):
+    _expect_dim(q, 3, "q")
+    _expect_dim(v, 3, "v")
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    _dtype_code(q)
+    _expect(k, (T, H, dk), q.dtype, "k")
+    _expect(v, (T, H, dv), q.dtype, "v")
+    _expect(beta, (T, H), torch.float32, "beta")
+    _expect(log_a, (T, H) if scalar_decay else (T, H, dk), torch.float32, "log_a")
+    _check_cu(cu_seqlens, T, cu_host)
+    n = cu_seqlens.numel() - 1
+    _expect(init_state, (n, H, dv, dk), torch.float32, "init_state")
+    _expect(out, (T, H, dv), q.dtype, "out")
+    _expect(final_state, (n, H, dv, dk), torch.float32, "final_state")
+    if snapshots is not None:
+        if snapshots.dim() != 4 or tuple(snapshots.shape[1:]) != (H, dv, dk) or \
+                snapshots.dtype != torch.float32:
+            raise ValueError(f"snapshots must be float32 [S, {H}, {dv}, {dk}]")
+        if cu_host is not None and snap_interval:
+            need = snapshot_count(cu_host, snap_interval)
+            if snapshots.shape[0] < need:
+                raise ValueError(f"snapshots holds {snapshots.shape[0]} slots, {need} needed")
+
+
 def _host_cu(cu_seqlens, cu_seqlens_host):
     if cu_seqlens_host is not None:
         return torch.as_tensor(cu_seqlens_host, dtype=torch.int32).contiguous()
@@ -207,6 +267,8 @@ def prefill(q, k, v, beta, log_a, cu_seqlens, *, scalar_decay=False, scale=1.0,
     """
     if q.dtype != k.dtype or q.dtype != v.dtype:
         raise TypeError("q, k and v must share a dtype")
+    _check_prefill_shapes(q, k, v, beta, log_a, cu_seqlens, scalar_decay, init_state, out,
+                          final_state, snapshots, cu_seqlens_host, snap_interval)
     _need_cuda(q, k, v, beta, log_a, cu_seqlens, init_state, out, final_state, snapshots,
                workspace)
     T, H, dk = q.shape
@@ -250,6 +312,12 @@ class PreparedPrefill:
     def __init__(self, q, k, v, beta, log_a, cu_seqlens, *, out, final_state, workspace,
                  scalar_decay=False, scale=1.0, init_state=None, snap_interval=0,
                  snapshots=None):
+        _check_prefill_shapes(q, k, v, beta, log_a, cu_seqlens, scalar_decay, init_state, out,
+                              final_state, snapshots)
+        if out is None or final_state is None or workspace is None:
+            raise ValueError("PreparedPrefill needs out, final_state and workspace")
+        if snap_interval and snapshots is None:
+            raise ValueError("snap_interval > 0 needs a snapshots buffer")
         _need_cuda(q, k, v, beta, log_a, cu_seqlens, out, final_state, workspace, init_state,
                    snapshots)
         self._keep = (q, k, v, beta, log_a, cu_seqlens, out, final_state, workspace,
@@ -278,9 +346,16 @@ def prefill_status(workspace) -> None:
 
 def cumdecay(log_a, cu_seqlens, *, scalar_decay=False, d_k=None, out=None):
     """Chunk-local cumulative log decay (the first prefill kernel on its own)."""
-    _need_cuda(log_a, cu_seqlens, out)
+    _expect_dim(log_a, 2 if scalar_decay else 3, "log_a")
+    if log_a.dtype != torch.float32:
+        raise TypeError("log_a must be float32")
     T, H = log_a.shape[0], log_a.shape[1]
+    if scalar_decay and d_k is None:
+        raise ValueError("a scalar gate needs d_k")
     dk = d_k if scalar_decay else log_a.shape[2]
+    _check_cu(cu_seqlens, T)
+    _expect(out, tuple(log_a.shape), torch.float32, "out")
+    _need_cuda(log_a, cu_seqlens, out)
     if out is None:
         out = torch.empty_like(log_a)
     _check(lib().gdr_cumdecay(cu_seqlens.numel() - 1, H, dk, T, _ptr(cu_seqlens), _ptr(log_a),
@@ -291,6 +366,9 @@ def cumdecay(log_a, cu_seqlens, *, scalar_decay=False, d_k=None, out=None):
 
 def chunk_factors(q, k, v, beta, log_a, cu_seqlens, *, scalar_decay=False, scale=1.0):
     """Per-chunk affine map of the state (Qt, PU, BS, NC, gamma) per chunk slot, fp32."""
+    if q.dtype != k.dtype or q.dtype != v.dtype:
+        raise TypeError("q, k and v must share a dtype")
+    _check_prefill_shapes(q, k, v, beta, log_a, cu_seqlens, scalar_decay)
     _need_cuda(q, k, v, beta, log_a, cu_seqlens)
     T, H, dk = q.shape
     dv = v.shape[-1]
@@ -315,11 +393,17 @@ def decode_step(state, q, k, v, beta, log_a, *, scalar_decay=False, scale=1.0, o
     Returns o [B, H, d_v] fp32."""
     if q.dtype != k.dtype or q.dtype != v.dtype:
         raise TypeError("q, k and v must share a dtype")
-    _need_cuda(state, q, k, v, beta, log_a, out)
-    if state.dtype != torch.float32:
-        raise TypeError("state must be float32")
+    _expect_dim(q, 3, "q")
+    _expect_dim(v, 3, "v")
     B, H, dk = q.shape
     dv = v.shape[-1]
+    _dtype_code(q)
+    _expect(k, (B, H, dk), q.dtype, "k")
+    _expect(beta, (B, H), torch.float32, "beta")
+    _expect(log_a, (B, H) if scalar_decay else (B, H, dk), torch.float32, "log_a")
+    _expect(state, (B, H, dv, dk), torch.float32, "state")
+    _expect(out, (B, H, dv), torch.float32, "out")
+    _need_cuda(state, q, k, v, beta, log_a, out)
     if out is None:
         out = torch.empty(B, H, dv, dtype=torch.float32, device=q.device)
     _check(lib().gdr_decode_step(B, H, dk, dv, _dtype_code(q), _ptr(q), _ptr(k), _ptr(v),
@@ -340,13 +424,19 @@ def decode_draft(state, q, k, v, beta, log_a, *, scalar_decay=False, scale=1.0, 
     """
     if q.dtype != k.dtype or q.dtype != v.dtype:
         raise TypeError("q, k and v must share a dtype")
-    _need_cuda(state, q, k, v, beta, log_a, out, token_states)
-    if state.dtype != torch.float32:
-        raise TypeError("state must be float32")
+    _expect_dim(q, 4, "q")
+    _expect_dim(v, 4, "v")
     B, K, H, dk = q.shape
     dv = v.shape[-1]
-    if tuple(state.shape) != (B, H, dv, dk):
-        raise ValueError(f"state must be [B, H, d_v, d_k] = {(B, H, dv, dk)}")
+    _dtype_code(q)
+    _expect(k, (B, K, H, dk), q.dtype, "k")
+    _expect(v, (B, K, H, dv), q.dtype, "v")
+    _expect(beta, (B, K, H), torch.float32, "beta")
+    _expect(log_a, (B, K, H) if scalar_decay else (B, K, H, dk), torch.float32, "log_a")
+    _expect(state, (B, H, dv, dk), torch.float32, "state")
+    _expect(out, (B, K, H, dv), torch.float32, "out")
+    _expect(token_states, (B, K, H, dv, dk), torch.float32, "token_states")
+    _need_cuda(state, q, k, v, beta, log_a, out, token_states)
     if out is None:
         out = torch.empty(B, K, H, dv, dtype=torch.float32, device=q.device)
     if token_states is None:
@@ -362,13 +452,12 @@ def decode_accept(state, token_states, n_accept):
     """Rollback after verification, in place: ``state[b]`` becomes
     ``token_states[b, n - 1]`` for n = n_accept[b] in 1 .. K and is left as it
     is for n = 0 (n clamped to [0, K]).  ``n_accept`` is a device int32 [B]."""
-    _need_cuda(state, token_states, n_accept)
-    if n_accept.dtype != torch.int32:
-        raise TypeError("n_accept must be int32")
+    _expect_dim(token_states, 5, "token_states")
     B, K, H, dv, dk = token_states.shape
-    if tuple(state.shape) != (B, H, dv, dk) or n_accept.numel() != B:
-        raise ValueError("state must be [B, H, d_v, d_k] and n_accept [B] for token_states "
-                         "[B, K, H, d_v, d_k]")
+    _expect(token_states, (B, K, H, dv, dk), torch.float32, "token_states")
+    _expect(state, (B, H, dv, dk), torch.float32, "state")
+    _expect(n_accept, (B,), torch.int32, "n_accept")
+    _need_cuda(state, token_states, n_accept)
     _check(lib().gdr_decode_accept(B, K, H, dk, dv, _ptr(n_accept), _ptr(token_states),
                                    _ptr(state), _stream(state.device)),
            "gdr_decode_accept")
@@ -388,7 +477,22 @@ def preprocess(xq, xk, xv, conv_q, conv_k, conv_v, beta_raw, a_raw, a_bias, cu_s
     """
     if xq.dtype != xk.dtype or xq.dtype != xv.dtype:
         raise TypeError("xq, xk and xv must share a dtype")
+    _expect_dim(xq, 3, "xq")
     T, H, d = xq.shape
+    _dtype_code(xq)
+    for name, t in (("xk", xk), ("xv", xv)):
+        _expect(t, (T, H, d), xq.dtype, name)
+    for name, t in (("conv_q", conv_q), ("conv_k", conv_k), ("conv_v", conv_v)):
+        _expect(t, (H * d, 4), torch.float32, name)
+    _expect(beta_raw, (T, H), torch.float32, "beta_raw")
+    _expect(a_raw, (T, H) if scalar_decay else (T, H, d), torch.float32, "a_raw")
+    _expect(a_bias, (H,) if scalar_decay else (H, d), torch.float32, "a_bias")
+    _check_cu(cu_seqlens, T)
+    if out:
+        for name in ("q", "k", "v"):
+            _expect(out.get(name), (T, H, d), xq.dtype, f"out[{name!r}]")
+        _expect(out.get("beta"), (T, H), torch.float32, "out['beta']")
+        _expect(out.get("log_a"), tuple(a_raw.shape), torch.float32, "out['log_a']")
     dev = xq.device
     out = dict(out or {})
     for name in ("q", "k", "v"):
@@ -400,9 +504,6 @@ def preprocess(xq, xk, xv, conv_q, conv_k, conv_v, beta_raw, a_raw, a_bias, cu_s
         out["log_a"] = torch.empty(a_raw.shape, device=dev)
     _need_cuda(xq, xk, xv, conv_q, conv_k, conv_v, beta_raw, a_raw, a_bias, cu_seqlens,
                *out.values())
-    for t in (conv_q, conv_k, conv_v, beta_raw, a_raw, a_bias):
-        if t.dtype != torch.float32:
-            raise TypeError("conv taps, beta_raw, a_raw and a_bias must be float32")
     a = PreprocessArgs()
     a.n_seqs, a.n_heads, a.d, a.total_tokens = cu_seqlens.numel() - 1, H, d, T
     a.cu_seqlens = cu_seqlens.data_ptr()
