@@ -16,9 +16,12 @@
 // earlier rows were just read by neighbouring warps and come from L1/L2, so
 // HBM sees each row about once).  The tap loads are unconditional (a tap
 // before the sequence start reads the current row and is then skipped), so
-// all twelve are in flight together instead of one after another.  The L2 norms are half-warp or quarter-warp
-// shuffle sums.  HBM-bound: read x_q, x_k, x_v, beta_raw, a_raw; write q, k,
-// v, beta, log a.
+// all twelve are in flight together instead of one after another.  The L2
+// norms are shuffle sums over the D / 8 lanes of a (token, head).  The HBM
+// traffic is x_q, x_k, x_v, beta_raw, a_raw read and q, k, v, beta, log a
+// written, once each; the conv taps' per-thread loads (eight 16-byte loads
+// whose lanes sit 128 bytes apart) cost more L1 wavefronts than that traffic
+// takes in HBM time, so the kernel is L1-bound at d 64.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -28,22 +31,12 @@ namespace {
 
 constexpr int kThreads = 256;
 
-// Eight consecutive values from p (16-byte aligned) as fp32.
+// Eight consecutive fp32 values from p (16-byte aligned).
 __device__ __forceinline__ void load8(const float* p, float* x) {
     const float4 a = __ldg(reinterpret_cast<const float4*>(p));
     const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
     x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
     x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-}
-__device__ __forceinline__ void load8(const __nv_bfloat16* p, float* x) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
-        x[2 * i] = f.x;
-        x[2 * i + 1] = f.y;
-    }
 }
 
 __device__ __forceinline__ void store8(float* p, const float* x) {
