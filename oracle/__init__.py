@@ -9,6 +9,8 @@ Contents
 --------
 * ``prefill`` / ``decode_step``: the token-by-token recurrence in plain C
   (``gdr_oracle.c``, fp64, OpenMP over (sequence, head)), wrapped with ctypes.
+* ``output_epilogue``: the per-head RMSNorm of o and the sigmoid output gate
+  that follow the mixer (numpy, fp64).
 * ``decode_draft`` / ``decode_accept``: speculative decoding with rollback --
   K draft tokens that keep the state after each token, then the state of the
   accepted prefix (same C file).
@@ -375,3 +377,18 @@ def preprocess(xq, xk, xv, conv_q, conv_k, conv_v, beta_raw, a_raw, a_bias, cu_s
     beta = sigmoid(f64(beta_raw))
     z = f64(a_raw) + f64(a_bias)[None]
     return dict(q=q, k=k, v=v, beta=beta, log_a=log_sigmoid(z))
+
+
+def output_epilogue(o, gate_raw, norm_weight, eps: float = 1e-6) -> np.ndarray:
+    """The mixer's output after its RMSNorm and output gate (fp64).
+
+    "kda-graft", section "Идея и архитектура": the graft adds an output gate
+    and an RMSNorm to each KDA layer; the page gives no formulas.  Readings:
+    the norm runs over the d_v channels of each (token, head) with one weight
+    vector [d_v] shared by the heads and eps = 1e-6; the gate is the sigmoid of
+    a raw gate projection [T, H, d_v]:
+        y = o / sqrt(mean_c o_c^2 + eps) * norm_weight * sigmoid(gate_raw)
+    """
+    o = f64(o)
+    ms = np.mean(o * o, axis=-1, keepdims=True)
+    return o / np.sqrt(ms + eps) * f64(norm_weight) * sigmoid(f64(gate_raw))
