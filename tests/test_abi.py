@@ -179,3 +179,18 @@ def test_prefill_stage_range_and_kernel_count(L):
 def test_static_workspace_is_declared_with_its_limit():
     src = open(os.path.join(ROOT, "include", "gdr.h")).read()
     assert "GDR_STATIC_WORKSPACE_BYTES" in src
+
+
+def test_header_is_plain_c():
+    """include/gdr.h is a C header: it compiles as C99 (and as C++17) with
+    warnings enabled, with no CUDA or torch include."""
+    import shutil
+    import subprocess
+    hdr = os.path.join(ROOT, "include", "gdr.h")
+    src = open(hdr).read()
+    assert "cuda" not in re.findall(r"#include\s*[<\"]([^>\"]+)", src.lower())
+    for cc, std, lang in (("gcc", "-std=c99", "c"), ("g++", "-std=c++17", "c++")):
+        if shutil.which(cc) is None:
+            pytest.skip(f"{cc} not available")
+        subprocess.run([cc, std, "-Wall", "-Wextra", "-Werror", "-fsyntax-only", "-x", lang, hdr],
+                       check=True)
