@@ -188,7 +188,8 @@ def test_header_is_plain_c():
     import subprocess
     hdr = os.path.join(ROOT, "include", "gdr.h")
     src = open(hdr).read()
-    assert "cuda" not in re.findall(r"#include\s*[<\"]([^>\"]+)", src.lower())
+    includes = re.findall(r"#include\s*[<\"]([^>\"]+)", src.lower())
+    assert not any("cuda" in inc or "torch" in inc for inc in includes), includes
     for cc, std, lang in (("gcc", "-std=c99", "c"), ("g++", "-std=c++17", "c++")):
         if shutil.which(cc) is None:
             pytest.skip(f"{cc} not available")
