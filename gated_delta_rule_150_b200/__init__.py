@@ -21,7 +21,7 @@ import torch
 
 __all__ = ["PrefillArgs", "PreparedPrefill", "prefill", "kernel_count", "decode_step",
            "decode_draft", "decode_accept", "PreprocessArgs", "preprocess", "cumdecay", "chunk_factors", "workspace_size",
-           "snapshot_count", "prefill_status", "lib", "GdrError", "LIB_PATH"]
+           "snapshot_count", "snapshot_offsets", "prefill_status", "lib", "GdrError", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_build", "libgdr.so")
 
@@ -47,7 +47,9 @@ class PrefillArgs(ctypes.Structure):
         ("beta", ctypes.c_void_p), ("log_a", ctypes.c_void_p), ("scalar_decay", ctypes.c_int),
         ("scale", ctypes.c_float), ("init_state", ctypes.c_void_p), ("o", ctypes.c_void_p),
         ("final_state", ctypes.c_void_p), ("snap_interval", ctypes.c_int),
-        ("snapshots", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
+        ("snapshots", ctypes.c_void_p), ("snap_offsets", ctypes.c_void_p),
+        ("gate_raw", ctypes.c_void_p), ("norm_weight", ctypes.c_void_p),
+        ("norm_eps", ctypes.c_float), ("workspace", ctypes.c_void_p),
         ("workspace_bytes", ctypes.c_size_t),
     ]
 
@@ -89,6 +91,12 @@ def lib():
             L.gdr_prefill_kernel_count.argtypes = [i, i, i, i, i64, i]
             L.gdr_snapshot_count.restype = i64
             L.gdr_snapshot_count.argtypes = [vp, i, i]
+            L.gdr_snapshot_offsets.restype = i
+            L.gdr_snapshot_offsets.argtypes = [vp, i, i, vp]
+            L.gdr_prefill_static_workspace.restype = i
+            L.gdr_prefill_static_workspace.argtypes = [ctypes.POINTER(PrefillArgs), vp]
+            L.gdr_prefill_static_status.restype = i
+            L.gdr_prefill_static_status.argtypes = [vp]
             L.gdr_prefill.restype = i
             L.gdr_prefill.argtypes = [ctypes.POINTER(PrefillArgs), vp]
             L.gdr_prefill_stages.restype = i
@@ -101,6 +109,9 @@ def lib():
             L.gdr_chunk_factors.argtypes = [ctypes.POINTER(PrefillArgs), vp, vp, vp, vp, vp, vp]
             L.gdr_decode_step.restype = i
             L.gdr_decode_step.argtypes = [i, i, i, i, i, vp, vp, vp, vp, vp, i, f, vp, vp, vp]
+            L.gdr_decode_step_gated.restype = i
+            L.gdr_decode_step_gated.argtypes = [i, i, i, i, i, vp, vp, vp, vp, vp, i, f, vp, vp,
+                                                vp, f, vp, vp]
             L.gdr_preprocess.restype = i
             L.gdr_preprocess.argtypes = [ctypes.POINTER(PreprocessArgs), vp]
             L.gdr_decode_draft.restype = i
@@ -140,6 +151,17 @@ def _need_cuda(*ts):
                 raise ValueError("all tensors must be CUDA tensors")
             if not t.is_contiguous():
                 raise ValueError("all tensors must be contiguous")
+
+
+def _check_snapshot_buffer(snapshots):
+    """Snapshots go to device memory or, for offload, to page-locked host
+    memory that the kernels write over the host link."""
+    if snapshots is None:
+        return
+    if not snapshots.is_contiguous():
+        raise ValueError("snapshots must be contiguous")
+    if not (snapshots.is_cuda or snapshots.is_pinned()):
+        raise ValueError("snapshots must be a CUDA tensor or pinned host memory")
 
 
 def _expect(t, shape, dtype, name):
@@ -228,8 +250,34 @@ def snapshot_count(cu_seqlens_host, snap_interval: int) -> int:
     return n
 
 
+def snapshot_offsets(cu_seqlens_host, snap_interval: int) -> torch.Tensor:
+    """First snapshot slot of every sequence (int64 [N+1], host); entry N is
+    the slot count.  Sequence n's m-th snapshot is slot offsets[n] + m - 1."""
+    cu = torch.as_tensor(cu_seqlens_host, dtype=torch.int32).contiguous()
+    out = torch.empty(cu.numel(), dtype=torch.int64)
+    _check(lib().gdr_snapshot_offsets(ctypes.c_void_p(cu.data_ptr()), cu.numel() - 1,
+                                      int(snap_interval), ctypes.c_void_p(out.data_ptr())),
+           "gdr_snapshot_offsets")
+    return out
+
+
+def _check_gate(gate_raw, norm_weight, norm_eps, o_shape, dtype):
+    """The output epilogue's inputs: raw gate shaped like o (o's dtype),
+    weight [d_v] fp32, eps >= 0; both or neither."""
+    if gate_raw is None and norm_weight is None:
+        return
+    if gate_raw is None or norm_weight is None:
+        raise ValueError("the output epilogue needs both gate_raw and norm_weight")
+    _expect(gate_raw, o_shape, dtype, "gate_raw")
+    _expect(norm_weight, (o_shape[-1],), torch.float32, "norm_weight")
+    if not norm_eps >= 0.0:
+        raise ValueError("norm_eps must be >= 0")
+    _need_cuda(gate_raw, norm_weight)
+
+
 def _prefill_args(q, k, v, beta, log_a, cu_seqlens, scalar_decay, scale, init_state,
-                  snap_interval, o, final_state, snapshots, workspace):
+                  snap_interval, o, final_state, snapshots, workspace, snap_offsets=None,
+                  gate_raw=None, norm_weight=None, norm_eps=1e-6):
     T, H, dk = q.shape
     a = PrefillArgs()
     a.n_seqs = cu_seqlens.numel() - 1
@@ -248,6 +296,10 @@ def _prefill_args(q, k, v, beta, log_a, cu_seqlens, scalar_decay, scale, init_st
     a.final_state = None if final_state is None else final_state.data_ptr()
     a.snap_interval = int(snap_interval)
     a.snapshots = None if snapshots is None else snapshots.data_ptr()
+    a.snap_offsets = None if snap_offsets is None else snap_offsets.data_ptr()
+    a.gate_raw = None if gate_raw is None else gate_raw.data_ptr()
+    a.norm_weight = None if norm_weight is None else norm_weight.data_ptr()
+    a.norm_eps = float(norm_eps)
     a.workspace = workspace.data_ptr()
     a.workspace_bytes = workspace.numel()
     return a
@@ -255,12 +307,18 @@ def _prefill_args(q, k, v, beta, log_a, cu_seqlens, scalar_decay, scale, init_st
 
 def prefill(q, k, v, beta, log_a, cu_seqlens, *, scalar_decay=False, scale=1.0,
             init_state=None, snap_interval=0, cu_seqlens_host=None, out=None,
-            final_state=None, snapshots=None, workspace=None, stages=(0, 1)):
+            final_state=None, snapshots=None, workspace=None, stages=(0, 1),
+            snap_offsets=None, gate_raw=None, norm_weight=None, norm_eps=1e-6):
     """Chunked prefill over a packed batch.  Returns (o, final_state, snapshots).
 
     ``cu_seqlens`` is a device int32 tensor [N+1]; its host copy (taken from
     ``cu_seqlens_host`` when given, else read back) sizes the snapshots.
     Output buffers and the workspace may be passed in to avoid allocation.
+    ``snap_offsets`` (device int64 [N+1], from ``snapshot_offsets``) gives
+    each sequence's first snapshot slot to the kernels; ``snapshots`` may be
+    pinned host memory (written by the kernels over the host link).
+    ``gate_raw`` [T, H, d_v] (q's dtype) with ``norm_weight`` [d_v] fp32 turns
+    on the output epilogue: o = RMSNorm(o) * norm_weight * sigmoid(gate_raw).
     ``stages`` = (first, last) runs only that range of the two stages
     (0 intra-chunk factors with the cumulative decay, 1 state pass), for
     timing them apart.
@@ -269,8 +327,12 @@ def prefill(q, k, v, beta, log_a, cu_seqlens, *, scalar_decay=False, scale=1.0,
         raise TypeError("q, k and v must share a dtype")
     _check_prefill_shapes(q, k, v, beta, log_a, cu_seqlens, scalar_decay, init_state, out,
                           final_state, snapshots, cu_seqlens_host, snap_interval)
-    _need_cuda(q, k, v, beta, log_a, cu_seqlens, init_state, out, final_state, snapshots,
-               workspace)
+    if snap_offsets is not None:
+        _expect(snap_offsets, (cu_seqlens.numel(),), torch.int64, "snap_offsets")
+    _check_gate(gate_raw, norm_weight, norm_eps, (q.shape[0], q.shape[1], v.shape[-1]), q.dtype)
+    _need_cuda(q, k, v, beta, log_a, cu_seqlens, init_state, out, final_state, workspace,
+               snap_offsets)
+    _check_snapshot_buffer(snapshots)
     T, H, dk = q.shape
     dv = v.shape[-1]
     n = cu_seqlens.numel() - 1
@@ -292,7 +354,8 @@ def prefill(q, k, v, beta, log_a, cu_seqlens, *, scalar_decay=False, scale=1.0,
         # no full interval in any sequence: any valid aligned pointer will do
         snap_arg = final_state
     a = _prefill_args(q, k, v, beta, log_a, cu_seqlens, scalar_decay, scale, init_state,
-                      snap_interval, out, final_state, snap_arg, workspace)
+                      snap_interval, out, final_state, snap_arg, workspace, snap_offsets,
+                      gate_raw, norm_weight, norm_eps)
     first, last = stages
     if (first, last) == (0, 1):
         _check(lib().gdr_prefill(ctypes.byref(a), _stream(dev)), "gdr_prefill")
@@ -311,20 +374,22 @@ class PreparedPrefill:
 
     def __init__(self, q, k, v, beta, log_a, cu_seqlens, *, out, final_state, workspace,
                  scalar_decay=False, scale=1.0, init_state=None, snap_interval=0,
-                 snapshots=None):
+                 snapshots=None, gate_raw=None, norm_weight=None, norm_eps=1e-6):
         _check_prefill_shapes(q, k, v, beta, log_a, cu_seqlens, scalar_decay, init_state, out,
                               final_state, snapshots)
         if out is None or final_state is None or workspace is None:
             raise ValueError("PreparedPrefill needs out, final_state and workspace")
+        _check_gate(gate_raw, norm_weight, norm_eps, tuple(out.shape), q.dtype)
         if snap_interval and snapshots is None:
             raise ValueError("snap_interval > 0 needs a snapshots buffer")
-        _need_cuda(q, k, v, beta, log_a, cu_seqlens, out, final_state, workspace, init_state,
-                   snapshots)
+        _need_cuda(q, k, v, beta, log_a, cu_seqlens, out, final_state, workspace, init_state)
+        _check_snapshot_buffer(snapshots)
         self._keep = (q, k, v, beta, log_a, cu_seqlens, out, final_state, workspace,
-                      init_state, snapshots)
+                      init_state, snapshots, gate_raw, norm_weight)
         self.args = _prefill_args(q, k, v, beta, log_a, cu_seqlens, scalar_decay, scale,
                                   init_state, snap_interval, out, final_state,
-                                  snapshots if snap_interval else None, workspace)
+                                  snapshots if snap_interval else None, workspace, None,
+                                  gate_raw, norm_weight, norm_eps)
         self.device = q.device
         self.out, self.final_state, self.snapshots, self.workspace = out, final_state, snapshots, workspace
         lib()
@@ -388,9 +453,11 @@ def chunk_factors(q, k, v, beta, log_a, cu_seqlens, *, scalar_decay=False, scale
     return f
 
 
-def decode_step(state, q, k, v, beta, log_a, *, scalar_decay=False, scale=1.0, out=None):
+def decode_step(state, q, k, v, beta, log_a, *, scalar_decay=False, scale=1.0, out=None,
+                gate_raw=None, norm_weight=None, norm_eps=1e-6):
     """One decode step; ``state`` [B, H, d_v, d_k] fp32 is updated in place.
-    Returns o [B, H, d_v] fp32."""
+    Returns o [B, H, d_v] fp32 (after the output epilogue when ``gate_raw``
+    [B, H, d_v] and ``norm_weight`` [d_v] are given)."""
     if q.dtype != k.dtype or q.dtype != v.dtype:
         raise TypeError("q, k and v must share a dtype")
     _expect_dim(q, 3, "q")
@@ -404,12 +471,21 @@ def decode_step(state, q, k, v, beta, log_a, *, scalar_decay=False, scale=1.0, o
     _expect(state, (B, H, dv, dk), torch.float32, "state")
     _expect(out, (B, H, dv), torch.float32, "out")
     _need_cuda(state, q, k, v, beta, log_a, out)
+    _check_gate(gate_raw, norm_weight, norm_eps, (B, H, dv), q.dtype)
     if out is None:
         out = torch.empty(B, H, dv, dtype=torch.float32, device=q.device)
-    _check(lib().gdr_decode_step(B, H, dk, dv, _dtype_code(q), _ptr(q), _ptr(k), _ptr(v),
-                                 _ptr(beta), _ptr(log_a), int(bool(scalar_decay)), float(scale),
-                                 _ptr(state), _ptr(out), _stream(q.device)),
-           "gdr_decode_step")
+    if gate_raw is None:
+        _check(lib().gdr_decode_step(B, H, dk, dv, _dtype_code(q), _ptr(q), _ptr(k), _ptr(v),
+                                     _ptr(beta), _ptr(log_a), int(bool(scalar_decay)), float(scale),
+                                     _ptr(state), _ptr(out), _stream(q.device)),
+               "gdr_decode_step")
+    else:
+        _check(lib().gdr_decode_step_gated(B, H, dk, dv, _dtype_code(q), _ptr(q), _ptr(k), _ptr(v),
+                                           _ptr(beta), _ptr(log_a), int(bool(scalar_decay)),
+                                           float(scale), _ptr(state), _ptr(gate_raw),
+                                           _ptr(norm_weight), float(norm_eps), _ptr(out),
+                                           _stream(q.device)),
+               "gdr_decode_step_gated")
     return out
 
 

@@ -63,5 +63,34 @@ def build(force: bool = False, verbose: bool = False, out: str = LIB, extra=()) 
     return out
 
 
+# A copy of the library for the bounded-wait test: the state-pass kernels wait,
+# at their second chunk, for a barrier nothing arrives on, with a 1 ms limit,
+# so that the timeout path (error word, drain, GDR_ERR_TIMEOUT) runs on demand.
+# Everything else is the regular library's objects.
+WAIT_TEST_LIB = os.path.join(OUT_DIR, "libgdr_waittest.so")
+WAIT_TEST_DEFINES = ["-DGDR_TEST_WAIT_LIMIT_NS=1000000"]
+
+
+def build_wait_test(force: bool = False) -> str:
+    build()
+    variant_src = os.path.join(CSRC, "state_pass.cu")
+    if not force and not _stale(WAIT_TEST_LIB, sources()):
+        return WAIT_TEST_LIB
+    vdir = os.path.join(OUT_DIR, "waittest")
+    os.makedirs(vdir, exist_ok=True)
+    vobj = os.path.join(vdir, "state_pass.o")
+    subprocess.run([_nvcc(), *NVCC_FLAGS, *WAIT_TEST_DEFINES, "-I", os.path.join(ROOT, "include"),
+                    "-I", CSRC, "-c", variant_src, "-o", vobj], check=True)
+    objs = [os.path.join(OUT_DIR, os.path.splitext(os.path.basename(src))[0] + ".o")
+            for src in sources() if src != variant_src] + [vobj]
+    tmp = WAIT_TEST_LIB + f".tmp{os.getpid()}"
+    subprocess.run([_nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared",
+                    "-Xcompiler", "-fPIC", "-o", tmp, *objs], check=True)
+    os.replace(tmp, WAIT_TEST_LIB)
+    return WAIT_TEST_LIB
+
+
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    if "--wait-test" in sys.argv:
+        print(build_wait_test(force="--force" in sys.argv))

@@ -47,13 +47,23 @@ __device__ __forceinline__ float sum16(float x) {
     return x;
 }
 
+// Output epilogue ("kda-graft", section "Идея и архитектура": each KDA layer
+// of the graft ends in an RMSNorm and an output gate): over the d_v outputs
+// of a (sequence, head), o = x / sqrt(mean x^2 + eps) * w * sigmoid(gate_raw).
+template <typename T>
+struct DecodeGate {
+    const T* gate;           // [B, H, d_v]
+    const float* weight;     // [d_v]
+    float eps;
+};
+
 // One CTA per (sequence, head).  Thread t handles row group t / 16 and the
 // float4 columns {t % 16 + 16 i}.  DK/64 float4 per thread per row.
-template <typename T, int DK, int DV, bool SCALAR>
+template <typename T, int DK, int DV, bool SCALAR, bool GATED>
 __global__ void __launch_bounds__(kThreads)
 decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                    const float* __restrict__ beta, const float* __restrict__ log_a, float scale,
-                   float* __restrict__ state, float* __restrict__ o) {
+                   float* __restrict__ state, float* __restrict__ o, const DecodeGate<T> og) {
     constexpr int NV = DK / (4 * kTPR);        // float4 per thread per row: 1 or 2
     constexpr int PASSES = DV / kRowsPerPass;  // 4 or 8
     const int bh = blockIdx.x;
@@ -93,6 +103,7 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
 #pragma unroll
     for (int p = 0; p < PASSES; ++p) vv[p] = to_f<T>(v[(size_t)bh * DV + rgrp + kRowsPerPass * p]);
 
+    float ov[PASSES];                          // this row group's outputs (epilogue)
 #pragma unroll
     for (int p = 0; p < PASSES; ++p) {
         const int row = rgrp + kRowsPerPass * p;
@@ -113,32 +124,58 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
             x.x += d * kk[i].x; x.y += d * kk[i].y; x.z += d * kk[i].z; x.w += d * kk[i].w;
             *reinterpret_cast<float4*>(S + (size_t)row * DK + 4 * (lane16 + kTPR * i)) = x;
         }
-        if (lane16 == 0) o[(size_t)bh * DV + row] = pq + d * kq;
+        if (GATED) ov[p] = pq + d * kq;
+        else if (lane16 == 0) o[(size_t)bh * DV + row] = pq + d * kq;
+    }
+    if (GATED) {
+        // mean square over the d_v outputs: one partial per row group
+        __shared__ float part[kRowsPerPass];
+        float ss = 0.f;
+#pragma unroll
+        for (int p = 0; p < PASSES; ++p) ss = fmaf(ov[p], ov[p], ss);
+        if (lane16 == 0) part[rgrp] = ss;
+        __syncthreads();
+        float tot = 0.f;
+#pragma unroll
+        for (int r = 0; r < kRowsPerPass; ++r) tot += part[r];
+        const float rstd = rsqrtf(tot * (1.f / DV) + og.eps);
+#pragma unroll
+        for (int p = 0; p < PASSES; ++p) {
+            if (lane16 != p) continue;             // pass p's row is stored by lane p
+            const int row = rgrp + kRowsPerPass * p;
+            const float g = to_f<T>(og.gate[(size_t)bh * DV + row]);
+            const float sig = 1.f / (1.f + __expf(-g));
+            o[(size_t)bh * DV + row] = ov[p] * rstd * __ldg(og.weight + row) * sig;
+        }
     }
 }
 
-template <typename T, int DK, int DV>
+template <typename T, int DK, int DV, bool GATED>
 cudaError_t launch_typed(int B, int H, const void* q, const void* k, const void* v,
                          const float* beta, const float* log_a, int scalar, float scale,
-                         float* state, float* o, cudaStream_t st) {
+                         float* state, float* o, const DecodeGate<T>& og, cudaStream_t st) {
     const dim3 grid((unsigned)(B * H));
     if (scalar)
-        decode_step_kernel<T, DK, DV, true><<<grid, kThreads, 0, st>>>(
-            (const T*)q, (const T*)k, (const T*)v, beta, log_a, scale, state, o);
+        decode_step_kernel<T, DK, DV, true, GATED><<<grid, kThreads, 0, st>>>(
+            (const T*)q, (const T*)k, (const T*)v, beta, log_a, scale, state, o, og);
     else
-        decode_step_kernel<T, DK, DV, false><<<grid, kThreads, 0, st>>>(
-            (const T*)q, (const T*)k, (const T*)v, beta, log_a, scale, state, o);
+        decode_step_kernel<T, DK, DV, false, GATED><<<grid, kThreads, 0, st>>>(
+            (const T*)q, (const T*)k, (const T*)v, beta, log_a, scale, state, o, og);
     return cudaGetLastError();
 }
 
-template <typename T>
+template <typename T, bool GATED>
 cudaError_t launch_dims(int B, int H, int dk, int dv, const void* q, const void* k,
                         const void* v, const float* beta, const float* log_a, int scalar,
-                        float scale, float* state, float* o, cudaStream_t st) {
-    if (dk == 64 && dv == 64) return launch_typed<T, 64, 64>(B, H, q, k, v, beta, log_a, scalar, scale, state, o, st);
-    if (dk == 64 && dv == 128) return launch_typed<T, 64, 128>(B, H, q, k, v, beta, log_a, scalar, scale, state, o, st);
-    if (dk == 128 && dv == 64) return launch_typed<T, 128, 64>(B, H, q, k, v, beta, log_a, scalar, scale, state, o, st);
-    return launch_typed<T, 128, 128>(B, H, q, k, v, beta, log_a, scalar, scale, state, o, st);
+                        float scale, float* state, float* o, const DecodeGate<T>& og,
+                        cudaStream_t st) {
+    if (dk == 64 && dv == 64)
+        return launch_typed<T, 64, 64, GATED>(B, H, q, k, v, beta, log_a, scalar, scale, state, o, og, st);
+    if (dk == 64 && dv == 128)
+        return launch_typed<T, 64, 128, GATED>(B, H, q, k, v, beta, log_a, scalar, scale, state, o, og, st);
+    if (dk == 128 && dv == 64)
+        return launch_typed<T, 128, 64, GATED>(B, H, q, k, v, beta, log_a, scalar, scale, state, o, og, st);
+    return launch_typed<T, 128, 128, GATED>(B, H, q, k, v, beta, log_a, scalar, scale, state, o, og, st);
 }
 
 }  // namespace
@@ -148,9 +185,24 @@ cudaError_t launch_decode(int B, int H, int dk, int dv, gdr_dtype dt, const void
                           const float* log_a, int scalar, float scale, float* state,
                           float* o, cudaStream_t st) {
     if (dt == GDR_BF16)
-        return launch_dims<__nv_bfloat16>(B, H, dk, dv, q, k, v, beta, log_a, scalar, scale,
-                                          state, o, st);
-    return launch_dims<float>(B, H, dk, dv, q, k, v, beta, log_a, scalar, scale, state, o, st);
+        return launch_dims<__nv_bfloat16, false>(B, H, dk, dv, q, k, v, beta, log_a, scalar, scale,
+                                                 state, o, DecodeGate<__nv_bfloat16>{}, st);
+    return launch_dims<float, false>(B, H, dk, dv, q, k, v, beta, log_a, scalar, scale, state, o,
+                                     DecodeGate<float>{}, st);
+}
+
+cudaError_t launch_decode_gated(int B, int H, int dk, int dv, gdr_dtype dt, const void* q,
+                                const void* k, const void* v, const float* beta,
+                                const float* log_a, int scalar, float scale, float* state,
+                                const void* gate_raw, const float* norm_weight, float norm_eps,
+                                float* o, cudaStream_t st) {
+    if (dt == GDR_BF16)
+        return launch_dims<__nv_bfloat16, true>(
+            B, H, dk, dv, q, k, v, beta, log_a, scalar, scale, state, o,
+            DecodeGate<__nv_bfloat16>{static_cast<const __nv_bfloat16*>(gate_raw), norm_weight, norm_eps}, st);
+    return launch_dims<float, true>(B, H, dk, dv, q, k, v, beta, log_a, scalar, scale, state, o,
+                                    DecodeGate<float>{static_cast<const float*>(gate_raw), norm_weight,
+                                                      norm_eps}, st);
 }
 
 }  // namespace gdr

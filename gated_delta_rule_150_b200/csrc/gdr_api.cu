@@ -27,7 +27,7 @@ gdr_status check_prefill_inputs(const gdr_prefill_args* a) {
         return GDR_ERR_INVALID_ARG;
     if (a->total_tokens > (int64_t)INT32_MAX) return GDR_ERR_INVALID_ARG;
     if (a->qkv_dtype != GDR_BF16 && a->qkv_dtype != GDR_F32) return GDR_ERR_INVALID_ARG;
-    if (!supported_width(a->d_k) || a->d_v != a->d_k) return GDR_ERR_UNSUPPORTED;
+    if (!supported_width(a->d_k) || !supported_width(a->d_v)) return GDR_ERR_UNSUPPORTED;
     if (!a->cu_seqlens || !aligned4(a->cu_seqlens)) return GDR_ERR_INVALID_ARG;
     if (a->total_tokens > 0) {
         const void* vec[] = {a->q, a->k, a->v};
@@ -41,8 +41,29 @@ gdr_status check_prefill_inputs(const gdr_prefill_args* a) {
     return GDR_OK;
 }
 
+// The address kernels use for `p`: a device (or managed) pointer as it is, a
+// page-locked host pointer as its mapped device address (the same value under
+// unified addressing).  Pageable host memory is rejected.
+gdr_status kernel_address(void* p, void** out) {
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return GDR_ERR_INVALID_ARG;
+    }
+    if (at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged) {
+        *out = p;
+        return GDR_OK;
+    }
+    if (at.type == cudaMemoryTypeHost && at.devicePointer) {
+        *out = at.devicePointer;
+        return aligned16(*out) ? GDR_OK : GDR_ERR_INVALID_ARG;
+    }
+    return GDR_ERR_INVALID_ARG;
+}
+
 gdr_status check_workspace(const gdr_prefill_args* a, WorkspaceLayout* lay) {
-    *lay = gdr::workspace_layout(a->n_seqs, a->n_heads, a->d_k, a->total_tokens, a->scalar_decay);
+    *lay = gdr::workspace_layout_dims(a->n_seqs, a->n_heads, a->d_k, a->d_v, a->total_tokens,
+                                      a->scalar_decay);
     if (!a->workspace || (reinterpret_cast<uintptr_t>(a->workspace) & 255u) != 0)
         return GDR_ERR_WORKSPACE;
     if (a->workspace_bytes < lay->total) return GDR_ERR_WORKSPACE;
@@ -70,8 +91,8 @@ int gdr_version(void) { return 100; }
 size_t gdr_prefill_workspace_size(int n_seqs, int n_heads, int d_k, int d_v,
                                   int64_t total_tokens, int scalar_decay) {
     if (n_seqs < 0 || n_heads <= 0 || total_tokens < 0) return 0;
-    if (!supported_width(d_k) || d_v != d_k) return 0;
-    return gdr::workspace_layout(n_seqs, n_heads, d_k, total_tokens, scalar_decay).total;
+    if (!supported_width(d_k) || !supported_width(d_v)) return 0;
+    return gdr::workspace_layout_dims(n_seqs, n_heads, d_k, d_v, total_tokens, scalar_decay).total;
 }
 
 int gdr_prefill_kernel_count(int n_seqs, int n_heads, int d_k, int d_v, int64_t total_tokens,
@@ -79,8 +100,11 @@ int gdr_prefill_kernel_count(int n_seqs, int n_heads, int d_k, int d_v, int64_t 
     if (gdr_prefill_workspace_size(n_seqs, n_heads, d_k, d_v, total_tokens, scalar_decay) == 0)
         return 0;
     if (n_seqs == 0) return 0;
+    const int D = d_k > d_v ? d_k : d_v;
     const int intra = total_tokens > 0 ? 1 : 0;
-    return intra + (gdr::segment_chunks(n_seqs, n_heads, total_tokens, d_k) > 0 ? 3 : 1);
+    // widening of the narrower side's inputs (d_k != d_v)
+    const int widen = (total_tokens > 0 && d_k != d_v) ? (d_k < d_v ? (scalar_decay ? 2 : 3) : 1) : 0;
+    return widen + intra + (gdr::segment_chunks(n_seqs, n_heads, total_tokens, D) > 0 ? 3 : 1);
 }
 
 int64_t gdr_snapshot_count(const int32_t* host_cu, int n_seqs, int snap_interval) {
@@ -95,6 +119,20 @@ int64_t gdr_snapshot_count(const int32_t* host_cu, int n_seqs, int snap_interval
     return total;
 }
 
+gdr_status gdr_snapshot_offsets(const int32_t* host_cu, int n_seqs, int snap_interval,
+                                int64_t* out) {
+    if (!host_cu || !out || n_seqs < 0 || snap_interval <= 0) return GDR_ERR_INVALID_ARG;
+    int64_t total = 0;
+    for (int n = 0; n < n_seqs; ++n) {
+        out[n] = total;
+        const int32_t len = host_cu[n + 1] - host_cu[n];
+        if (len < 0) return GDR_ERR_INVALID_ARG;
+        total += len / snap_interval;
+    }
+    out[n_seqs] = total;
+    return GDR_OK;
+}
+
 gdr_status gdr_prefill_stages(const gdr_prefill_args* a, int first, int last, void* stream) {
     if (first < 0 || last > 1 || first > last) return GDR_ERR_INVALID_ARG;
     gdr_status s = check_prefill_inputs(a);
@@ -104,21 +142,55 @@ gdr_status gdr_prefill_stages(const gdr_prefill_args* a, int first, int last, vo
     if (a->init_state && !aligned16(a->init_state)) return GDR_ERR_INVALID_ARG;
     if (a->snap_interval > 0 && (!a->snapshots || !aligned16(a->snapshots)))
         return GDR_ERR_INVALID_ARG;
+    if (a->snap_offsets && (reinterpret_cast<uintptr_t>(a->snap_offsets) & 7u) != 0)
+        return GDR_ERR_INVALID_ARG;
+    if (a->gate_raw) {
+        if (!aligned16(a->gate_raw) || !a->norm_weight || !aligned16(a->norm_weight))
+            return GDR_ERR_INVALID_ARG;
+        if (!(a->norm_eps >= 0.f) || a->norm_eps > 3.0e38f) return GDR_ERR_INVALID_ARG;
+    }
     WorkspaceLayout lay;
     s = check_workspace(a, &lay);
     if (s != GDR_OK) return s;
     if (a->n_seqs == 0) return GDR_OK;
+    gdr_prefill_args args = *a;
+    if (last >= 1 && a->snap_interval > 0) {
+        s = kernel_address(a->snapshots, reinterpret_cast<void**>(&args.snapshots));
+        if (s != GDR_OK) return s;
+    }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    uint8_t* ws = static_cast<uint8_t*>(a->workspace);
+    uint8_t* ws = static_cast<uint8_t*>(args.workspace);
     uint32_t* err = reinterpret_cast<uint32_t*>(ws + lay.err_off);
     uint8_t* rec = ws + lay.rec_off;
     if (first == 0 && cudaMemsetAsync(err, 0, sizeof(uint32_t), st) != cudaSuccess)
         return GDR_ERR_CUDA;
-    if (first == 0 && a->total_tokens > 0) {
-        s = from_cuda(gdr::launch_intra_chunk(*a, rec, err, st));
+    if (first == 0 && args.total_tokens > 0) {
+        // d_k != d_v: the intra-chunk kernel reads inputs widened to D = max
+        gdr_prefill_args sq = args;
+        if (a->d_k != a->d_v) {
+            const int D = a->d_k > a->d_v ? a->d_k : a->d_v;
+            const int elem = a->qkv_dtype == GDR_BF16 ? 2 : 4;
+            const int64_t rows = a->total_tokens * a->n_heads;
+            if (a->d_k < D) {
+                s = from_cuda(gdr::launch_widen(a->q, ws + lay.wq_off, rows, a->d_k, D, elem, st));
+                if (s == GDR_OK)
+                    s = from_cuda(gdr::launch_widen(a->k, ws + lay.wk_off, rows, a->d_k, D, elem, st));
+                if (s == GDR_OK && !a->scalar_decay)
+                    s = from_cuda(gdr::launch_widen(a->log_a, ws + lay.wg_off, rows, a->d_k, D, 4, st));
+                sq.q = ws + lay.wq_off;
+                sq.k = ws + lay.wk_off;
+                if (!a->scalar_decay) sq.log_a = reinterpret_cast<const float*>(ws + lay.wg_off);
+            } else {
+                s = from_cuda(gdr::launch_widen(a->v, ws + lay.wv_off, rows, a->d_v, D, elem, st));
+                sq.v = ws + lay.wv_off;
+            }
+            if (s != GDR_OK) return s;
+            sq.d_k = sq.d_v = D;
+        }
+        s = from_cuda(gdr::launch_intra_chunk(sq, rec, err, st));
         if (s != GDR_OK) return s;
     }
-    if (last >= 1) return from_cuda(gdr::launch_state_pass(*a, rec, lay, ws, err, st));
+    if (last >= 1) return from_cuda(gdr::launch_state_pass(args, rec, lay, ws, err, st));
     return GDR_OK;
 }
 
@@ -153,6 +225,7 @@ gdr_status gdr_chunk_factors(const gdr_prefill_args* a, float* Qt, float* PU, fl
                              float* NC, float* gamma, void* stream) {
     gdr_status s = check_prefill_inputs(a);
     if (s != GDR_OK) return s;
+    if (a->d_k != a->d_v) return GDR_ERR_UNSUPPORTED;
     WorkspaceLayout lay;
     s = check_workspace(a, &lay);
     if (s != GDR_OK) return s;
@@ -188,6 +261,30 @@ gdr_status gdr_decode_step(int batch, int n_heads, int d_k, int d_v, gdr_dtype q
     return from_cuda(gdr::launch_decode(batch, n_heads, d_k, d_v, qkv_dtype, q, k, v, beta, log_a,
                                         scalar_decay, scale, state, o,
                                         static_cast<cudaStream_t>(stream)));
+}
+
+gdr_status gdr_decode_step_gated(int batch, int n_heads, int d_k, int d_v, gdr_dtype qkv_dtype,
+                                 const void* q, const void* k, const void* v, const float* beta,
+                                 const float* log_a, int scalar_decay, float scale, float* state,
+                                 const void* gate_raw, const float* norm_weight, float norm_eps,
+                                 float* o, void* stream) {
+    if (batch < 0 || n_heads <= 0 || d_k <= 0 || d_v <= 0) return GDR_ERR_INVALID_ARG;
+    if (qkv_dtype != GDR_BF16 && qkv_dtype != GDR_F32) return GDR_ERR_INVALID_ARG;
+    if (!supported_width(d_k) || !supported_width(d_v)) return GDR_ERR_UNSUPPORTED;
+    if ((int64_t)batch * n_heads > (int64_t)INT32_MAX) return GDR_ERR_INVALID_ARG;
+    if (batch == 0) return GDR_OK;
+    const void* vec[] = {q, k, state, norm_weight};
+    for (const void* p : vec)
+        if (!p || !aligned16(p)) return GDR_ERR_INVALID_ARG;
+    if (!v || !aligned_elem(v, qkv_dtype) || !beta || !aligned4(beta) || !o || !aligned4(o))
+        return GDR_ERR_INVALID_ARG;
+    if (!gate_raw || !aligned_elem(gate_raw, qkv_dtype)) return GDR_ERR_INVALID_ARG;
+    if (!(norm_eps >= 0.f) || norm_eps > 3.0e38f) return GDR_ERR_INVALID_ARG;
+    if (!log_a || !(scalar_decay ? aligned4(log_a) : aligned16(log_a))) return GDR_ERR_INVALID_ARG;
+    return from_cuda(gdr::launch_decode_gated(batch, n_heads, d_k, d_v, qkv_dtype, q, k, v, beta,
+                                              log_a, scalar_decay, scale, state, gate_raw,
+                                              norm_weight, norm_eps, o,
+                                              static_cast<cudaStream_t>(stream)));
 }
 
 gdr_status gdr_preprocess(const gdr_preprocess_args* a, void* stream) {

@@ -116,6 +116,9 @@ struct WorkspaceLayout {
     int64_t n_seg_slots;
     int seg_chunks;
     size_t rec_bytes;
+    // d_k != d_v: the narrower side's inputs widened to D = max(d_k, d_v)
+    // (zero channels), each [T, H, D] with 4 bytes per element reserved
+    size_t wq_off, wk_off, wg_off, wv_off;   // 0 when not used
     size_t total;
 };
 
@@ -132,6 +135,27 @@ inline WorkspaceLayout workspace_layout(int n_seqs, int H, int D, int64_t T, int
     w.seg_chunks = segment_chunks(n_seqs, H, T, D);
     w.n_seg_slots = n_segment_slots(T, n_seqs, w.seg_chunks);
     w.total = w.seg_off + (size_t)w.n_seg_slots * (size_t)H * 3u * (size_t)D * D * sizeof(float);
+    w.wq_off = w.wk_off = w.wg_off = w.wv_off = 0;
+    return w;
+}
+
+// Workspace of a prefill with key width dk and value width dv: the square
+// layout for D = max(dk, dv), then (dk != dv) the widened inputs.
+inline WorkspaceLayout workspace_layout_dims(int n_seqs, int H, int dk, int dv, int64_t T,
+                                             int scalar) {
+    const int D = dk > dv ? dk : dv;
+    WorkspaceLayout w = workspace_layout(n_seqs, H, D, T, scalar);
+    if (dk == dv) return w;
+    const size_t arr = align_up((size_t)T * (size_t)H * (size_t)D * 4u, 1024);
+    size_t off = align_up(w.total, 1024);
+    if (dk < D) {
+        w.wq_off = off; off += arr;
+        w.wk_off = off; off += arr;
+        if (!scalar) { w.wg_off = off; off += arr; }
+    } else {
+        w.wv_off = off; off += arr;
+    }
+    w.total = off;
     return w;
 }
 
@@ -155,7 +179,18 @@ cudaError_t launch_decode(int B, int H, int dk, int dv, gdr_dtype dt, const void
                           const float* log_a, int scalar, float scale, float* state,
                           float* o, cudaStream_t st);
 
+cudaError_t launch_decode_gated(int B, int H, int dk, int dv, gdr_dtype dt, const void* q,
+                                const void* k, const void* v, const float* beta,
+                                const float* log_a, int scalar, float scale, float* state,
+                                const void* gate_raw, const float* norm_weight, float norm_eps,
+                                float* o, cudaStream_t st);
+
 cudaError_t launch_preprocess(const gdr_preprocess_args& a, cudaStream_t st);
+
+// Copy rows of width w of a [rows, w] array into [rows, D] with zeros past w
+// (elem = 2 or 4 bytes; w and D multiples of 64).
+cudaError_t launch_widen(const void* src, void* dst, int64_t rows, int w, int D, int elem,
+                         cudaStream_t st);
 
 cudaError_t launch_decode_draft(int B, int K, int H, int dk, int dv, gdr_dtype dt, const void* q,
                                 const void* k, const void* v, const float* beta,

@@ -410,9 +410,14 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
-    if (cur.idx >= 0 && warp == kLoadWarp)
+    // requests of inputs (load warp) and MMA commits (thread 0) so far: on a
+    // timed-out wait the last of each is drained before the CTA exits
+    uint32_t in_issued = 0, mma_commits = 0;
+    if (cur.idx >= 0 && warp == kLoadWarp) {
         issue_inputs<D, InT, SCALAR, L>(sm, &in_bar[0], &in_bar[1], maps, beta, log_a, H, cur, lane,
                                         keep_records != 0);
+        ++in_issued;
+    }
     const uint32_t tmem = tmem_slot;
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
     const int wgrp = warp >> 2;                               // warp group (0 .. NG - 1)
@@ -684,6 +689,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                 mma_bf16(tmem, sw128_desc(aXA, 128, 0, 16 * kk), sw128_desc(aXA, 128, 64, 16 * kk), id, kk > 0);
         }
         mma_commit(&mma_bar);
+        ++mma_commits;
     }
     failed = !mbar_wait(&mma_bar, phase);
     phase ^= 1u;
@@ -766,9 +772,11 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     if (warp == kLoadWarp) {
         const Item nxt = s_item[(iter + 1) & 1];
         fence_proxy_async_smem();             // this item's reads of region 1 come first
-        if (nxt.idx >= 0)
+        if (nxt.idx >= 0) {
             issue_inputs<D, InT, SCALAR, L>(sm, &in_bar[0], &in_bar[1], maps, beta, log_a, H, nxt, lane,
                                             keep_records != 0);
+            ++in_issued;
+        }
         if (lane == 0)
             s_item[iter & 1] = nxt.idx >= 0 ? find_item(cu, n_seqs, H, n_items, nxt.idx + gridDim.x) : nxt;
     }
@@ -878,6 +886,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                 mma_bf16(tmem + 64 * half, sw128_desc(aB, 2 * D, 128 * half, 16 * kk),
                          sw128_desc(aT, 64, 0, 16 * kk), id, kk > 0);
         mma_commit(&mma_bar);
+        ++mma_commits;
     }
     if (!failed && !mbar_wait(&mma_bar, phase)) failed = true;
     phase ^= 1u;
@@ -925,6 +934,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
             mma_bf16(tmem + 3 * D, sw128_desc(aWU, 2 * D, D, 16 * kk), sw128_desc(aKd, D, 0, 16 * kk), id_dd, kk > 0);
         }
         mma_commit(&mma_bar);
+        ++mma_commits;
     }
     if (!failed && !mbar_wait(&mma_bar, phase)) failed = true;
     phase ^= 1u;
@@ -1012,6 +1022,17 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     }
 
     pdl_launch_dependents();
+    if (failed) {
+        // a wait gave up: nothing this CTA started may still be running when it
+        // releases its tensor memory and exits -- the last committed MMA and
+        // the last requested inputs (at most one of each is outstanding; these
+        // waits are bounded too)
+        if (tid == 0 && mma_commits > 0) (void)mbar_wait(&mma_bar, (mma_commits - 1u) & 1u);
+        if (warp == kLoadWarp && lane == 0 && in_issued > 0) {
+            if (!SCALAR) (void)mbar_wait(&in_bar[0], (in_issued - 1u) & 1u);
+            if (L::kStageQKV) (void)mbar_wait(&in_bar[1], (in_issued - 1u) & 1u);
+        }
+    }
     cp_async_wait_all();
     if (tid == 0) bulk_wait_group0();
     tc_fence_before_sync();

@@ -54,6 +54,44 @@ template <> struct Out8<__nv_bfloat16> {
     }
 };
 
+// Barrier of warps w and w + 4 (w = sub in 0..3) on named barrier 1 + w.
+template <int ID>
+__device__ __forceinline__ void pair_bar_id() {
+    asm volatile("bar.sync %0, 64;" ::"n"(ID) : "memory");
+}
+__device__ __forceinline__ void pair_bar(int sub) {
+    if (sub == 0) pair_bar_id<1>();
+    else if (sub == 1) pair_bar_id<2>();
+    else if (sub == 2) pair_bar_id<3>();
+    else pair_bar_id<4>();
+}
+
+template <typename T> struct In8;
+template <> struct In8<float> {
+    static __device__ __forceinline__ void load(const float* p, float (&x)[8]) {
+        const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+        const float4 b = __ldg(reinterpret_cast<const float4*>(p + 4));
+        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+    }
+};
+template <> struct In8<__nv_bfloat16> {
+    static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&x)[8]) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+        const float2 a = unpack_bf16(u.x), b = unpack_bf16(u.y), c = unpack_bf16(u.z), d = unpack_bf16(u.w);
+        x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y; x[4] = c.x; x[5] = c.y; x[6] = d.x; x[7] = d.y;
+    }
+};
+
+// Output epilogue of the mixer ("kda-graft", section "Идея и архитектура":
+// every KDA layer of the graft ends in an RMSNorm and an output gate):
+//     y = o / sqrt(mean_c o_c^2 + eps) * w * sigmoid(gate_raw)
+// over the d_v channels of each (token, head), w [d_v] shared by the heads.
+struct OutputGate {
+    const void* gate;        // [T, H, d_v], the outputs' dtype; NULL: no epilogue
+    const float* weight;     // [d_v]
+    float eps;
+};
+
 template <int D, int MODE>
 struct PassLayout {
     static constexpr RecordLayout R = record_layout(D);
@@ -80,8 +118,9 @@ __global__ void __launch_bounds__(kThreads, (D == 64) ? 2 : 1)
 state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                   const uint8_t* __restrict__ records, const float* init_state,
                   OutT* __restrict__ o, float* final_state, int snap_interval,
-                  float* __restrict__ snapshots, int seg_chunks, float* seg_ws,
-                  uint32_t* err, int keep_records) {
+                  float* __restrict__ snapshots, const int64_t* __restrict__ snap_offsets,
+                  int seg_chunks, float* seg_ws, uint32_t* err, int keep_records,
+                  const __grid_constant__ OutputGate og, int dk, int dv) {
     using L = PassLayout<D, MODE>;
     constexpr RecordLayout R = record_layout(D);
     constexpr int ST = L::kStages;
@@ -96,8 +135,15 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     uint8_t* sm = align_smem<1024>(smem_raw);
     __shared__ uint64_t full[ST];
     __shared__ uint64_t mma_bar;
+#ifdef GDR_TEST_WAIT_LIMIT_NS
+    // test builds only: a barrier nothing arrives on, waited for with a short
+    // limit at the second chunk, so that the timeout path runs on demand
+    __shared__ uint64_t never_bar;
+#endif
     __shared__ uint32_t tmem_slot;
     __shared__ int64_t snap_base_s;
+    // epilogue: partial sums of squares of the output rows, [chunk parity][half][row]
+    __shared__ float ssq_s[L::kOut ? 2 * 2 * 64 : 1];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int sub = warp & 3, half = warp >> 2;
@@ -164,6 +210,9 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
 #pragma unroll
         for (int s = 0; s < ST; ++s) mbar_init(&full[s], 1);
         mbar_init(&mma_bar, 1);
+#ifdef GDR_TEST_WAIT_LIMIT_NS
+        mbar_init(&never_bar, 1);
+#endif
         fence_mbar_init();
         // the first records start arriving while the initial state is loaded
         for (int c = 0; c < ST && c < nchunks; ++c) issue_copy(c);
@@ -171,33 +220,43 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     }
     if (warp == 0) {
         tmem_alloc(&tmem_slot, kTmemCols);
+        // first snapshot slot of sequence n: the caller's offsets, or the sum
+        // of the earlier sequences' snapshot counts
         int64_t acc = 0;
-        if (kOut && snap_interval > 0)
+        if (kOut && snap_interval > 0 && !snap_offsets)
             for (int m = lane; m < n; m += 32) acc += (__ldg(cu + m + 1) - __ldg(cu + m)) / snap_interval;
 #pragma unroll
         for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (kOut && snap_interval > 0 && snap_offsets) acc = __ldg(snap_offsets + n);
         if (lane == 0) snap_base_s = acc;
     }
 
     // ---- initial state --------------------------------------------------------
-    // S[t][j]: tile t (0 = S, 1 = X for kLocal with two products), column cb + j
+    // S[t][j]: tile t (0 = S, 1 = X for kLocal with two products), column cb + j.
+    // The caller's states are d_v x d_k; with d_k != d_v the kernel works on
+    // D x D (D = max) and the extra rows / columns stay zero.
     float S[kNT][CW];
-    const size_t state_off = ((size_t)n * H + h) * D * D;
+    const size_t state_off = ((size_t)n * H + h) * dv * dk;     // caller's layout
     const float* src = nullptr;
-    size_t src_off = state_off;
+    bool src_user = true;                                         // caller's layout or E
     if (MODE == kFull) src = init_state;
     if (MODE == kApply) {
         if (s0 == seg_start) src = init_state;
-        else { src = seg_base + 2u * D * D; src_off = 0; }       // E: this segment's start state
+        else { src = seg_base + 2u * D * D; src_user = false; }  // E: this segment's start state
     }
+    const bool row_in = srow < dv;                                // a row of the caller's state
 #pragma unroll
     for (int t = 0; t < kNT; ++t) {
         const bool x_tile = (MODE == kLocal) && (t == 1 || is_x);
 #pragma unroll
         for (int j = 0; j < CW; j += 4) {
             float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (MODE != kLocal && active && src)
-                x = *reinterpret_cast<const float4*>(src + src_off + (size_t)srow * D + cb + j);
+            if (MODE != kLocal && active && src) {
+                if (!src_user)
+                    x = *reinterpret_cast<const float4*>(src + (size_t)srow * D + cb + j);
+                else if (row_in && cb + j < dk)
+                    x = *reinterpret_cast<const float4*>(src + state_off + (size_t)srow * dk + cb + j);
+            }
             if (x_tile) {
                 const int c = cb + j;
                 x = make_float4(c + 0 == srow ? 1.f : 0.f, c + 1 == srow ? 1.f : 0.f,
@@ -269,6 +328,9 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         const int t0 = s0 + k * kChunk;
         const int len = min(kChunk, s1 - t0);
         if (!mbar_wait(&full[st], (uint32_t)(k / ST) & 1)) failed = true;
+#ifdef GDR_TEST_WAIT_LIMIT_NS
+        if (k == 1 && !mbar_wait_for(&never_bar, 0u, (uint64_t)GDR_TEST_WAIT_LIMIT_NS)) failed = true;
+#endif
         const float* gam = reinterpret_cast<const float*>(stage(st) + L::kGamma);
         const uint8_t* nc = stage(st) + R.NC;
         // gamma and this row's NC, read while the MMAs of chunk k finish
@@ -377,13 +439,51 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
             const int kabs = chunk0 + k;
             if (snap_interval > 0 && len == kChunk && ((kabs + 1) * kChunk) % snap_interval == 0 && active) {
                 const int64_t slot = snap_base + ((int64_t)(kabs + 1) * kChunk) / snap_interval - 1;
-                float* dst = snapshots + ((size_t)slot * H + h) * D * D + (size_t)srow * D + cb;
+                float* dst = snapshots + ((size_t)slot * H + h) * dv * dk + (size_t)srow * dk + cb;
 #pragma unroll
                 for (int j = 0; j < CW; j += 4)
-                    *reinterpret_cast<float4*>(dst + j) = make_float4(S[0][j], S[0][j + 1], S[0][j + 2], S[0][j + 3]);
+                    if (row_in && cb + j < dk)
+                        *reinterpret_cast<float4*>(dst + j) = make_float4(S[0][j], S[0][j + 1], S[0][j + 2], S[0][j + 3]);
             }
             const uint8_t* pu = stage(st) + R.PU;
-            OutT* orow_ptr = o + ((size_t)(t0 + orow) * H + h) * D + cb;
+            OutT* orow_ptr = o + ((size_t)(t0 + orow) * H + h) * dv + cb;
+            if (og.gate) {
+                // o = Qt S0^T + PU in place, then the row's RMS: the two halves
+                // of a row (warps w and w + 4, same lane) swap their partial sums
+                // of squares through shared memory behind a barrier of the pair
+                float ss = 0.f;
+#pragma unroll
+                for (int j = 0; j < CW; j += 8) {
+                    const uint4 u = *reinterpret_cast<const uint4*>(pu + sw128_chunk(64, orow & 63, (cb + j) / 8));
+                    const float2 p0 = unpack_bf16(u.x), p1 = unpack_bf16(u.y);
+                    const float2 p2 = unpack_bf16(u.z), p3 = unpack_bf16(u.w);
+                    ov[j + 0] += p0.x; ov[j + 1] += p0.y; ov[j + 2] += p1.x; ov[j + 3] += p1.y;
+                    ov[j + 4] += p2.x; ov[j + 5] += p2.y; ov[j + 6] += p3.x; ov[j + 7] += p3.y;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) ss = fmaf(ov[j + e], ov[j + e], ss);
+                }
+                float* ssq = ssq_s + (k & 1) * 128;
+                if (oactive) ssq[half * 64 + orow] = ss;
+                pair_bar(sub);
+                const float tot = ss + (oactive ? ssq[(half ^ 1) * 64 + orow] : 0.f);
+                const float rstd = rsqrtf(tot / (float)dv + og.eps);
+                if (oactive && orow < len) {
+                    const OutT* g = static_cast<const OutT*>(og.gate) + ((size_t)(t0 + orow) * H + h) * dv + cb;
+#pragma unroll
+                    for (int j = 0; j < CW; j += 8) {
+                        if (cb + j >= dv) continue;
+                        float gv[8], wv[8], x[8];
+                        In8<OutT>::load(g + j, gv);
+                        In8<float>::load(og.weight + cb + j, wv);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const float sig = 1.f / (1.f + __expf(-gv[e]));
+                            x[e] = ov[j + e] * rstd * wv[e] * sig;
+                        }
+                        Out8<OutT>::store(orow_ptr + j, x);
+                    }
+                }
+            } else {
 #pragma unroll
             for (int p = 0; p < CW / 16; ++p) {
                 const float* y = ov + 16 * p;
@@ -392,7 +492,7 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                               *reinterpret_cast<float(*)[16]>(ov + 16 * p));
                     tmem_ld_wait();
                 }
-                if (oactive && orow < len) {
+                if (oactive && orow < len && cb + 16 * p < dv) {
 #pragma unroll
                     for (int jj = 0; jj < 2; ++jj) {
                         const int j = 16 * p + 8 * jj;
@@ -406,6 +506,7 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                         Out8<OutT>::store(orow_ptr + j, x);
                     }
                 }
+            }
             }
         }
         // With two stages this chunk's stage is refilled now, once every
@@ -427,17 +528,18 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     if (failed) {
         if (tid == 0) atomicOr(err, 1u);
     } else if (active) {
-        auto store_row = [&](float* dst, int t) {
+        auto store_row = [&](float* dst, int t, int ncols) {
 #pragma unroll
             for (int j = 0; j < CW; j += 4)
-                *reinterpret_cast<float4*>(dst + j) = make_float4(S[t][j], S[t][j + 1], S[t][j + 2], S[t][j + 3]);
+                if (cb + j < ncols)
+                    *reinterpret_cast<float4*>(dst + j) = make_float4(S[t][j], S[t][j + 1], S[t][j + 2], S[t][j + 3]);
         };
-        if (MODE == kFull || (MODE == kApply && s1 == __ldg(cu + n + 1)))
-            store_row(final_state + state_off + (size_t)srow * D + cb, 0);
+        if ((MODE == kFull || (MODE == kApply && s1 == __ldg(cu + n + 1))) && row_in)
+            store_row(final_state + state_off + (size_t)srow * dk + cb, 0, dk);
         if (MODE == kLocal) {
             // N (rows of S) then M (rows of X) of this segment's affine map
-            store_row(seg_base + (is_x ? (size_t)D * D : 0) + (size_t)srow * D + cb, 0);
-            if (kNT == 2) store_row(seg_base + (size_t)D * D + (size_t)srow * D + cb, kNT - 1);
+            store_row(seg_base + (is_x ? (size_t)D * D : 0) + (size_t)srow * D + cb, 0, D);
+            if (kNT == 2) store_row(seg_base + (size_t)D * D + (size_t)srow * D + cb, kNT - 1, D);
         }
     }
     // error path: no copy or MMA of this CTA may still be in flight when it
@@ -489,7 +591,7 @@ struct CombineLayout {
 template <int D>
 __global__ void __launch_bounds__(kCombineThreads)
 combine_kernel(const int32_t* __restrict__ cu, int H, int seg_chunks, const float* init_state,
-               float* final_state, float* seg_ws, uint32_t* err) {
+               float* final_state, float* seg_ws, uint32_t* err, int dk, int dv) {
     using L = CombineLayout<D>;
     constexpr int RB = kCombineRows;
     constexpr int NT = kCombineThreads;
@@ -506,13 +608,15 @@ combine_kernel(const int32_t* __restrict__ cu, int H, int seg_chunks, const floa
     const int s0 = __ldg(cu + n), s1 = __ldg(cu + n + 1);
     const int span = kChunk * seg_chunks;
     const int nseg = (s1 - s0 + span - 1) / span;
-    const size_t state_off = ((size_t)n * H + h) * D * D;
-    const size_t row_off = (size_t)(rb * RB + j) * D + c0;              // this lane's row, slab start
+    // the caller's states are d_v x d_k; the maps and E are D x D (D = max)
+    const size_t state_off = ((size_t)n * H + h) * dv * dk;
+    const size_t row_off = (size_t)(rb * RB + j) * dk + c0;             // this lane's row, slab start
     (void)err;
     if (nseg == 0) {
-        if (kq == 0) {
+        if (kq == 0 && rb * RB + j < dv) {
 #pragma unroll
             for (int c = 0; c < CW; c += 4) {
+                if (c0 + c >= dk) continue;
                 float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (init_state) x = *reinterpret_cast<const float4*>(init_state + state_off + row_off + c);
                 *reinterpret_cast<float4*>(final_state + state_off + row_off + c) = x;
@@ -538,7 +642,8 @@ combine_kernel(const int32_t* __restrict__ cu, int H, int seg_chunks, const floa
     };
     for (int c = tid; c < RB * D; c += NT) {
         const int r = c / D, col = c % D;
-        e[r * L::kLdE + col] = init_state ? init_state[state_off + (size_t)(rb * RB + r) * D + col] : 0.f;
+        const bool in = init_state && rb * RB + r < dv && col < dk;
+        e[r * L::kLdE + col] = in ? init_state[state_off + (size_t)(rb * RB + r) * dk + col] : 0.f;
     }
     // steps 0 .. NB-2 in flight (one commit group per step, empty past the end)
 #pragma unroll
@@ -628,8 +733,9 @@ cudaError_t launch_mode(const gdr_prefill_args& a, const uint8_t* records,
     // slower with it
     return launch_pdl(MODE == kFull, kern, grid, dim3(kThreads), smem, st, a.cu_seqlens, a.n_seqs, a.n_heads,
                       records, a.init_state, static_cast<OutT*>(a.o), a.final_state,
-                      a.snap_interval, a.snapshots, lay.seg_chunks, seg_ws, err,
-                      records_fit_l2(lay.n_slots, a.n_heads, D) ? 1 : 0);
+                      a.snap_interval, a.snapshots, a.snap_offsets, lay.seg_chunks, seg_ws, err,
+                      records_fit_l2(lay.n_slots, a.n_heads, D) ? 1 : 0,
+                      OutputGate{a.gate_raw, a.norm_weight, a.norm_eps}, a.d_k, a.d_v);
 }
 
 template <int D, typename OutT>
@@ -645,7 +751,8 @@ cudaError_t launch_typed(const gdr_prefill_args& a, const uint8_t* records,
     if (e != cudaSuccess) return e;
     e = launch_pdl(false, ck, dim3((unsigned)a.n_seqs * (unsigned)a.n_heads, D / kCombineRows),
                    dim3(kCombineThreads), CombineLayout<D>::dyn_bytes, st, a.cu_seqlens,
-                   a.n_heads, lay.seg_chunks, a.init_state, a.final_state, seg_ws, err);
+                   a.n_heads, lay.seg_chunks, a.init_state, a.final_state, seg_ws, err, a.d_k,
+                   a.d_v);
     if (e != cudaSuccess) return e;
     return launch_mode<D, OutT, kApply>(a, records, lay, seg_ws, err, st);
 }
@@ -656,7 +763,7 @@ cudaError_t launch_state_pass(const gdr_prefill_args& a, const uint8_t* records,
                               const WorkspaceLayout& lay, uint8_t* ws, uint32_t* err,
                               cudaStream_t st) {
     if ((int64_t)a.n_seqs * a.n_heads == 0) return cudaSuccess;
-    if (a.d_k == 64)
+    if (a.d_k == 64 && a.d_v == 64)       // else D = 128 (d_k, d_v in {64, 128})
         return a.qkv_dtype == GDR_BF16 ? launch_typed<64, __nv_bfloat16>(a, records, lay, ws, err, st)
                                        : launch_typed<64, float>(a, records, lay, ws, err, st);
     return a.qkv_dtype == GDR_BF16 ? launch_typed<128, __nv_bfloat16>(a, records, lay, ws, err, st)

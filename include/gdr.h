@@ -85,7 +85,14 @@ typedef struct {
     int n_seqs;                 /* N >= 0 sequences packed by cu_seqlens */
     int n_heads;                /* H >= 1 */
     int d_k;                    /* key/query width: 64 or 128 */
-    int d_v;                    /* value width: must equal d_k in this build */
+    int d_v;                    /* value width: 64 or 128, any pairing with d_k.  With
+                                   d_k != d_v the kernels run at D = max(d_k, d_v) on
+                                   inputs whose narrower side is copied, widened with
+                                   zero channels, into the workspace (exact: zero key
+                                   channels leave the other columns of S untouched and
+                                   stay zero; rows of S evolve independently, and a
+                                   zero value row stays zero); states and o keep the
+                                   caller's d_v x d_k and d_v layouts. */
     int64_t total_tokens;       /* T_tot = cu_seqlens[N]; host copy of the device value */
     const int32_t* cu_seqlens;  /* device [N+1]: 0 = cu[0] <= cu[1] <= ... <= cu[N] = T_tot */
     gdr_dtype qkv_dtype;        /* dtype of q, k, v and o */
@@ -107,7 +114,20 @@ typedef struct {
                                    sequence, m = 1 .. floor(L_n / snap_interval),
                                    sequences in order ("Co stan rekurencyjny zmienia przy
                                    serwowaniu", point 1: a prefix is reused from the
-                                   snapshot taken at its end). */
+                                   snapshot taken at its end).  May be pinned host
+                                   memory (see "Snapshot offload" below). */
+    const int64_t* snap_offsets;/* device [N+1] or NULL: first snapshot slot of each
+                                   sequence, as gdr_snapshot_offsets returns it
+                                   (NULL: the kernels sum the sequence lengths) */
+    const void* gate_raw;       /* device [T_tot, H, d_v], dtype qkv_dtype, or NULL.  When
+                                   given, o receives the mixer's output after its RMSNorm
+                                   and output gate ("kda-graft", section "Идея и
+                                   архитектура": each KDA layer ends in both), per token
+                                   and head over the d_v channels:
+                                     o = x / sqrt(mean_c x_c^2 + norm_eps) * norm_weight
+                                           * sigmoid(gate_raw),   x = S_t (scale q_t) */
+    const float* norm_weight;   /* device [d_v] fp32, shared by the heads (with gate_raw) */
+    float norm_eps;             /* RMSNorm epsilon >= 0 (with gate_raw), e.g. 1e-6f */
     void* workspace;            /* device scratch, >= gdr_prefill_workspace_size(...) bytes,
                                    256-byte aligned; contents on entry do not matter */
     size_t workspace_bytes;
@@ -121,13 +141,47 @@ size_t gdr_prefill_workspace_size(int n_seqs, int n_heads, int d_k, int d_v,
  * Number of kernel launches gdr_prefill enqueues for these sizes (0 on bad
  * sizes): the intra-chunk kernel plus one state pass, or three (zero-state
  * pass, chaining of segment maps, replay) when long sequences with few
- * (sequence, head) pairs are cut into segments.
+ * (sequence, head) pairs are cut into segments; with d_k != d_v, plus one
+ * widening copy per widened input (q, k and a per-channel log_a, or v).
  */
 int gdr_prefill_kernel_count(int n_seqs, int n_heads, int d_k, int d_v, int64_t total_tokens,
                              int scalar_decay);
 
 /* Number of snapshot slots for host-side cu_seqlens [N+1] (-1 on bad input). */
 int64_t gdr_snapshot_count(const int32_t* host_cu_seqlens, int n_seqs, int snap_interval);
+
+/*
+ * Where each sequence's snapshots start ("Co stan rekurencyjny zmienia przy
+ * serwowaniu", point 1: a request whose prompt extends a stored prefix resumes
+ * from the snapshot at the prefix's end, so a caller must find sequence n's
+ * m-th snapshot).  host_cu_seqlens [N+1] and host_offsets_out [N+1] are host
+ * memory.  On return host_offsets_out[n] = sum over sequences m < n of
+ * floor(L_m / snap_interval); sequence n's m-th snapshot (m = 1 .. floor(L_n /
+ * snap_interval), the state after its first m * snap_interval tokens) is slot
+ * host_offsets_out[n] + m - 1 of gdr_prefill_args.snapshots, and
+ * host_offsets_out[N] is the slot count.  A copy of the array on the device
+ * may be passed as gdr_prefill_args.snap_offsets.  Errors: GDR_ERR_INVALID_ARG
+ * for a null pointer, n_seqs < 0, snap_interval <= 0 or a decreasing
+ * cu_seqlens (host_offsets_out is then left unspecified).
+ */
+gdr_status gdr_snapshot_offsets(const int32_t* host_cu_seqlens, int n_seqs, int snap_interval,
+                                int64_t* host_offsets_out);
+
+/*
+ * Snapshot offload.  A serving engine keeps prefix snapshots in host memory
+ * ("Co stan rekurencyjny zmienia przy serwowaniu", point 1: dozens of
+ * checkpoints of ~149 MiB each; saving them was made asynchronous so that it
+ * stops stalling prefill).  gdr_prefill_args.snapshots may therefore point to
+ * page-locked host memory (cudaHostAlloc / cudaMallocHost, or cudaHostRegister
+ * with cudaHostRegisterMapped): the state-pass kernel then writes every
+ * snapshot straight into host memory over the host link while it runs, as
+ * soon as that snapshot's state is known.  No device staging buffer, copy
+ * engine transfer, extra stream or host synchronisation is involved, and the
+ * prefill never waits for a copy; the snapshots are complete in host memory
+ * when the prefill's last kernel has completed (an event recorded after
+ * gdr_prefill on the same stream marks that).  Pageable host memory is
+ * rejected with GDR_ERR_INVALID_ARG.
+ */
 
 /*
  * Enqueue a prefill.  Outputs: o, final_state and (if snap_interval > 0)
@@ -166,11 +220,34 @@ gdr_status gdr_prefill_stages(const gdr_prefill_args* args, int first, int last,
  * array's device address (cudaGetSymbolAddress) with that device current;
  * make that first call before any stream capture.  All calls share the one
  * array: calls that may overlap on the GPU (other streams, other host threads)
- * race and must be serialised by the caller.  gdr_prefill_status needs a
- * workspace pointer and does not apply to this path.
+ * race and must be serialised by the caller.  Use gdr_prefill_static_status
+ * (not gdr_prefill_status) to learn whether the call's kernels completed.
+ *
+ * Size limit: gdr_prefill_workspace_size(...) <= GDR_STATIC_WORKSPACE_BYTES,
+ * where the workspace is 1 KiB + (floor(T/64) + N) * H * R(d) bytes of chunk
+ * records, R(64) = 33 792 and R(128) = 99 328, plus, when long sequences with
+ * few (sequence, head) pairs are cut into segments, 12 d^2 bytes per segment
+ * slot and head.  For one sequence that is up to 7 424 tokens at 14 heads and
+ * d 64 (the 8 192-token Qwen2.5-0.5B graft layer does not fit), 60 480 tokens
+ * at 2 heads and d 64, and 1 984 tokens at 16 heads and d 128.
+ *
+ * The device address of the array is looked up again (cudaGetSymbolAddress)
+ * on every call made while `stream` is not capturing, so a context re-created
+ * after cudaDeviceReset is handled; while capturing, the address from the last
+ * call on that device outside capture is used.
  */
 #define GDR_STATIC_WORKSPACE_BYTES (64u << 20)
 gdr_status gdr_prefill_static_workspace(const gdr_prefill_args* args, void* stream);
+
+/*
+ * Status the device side of the most recent gdr_prefill_static_workspace call
+ * on the current device recorded: GDR_OK, or GDR_ERR_TIMEOUT if one of its
+ * kernels abandoned a bounded wait (the outputs of that call are then
+ * undefined).  Reads one word of the library's array (no allocation) and
+ * synchronises `stream`, so it cannot be called while `stream` is capturing;
+ * GDR_ERR_CUDA if the read fails.
+ */
+gdr_status gdr_prefill_static_status(void* stream);
 
 /*
  * Status the device side of the most recent gdr_prefill on this workspace
@@ -209,6 +286,7 @@ gdr_status gdr_cumdecay(int n_seqs, int n_heads, int d_k, int64_t total_tokens,
  * Rows past the end of a partial chunk are zero.  `workspace` as for
  * gdr_prefill with the same arguments; q, k, v, beta, log_a, cu_seqlens,
  * scalar_decay and scale are read from `args`, its outputs are ignored.
+ * d_k must equal d_v here (GDR_ERR_UNSUPPORTED otherwise).
  */
 gdr_status gdr_chunk_factors(const gdr_prefill_args* args, float* Qt, float* PU, float* BS,
                              float* NC, float* gamma, void* stream);
@@ -229,6 +307,22 @@ gdr_status gdr_decode_step(int batch, int n_heads, int d_k, int d_v, gdr_dtype q
                            const void* q, const void* k, const void* v, const float* beta,
                            const float* log_a, int scalar_decay, float scale, float* state,
                            float* o, void* stream);
+
+/*
+ * gdr_decode_step followed by the output epilogue of gdr_prefill_args.gate_raw
+ * (RMSNorm over the d_v channels of each (sequence, head), weight shared by
+ * the heads, then the sigmoid output gate):
+ *   gate_raw     device [B, H, d_v], dtype qkv_dtype
+ *   norm_weight  device [d_v] fp32
+ *   norm_eps     >= 0
+ *   o            device [B, H, d_v] fp32 (output): the gated, normalised output
+ * Other arguments, results and errors as for gdr_decode_step.
+ */
+gdr_status gdr_decode_step_gated(int batch, int n_heads, int d_k, int d_v, gdr_dtype qkv_dtype,
+                                 const void* q, const void* k, const void* v, const float* beta,
+                                 const float* log_a, int scalar_decay, float scale, float* state,
+                                 const void* gate_raw, const float* norm_weight, float norm_eps,
+                                 float* o, void* stream);
 
 /* ------------------------------------------------------------------------
  * Input activations: the recurrence's q, k, v, beta and log a from raw

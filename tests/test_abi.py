@@ -134,7 +134,8 @@ def test_prefill_rejects_bad_arguments(L):
     pre = lambda a: L.gdr_prefill(ctypes.byref(a), None)
     assert pre(_args(n_heads=0)) == 1
     assert pre(_args(d_k=96, d_v=96)) == 2
-    assert pre(_args(d_v=128)) == 2
+    assert pre(_args(d_v=96)) == 2
+    assert pre(_args(d_k=128, d_v=32)) == 2
     assert pre(_args(q=None)) == 1
     assert pre(_args(k=0x30004)) == 1
     assert pre(_args(snap_interval=100, snapshots=0x90000)) == 1
@@ -153,6 +154,14 @@ def test_workspace_size_grows_with_tokens(L):
     assert 0 < s1 < s2
     assert gdr.workspace_size(1, 14, 96, 96, 8192) == 0
     assert gdr.workspace_size(1, 14, 128, 128, 8192, True) <= gdr.workspace_size(1, 14, 128, 128, 8192, False)
+    # d_k != d_v: the square layout at D = 128 plus the widened inputs
+    sq = gdr.workspace_size(1, 14, 128, 128, 8192)
+    assert gdr.workspace_size(1, 14, 64, 128, 8192) == sq + 3 * 8192 * 14 * 128 * 4
+    assert gdr.workspace_size(1, 14, 64, 128, 8192, True) == \
+        gdr.workspace_size(1, 14, 128, 128, 8192, True) + 2 * 8192 * 14 * 128 * 4
+    assert gdr.workspace_size(1, 14, 128, 64, 8192) == sq + 8192 * 14 * 128 * 4
+    assert gdr.kernel_count(32, 32, 64, 128, 278000) == 2 + 3
+    assert gdr.kernel_count(32, 32, 128, 64, 278000) == 2 + 1
 
 
 def test_snapshot_count_matches_oracle(L):
@@ -195,3 +204,43 @@ def test_header_is_plain_c():
             pytest.skip(f"{cc} not available")
         subprocess.run([cc, std, "-Wall", "-Wextra", "-Werror", "-fsyntax-only", "-x", lang, hdr],
                        check=True)
+
+
+def _enumerate_offsets(lengths, iv):
+    """Host enumeration: walk every sequence's snapshot positions in order."""
+    offsets, slot = [], 0
+    for L in lengths:
+        offsets.append(slot)
+        for end in range(iv, L + 1, iv):
+            slot += 1
+    return offsets + [slot]
+
+
+def test_snapshot_offsets_match_enumeration(L):
+    for lengths, iv in (([4096, 100, 8192, 0, 4095], 4096), ([64, 128, 1, 0, 640], 64),
+                        ([0], 128), ([], 64), ([300, 257, 1024], 128)):
+        cu = torch.tensor([0] + [int(x) for x in torch.tensor(lengths, dtype=torch.int64).cumsum(0)],
+                          dtype=torch.int32)
+        got = gdr.snapshot_offsets(cu, iv)
+        assert got.tolist() == _enumerate_offsets(lengths, iv)
+        assert int(got[-1]) == gdr.snapshot_count(cu, iv)
+
+
+def test_snapshot_offsets_reject_bad_arguments(L):
+    cu = torch.tensor([0, 64, 32], dtype=torch.int32)             # decreasing
+    out = torch.empty(3, dtype=torch.int64)
+    call = lambda c, n, iv, o: L.gdr_snapshot_offsets(c, n, iv, o)
+    p_cu, p_out = ctypes.c_void_p(cu.data_ptr()), ctypes.c_void_p(out.data_ptr())
+    assert call(p_cu, 2, 64, p_out) == 1
+    ok = torch.tensor([0, 64, 128], dtype=torch.int32)
+    p_ok = ctypes.c_void_p(ok.data_ptr())
+    assert call(p_ok, 2, 0, p_out) == 1
+    assert call(p_ok, -1, 64, p_out) == 1
+    assert call(None, 2, 64, p_out) == 1
+    assert call(p_ok, 2, 64, None) == 1
+    assert call(p_ok, 2, 64, p_out) == 0 and out.tolist() == [0, 1, 2]
+
+
+def test_prefill_rejects_misaligned_snapshot_offsets(L):
+    pre = lambda a: L.gdr_prefill(ctypes.byref(a), None)
+    assert pre(_args(snap_interval=128, snapshots=0x90000, snap_offsets=0xA0004)) == 1

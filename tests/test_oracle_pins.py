@@ -418,3 +418,34 @@ def test_every_planted_mistake_is_caught(mutant):
         except AssertionError:
             caught.append(pin.__name__)
     assert caught, f"mutant {mutant} passed every pin"
+
+
+def test_zero_channel_widening_is_exact():
+    """Widening the key side (q = k = 0, log a = 0) or the value side (v = 0)
+    with zero channels changes nothing in the original channels and leaves the
+    extra state rows / columns at zero -- the property that lets a d_k != d_v
+    prefill run on square D x D states, D = max(d_k, d_v)."""
+    import workloads as wl
+
+    def widen(x, D):
+        y = torch.zeros(*x.shape[:-1], D, dtype=x.dtype)
+        y[..., :x.shape[-1]] = x
+        return y
+
+    for dk, dv in ((64, 128), (128, 64)):
+        w = wl.shrink(wl.VARLEN, n_heads=2, d_k=dk, d_v=dv, lengths=(70, 5, 64), init_std=0.1,
+                      snap_interval=64)
+        x = wl.make_prefill_inputs(w)
+        ref = oracle.prefill(x["q"], x["k"], x["v"], x["beta"], x["log_a"], x["cu_seqlens"],
+                             init_state=x["init_state"], snap_interval=64)
+        D = max(dk, dv)
+        init = torch.zeros(3, 2, D, D)
+        init[:, :, :dv, :dk] = x["init_state"]
+        wide = oracle.prefill(widen(x["q"], D), widen(x["k"], D), widen(x["v"], D), x["beta"],
+                              widen(x["log_a"], D), x["cu_seqlens"], init_state=init,
+                              snap_interval=64)
+        assert np.array_equal(wide["o"][..., :dv], ref["o"])
+        assert not wide["o"][..., dv:].any()
+        for name in ("final_state", "snapshots"):
+            assert np.array_equal(wide[name][..., :dv, :dk], ref[name])
+            assert not wide[name][..., dv:, :].any() and not wide[name][..., :, dk:].any()

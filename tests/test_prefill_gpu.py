@@ -292,3 +292,41 @@ def test_varlen_full_size_sampled_heads():
     inp = wl.make_prefill_inputs(wl.VARLEN, draw_device="cuda", device="cuda")
     o, fin, s = _gpu_prefill(inp)
     _check(inp, o, fin, s, heads=[5], what="varlen")
+
+
+@pytest.mark.parametrize("dk,dv,scalar,lengths,heads,snap", [
+    (64, 128, False, (300, 0, 129, 512, 64), 3, 128),     # one pass, wider values
+    (128, 64, False, (300, 1, 257, 700), 3, 64),          # one pass, wider keys
+    (64, 128, True, (2000, 700), 1, 256),                 # segmented, scalar gate
+    (128, 64, True, (3000, 65), 1, 0),                    # segmented, scalar gate
+    (128, 64, False, (1800, 0, 900), 1, 512),             # segmented, per-channel gate
+])
+def test_mixed_key_and_value_widths(dk, dv, scalar, lengths, heads, snap):
+    """d_k != d_v: o [T, H, d_v], states [N, H, d_v, d_k], snapshots, against
+    the oracle's rectangular recurrence."""
+    base = wl.GDN_LONG if scalar else wl.VARLEN
+    w = wl.shrink(base, n_heads=heads, d_k=dk, d_v=dv, lengths=lengths, init_std=0.1,
+                  snap_interval=snap, scale=0.9)
+    inp = wl.make_prefill_inputs(w)
+    o, fin, s = _gpu_prefill(inp)
+    assert tuple(o.shape) == (sum(lengths), heads, dv)
+    assert tuple(fin.shape) == (len(lengths), heads, dv, dk)
+    _check(inp, o, fin, s, what=f"d_k {dk} d_v {dv} scalar={scalar}")
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 128), (128, 64)])
+def test_mixed_widths_with_output_epilogue(dk, dv):
+    gdr = _gdr()
+    w = wl.shrink(wl.VARLEN, n_heads=2, d_k=dk, d_v=dv, lengths=(300, 129), init_std=0.1,
+                  snap_interval=0)
+    inp = wl.make_prefill_inputs(w)
+    g = wl.make_output_gate(inp["q"].shape[0], 2, dv, inp["q"].dtype, seed=88)
+    d = _to(inp, "cuda")
+    y, _, _ = gdr.prefill(d["q"], d["k"], d["v"], d["beta"], d["log_a"], d["cu_seqlens"],
+                          init_state=d["init_state"], gate_raw=g["gate_raw"].cuda(),
+                          norm_weight=g["norm_weight"].cuda(), norm_eps=1e-6)
+    torch.cuda.synchronize()
+    ref = oracle.prefill(inp["q"], inp["k"], inp["v"], inp["beta"], inp["log_a"],
+                         inp["cu_seqlens"], init_state=inp["init_state"])
+    y_ref = oracle.output_epilogue(ref["o"], g["gate_raw"], g["norm_weight"], 1e-6)
+    assert_close_rel(y, y_ref, TOL, f"gated o, d_k {dk} d_v {dv}")

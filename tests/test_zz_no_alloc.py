@@ -4,9 +4,12 @@ paths where allocation is forbidden).  It uses a fixed array inside the
 library instead of a caller workspace.
 
 Called through the C ABI twice in a row with different inputs; each result
-must match gdr_prefill's on the same inputs within the prefill tolerance of
-the other tests.  The file sorts last so that a run stopping at the first
-failure has run every other test before it.
+must equal gdr_prefill's on the same inputs bit for bit (both run the same
+kernels on the same inputs), and gdr_prefill_static_status must report that
+the kernels completed.  A CUDA graph captured around the call (after a first
+call outside capture) replays on new inputs with the same results.  The file
+sorts last so that a run stopping at the first failure has run every other
+test before it.
 """
 import ctypes
 
@@ -25,6 +28,8 @@ def _lib():
     L = gdr.lib()
     L.gdr_prefill_static_workspace.restype = ctypes.c_int
     L.gdr_prefill_static_workspace.argtypes = [ctypes.POINTER(gdr.PrefillArgs), ctypes.c_void_p]
+    L.gdr_prefill_static_status.restype = ctypes.c_int
+    L.gdr_prefill_static_status.argtypes = [ctypes.c_void_p]
     return gdr, L
 
 
@@ -76,10 +81,44 @@ def test_static_workspace_matches_prefill_twice():
         o = torch.full_like(o_ref, float("nan"))
         f = torch.full_like(f_ref, float("nan"))
         assert L.gdr_prefill_static_workspace(ctypes.byref(_args(gdr, d, o, f)), st) == 0
+        assert L.gdr_prefill_static_status(st) == 0          # no kernel gave up a wait
         torch.cuda.synchronize()
         assert not torch.isnan(o).any() and not torch.isnan(f).any()
-        assert _rel(o, o_ref) <= TOL
-        assert _rel(f, f_ref) <= TOL
+        assert torch.equal(o, o_ref) and torch.equal(f, f_ref)
+        assert _rel(o, o_ref) <= TOL and _rel(f, f_ref) <= TOL
+
+
+def test_static_workspace_under_graph_capture():
+    """The caller this entry point exists for: code captured into a CUDA
+    graph, where no allocation may happen.  One call outside capture first,
+    then capture, then replay on inputs copied into the captured buffers."""
+    gdr, L = _lib()
+    first = _inputs(4545, (300, 129), False)
+    second = _inputs(4646, (300, 129), False)
+    T, H, dk = first["q"].shape
+    n = first["cu_seqlens"].numel() - 1
+    o = torch.empty(T, H, 64, dtype=first["q"].dtype, device="cuda")
+    f = torch.empty(n, H, 64, dk, device="cuda")
+    a = _args(gdr, first, o, f)
+    st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert L.gdr_prefill_static_workspace(ctypes.byref(a), st) == 0
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        cap = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        assert L.gdr_prefill_static_workspace(ctypes.byref(a), cap) == 0
+    for name in ("q", "k", "v", "beta", "log_a", "init_state"):
+        first[name].copy_(second[name])
+    g.replay()
+    torch.cuda.synchronize()
+    assert L.gdr_prefill_static_status(st) == 0
+    o_ref = torch.empty_like(o)
+    f_ref = torch.empty_like(f)
+    ws = torch.empty(gdr.workspace_size(n, H, dk, 64, T, 0), dtype=torch.uint8, device="cuda")
+    assert L.gdr_prefill(ctypes.byref(_args(gdr, second, o_ref, f_ref, ws)), st) == 0
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_ref) and torch.equal(f, f_ref)
+    del g
 
 
 def test_static_workspace_rejects_oversized_request():

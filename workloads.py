@@ -268,3 +268,16 @@ def make_preprocess_inputs(w: PrefillWorkload, device="cpu", lengths=None, draw_
                 "cu_seqlens"):
         out[key] = out[key].to(dev).contiguous()
     return out
+
+
+def make_output_gate(T: int, H: int, d_v: int, dtype: torch.dtype, seed: int, device="cpu",
+                     draw_device=None) -> dict:
+    """Inputs of the output epilogue (RMSNorm and output gate, "kda-graft",
+    section "Идея и архитектура"): a raw gate projection gate_raw [T, H, d_v]
+    ~ N(0, 1) in the outputs' dtype and an RMSNorm weight [d_v] = 1 + N(0, 0.1)
+    in fp32 (a trained norm weight stays near its initial value of 1)."""
+    gen = torch.Generator(device=draw_device or "cpu").manual_seed(seed)
+    dd = draw_device or "cpu"
+    gate = torch.randn(T, H, d_v, generator=gen, device=dd).to(dtype)
+    weight = 1.0 + 0.1 * torch.randn(d_v, generator=gen, device=dd)
+    return {"gate_raw": gate.to(device), "norm_weight": weight.to(device)}
