@@ -3,12 +3,15 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl gdr|reference]
 
-One JSON line on rank 0.  A "step" is one chunked prefill (cumulative decay,
-intra-chunk factors, sequential state pass: three kernels) over one batch of
-the Qwen2.5-0.5B KDA-graft layer workload (1 sequence x 8192 tokens, 14 heads,
-d_k = d_v = 64, bf16 q/k/v, fp32 beta/log_a/state).  ``value`` is prefill
-tokens/s over all ranks (each rank runs its own batch: weak scaling, no
-collective on the data path).  The same run also measures:
+One JSON line on rank 0.  A "step" is one chunked prefill over one batch of
+the largest workload, the varlen mixed batch (32 sequences of 1024..16384
+tokens packed by cu_seqlens, 32 heads, d_k = d_v = 128, bf16 q/k/v, fp32
+beta/log_a/state, per-sequence initial states): the intra-chunk kernel (with
+the chunk-local cumulative decay fused in) and the sequential state pass, two
+launches (four when the pass is segmented).  ``value`` is prefill tokens/s
+over all ranks (each rank runs its own batch: weak scaling, no collective on
+the data path).  ``--workload`` picks another prefill workload for the main
+line.  The same run also measures:
 
 * ``decode``: the decode step on 256 sequences x 14 heads x 64 x 64 fp32 states,
   state bytes streamed per second (four state sets rotated so that the 235 MB
@@ -22,9 +25,14 @@ collective on the data path).  The same run also measures:
 * ``roofline``: the step's dominant kernel, timed alone with CUDA events;
 * ``e2e``: the same prefill through the public API with pinned host buffers,
   host<->device copies inside the timed region;
-* ``cpu_baseline``: the fp64 oracle on the host cores, same workload;
-* ``extra``: the other prefill workloads (tiny fp32, 65K-token scalar gate with
-  snapshots, 32-sequence varlen batch), a few steps each.
+* ``cpu_baseline``: the fp64 oracle on the host cores, a bounded sample of the
+  same workload; ``cpu_baselines``: the same for the graft layer, the long
+  Gated DeltaNet prefill and the decode step;
+* ``extra``: the other prefill workloads (tiny fp32, the Qwen2.5-0.5B graft
+  layer, the 65K-token scalar gate with snapshots), each with its own
+  roofline block; the graft layer also with the output epilogue (RMSNorm and
+  output gate) and the long prefill also with its snapshots offloaded to
+  pinned host memory.
 
 ``--impl reference`` times the fp64 CPU oracle alone (rank 0; other ranks exit).
 """
@@ -153,6 +161,64 @@ class ClockSampler:
                 "samples": len(window), "samples_inside_timed_region": len(inside)}
 
 
+class NvmlClockSampler:
+    """SM clock and clock-event reasons read through NVML (read-only queries)
+    by a thread every ~2 ms between start() and stop(), so that even a timed
+    region of a few milliseconds holds samples.  Falls back to None when NVML
+    is unavailable (the nvidia-smi sampler above then covers the run)."""
+    REASONS = (("hw_slowdown", 0x8), ("sw_thermal_slowdown", 0x20),
+               ("hw_thermal_slowdown", 0x40), ("hw_power_brake_slowdown", 0x80),
+               ("sw_power_cap", 0x4))
+
+    def __init__(self, cuda_index: int):
+        import threading
+        self.rows, self.ok, self._stop = [], False, threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            try:
+                pr = torch.cuda.get_device_properties(cuda_index)
+                bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(cuda_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+        self.thread = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.rows.append((time.perf_counter(), mhz, rs))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def start(self):
+        if self.ok:
+            self.thread.start()
+        return self
+
+    def stop(self, t0: float, t1: float):
+        if not self.ok:
+            return None
+        self._stop.set()
+        self.thread.join(timeout=5)
+        inside = [r for r in self.rows if t0 <= r[0] <= t1]
+        if not inside:
+            return None
+        reasons = sorted({n for r in inside for n, bit in self.REASONS if r[2] & bit})
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples_inside_timed_region": len(inside),
+                "source": "nvml, every ~2 ms"}
+
+
 # ---------------------------------------------------------------------------
 # distributed plumbing (one process per GPU, torchrun)
 # ---------------------------------------------------------------------------
@@ -209,9 +275,13 @@ class PrefillSets:
     """R independent input sets (rotated every step), outputs and workspaces."""
 
     def __init__(self, gdr, w: wl.PrefillWorkload, n_sets: int, rank: int):
+        """n_sets = 0: one set when its buffers alone exceed L2, else enough
+        sets (at most 4) that the rotation's footprint exceeds L2 where
+        possible."""
         self.w = w
         self.sets = []
-        for i in range(n_sets):
+        i = 0
+        while i < (n_sets or 4):
             wi = wl.shrink(w, seed=rank_seed(w.seed, i, rank))
             inp = wl.make_prefill_inputs(wi, device="cuda", draw_device="cuda")
             T, H, dk = inp["q"].shape
@@ -229,6 +299,10 @@ class PrefillSets:
                                        init_state=inp["init_state"], snap_interval=w.snap_interval,
                                        snapshots=snaps)
             self.sets.append(dict(inp=inp, prep=prep, n_snap=ns, T=T, H=H, dk=dk, dv=dv, n=n))
+            i += 1
+            one = sum(t.numel() * t.element_size() for t in prep._keep if torch.is_tensor(t))
+            if not n_sets and one * i > 2 * L2_BYTES:
+                break
         s0 = self.sets[0]
         self.T, self.H, self.dk, self.dv, self.n = s0["T"], s0["H"], s0["dk"], s0["dv"], s0["n"]
         elem = 2 if w.qkv_dtype == torch.bfloat16 else 4
@@ -239,6 +313,8 @@ class PrefillSets:
                                             s0["n_snap"]))
         self.footprint = sum(sum(t.numel() * t.element_size() for t in s["prep"]._keep
                                  if torch.is_tensor(t)) for s in self.sets)
+        self.l2 = (f"{len(self.sets)} rotating input set(s), {self.footprint / 2**20:.0f} MiB "
+                   f"{'>' if self.footprint > L2_BYTES else '<='} 126 MiB L2")
 
     def step(self, i, stages=(0, 1)):
         self.sets[i % len(self.sets)]["prep"].run(stages)
@@ -286,62 +362,153 @@ def recorded_traffic(kernel: str, workload: str):
 # ---------------------------------------------------------------------------
 # arms
 # ---------------------------------------------------------------------------
+def oracle_cores() -> int:
+    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count()))
+
+
+def _host_inputs(inp: dict, heads) -> dict:
+    """The sampled heads of a prefill batch, on the host (same bits)."""
+    out = {}
+    for k_ in ("q", "k", "v", "beta", "log_a"):
+        out[k_] = inp[k_][:, heads].cpu()
+    out["init_state"] = None if inp["init_state"] is None else inp["init_state"][:, heads].cpu()
+    out["cu_seqlens"] = inp["cu_seqlens"].cpu()
+    return out
+
+
+def oracle_prefill_sample(w: wl.PrefillWorkload, inp: dict, budget_s: float, steps: int = 0):
+    """Time the fp64 oracle on a bounded sample of workload ``w``: all of its
+    sequences, on as many heads as fit the time budget (one head's cost is
+    measured first).  Returns (tokens/s scaled to all heads, sample text,
+    seconds per pass)."""
+    import oracle
+    H = inp["q"].shape[1]
+    T = inp["q"].shape[0]
+
+    def run(heads):
+        x = _host_inputs(inp, heads)
+        t0 = time.perf_counter()
+        oracle.prefill(x["q"], x["k"], x["v"], x["beta"], x["log_a"], x["cu_seqlens"],
+                       scalar_decay=w.scalar_decay, scale=w.scale, init_state=x["init_state"],
+                       snap_interval=w.snap_interval)
+        return time.perf_counter() - t0
+
+    t1 = run([0])
+    n_heads = max(1, min(H, int(budget_s / max(t1, 1e-6))))
+    heads = list(range(n_heads))
+    passes = max(1, steps) if steps else max(1, min(20, int(budget_s / max(t1 * n_heads, 1e-6))))
+    dt = sum(run(heads) for _ in range(passes)) / passes
+    value = T * n_heads / H / dt
+    sample = (f"{passes} pass(es) over heads 0..{n_heads - 1} of {H}, all {T} tokens of "
+              f"{len(inp['lengths'])} sequence(s) of {w.name}, fp64; tokens/s = tokens x "
+              f"sampled heads / {H} / seconds")
+    return value, sample, dt
+
+
 def run_reference(args):
-    """The fp64 CPU oracle as the reference arm (rank 0 only)."""
+    """The fp64 CPU oracle as the reference arm (rank 0 only), on the main
+    line's workload, metric and unit.  The sample: every sequence and token of
+    the workload, on as many heads as fit the time budget (drawn with the
+    workload's shapes and distributions for that many heads; the oracle's
+    cost does not depend on the values)."""
     world, rank, _ = dist_env()
     if rank != 0:
         return
     import oracle
-    w = wl.GRAFT_LAYER
-    inp = wl.make_prefill_inputs(w)
-    T, H = inp["q"].shape[0], inp["q"].shape[1]
+    w = {**wl.PREFILL_WORKLOADS, **wl.PROFILE_CASES}[args.workload]
+    H = w.n_heads
 
-    def run(heads):
-        oracle.prefill(inp["q"][:, heads], inp["k"][:, heads], inp["v"][:, heads],
-                       inp["beta"][:, heads], inp["log_a"][:, heads], inp["cu_seqlens"])
+    def sample(n_heads):
+        return wl.make_prefill_inputs(wl.shrink(w, n_heads=n_heads))
 
-    # bounded sample: all heads if one pass takes <= 2 s, else the first few
-    t0 = time.perf_counter()
-    run(list(range(H)))
-    t_full = time.perf_counter() - t0
-    heads = list(range(H)) if t_full <= 2.0 else list(range(max(1, int(H * 2.0 / t_full))))
-    for _ in range(max(0, args.warmup - 1)):
-        run(heads)
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        run(heads)
-    dt = (time.perf_counter() - t0) / args.steps
-    value = T * len(heads) / H / dt          # tokens/s (token-heads/s over H)
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count()))
+    def run(x):
+        t0 = time.perf_counter()
+        oracle.prefill(x["q"], x["k"], x["v"], x["beta"], x["log_a"], x["cu_seqlens"],
+                       scalar_decay=w.scalar_decay, scale=w.scale, init_state=x["init_state"],
+                       snap_interval=w.snap_interval)
+        return time.perf_counter() - t0
+
+    budget = 8.0
+    t1 = run(sample(1))
+    n = max(1, min(H, int(budget / max(t1, 1e-6))))
+    x = sample(n)
+    for _ in range(max(0, args.warmup - 3)):
+        run(x)
+    passes = max(1, min(args.steps, int(3 * budget / max(t1 * n, 1e-6))))
+    dt = sum(run(x) for _ in range(passes)) / passes
+    T = x["q"].shape[0]
+    value = T * n / H / dt
+    sample_text = (f"{passes} pass(es) over {n} of {H} heads (drawn with the workload's shapes "
+                   f"and distributions), all {T} tokens of {len(x['lengths'])} sequence(s) of "
+                   f"{w.name}, fp64; tokens/s = tokens x {n} / {H} / seconds")
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "n_seqs": 1, "seq_len": T, "heads": H, "d_k": w.d_k,
-                       "d_v": w.d_v, "parallelism": "none (host cores)"},
-            "cpu_baseline": {"value": round(value, 1), "unit": "tokens/s", "cores": cores,
-                             "kind": "oracle",
-                             "sample": f"{len(heads)} of {H} heads x {T} tokens per step"},
+            "config": {"workload": w.name, "n_seqs": len(x["lengths"]), "tokens": T,
+                       "heads": H, "d_k": w.d_k, "d_v": w.d_v,
+                       "parallelism": "none (host cores)"},
+            "cpu_baseline": {"value": round(value, 1), "unit": "tokens/s", "cores": oracle_cores(),
+                             "kind": "oracle", "sample": sample_text},
             "e2e": {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-def cpu_baseline_graft(budget_s: float = 12.0) -> dict:
+def cpu_baseline_prefill(w: wl.PrefillWorkload, inp: dict, budget_s: float) -> dict:
+    value, sample, _ = oracle_prefill_sample(w, inp, budget_s)
+    return {"value": round(value, 1), "unit": "tokens/s", "cores": oracle_cores(),
+            "kind": "oracle", "sample": sample}
+
+
+def cpu_baseline_decode(budget_s: float) -> dict:
+    """The oracle's decode step on a sample of the decode workload's
+    sequences: state GB/s counted with the same bytes per head-state and step
+    as the GPU line."""
     import oracle
-    w = wl.GRAFT_LAYER
-    inp = wl.make_prefill_inputs(w)
-    T, H = inp["q"].shape[0], inp["q"].shape[1]
-    n, t0 = 0, time.perf_counter()
+    w = wl.DECODE
+    inp = wl.make_decode_inputs(w, steps=4)
+    B = w.batch
+    state = inp["state"].double().numpy()
+    elem = 2 if w.qkv_dtype == torch.bfloat16 else 4
+    per = decode_bytes_per_head_state(w.d_k, w.d_v, elem, w.scalar_decay)
+    b, n_steps, t_total = 16, 0, 0.0
     while True:
-        oracle.prefill(inp["q"], inp["k"], inp["v"], inp["beta"], inp["log_a"], inp["cu_seqlens"])
-        n += 1
-        if time.perf_counter() - t0 > budget_s or n >= 20:
-            break
-    dt = (time.perf_counter() - t0) / n
-    return {"value": round(T / dt, 1), "unit": "tokens/s",
-            "cores": int(os.environ.get("OMP_NUM_THREADS", os.cpu_count())), "kind": "oracle",
-            "sample": f"{n} full passes of {w.name} ({T} tokens x {H} heads), fp64"}
+        t0 = time.perf_counter()
+        oracle.decode_step(state[:b], inp["q"][0][:b], inp["k"][0][:b], inp["v"][0][:b],
+                           inp["beta"][0][:b], inp["log_a"][0][:b], scalar_decay=w.scalar_decay)
+        dt = time.perf_counter() - t0
+        if dt * B / b * 2 < budget_s and b < B:
+            b = min(B, 2 * b)
+            continue
+        n_steps, t_total = 1, dt
+        while t_total < budget_s and n_steps < 64:
+            t0 = time.perf_counter()
+            oracle.decode_step(state[:b], inp["q"][n_steps % 4][:b], inp["k"][n_steps % 4][:b],
+                               inp["v"][n_steps % 4][:b], inp["beta"][n_steps % 4][:b],
+                               inp["log_a"][n_steps % 4][:b], scalar_decay=w.scalar_decay)
+            t_total += time.perf_counter() - t0
+            n_steps += 1
+        break
+    units = b * w.n_heads * n_steps
+    gbs = per * units / t_total / 1e9
+    return {"value": round(gbs, 4), "unit": "GB/s (state bytes per head-state and step)",
+            "cores": oracle_cores(), "kind": "oracle",
+            "sample": f"{n_steps} decode step(s) of {b} of {B} sequences x {w.n_heads} heads "
+                      f"of {w.name}, fp64, {per} B per head-state and step"}
+
+
+def dominant_roofline(ps: "PrefillSets", st_ms: list, pk: dict) -> dict:
+    """Roofline block of the step's dominant kernel (the slower stage, timed
+    alone): the whole step's algorithmic bytes over that kernel's time."""
+    dom = max(range(len(STAGES)), key=lambda s_: st_ms[s_])
+    roof = roofline_obj(ps.bytes, ps.flops, st_ms[dom], pk,
+                        recorded_traffic(STAGES[dom], ps.w.name))
+    roof["kernel"] = STAGES[dom]
+    roof["kernel_ms"] = round(st_ms[dom], 4)
+    roof["algorithmic_bytes_per_step"] = ps.bytes
+    roof["algorithmic_flops_per_step"] = ps.flops
+    return roof
 
 
 def run_gdr(args):
@@ -354,65 +521,72 @@ def run_gdr(args):
     stream = torch.cuda.current_stream()
     pk = peaks()
 
-    # ---- main workload: graft-layer prefill, 4 rotating input sets ----------
-    n_sets = args.sets or (4 if args.workload != wl.VARLEN.name else 1)
-    ps = PrefillSets(gdr, {**wl.PREFILL_WORKLOADS, **wl.PROFILE_CASES}[args.workload], n_sets, rank)
+    # ---- main workload (default: the varlen batch, inputs larger than L2) ----
+    w_main = {**wl.PREFILL_WORKLOADS, **wl.PROFILE_CASES}[args.workload]
+    ps = PrefillSets(gdr, w_main, args.sets or 0, rank)
     for i in range(args.warmup):
         ps.step(i)
     torch.cuda.synchronize()
     sampler = ClockSampler(local)
+    nvml = NvmlClockSampler(local).start()
     time.sleep(0.3)
     barrier(world)
     torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t_wall0 = datetime.datetime.now()
+    t_wall0, t_perf0 = datetime.datetime.now(), time.perf_counter()
     start.record(stream)
     for i in range(args.steps):
         ps.step(i)
     end.record(stream)
     torch.cuda.synchronize()
-    t_wall1 = datetime.datetime.now()
+    t_wall1, t_perf1 = datetime.datetime.now(), time.perf_counter()
     barrier(world)
-    clocks = sampler.stop(t_wall0, t_wall1)
+    clocks = nvml.stop(t_perf0, t_perf1) or sampler.stop(t_wall0, t_wall1)
+    if nvml.ok:
+        sampler.stop(t_wall0, t_wall1)
     ms_local = start.elapsed_time(end)
     ms_total = max_over_ranks(ms_local, world)
     ms_step = ms_total / args.steps
     value = job_throughput(ps.T, world, args.steps, ms_total)
-
     launches_per_step = gdr.kernel_count(ps.n, ps.H, ps.dk, ps.dv, ps.T, ps.w.scalar_decay)
-    # the cumulative-decay kernel on its own (inside the prefill it is fused
-    # into the intra-chunk stage)
-    la, cu0 = ps.sets[0]["inp"]["log_a"], ps.sets[0]["inp"]["cu_seqlens"]
-    g_out = torch.empty_like(la)
-    stage_report_cum = round(timed(lambda i: gdr.cumdecay(la, cu0, out=g_out, d_k=ps.dk,
-                                                          scalar_decay=ps.w.scalar_decay),
-                                   50, stream), 4)
 
     # ---- the prefill stages alone -> dominant kernel roofline -------------------
-    names = list(STAGES)
-    st_ms = stage_times(ps, max(20, min(args.steps, 200)), stream)
-    dom = max(range(len(names)), key=lambda s: st_ms[s])
-    roof = roofline_obj(ps.bytes, ps.flops, st_ms[dom], pk,
-                        recorded_traffic(names[dom], ps.w.name))
-    roof["kernel"] = names[dom]
-    roof["kernel_ms"] = round(st_ms[dom], 4)
-    stage_report = {names[s]: round(st_ms[s], 4) for s in range(len(names))}
-    stage_report["cumdecay_standalone"] = stage_report_cum
+    st_ms = stage_times(ps, max(10, min(args.steps, 200)), stream)
+    roof = dominant_roofline(ps, st_ms, pk)
+    stage_report = {STAGES[s_]: round(st_ms[s_], 4) for s_ in range(len(STAGES))}
+    la, cu0 = ps.sets[0]["inp"]["log_a"], ps.sets[0]["inp"]["cu_seqlens"]
+    g_out = torch.empty_like(la)
+    stage_report["cumdecay_standalone"] = round(
+        timed(lambda i: gdr.cumdecay(la, cu0, out=g_out, d_k=ps.dk,
+                                     scalar_decay=ps.w.scalar_decay), 10, stream), 4)
     path_roof = roofline_obj(ps.bytes, ps.flops, ms_step, pk)
+    main_inp = ps.sets[0]["inp"]
+    config = {"workload": w_main.name, "n_seqs": ps.n, "tokens": ps.T, "heads": ps.H,
+              "d_k": ps.dk, "d_v": ps.dv, "parallelism": "replicas" if world > 1 else "none",
+              "l2": ps.l2}
+    del g_out
 
-    extra = {}
-    decode = None
-    spec = None
-    pre = None
+    extra, decode, spec, pre = {}, None, None, None
     if not args.no_extra:
         decode = bench_decode(gdr, stream, pk, args)
         spec = bench_spec_decode(gdr, stream, pk, args)
         pre = bench_preprocess(gdr, stream, pk, args)
-        for w in (wl.TINY_KDA, wl.GDN_LONG, wl.VARLEN):
-            extra[w.name] = bench_prefill_workload(gdr, w, stream, pk, rank, args)
-    e2e = bench_e2e(gdr, stream, args)
+        for w in (wl.TINY_KDA, wl.GRAFT_LAYER, wl.GDN_LONG, wl.VARLEN):
+            if w.name != w_main.name:
+                extra[w.name] = bench_prefill_workload(gdr, w, stream, pk, rank, args)
+    e2e = None if args.no_e2e else bench_e2e(gdr, w_main, stream, args)
 
-    cpu = cpu_baseline_graft() if (rank == 0 and world == 1 and not args.no_cpu) else None
+    cpu, cpus = None, None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline_prefill(w_main, main_inp, 8.0)
+        cpus = {"decode_" + wl.DECODE.name: cpu_baseline_decode(4.0)}
+        for w in (wl.GRAFT_LAYER, wl.GDN_LONG):
+            if w.name != w_main.name:
+                inp = wl.make_prefill_inputs(w, device="cuda", draw_device="cuda")
+                cpus[w.name] = cpu_baseline_prefill(w, inp, 4.0)
+                del inp
+    del ps, main_inp
+    torch.cuda.empty_cache()
     if rank != 0:
         if world > 1:
             torch.distributed.destroy_process_group()
@@ -422,9 +596,7 @@ def run_gdr(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": ps.w.name, "n_seqs": ps.n, "seq_len": ps.T, "heads": ps.H,
-                   "d_k": ps.dk, "d_v": ps.dv, "parallelism": "replicas" if world > 1 else "none",
-                   "l2": f"4 rotating input sets, {ps.footprint / 2**20:.0f} MiB > 126 MiB L2"},
+        "config": config,
         "roofline": roof,
         "path_roofline": path_roof,
         "kernel_ms": stage_report,
@@ -435,6 +607,7 @@ def run_gdr(args):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
         "cpu_baseline": cpu,
+        "cpu_baselines": cpus,
         "extra": extra,
         "gpu": torch.cuda.get_device_name(),
     }
@@ -444,19 +617,73 @@ def run_gdr(args):
 
 
 def bench_prefill_workload(gdr, w, stream, pk, rank, args):
-    ps = PrefillSets(gdr, w, 1 if w is not wl.TINY_KDA else 4, rank)
-    n = 3 if ps.T > 100000 else 20
+    """One prefill workload: whole step, its two stages alone, the dominant
+    kernel's roofline; the graft layer also with the output epilogue, the long
+    Gated DeltaNet prefill also with its snapshots in pinned host memory."""
+    ps = PrefillSets(gdr, w, 0, rank)
+    n = 3 if ps.T > 100000 else (10 if ps.T > 20000 else 20)
     for i in range(2):
         ps.step(i)
     ms = timed(lambda i: ps.step(i), n, stream)
     st = stage_times(ps, n, stream)
     res = {"tokens_per_s": round(ps.T / (ms * 1e-3), 1), "ms_per_step": round(ms, 4),
-           "kernel_ms": {k: round(v, 4) for k, v in zip(STAGES, st)},
+           "kernel_ms": {k_: round(v_, 4) for k_, v_ in zip(STAGES, st)},
+           "roofline": dominant_roofline(ps, st, pk),
            "path_roofline": roofline_obj(ps.bytes, ps.flops, ms, pk), "tokens": ps.T,
-           "sequences": ps.n, "inputs_exceed_l2": ps.footprint > L2_BYTES}
+           "sequences": ps.n, "l2": ps.l2, "steps": n}
+    if w is wl.GRAFT_LAYER:
+        res["output_epilogue"] = bench_epilogue(gdr, ps, stream, ms, n)
+    if w.snap_interval:
+        res["snapshot_offload"] = bench_offload(gdr, ps, stream, ms, n)
     del ps
     torch.cuda.empty_cache()
     return res
+
+
+def bench_epilogue(gdr, ps, stream, ms_plain, n):
+    """The same prefill with the RMSNorm and output gate fused into the
+    output store (gate_raw [T, H, d_v] bf16 and norm weight [d_v])."""
+    gated = []
+    for i, s_ in enumerate(ps.sets):
+        inp = s_["inp"]
+        g = wl.make_output_gate(s_["T"], s_["H"], s_["dv"], inp["q"].dtype, seed=5000 + i,
+                                device="cuda", draw_device="cuda")
+        p = s_["prep"]
+        gated.append((g, gdr.PreparedPrefill(
+            inp["q"], inp["k"], inp["v"], inp["beta"], inp["log_a"], inp["cu_seqlens"],
+            out=p.out, final_state=p.final_state, workspace=p.workspace,
+            scalar_decay=ps.w.scalar_decay, scale=ps.w.scale, init_state=inp["init_state"],
+            snap_interval=ps.w.snap_interval, snapshots=p.snapshots, gate_raw=g["gate_raw"],
+            norm_weight=g["norm_weight"])))
+    for i in range(2):
+        gated[i % len(gated)][1].run()
+    ms = timed(lambda i: gated[i % len(gated)][1].run(), n, stream)
+    gate_bytes = gated[0][0]["gate_raw"].numel() * gated[0][0]["gate_raw"].element_size()
+    return {"ms_per_step": round(ms, 4), "plain_ms_per_step": round(ms_plain, 4),
+            "overhead_frac": round(ms / ms_plain - 1.0, 4), "gate_bytes_per_step": gate_bytes}
+
+
+def bench_offload(gdr, ps, stream, ms_plain, n):
+    """The same prefill with its snapshots written by the state-pass kernel
+    straight into pinned host memory (no device copy, no copy stream)."""
+    runs = []
+    for s_ in ps.sets:
+        inp, p = s_["inp"], s_["prep"]
+        host = torch.empty(tuple(p.snapshots.shape), dtype=torch.float32).pin_memory()
+        runs.append((host, gdr.PreparedPrefill(
+            inp["q"], inp["k"], inp["v"], inp["beta"], inp["log_a"], inp["cu_seqlens"],
+            out=p.out, final_state=p.final_state, workspace=p.workspace,
+            scalar_decay=ps.w.scalar_decay, scale=ps.w.scale, init_state=inp["init_state"],
+            snap_interval=ps.w.snap_interval, snapshots=host)))
+    for i in range(2):
+        runs[i % len(runs)][1].run()
+    ms = timed(lambda i: runs[i % len(runs)][1].run(), n, stream)
+    torch.cuda.synchronize()
+    same = bool(torch.equal(runs[0][0], ps.sets[0]["prep"].snapshots.cpu())) if len(runs) == 1 else None
+    nbytes = runs[0][0].numel() * 4
+    return {"ms_per_step": round(ms, 4), "device_snapshots_ms_per_step": round(ms_plain, 4),
+            "overhead_frac": round(ms / ms_plain - 1.0, 4), "host_bytes_per_step": nbytes,
+            "bitwise_equal_to_device_snapshots": same}
 
 
 def bench_decode(gdr, stream, pk, args):
@@ -577,11 +804,22 @@ def bench_preprocess(gdr, stream, pk, args):
         pre(i)
         sets[i % 4][2].run()
 
+    def plain(i):
+        sets[i % 4][2].run()
+
+    def fused(i):
+        inp, _, prep = sets[i % 4]
+        gdr.prefill_from_projections(*(inp[n_] for n_ in names), out=prep.out,
+                                     final_state=prep.final_state, workspace=prep.workspace)
+
     for i in range(8):
         layer(i)
+        fused(i)
     n = 200
     ms_p = timed(pre, n, stream)
     ms_l = timed(layer, n, stream)
+    ms_plain = timed(plain, n, stream)
+    ms_f = timed(fused, n, stream)
     T, H, d = sets[0][0]["xq"].shape
     elem = 2 if w.qkv_dtype == torch.bfloat16 else 4
     per = preprocess_bytes_per_token_head(d, elem, w.scalar_decay)
@@ -593,31 +831,45 @@ def bench_preprocess(gdr, stream, pk, args):
                         "traffic": recorded_traffic("preprocess", w.name)},
            "with_prefill": {"ms_per_step": round(ms_l, 5),
                             "tokens_per_s": round(T / (ms_l * 1e-3), 1)},
+           "fused_prefill_from_projections": {
+               "ms_per_step": round(ms_f, 5), "tokens_per_s": round(T / (ms_f * 1e-3), 1),
+               "plain_prefill_ms": round(ms_plain, 5),
+               "over_plain_prefill": round(ms_f / ms_plain - 1.0, 4)},
            "l2": "4 rotating input and output sets, 4 x 148 MB > 126 MB L2", "steps": n}
     del sets
     torch.cuda.empty_cache()
     return res
 
 
-def bench_e2e(gdr, stream, args):
-    """Prefill through the public API from pinned host buffers: H2D of the
-    inputs, the prefill, D2H of o and the final state, every step."""
-    w = wl.GRAFT_LAYER
-    host = wl.make_prefill_inputs(w)
-    pinned = {k: host[k].pin_memory() for k in ("q", "k", "v", "beta", "log_a", "cu_seqlens")}
-    dev = {k: torch.empty_like(v, device="cuda") for k, v in pinned.items()}
-    T, H, dk = host["q"].shape
-    dv = host["v"].shape[-1]
-    out = torch.empty(T, H, dv, dtype=host["q"].dtype, device="cuda")
-    fin = torch.empty(1, H, dv, dk, device="cuda")
-    ws = torch.empty(gdr.workspace_size(1, H, dk, dv, T), dtype=torch.uint8, device="cuda")
+def bench_e2e(gdr, w, stream, args):
+    """The main workload's prefill through the public API from pinned host
+    buffers: H2D of the inputs, the prefill, D2H of o and the final states,
+    every step."""
+    dev0 = wl.make_prefill_inputs(w, device="cuda", draw_device="cuda")
+    names = [k_ for k_ in ("q", "k", "v", "beta", "log_a", "cu_seqlens", "init_state")
+             if dev0.get(k_) is not None]
+    pinned = {k_: dev0[k_].cpu().pin_memory() for k_ in names}
+    dev = {k_: torch.empty_like(dev0[k_]) for k_ in names}
+    del dev0
+    T, H, dk = pinned["q"].shape
+    dv = pinned["v"].shape[-1]
+    n = pinned["cu_seqlens"].numel() - 1
+    out = torch.empty(T, H, dv, dtype=pinned["q"].dtype, device="cuda")
+    fin = torch.empty(n, H, dv, dk, device="cuda")
+    ns = gdr.snapshot_count(pinned["cu_seqlens"], w.snap_interval) if w.snap_interval else 0
+    snaps = torch.empty(max(ns, 1), H, dv, dk, device="cuda") if w.snap_interval else None
+    ws = torch.empty(gdr.workspace_size(n, H, dk, dv, T, w.scalar_decay), dtype=torch.uint8,
+                     device="cuda")
     out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     fin_h = torch.empty(fin.shape, dtype=fin.dtype).pin_memory()
     prep = gdr.PreparedPrefill(dev["q"], dev["k"], dev["v"], dev["beta"], dev["log_a"],
-                               dev["cu_seqlens"], out=out, final_state=fin, workspace=ws)
+                               dev["cu_seqlens"], out=out, final_state=fin, workspace=ws,
+                               scalar_decay=w.scalar_decay, scale=w.scale,
+                               init_state=dev.get("init_state"), snap_interval=w.snap_interval,
+                               snapshots=snaps)
 
     def step(_):
-        for k_ in pinned:
+        for k_ in names:
             dev[k_].copy_(pinned[k_], non_blocking=True)
         prep.run()
         out_h.copy_(out, non_blocking=True)
@@ -625,12 +877,16 @@ def bench_e2e(gdr, stream, args):
 
     for i in range(3):
         step(i)
-    n = max(5, min(args.steps, 50))
-    ms = timed(step, n, stream)
+    n_steps = max(5, min(args.steps, 20))
+    ms = timed(step, n_steps, stream)
     h2d = sum(t.numel() * t.element_size() for t in pinned.values())
     d2h = out_h.numel() * out_h.element_size() + fin_h.numel() * fin_h.element_size()
-    return {"value": round(T / (ms * 1e-3), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 4), "steps": n}
+    res = {"value": round(T / (ms * 1e-3), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 4), "steps": n_steps,
+           "workload": w.name}
+    del pinned, dev, out, fin, ws, out_h, fin_h, prep, snaps
+    torch.cuda.empty_cache()
+    return res
 
 
 def main():
@@ -641,17 +897,20 @@ def main():
     p.add_argument("--impl", choices=["gdr", "reference"], default="gdr")
     p.add_argument("--no-extra", action="store_true", help="skip decode and the other workloads")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    p.add_argument("--no-e2e", action="store_true",
+                   help="skip the end-to-end measurement (for profiling runs)")
     p.add_argument("--only-decode", action="store_true",
                    help="run only the decode measurement (for profiling)")
     p.add_argument("--only-spec", action="store_true",
                    help="run only the speculative-decoding measurement (for profiling)")
     p.add_argument("--only-preprocess", action="store_true",
                    help="run only the input-activation measurement (for profiling)")
-    p.add_argument("--workload", default=wl.GRAFT_LAYER.name,
+    p.add_argument("--workload", default=wl.VARLEN.name,
                    choices=sorted(wl.PREFILL_WORKLOADS) + sorted(wl.PROFILE_CASES),
-                   help="prefill workload of the main line (default: the graft layer)")
+                   help="prefill workload of the main line (default: the varlen batch, the "
+                        "largest workload)")
     p.add_argument("--sets", type=int, default=0,
-                   help="rotating input sets of the main line (default 4; 1 for varlen)")
+                   help="rotating input sets of the main line (default: enough to exceed L2)")
     args = p.parse_args()
     if args.warmup < 3:
         p.error("--warmup must be >= 3")

@@ -20,7 +20,8 @@ import threading
 import torch
 
 __all__ = ["PrefillArgs", "PreparedPrefill", "prefill", "kernel_count", "decode_step",
-           "decode_draft", "decode_accept", "PreprocessArgs", "preprocess", "cumdecay", "chunk_factors", "workspace_size",
+           "decode_draft", "decode_accept", "PreprocessArgs", "preprocess", "Projections",
+           "prefill_from_projections", "cumdecay", "chunk_factors", "workspace_size",
            "snapshot_count", "snapshot_offsets", "prefill_status", "lib", "GdrError", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_build", "libgdr.so")
@@ -51,6 +52,15 @@ class PrefillArgs(ctypes.Structure):
         ("gate_raw", ctypes.c_void_p), ("norm_weight", ctypes.c_void_p),
         ("norm_eps", ctypes.c_float), ("workspace", ctypes.c_void_p),
         ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
+class Projections(ctypes.Structure):
+    """Mirror of ``gdr_projections`` (include/gdr.h)."""
+    _fields_ = [
+        ("xq", ctypes.c_void_p), ("xk", ctypes.c_void_p), ("xv", ctypes.c_void_p),
+        ("conv_q", ctypes.c_void_p), ("conv_k", ctypes.c_void_p), ("conv_v", ctypes.c_void_p),
+        ("beta_raw", ctypes.c_void_p), ("a_raw", ctypes.c_void_p), ("a_bias", ctypes.c_void_p),
     ]
 
 
@@ -112,6 +122,9 @@ def lib():
             L.gdr_decode_step_gated.restype = i
             L.gdr_decode_step_gated.argtypes = [i, i, i, i, i, vp, vp, vp, vp, vp, i, f, vp, vp,
                                                 vp, f, vp, vp]
+            L.gdr_prefill_from_projections.restype = i
+            L.gdr_prefill_from_projections.argtypes = [ctypes.POINTER(PrefillArgs),
+                                                       ctypes.POINTER(Projections), vp]
             L.gdr_preprocess.restype = i
             L.gdr_preprocess.argtypes = [ctypes.POINTER(PreprocessArgs), vp]
             L.gdr_decode_draft.restype = i
@@ -592,3 +605,70 @@ def preprocess(xq, xk, xv, conv_q, conv_k, conv_v, beta_raw, a_raw, a_bias, cu_s
     a.beta, a.log_a = out["beta"].data_ptr(), out["log_a"].data_ptr()
     _check(lib().gdr_preprocess(ctypes.byref(a), _stream(dev)), "gdr_preprocess")
     return out
+
+
+def prefill_from_projections(xq, xk, xv, conv_q, conv_k, conv_v, beta_raw, a_raw, a_bias,
+                             cu_seqlens, *, scalar_decay=False, scale=1.0, init_state=None,
+                             snap_interval=0, cu_seqlens_host=None, out=None, final_state=None,
+                             snapshots=None, workspace=None, gate_raw=None, norm_weight=None,
+                             norm_eps=1e-6):
+    """``preprocess`` and ``prefill`` in one: the input activations (conv-4, L2
+    norm of q and k, beta and log-decay gates) are applied inside the
+    prefill's first kernel.  Raw projections as for ``preprocess`` (bf16);
+    the other arguments and the result (o, final_state, snapshots) as for
+    ``prefill``."""
+    if xq.dtype != torch.bfloat16 or xk.dtype != xq.dtype or xv.dtype != xq.dtype:
+        raise TypeError("the fused path takes bf16 projections")
+    _expect_dim(xq, 3, "xq")
+    T, H, d = xq.shape
+    for name, t in (("xk", xk), ("xv", xv)):
+        _expect(t, (T, H, d), xq.dtype, name)
+    for name, t in (("conv_q", conv_q), ("conv_k", conv_k), ("conv_v", conv_v)):
+        _expect(t, (H * d, 4), torch.float32, name)
+    _expect(beta_raw, (T, H), torch.float32, "beta_raw")
+    _expect(a_raw, (T, H) if scalar_decay else (T, H, d), torch.float32, "a_raw")
+    _expect(a_bias, (H,) if scalar_decay else (H, d), torch.float32, "a_bias")
+    _check_cu(cu_seqlens, T, cu_seqlens_host)
+    n = cu_seqlens.numel() - 1
+    _expect(init_state, (n, H, d, d), torch.float32, "init_state")
+    _expect(out, (T, H, d), xq.dtype, "out")
+    _expect(final_state, (n, H, d, d), torch.float32, "final_state")
+    _check_gate(gate_raw, norm_weight, norm_eps, (T, H, d), xq.dtype)
+    _need_cuda(xq, xk, xv, conv_q, conv_k, conv_v, beta_raw, a_raw, a_bias, cu_seqlens,
+               init_state, out, final_state, workspace)
+    _check_snapshot_buffer(snapshots)
+    dev = xq.device
+    if out is None:
+        out = torch.empty(T, H, d, dtype=xq.dtype, device=dev)
+    if final_state is None:
+        final_state = torch.empty(n, H, d, d, dtype=torch.float32, device=dev)
+    if snap_interval and snapshots is None:
+        ns = snapshot_count(_host_cu(cu_seqlens, cu_seqlens_host), snap_interval)
+        snapshots = torch.empty(max(ns, 1), H, d, d, dtype=torch.float32, device=dev)[:ns]
+    if workspace is None:
+        workspace = torch.empty(workspace_size(n, H, d, d, T, scalar_decay), dtype=torch.uint8,
+                                device=dev)
+    snap_arg = snapshots if (snap_interval and snapshots is not None and snapshots.numel()) else None
+    if snap_interval and snap_arg is None:
+        snap_arg = final_state
+    a = PrefillArgs()
+    a.n_seqs, a.n_heads, a.d_k, a.d_v, a.total_tokens = n, H, d, d, T
+    a.cu_seqlens = cu_seqlens.data_ptr()
+    a.qkv_dtype = GDR_BF16
+    a.scalar_decay = int(bool(scalar_decay))
+    a.scale = float(scale)
+    a.init_state = None if init_state is None else init_state.data_ptr()
+    a.o, a.final_state = out.data_ptr(), final_state.data_ptr()
+    a.snap_interval = int(snap_interval)
+    a.snapshots = None if snap_arg is None else snap_arg.data_ptr()
+    a.gate_raw = None if gate_raw is None else gate_raw.data_ptr()
+    a.norm_weight = None if norm_weight is None else norm_weight.data_ptr()
+    a.norm_eps = float(norm_eps)
+    a.workspace, a.workspace_bytes = workspace.data_ptr(), workspace.numel()
+    p = Projections()
+    p.xq, p.xk, p.xv = xq.data_ptr(), xk.data_ptr(), xv.data_ptr()
+    p.conv_q, p.conv_k, p.conv_v = conv_q.data_ptr(), conv_k.data_ptr(), conv_v.data_ptr()
+    p.beta_raw, p.a_raw, p.a_bias = beta_raw.data_ptr(), a_raw.data_ptr(), a_bias.data_ptr()
+    _check(lib().gdr_prefill_from_projections(ctypes.byref(a), ctypes.byref(p), _stream(dev)),
+           "gdr_prefill_from_projections")
+    return out, final_state, snapshots

@@ -16,7 +16,13 @@ bool aligned_elem(const void* p, gdr_dtype dt) {
     return (reinterpret_cast<uintptr_t>(p) & (dt == GDR_BF16 ? 1u : 3u)) == 0;
 }
 
-gdr_status from_cuda(cudaError_t e) { return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA; }
+// A failed launch also leaves the runtime's last-error state set; it is
+// cleared here so that the next call's launch check does not report it again.
+gdr_status from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return GDR_OK;
+    (void)cudaGetLastError();
+    return GDR_ERR_CUDA;
+}
 
 bool supported_width(int d) { return d == 64 || d == 128; }
 
@@ -67,6 +73,23 @@ gdr_status check_workspace(const gdr_prefill_args* a, WorkspaceLayout* lay) {
     if (!a->workspace || (reinterpret_cast<uintptr_t>(a->workspace) & 255u) != 0)
         return GDR_ERR_WORKSPACE;
     if (a->workspace_bytes < lay->total) return GDR_ERR_WORKSPACE;
+    return GDR_OK;
+}
+
+// Checks of the prefill's outputs and options (not of its inputs).
+gdr_status check_prefill_outputs(const gdr_prefill_args* a) {
+    if (!a->final_state || !aligned16(a->final_state)) return GDR_ERR_INVALID_ARG;
+    if (a->total_tokens > 0 && (!a->o || !aligned_elem(a->o, a->qkv_dtype))) return GDR_ERR_INVALID_ARG;
+    if (a->init_state && !aligned16(a->init_state)) return GDR_ERR_INVALID_ARG;
+    if (a->snap_interval > 0 && (!a->snapshots || !aligned16(a->snapshots)))
+        return GDR_ERR_INVALID_ARG;
+    if (a->snap_offsets && (reinterpret_cast<uintptr_t>(a->snap_offsets) & 7u) != 0)
+        return GDR_ERR_INVALID_ARG;
+    if (a->gate_raw) {
+        if (!aligned16(a->gate_raw) || !a->norm_weight || !aligned16(a->norm_weight))
+            return GDR_ERR_INVALID_ARG;
+        if (!(a->norm_eps >= 0.f) || a->norm_eps > 3.0e38f) return GDR_ERR_INVALID_ARG;
+    }
     return GDR_OK;
 }
 
@@ -131,6 +154,49 @@ gdr_status gdr_snapshot_offsets(const int32_t* host_cu, int n_seqs, int snap_int
     }
     out[n_seqs] = total;
     return GDR_OK;
+}
+
+gdr_status gdr_prefill_from_projections(const gdr_prefill_args* a, const gdr_projections* p,
+                                        void* stream) {
+    if (!a || !p) return GDR_ERR_INVALID_ARG;
+    // the raw tensors take the places of q, k, v, beta and log a
+    gdr_prefill_args r = *a;
+    r.q = p->xq;
+    r.k = p->xk;
+    r.v = p->xv;
+    r.beta = p->beta_raw;
+    r.log_a = p->a_raw;
+    gdr_status s = check_prefill_inputs(&r);
+    if (s != GDR_OK) return s;
+    if (r.qkv_dtype != GDR_BF16 || r.d_k != r.d_v) return GDR_ERR_UNSUPPORTED;
+    if (r.total_tokens > 0) {
+        const void* taps[] = {p->conv_q, p->conv_k, p->conv_v};
+        for (const void* t : taps)
+            if (!t || !aligned16(t)) return GDR_ERR_INVALID_ARG;
+        if (!p->a_bias || !(r.scalar_decay ? aligned4(p->a_bias) : aligned16(p->a_bias)))
+            return GDR_ERR_INVALID_ARG;
+    }
+    s = check_prefill_outputs(&r);
+    if (s != GDR_OK) return s;
+    WorkspaceLayout lay;
+    s = check_workspace(&r, &lay);
+    if (s != GDR_OK) return s;
+    if (r.n_seqs == 0) return GDR_OK;
+    if (r.snap_interval > 0) {
+        s = kernel_address(a->snapshots, reinterpret_cast<void**>(&r.snapshots));
+        if (s != GDR_OK) return s;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(r.workspace);
+    uint32_t* err = reinterpret_cast<uint32_t*>(ws + lay.err_off);
+    uint8_t* rec = ws + lay.rec_off;
+    if (cudaMemsetAsync(err, 0, sizeof(uint32_t), st) != cudaSuccess) return from_cuda(cudaErrorUnknown);
+    if (r.total_tokens > 0) {
+        s = from_cuda(gdr::launch_intra_chunk_raw(r, p->conv_q, p->conv_k, p->conv_v, p->a_bias, rec,
+                                                  err, st));
+        if (s != GDR_OK) return s;
+    }
+    return from_cuda(gdr::launch_state_pass(r, rec, lay, ws, err, st));
 }
 
 gdr_status gdr_prefill_stages(const gdr_prefill_args* a, int first, int last, void* stream) {

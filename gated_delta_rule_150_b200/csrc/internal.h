@@ -166,6 +166,10 @@ cudaError_t launch_cumdecay(int n_seqs, int H, int D, int64_t T, const int32_t* 
 cudaError_t launch_intra_chunk(const gdr_prefill_args& a, uint8_t* records, uint32_t* err,
                                cudaStream_t st);
 
+cudaError_t launch_intra_chunk_raw(const gdr_prefill_args& a, const float* wq, const float* wk,
+                                   const float* wv, const float* a_bias, uint8_t* records,
+                                   uint32_t* err, cudaStream_t st);
+
 cudaError_t launch_state_pass(const gdr_prefill_args& a, const uint8_t* records,
                               const WorkspaceLayout& lay, uint8_t* ws, uint32_t* err,
                               cudaStream_t st);

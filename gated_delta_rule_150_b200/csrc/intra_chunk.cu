@@ -68,7 +68,17 @@ constexpr int kLd = 68;                       // row stride (floats) of the fp32
 __host__ __device__ constexpr uint32_t al1024(uint32_t x) { return (x + 1023u) & ~1023u; }
 __host__ __device__ constexpr uint32_t umax(uint32_t a, uint32_t b) { return a > b ? a : b; }
 
-template <int D, typename InT, bool SCALAR>
+// Gate activations of the fused input path (raw projections).
+__device__ __forceinline__ float log_sigmoid_f(float z) {
+    return fminf(z, 0.f) - log1pf(__expf(-fabsf(z)));
+}
+
+__device__ __forceinline__ float sigmoid_f(float z) {
+    const float e = __expf(-fabsf(z));
+    return z >= 0.f ? 1.0f / (1.0f + e) : e / (1.0f + e);
+}
+
+template <int D, typename InT, bool SCALAR, bool RAW = false>
 struct IntraLayout {
     static constexpr uint32_t elem = sizeof(InT);
     // fp32 q/k/v at d 128 do not fit next to everything else: read from global
@@ -88,9 +98,10 @@ struct IntraLayout {
     static constexpr uint32_t op_bytes = SCALAR ? 256u * D : 576u * D;
     static constexpr uint32_t As = r1;                        // fp32 [64][kLd]
     static constexpr uint32_t Pt = As + 64u * kLd * 4u;       // bf16 [64][64]
-    static constexpr uint32_t Tb = Pt + 8192u;                // bf16 [64][64]
-    static constexpr uint32_t Yt = Tb + 8192u;                // fp32 [32][32] scratch
-    static constexpr uint32_t solve_bytes = 64u * kLd * 4u + 16384u + 4096u;
+    static constexpr uint32_t Tb = Pt + 8192u;                // bf16 [64][64] (d 128)
+    static constexpr uint32_t Yt = Tb + 8192u;                // fp32 [32][32] scratch (d 128)
+    // d 64 applies (I + A)^-1 by substitution on B: no T tile, no scratch
+    static constexpr uint32_t solve_bytes = 64u * kLd * 4u + (D == 64 ? 8192u : 16384u + 4096u);
     static constexpr uint32_t Rec = r1;                       // record staging
     static constexpr uint32_t rec_bytes = record_layout(D).bytes;
     static constexpr uint32_t r2 = al1024(umax(umax(op_bytes, solve_bytes),
@@ -103,13 +114,16 @@ struct IntraLayout {
     static constexpr uint32_t Gl = Qgs + 128u * D;            // fp32 [D] g_last
     static constexpr uint32_t Bs = Gl + 4u * D;               // fp32 [64] beta
     static constexpr uint32_t Gs = Bs + 256u;                 // fp32 [64] g (scalar decay)
-    // fp32 scan partials [1024 B], live only during the scan: in region 2
-    // past the operands and the (possibly still draining) record when it fits
-    static constexpr uint32_t free2 = umax(op_bytes, rec_bytes);
+    // fp32 partials of the per-channel scan [1024 B]: that scan runs only for
+    // a CTA's first item (later items are scanned during the previous item's
+    // solve, without partials), when nothing else is in region 2
     static constexpr uint32_t kPtotBytes = 4u * threads_for<D, SCALAR>();
-    static constexpr bool kPtotInR2 = free2 + kPtotBytes <= r2;
-    static constexpr uint32_t Ptot = kPtotInR2 ? r1 + free2 : Gs + 256u;
-    static constexpr uint32_t bytes = Gs + 256u + (kPtotInR2 ? 0u : kPtotBytes);
+    static constexpr uint32_t Ptot = r1;
+    // raw projections (fused input activations): the three rows before the
+    // chunk of x_q, x_k, x_v, each [3][D] (zeros before the sequence start)
+    static constexpr uint32_t Halo = Gs + 256u;
+    static constexpr uint32_t halo_bytes = RAW ? 3u * 3u * D * elem : 0u;
+    static constexpr uint32_t bytes = Halo + halo_bytes;
     // at d 128 the 512 TMEM columns of a CTA allow one CTA per SM: request
     // enough shared memory that a second one is never scheduled
     static constexpr uint32_t dyn_bytes = (D == 128) ? umax(bytes + 1024u, 118784u) : bytes + 1024u;
@@ -117,6 +131,8 @@ struct IntraLayout {
         return KT0 + 32u * D * (uint32_t)(b * (b + 1) / 2);
     }
     static_assert(dyn_bytes <= 232448u, "shared memory budget");
+    static_assert(kPtotBytes <= r2, "scan partials fit in region 2");
+    static_assert(!RAW || kStageQKV, "raw projections are staged");
     static_assert((64u * kLd * 4u) % 1024u == 0u, "Pt alignment");
     static_assert(Rec + rec_bytes <= Qgs, "record staging stays below Qgs");
     // TMEM is allocated once per persistent CTA: never more CTAs on an SM
@@ -230,8 +246,9 @@ __device__ __forceinline__ bool bar_or(int id, int count, bool pred) {
 // by NS threads (t = 0 .. NS-1): 128 / D row parts per channel, the parts
 // joined by a shuffle.  Rows past len add 0.  Returns whether this thread saw
 // a log a below -kMaxFactorExp / 8.
-template <int D, int NS>
-__device__ __forceinline__ bool scan_channels(float* sG, int len, int t) {
+template <int D, int NS, bool RAW>
+__device__ __forceinline__ bool scan_channels(float* sG, int len, int t,
+                                              const float* __restrict__ bias) {
     static_assert(NS == 128 && (D == 64 || D == 128), "two parts of 32 rows (d 64) or one of 64");
     constexpr int P = NS / D, RP = 64 / P;
     // D = 64: channel c = 16 (t / 32) + (t % 32) / 2, part = t % 2; D = 128: c = t
@@ -240,8 +257,10 @@ __device__ __forceinline__ bool scan_channels(float* sG, int len, int t) {
     bool bad = false;
     float run = 0.f;
 #pragma unroll 4
+    const float bc = RAW ? __ldg(bias + c) : 0.f;
     for (int r = part * RP; r < (part + 1) * RP; ++r) {
-        const float la = r < len ? sG[r * D + c] : 0.f;
+        // raw projections: log a = log_sigmoid(a_raw + bias) on the fly
+        const float la = r < len ? (RAW ? log_sigmoid_f(sG[r * D + c] + bc) : sG[r * D + c]) : 0.f;
         bad |= la < -kMaxFactorExp / 8.f;
         run += la;
         sG[r * D + c] = run;
@@ -260,13 +279,14 @@ __device__ __forceinline__ bool scan_channels(float* sG, int len, int t) {
 struct Item {
     int64_t idx;
     int h, start, len;
+    int sstart;                 // first token of the chunk's sequence
 };
 
 // The first item at or after `from`, stepping by the grid size, whose chunk
 // slot holds a chunk (the slot map leaves one unused slot per sequence).
 __device__ __forceinline__ Item find_item(const int32_t* __restrict__ cu, int n_seqs, int H,
                                           int64_t n_items, int64_t from) {
-    Item it{-1, 0, 0, 0};
+    Item it{-1, 0, 0, 0, 0};
     for (int64_t i = from; i < n_items; i += gridDim.x) {
         int seq, start, len;
         if (slot_to_chunk(cu, n_seqs, i / H, &seq, &start, &len)) {
@@ -274,6 +294,7 @@ __device__ __forceinline__ Item find_item(const int32_t* __restrict__ cu, int n_
             it.h = (int)(i % H);
             it.start = start;
             it.len = len;
+            it.sstart = __ldg(cu + seq);
             break;
         }
     }
@@ -288,14 +309,27 @@ struct InputMaps {
     CUtensorMap q, k, v, g;
 };
 
+// Fused input activations ("kda-graft", section "Идея и архитектура": a
+// width-4 conv initialised as an identity tap, the alpha gate with bias +5,
+// beta): the maps above then read the raw projections x_q, x_k, x_v and
+// a_raw, beta comes from beta_raw, and these are the per-head parameters.
+struct RawParams {
+    const float* wq;            // [H D, 4] conv taps (tap 3 = current token)
+    const float* wk;
+    const float* wv;
+    const float* a_bias;        // [H, D], or [H] with a scalar gate
+};
+
+
 // Issue the copies of one item's inputs, from one warp: lane 0 starts the
 // tiled TMA loads of log a (completing on bar_g) and of q, k, v (on bar_qkv);
 // beta and the scalar log a go by 4-byte cp.async with zero fill.
-template <int D, typename InT, bool SCALAR, typename L>
+template <int D, typename InT, bool SCALAR, bool RAW, typename L>
 __device__ __forceinline__ void issue_inputs(uint8_t* sm, uint64_t* bar_g, uint64_t* bar_qkv,
                                              const InputMaps& maps, const float* __restrict__ beta,
                                              const float* __restrict__ log_a, int H, const Item& it,
-                                             int lane, bool hint) {
+                                             int lane, bool hint, const InT* __restrict__ xq,
+                                             const InT* __restrict__ xk, const InT* __restrict__ xv) {
     if (lane == 0) {
         const int x = it.h * D;
         const uint64_t pol = l2_policy_evict_first();             // inputs are read once
@@ -321,7 +355,62 @@ __device__ __forceinline__ void issue_inputs(uint8_t* sm, uint64_t* bar_g, uint6
         cp_async4(sm + L::Bs + 4 * t, beta + o, n);
         if (SCALAR) cp_async4(sm + L::Gs + 4 * t, log_a + o, n);
     }
+    if (RAW) {
+        // the three raw rows before the chunk, zeros before the sequence start
+        constexpr int kPer = D * (int)sizeof(InT) / 16;           // 16-byte pieces per row
+        for (int i = lane; i < 3 * 3 * kPer; i += 32) {
+            const int tsr = i / (3 * kPer), j = (i / kPer) % 3, piece = i % kPer;
+            const int tok = it.start - 3 + j;
+            const InT* src = tsr == 0 ? xq : (tsr == 1 ? xk : xv);
+            const bool in = tok >= it.sstart;
+            const size_t off = ((size_t)(in ? tok : it.start) * H + it.h) * D;
+            cp_async16(sm + L::Halo + ((tsr * 3 + j) * D) * sizeof(InT) + 16 * piece,
+                       reinterpret_cast<const uint8_t*>(src + off) + 16 * piece, in ? 16u : 0u);
+        }
+    }
     cp_async_commit();
+}
+
+// [W | U] = (I + A)^-1 B, one column at a time (d 64: 2D = 128 columns, one
+// per thread of warps 0-3), by forward substitution in fp32:
+//     x_r = b_r - sum_{i<r} A[r, i] x_i,        r = 1 .. 63,
+// where column c of B = [diag(beta)(K * Gamma) | diag(beta) V] is row c of the
+// bf16 tile Bt.  A (fp32, zero on and above the diagonal, row stride kLd) is
+// read as float4 rows that every lane shares (broadcast); the column stays in
+// registers.  No barrier is needed (each thread owns its column), and the
+// result overwrites row c of Bt as row c of the bf16 tile [W | U]^T.  This is
+// the same T = (I + A)^-1 the blocked solve forms, applied to B directly and
+// without rounding T to bf16 first.
+template <int D>
+__device__ __forceinline__ void substitute_column(const float* __restrict__ As, uint8_t* Bt, int c) {
+    float x[64];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const uint4 u = *reinterpret_cast<const uint4*>(Bt + sw128_chunk(2 * D, c, j));
+        const float2 a = unpack_bf16(u.x), b = unpack_bf16(u.y), e = unpack_bf16(u.z), f = unpack_bf16(u.w);
+        x[8 * j + 0] = a.x; x[8 * j + 1] = a.y; x[8 * j + 2] = b.x; x[8 * j + 3] = b.y;
+        x[8 * j + 4] = e.x; x[8 * j + 5] = e.y; x[8 * j + 6] = f.x; x[8 * j + 7] = f.y;
+    }
+#pragma unroll
+    for (int r = 1; r < 64; ++r) {
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+        for (int i4 = 0; i4 < (r + 3) / 4; ++i4) {
+            const float4 a = *reinterpret_cast<const float4*>(As + r * kLd + 4 * i4);
+            a0 = fmaf(a.x, x[4 * i4 + 0], a0);
+            a1 = fmaf(a.y, x[4 * i4 + 1], a1);
+            a2 = fmaf(a.z, x[4 * i4 + 2], a2);
+            a3 = fmaf(a.w, x[4 * i4 + 3], a3);
+        }
+        x[r] -= (a0 + a1) + (a2 + a3);
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        float y[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) y[e] = x[8 * j + e];
+        *reinterpret_cast<uint4*>(Bt + sw128_chunk(2 * D, c, j)) = pack8(y);
+    }
 }
 
 // Read the A/P products of this thread's row from TMEM (per-channel decay).
@@ -356,14 +445,17 @@ __device__ __forceinline__ void load_ap_row(uint32_t taddr, int b, float (&v)[64
     }
 }
 
-template <int D, typename InT, bool SCALAR>
+// RAW: q, k, v, beta and log_a are the raw projections x_q, x_k, x_v,
+// beta_raw and a_raw; the input activations are applied on the fly (`rp`).
+template <int D, typename InT, bool SCALAR, bool RAW>
 __global__ void __launch_bounds__(threads_for<D, SCALAR>(), (D == 64) ? 2 : 1)
 intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                    const InT* __restrict__ q, const InT* __restrict__ k, const InT* __restrict__ v,
                    const float* __restrict__ beta, const float* __restrict__ log_a, float scale,
                    int64_t n_items, uint8_t* __restrict__ records, uint32_t* err,
-                   const __grid_constant__ InputMaps maps, int keep_records) {
-    using L = IntraLayout<D, InT, SCALAR>;
+                   const __grid_constant__ InputMaps maps, int keep_records,
+                   const __grid_constant__ RawParams rp) {
+    using L = IntraLayout<D, InT, SCALAR, RAW>;
     constexpr RecordLayout R = record_layout(D);
     constexpr int CG = D / 8;              // channel groups of 8
     constexpr int NT = threads_for<D, SCALAR>();
@@ -414,8 +506,8 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     // timed-out wait the last of each is drained before the CTA exits
     uint32_t in_issued = 0, mma_commits = 0;
     if (cur.idx >= 0 && warp == kLoadWarp) {
-        issue_inputs<D, InT, SCALAR, L>(sm, &in_bar[0], &in_bar[1], maps, beta, log_a, H, cur, lane,
-                                        keep_records != 0);
+        issue_inputs<D, InT, SCALAR, RAW, L>(sm, &in_bar[0], &in_bar[1], maps, beta, log_a, H, cur,
+                                             lane, keep_records != 0, q, k, v);
         ++in_issued;
     }
     const uint32_t tmem = tmem_slot;
@@ -461,10 +553,12 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         constexpr int P = NT / D, RP = 64 / P;                // row parts per channel
         float* Ptot = reinterpret_cast<float*>(sm + L::Ptot);
         const int c = tid % D, part = tid / D;
+        const float bc = RAW ? __ldg(rp.a_bias + (size_t)h * D + c) : 0.f;
         float run = 0.f;
 #pragma unroll 4
         for (int r = part * RP; r < (part + 1) * RP; ++r) {
-            const float la = r < len ? sG[r * D + c] : 0.f;   // rows past the end add 0
+            // rows past the end add 0; raw projections: log a = log_sigmoid(a_raw + bias)
+            const float la = r < len ? (RAW ? log_sigmoid_f(sG[r * D + c] + bc) : sG[r * D + c]) : 0.f;
             bad |= la < -kMaxFactorExp / 8.f;
             run += la;
             sG[r * D + c] = run;
@@ -478,7 +572,12 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
             for (int r = part * RP; r < (part + 1) * RP; ++r) sG[r * D + c] += off;
         }
     } else if (warp == 0) {
-        const float x0 = Gs[2 * lane], x1 = Gs[2 * lane + 1];
+        float x0 = Gs[2 * lane], x1 = Gs[2 * lane + 1];
+        if (RAW) {
+            const float bh = __ldg(rp.a_bias + h);
+            x0 = 2 * lane < len ? log_sigmoid_f(x0 + bh) : 0.f;
+            x1 = 2 * lane + 1 < len ? log_sigmoid_f(x1 + bh) : 0.f;
+        }
         const float pair = x0 + x1;
         float incl = pair;
 #pragma unroll
@@ -535,7 +634,76 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         }
     }
 
-    // ---- operands and per-token outputs -------------------------------------
+    // ---- raw projections: conv-4, L2 norm of q and k, beta ----------------------
+    // (the input activations, "kda-graft", section "Идея и архитектура").  Row
+    // r of the chunk reads raw rows r-3 .. r (the three before the chunk from
+    // the halo, zero before the sequence start); tap 3 is the current token.
+    // The staged q, k, v rows are replaced by their activated values once
+    // every thread has read the raw rows it needs.  Each thread keeps the rows
+    // and channels it builds the operands from below.
+    if constexpr (RAW) {
+        if (tid < len) Bs[tid] = sigmoid_f(Bs[tid]);
+        float y[3][RPT][8];
+#pragma unroll
+        for (int tsr = 0; tsr < 3; ++tsr) {
+            const InT* stg = reinterpret_cast<const InT*>(sm + (tsr == 0 ? L::sQ : (tsr == 1 ? L::sK : L::sV)));
+            const InT* hal = reinterpret_cast<const InT*>(sm + L::Halo) + tsr * 3 * D;
+            const float* wsrc = tsr == 0 ? rp.wq : (tsr == 1 ? rp.wk : rp.wv);
+            float w[8][4];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float4 f = __ldg(reinterpret_cast<const float4*>(wsrc + ((size_t)h * D + c0 + e) * 4));
+                w[e][0] = f.x; w[e][1] = f.y; w[e][2] = f.z; w[e][3] = f.w;
+            }
+#pragma unroll
+            for (int u = 0; u < RPT; ++u) {
+                const int r = r0 + u;
+                float x[4][8];                    // x[j]: raw row r - 3 + j
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int rr = r - 3 + j;
+                    Vec8<InT>::load(rr >= 0 ? stg + (size_t)rr * D + c0 : hal + (size_t)(rr + 3) * D + c0, x[j]);
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    float acc = w[e][3] * x[3][e];
+                    acc = fmaf(w[e][2], x[2][e], acc);
+                    acc = fmaf(w[e][1], x[1][e], acc);
+                    acc = fmaf(w[e][0], x[0][e], acc);
+                    y[tsr][u][e] = acc;
+                }
+                if (tsr < 2) {
+                    // L2 norm over the row's D channels: CG consecutive lanes
+                    float ss = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) ss = fmaf(y[tsr][u][e], y[tsr][u][e], ss);
+#pragma unroll
+                    for (int m = 1; m < CG; m <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+                    const float inv = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) y[tsr][u][e] *= inv;
+                }
+            }
+        }
+        __syncthreads();                      // every raw row has been read
+#pragma unroll
+        for (int tsr = 0; tsr < 3; ++tsr) {
+            uint8_t* stg = sm + (tsr == 0 ? L::sQ : (tsr == 1 ? L::sK : L::sV));
+#pragma unroll
+            for (int u = 0; u < RPT; ++u)
+                *reinterpret_cast<uint4*>(stg + ((size_t)(r0 + u) * D + c0) * sizeof(InT)) = pack8(y[tsr][u]);
+        }
+        // the operand passes below read only this thread's rows and channels;
+        // beta and other threads' rows are read after the next barrier
+    }
+
+    // ---- operands -------------------------------------------------------------
+    // Pass 1 builds what the A/P products read (scaled query and key rows, the
+    // key tiles); their MMA is issued at once, and pass 2 builds the operands
+    // of the later products (Qg and the transposed diag(beta)(K Gamma),
+    // diag(beta) V and Kd) while it runs.  Pass 2 recomputes the row factors
+    // (the same values: the operations are the same), which is cheaper than
+    // keeping them live across the MMA issue.
     uint8_t* XA = sm + L::XA;
     uint8_t* Bt = sm + L::Bt;
     uint8_t* Kdt = sm + L::Kdt;
@@ -545,26 +713,22 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
 #pragma unroll
         for (int e = 0; e < 8; ++e) { em[e] = __expf(mj[e]); eld[e] = __expf(gl[e] - mj[e]); }
     }
-    uint32_t pb1[8][RPT / 2], pb2[8][RPT / 2], pkd[8][RPT / 2];   // transposed bf16 pairs
-    float p_b1[8], p_bv[8], p_kd[8];                               // even row of the pair
-#pragma unroll
-    for (int u = 0; u < RPT; ++u) {
-        const int r = r0 + u;
-        const bool valid = r < len;
-        float qv[8], kv[8], vv[8], gr[8];
-        const float br = Bs[r];
+    // this thread's row r of q, k (and v): staged, from global, or zeros past the end
+    auto load_row = [&](int r, bool valid, float (&qv)[8], float (&kv)[8], float (&vv)[8], bool with_v) {
         if (valid && L::kStageQKV) {
             Vec8<InT>::load(reinterpret_cast<const InT*>(sm + L::sQ) + (size_t)r * D + c0, qv);
             Vec8<InT>::load(reinterpret_cast<const InT*>(sm + L::sK) + (size_t)r * D + c0, kv);
-            Vec8<InT>::load(reinterpret_cast<const InT*>(sm + L::sV) + (size_t)r * D + c0, vv);
+            if (with_v) Vec8<InT>::load(reinterpret_cast<const InT*>(sm + L::sV) + (size_t)r * D + c0, vv);
         } else if (valid) {
             Vec8<InT>::load(q + base + (size_t)r * tok_stride + c0, qv);
             Vec8<InT>::load(k + base + (size_t)r * tok_stride + c0, kv);
-            Vec8<InT>::load(v + base + (size_t)r * tok_stride + c0, vv);
+            if (with_v) Vec8<InT>::load(v + base + (size_t)r * tok_stride + c0, vv);
         } else {
 #pragma unroll
             for (int e = 0; e < 8; ++e) qv[e] = kv[e] = vv[e] = 0.f;
         }
+    };
+    auto load_g = [&](int r, bool valid, float (&gr)[8]) {
         if (!SCALAR) {
             if (valid) load8f(sG + (size_t)r * D + c0, gr);
             else {
@@ -575,7 +739,16 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
 #pragma unroll
             for (int e = 0; e < 8; ++e) gr[e] = Gs[r];
         }
-        float xq[8], xk[8], kk0[8], b1[8], qg[8], kd[8];
+    };
+    // pass 1: A-side operand rows r (queries) and 64 + r (keys), key tiles
+#pragma unroll
+    for (int u = 0; u < RPT; ++u) {
+        const int r = r0 + u;
+        const bool valid = r < len;
+        float qv[8], kv[8], vv[8], gr[8];
+        load_row(r, valid, qv, kv, vv, false);
+        load_g(r, valid, gr);
+        float xq[8], xk[8], kk0[8];
         if (!SCALAR && !bad_chunk) {
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
@@ -584,34 +757,14 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                 xq[e] = scale * qv[e] * F;
                 xk[e] = kv[e] * F;
                 kk0[e] = kv[e] * Fi;
-                b1[e] = br * xk[e] * em[e];
-                qg[e] = xq[e] * em[e];
-                kd[e] = kk0[e] * eld[e];
             }
         } else if (SCALAR) {
-            const float G = __expf(gr[0]), Ed = __expf(gl[0] - gr[0]);   // one gate per row
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                xq[e] = scale * qv[e];
-                xk[e] = kv[e];
-                kk0[e] = 0.f;
-                b1[e] = br * kv[e] * G;
-                qg[e] = scale * qv[e] * G;
-                kd[e] = kv[e] * Ed;
-            }
+            for (int e = 0; e < 8; ++e) { xq[e] = scale * qv[e]; xk[e] = kv[e]; kk0[e] = 0.f; }
         } else {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float G = __expf(gr[e]);
-                xq[e] = 0.f;
-                xk[e] = 0.f;
-                kk0[e] = 0.f;
-                b1[e] = br * kv[e] * G;
-                qg[e] = scale * qv[e] * G;
-                kd[e] = kv[e] * __expf(gl[e] - gr[e]);
-            }
+            for (int e = 0; e < 8; ++e) xq[e] = xk[e] = kk0[e] = 0.f;
         }
-        // A-side operand rows r (queries) and 64 + r (keys)
         *reinterpret_cast<uint4*>(XA + sw128_chunk(128, r, cg)) = pack8(xq);
         *reinterpret_cast<uint4*>(XA + sw128_chunk(128, 64 + r, cg)) = pack8(xk);
         if (!SCALAR) {
@@ -623,6 +776,74 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
 #pragma unroll
                 for (int e = 0; e < 8; ++e) kb[e] = (b == jb) ? kk0[e] : kk0[e] * ecross[b][e];
                 *reinterpret_cast<uint4*>(sm + L::kt_off(b) + sw128_chunk(16 * (b + 1), r, cg)) = pack8(kb);
+            }
+        }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+
+    // ---- decay-weighted Q K^T and K K^T on the tensor cores ------------------
+    if (tid == 0) {
+        const uint32_t aXA = smem_u32(XA);
+        if (!SCALAR) {
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const uint32_t id = idesc_bf16_f32(128, 16 * (b + 1));
+                const uint32_t aK = smem_u32(sm + L::kt_off(b));
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_bf16(tmem + ap_col(b), sw128_desc(aXA, 128, 0, 16 * kk),
+                             sw128_desc(aK, 16 * (b + 1), 0, 16 * kk), id, kk > 0);
+            }
+        } else {
+            const uint32_t id = idesc_bf16_f32(128, 64);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+                mma_bf16(tmem, sw128_desc(aXA, 128, 0, 16 * kk), sw128_desc(aXA, 128, 64, 16 * kk), id, kk > 0);
+        }
+        mma_commit(&mma_bar);
+        ++mma_commits;
+    }
+
+    // ---- pass 2, under the A/P MMA: Qg rows, transposed B1, B2, Kd ------------
+    uint32_t pb1[8][RPT / 2], pb2[8][RPT / 2], pkd[8][RPT / 2];   // transposed bf16 pairs
+    float p_b1[8], p_bv[8], p_kd[8];                               // even row of the pair
+#pragma unroll
+    for (int u = 0; u < RPT; ++u) {
+        const int r = r0 + u;
+        const bool valid = r < len;
+        float qv[8], kv[8], vv[8], gr[8];
+        const float br = Bs[r];
+        load_row(r, valid, qv, kv, vv, true);
+        load_g(r, valid, gr);
+        float b1[8], qg[8], kd[8];
+        if (!SCALAR && !bad_chunk) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float d = gr[e] - mj[e];
+                const float F = __expf(d), Fi = __expf(-d);
+                const float xq = scale * qv[e] * F, xk = kv[e] * F, kk0 = kv[e] * Fi;
+                b1[e] = br * xk * em[e];
+                qg[e] = xq * em[e];
+                kd[e] = kk0 * eld[e];
+            }
+        } else if (SCALAR) {
+            const float G = __expf(gr[0]), Ed = __expf(gl[0] - gr[0]);   // one gate per row
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                b1[e] = br * kv[e] * G;
+                qg[e] = scale * qv[e] * G;
+                kd[e] = kv[e] * Ed;
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float G = __expf(gr[e]);
+                b1[e] = br * kv[e] * G;
+                qg[e] = scale * qv[e] * G;
+                kd[e] = kv[e] * __expf(gl[e] - gr[e]);
             }
         }
         *reinterpret_cast<uint4*>(Qgs + sw128_chunk(64, r, cg)) = pack8(qg);
@@ -664,33 +885,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
             *reinterpret_cast<uint32_t*>(Kdt + o3) = pkd[e][0];
         }
     }
-    fence_proxy_async_smem();
-    tc_fence_before_sync();
-    __syncthreads();
-    tc_fence_after_sync();
-
-    // ---- decay-weighted Q K^T and K K^T on the tensor cores ------------------
-    if (tid == 0) {
-        const uint32_t aXA = smem_u32(XA);
-        if (!SCALAR) {
-#pragma unroll
-            for (int b = 0; b < 4; ++b) {
-                const uint32_t id = idesc_bf16_f32(128, 16 * (b + 1));
-                const uint32_t aK = smem_u32(sm + L::kt_off(b));
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    mma_bf16(tmem + ap_col(b), sw128_desc(aXA, 128, 0, 16 * kk),
-                             sw128_desc(aK, 16 * (b + 1), 0, 16 * kk), id, kk > 0);
-            }
-        } else {
-            const uint32_t id = idesc_bf16_f32(128, 64);
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk)
-                mma_bf16(tmem, sw128_desc(aXA, 128, 0, 16 * kk), sw128_desc(aXA, 128, 64, 16 * kk), id, kk > 0);
-        }
-        mma_commit(&mma_bar);
-        ++mma_commits;
-    }
+    fence_proxy_async_smem();         // read by later MMAs, after the next barrier
     failed = !mbar_wait(&mma_bar, phase);
     phase ^= 1u;
     tc_fence_after_sync();
@@ -734,10 +929,22 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                 float acc = 0.f;
                 if (i <= lim && rr < len) {
                     for (int c = 0; c < D; ++c) {
-                        const size_t tr = base + (size_t)rr * tok_stride + c;
-                        const size_t ti = base + (size_t)i * tok_stride + c;
-                        const float xr = is_p ? scale * (float)q[tr] : (float)k[tr];
-                        acc += xr * (float)k[ti] * expf(sG[rr * D + c] - sG[i * D + c]);
+                        // q and k as staged (the same values as in memory; with
+                        // raw projections, the activated ones)
+                        float qr, kr, ki;
+                        if (L::kStageQKV) {
+                            const InT* sq = reinterpret_cast<const InT*>(sm + L::sQ);
+                            const InT* sk = reinterpret_cast<const InT*>(sm + L::sK);
+                            qr = (float)sq[rr * D + c];
+                            kr = (float)sk[rr * D + c];
+                            ki = (float)sk[i * D + c];
+                        } else {
+                            qr = (float)q[base + (size_t)rr * tok_stride + c];
+                            kr = (float)k[base + (size_t)rr * tok_stride + c];
+                            ki = (float)k[base + (size_t)i * tok_stride + c];
+                        }
+                        const float xr = is_p ? scale * qr : kr;
+                        acc += xr * ki * expf(sG[rr * D + c] - sG[i * D + c]);
                     }
                 }
                 v32[il] = acc;
@@ -773,23 +980,29 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         const Item nxt = s_item[(iter + 1) & 1];
         fence_proxy_async_smem();             // this item's reads of region 1 come first
         if (nxt.idx >= 0) {
-            issue_inputs<D, InT, SCALAR, L>(sm, &in_bar[0], &in_bar[1], maps, beta, log_a, H, nxt, lane,
-                                            keep_records != 0);
+            issue_inputs<D, InT, SCALAR, RAW, L>(sm, &in_bar[0], &in_bar[1], maps, beta, log_a, H, nxt,
+                                                 lane, keep_records != 0, q, k, v);
             ++in_issued;
         }
         if (lane == 0)
             s_item[iter & 1] = nxt.idx >= 0 ? find_item(cu, n_seqs, H, n_items, nxt.idx + gridDim.x) : nxt;
     }
 
-    // ---- T = (I + A)^-1: 16x16 diagonal blocks, then block merges -----------
+    // ---- [W | U] = (I + A)^-1 B ------------------------------------------------
+    // d 64: forward substitution on the 128 columns of B (substitute_column),
+    // straight into the tile [W | U]^T.  d 128: T = (I + A)^-1 by the blocked
+    // solve below (16x16 diagonal blocks, then block merges), then one MMA.
     // T overwrites A in As block by block, each block once the phases that
     // still read it have passed a barrier.  Every phase also writes its bf16
     // copy straight into the operand tile Tb, whose blocks above the
     // diagonal are zeroed here.
     // Warps 0-3 solve (named barrier 1); warps 4-7 meanwhile scan the next
     // item's log a, which the loader warp has just requested.
+    constexpr bool kSubst = (D == 64);
     uint8_t* Tb = sm + L::Tb;
-    if (tid < 128) {
+    if (kSubst && tid < 2 * D) {
+        substitute_column<D>(As, Bt, tid);
+    } else if (!kSubst && tid < 128) {
         if (tid >= 64) {
             // (row, chunk) pairs of the zero blocks (b, j > b): 96 + 64 + 32
 #pragma unroll
@@ -865,7 +1078,8 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         bool nbad = false;
         if (nx.idx >= 0) {
             if (!mbar_wait(&in_bar[0], in_phase)) failed = true;
-            nbad = scan_channels<D, 128>(sG, nx.len, tid - 128);
+            nbad = scan_channels<D, 128, RAW>(sG, nx.len, tid - 128,
+                                              RAW ? rp.a_bias + (size_t)nx.h * D : nullptr);
         }
         nbad = bar_or(2, 128, nbad);
         if (tid == 128) s_bad_next = nbad ? 1 : 0;
@@ -875,7 +1089,8 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     failed = __syncthreads_or(failed);
     tc_fence_after_sync();
 
-    // ---- [W | U]^T = [diag(b)(K*Gamma) | diag(b)V]^T T^T ---------------------
+    // ---- [W | U]^T = [diag(b)(K*Gamma) | diag(b)V]^T T^T (d 128) -------------
+    if constexpr (!kSubst) {
     if (tid == 0 && !failed) {
         const uint32_t id = idesc_bf16_f32(128, 64);
         const uint32_t aB = smem_u32(Bt), aT = smem_u32(sm + L::Tb);
@@ -921,6 +1136,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     tc_fence_before_sync();
     failed = __syncthreads_or(failed);
     tc_fence_after_sync();
+    }
 
     // ---- P [W | U], Kd^T W, U^T Kd --------------------------------------------
     if (tid == 0 && !failed) {
@@ -1100,11 +1316,12 @@ cudaError_t token_map(EncodeTiledFn enc, CUtensorMap* m, const void* base, CUten
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int D, typename InT, bool SCALAR>
-cudaError_t launch_typed(const gdr_prefill_args& a, uint8_t* records, uint32_t* err,
-                         cudaStream_t st) {
-    auto kern = intra_chunk_kernel<D, InT, SCALAR>;
-    const uint32_t smem = IntraLayout<D, InT, SCALAR>::dyn_bytes;
+template <int D, typename InT, bool SCALAR, bool RAW>
+cudaError_t launch_typed(const gdr_prefill_args& a, const RawParams& rp, uint8_t* records,
+                         uint32_t* err, cudaStream_t st) {
+    auto kern = intra_chunk_kernel<D, InT, SCALAR, RAW>;
+    using Lay = IntraLayout<D, InT, SCALAR, RAW>;
+    const uint32_t smem = Lay::dyn_bytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     // all of the unified L1 / shared memory as shared memory, so that the
@@ -1142,7 +1359,7 @@ cudaError_t launch_typed(const gdr_prefill_args& a, uint8_t* records, uint32_t* 
     InputMaps maps;
     memset(&maps, 0, sizeof(maps));
     const CUtensorMapDataType dt = sizeof(InT) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-    if (IntraLayout<D, InT, SCALAR>::kStageQKV) {
+    if (Lay::kStageQKV) {
         if ((e = token_map(enc, &maps.q, a.q, dt, sizeof(InT), a.total_tokens, a.n_heads, D)) != cudaSuccess) return e;
         if ((e = token_map(enc, &maps.k, a.k, dt, sizeof(InT), a.total_tokens, a.n_heads, D)) != cudaSuccess) return e;
         if ((e = token_map(enc, &maps.v, a.v, dt, sizeof(InT), a.total_tokens, a.n_heads, D)) != cudaSuccess) return e;
@@ -1154,14 +1371,14 @@ cudaError_t launch_typed(const gdr_prefill_args& a, uint8_t* records, uint32_t* 
     return launch_pdl(true, kern, dim3(grid), dim3(threads_for<D, SCALAR>()), smem, st, a.cu_seqlens,
                       a.n_seqs, a.n_heads, (const InT*)a.q, (const InT*)a.k, (const InT*)a.v, a.beta,
                       a.log_a, a.scale, n_items, records, err, maps,
-                      records_fit_l2(n_chunk_slots(a.total_tokens, a.n_seqs), a.n_heads, D) ? 1 : 0);
+                      records_fit_l2(n_chunk_slots(a.total_tokens, a.n_seqs), a.n_heads, D) ? 1 : 0, rp);
 }
 
-template <int D, typename InT>
-cudaError_t launch_decay(const gdr_prefill_args& a, uint8_t* records, uint32_t* err,
-                         cudaStream_t st) {
-    return a.scalar_decay ? launch_typed<D, InT, true>(a, records, err, st)
-                          : launch_typed<D, InT, false>(a, records, err, st);
+template <int D, typename InT, bool RAW>
+cudaError_t launch_decay(const gdr_prefill_args& a, const RawParams& rp, uint8_t* records,
+                         uint32_t* err, cudaStream_t st) {
+    return a.scalar_decay ? launch_typed<D, InT, true, RAW>(a, rp, records, err, st)
+                          : launch_typed<D, InT, false, RAW>(a, rp, records, err, st);
 }
 
 }  // namespace
@@ -1169,11 +1386,24 @@ cudaError_t launch_decay(const gdr_prefill_args& a, uint8_t* records, uint32_t* 
 cudaError_t launch_intra_chunk(const gdr_prefill_args& a, uint8_t* records, uint32_t* err,
                                cudaStream_t st) {
     if (n_chunk_slots(a.total_tokens, a.n_seqs) == 0) return cudaSuccess;
+    const RawParams none{};
     if (a.d_k == 64)
-        return a.qkv_dtype == GDR_BF16 ? launch_decay<64, __nv_bfloat16>(a, records, err, st)
-                                       : launch_decay<64, float>(a, records, err, st);
-    return a.qkv_dtype == GDR_BF16 ? launch_decay<128, __nv_bfloat16>(a, records, err, st)
-                                   : launch_decay<128, float>(a, records, err, st);
+        return a.qkv_dtype == GDR_BF16 ? launch_decay<64, __nv_bfloat16, false>(a, none, records, err, st)
+                                       : launch_decay<64, float, false>(a, none, records, err, st);
+    return a.qkv_dtype == GDR_BF16 ? launch_decay<128, __nv_bfloat16, false>(a, none, records, err, st)
+                                   : launch_decay<128, float, false>(a, none, records, err, st);
+}
+
+// The same stage from raw projections (bf16 only): a's q, k, v, beta and
+// log_a are x_q, x_k, x_v, beta_raw and a_raw.
+cudaError_t launch_intra_chunk_raw(const gdr_prefill_args& a, const float* wq, const float* wk,
+                                   const float* wv, const float* a_bias, uint8_t* records,
+                                   uint32_t* err, cudaStream_t st) {
+    if (n_chunk_slots(a.total_tokens, a.n_seqs) == 0) return cudaSuccess;
+    if (a.qkv_dtype != GDR_BF16) return cudaErrorInvalidValue;
+    const RawParams rp{wq, wk, wv, a_bias};
+    return a.d_k == 64 ? launch_decay<64, __nv_bfloat16, true>(a, rp, records, err, st)
+                       : launch_decay<128, __nv_bfloat16, true>(a, rp, records, err, st);
 }
 
 cudaError_t launch_unpack_records(const gdr_prefill_args& a, const uint8_t* records, float* Qt,

@@ -9,19 +9,16 @@
 // k normalised per (token, head) after it as y / max(||y||, 1e-12), the conv
 // restarting from zero history at every sequence start.
 //
-// Layout of the work: D / 8 consecutive threads own one (token, head) and
-// eight consecutive channels each, so a warp reads and writes whole
-// contiguous rows of [T, H, D].  Each thread reads its channels of the
-// current token and up to three earlier ones of the same sequence (the
-// earlier rows were just read by neighbouring warps and come from L1/L2, so
-// HBM sees each row about once).  The tap loads are unconditional (a tap
-// before the sequence start reads the current row and is then skipped), so
-// all twelve are in flight together instead of one after another.  The L2
-// norms are shuffle sums over the D / 8 lanes of a (token, head).  The HBM
-// traffic is x_q, x_k, x_v, beta_raw, a_raw read and q, k, v, beta, log a
-// written, once each; the conv taps' per-thread loads (eight 16-byte loads
-// whose lanes sit 128 bytes apart) cost more L1 wavefronts than that traffic
-// takes in HBM time, so the kernel is L1-bound at d 64.
+// Layout of the work: one warp per (head, span of kSpan tokens).  Lane l
+// owns channels [l C, l C + C) of the head, C = D / 32 (2 at d 64, 4 at
+// d 128), so a warp's access to one (token, head) row of x_q, x_k, x_v, q, k,
+// v or log a is one contiguous, coalesced row.  The lane keeps its channels'
+// conv taps in registers and walks the span's tokens in order with the last
+// three raw rows of x_q, x_k and x_v in a register window, so every raw row
+// is read from memory once (plus a three-row halo per span); the window is
+// cleared at every sequence start.  Loads run kPref tokens ahead of the
+// arithmetic.  L2 norms are warp sums.  The HBM traffic is x_q, x_k, x_v,
+// beta_raw and a_raw read and q, k, v, beta, log a written, once each.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -31,116 +28,63 @@ namespace {
 
 constexpr int kThreads = 256;
 
-// Eight consecutive fp32 values from p (16-byte aligned).
-__device__ __forceinline__ void load8(const float* p, float* x) {
-    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
-    const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
-    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-}
+constexpr int kSpan = 32;          // tokens per warp
+constexpr int kPref = 4;           // tokens of loads in flight ahead of the arithmetic
 
-__device__ __forceinline__ void store8(float* p, const float* x) {
-    reinterpret_cast<float4*>(p)[0] = make_float4(x[0], x[1], x[2], x[3]);
-    reinterpret_cast<float4*>(p)[1] = make_float4(x[4], x[5], x[6], x[7]);
-}
-__device__ __forceinline__ void store8(__nv_bfloat16* p, const float* x) {
-    uint32_t w[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const __nv_bfloat162 b = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
-        w[i] = *reinterpret_cast<const uint32_t*>(&b);
-    }
-    *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
-}
-
-// First token of the sequence holding token t: cu[n] for the largest n with
-// cu[n] <= t (empty sequences share their start with the next one).
-__device__ __forceinline__ int64_t seq_start(const int32_t* __restrict__ cu, int n_seqs,
-                                             int64_t t) {
-    int lo = 0, hi = n_seqs - 1, found = 0;
-    while (lo <= hi) {
-        const int mid = (lo + hi) >> 1;
-        if ((int64_t)__ldg(cu + mid) <= t) { found = mid; lo = mid + 1; } else { hi = mid - 1; }
-    }
-    return __ldg(cu + found);
-}
-
-// Eight consecutive raw values of x_q / x_k / x_v, held as loaded (16 bytes
-// of bf16 or 32 bytes of fp32) until the conv uses them.
-template <typename T>
-struct Raw8;
-template <>
-struct Raw8<__nv_bfloat16> {
-    uint4 u;
-    __device__ __forceinline__ void load(const __nv_bfloat16* p) {
-        u = __ldg(reinterpret_cast<const uint4*>(p));
-    }
-    __device__ __forceinline__ void to_f32(float* x) const {
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
-            x[2 * i] = f.x;
-            x[2 * i + 1] = f.y;
-        }
+// C consecutive channels of one row, as loaded (bf16 or fp32).
+template <typename T, int C> struct RowC;
+template <> struct RowC<__nv_bfloat16, 2> {
+    uint32_t u;
+    __device__ __forceinline__ void load(const __nv_bfloat16* p) { u = __ldg(reinterpret_cast<const uint32_t*>(p)); }
+    __device__ __forceinline__ void get(float* x) const {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u));
+        x[0] = f.x; x[1] = f.y;
     }
 };
-template <>
-struct Raw8<float> {
-    float4 a, b;
-    __device__ __forceinline__ void load(const float* p) {
-        a = __ldg(reinterpret_cast<const float4*>(p));
-        b = __ldg(reinterpret_cast<const float4*>(p) + 1);
-    }
-    __device__ __forceinline__ void to_f32(float* x) const {
-        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-        x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+template <> struct RowC<__nv_bfloat16, 4> {
+    uint2 u;
+    __device__ __forceinline__ void load(const __nv_bfloat16* p) { u = __ldg(reinterpret_cast<const uint2*>(p)); }
+    __device__ __forceinline__ void get(float* x) const {
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+        x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
     }
 };
+template <> struct RowC<float, 2> {
+    float2 u;
+    __device__ __forceinline__ void load(const float* p) { u = __ldg(reinterpret_cast<const float2*>(p)); }
+    __device__ __forceinline__ void get(float* x) const { x[0] = u.x; x[1] = u.y; }
+};
+template <> struct RowC<float, 4> {
+    float4 u;
+    __device__ __forceinline__ void load(const float* p) { u = __ldg(reinterpret_cast<const float4*>(p)); }
+    __device__ __forceinline__ void get(float* x) const { x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w; }
+};
 
-// y[0..7] = sum over the taps j = 0..3 with t - 3 + j >= s of
-// w[c][j] * x[t - 3 + j][c], c = c0 .. c0 + 7 (w row-major [H D, 4]); r[j]
-// holds tap j's values (any row when the tap is before the sequence start).
-template <typename T, int D>
-__device__ __forceinline__ void conv4(const Raw8<T> (&r)[4], const float* __restrict__ w,
-                                      int64_t t, int64_t s, int h, int c0, float* y) {
-    float wt[8][4];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        const float4 f = __ldg(reinterpret_cast<const float4*>(w + ((size_t)h * D + c0 + e) * 4));
-        wt[e][0] = f.x; wt[e][1] = f.y; wt[e][2] = f.z; wt[e][3] = f.w;
-    }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) y[e] = 0.f;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        if (t - 3 + j >= s) {
-            float x[8];
-            r[j].to_f32(x);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) y[e] = fmaf(wt[e][j], x[e], y[e]);
-        }
-    }
+template <int C> __device__ __forceinline__ void storeC(float* p, const float* x);
+template <> __device__ __forceinline__ void storeC<2>(float* p, const float* x) {
+    *reinterpret_cast<float2*>(p) = make_float2(x[0], x[1]);
+}
+template <> __device__ __forceinline__ void storeC<4>(float* p, const float* x) {
+    *reinterpret_cast<float4*>(p) = make_float4(x[0], x[1], x[2], x[3]);
+}
+template <int C> __device__ __forceinline__ void storeC(__nv_bfloat16* p, const float* x);
+template <> __device__ __forceinline__ void storeC<2>(__nv_bfloat16* p, const float* x) {
+    const __nv_bfloat162 b = __floats2bfloat162_rn(x[0], x[1]);
+    *reinterpret_cast<__nv_bfloat162*>(p) = b;
+}
+template <> __device__ __forceinline__ void storeC<4>(__nv_bfloat16* p, const float* x) {
+    const __nv_bfloat162 a = __floats2bfloat162_rn(x[0], x[1]), b = __floats2bfloat162_rn(x[2], x[3]);
+    uint2 u;
+    u.x = *reinterpret_cast<const uint32_t*>(&a);
+    u.y = *reinterpret_cast<const uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(p) = u;
 }
 
-// Sum over the G = D / 8 lanes of this (token, head) group (G divides 32 and
-// groups are G-aligned, so xor offsets below G stay inside the group).
-template <int G>
-__device__ __forceinline__ float group_sum(float v) {
+__device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
-    for (int m = G / 2; m >= 1; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
+    for (int m = 16; m >= 1; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
     return v;
-}
-
-template <int G>
-__device__ __forceinline__ void l2_normalise(float* y) {
-    float ss = 0.f;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) ss = fmaf(y[e], y[e], ss);
-    ss = group_sum<G>(ss);
-    const float inv = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) y[e] *= inv;
 }
 
 __device__ __forceinline__ float log_sigmoid(float z) {
@@ -152,88 +96,162 @@ __device__ __forceinline__ float sigmoid(float z) {
     return z >= 0.f ? 1.0f / (1.0f + e) : e / (1.0f + e);
 }
 
-// Grid-stride over (token, head) units, warp-uniform: every lane of a warp
-// runs the same iterations; lanes past the end work on the last unit (so
-// every address is valid), join the shuffles and store nothing.  All global
-// loads of an iteration are issued before any of them is used.
+// Inputs of one token for one lane, as loaded.
+template <typename T, int C, bool SCALAR>
+struct TokenIn {
+    RowC<T, C> xq, xk, xv;
+    RowC<float, C> a;          // a_raw (per-channel gate)
+    float a_s, b;              // a_raw (scalar gate), beta_raw
+    __device__ __forceinline__ void load(const T* xq_, const T* xk_, const T* xv_,
+                                         const float* a_raw, const float* beta_raw, int64_t t,
+                                         int H, int h, int c0) {
+        const size_t off = ((size_t)t * H + h) * (C * 32) + c0;
+        xq.load(xq_ + off);
+        xk.load(xk_ + off);
+        xv.load(xv_ + off);
+        if (SCALAR) a_s = __ldg(a_raw + (size_t)t * H + h);
+        else a.load(a_raw + off);
+        b = __ldg(beta_raw + (size_t)t * H + h);
+    }
+};
+
+// Causal width-4 conv of one lane's channels with a window of the three
+// previous raw rows (w0 = oldest): y = w[0] x_{t-3} + w[1] x_{t-2} +
+// w[2] x_{t-1} + w[3] x_t, then the window advances.
+template <int C>
+__device__ __forceinline__ void conv_step(const float (&w)[C][4], float (&win)[3][C],
+                                          const float* x, float* y) {
+#pragma unroll
+    for (int e = 0; e < C; ++e) {
+        float acc = w[e][3] * x[e];
+        acc = fmaf(w[e][2], win[2][e], acc);
+        acc = fmaf(w[e][1], win[1][e], acc);
+        acc = fmaf(w[e][0], win[0][e], acc);
+        y[e] = acc;
+        win[0][e] = win[1][e];
+        win[1][e] = win[2][e];
+        win[2][e] = x[e];
+    }
+}
+
 template <typename T, int D, bool SCALAR>
-__global__ void __launch_bounds__(kThreads, 2)
-preprocess_kernel(int n_seqs, int H, int64_t units, const int32_t* __restrict__ cu,
+__global__ void __launch_bounds__(kThreads)
+preprocess_kernel(int n_seqs, int H, int64_t T_tot, int64_t n_units, const int32_t* __restrict__ cu,
                   const T* __restrict__ xq, const T* __restrict__ xk, const T* __restrict__ xv,
                   const float* __restrict__ wq, const float* __restrict__ wk,
                   const float* __restrict__ wv, const float* __restrict__ beta_raw,
                   const float* __restrict__ a_raw, const float* __restrict__ a_bias,
                   T* __restrict__ q, T* __restrict__ k, T* __restrict__ v,
                   float* __restrict__ beta, float* __restrict__ log_a) {
-    constexpr int G = D / 8;                   // threads per (token, head)
-    constexpr int kUnitsPerWarp = 32 / G;
+    constexpr int C = D / 32;                  // channels per lane
     const int lane = threadIdx.x & 31;
-    const int sub = lane % G;                  // channel group: channels 8 sub .. 8 sub + 7
-    const int c0 = 8 * sub;
-    const int64_t warp = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / 32;
-    const int64_t n_warps = (int64_t)gridDim.x * kThreads / 32;
-    for (int64_t base = warp * kUnitsPerWarp; base < units; base += n_warps * kUnitsPerWarp) {
-        const int64_t u0 = base + lane / G;
-        const bool valid = u0 < units;
-        const int64_t u = valid ? u0 : units - 1;
-        const int64_t t = u / H;
-        const int h = (int)(u - t * H);
-        const int64_t s = seq_start(cu, n_seqs, t);
+    const int64_t unit = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / 32;
+    if (unit >= n_units) return;               // whole warps leave together
+    const int h = (int)(unit % H);
+    const int64_t t0 = (unit / H) * kSpan;
+    const int64_t t1 = t0 + kSpan < T_tot ? t0 + kSpan : T_tot;
+    const int c0 = C * lane;
 
-        Raw8<T> rq[4], rk[4], rv[4];
+    // this lane's taps and gate bias
+    float tq[C][4], tk[C][4], tv[C][4], bias[C];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int64_t tt = (t - 3 + j >= s) ? t - 3 + j : t;   // a valid row either way
+    for (int e = 0; e < C; ++e) {
+        const size_t r = ((size_t)h * D + c0 + e) * 4;
+        const float4 fq = __ldg(reinterpret_cast<const float4*>(wq + r));
+        const float4 fk = __ldg(reinterpret_cast<const float4*>(wk + r));
+        const float4 fv = __ldg(reinterpret_cast<const float4*>(wv + r));
+        tq[e][0] = fq.x; tq[e][1] = fq.y; tq[e][2] = fq.z; tq[e][3] = fq.w;
+        tk[e][0] = fk.x; tk[e][1] = fk.y; tk[e][2] = fk.z; tk[e][3] = fk.w;
+        tv[e][0] = fv.x; tv[e][1] = fv.y; tv[e][2] = fv.z; tv[e][3] = fv.w;
+        bias[e] = SCALAR ? 0.f : __ldg(a_bias + (size_t)h * D + c0 + e);
+    }
+    const float bias_s = SCALAR ? __ldg(a_bias + h) : 0.f;
+
+    // the sequence holding t0: the largest n with cu[n] <= t0
+    int n = 0;
+    {
+        int lo = 0, hi = n_seqs - 1;
+        while (lo <= hi) {
+            const int mid = (lo + hi) >> 1;
+            if ((int64_t)__ldg(cu + mid) <= t0) { n = mid; lo = mid + 1; } else { hi = mid - 1; }
+        }
+    }
+    const int64_t s = __ldg(cu + n);
+    int64_t next = __ldg(cu + n + 1);          // start of the next sequence
+
+    // window: the three raw rows before t0 that belong to t0's sequence
+    float wq_[3][C], wk_[3][C], wv_[3][C];
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+        const int64_t tt = t0 - 3 + j;
+        if (tt >= s) {
+            RowC<T, C> a, b, c;
             const size_t off = ((size_t)tt * H + h) * D + c0;
-            rq[j].load(xq + off);
-            rk[j].load(xk + off);
-            rv[j].load(xv + off);
-        }
-        const size_t row = (size_t)u * D + c0;
-        float z[8];
-        if (SCALAR) {
-            z[0] = __ldg(a_raw + u) + __ldg(a_bias + h);
+            a.load(xq + off); b.load(xk + off); c.load(xv + off);
+            a.get(wq_[j]); b.get(wk_[j]); c.get(wv_[j]);
         } else {
-            float bz[8];
-            load8(a_raw + row, z);
-            load8(a_bias + (size_t)h * D + c0, bz);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) z[e] += bz[e];
+            for (int e = 0; e < C; ++e) wq_[j][e] = wk_[j][e] = wv_[j][e] = 0.f;
         }
-        const float br = __ldg(beta_raw + u);
+    }
 
-        float yq[8], yk[8], yv[8];
-        conv4<T, D>(rq, wq, t, s, h, c0, yq);
-        conv4<T, D>(rk, wk, t, s, h, c0, yk);
-        conv4<T, D>(rv, wv, t, s, h, c0, yv);
-        l2_normalise<G>(yq);
-        l2_normalise<G>(yk);
-        if (!valid) continue;
-        store8(q + row, yq);
-        store8(k + row, yk);
-        store8(v + row, yv);
-        if (SCALAR) {
-            if (sub == 0) log_a[u] = log_sigmoid(z[0]);
-        } else {
+    // loads kPref tokens ahead (ring of kPref slots, index t % kPref)
+    TokenIn<T, C, SCALAR> ring[kPref];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) z[e] = log_sigmoid(z[e]);
-            store8(log_a + row, z);
+    for (int i = 0; i < kPref; ++i)
+        if (t0 + i < t1) ring[i].load(xq, xk, xv, a_raw, beta_raw, t0 + i, H, h, c0);
+
+    for (int64_t tb = t0; tb < t1; tb += kPref) {
+#pragma unroll
+        for (int i = 0; i < kPref; ++i) {
+            const int64_t t = tb + i;
+            if (t >= t1) break;
+            const TokenIn<T, C, SCALAR> in = ring[i];
+            if (t + kPref < t1) ring[i].load(xq, xk, xv, a_raw, beta_raw, t + kPref, H, h, c0);
+            if (t == next) {                   // a sequence starts here: clear the window
+                while (n + 1 < n_seqs && (int64_t)__ldg(cu + n + 1) <= t) ++n;
+                next = __ldg(cu + n + 1);
+#pragma unroll
+                for (int j = 0; j < 3; ++j)
+#pragma unroll
+                    for (int e = 0; e < C; ++e) wq_[j][e] = wk_[j][e] = wv_[j][e] = 0.f;
+            }
+            float x[C], yq[C], yk[C], yv[C];
+            in.xq.get(x); conv_step<C>(tq, wq_, x, yq);
+            in.xk.get(x); conv_step<C>(tk, wk_, x, yk);
+            in.xv.get(x); conv_step<C>(tv, wv_, x, yv);
+            float sq = 0.f, sk = 0.f;
+#pragma unroll
+            for (int e = 0; e < C; ++e) { sq = fmaf(yq[e], yq[e], sq); sk = fmaf(yk[e], yk[e], sk); }
+            sq = warp_sum(sq);
+            sk = warp_sum(sk);
+            const float iq = 1.0f / fmaxf(sqrtf(sq), 1e-12f), ik = 1.0f / fmaxf(sqrtf(sk), 1e-12f);
+#pragma unroll
+            for (int e = 0; e < C; ++e) { yq[e] *= iq; yk[e] *= ik; }
+            const size_t row = ((size_t)t * H + h) * D + c0;
+            storeC<C>(q + row, yq);
+            storeC<C>(k + row, yk);
+            storeC<C>(v + row, yv);
+            if (SCALAR) {
+                if (lane == 0) log_a[(size_t)t * H + h] = log_sigmoid(in.a_s + bias_s);
+            } else {
+                float z[C];
+                in.a.get(z);
+#pragma unroll
+                for (int e = 0; e < C; ++e) z[e] = log_sigmoid(z[e] + bias[e]);
+                storeC<C>(log_a + row, z);
+            }
+            if (lane == 1) beta[(size_t)t * H + h] = sigmoid(in.b);
         }
-        if (sub == 0) beta[u] = sigmoid(br);
     }
 }
 
 template <typename T, int D>
 cudaError_t launch_typed(const gdr_preprocess_args& a, cudaStream_t st) {
-    const int64_t units = a.total_tokens * a.n_heads;
-    constexpr int G = D / 8;
-    const int64_t warps = (units * G + 31) / 32;
-    int64_t blocks = (warps + kThreads / 32 - 1) / (kThreads / 32);
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t cap = (int64_t)sms * 8;      // eight 256-thread CTAs per SM
-    if (blocks > cap) blocks = cap;
+    const int64_t spans = (a.total_tokens + kSpan - 1) / kSpan;
+    const int64_t n_units = spans * a.n_heads;             // one warp each
+    const int64_t blocks = (n_units + kThreads / 32 - 1) / (kThreads / 32);
+    if (blocks > (int64_t)INT32_MAX) return cudaErrorInvalidValue;
     const dim3 grid((unsigned)blocks);
     auto* xq = static_cast<const T*>(a.xq);
     auto* xk = static_cast<const T*>(a.xk);
@@ -243,12 +261,12 @@ cudaError_t launch_typed(const gdr_preprocess_args& a, cudaStream_t st) {
     auto* v = static_cast<T*>(a.v);
     if (a.scalar_decay)
         preprocess_kernel<T, D, true><<<grid, kThreads, 0, st>>>(
-            a.n_seqs, a.n_heads, units, a.cu_seqlens, xq, xk, xv, a.conv_q, a.conv_k, a.conv_v,
-            a.beta_raw, a.a_raw, a.a_bias, q, k, v, a.beta, a.log_a);
+            a.n_seqs, a.n_heads, a.total_tokens, n_units, a.cu_seqlens, xq, xk, xv, a.conv_q,
+            a.conv_k, a.conv_v, a.beta_raw, a.a_raw, a.a_bias, q, k, v, a.beta, a.log_a);
     else
         preprocess_kernel<T, D, false><<<grid, kThreads, 0, st>>>(
-            a.n_seqs, a.n_heads, units, a.cu_seqlens, xq, xk, xv, a.conv_q, a.conv_k, a.conv_v,
-            a.beta_raw, a.a_raw, a.a_bias, q, k, v, a.beta, a.log_a);
+            a.n_seqs, a.n_heads, a.total_tokens, n_units, a.cu_seqlens, xq, xk, xv, a.conv_q,
+            a.conv_k, a.conv_v, a.beta_raw, a.a_raw, a.a_bias, q, k, v, a.beta, a.log_a);
     return cudaGetLastError();
 }
 

@@ -142,8 +142,6 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
 #endif
     __shared__ uint32_t tmem_slot;
     __shared__ int64_t snap_base_s;
-    // epilogue: partial sums of squares of the output rows, [chunk parity][half][row]
-    __shared__ float ssq_s[L::kOut ? 2 * 2 * 64 : 1];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int sub = warp & 3, half = warp >> 2;
@@ -462,7 +460,10 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
 #pragma unroll
                     for (int e = 0; e < 8; ++e) ss = fmaf(ov[j + e], ov[j + e], ss);
                 }
-                float* ssq = ssq_s + (k & 1) * 128;
+                // [half][row] partial sums, in this stage's Qt part: the O MMA
+                // that read it has completed, and the stage is refilled only
+                // after a later barrier (shared memory is full at d 128)
+                float* ssq = reinterpret_cast<float*>(stage(st) + R.Qt);
                 if (oactive) ssq[half * 64 + orow] = ss;
                 pair_bar(sub);
                 const float tot = ss + (oactive ? ssq[(half ^ 1) * 64 + orow] : 0.f);

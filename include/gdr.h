@@ -372,6 +372,38 @@ typedef struct {
 gdr_status gdr_preprocess(const gdr_preprocess_args* args, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Prefill from raw projections: gdr_preprocess's input activations (width-4
+ * conv, L2 norm of q and k, beta = sigmoid(beta_raw), log a =
+ * log_sigmoid(a_raw + a_bias)) applied inside the prefill's first stage, so
+ * that q, k, v, beta and log a are never written to memory ("kda-graft",
+ * section "Идея и архитектура": the activations sit right before the
+ * recurrence).  The results equal gdr_preprocess followed by gdr_prefill up
+ * to the summation order of the L2 norms.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+    const void* xq;             /* device [T_tot, H, d] raw projections, bf16 */
+    const void* xk;             /* device [T_tot, H, d] */
+    const void* xv;             /* device [T_tot, H, d] */
+    const float* conv_q;        /* device [H d, 4] fp32 taps (row h d + c; tap 3 = current token) */
+    const float* conv_k;        /* device [H d, 4] */
+    const float* conv_v;        /* device [H d, 4] */
+    const float* beta_raw;      /* device [T_tot, H] */
+    const float* a_raw;         /* device [T_tot, H, d], or [T_tot, H] if args->scalar_decay */
+    const float* a_bias;        /* device [H, d], or [H] if args->scalar_decay */
+} gdr_projections;
+
+/*
+ * Enqueue a prefill whose inputs are raw projections.  `args` as for
+ * gdr_prefill, with its q, k, v, beta and log_a ignored (may be NULL);
+ * qkv_dtype must be GDR_BF16 and d_k == d_v (64 or 128), else
+ * GDR_ERR_UNSUPPORTED.  xq, xk, xv, the conv taps and (per-channel gate)
+ * a_raw and a_bias must be 16-byte aligned.  Outputs, workspace (same size as
+ * gdr_prefill's) and errors as for gdr_prefill.
+ */
+gdr_status gdr_prefill_from_projections(const gdr_prefill_args* args, const gdr_projections* proj,
+                                        void* stream);
+
+/* ------------------------------------------------------------------------
  * Speculative decoding with rollback ("Modele hybrydowe", section "Co stan
  * rekurencyjny zmienia przy serwowaniu", point 2: a KV cache drops rejected
  * draft tokens, but the recurrent state has already absorbed them, so the

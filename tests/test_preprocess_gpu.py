@@ -97,3 +97,54 @@ def test_preprocess_no_tokens_is_noop():
     d = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in inp.items()}
     out = gdr.preprocess(*(d[a] for a in ARGS))
     assert out["q"].shape == (0, 2, 64)
+
+
+def _fused_vs_chain(w, lengths, snap=0, init=False):
+    """The fused prefill from raw projections against (a) the oracle's prefill
+    of the oracle's activations (cast to bf16) at the prefill bound 2e-2 max
+    |ref|, and (b) the two-kernel chain preprocess -> prefill."""
+    gdr = _gdr()
+    inp = wl.make_preprocess_inputs(w, lengths=lengths)
+    d = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in inp.items()}
+    H, dd = w.n_heads, w.d_k
+    n = len(inp["lengths"])
+    init_state = (0.1 * torch.randn(n, H, dd, dd, generator=torch.Generator().manual_seed(5))
+                  if init else None)
+    ini = None if init_state is None else init_state.cuda()
+    kw = dict(scalar_decay=w.scalar_decay, init_state=ini, snap_interval=snap,
+              cu_seqlens_host=inp["cu_seqlens"])
+    o, fin, snaps = gdr.prefill_from_projections(*(d[a] for a in ARGS), **kw)
+    act = gdr.preprocess(*(d[a] for a in ARGS), scalar_decay=w.scalar_decay)
+    o2, fin2, snaps2 = gdr.prefill(act["q"], act["k"], act["v"], act["beta"], act["log_a"],
+                                   d["cu_seqlens"], **kw)
+    torch.cuda.synchronize()
+    ref_act = oracle.preprocess(*(inp[a] for a in ARGS), scalar_decay=w.scalar_decay)
+    cast = {m: torch.from_numpy(ref_act[m]).to(torch.bfloat16) for m in ("q", "k", "v")}
+    ref = oracle.prefill(cast["q"], cast["k"], cast["v"], ref_act["beta"], ref_act["log_a"],
+                         inp["cu_seqlens"], scalar_decay=w.scalar_decay, init_state=init_state,
+                         snap_interval=snap)
+    pairs = [("o", o, ref["o"]), ("final_state", fin, ref["final_state"])]
+    if snap:
+        pairs.append(("snapshots", snaps, ref["snapshots"]))
+    for name, x, r in pairs:
+        err = np.abs(x.double().cpu().numpy() - r).max() / np.abs(r).max()
+        assert err <= 2e-2, f"fused {name}: {err:.3e}"
+    # the chain of two kernels computes the same (up to the norms' summation order)
+    for name, x, y in (("o", o, o2), ("final_state", fin, fin2)):
+        err = (x.double() - y.double()).abs().max().item() / y.double().abs().max().item()
+        assert err <= 2e-2, f"fused vs chain {name}: {err:.3e}"
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("scalar", [False, True])
+def test_fused_prefill_from_projections(d, scalar):
+    """Ragged sequences (1, 2, 3 tokens, empty, chunk-crossing lengths),
+    initial states and snapshots: the conv's history restarts at each
+    sequence start, including inside a chunk, and crosses chunk boundaries."""
+    w = wl.shrink(wl.PREPROCESS, n_heads=3, d_k=d, d_v=d, scalar_decay=scalar, seed=1110)
+    _fused_vs_chain(w, [1, 2, 3, 0, 130, 64, 200, 5], snap=64, init=True)
+
+
+def test_fused_prefill_graft_layer_shape():
+    """The graft layer's shape (8192 tokens x 14 heads x 64), one sequence."""
+    _fused_vs_chain(wl.PREPROCESS, None)
