@@ -664,26 +664,51 @@ def bench_epilogue(gdr, ps, stream, ms_plain, n):
 
 
 def bench_offload(gdr, ps, stream, ms_plain, n):
-    """The same prefill with its snapshots written by the state-pass kernel
-    straight into pinned host memory (no device copy, no copy stream)."""
-    runs = []
-    for s_ in ps.sets:
-        inp, p = s_["inp"], s_["prep"]
-        host = torch.empty(tuple(p.snapshots.shape), dtype=torch.float32).pin_memory()
-        runs.append((host, gdr.PreparedPrefill(
+    """The same prefill with its snapshots offloaded to pinned host memory:
+    (a) written by the state-pass kernel straight into host memory; (b) written
+    to device memory and copied on a second stream while the next prefill runs
+    (two device snapshot buffers alternate, so a prefill never overwrites a
+    buffer being copied)."""
+    s0 = ps.sets[0]
+    inp, p = s0["inp"], s0["prep"]
+    shape = tuple(p.snapshots.shape)
+    hosts = [torch.empty(shape, dtype=torch.float32).pin_memory() for _ in range(2)]
+
+    def prepared(snaps):
+        return gdr.PreparedPrefill(
             inp["q"], inp["k"], inp["v"], inp["beta"], inp["log_a"], inp["cu_seqlens"],
             out=p.out, final_state=p.final_state, workspace=p.workspace,
             scalar_decay=ps.w.scalar_decay, scale=ps.w.scale, init_state=inp["init_state"],
-            snap_interval=ps.w.snap_interval, snapshots=host)))
+            snap_interval=ps.w.snap_interval, snapshots=snaps)
+
+    direct = [prepared(h) for h in hosts]
+    devs = [p.snapshots, torch.empty_like(p.snapshots)]
+    viadev = [prepared(d_) for d_ in devs]
+    copy_stream = torch.cuda.Stream()
+    events = [torch.cuda.Event() for _ in range(2)]
+
+    def run_direct(i):
+        direct[i % 2].run()
+
+    def run_copy(i):
+        viadev[i % 2].run()
+        gdr.snapshot_offload(devs[i % 2], hosts[i % 2], copy_stream, events[i % 2], stream)
+
     for i in range(2):
-        runs[i % len(runs)][1].run()
-    ms = timed(lambda i: runs[i % len(runs)][1].run(), n, stream)
+        run_direct(i)
+        run_copy(i)
+    ms_direct = timed(run_direct, n, stream)
     torch.cuda.synchronize()
-    same = bool(torch.equal(runs[0][0], ps.sets[0]["prep"].snapshots.cpu())) if len(runs) == 1 else None
-    nbytes = runs[0][0].numel() * 4
-    return {"ms_per_step": round(ms, 4), "device_snapshots_ms_per_step": round(ms_plain, 4),
-            "overhead_frac": round(ms / ms_plain - 1.0, 4), "host_bytes_per_step": nbytes,
-            "bitwise_equal_to_device_snapshots": same}
+    ms_copy = timed(run_copy, n, stream)
+    torch.cuda.synchronize()
+    same = bool(torch.equal(hosts[(n - 1) % 2], devs[(n - 1) % 2].cpu()))
+    nbytes = hosts[0].numel() * 4
+    return {"device_snapshots_ms_per_step": round(ms_plain, 4), "host_bytes_per_step": nbytes,
+            "copy_stream": {"ms_per_step": round(ms_copy, 4),
+                            "overhead_frac": round(ms_copy / ms_plain - 1.0, 4),
+                            "host_copy_equals_device": same},
+            "direct_host_stores": {"ms_per_step": round(ms_direct, 4),
+                                   "overhead_frac": round(ms_direct / ms_plain - 1.0, 4)}}
 
 
 def bench_decode(gdr, stream, pk, args):

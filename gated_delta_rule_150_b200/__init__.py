@@ -22,7 +22,7 @@ import torch
 __all__ = ["PrefillArgs", "PreparedPrefill", "prefill", "kernel_count", "decode_step",
            "decode_draft", "decode_accept", "PreprocessArgs", "preprocess", "Projections",
            "prefill_from_projections", "cumdecay", "chunk_factors", "workspace_size",
-           "snapshot_count", "snapshot_offsets", "prefill_status", "lib", "GdrError", "LIB_PATH"]
+           "snapshot_count", "snapshot_offsets", "snapshot_offload", "prefill_status", "lib", "GdrError", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_build", "libgdr.so")
 
@@ -103,6 +103,8 @@ def lib():
             L.gdr_snapshot_count.argtypes = [vp, i, i]
             L.gdr_snapshot_offsets.restype = i
             L.gdr_snapshot_offsets.argtypes = [vp, i, i, vp]
+            L.gdr_snapshot_offload.restype = i
+            L.gdr_snapshot_offload.argtypes = [vp, vp, ctypes.c_size_t, vp, vp, vp]
             L.gdr_prefill_static_workspace.restype = i
             L.gdr_prefill_static_workspace.argtypes = [ctypes.POINTER(PrefillArgs), vp]
             L.gdr_prefill_static_status.restype = i
@@ -672,3 +674,25 @@ def prefill_from_projections(xq, xk, xv, conv_q, conv_k, conv_v, beta_raw, a_raw
     _check(lib().gdr_prefill_from_projections(ctypes.byref(a), ctypes.byref(p), _stream(dev)),
            "gdr_prefill_from_projections")
     return out, final_state, snapshots
+
+
+def snapshot_offload(dev_snapshots, host_snapshots, copy_stream, event, compute_stream=None):
+    """Copy the snapshots a prefill wrote (device) into pinned host memory on
+    ``copy_stream`` (a torch.cuda.Stream), after the work enqueued so far on
+    ``compute_stream`` (default: the current stream), ordered by ``event``
+    (a torch.cuda.Event).  Later prefills on compute_stream do not wait."""
+    if not dev_snapshots.is_cuda or not host_snapshots.is_pinned():
+        raise ValueError("dev_snapshots must be a CUDA tensor and host_snapshots pinned host memory")
+    if dev_snapshots.numel() != host_snapshots.numel() or dev_snapshots.dtype != torch.float32 or \
+            host_snapshots.dtype != torch.float32:
+        raise ValueError("snapshot buffers must be float32 of equal size")
+    if not dev_snapshots.is_contiguous() or not host_snapshots.is_contiguous():
+        raise ValueError("snapshot buffers must be contiguous")
+    cs = compute_stream if compute_stream is not None else torch.cuda.current_stream(dev_snapshots.device)
+    if not event.cuda_event:            # torch creates the event on its first record
+        event.record(cs)
+    _check(lib().gdr_snapshot_offload(_ptr(dev_snapshots), _ptr(host_snapshots),
+                                      dev_snapshots.numel() * 4, ctypes.c_void_p(cs.cuda_stream),
+                                      ctypes.c_void_p(copy_stream.cuda_stream),
+                                      ctypes.c_void_p(event.cuda_event)),
+           "gdr_snapshot_offload")

@@ -264,6 +264,22 @@ gdr_status gdr_prefill(const gdr_prefill_args* a, void* stream) {
     return gdr_prefill_stages(a, 0, 1, stream);
 }
 
+gdr_status gdr_snapshot_offload(const float* dev_snapshots, float* host_snapshots, size_t bytes,
+                                void* compute_stream, void* copy_stream, void* event) {
+    if (!event || compute_stream == copy_stream) return GDR_ERR_INVALID_ARG;
+    if (bytes > 0 && (!dev_snapshots || !host_snapshots || !aligned16(dev_snapshots) ||
+                      !aligned16(host_snapshots)))
+        return GDR_ERR_INVALID_ARG;
+    cudaEvent_t ev = static_cast<cudaEvent_t>(event);
+    cudaStream_t cs = static_cast<cudaStream_t>(compute_stream);
+    cudaStream_t xs = static_cast<cudaStream_t>(copy_stream);
+    gdr_status s = from_cuda(cudaEventRecord(ev, cs));
+    if (s != GDR_OK || bytes == 0) return s;
+    s = from_cuda(cudaStreamWaitEvent(xs, ev, 0));
+    if (s != GDR_OK) return s;
+    return from_cuda(cudaMemcpyAsync(host_snapshots, dev_snapshots, bytes, cudaMemcpyDeviceToHost, xs));
+}
+
 gdr_status gdr_prefill_status(const void* workspace, void* stream) {
     if (!workspace) return GDR_ERR_INVALID_ARG;
     uint32_t word = 0;

@@ -98,10 +98,9 @@ struct IntraLayout {
     static constexpr uint32_t op_bytes = SCALAR ? 256u * D : 576u * D;
     static constexpr uint32_t As = r1;                        // fp32 [64][kLd]
     static constexpr uint32_t Pt = As + 64u * kLd * 4u;       // bf16 [64][64]
-    static constexpr uint32_t Tb = Pt + 8192u;                // bf16 [64][64] (d 128)
-    static constexpr uint32_t Yt = Tb + 8192u;                // fp32 [32][32] scratch (d 128)
-    // d 64 applies (I + A)^-1 by substitution on B: no T tile, no scratch
-    static constexpr uint32_t solve_bytes = 64u * kLd * 4u + (D == 64 ? 8192u : 16384u + 4096u);
+    static constexpr uint32_t Tb = Pt + 8192u;                // bf16 [64][64]
+    static constexpr uint32_t Yt = Tb + 8192u;                // fp32 [32][32] scratch
+    static constexpr uint32_t solve_bytes = 64u * kLd * 4u + 16384u + 4096u;
     static constexpr uint32_t Rec = r1;                       // record staging
     static constexpr uint32_t rec_bytes = record_layout(D).bytes;
     static constexpr uint32_t r2 = al1024(umax(umax(op_bytes, solve_bytes),
@@ -119,11 +118,13 @@ struct IntraLayout {
     // solve, without partials), when nothing else is in region 2
     static constexpr uint32_t kPtotBytes = 4u * threads_for<D, SCALAR>();
     static constexpr uint32_t Ptot = r1;
-    // raw projections (fused input activations): the three rows before the
-    // chunk of x_q, x_k, x_v, each [3][D] (zeros before the sequence start)
-    static constexpr uint32_t Halo = Gs + 256u;
-    static constexpr uint32_t halo_bytes = RAW ? 3u * 3u * D * elem : 0u;
-    static constexpr uint32_t bytes = Halo + halo_bytes;
+    // raw projections (fused input activations): the three raw rows before
+    // the chunk of x_q, x_k, x_v, [3 tensors][3 rows][D]; fetched at the item
+    // start into the solve's scratch Yt (free until the solve; outside the
+    // record staging) at d 64, past everything else at d 128
+    static constexpr uint32_t halo_bytes = RAW ? 9u * D * elem : 0u;
+    static constexpr uint32_t Halo = (D == 64) ? Yt : Gs + 256u;
+    static constexpr uint32_t bytes = Gs + 256u + ((RAW && D != 64) ? halo_bytes : 0u);
     // at d 128 the 512 TMEM columns of a CTA allow one CTA per SM: request
     // enough shared memory that a second one is never scheduled
     static constexpr uint32_t dyn_bytes = (D == 128) ? umax(bytes + 1024u, 118784u) : bytes + 1024u;
@@ -133,6 +134,8 @@ struct IntraLayout {
     static_assert(dyn_bytes <= 232448u, "shared memory budget");
     static_assert(kPtotBytes <= r2, "scan partials fit in region 2");
     static_assert(!RAW || kStageQKV, "raw projections are staged");
+    static_assert(D != 64 || !RAW || (Yt + halo_bytes <= r1 + r2 && Yt >= Rec + rec_bytes),
+                  "halo fits in the solve scratch, outside the record staging");
     static_assert((64u * kLd * 4u) % 1024u == 0u, "Pt alignment");
     static_assert(Rec + rec_bytes <= Qgs, "record staging stays below Qgs");
     // TMEM is allocated once per persistent CTA: never more CTAs on an SM
@@ -147,13 +150,19 @@ __host__ __device__ constexpr uint32_t ap_col(int b) { return (uint32_t)(8 * b *
 
 template <typename T> struct Vec8;
 template <> struct Vec8<__nv_bfloat16> {
-    static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&x)[8]) {
-        const uint4 u = *reinterpret_cast<const uint4*>(p);
+    static __device__ __forceinline__ void load_reg(const uint4 u, float (&x)[8]) {
         float2 a = unpack_bf16(u.x), b = unpack_bf16(u.y), c = unpack_bf16(u.z), d = unpack_bf16(u.w);
         x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y; x[4] = c.x; x[5] = c.y; x[6] = d.x; x[7] = d.y;
     }
+    static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&x)[8]) {
+        load_reg(*reinterpret_cast<const uint4*>(p), x);
+    }
 };
 template <> struct Vec8<float> {
+    static __device__ __forceinline__ void load_reg(const uint4, float (&x)[8]) {   // not used for fp32
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = 0.f;
+    }
     static __device__ __forceinline__ void load(const float* p, float (&x)[8]) {
         const float4 a = *reinterpret_cast<const float4*>(p);
         const float4 b = *reinterpret_cast<const float4*>(p + 4);
@@ -256,8 +265,8 @@ __device__ __forceinline__ bool scan_channels(float* sG, int len, int t,
     const int part = (P == 1) ? 0 : (t & 1);
     bool bad = false;
     float run = 0.f;
-#pragma unroll 4
     const float bc = RAW ? __ldg(bias + c) : 0.f;
+#pragma unroll 4
     for (int r = part * RP; r < (part + 1) * RP; ++r) {
         // raw projections: log a = log_sigmoid(a_raw + bias) on the fly
         const float la = r < len ? (RAW ? log_sigmoid_f(sG[r * D + c] + bc) : sG[r * D + c]) : 0.f;
@@ -328,8 +337,7 @@ template <int D, typename InT, bool SCALAR, bool RAW, typename L>
 __device__ __forceinline__ void issue_inputs(uint8_t* sm, uint64_t* bar_g, uint64_t* bar_qkv,
                                              const InputMaps& maps, const float* __restrict__ beta,
                                              const float* __restrict__ log_a, int H, const Item& it,
-                                             int lane, bool hint, const InT* __restrict__ xq,
-                                             const InT* __restrict__ xk, const InT* __restrict__ xv) {
+                                             int lane, bool hint) {
     if (lane == 0) {
         const int x = it.h * D;
         const uint64_t pol = l2_policy_evict_first();             // inputs are read once
@@ -355,62 +363,7 @@ __device__ __forceinline__ void issue_inputs(uint8_t* sm, uint64_t* bar_g, uint6
         cp_async4(sm + L::Bs + 4 * t, beta + o, n);
         if (SCALAR) cp_async4(sm + L::Gs + 4 * t, log_a + o, n);
     }
-    if (RAW) {
-        // the three raw rows before the chunk, zeros before the sequence start
-        constexpr int kPer = D * (int)sizeof(InT) / 16;           // 16-byte pieces per row
-        for (int i = lane; i < 3 * 3 * kPer; i += 32) {
-            const int tsr = i / (3 * kPer), j = (i / kPer) % 3, piece = i % kPer;
-            const int tok = it.start - 3 + j;
-            const InT* src = tsr == 0 ? xq : (tsr == 1 ? xk : xv);
-            const bool in = tok >= it.sstart;
-            const size_t off = ((size_t)(in ? tok : it.start) * H + it.h) * D;
-            cp_async16(sm + L::Halo + ((tsr * 3 + j) * D) * sizeof(InT) + 16 * piece,
-                       reinterpret_cast<const uint8_t*>(src + off) + 16 * piece, in ? 16u : 0u);
-        }
-    }
     cp_async_commit();
-}
-
-// [W | U] = (I + A)^-1 B, one column at a time (d 64: 2D = 128 columns, one
-// per thread of warps 0-3), by forward substitution in fp32:
-//     x_r = b_r - sum_{i<r} A[r, i] x_i,        r = 1 .. 63,
-// where column c of B = [diag(beta)(K * Gamma) | diag(beta) V] is row c of the
-// bf16 tile Bt.  A (fp32, zero on and above the diagonal, row stride kLd) is
-// read as float4 rows that every lane shares (broadcast); the column stays in
-// registers.  No barrier is needed (each thread owns its column), and the
-// result overwrites row c of Bt as row c of the bf16 tile [W | U]^T.  This is
-// the same T = (I + A)^-1 the blocked solve forms, applied to B directly and
-// without rounding T to bf16 first.
-template <int D>
-__device__ __forceinline__ void substitute_column(const float* __restrict__ As, uint8_t* Bt, int c) {
-    float x[64];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const uint4 u = *reinterpret_cast<const uint4*>(Bt + sw128_chunk(2 * D, c, j));
-        const float2 a = unpack_bf16(u.x), b = unpack_bf16(u.y), e = unpack_bf16(u.z), f = unpack_bf16(u.w);
-        x[8 * j + 0] = a.x; x[8 * j + 1] = a.y; x[8 * j + 2] = b.x; x[8 * j + 3] = b.y;
-        x[8 * j + 4] = e.x; x[8 * j + 5] = e.y; x[8 * j + 6] = f.x; x[8 * j + 7] = f.y;
-    }
-#pragma unroll
-    for (int r = 1; r < 64; ++r) {
-        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-        for (int i4 = 0; i4 < (r + 3) / 4; ++i4) {
-            const float4 a = *reinterpret_cast<const float4*>(As + r * kLd + 4 * i4);
-            a0 = fmaf(a.x, x[4 * i4 + 0], a0);
-            a1 = fmaf(a.y, x[4 * i4 + 1], a1);
-            a2 = fmaf(a.z, x[4 * i4 + 2], a2);
-            a3 = fmaf(a.w, x[4 * i4 + 3], a3);
-        }
-        x[r] -= (a0 + a1) + (a2 + a3);
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        float y[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) y[e] = x[8 * j + e];
-        *reinterpret_cast<uint4*>(Bt + sw128_chunk(2 * D, c, j)) = pack8(y);
-    }
 }
 
 // Read the A/P products of this thread's row from TMEM (per-channel decay).
@@ -507,7 +460,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     uint32_t in_issued = 0, mma_commits = 0;
     if (cur.idx >= 0 && warp == kLoadWarp) {
         issue_inputs<D, InT, SCALAR, RAW, L>(sm, &in_bar[0], &in_bar[1], maps, beta, log_a, H, cur,
-                                             lane, keep_records != 0, q, k, v);
+                                             lane, keep_records != 0);
         ++in_issued;
     }
     const uint32_t tmem = tmem_slot;
@@ -526,6 +479,27 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     const int h = cur.h, start = cur.start, len = cur.len;
     uint8_t* rec = records + (size_t)cur.idx * R.bytes;       // item = slot * H + h
     const size_t base = (size_t)start * tok_stride + (size_t)h * D;
+
+    // raw projections: the first row group fetches the three raw rows before
+    // the chunk (x_q, x_k, x_v; zeros before the sequence start) by cp.async
+    // now, so that the copies are in flight during the waits below
+    if constexpr (RAW) {
+        if (tid < CG) {
+#pragma unroll
+            for (int j = 0; j < 3; ++j) {
+                const int tok = start - 3 + j;
+                const bool in = tok >= cur.sstart;
+                const size_t off = ((size_t)(in ? tok : start) * H + h) * D + 8 * tid;
+#pragma unroll
+                for (int tsr = 0; tsr < 3; ++tsr) {
+                    const InT* src = tsr == 0 ? q : (tsr == 1 ? k : v);
+                    cp_async16(sm + L::Halo + ((size_t)(tsr * 3 + j) * D + 8 * tid) * sizeof(InT), src + off,
+                               in ? 16u : 0u);
+                }
+            }
+            cp_async_commit();
+        }
+    }
 
     // ---- this item's log a and beta have landed --------------------------------
     {
@@ -627,6 +601,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         const bool ok = !L::kStageQKV || mbar_wait(&in_bar[1], in_phase);
         in_phase ^= 1u;
         if (tid == 0) bulk_wait_group_read0();
+        if (RAW && tid < CG) cp_async_wait_all();      // the halo rows
         failed = __syncthreads_or(!ok);
         if (failed) {
             if (tid == 0) atomicOr(err, 1u);
@@ -643,11 +618,10 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     // and channels it builds the operands from below.
     if constexpr (RAW) {
         if (tid < len) Bs[tid] = sigmoid_f(Bs[tid]);
-        float y[3][RPT][8];
+        uint4 y[3][RPT];                      // activated rows, as bf16 (how they are stored)
 #pragma unroll
         for (int tsr = 0; tsr < 3; ++tsr) {
             const InT* stg = reinterpret_cast<const InT*>(sm + (tsr == 0 ? L::sQ : (tsr == 1 ? L::sK : L::sV)));
-            const InT* hal = reinterpret_cast<const InT*>(sm + L::Halo) + tsr * 3 * D;
             const float* wsrc = tsr == 0 ? rp.wq : (tsr == 1 ? rp.wk : rp.wv);
             float w[8][4];
 #pragma unroll
@@ -662,27 +636,30 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const int rr = r - 3 + j;
+                    const InT* hal = reinterpret_cast<const InT*>(sm + L::Halo) + (size_t)tsr * 3 * D;
                     Vec8<InT>::load(rr >= 0 ? stg + (size_t)rr * D + c0 : hal + (size_t)(rr + 3) * D + c0, x[j]);
                 }
+                float yy[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     float acc = w[e][3] * x[3][e];
                     acc = fmaf(w[e][2], x[2][e], acc);
                     acc = fmaf(w[e][1], x[1][e], acc);
                     acc = fmaf(w[e][0], x[0][e], acc);
-                    y[tsr][u][e] = acc;
+                    yy[e] = acc;
                 }
                 if (tsr < 2) {
                     // L2 norm over the row's D channels: CG consecutive lanes
                     float ss = 0.f;
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) ss = fmaf(y[tsr][u][e], y[tsr][u][e], ss);
+                    for (int e = 0; e < 8; ++e) ss = fmaf(yy[e], yy[e], ss);
 #pragma unroll
                     for (int m = 1; m < CG; m <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
                     const float inv = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) y[tsr][u][e] *= inv;
+                    for (int e = 0; e < 8; ++e) yy[e] *= inv;
                 }
+                y[tsr][u] = pack8(yy);
             }
         }
         __syncthreads();                      // every raw row has been read
@@ -691,19 +668,13 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
             uint8_t* stg = sm + (tsr == 0 ? L::sQ : (tsr == 1 ? L::sK : L::sV));
 #pragma unroll
             for (int u = 0; u < RPT; ++u)
-                *reinterpret_cast<uint4*>(stg + ((size_t)(r0 + u) * D + c0) * sizeof(InT)) = pack8(y[tsr][u]);
+                *reinterpret_cast<uint4*>(stg + ((size_t)(r0 + u) * D + c0) * sizeof(InT)) = y[tsr][u];
         }
         // the operand passes below read only this thread's rows and channels;
         // beta and other threads' rows are read after the next barrier
     }
 
-    // ---- operands -------------------------------------------------------------
-    // Pass 1 builds what the A/P products read (scaled query and key rows, the
-    // key tiles); their MMA is issued at once, and pass 2 builds the operands
-    // of the later products (Qg and the transposed diag(beta)(K Gamma),
-    // diag(beta) V and Kd) while it runs.  Pass 2 recomputes the row factors
-    // (the same values: the operations are the same), which is cheaper than
-    // keeping them live across the MMA issue.
+    // ---- operands and per-token outputs -------------------------------------
     uint8_t* XA = sm + L::XA;
     uint8_t* Bt = sm + L::Bt;
     uint8_t* Kdt = sm + L::Kdt;
@@ -713,22 +684,26 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
 #pragma unroll
         for (int e = 0; e < 8; ++e) { em[e] = __expf(mj[e]); eld[e] = __expf(gl[e] - mj[e]); }
     }
-    // this thread's row r of q, k (and v): staged, from global, or zeros past the end
-    auto load_row = [&](int r, bool valid, float (&qv)[8], float (&kv)[8], float (&vv)[8], bool with_v) {
+    uint32_t pb1[8][RPT / 2], pb2[8][RPT / 2], pkd[8][RPT / 2];   // transposed bf16 pairs
+    float p_b1[8], p_bv[8], p_kd[8];                               // even row of the pair
+#pragma unroll
+    for (int u = 0; u < RPT; ++u) {
+        const int r = r0 + u;
+        const bool valid = r < len;
+        float qv[8], kv[8], vv[8], gr[8];
+        const float br = Bs[r];
         if (valid && L::kStageQKV) {
             Vec8<InT>::load(reinterpret_cast<const InT*>(sm + L::sQ) + (size_t)r * D + c0, qv);
             Vec8<InT>::load(reinterpret_cast<const InT*>(sm + L::sK) + (size_t)r * D + c0, kv);
-            if (with_v) Vec8<InT>::load(reinterpret_cast<const InT*>(sm + L::sV) + (size_t)r * D + c0, vv);
+            Vec8<InT>::load(reinterpret_cast<const InT*>(sm + L::sV) + (size_t)r * D + c0, vv);
         } else if (valid) {
             Vec8<InT>::load(q + base + (size_t)r * tok_stride + c0, qv);
             Vec8<InT>::load(k + base + (size_t)r * tok_stride + c0, kv);
-            if (with_v) Vec8<InT>::load(v + base + (size_t)r * tok_stride + c0, vv);
+            Vec8<InT>::load(v + base + (size_t)r * tok_stride + c0, vv);
         } else {
 #pragma unroll
             for (int e = 0; e < 8; ++e) qv[e] = kv[e] = vv[e] = 0.f;
         }
-    };
-    auto load_g = [&](int r, bool valid, float (&gr)[8]) {
         if (!SCALAR) {
             if (valid) load8f(sG + (size_t)r * D + c0, gr);
             else {
@@ -739,16 +714,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
 #pragma unroll
             for (int e = 0; e < 8; ++e) gr[e] = Gs[r];
         }
-    };
-    // pass 1: A-side operand rows r (queries) and 64 + r (keys), key tiles
-#pragma unroll
-    for (int u = 0; u < RPT; ++u) {
-        const int r = r0 + u;
-        const bool valid = r < len;
-        float qv[8], kv[8], vv[8], gr[8];
-        load_row(r, valid, qv, kv, vv, false);
-        load_g(r, valid, gr);
-        float xq[8], xk[8], kk0[8];
+        float xq[8], xk[8], kk0[8], b1[8], qg[8], kd[8];
         if (!SCALAR && !bad_chunk) {
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
@@ -757,14 +723,34 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                 xq[e] = scale * qv[e] * F;
                 xk[e] = kv[e] * F;
                 kk0[e] = kv[e] * Fi;
+                b1[e] = br * xk[e] * em[e];
+                qg[e] = xq[e] * em[e];
+                kd[e] = kk0[e] * eld[e];
             }
         } else if (SCALAR) {
+            const float G = __expf(gr[0]), Ed = __expf(gl[0] - gr[0]);   // one gate per row
 #pragma unroll
-            for (int e = 0; e < 8; ++e) { xq[e] = scale * qv[e]; xk[e] = kv[e]; kk0[e] = 0.f; }
+            for (int e = 0; e < 8; ++e) {
+                xq[e] = scale * qv[e];
+                xk[e] = kv[e];
+                kk0[e] = 0.f;
+                b1[e] = br * kv[e] * G;
+                qg[e] = scale * qv[e] * G;
+                kd[e] = kv[e] * Ed;
+            }
         } else {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) xq[e] = xk[e] = kk0[e] = 0.f;
+            for (int e = 0; e < 8; ++e) {
+                const float G = __expf(gr[e]);
+                xq[e] = 0.f;
+                xk[e] = 0.f;
+                kk0[e] = 0.f;
+                b1[e] = br * kv[e] * G;
+                qg[e] = scale * qv[e] * G;
+                kd[e] = kv[e] * __expf(gl[e] - gr[e]);
+            }
         }
+        // A-side operand rows r (queries) and 64 + r (keys)
         *reinterpret_cast<uint4*>(XA + sw128_chunk(128, r, cg)) = pack8(xq);
         *reinterpret_cast<uint4*>(XA + sw128_chunk(128, 64 + r, cg)) = pack8(xk);
         if (!SCALAR) {
@@ -776,74 +762,6 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
 #pragma unroll
                 for (int e = 0; e < 8; ++e) kb[e] = (b == jb) ? kk0[e] : kk0[e] * ecross[b][e];
                 *reinterpret_cast<uint4*>(sm + L::kt_off(b) + sw128_chunk(16 * (b + 1), r, cg)) = pack8(kb);
-            }
-        }
-    }
-    fence_proxy_async_smem();
-    tc_fence_before_sync();
-    __syncthreads();
-    tc_fence_after_sync();
-
-    // ---- decay-weighted Q K^T and K K^T on the tensor cores ------------------
-    if (tid == 0) {
-        const uint32_t aXA = smem_u32(XA);
-        if (!SCALAR) {
-#pragma unroll
-            for (int b = 0; b < 4; ++b) {
-                const uint32_t id = idesc_bf16_f32(128, 16 * (b + 1));
-                const uint32_t aK = smem_u32(sm + L::kt_off(b));
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    mma_bf16(tmem + ap_col(b), sw128_desc(aXA, 128, 0, 16 * kk),
-                             sw128_desc(aK, 16 * (b + 1), 0, 16 * kk), id, kk > 0);
-            }
-        } else {
-            const uint32_t id = idesc_bf16_f32(128, 64);
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk)
-                mma_bf16(tmem, sw128_desc(aXA, 128, 0, 16 * kk), sw128_desc(aXA, 128, 64, 16 * kk), id, kk > 0);
-        }
-        mma_commit(&mma_bar);
-        ++mma_commits;
-    }
-
-    // ---- pass 2, under the A/P MMA: Qg rows, transposed B1, B2, Kd ------------
-    uint32_t pb1[8][RPT / 2], pb2[8][RPT / 2], pkd[8][RPT / 2];   // transposed bf16 pairs
-    float p_b1[8], p_bv[8], p_kd[8];                               // even row of the pair
-#pragma unroll
-    for (int u = 0; u < RPT; ++u) {
-        const int r = r0 + u;
-        const bool valid = r < len;
-        float qv[8], kv[8], vv[8], gr[8];
-        const float br = Bs[r];
-        load_row(r, valid, qv, kv, vv, true);
-        load_g(r, valid, gr);
-        float b1[8], qg[8], kd[8];
-        if (!SCALAR && !bad_chunk) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float d = gr[e] - mj[e];
-                const float F = __expf(d), Fi = __expf(-d);
-                const float xq = scale * qv[e] * F, xk = kv[e] * F, kk0 = kv[e] * Fi;
-                b1[e] = br * xk * em[e];
-                qg[e] = xq * em[e];
-                kd[e] = kk0 * eld[e];
-            }
-        } else if (SCALAR) {
-            const float G = __expf(gr[0]), Ed = __expf(gl[0] - gr[0]);   // one gate per row
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                b1[e] = br * kv[e] * G;
-                qg[e] = scale * qv[e] * G;
-                kd[e] = kv[e] * Ed;
-            }
-        } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float G = __expf(gr[e]);
-                b1[e] = br * kv[e] * G;
-                qg[e] = scale * qv[e] * G;
-                kd[e] = kv[e] * __expf(gl[e] - gr[e]);
             }
         }
         *reinterpret_cast<uint4*>(Qgs + sw128_chunk(64, r, cg)) = pack8(qg);
@@ -885,7 +803,33 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
             *reinterpret_cast<uint32_t*>(Kdt + o3) = pkd[e][0];
         }
     }
-    fence_proxy_async_smem();         // read by later MMAs, after the next barrier
+    fence_proxy_async_smem();
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+
+    // ---- decay-weighted Q K^T and K K^T on the tensor cores ------------------
+    if (tid == 0) {
+        const uint32_t aXA = smem_u32(XA);
+        if (!SCALAR) {
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const uint32_t id = idesc_bf16_f32(128, 16 * (b + 1));
+                const uint32_t aK = smem_u32(sm + L::kt_off(b));
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_bf16(tmem + ap_col(b), sw128_desc(aXA, 128, 0, 16 * kk),
+                             sw128_desc(aK, 16 * (b + 1), 0, 16 * kk), id, kk > 0);
+            }
+        } else {
+            const uint32_t id = idesc_bf16_f32(128, 64);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+                mma_bf16(tmem, sw128_desc(aXA, 128, 0, 16 * kk), sw128_desc(aXA, 128, 64, 16 * kk), id, kk > 0);
+        }
+        mma_commit(&mma_bar);
+        ++mma_commits;
+    }
     failed = !mbar_wait(&mma_bar, phase);
     phase ^= 1u;
     tc_fence_after_sync();
@@ -981,28 +925,22 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         fence_proxy_async_smem();             // this item's reads of region 1 come first
         if (nxt.idx >= 0) {
             issue_inputs<D, InT, SCALAR, RAW, L>(sm, &in_bar[0], &in_bar[1], maps, beta, log_a, H, nxt,
-                                                 lane, keep_records != 0, q, k, v);
+                                                 lane, keep_records != 0);
             ++in_issued;
         }
         if (lane == 0)
             s_item[iter & 1] = nxt.idx >= 0 ? find_item(cu, n_seqs, H, n_items, nxt.idx + gridDim.x) : nxt;
     }
 
-    // ---- [W | U] = (I + A)^-1 B ------------------------------------------------
-    // d 64: forward substitution on the 128 columns of B (substitute_column),
-    // straight into the tile [W | U]^T.  d 128: T = (I + A)^-1 by the blocked
-    // solve below (16x16 diagonal blocks, then block merges), then one MMA.
+    // ---- T = (I + A)^-1: 16x16 diagonal blocks, then block merges -----------
     // T overwrites A in As block by block, each block once the phases that
     // still read it have passed a barrier.  Every phase also writes its bf16
     // copy straight into the operand tile Tb, whose blocks above the
     // diagonal are zeroed here.
     // Warps 0-3 solve (named barrier 1); warps 4-7 meanwhile scan the next
     // item's log a, which the loader warp has just requested.
-    constexpr bool kSubst = (D == 64);
     uint8_t* Tb = sm + L::Tb;
-    if (kSubst && tid < 2 * D) {
-        substitute_column<D>(As, Bt, tid);
-    } else if (!kSubst && tid < 128) {
+    if (tid < 128) {
         if (tid >= 64) {
             // (row, chunk) pairs of the zero blocks (b, j > b): 96 + 64 + 32
 #pragma unroll
@@ -1089,8 +1027,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     failed = __syncthreads_or(failed);
     tc_fence_after_sync();
 
-    // ---- [W | U]^T = [diag(b)(K*Gamma) | diag(b)V]^T T^T (d 128) -------------
-    if constexpr (!kSubst) {
+    // ---- [W | U]^T = [diag(b)(K*Gamma) | diag(b)V]^T T^T ---------------------
     if (tid == 0 && !failed) {
         const uint32_t id = idesc_bf16_f32(128, 64);
         const uint32_t aB = smem_u32(Bt), aT = smem_u32(sm + L::Tb);
@@ -1101,6 +1038,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                 mma_bf16(tmem + 64 * half, sw128_desc(aB, 2 * D, 128 * half, 16 * kk),
                          sw128_desc(aT, 64, 0, 16 * kk), id, kk > 0);
         mma_commit(&mma_bar);
+        ++mma_commits;
         ++mma_commits;
     }
     if (!failed && !mbar_wait(&mma_bar, phase)) failed = true;
@@ -1136,7 +1074,6 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     tc_fence_before_sync();
     failed = __syncthreads_or(failed);
     tc_fence_after_sync();
-    }
 
     // ---- P [W | U], Kd^T W, U^T Kd --------------------------------------------
     if (tid == 0 && !failed) {

@@ -113,7 +113,9 @@ struct PassLayout {
     static_assert(dyn_bytes + 128u <= 232448u, "shared memory budget");
 };
 
-template <int D, typename OutT, int MODE>
+// GATED: the output epilogue is applied (og.gate is set); a template
+// parameter so that the plain kernels keep their register allocation.
+template <int D, typename OutT, int MODE, bool GATED>
 __global__ void __launch_bounds__(kThreads, (D == 64) ? 2 : 1)
 state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                   const uint8_t* __restrict__ records, const float* init_state,
@@ -321,10 +323,22 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     }
     int mmas_waited = 0;
 
+    // output epilogue with bf16 outputs: this chunk's raw gate values are
+    // loaded at the top of its iteration, so that the loads complete during
+    // the waits and the state update instead of on the output path
+    constexpr bool kGatePre = GATED && kOut && sizeof(OutT) == 2;
+    constexpr int kGateVec = kGatePre ? CW / 8 : 1;
     for (int k = 0; k < nchunks; ++k) {
         const int st = k % ST;
         const int t0 = s0 + k * kChunk;
         const int len = min(kChunk, s1 - t0);
+        uint4 gpre[kGateVec];
+        if (kGatePre && GATED && oactive && orow < len && cb < dv) {
+            const uint4* g = reinterpret_cast<const uint4*>(static_cast<const OutT*>(og.gate) +
+                                                            ((size_t)(t0 + orow) * H + h) * dv + cb);
+#pragma unroll
+            for (int i = 0; i < kGateVec; ++i) gpre[i] = __ldg(g + i);
+        }
         if (!mbar_wait(&full[st], (uint32_t)(k / ST) & 1)) failed = true;
 #ifdef GDR_TEST_WAIT_LIMIT_NS
         if (k == 1 && !mbar_wait_for(&never_bar, 0u, (uint64_t)GDR_TEST_WAIT_LIMIT_NS)) failed = true;
@@ -445,7 +459,7 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
             }
             const uint8_t* pu = stage(st) + R.PU;
             OutT* orow_ptr = o + ((size_t)(t0 + orow) * H + h) * dv + cb;
-            if (og.gate) {
+            if (GATED) {
                 // o = Qt S0^T + PU in place, then the row's RMS: the two halves
                 // of a row (warps w and w + 4, same lane) swap their partial sums
                 // of squares through shared memory behind a barrier of the pair
@@ -474,7 +488,15 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                     for (int j = 0; j < CW; j += 8) {
                         if (cb + j >= dv) continue;
                         float gv[8], wv[8], x[8];
-                        In8<OutT>::load(g + j, gv);
+                        if (kGatePre) {
+                            const uint4 u = gpre[j / 8];
+                            const float2 a = unpack_bf16(u.x), b = unpack_bf16(u.y);
+                            const float2 c = unpack_bf16(u.z), d = unpack_bf16(u.w);
+                            gv[0] = a.x; gv[1] = a.y; gv[2] = b.x; gv[3] = b.y;
+                            gv[4] = c.x; gv[5] = c.y; gv[6] = d.x; gv[7] = d.y;
+                        } else {
+                            In8<OutT>::load(g + j, gv);
+                        }
                         In8<float>::load(og.weight + cb + j, wv);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
@@ -720,10 +742,10 @@ combine_kernel(const int32_t* __restrict__ cu, int H, int seg_chunks, const floa
     cp_async_wait_all();
 }
 
-template <int D, typename OutT, int MODE>
-cudaError_t launch_mode(const gdr_prefill_args& a, const uint8_t* records,
-                        const WorkspaceLayout& lay, float* seg_ws, uint32_t* err, cudaStream_t st) {
-    auto kern = state_pass_kernel<D, OutT, MODE>;
+template <int D, typename OutT, int MODE, bool GATED>
+cudaError_t launch_gated(const gdr_prefill_args& a, const uint8_t* records,
+                         const WorkspaceLayout& lay, float* seg_ws, uint32_t* err, cudaStream_t st) {
+    auto kern = state_pass_kernel<D, OutT, MODE, GATED>;
     const uint32_t smem = PassLayout<D, MODE>::dyn_bytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -737,6 +759,16 @@ cudaError_t launch_mode(const gdr_prefill_args& a, const uint8_t* records,
                       a.snap_interval, a.snapshots, a.snap_offsets, lay.seg_chunks, seg_ws, err,
                       records_fit_l2(lay.n_slots, a.n_heads, D) ? 1 : 0,
                       OutputGate{a.gate_raw, a.norm_weight, a.norm_eps}, a.d_k, a.d_v);
+}
+
+template <int D, typename OutT, int MODE>
+cudaError_t launch_mode(const gdr_prefill_args& a, const uint8_t* records,
+                        const WorkspaceLayout& lay, float* seg_ws, uint32_t* err, cudaStream_t st) {
+    // the zero-state pass writes no outputs: never gated
+    if constexpr (MODE != kLocal) {
+        if (a.gate_raw) return launch_gated<D, OutT, MODE, true>(a, records, lay, seg_ws, err, st);
+    }
+    return launch_gated<D, OutT, MODE, false>(a, records, lay, seg_ws, err, st);
 }
 
 template <int D, typename OutT>

@@ -244,3 +244,12 @@ def test_snapshot_offsets_reject_bad_arguments(L):
 def test_prefill_rejects_misaligned_snapshot_offsets(L):
     pre = lambda a: L.gdr_prefill(ctypes.byref(a), None)
     assert pre(_args(snap_interval=128, snapshots=0x90000, snap_offsets=0xA0004)) == 1
+
+
+def test_snapshot_offload_rejects_bad_arguments(L):
+    f = lambda d, h, n, cs, xs, ev: L.gdr_snapshot_offload(d, h, n, cs, xs, ev)
+    d, h, ev = _fake(1), _fake(2), _fake(3)
+    assert f(d, h, 1024, _fake(4), _fake(5), None) == 1          # no event
+    assert f(d, h, 1024, _fake(4), _fake(4), ev) == 1            # same stream
+    assert f(None, h, 1024, _fake(4), _fake(5), ev) == 1
+    assert f(ctypes.c_void_p(0x10008), h, 1024, _fake(4), _fake(5), ev) == 1
