@@ -144,7 +144,7 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
             if (lane16 != p) continue;             // pass p's row is stored by lane p
             const int row = rgrp + kRowsPerPass * p;
             const float g = to_f<T>(og.gate[(size_t)bh * DV + row]);
-            const float sig = 1.f / (1.f + __expf(-g));
+            const float sig = __fdividef(1.f, 1.f + __expf(-g));
             o[(size_t)bh * DV + row] = ov[p] * rstd * __ldg(og.weight + row) * sig;
         }
     }

@@ -118,13 +118,15 @@ struct IntraLayout {
     // solve, without partials), when nothing else is in region 2
     static constexpr uint32_t kPtotBytes = 4u * threads_for<D, SCALAR>();
     static constexpr uint32_t Ptot = r1;
-    // raw projections (fused input activations): the three raw rows before
-    // the chunk of x_q, x_k, x_v, [3 tensors][3 rows][D]; fetched at the item
-    // start into the solve's scratch Yt (free until the solve; outside the
-    // record staging) at d 64, past everything else at d 128
+    // raw projections (fused input activations): the item's conv taps
+    // [3 tensors][D][4] fp32 and the three raw rows before the chunk of x_q,
+    // x_k, x_v [3][3][D], fetched at the item start into the Qg tile (dead
+    // from the previous item's map MMAs on, outside its record staging, and
+    // written only by this item's operand build, after their last use)
+    static constexpr uint32_t Taps = Qgs;
+    static constexpr uint32_t Halo = Taps + 3u * D * 16u;
     static constexpr uint32_t halo_bytes = RAW ? 9u * D * elem : 0u;
-    static constexpr uint32_t Halo = (D == 64) ? Yt : Gs + 256u;
-    static constexpr uint32_t bytes = Gs + 256u + ((RAW && D != 64) ? halo_bytes : 0u);
+    static constexpr uint32_t bytes = Gs + 256u;
     // at d 128 the 512 TMEM columns of a CTA allow one CTA per SM: request
     // enough shared memory that a second one is never scheduled
     static constexpr uint32_t dyn_bytes = (D == 128) ? umax(bytes + 1024u, 118784u) : bytes + 1024u;
@@ -134,8 +136,8 @@ struct IntraLayout {
     static_assert(dyn_bytes <= 232448u, "shared memory budget");
     static_assert(kPtotBytes <= r2, "scan partials fit in region 2");
     static_assert(!RAW || kStageQKV, "raw projections are staged");
-    static_assert(D != 64 || !RAW || (Yt + halo_bytes <= r1 + r2 && Yt >= Rec + rec_bytes),
-                  "halo fits in the solve scratch, outside the record staging");
+    static_assert(!RAW || (Halo + halo_bytes <= Qgs + 128u * D && Taps >= Rec + rec_bytes),
+                  "taps and halo fit in the Qg tile, outside the record staging");
     static_assert((64u * kLd * 4u) % 1024u == 0u, "Pt alignment");
     static_assert(Rec + rec_bytes <= Qgs, "record staging stays below Qgs");
     // TMEM is allocated once per persistent CTA: never more CTAs on an SM
@@ -480,10 +482,16 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     uint8_t* rec = records + (size_t)cur.idx * R.bytes;       // item = slot * H + h
     const size_t base = (size_t)start * tok_stride + (size_t)h * D;
 
-    // raw projections: the first row group fetches the three raw rows before
-    // the chunk (x_q, x_k, x_v; zeros before the sequence start) by cp.async
-    // now, so that the copies are in flight during the waits below
+    // raw projections: the CTA fetches this head's conv taps and the first row
+    // group the three raw rows before the chunk (x_q, x_k, x_v; zeros before
+    // the sequence start) by cp.async now, so that the copies are in flight
+    // during the waits below
     if constexpr (RAW) {
+        for (int i = tid; i < 3 * D; i += NT) {
+            const int tsr = i / D, c = i % D;
+            const float* wsrc = tsr == 0 ? rp.wq : (tsr == 1 ? rp.wk : rp.wv);
+            cp_async16(sm + L::Taps + 16u * i, wsrc + ((size_t)h * D + c) * 4, 16u);
+        }
         if (tid < CG) {
 #pragma unroll
             for (int j = 0; j < 3; ++j) {
@@ -497,8 +505,8 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                                in ? 16u : 0u);
                 }
             }
-            cp_async_commit();
         }
+        cp_async_commit();
     }
 
     // ---- this item's log a and beta have landed --------------------------------
@@ -601,7 +609,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         const bool ok = !L::kStageQKV || mbar_wait(&in_bar[1], in_phase);
         in_phase ^= 1u;
         if (tid == 0) bulk_wait_group_read0();
-        if (RAW && tid < CG) cp_async_wait_all();      // the halo rows
+        if (RAW) cp_async_wait_all();                  // taps and halo rows
         failed = __syncthreads_or(!ok);
         if (failed) {
             if (tid == 0) atomicOr(err, 1u);
@@ -622,11 +630,11 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
 #pragma unroll
         for (int tsr = 0; tsr < 3; ++tsr) {
             const InT* stg = reinterpret_cast<const InT*>(sm + (tsr == 0 ? L::sQ : (tsr == 1 ? L::sK : L::sV)));
-            const float* wsrc = tsr == 0 ? rp.wq : (tsr == 1 ? rp.wk : rp.wv);
+            const float* wsm = reinterpret_cast<const float*>(sm + L::Taps) + ((size_t)tsr * D + c0) * 4;
             float w[8][4];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                const float4 f = __ldg(reinterpret_cast<const float4*>(wsrc + ((size_t)h * D + c0 + e) * 4));
+                const float4 f = *reinterpret_cast<const float4*>(wsm + 4 * e);
                 w[e][0] = f.x; w[e][1] = f.y; w[e][2] = f.z; w[e][3] = f.w;
             }
 #pragma unroll

@@ -500,7 +500,7 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                         In8<float>::load(og.weight + cb + j, wv);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
-                            const float sig = 1.f / (1.f + __expf(-gv[e]));
+                            const float sig = __fdividef(1.f, 1.f + __expf(-gv[e]));
                             x[e] = ov[j + e] * rstd * wv[e] * sig;
                         }
                         Out8<OutT>::store(orow_ptr + j, x);
