@@ -211,12 +211,15 @@ class NvmlClockSampler:
         self._stop.set()
         self.thread.join(timeout=5)
         inside = [r for r in self.rows if t0 <= r[0] <= t1]
-        if not inside:
+        # a timed region shorter than the sampling interval: the samples
+        # nearest to it
+        window = inside or sorted(self.rows, key=lambda r: abs(r[0] - t0))[:3]
+        if not window:
             return None
-        reasons = sorted({n for r in inside for n, bit in self.REASONS if r[2] & bit})
-        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": self.max_mhz,
-                "reasons": reasons, "samples_inside_timed_region": len(inside),
-                "source": "nvml, every ~2 ms"}
+        reasons = sorted({n for r in window for n, bit in self.REASONS if r[2] & bit})
+        return {"sm_mhz": statistics.median(r[1] for r in window), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(window),
+                "samples_inside_timed_region": len(inside), "source": "nvml, every ~2 ms"}
 
 
 # ---------------------------------------------------------------------------
@@ -541,9 +544,9 @@ def run_gdr(args):
     torch.cuda.synchronize()
     t_wall1, t_perf1 = datetime.datetime.now(), time.perf_counter()
     barrier(world)
-    clocks = nvml.stop(t_perf0, t_perf1) or sampler.stop(t_wall0, t_wall1)
-    if nvml.ok:
-        sampler.stop(t_wall0, t_wall1)
+    clocks_nvml = nvml.stop(t_perf0, t_perf1)
+    clocks_smi = sampler.stop(t_wall0, t_wall1)
+    clocks = clocks_nvml or clocks_smi
     ms_local = start.elapsed_time(end)
     ms_total = max_over_ranks(ms_local, world)
     ms_step = ms_total / args.steps

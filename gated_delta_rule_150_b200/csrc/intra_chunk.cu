@@ -119,7 +119,7 @@ struct IntraLayout {
     static constexpr uint32_t kPtotBytes = 4u * threads_for<D, SCALAR>();
     static constexpr uint32_t Ptot = r1;
     // raw projections (fused input activations): the item's conv taps
-    // [3 tensors][D][4] fp32 and the three raw rows before the chunk of x_q,
+    // [3 tensors][4 taps][D] fp32 and the three raw rows before the chunk of x_q,
     // x_k, x_v [3][3][D], fetched at the item start into the Qg tile (dead
     // from the previous item's map MMAs on, outside its record staging, and
     // written only by this item's operand build, after their last use)
@@ -284,6 +284,38 @@ __device__ __forceinline__ bool scan_channels(float* sG, int len, int t,
         }
     }
     return bad;
+}
+
+// Reference points of this thread's channels c0 .. c0 + 7: g_last, the
+// midpoint m_jb of its 16-row block and exp(m_b - m_jb) for later blocks b
+// (per-channel decay; with a scalar decay g_last only); g_last also goes to Gl.
+template <int D, bool SCALAR>
+__device__ __forceinline__ void reference_points(const float* sG, const float* Gs, float* Gl,
+                                                 int len, int jb, int c0, int rg, int tid,
+                                                 float (&gl)[8], float (&mj)[8],
+                                                 float (&ecross)[4][8]) {
+    if (!SCALAR) {
+        load8f(sG + (size_t)(len - 1) * D + c0, gl);
+        load8f(sG + (size_t)min(16 * jb + 8, len - 1) * D + c0, mj);
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            if (b > jb) {
+                float mb[8];
+                load8f(sG + (size_t)min(16 * b + 8, len - 1) * D + c0, mb);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) ecross[b][e] = __expf(mb[e] - mj[e]);
+            }
+        }
+        if (rg == 0) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) Gl[c0 + e] = gl[e];
+        }
+    } else {
+        const float glast = Gs[len - 1];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) gl[e] = glast;
+        if (tid < D) Gl[tid] = glast;
+    }
 }
 
 // One unit of work: chunk slot idx / H of head idx % H (idx < 0: none).
@@ -486,11 +518,17 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     // group the three raw rows before the chunk (x_q, x_k, x_v; zeros before
     // the sequence start) by cp.async now, so that the copies are in flight
     // during the waits below
+    constexpr int kTapsPer = RAW ? (3 * 4 * D + NT - 1) / NT : 1;
+    float taps[kTapsPer];                     // this thread's share, stored tap-major below
     if constexpr (RAW) {
-        for (int i = tid; i < 3 * D; i += NT) {
-            const int tsr = i / D, c = i % D;
-            const float* wsrc = tsr == 0 ? rp.wq : (tsr == 1 ? rp.wk : rp.wv);
-            cp_async16(sm + L::Taps + 16u * i, wsrc + ((size_t)h * D + c) * 4, 16u);
+#pragma unroll
+        for (int u = 0; u < kTapsPer; ++u) {
+            const int i = tid + u * NT;
+            if (i < 3 * 4 * D) {
+                const int tsr = i / (4 * D), j = (i / D) % 4, c = i % D;
+                const float* wsrc = tsr == 0 ? rp.wq : (tsr == 1 ? rp.wk : rp.wv);
+                taps[u] = __ldg(wsrc + ((size_t)h * D + c) * 4 + j);
+            }
         }
         if (tid < CG) {
 #pragma unroll
@@ -579,37 +617,23 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     const int jb = r0 / 16;                                   // this thread's 16-row block
 
     // ---- reference points: g_last, block midpoints m_b -------------------------
+    // (with raw projections computed after the input activations, so that
+    // these registers are not live through them)
     float gl[8], mj[8];
     float ecross[4][8];                       // exp(m_b - m_jb) for b > jb (per-channel)
-    if (!SCALAR) {
-        load8f(sG + (size_t)(len - 1) * D + c0, gl);
-        load8f(sG + (size_t)min(16 * jb + 8, len - 1) * D + c0, mj);
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            if (b > jb) {
-                float mb[8];
-                load8f(sG + (size_t)min(16 * b + 8, len - 1) * D + c0, mb);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) ecross[b][e] = __expf(mb[e] - mj[e]);
-            }
-        }
-        if (rg == 0) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) Gl[c0 + e] = gl[e];
-        }
-    } else {
-        const float glast = Gs[len - 1];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) gl[e] = glast;
-        if (tid < D) Gl[tid] = glast;
-    }
+    if (!RAW) reference_points<D, SCALAR>(sG, Gs, Gl, len, jb, c0, rg, tid, gl, mj, ecross);
     // q, k, v have landed and the previous record's bulk store has finished
     // reading the region the operands go to
     {
         const bool ok = !L::kStageQKV || mbar_wait(&in_bar[1], in_phase);
         in_phase ^= 1u;
         if (tid == 0) bulk_wait_group_read0();
-        if (RAW) cp_async_wait_all();                  // taps and halo rows
+        if constexpr (RAW) {
+            cp_async_wait_all();                       // the halo rows
+#pragma unroll
+            for (int u = 0; u < kTapsPer; ++u)         // the taps, tap-major
+                if (tid + u * NT < 3 * 4 * D) reinterpret_cast<float*>(sm + L::Taps)[tid + u * NT] = taps[u];
+        }
         failed = __syncthreads_or(!ok);
         if (failed) {
             if (tid == 0) atomicOr(err, 1u);
@@ -630,12 +654,14 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
 #pragma unroll
         for (int tsr = 0; tsr < 3; ++tsr) {
             const InT* stg = reinterpret_cast<const InT*>(sm + (tsr == 0 ? L::sQ : (tsr == 1 ? L::sK : L::sV)));
-            const float* wsm = reinterpret_cast<const float*>(sm + L::Taps) + ((size_t)tsr * D + c0) * 4;
+            const float* wsm = reinterpret_cast<const float*>(sm + L::Taps) + (size_t)tsr * 4 * D + c0;
             float w[8][4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float4 f = *reinterpret_cast<const float4*>(wsm + 4 * e);
-                w[e][0] = f.x; w[e][1] = f.y; w[e][2] = f.z; w[e][3] = f.w;
+            for (int j = 0; j < 4; ++j) {
+                float t8[8];
+                load8f(wsm + (size_t)j * D, t8);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) w[e][j] = t8[e];
             }
 #pragma unroll
             for (int u = 0; u < RPT; ++u) {
@@ -680,6 +706,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         }
         // the operand passes below read only this thread's rows and channels;
         // beta and other threads' rows are read after the next barrier
+        reference_points<D, SCALAR>(sG, Gs, Gl, len, jb, c0, rg, tid, gl, mj, ecross);
     }
 
     // ---- operands and per-token outputs -------------------------------------

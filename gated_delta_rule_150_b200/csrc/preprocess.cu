@@ -9,83 +9,40 @@
 // k normalised per (token, head) after it as y / max(||y||, 1e-12), the conv
 // restarting from zero history at every sequence start.
 //
-// Layout of the work: one warp per (head, span of kSpan tokens).  Lane l
-// owns channels [l C, l C + C) of the head, C = D / 32 (2 at d 64, 4 at
-// d 128), so a warp's access to one (token, head) row of x_q, x_k, x_v, q, k,
-// v or log a is one contiguous, coalesced row.  The lane keeps its channels'
-// conv taps in registers and walks the span's tokens in order with the last
-// three raw rows of x_q, x_k and x_v in a register window, so every raw row
-// is read from memory once (plus a three-row halo per span); the window is
-// cleared at every sequence start.  Loads run kPref tokens ahead of the
-// arithmetic.  L2 norms are warp sums.  The HBM traffic is x_q, x_k, x_v,
-// beta_raw and a_raw read and q, k, v, beta, log a written, once each.
+// Layout of the work: one CTA per (head, block of kTok tokens).  It first
+// stages, by 16-byte cp.async from every thread, the raw rows of x_q, x_k and
+// x_v for tokens [t0 - 3, t0 + kTok) (the three before the block for the
+// conv), the block's a_raw rows, beta_raw and the head's conv taps and gate
+// bias: about 45 KB per CTA at d 64, all in flight at once, so the kernel
+// keeps enough bytes moving to stream at HBM speed.  Then D / 8 threads own
+// a token (eight channels each) and compute its outputs from shared memory;
+// a tap that reaches before the token's sequence start is skipped.  L2 norms
+// are shuffle sums over the token's D / 8 lanes.  Outputs go straight to
+// global memory, each token row written by D / 8 neighbouring threads.  HBM
+// traffic: x_q, x_k, x_v, beta_raw and a_raw read (plus a three-row halo per
+// block), q, k, v, beta and log a written.
 #include <cuda_bf16.h>
 
 #include "internal.h"
+#include "sm100.cuh"
 
 namespace gdr {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kTok = 64;            // tokens per CTA
 
-constexpr int kSpan = 32;          // tokens per warp
-constexpr int kPref = 4;           // tokens of loads in flight ahead of the arithmetic
-
-// C consecutive channels of one row, as loaded (bf16 or fp32).
-template <typename T, int C> struct RowC;
-template <> struct RowC<__nv_bfloat16, 2> {
-    uint32_t u;
-    __device__ __forceinline__ void load(const __nv_bfloat16* p) { u = __ldg(reinterpret_cast<const uint32_t*>(p)); }
-    __device__ __forceinline__ void get(float* x) const {
-        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u));
-        x[0] = f.x; x[1] = f.y;
-    }
+template <typename T, int D, bool SCALAR>
+struct PreLayout {
+    static constexpr uint32_t kRows = kTok + 3;                    // staged raw rows
+    static constexpr uint32_t X = 0;                               // [3][kRows][D] raw x
+    static constexpr uint32_t A = X + 3u * kRows * D * sizeof(T);  // [kTok][D] a_raw (or [kTok])
+    static constexpr uint32_t a_bytes = SCALAR ? 4u * kTok : 4u * kTok * D;
+    static constexpr uint32_t B = A + ((a_bytes + 15u) & ~15u);    // [kTok] beta_raw
+    static constexpr uint32_t W = B + 4u * kTok;                   // [3][4][D] taps, tap-major
+    static constexpr uint32_t Bias = W + 3u * D * 16u;             // [D] (or [1]) gate bias
+    static constexpr uint32_t bytes = Bias + 4u * D;
 };
-template <> struct RowC<__nv_bfloat16, 4> {
-    uint2 u;
-    __device__ __forceinline__ void load(const __nv_bfloat16* p) { u = __ldg(reinterpret_cast<const uint2*>(p)); }
-    __device__ __forceinline__ void get(float* x) const {
-        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
-        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
-        x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
-    }
-};
-template <> struct RowC<float, 2> {
-    float2 u;
-    __device__ __forceinline__ void load(const float* p) { u = __ldg(reinterpret_cast<const float2*>(p)); }
-    __device__ __forceinline__ void get(float* x) const { x[0] = u.x; x[1] = u.y; }
-};
-template <> struct RowC<float, 4> {
-    float4 u;
-    __device__ __forceinline__ void load(const float* p) { u = __ldg(reinterpret_cast<const float4*>(p)); }
-    __device__ __forceinline__ void get(float* x) const { x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w; }
-};
-
-template <int C> __device__ __forceinline__ void storeC(float* p, const float* x);
-template <> __device__ __forceinline__ void storeC<2>(float* p, const float* x) {
-    *reinterpret_cast<float2*>(p) = make_float2(x[0], x[1]);
-}
-template <> __device__ __forceinline__ void storeC<4>(float* p, const float* x) {
-    *reinterpret_cast<float4*>(p) = make_float4(x[0], x[1], x[2], x[3]);
-}
-template <int C> __device__ __forceinline__ void storeC(__nv_bfloat16* p, const float* x);
-template <> __device__ __forceinline__ void storeC<2>(__nv_bfloat16* p, const float* x) {
-    const __nv_bfloat162 b = __floats2bfloat162_rn(x[0], x[1]);
-    *reinterpret_cast<__nv_bfloat162*>(p) = b;
-}
-template <> __device__ __forceinline__ void storeC<4>(__nv_bfloat16* p, const float* x) {
-    const __nv_bfloat162 a = __floats2bfloat162_rn(x[0], x[1]), b = __floats2bfloat162_rn(x[2], x[3]);
-    uint2 u;
-    u.x = *reinterpret_cast<const uint32_t*>(&a);
-    u.y = *reinterpret_cast<const uint32_t*>(&b);
-    *reinterpret_cast<uint2*>(p) = u;
-}
-
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
-    return v;
-}
 
 __device__ __forceinline__ float log_sigmoid(float z) {
     return fminf(z, 0.f) - log1pf(expf(-fabsf(z)));
@@ -96,178 +53,182 @@ __device__ __forceinline__ float sigmoid(float z) {
     return z >= 0.f ? 1.0f / (1.0f + e) : e / (1.0f + e);
 }
 
-// Inputs of one token for one lane, as loaded.
-template <typename T, int C, bool SCALAR>
-struct TokenIn {
-    RowC<T, C> xq, xk, xv;
-    RowC<float, C> a;          // a_raw (per-channel gate)
-    float a_s, b;              // a_raw (scalar gate), beta_raw
-    __device__ __forceinline__ void load(const T* xq_, const T* xk_, const T* xv_,
-                                         const float* a_raw, const float* beta_raw, int64_t t,
-                                         int H, int h, int c0) {
-        const size_t off = ((size_t)t * H + h) * (C * 32) + c0;
-        xq.load(xq_ + off);
-        xk.load(xk_ + off);
-        xv.load(xv_ + off);
-        if (SCALAR) a_s = __ldg(a_raw + (size_t)t * H + h);
-        else a.load(a_raw + off);
-        b = __ldg(beta_raw + (size_t)t * H + h);
+template <typename T> struct Vec8;
+template <> struct Vec8<__nv_bfloat16> {
+    static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&x)[8]) {
+        const uint4 u = *reinterpret_cast<const uint4*>(p);
+        const float2 a = unpack_bf16(u.x), b = unpack_bf16(u.y), c = unpack_bf16(u.z), d = unpack_bf16(u.w);
+        x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y; x[4] = c.x; x[5] = c.y; x[6] = d.x; x[7] = d.y;
+    }
+    static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&x)[8]) {
+        uint4 u;
+        u.x = pack_bf16(x[0], x[1]); u.y = pack_bf16(x[2], x[3]);
+        u.z = pack_bf16(x[4], x[5]); u.w = pack_bf16(x[6], x[7]);
+        *reinterpret_cast<uint4*>(p) = u;
+    }
+};
+template <> struct Vec8<float> {
+    static __device__ __forceinline__ void load(const float* p, float (&x)[8]) {
+        const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
+        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+    }
+    static __device__ __forceinline__ void store(float* p, const float (&x)[8]) {
+        *reinterpret_cast<float4*>(p) = make_float4(x[0], x[1], x[2], x[3]);
+        *reinterpret_cast<float4*>(p + 4) = make_float4(x[4], x[5], x[6], x[7]);
     }
 };
 
-// Causal width-4 conv of one lane's channels with a window of the three
-// previous raw rows (w0 = oldest): y = w[0] x_{t-3} + w[1] x_{t-2} +
-// w[2] x_{t-1} + w[3] x_t, then the window advances.
-template <int C>
-__device__ __forceinline__ void conv_step(const float (&w)[C][4], float (&win)[3][C],
-                                          const float* x, float* y) {
+// Sum over the G = D / 8 lanes of a token (G divides 32; groups are G-aligned).
+template <int G>
+__device__ __forceinline__ float group_sum(float v) {
 #pragma unroll
-    for (int e = 0; e < C; ++e) {
-        float acc = w[e][3] * x[e];
-        acc = fmaf(w[e][2], win[2][e], acc);
-        acc = fmaf(w[e][1], win[1][e], acc);
-        acc = fmaf(w[e][0], win[0][e], acc);
-        y[e] = acc;
-        win[0][e] = win[1][e];
-        win[1][e] = win[2][e];
-        win[2][e] = x[e];
-    }
+    for (int m = G / 2; m >= 1; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
+    return v;
 }
 
 template <typename T, int D, bool SCALAR>
 __global__ void __launch_bounds__(kThreads)
-preprocess_kernel(int n_seqs, int H, int64_t T_tot, int64_t n_units, const int32_t* __restrict__ cu,
+preprocess_kernel(int n_seqs, int H, int64_t T_tot, const int32_t* __restrict__ cu,
                   const T* __restrict__ xq, const T* __restrict__ xk, const T* __restrict__ xv,
                   const float* __restrict__ wq, const float* __restrict__ wk,
                   const float* __restrict__ wv, const float* __restrict__ beta_raw,
                   const float* __restrict__ a_raw, const float* __restrict__ a_bias,
                   T* __restrict__ q, T* __restrict__ k, T* __restrict__ v,
                   float* __restrict__ beta, float* __restrict__ log_a) {
-    constexpr int C = D / 32;                  // channels per lane
-    const int lane = threadIdx.x & 31;
-    const int64_t unit = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / 32;
-    if (unit >= n_units) return;               // whole warps leave together
-    const int h = (int)(unit % H);
-    const int64_t t0 = (unit / H) * kSpan;
-    const int64_t t1 = t0 + kSpan < T_tot ? t0 + kSpan : T_tot;
-    const int c0 = C * lane;
+    using L = PreLayout<T, D, SCALAR>;
+    constexpr int G = D / 8;                       // threads per token
+    constexpr int TPP = kThreads / G;              // tokens per pass
+    constexpr int kPer = D * (int)sizeof(T) / 16;  // 16-byte pieces per raw row
+    extern __shared__ __align__(16) uint8_t sm[];
+    const int tid = threadIdx.x;
+    const int h = blockIdx.y;
+    const int64_t t0 = (int64_t)blockIdx.x * kTok;
+    const int ntok = (int)(T_tot - t0 < kTok ? T_tot - t0 : kTok);
 
-    // this lane's taps and gate bias
-    float tq[C][4], tk[C][4], tv[C][4], bias[C];
-#pragma unroll
-    for (int e = 0; e < C; ++e) {
-        const size_t r = ((size_t)h * D + c0 + e) * 4;
-        const float4 fq = __ldg(reinterpret_cast<const float4*>(wq + r));
-        const float4 fk = __ldg(reinterpret_cast<const float4*>(wk + r));
-        const float4 fv = __ldg(reinterpret_cast<const float4*>(wv + r));
-        tq[e][0] = fq.x; tq[e][1] = fq.y; tq[e][2] = fq.z; tq[e][3] = fq.w;
-        tk[e][0] = fk.x; tk[e][1] = fk.y; tk[e][2] = fk.z; tk[e][3] = fk.w;
-        tv[e][0] = fv.x; tv[e][1] = fv.y; tv[e][2] = fv.z; tv[e][3] = fv.w;
-        bias[e] = SCALAR ? 0.f : __ldg(a_bias + (size_t)h * D + c0 + e);
+    // ---- stage everything the block reads -----------------------------------------
+    for (int i = tid; i < 3 * (kTok + 3) * kPer; i += kThreads) {
+        const int tsr = i / ((kTok + 3) * kPer), rem = i % ((kTok + 3) * kPer);
+        const int row = rem / kPer, piece = rem % kPer;
+        const int64_t tok = t0 - 3 + row;
+        const bool in = tok >= 0 && tok < T_tot;
+        const T* x = tsr == 0 ? xq : (tsr == 1 ? xk : xv);
+        const T* src = x + ((in ? tok : 0) * H + h) * (int64_t)D;
+        cp_async16(sm + L::X + ((size_t)(tsr * (kTok + 3) + row) * D) * sizeof(T) + 16 * piece,
+                   reinterpret_cast<const uint8_t*>(src) + 16 * piece, in ? 16u : 0u);
     }
-    const float bias_s = SCALAR ? __ldg(a_bias + h) : 0.f;
+    if (SCALAR) {
+        for (int i = tid; i < kTok; i += kThreads)
+            cp_async4(sm + L::A + 4 * i, a_raw + ((i < ntok ? t0 + i : 0) * H + h), i < ntok ? 4u : 0u);
+    } else {
+        for (int i = tid; i < kTok * D / 4; i += kThreads) {
+            const int row = i / (D / 4), piece = i % (D / 4);
+            const bool in = row < ntok;
+            cp_async16(sm + L::A + 16 * i,
+                       a_raw + ((in ? t0 + row : 0) * H + h) * (int64_t)D + 4 * piece, in ? 16u : 0u);
+        }
+    }
+    for (int i = tid; i < kTok; i += kThreads)
+        cp_async4(sm + L::B + 4 * i, beta_raw + ((i < ntok ? t0 + i : 0) * H + h), i < ntok ? 4u : 0u);
+    // taps transposed to [tensor][tap][channel], so that a thread's eight
+    // channels of one tap are two 16-byte words
+    for (int i = tid; i < 3 * 4 * D; i += kThreads) {
+        const int tsr = i / (4 * D), j = (i / D) % 4, c = i % D;
+        const float* w = tsr == 0 ? wq : (tsr == 1 ? wk : wv);
+        reinterpret_cast<float*>(sm + L::W)[i] = __ldg(w + ((size_t)h * D + c) * 4 + j);
+    }
+    if (SCALAR) {
+        if (tid == 0) cp_async4(sm + L::Bias, a_bias + h, 4u);
+    } else {
+        for (int i = tid; i < D / 4; i += kThreads)
+            cp_async16(sm + L::Bias + 16 * i, a_bias + (size_t)h * D + 4 * i, 16u);
+    }
+    cp_async_commit();
+    cp_async_wait_all();
+    __syncthreads();
 
-    // the sequence holding t0: the largest n with cu[n] <= t0
-    int n = 0;
-    {
-        int lo = 0, hi = n_seqs - 1;
+    // ---- outputs: thread (token r, channels c0 .. c0 + 7) -----------------------------
+    const int cg = tid % G, c0 = 8 * cg;
+    const T* X = reinterpret_cast<const T*>(sm + L::X);
+    const float* Wt = reinterpret_cast<const float*>(sm + L::W);
+    const float* Av = reinterpret_cast<const float*>(sm + L::A);
+    const float* Bv = reinterpret_cast<const float*>(sm + L::B);
+    const float* Bias = reinterpret_cast<const float*>(sm + L::Bias);
+#pragma unroll 1
+    for (int r = tid / G; r < kTok; r += TPP) {
+        if (r >= ntok) break;                      // uniform over the token's lanes
+        const int64_t t = t0 + r;
+        // first token of t's sequence: cu[n] for the largest n with cu[n] <= t
+        int lo = 0, hi = n_seqs - 1, n = 0;
         while (lo <= hi) {
             const int mid = (lo + hi) >> 1;
-            if ((int64_t)__ldg(cu + mid) <= t0) { n = mid; lo = mid + 1; } else { hi = mid - 1; }
+            if ((int64_t)__ldg(cu + mid) <= t) { n = mid; lo = mid + 1; } else { hi = mid - 1; }
         }
-    }
-    const int64_t s = __ldg(cu + n);
-    int64_t next = __ldg(cu + n + 1);          // start of the next sequence
-
-    // window: the three raw rows before t0 that belong to t0's sequence
-    float wq_[3][C], wk_[3][C], wv_[3][C];
+        const int64_t s = __ldg(cu + n);
+        float y[3][8];
 #pragma unroll
-    for (int j = 0; j < 3; ++j) {
-        const int64_t tt = t0 - 3 + j;
-        if (tt >= s) {
-            RowC<T, C> a, b, c;
-            const size_t off = ((size_t)tt * H + h) * D + c0;
-            a.load(xq + off); b.load(xk + off); c.load(xv + off);
-            a.get(wq_[j]); b.get(wk_[j]); c.get(wv_[j]);
+        for (int tsr = 0; tsr < 3; ++tsr) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) y[tsr][e] = 0.f;
+            // taps 3 .. 0 on rows t, t - 1, t - 2, t - 3 (staged row r + j is token t - 3 + j)
+#pragma unroll
+            for (int j = 3; j >= 0; --j) {
+                if (t - 3 + j < s) continue;
+                float x[8], w[8];
+                Vec8<T>::load(X + ((size_t)(tsr * (kTok + 3) + r + j)) * D + c0, x);
+                Vec8<float>::load(Wt + (size_t)(tsr * 4 + j) * D + c0, w);
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    y[tsr][e] = (j == 3) ? w[e] * x[e] : fmaf(w[e], x[e], y[tsr][e]);
+            }
+        }
+#pragma unroll
+        for (int tsr = 0; tsr < 2; ++tsr) {
+            float ss = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) ss = fmaf(y[tsr][e], y[tsr][e], ss);
+            ss = group_sum<G>(ss);
+            const float inv = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) y[tsr][e] *= inv;
+        }
+        const size_t row = ((size_t)t * H + h) * D + c0;
+        Vec8<T>::store(q + row, y[0]);
+        Vec8<T>::store(k + row, y[1]);
+        Vec8<T>::store(v + row, y[2]);
+        if (SCALAR) {
+            if (cg == 0) log_a[(size_t)t * H + h] = log_sigmoid(Av[r] + Bias[0]);
         } else {
+            float z[8], bz[8];
+            Vec8<float>::load(Av + (size_t)r * D + c0, z);
+            Vec8<float>::load(Bias + c0, bz);
 #pragma unroll
-            for (int e = 0; e < C; ++e) wq_[j][e] = wk_[j][e] = wv_[j][e] = 0.f;
+            for (int e = 0; e < 8; ++e) z[e] = log_sigmoid(z[e] + bz[e]);
+            Vec8<float>::store(log_a + row, z);
         }
+        if (cg == 0) beta[(size_t)t * H + h] = sigmoid(Bv[r]);
     }
+}
 
-    // loads kPref tokens ahead (ring of kPref slots, index t % kPref)
-    TokenIn<T, C, SCALAR> ring[kPref];
-#pragma unroll
-    for (int i = 0; i < kPref; ++i)
-        if (t0 + i < t1) ring[i].load(xq, xk, xv, a_raw, beta_raw, t0 + i, H, h, c0);
-
-    for (int64_t tb = t0; tb < t1; tb += kPref) {
-#pragma unroll
-        for (int i = 0; i < kPref; ++i) {
-            const int64_t t = tb + i;
-            if (t >= t1) break;
-            const TokenIn<T, C, SCALAR> in = ring[i];
-            if (t + kPref < t1) ring[i].load(xq, xk, xv, a_raw, beta_raw, t + kPref, H, h, c0);
-            if (t == next) {                   // a sequence starts here: clear the window
-                while (n + 1 < n_seqs && (int64_t)__ldg(cu + n + 1) <= t) ++n;
-                next = __ldg(cu + n + 1);
-#pragma unroll
-                for (int j = 0; j < 3; ++j)
-#pragma unroll
-                    for (int e = 0; e < C; ++e) wq_[j][e] = wk_[j][e] = wv_[j][e] = 0.f;
-            }
-            float x[C], yq[C], yk[C], yv[C];
-            in.xq.get(x); conv_step<C>(tq, wq_, x, yq);
-            in.xk.get(x); conv_step<C>(tk, wk_, x, yk);
-            in.xv.get(x); conv_step<C>(tv, wv_, x, yv);
-            float sq = 0.f, sk = 0.f;
-#pragma unroll
-            for (int e = 0; e < C; ++e) { sq = fmaf(yq[e], yq[e], sq); sk = fmaf(yk[e], yk[e], sk); }
-            sq = warp_sum(sq);
-            sk = warp_sum(sk);
-            const float iq = 1.0f / fmaxf(sqrtf(sq), 1e-12f), ik = 1.0f / fmaxf(sqrtf(sk), 1e-12f);
-#pragma unroll
-            for (int e = 0; e < C; ++e) { yq[e] *= iq; yk[e] *= ik; }
-            const size_t row = ((size_t)t * H + h) * D + c0;
-            storeC<C>(q + row, yq);
-            storeC<C>(k + row, yk);
-            storeC<C>(v + row, yv);
-            if (SCALAR) {
-                if (lane == 0) log_a[(size_t)t * H + h] = log_sigmoid(in.a_s + bias_s);
-            } else {
-                float z[C];
-                in.a.get(z);
-#pragma unroll
-                for (int e = 0; e < C; ++e) z[e] = log_sigmoid(z[e] + bias[e]);
-                storeC<C>(log_a + row, z);
-            }
-            if (lane == 1) beta[(size_t)t * H + h] = sigmoid(in.b);
-        }
-    }
+template <typename T, int D, bool SCALAR>
+cudaError_t launch_kernel(const gdr_preprocess_args& a, cudaStream_t st) {
+    auto kern = preprocess_kernel<T, D, SCALAR>;
+    constexpr uint32_t smem = PreLayout<T, D, SCALAR>::bytes;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t blocks = (a.total_tokens + kTok - 1) / kTok;
+    if (blocks > (int64_t)INT32_MAX || a.n_heads > 65535) return cudaErrorInvalidValue;
+    const dim3 grid((unsigned)blocks, (unsigned)a.n_heads);
+    kern<<<grid, kThreads, smem, st>>>(
+        a.n_seqs, a.n_heads, a.total_tokens, a.cu_seqlens, static_cast<const T*>(a.xq),
+        static_cast<const T*>(a.xk), static_cast<const T*>(a.xv), a.conv_q, a.conv_k, a.conv_v,
+        a.beta_raw, a.a_raw, a.a_bias, static_cast<T*>(a.q), static_cast<T*>(a.k),
+        static_cast<T*>(a.v), a.beta, a.log_a);
+    return cudaGetLastError();
 }
 
 template <typename T, int D>
 cudaError_t launch_typed(const gdr_preprocess_args& a, cudaStream_t st) {
-    const int64_t spans = (a.total_tokens + kSpan - 1) / kSpan;
-    const int64_t n_units = spans * a.n_heads;             // one warp each
-    const int64_t blocks = (n_units + kThreads / 32 - 1) / (kThreads / 32);
-    if (blocks > (int64_t)INT32_MAX) return cudaErrorInvalidValue;
-    const dim3 grid((unsigned)blocks);
-    auto* xq = static_cast<const T*>(a.xq);
-    auto* xk = static_cast<const T*>(a.xk);
-    auto* xv = static_cast<const T*>(a.xv);
-    auto* q = static_cast<T*>(a.q);
-    auto* k = static_cast<T*>(a.k);
-    auto* v = static_cast<T*>(a.v);
-    if (a.scalar_decay)
-        preprocess_kernel<T, D, true><<<grid, kThreads, 0, st>>>(
-            a.n_seqs, a.n_heads, a.total_tokens, n_units, a.cu_seqlens, xq, xk, xv, a.conv_q,
-            a.conv_k, a.conv_v, a.beta_raw, a.a_raw, a.a_bias, q, k, v, a.beta, a.log_a);
-    else
-        preprocess_kernel<T, D, false><<<grid, kThreads, 0, st>>>(
-            a.n_seqs, a.n_heads, a.total_tokens, n_units, a.cu_seqlens, xq, xk, xv, a.conv_q,
-            a.conv_k, a.conv_v, a.beta_raw, a.a_raw, a.a_bias, q, k, v, a.beta, a.log_a);
-    return cudaGetLastError();
+    return a.scalar_decay ? launch_kernel<T, D, true>(a, st) : launch_kernel<T, D, false>(a, st);
 }
 
 }  // namespace
