@@ -871,48 +871,102 @@ def bench_preprocess(gdr, stream, pk, args):
 
 def bench_e2e(gdr, w, stream, args):
     """The main workload's prefill through the public API from pinned host
-    buffers: H2D of the inputs, the prefill, D2H of o and the final states,
-    every step."""
+    buffers, every step: H2D of the inputs, the prefill, D2H of o and the
+    final states.  Timed twice: all on one stream, and pipelined over three
+    streams (step i+1's H2D and step i-1's D2H overlap step i's prefill; two
+    device buffer sets alternate, ordered by events) -- ``value`` is the
+    pipelined figure, each step still moving all of its bytes."""
     dev0 = wl.make_prefill_inputs(w, device="cuda", draw_device="cuda")
     names = [k_ for k_ in ("q", "k", "v", "beta", "log_a", "cu_seqlens", "init_state")
              if dev0.get(k_) is not None]
     pinned = {k_: dev0[k_].cpu().pin_memory() for k_ in names}
-    dev = {k_: torch.empty_like(dev0[k_]) for k_ in names}
-    del dev0
     T, H, dk = pinned["q"].shape
     dv = pinned["v"].shape[-1]
     n = pinned["cu_seqlens"].numel() - 1
-    out = torch.empty(T, H, dv, dtype=pinned["q"].dtype, device="cuda")
-    fin = torch.empty(n, H, dv, dk, device="cuda")
-    ns = gdr.snapshot_count(pinned["cu_seqlens"], w.snap_interval) if w.snap_interval else 0
-    snaps = torch.empty(max(ns, 1), H, dv, dk, device="cuda") if w.snap_interval else None
     ws = torch.empty(gdr.workspace_size(n, H, dk, dv, T, w.scalar_decay), dtype=torch.uint8,
                      device="cuda")
-    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    fin_h = torch.empty(fin.shape, dtype=fin.dtype).pin_memory()
-    prep = gdr.PreparedPrefill(dev["q"], dev["k"], dev["v"], dev["beta"], dev["log_a"],
-                               dev["cu_seqlens"], out=out, final_state=fin, workspace=ws,
-                               scalar_decay=w.scalar_decay, scale=w.scale,
-                               init_state=dev.get("init_state"), snap_interval=w.snap_interval,
-                               snapshots=snaps)
+    ns = gdr.snapshot_count(pinned["cu_seqlens"], w.snap_interval) if w.snap_interval else 0
+    bufs = []
+    for b in range(2):
+        dev = dev0 if b == 0 else {k_: torch.empty_like(dev0[k_]) for k_ in names}
+        dev = {k_: dev[k_] for k_ in names}
+        out = torch.empty(T, H, dv, dtype=pinned["q"].dtype, device="cuda")
+        fin = torch.empty(n, H, dv, dk, device="cuda")
+        snaps = torch.empty(max(ns, 1), H, dv, dk, device="cuda") if w.snap_interval else None
+        prep = gdr.PreparedPrefill(dev["q"], dev["k"], dev["v"], dev["beta"], dev["log_a"],
+                                   dev["cu_seqlens"], out=out, final_state=fin, workspace=ws,
+                                   scalar_decay=w.scalar_decay, scale=w.scale,
+                                   init_state=dev.get("init_state"),
+                                   snap_interval=w.snap_interval, snapshots=snaps)
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        fin_h = torch.empty(fin.shape, dtype=fin.dtype).pin_memory()
+        bufs.append(dict(dev=dev, out=out, fin=fin, prep=prep, out_h=out_h, fin_h=fin_h,
+                         loaded=torch.cuda.Event(), done=torch.cuda.Event(),
+                         read=torch.cuda.Event()))
+    del dev0
 
-    def step(_):
+    def serial(i):
+        b = bufs[0]
         for k_ in names:
-            dev[k_].copy_(pinned[k_], non_blocking=True)
-        prep.run()
-        out_h.copy_(out, non_blocking=True)
-        fin_h.copy_(fin, non_blocking=True)
+            b["dev"][k_].copy_(pinned[k_], non_blocking=True)
+        b["prep"].run()
+        b["out_h"].copy_(b["out"], non_blocking=True)
+        b["fin_h"].copy_(b["fin"], non_blocking=True)
+
+    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def pipelined(i):
+        b = bufs[i % 2]
+        with torch.cuda.stream(h2d):
+            if i >= 2:
+                h2d.wait_event(b["done"])            # prefill i-2 has read these inputs
+            for k_ in names:
+                b["dev"][k_].copy_(pinned[k_], non_blocking=True)
+            b["loaded"].record(h2d)
+        stream.wait_event(b["loaded"])
+        if i >= 2:
+            stream.wait_event(b["read"])             # D2H of step i-2 has read o, final
+        b["prep"].run(stream=stream)
+        b["done"].record(stream)
+        with torch.cuda.stream(d2h):
+            d2h.wait_event(b["done"])
+            b["out_h"].copy_(b["out"], non_blocking=True)
+            b["fin_h"].copy_(b["fin"], non_blocking=True)
+            b["read"].record(d2h)
+
+    def timed_streams(fn, n_steps):
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        start.record(stream)
+        h2d.wait_event(start)
+        d2h.wait_event(start)
+        for i in range(n_steps):
+            fn(i)
+        stream.wait_stream(h2d)
+        stream.wait_stream(d2h)
+        end.record(stream)
+        torch.cuda.synchronize()
+        return start.elapsed_time(end) / n_steps
 
     for i in range(3):
-        step(i)
+        serial(i)
+    for i in range(4):
+        pipelined(i)
+    torch.cuda.synchronize()
     n_steps = max(5, min(args.steps, 20))
-    ms = timed(step, n_steps, stream)
-    h2d = sum(t.numel() * t.element_size() for t in pinned.values())
-    d2h = out_h.numel() * out_h.element_size() + fin_h.numel() * fin_h.element_size()
-    res = {"value": round(T / (ms * 1e-3), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 4), "steps": n_steps,
-           "workload": w.name}
-    del pinned, dev, out, fin, ws, out_h, fin_h, prep, snaps
+    ms_serial = timed_streams(serial, n_steps)
+    ms = timed_streams(pipelined, n_steps)
+    h2d_bytes = sum(t.numel() * t.element_size() for t in pinned.values())
+    b0 = bufs[0]
+    d2h_bytes = b0["out_h"].numel() * b0["out_h"].element_size() + \
+        b0["fin_h"].numel() * b0["fin_h"].element_size()
+    res = {"value": round(T / (ms * 1e-3), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d_bytes,
+           "d2h_bytes_per_step": d2h_bytes, "ms_per_step": round(ms, 4),
+           "serial_one_stream": {"ms_per_step": round(ms_serial, 4),
+                                 "tokens_per_s": round(T / (ms_serial * 1e-3), 1)},
+           "steps": n_steps, "workload": w.name,
+           "pipelining": "H2D, prefill and D2H on three streams, two buffer sets"}
+    del pinned, bufs, ws
     torch.cuda.empty_cache()
     return res
 

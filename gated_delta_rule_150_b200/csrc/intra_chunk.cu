@@ -69,8 +69,11 @@ __host__ __device__ constexpr uint32_t al1024(uint32_t x) { return (x + 1023u) &
 __host__ __device__ constexpr uint32_t umax(uint32_t a, uint32_t b) { return a > b ? a : b; }
 
 // Gate activations of the fused input path (raw projections).
+// log(1 + e) with the fast log: e = exp(-|z|) is in (0, 1], so 1 + e is in
+// (1, 2] where __logf's absolute error is a few 1e-8 -- far inside what the
+// bf16 operands built from log a resolve
 __device__ __forceinline__ float log_sigmoid_f(float z) {
-    return fminf(z, 0.f) - log1pf(__expf(-fabsf(z)));
+    return fminf(z, 0.f) - __logf(1.f + __expf(-fabsf(z)));
 }
 
 __device__ __forceinline__ float sigmoid_f(float z) {
@@ -815,6 +818,10 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
             }
         }
     }
+    // B1^T rows c, B2^T rows D + c, Kd^T rows c (token columns r0 .. r0 + RPT - 1):
+    // stored here at d 64; at d 128 while the A/P MMA runs (measured 4 % faster there,
+    // no gain at d 64, where keeping the pairs live across the MMA issue spills)
+    if constexpr (D == 64) {
     // B1^T rows c, B2^T rows D + c, Kd^T rows c; token columns r0 .. r0 + RPT - 1.
     // Step e of lane group cg writes channel c0 + (e ^ s), s = cg mod 8, so the
     // lanes of a warp hit 8 different swizzle positions instead of one.
@@ -837,6 +844,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
             *reinterpret_cast<uint32_t*>(Bt + o2) = pb2[e][0];
             *reinterpret_cast<uint32_t*>(Kdt + o3) = pkd[e][0];
         }
+    }
     }
     fence_proxy_async_smem();
     tc_fence_before_sync();
@@ -864,6 +872,32 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         }
         mma_commit(&mma_bar);
         ++mma_commits;
+    }
+    if constexpr (D != 64) {
+    // B1^T rows c, B2^T rows D + c, Kd^T rows c; token columns r0 .. r0 + RPT - 1.
+    // Step e of lane group cg writes channel c0 + (e ^ s), s = cg mod 8, so the
+    // lanes of a warp hit 8 different swizzle positions instead of one.
+    const int s8 = cg & 7;
+    xor_permute(pb1, s8);
+    xor_permute(pb2, s8);
+    xor_permute(pkd, s8);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const int c = c0 + (e ^ s8);
+        const uint32_t o1 = sw128_chunk(2 * D, c, r0 / 8) + (r0 % 8) * 2;
+        const uint32_t o2 = sw128_chunk(2 * D, D + c, r0 / 8) + (r0 % 8) * 2;
+        const uint32_t o3 = sw128_chunk(D, c, r0 / 8) + (r0 % 8) * 2;
+        if constexpr (RPT == 4) {
+            *reinterpret_cast<uint2*>(Bt + o1) = make_uint2(pb1[e][0], pb1[e][RPT / 2 - 1]);
+            *reinterpret_cast<uint2*>(Bt + o2) = make_uint2(pb2[e][0], pb2[e][RPT / 2 - 1]);
+            *reinterpret_cast<uint2*>(Kdt + o3) = make_uint2(pkd[e][0], pkd[e][RPT / 2 - 1]);
+        } else {
+            *reinterpret_cast<uint32_t*>(Bt + o1) = pb1[e][0];
+            *reinterpret_cast<uint32_t*>(Bt + o2) = pb2[e][0];
+            *reinterpret_cast<uint32_t*>(Kdt + o3) = pkd[e][0];
+        }
+    }
+        fence_proxy_async_smem();     // read by later MMAs, after the next barrier
     }
     failed = !mbar_wait(&mma_bar, phase);
     phase ^= 1u;
