@@ -374,6 +374,8 @@ gdr_status gdr_preprocess(const gdr_preprocess_args* a, void* stream) {
     if (a->n_seqs < 0 || a->n_heads <= 0 || a->d <= 0 || a->total_tokens < 0 ||
         a->total_tokens > (int64_t)INT32_MAX)
         return GDR_ERR_INVALID_ARG;
+    // one CTA per (32-token block, head)
+    if ((a->total_tokens + 31) / 32 * (int64_t)a->n_heads > (int64_t)INT32_MAX) return GDR_ERR_INVALID_ARG;
     if (a->io_dtype != GDR_BF16 && a->io_dtype != GDR_F32) return GDR_ERR_INVALID_ARG;
     if (!supported_width(a->d)) return GDR_ERR_UNSUPPORTED;
     if (a->total_tokens == 0) return GDR_OK;

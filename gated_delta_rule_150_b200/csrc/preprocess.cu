@@ -9,7 +9,12 @@
 // k normalised per (token, head) after it as y / max(||y||, 1e-12), the conv
 // restarting from zero history at every sequence start.
 //
-// Layout of the work: one CTA per (head, block of kTok tokens).  It first
+// Layout of the work: one CTA per (head, block of kTok tokens), heads
+// fastest in the launch order, so that the CTAs resident at one time read
+// every head of the same tokens: contiguous runs of H * D elements per
+// token instead of one head's D elements every H * D (measured 7 % faster at
+// d 64 and 5 % at d 128 than token blocks fastest, the difference being DRAM
+// page locality).  It first
 // stages, by 16-byte cp.async from every thread, the raw rows of x_q, x_k and
 // x_v for tokens [t0 - 3, t0 + kTok) (the three before the block for the
 // conv), the block's a_raw rows, beta_raw and the head's conv taps and gate
@@ -30,7 +35,7 @@ namespace gdr {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kTok = 64;            // tokens per CTA
+constexpr int kTok = 32;            // tokens per CTA (32 measured faster than 64)
 
 template <typename T, int D, bool SCALAR>
 struct PreLayout {
@@ -44,8 +49,12 @@ struct PreLayout {
     static constexpr uint32_t bytes = Bias + 4u * D;
 };
 
+// log(1 + e) with the fast log: e = exp(-|z|) is in (0, 1], so 1 + e is in
+// (1, 2], where __logf's absolute error is documented below 2^-21.4 (about
+// 4e-7), inside the 2e-6 absolute bound the outputs are held to (measured
+// 4-6 % faster than log1pf)
 __device__ __forceinline__ float log_sigmoid(float z) {
-    return fminf(z, 0.f) - log1pf(expf(-fabsf(z)));
+    return fminf(z, 0.f) - __logf(1.f + __expf(-fabsf(z)));
 }
 
 __device__ __forceinline__ float sigmoid(float z) {
@@ -79,10 +88,14 @@ template <> struct Vec8<float> {
 };
 
 // Sum over the G = D / 8 lanes of a token (G divides 32; groups are G-aligned).
+// The shuffles name only the token's own lanes: in a ragged last block the
+// lanes of tokens past its end have left the token loop.
 template <int G>
 __device__ __forceinline__ float group_sum(float v) {
+    const unsigned lane = threadIdx.x & 31u;
+    const unsigned mask = G == 32 ? 0xffffffffu : ((1u << G) - 1u) << (lane & ~(unsigned)(G - 1));
 #pragma unroll
-    for (int m = G / 2; m >= 1; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
+    for (int m = G / 2; m >= 1; m >>= 1) v += __shfl_xor_sync(mask, v, m);
     return v;
 }
 
@@ -101,8 +114,8 @@ preprocess_kernel(int n_seqs, int H, int64_t T_tot, const int32_t* __restrict__ 
     constexpr int kPer = D * (int)sizeof(T) / 16;  // 16-byte pieces per raw row
     extern __shared__ __align__(16) uint8_t sm[];
     const int tid = threadIdx.x;
-    const int h = blockIdx.y;
-    const int64_t t0 = (int64_t)blockIdx.x * kTok;
+    const int h = (int)(blockIdx.x % (unsigned)H);
+    const int64_t t0 = (int64_t)(blockIdx.x / (unsigned)H) * kTok;
     const int ntok = (int)(T_tot - t0 < kTok ? T_tot - t0 : kTok);
 
     // ---- stage everything the block reads -----------------------------------------
@@ -215,9 +228,11 @@ cudaError_t launch_kernel(const gdr_preprocess_args& a, cudaStream_t st) {
     constexpr uint32_t smem = PreLayout<T, D, SCALAR>::bytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const int64_t blocks = (a.total_tokens + kTok - 1) / kTok;
-    if (blocks > (int64_t)INT32_MAX || a.n_heads > 65535) return cudaErrorInvalidValue;
-    const dim3 grid((unsigned)blocks, (unsigned)a.n_heads);
+    // one CTA per (token block, head), heads fastest
+    const int64_t ctas = (a.total_tokens + kTok - 1) / kTok * (int64_t)a.n_heads;
+    if (ctas == 0) return cudaSuccess;
+    if (ctas > (int64_t)INT32_MAX) return cudaErrorInvalidValue;
+    const dim3 grid((unsigned)ctas);
     kern<<<grid, kThreads, smem, st>>>(
         a.n_seqs, a.n_heads, a.total_tokens, a.cu_seqlens, static_cast<const T*>(a.xq),
         static_cast<const T*>(a.xk), static_cast<const T*>(a.xv), a.conv_q, a.conv_k, a.conv_v,

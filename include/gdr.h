@@ -386,8 +386,9 @@ typedef struct {
  * Enqueue the input activations.  Outputs must not overlap the inputs.
  * Errors: GDR_ERR_INVALID_ARG (null or misaligned pointer -- xq, xk, xv, the
  * conv taps, q, k, v and, with a per-channel gate, a_raw, a_bias and log_a
- * need 16-byte alignment -- or bad sizes), GDR_ERR_UNSUPPORTED (d not 64 or
- * 128), GDR_ERR_CUDA on a failed launch.  T_tot == 0 is a no-op.
+ * need 16-byte alignment -- or bad sizes, including ceil(T_tot / 32) * H
+ * above 2^31 - 1), GDR_ERR_UNSUPPORTED (d not 64 or 128), GDR_ERR_CUDA on a
+ * failed launch.  T_tot == 0 is a no-op.
  */
 gdr_status gdr_preprocess(const gdr_preprocess_args* args, void* stream);
 
