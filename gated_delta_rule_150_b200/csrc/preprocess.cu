@@ -87,6 +87,20 @@ template <> struct Vec8<float> {
     }
 };
 
+// The fp32 rows in shared memory (taps, a_raw, gate bias) store 16-byte word
+// w (channels 4w .. 4w + 3) at word w ^ ((w >> 3) & 1).  A thread reads
+// words 2 cg and 2 cg + 1 (its channels 8 cg .. 8 cg + 7); in the plain order
+// the eight lanes of a quarter-warp would hit every bank group twice (words
+// 32 bytes apart), swizzled they hit each once, and eight consecutive words
+// written by consecutive lanes stay in distinct bank groups too.
+__device__ __forceinline__ int swz_word(int w) { return w ^ ((w >> 3) & 1); }
+
+__device__ __forceinline__ void load8_swz(const float* row, int cg, float (&x)[8]) {
+    const float4 a = *reinterpret_cast<const float4*>(row + 4 * swz_word(2 * cg));
+    const float4 b = *reinterpret_cast<const float4*>(row + 4 * swz_word(2 * cg + 1));
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+
 // Sum over the G = D / 8 lanes of a token (G divides 32; groups are G-aligned).
 // The shuffles name only the token's own lanes: in a ragged last block the
 // lanes of tokens past its end have left the token loop.
@@ -136,24 +150,25 @@ preprocess_kernel(int n_seqs, int H, int64_t T_tot, const int32_t* __restrict__ 
         for (int i = tid; i < kTok * D / 4; i += kThreads) {
             const int row = i / (D / 4), piece = i % (D / 4);
             const bool in = row < ntok;
-            cp_async16(sm + L::A + 16 * i,
+            cp_async16(sm + L::A + 4 * (row * D + 4 * swz_word(piece)),
                        a_raw + ((in ? t0 + row : 0) * H + h) * (int64_t)D + 4 * piece, in ? 16u : 0u);
         }
     }
     for (int i = tid; i < kTok; i += kThreads)
         cp_async4(sm + L::B + 4 * i, beta_raw + ((i < ntok ? t0 + i : 0) * H + h), i < ntok ? 4u : 0u);
-    // taps transposed to [tensor][tap][channel], so that a thread's eight
-    // channels of one tap are two 16-byte words
+    // taps transposed to [tensor][tap][channel] (16-byte words swizzled as
+    // above), so that a thread's eight channels of one tap are two 16-byte words
     for (int i = tid; i < 3 * 4 * D; i += kThreads) {
         const int tsr = i / (4 * D), j = (i / D) % 4, c = i % D;
         const float* w = tsr == 0 ? wq : (tsr == 1 ? wk : wv);
-        reinterpret_cast<float*>(sm + L::W)[i] = __ldg(w + ((size_t)h * D + c) * 4 + j);
+        reinterpret_cast<float*>(sm + L::W)[(tsr * 4 + j) * D + 4 * swz_word(c / 4) + c % 4] =
+            __ldg(w + ((size_t)h * D + c) * 4 + j);
     }
     if (SCALAR) {
         if (tid == 0) cp_async4(sm + L::Bias, a_bias + h, 4u);
     } else {
         for (int i = tid; i < D / 4; i += kThreads)
-            cp_async16(sm + L::Bias + 16 * i, a_bias + (size_t)h * D + 4 * i, 16u);
+            cp_async16(sm + L::Bias + 16 * swz_word(i), a_bias + (size_t)h * D + 4 * i, 16u);
     }
     cp_async_commit();
     cp_async_wait_all();
@@ -188,7 +203,7 @@ preprocess_kernel(int n_seqs, int H, int64_t T_tot, const int32_t* __restrict__ 
                 if (t - 3 + j < s) continue;
                 float x[8], w[8];
                 Vec8<T>::load(X + ((size_t)(tsr * (kTok + 3) + r + j)) * D + c0, x);
-                Vec8<float>::load(Wt + (size_t)(tsr * 4 + j) * D + c0, w);
+                load8_swz(Wt + (size_t)(tsr * 4 + j) * D, cg, w);
 #pragma unroll
                 for (int e = 0; e < 8; ++e)
                     y[tsr][e] = (j == 3) ? w[e] * x[e] : fmaf(w[e], x[e], y[tsr][e]);
@@ -212,8 +227,8 @@ preprocess_kernel(int n_seqs, int H, int64_t T_tot, const int32_t* __restrict__ 
             if (cg == 0) log_a[(size_t)t * H + h] = log_sigmoid(Av[r] + Bias[0]);
         } else {
             float z[8], bz[8];
-            Vec8<float>::load(Av + (size_t)r * D + c0, z);
-            Vec8<float>::load(Bias + c0, bz);
+            load8_swz(Av + (size_t)r * D, cg, z);
+            load8_swz(Bias, cg, bz);
 #pragma unroll
             for (int e = 0; e < 8; ++e) z[e] = log_sigmoid(z[e] + bz[e]);
             Vec8<float>::store(log_a + row, z);
