@@ -559,6 +559,7 @@ def run_gdr(args):
     stage_report = {STAGES[s_]: round(st_ms[s_], 4) for s_ in range(len(STAGES))}
     la, cu0 = ps.sets[0]["inp"]["log_a"], ps.sets[0]["inp"]["cu_seqlens"]
     g_out = torch.empty_like(la)
+    gdr.cumdecay(la, cu0, out=g_out, d_k=ps.dk, scalar_decay=ps.w.scalar_decay)   # warm-up
     stage_report["cumdecay_standalone"] = round(
         timed(lambda i: gdr.cumdecay(la, cu0, out=g_out, d_k=ps.dk,
                                      scalar_decay=ps.w.scalar_decay), 10, stream), 4)
