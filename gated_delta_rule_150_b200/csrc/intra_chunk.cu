@@ -370,12 +370,15 @@ struct RawParams {
 // Issue the copies of one item's inputs, from one warp: lane 0 starts the
 // tiled TMA loads of log a (completing on bar_g) and of q, k, v (on bar_qkv);
 // beta and the scalar log a go by 4-byte cp.async with zero fill.
+// The inputs of item `it`: with `tiles`, the per-channel decay tile and q,
+// k, v (region 1) by 2-D TMA from lane 0; always beta (and a scalar log a)
+// by cp.async from every lane.
 template <int D, typename InT, bool SCALAR, bool RAW, typename L>
 __device__ __forceinline__ void issue_inputs(uint8_t* sm, uint64_t* bar_g, uint64_t* bar_qkv,
                                              const InputMaps& maps, const float* __restrict__ beta,
                                              const float* __restrict__ log_a, int H, const Item& it,
-                                             int lane, bool hint) {
-    if (lane == 0) {
+                                             int lane, bool hint, bool tiles) {
+    if (lane == 0 && tiles) {
         const int x = it.h * D;
         const uint64_t pol = l2_policy_evict_first();             // inputs are read once
         if (!SCALAR) {
@@ -492,13 +495,14 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
-    // requests of inputs (load warp) and MMA commits (thread 0) so far: on a
-    // timed-out wait the last of each is drained before the CTA exits
-    uint32_t in_issued = 0, mma_commits = 0;
+    // requests of decay tiles and of the other inputs (load warp) and MMA
+    // commits (thread 0) so far: on a timed-out wait the last of each is
+    // drained before the CTA exits
+    uint32_t tiles_issued = 0, mma_commits = 0;
     if (cur.idx >= 0 && warp == kLoadWarp) {
         issue_inputs<D, InT, SCALAR, RAW, L>(sm, &in_bar[0], &in_bar[1], maps, beta, log_a, H, cur,
-                                             lane, keep_records != 0);
-        ++in_issued;
+                                             lane, keep_records != 0, true);
+        ++tiles_issued;
     }
     const uint32_t tmem = tmem_slot;
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
@@ -851,6 +855,43 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     __syncthreads();
     tc_fence_after_sync();
 
+    // ---- the next item's decay tile and q, k, v -------------------------------
+    // This item read region 1 (g, q, k, v) in the operand build above; only a
+    // chunk with extreme decay reads it again (the exact path of the A/P
+    // readout), and there the tiles keep the late request with beta (which
+    // the readout reads).  Otherwise they are requested now, so that the
+    // decay tile has landed when warps 4-7 scan it during the solve.
+    const bool tiles_early = SCALAR || !bad_chunk;
+    if (tiles_early && warp == kLoadWarp) {
+        const Item nxt = s_item[(iter + 1) & 1];
+        if (nxt.idx >= 0) {
+            fence_proxy_async_smem();             // the operand build's reads of region 1 come first
+            if (lane == 0) {
+                const int x = nxt.h * D;
+                const uint64_t pol = l2_policy_evict_first();
+                const bool hint = keep_records != 0;
+                if (!SCALAR) {
+                    mbar_arrive_expect_tx(&in_bar[0], 64u * D * 4u);
+                    if (hint) tma_load_2d_hint(sm + L::sG, &maps.g, x, nxt.start, &in_bar[0], pol);
+                    else tma_load_2d(sm + L::sG, &maps.g, x, nxt.start, &in_bar[0]);
+                }
+                if (L::kStageQKV) {
+                    mbar_arrive_expect_tx(&in_bar[1], 3u * 64u * D * (uint32_t)sizeof(InT));
+                    if (hint) {
+                        tma_load_2d_hint(sm + L::sQ, &maps.q, x, nxt.start, &in_bar[1], pol);
+                        tma_load_2d_hint(sm + L::sK, &maps.k, x, nxt.start, &in_bar[1], pol);
+                        tma_load_2d_hint(sm + L::sV, &maps.v, x, nxt.start, &in_bar[1], pol);
+                    } else {
+                        tma_load_2d(sm + L::sQ, &maps.q, x, nxt.start, &in_bar[1]);
+                        tma_load_2d(sm + L::sK, &maps.k, x, nxt.start, &in_bar[1]);
+                        tma_load_2d(sm + L::sV, &maps.v, x, nxt.start, &in_bar[1]);
+                    }
+                }
+            }
+            ++tiles_issued;
+        }
+    }
+
     // ---- decay-weighted Q K^T and K K^T on the tensor cores ------------------
     if (tid == 0) {
         const uint32_t aXA = smem_u32(XA);
@@ -987,15 +1028,16 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     }
     __syncthreads();
 
-    // region 1 and beta are free: stage the next item's inputs
-    // and look up the item after it (read by every thread at this item's end)
+    // region 1 and beta are free: stage the next item's beta (and its tiles
+    // if they were not requested during the A/P MMA) and look up the item
+    // after it (read by every thread at this item's end)
     if (warp == kLoadWarp) {
         const Item nxt = s_item[(iter + 1) & 1];
         fence_proxy_async_smem();             // this item's reads of region 1 come first
         if (nxt.idx >= 0) {
             issue_inputs<D, InT, SCALAR, RAW, L>(sm, &in_bar[0], &in_bar[1], maps, beta, log_a, H, nxt,
-                                                 lane, keep_records != 0);
-            ++in_issued;
+                                                 lane, keep_records != 0, !tiles_early);
+            if (!tiles_early) ++tiles_issued;
         }
         if (lane == 0)
             s_item[iter & 1] = nxt.idx >= 0 ? find_item(cu, n_seqs, H, n_items, nxt.idx + gridDim.x) : nxt;
@@ -1250,9 +1292,9 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         // the last requested inputs (at most one of each is outstanding; these
         // waits are bounded too)
         if (tid == 0 && mma_commits > 0) (void)mbar_wait(&mma_bar, (mma_commits - 1u) & 1u);
-        if (warp == kLoadWarp && lane == 0 && in_issued > 0) {
-            if (!SCALAR) (void)mbar_wait(&in_bar[0], (in_issued - 1u) & 1u);
-            if (L::kStageQKV) (void)mbar_wait(&in_bar[1], (in_issued - 1u) & 1u);
+        if (warp == kLoadWarp && lane == 0 && tiles_issued > 0) {
+            if (!SCALAR) (void)mbar_wait(&in_bar[0], (tiles_issued - 1u) & 1u);
+            if (L::kStageQKV) (void)mbar_wait(&in_bar[1], (tiles_issued - 1u) & 1u);
         }
     }
     cp_async_wait_all();
