@@ -14,9 +14,13 @@
 //
 // Memory roofline: per head-state 2 * 4 * d_v * d_k bytes of state plus the
 // token's inputs and the output row; no reuse, so the kernel is HBM-bound.
+// Launched with programmatic stream serialization: back-to-back steps (the
+// layers of a decode pass) schedule their CTAs while the previous step's last
+// wave drains, each waiting for that step's memory before its first access.
 #include <cuda_bf16.h>
 
 #include "internal.h"
+#include "sm100.cuh"
 
 namespace gdr {
 namespace {
@@ -66,6 +70,8 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
                    float* __restrict__ state, float* __restrict__ o, const DecodeGate<T> og) {
     constexpr int NV = DK / (4 * kTPR);        // float4 per thread per row: 1 or 2
     constexpr int PASSES = DV / kRowsPerPass;  // 4 or 8
+    pdl_launch_dependents();
+    pdl_wait();                                // the previous kernel's writes are visible
     const int bh = blockIdx.x;
     const int lane16 = threadIdx.x % kTPR;
     const int rgrp = threadIdx.x / kTPR;
@@ -156,12 +162,10 @@ cudaError_t launch_typed(int B, int H, const void* q, const void* k, const void*
                          float* state, float* o, const DecodeGate<T>& og, cudaStream_t st) {
     const dim3 grid((unsigned)(B * H));
     if (scalar)
-        decode_step_kernel<T, DK, DV, true, GATED><<<grid, kThreads, 0, st>>>(
-            (const T*)q, (const T*)k, (const T*)v, beta, log_a, scale, state, o, og);
-    else
-        decode_step_kernel<T, DK, DV, false, GATED><<<grid, kThreads, 0, st>>>(
-            (const T*)q, (const T*)k, (const T*)v, beta, log_a, scale, state, o, og);
-    return cudaGetLastError();
+        return launch_pdl(true, decode_step_kernel<T, DK, DV, true, GATED>, grid, dim3(kThreads), 0, st,
+                          (const T*)q, (const T*)k, (const T*)v, beta, log_a, scale, state, o, og);
+    return launch_pdl(true, decode_step_kernel<T, DK, DV, false, GATED>, grid, dim3(kThreads), 0, st,
+                      (const T*)q, (const T*)k, (const T*)v, beta, log_a, scale, state, o, og);
 }
 
 template <typename T, bool GATED>

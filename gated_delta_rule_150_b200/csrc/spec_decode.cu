@@ -19,6 +19,7 @@
 #include <cuda_bf16.h>
 
 #include "internal.h"
+#include "sm100.cuh"
 
 namespace gdr {
 namespace {
@@ -100,6 +101,8 @@ decode_draft_kernel(int H, int K, const T* __restrict__ q, const T* __restrict__
                     float* __restrict__ o, float* __restrict__ token_states) {
     constexpr int PASSES = DV / (RS * kRowsPerPass);
     static_assert(PASSES >= 1 && PASSES * RS * kRowsPerPass == DV, "row split");
+    pdl_launch_dependents();
+    pdl_wait();                                // the previous kernel's writes are visible
     using Tok = TokenIn<T, DK, DV, PASSES, SCALAR>;
     constexpr int NV = Tok::NV;
     const int bh = blockIdx.x / RS;
@@ -174,6 +177,8 @@ decode_draft_kernel(int H, int K, const T* __restrict__ q, const T* __restrict__
 __global__ void __launch_bounds__(kThreads)
 decode_accept_kernel(int H, int K, int n4, const int32_t* __restrict__ n_accept,
                      const float* __restrict__ token_states, float* __restrict__ state) {
+    pdl_launch_dependents();
+    pdl_wait();                                // the draft's kept states are visible
     const int bh = blockIdx.x;
     const int b = bh / H;
     const int h = bh - b * H;
@@ -210,12 +215,10 @@ cudaError_t draft_typed(int B, int K, int H, const void* q, const void* k, const
                         const float* state, float* o, float* ts, cudaStream_t st) {
     const dim3 grid((unsigned)((int64_t)B * H * kRowSplit));
     if (scalar)
-        decode_draft_kernel<T, DK, DV, true, kRowSplit><<<grid, kThreads, 0, st>>>(
-            H, K, (const T*)q, (const T*)k, (const T*)v, beta, log_a, scale, state, o, ts);
-    else
-        decode_draft_kernel<T, DK, DV, false, kRowSplit><<<grid, kThreads, 0, st>>>(
-            H, K, (const T*)q, (const T*)k, (const T*)v, beta, log_a, scale, state, o, ts);
-    return cudaGetLastError();
+        return launch_pdl(true, decode_draft_kernel<T, DK, DV, true, kRowSplit>, grid, dim3(kThreads), 0,
+                          st, H, K, (const T*)q, (const T*)k, (const T*)v, beta, log_a, scale, state, o, ts);
+    return launch_pdl(true, decode_draft_kernel<T, DK, DV, false, kRowSplit>, grid, dim3(kThreads), 0, st,
+                      H, K, (const T*)q, (const T*)k, (const T*)v, beta, log_a, scale, state, o, ts);
 }
 
 template <typename T>
@@ -246,9 +249,8 @@ cudaError_t launch_decode_draft(int B, int K, int H, int dk, int dv, gdr_dtype d
 
 cudaError_t launch_decode_accept(int B, int K, int H, int dk, int dv, const int32_t* n_accept,
                                  const float* token_states, float* state, cudaStream_t st) {
-    decode_accept_kernel<<<(unsigned)(B * H), kThreads, 0, st>>>(H, K, dk * dv / 4, n_accept,
-                                                                 token_states, state);
-    return cudaGetLastError();
+    return launch_pdl(true, decode_accept_kernel, dim3((unsigned)(B * H)), dim3(kThreads), 0, st, H, K,
+                      dk * dv / 4, n_accept, token_states, state);
 }
 
 }  // namespace gdr
