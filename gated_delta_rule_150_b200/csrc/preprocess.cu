@@ -128,6 +128,8 @@ preprocess_kernel(int n_seqs, int H, int64_t T_tot, const int32_t* __restrict__ 
     constexpr int kPer = D * (int)sizeof(T) / 16;  // 16-byte pieces per raw row
     extern __shared__ __align__(16) uint8_t sm[];
     const int tid = threadIdx.x;
+    pdl_launch_dependents();
+    pdl_wait();                                    // the previous kernel's writes are visible
     const int h = (int)(blockIdx.x % (unsigned)H);
     const int64_t t0 = (int64_t)(blockIdx.x / (unsigned)H) * kTok;
     const int ntok = (int)(T_tot - t0 < kTok ? T_tot - t0 : kTok);
@@ -247,13 +249,12 @@ cudaError_t launch_kernel(const gdr_preprocess_args& a, cudaStream_t st) {
     const int64_t ctas = (a.total_tokens + kTok - 1) / kTok * (int64_t)a.n_heads;
     if (ctas == 0) return cudaSuccess;
     if (ctas > (int64_t)INT32_MAX) return cudaErrorInvalidValue;
-    const dim3 grid((unsigned)ctas);
-    kern<<<grid, kThreads, smem, st>>>(
-        a.n_seqs, a.n_heads, a.total_tokens, a.cu_seqlens, static_cast<const T*>(a.xq),
-        static_cast<const T*>(a.xk), static_cast<const T*>(a.xv), a.conv_q, a.conv_k, a.conv_v,
-        a.beta_raw, a.a_raw, a.a_bias, static_cast<T*>(a.q), static_cast<T*>(a.k),
-        static_cast<T*>(a.v), a.beta, a.log_a);
-    return cudaGetLastError();
+    // early launch: the CTAs take the SMs the previous kernel's last CTAs leave
+    return launch_pdl(true, kern, dim3((unsigned)ctas), dim3(kThreads), smem, st, a.n_seqs, a.n_heads,
+                      a.total_tokens, a.cu_seqlens, static_cast<const T*>(a.xq),
+                      static_cast<const T*>(a.xk), static_cast<const T*>(a.xv), a.conv_q, a.conv_k,
+                      a.conv_v, a.beta_raw, a.a_raw, a.a_bias, static_cast<T*>(a.q),
+                      static_cast<T*>(a.k), static_cast<T*>(a.v), a.beta, a.log_a);
 }
 
 template <typename T, int D>
