@@ -23,7 +23,8 @@
 //
 // Structure.  A persistent kernel: as many CTAs as fit (two per SM at d 64,
 // one at d 128) take the items round-robin.  A loader warp requests the next
-// item's q, k, v and log a by 2-D TMA while the current item is finished;
+// item's q, k, v and log a by 2-D TMA as soon as the current item's operand
+// build has read its own (while the A/P MMA runs);
 // the chunk-local cumulative decay (the standalone cumdecay kernel's
 // quantity) is summed in shared memory, for per-channel decay by warps 4-7
 // during the previous item's triangular solve; the record leaves by two bulk
