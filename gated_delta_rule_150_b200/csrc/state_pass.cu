@@ -108,7 +108,11 @@ struct PassLayout {
     static constexpr uint32_t kStride = kOut ? R.bytes : 4u * D * D + 1024u;
     static constexpr uint32_t bytes = Rec0 + (kStages - 1) * kStride + kGamma + 4u * D;
     static constexpr uint32_t dyn_bytes = bytes + 1024u;
-    static constexpr uint32_t tx_bytes = kOut ? R.used : 4u * D * D + 4u * D;
+    // record parts (see the kernel): split at d 128 only
+    static constexpr bool kSplit = (D == 128);
+    static constexpr uint32_t tx_whole = kOut ? R.used : 4u * D * D + 4u * D;
+    static constexpr uint32_t tx_a = kSplit ? 2u * D * D + (kOut ? 128u * D : 0u) : tx_whole;   // BS (Qt)
+    static constexpr uint32_t tx_b = 2u * D * D + (kOut ? R.used - R.PU : 4u * D);              // NC, (PU,) gamma
     static_assert(kStride % 1024u == 0u && Rec0 % 1024u == 0u, "tile alignment");
     static_assert(dyn_bytes + 128u <= 232448u, "shared memory budget");
 };
@@ -127,6 +131,7 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     constexpr RecordLayout R = record_layout(D);
     constexpr int ST = L::kStages;
     constexpr bool kOut = L::kOut;
+    constexpr bool kSplit = L::kSplit;
     // M of the state product: D rows (kLocal, D = 64: S and X stacked, 128 rows;
     // kLocal, D = 128: two products of 128 rows)
     constexpr int kMS = (MODE == kLocal && D == 64) ? 128 : D;
@@ -135,7 +140,9 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     constexpr int CW = D / 2;                                       // columns per thread
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align_smem<1024>(smem_raw);
-    __shared__ uint64_t full[ST];
+    // record parts of each stage: A = the MMA's operands (BS, and Qt with
+    // outputs), B = the rest (NC, gamma, and PU with outputs)
+    __shared__ uint64_t full_a[ST], full_b[ST];
     __shared__ uint64_t mma_bar;
 #ifdef GDR_TEST_WAIT_LIMIT_NS
     // test builds only: a barrier nothing arrives on, waited for with a short
@@ -181,42 +188,65 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         return records + ((size_t)slot * H + h) * R.bytes;
     };
     auto stage = [&](int s) { return sm + L::Rec0 + (uint32_t)s * L::kStride; };
-    // A CTA's bulk copies are served one after another and their issue can
-    // block for a while: one copy per record, issued where thread 0 has slack.
-    auto issue_copy = [&](int c) {       // thread 0 only
+    // At d 128 (two stages) each record comes in two parts with a barrier
+    // each, so that a stage's operand part can be refilled as soon as the MMA
+    // that read it has completed, a whole chunk earlier than the rest, whose
+    // last reader is the chunk's output step: part A = BS (and Qt), part B =
+    // NC, gamma (and PU) -- 15 % off the single pass at d 128.  At d 64 three
+    // stages hide the copies already and one copy per record (part A is the
+    // whole record, no part B) measured faster.  A CTA's bulk copies are served
+    // one after another.  Thread 0 only.
+    auto policy = [&]() {
+        // a record set that fits in L2: the state-only pass leaves it there
+        // for the replay, the passes with outputs read it for the last time
+        return (MODE == kLocal) ? l2_policy_evict_last() : l2_policy_evict_first();
+    };
+    auto copy = [&](uint8_t* dst, const uint8_t* src, uint32_t n, uint64_t* bar) {
+        if (keep_records) bulk_g2s_hint(dst, src, n, bar, policy());
+        else bulk_g2s(dst, src, n, bar);
+    };
+    auto issue_a = [&](int c) {
         const int s = c % ST;
         const uint8_t* r = record_of(c);
-        mbar_arrive_expect_tx(&full[s], L::tx_bytes);
-        if (keep_records) {
-            // a record set that fits in L2: the state-only pass leaves it there
-            // for the replay, the passes with outputs read it for the last time
-            const uint64_t pol = (MODE == kLocal) ? l2_policy_evict_last() : l2_policy_evict_first();
-            if (kOut) {
-                bulk_g2s_hint(stage(s), r, R.used, &full[s], pol);
-            } else {
-                bulk_g2s_hint(stage(s) + R.BS, r + R.BS, 4u * D * D, &full[s], pol);   // BS and NC
-                bulk_g2s_hint(stage(s) + L::kGamma, r + R.gamma, 4u * D, &full[s], pol);
-            }
-        } else if (kOut) {
-            bulk_g2s(stage(s), r, R.used, &full[s]);
+        mbar_arrive_expect_tx(&full_a[s], L::tx_a);
+        if (!kSplit && kOut) {
+            copy(stage(s), r, R.used, &full_a[s]);                               // the whole record
+        } else if (!kSplit) {
+            copy(stage(s) + R.BS, r + R.BS, 4u * D * D, &full_a[s]);              // BS and NC
+            copy(stage(s) + L::kGamma, r + R.gamma, 4u * D, &full_a[s]);
         } else {
-            bulk_g2s(stage(s) + R.BS, r + R.BS, 4u * D * D, &full[s]);     // BS and NC
-            bulk_g2s(stage(s) + L::kGamma, r + R.gamma, 4u * D, &full[s]);
+            copy(stage(s) + R.BS, r + R.BS, 2u * D * D, &full_a[s]);
+            if (kOut) copy(stage(s) + R.Qt, r + R.Qt, 128u * D, &full_a[s]);
         }
     };
+    auto issue_b = [&](int c) {
+        const int s = c % ST;
+        const uint8_t* r = record_of(c);
+        mbar_arrive_expect_tx(&full_b[s], L::tx_b);
+        copy(stage(s) + R.NC, r + R.NC, 2u * D * D, &full_b[s]);
+        if (kOut) copy(stage(s) + R.PU, r + R.PU, R.used - R.PU, &full_b[s]);        // PU and gamma
+        else copy(stage(s) + L::kGamma, r + R.gamma, 4u * D, &full_b[s]);
+    };
 
-    int copies_issued = 0;                                          // thread 0's bookkeeping
+    int a_issued = 0, b_issued = 0;                                 // thread 0's bookkeeping
     if (tid == 0) {
 #pragma unroll
-        for (int s = 0; s < ST; ++s) mbar_init(&full[s], 1);
+        for (int s = 0; s < ST; ++s) {
+            mbar_init(&full_a[s], 1);
+            mbar_init(&full_b[s], 1);
+        }
         mbar_init(&mma_bar, 1);
 #ifdef GDR_TEST_WAIT_LIMIT_NS
         mbar_init(&never_bar, 1);
 #endif
         fence_mbar_init();
         // the first records start arriving while the initial state is loaded
-        for (int c = 0; c < ST && c < nchunks; ++c) issue_copy(c);
-        copies_issued = min(ST, nchunks);
+        for (int c = 0; c < ST && c < nchunks; ++c) {
+            issue_a(c);
+            if (kSplit) issue_b(c);
+        }
+        a_issued = min(ST, nchunks);
+        b_issued = kSplit ? a_issued : 0;
     }
     if (warp == 0) {
         tmem_alloc(&tmem_slot, kTmemCols);
@@ -314,10 +344,10 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     };
 
     bool failed = false;
-    int copies_waited = 0, mmas_issued = 0;                         // thread 0's bookkeeping
+    int a_waited = 0, b_waited = 0, mmas_issued = 0;                // thread 0's bookkeeping
     if (tid == 0 && nchunks > 0) {
-        if (!mbar_wait(&full[0], 0)) failed = true;
-        copies_waited = 1;
+        if (!mbar_wait(&full_a[0], 0)) failed = true;
+        a_waited = 1;
         issue_mma(0);
         mmas_issued = 1;
     }
@@ -339,7 +369,8 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
 #pragma unroll
             for (int i = 0; i < kGateVec; ++i) gpre[i] = __ldg(g + i);
         }
-        if (!mbar_wait(&full[st], (uint32_t)(k / ST) & 1)) failed = true;
+        if (!mbar_wait(kSplit ? &full_b[st] : &full_a[st], (uint32_t)(k / ST) & 1)) failed = true;
+        if (tid == 0 && kSplit) b_waited = k + 1;
 #ifdef GDR_TEST_WAIT_LIMIT_NS
         if (k == 1 && !mbar_wait_for(&never_bar, 0u, (uint64_t)GDR_TEST_WAIT_LIMIT_NS)) failed = true;
 #endif
@@ -370,6 +401,11 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         if (!mbar_wait(&mma_bar, (uint32_t)k & 1)) failed = true;
         mmas_waited = k + 1;
         tc_fence_after_sync();
+        // the MMAs of chunk k have read this stage's part A: refill it
+        if (kSplit && tid == 0 && !failed && k + ST < nchunks) {
+            issue_a(k + ST);
+            a_issued = k + ST + 1;
+        }
 
         // ---- state: S = S * gamma + Z (+ NC for S rows), critical path ----------
 #pragma unroll
@@ -433,8 +469,8 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         if (__syncthreads_or(failed)) { failed = true; break; }
         tc_fence_after_sync();
         if (tid == 0 && k + 1 < nchunks) {
-            if (!mbar_wait(&full[(k + 1) % ST], (uint32_t)((k + 1) / ST) & 1)) failed = true;
-            copies_waited = k + 2;
+            if (!mbar_wait(&full_a[(k + 1) % ST], (uint32_t)((k + 1) / ST) & 1)) failed = true;
+            a_waited = k + 2;
             issue_mma(k + 1);
             mmas_issued = k + 2;
         }
@@ -442,8 +478,13 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         // barrier, its reads fenced before it) takes record k-1+ST now, under
         // the MMAs just issued
         if (ST >= 3 && tid == 0 && k >= 1 && k - 1 + ST < nchunks) {
-            issue_copy(k - 1 + ST);
-            copies_issued = k + ST;
+            if (kSplit) {
+                issue_b(k - 1 + ST);
+                b_issued = k + ST;
+            } else {
+                issue_a(k - 1 + ST);
+                a_issued = k + ST;
+            }
         }
 
         if (kOut) {
@@ -474,10 +515,11 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
 #pragma unroll
                     for (int e = 0; e < 8; ++e) ss = fmaf(ov[j + e], ov[j + e], ss);
                 }
-                // [half][row] partial sums, in this stage's Qt part: the O MMA
-                // that read it has completed, and the stage is refilled only
-                // after a later barrier (shared memory is full at d 128)
-                float* ssq = reinterpret_cast<float*>(stage(st) + R.Qt);
+                // [half][row] partial sums, in this stage's NC part: the state
+                // update that read it is done (barrier above), and part B is
+                // refilled only after a later barrier (shared memory is full
+                // at d 128; part A may already be refilling)
+                float* ssq = reinterpret_cast<float*>(stage(st) + R.NC);
                 if (oactive) ssq[half * 64 + orow] = ss;
                 pair_bar(sub);
                 const float tot = ss + (oactive ? ssq[(half ^ 1) * 64 + orow] : 0.f);
@@ -541,8 +583,13 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
             tc_fence_before_sync();
             if (__syncthreads_or(failed)) { failed = true; break; }
             if (tid == 0 && k + ST < nchunks) {
-                issue_copy(k + ST);
-                copies_issued = k + ST + 1;
+                if (kSplit) {
+                    issue_b(k + ST);
+                    b_issued = k + ST + 1;
+                } else {
+                    issue_a(k + ST);
+                    a_issued = k + ST + 1;
+                }
             }
         }
     }
@@ -569,7 +616,8 @@ state_pass_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     // exits (each of these waits is bounded too)
     if (tid == 0 && failed) {
         for (int c = mmas_waited; c < mmas_issued; ++c) mbar_wait(&mma_bar, (uint32_t)c & 1);
-        for (int c = copies_waited; c < copies_issued; ++c) mbar_wait(&full[c % ST], (uint32_t)(c / ST) & 1);
+        for (int c = a_waited; c < a_issued; ++c) mbar_wait(&full_a[c % ST], (uint32_t)(c / ST) & 1);
+        for (int c = b_waited; c < b_issued; ++c) mbar_wait(&full_b[c % ST], (uint32_t)(c / ST) & 1);
     }
     tc_fence_before_sync();
     __syncthreads();
