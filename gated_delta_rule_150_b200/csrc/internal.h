@@ -90,10 +90,13 @@ inline int segment_chunks(int n_seqs, int H, int64_t T, int D) {
     if (n_seqs <= 0 || T <= 0) return 0;
     const int64_t pairs = (int64_t)n_seqs * H;
     // about two CTAs per SM (the state-pass kernels fit two per SM at d = 64;
-    // at d = 128 two waves of shorter segments beat one wave of longer ones)
+    // at d = 128 two waves of shorter segments beat one wave of longer ones),
+    // never more: a CTA past the last full wave costs a whole segment's time
+    // (16 heads at d 128: 19 segments = 304 CTAs, 8 of them in a third wave)
     (void)D;
     const int64_t target_ctas = 2 * 148;
-    int64_t segs = (target_ctas + pairs - 1) / pairs;
+    int64_t segs = target_ctas / pairs;
+    if (segs <= 1) return 0;                  // enough pairs for one pass
     if (segs > 32) segs = 32;
     const int64_t avg_chunks = (T / n_seqs + kChunk - 1) / kChunk;
     int64_t sc = (avg_chunks + segs - 1) / segs;

@@ -180,6 +180,8 @@ def test_prefill_stage_range_and_kernel_count(L):
     # one intra-chunk kernel + one state pass, or + three when segmented
     assert gdr.kernel_count(1, 14, 64, 64, 8192) == 4          # 14 long heads: segmented
     assert gdr.kernel_count(32, 32, 128, 128, 278000) == 2     # many pairs: one pass
+    assert gdr.kernel_count(300, 1, 64, 64, 300 * 4096) == 2   # more pairs than the CTA target
+    assert gdr.kernel_count(1, 16, 128, 128, 65536, True) == 4  # 16 long heads: segmented
     assert gdr.kernel_count(1, 2, 64, 64, 256) == 2            # short: one pass
     assert gdr.kernel_count(1, 2, 64, 64, 0) == 1              # no tokens: state copy only
     assert gdr.kernel_count(1, 2, 96, 96, 256) == 0            # unsupported width
