@@ -144,6 +144,8 @@ struct IntraLayout {
                   "taps and halo fit in the Qg tile, outside the record staging");
     static_assert((64u * kLd * 4u) % 1024u == 0u, "Pt alignment");
     static_assert(Rec + rec_bytes <= Qgs, "record staging stays below Qgs");
+    static_assert(!(SCALAR && D == 128) || XA + op_bytes <= Rec + record_layout(D).Qt,
+                  "scalar d 128: the operand build writes only what the first record store reads");
     // TMEM is allocated once per persistent CTA: never more CTAs on an SM
     // than its 512 columns hold (2 x 256 at d 64, 1 x 512 at d 128)
     static_assert(3u * (dyn_bytes + 1088u) > 233472u, "at most two CTAs per SM");
@@ -514,6 +516,8 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     // per-channel decay at 8 warps: the next item's scan runs on warps 4-7
     // while warps 0-3 do the triangular solve
     constexpr bool kEarlyScan = !SCALAR && NT == 256;
+    // (see the wait for the previous record's stores at the operand build)
+    constexpr bool kLateRecWait = SCALAR && D == 128;
     bool pre_scanned = false;                                 // this item's g is already in sG
     bool failed = false;
 
@@ -635,7 +639,15 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     {
         const bool ok = !L::kStageQKV || mbar_wait(&in_bar[1], in_phase);
         in_phase ^= 1u;
-        if (tid == 0) bulk_wait_group_read0();
+        // the previous record's bulk stores have read the staging area the
+        // operands go to.  With the scalar gate at d 128 the operand build
+        // writes only the part of region 2 the first store read (BS, NC); the
+        // second store (Qt, PU, gamma) reaches into Bt and Kdt, written after
+        // the barrier below, so it is waited for just before that barrier.
+        if (tid == 0) {
+            if constexpr (kLateRecWait) bulk_wait_group_read<1>();
+            else bulk_wait_group_read0();
+        }
         if constexpr (RAW) {
             cp_async_wait_all();                       // the halo rows
 #pragma unroll
@@ -850,6 +862,9 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
             *reinterpret_cast<uint32_t*>(Kdt + o3) = pkd[e][0];
         }
     }
+    }
+    if constexpr (kLateRecWait) {
+        if (tid == 0) bulk_wait_group_read0();
     }
     fence_proxy_async_smem();
     tc_fence_before_sync();
