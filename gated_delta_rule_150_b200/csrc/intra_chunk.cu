@@ -137,7 +137,7 @@ struct IntraLayout {
     __host__ __device__ static constexpr uint32_t kt_off(int b) {
         return KT0 + 32u * D * (uint32_t)(b * (b + 1) / 2);
     }
-    static_assert(dyn_bytes <= 232448u, "shared memory budget");
+    static_assert(dyn_bytes + 256u <= 232448u, "shared memory budget (with the kernel's static variables)");
     static_assert(kPtotBytes <= r2, "scan partials fit in region 2");
     static_assert(!RAW || kStageQKV, "raw projections are staged");
     static_assert(!RAW || (Halo + halo_bytes <= Qgs + 128u * D && Taps >= Rec + rec_bytes),
