@@ -1045,8 +1045,9 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     __syncthreads();
 
     // region 1 and beta are free: stage the next item's beta (and its tiles
-    // if they were not requested during the A/P MMA) and look up the item
-    // after it (read by every thread at this item's end)
+    // if they were not requested during the A/P MMA) and, except with raw
+    // projections (below), look up the item after it (read by every thread at
+    // this item's end)
     if (warp == kLoadWarp) {
         const Item nxt = s_item[(iter + 1) & 1];
         fence_proxy_async_smem();             // this item's reads of region 1 come first
@@ -1055,7 +1056,7 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                                                  lane, keep_records != 0, !tiles_early);
             if (!tiles_early) ++tiles_issued;
         }
-        if (lane == 0)
+        if (!RAW && lane == 0)
             s_item[iter & 1] = nxt.idx >= 0 ? find_item(cu, n_seqs, H, n_items, nxt.idx + gridDim.x) : nxt;
     }
 
@@ -1068,6 +1069,17 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
     // item's log a, which the loader warp has just requested.
     uint8_t* Tb = sm + L::Tb;
     if (tid < 128) {
+        // with raw projections the item after the next one (a chain of
+        // dependent loads of cu_seqlens) is looked up by warp 2, idle while
+        // warps 0-1 solve the diagonal blocks, instead of by the loader warp:
+        // there the next item's decay scan (with its log_sigmoid) outlasts the
+        // solve, and the loader warp's share of it would finish last (1-2.5 %
+        // faster); with ready inputs the scan ends first and the lookup on
+        // warp 2 would only delay the solve (1 % slower)
+        if (RAW && tid == 64) {
+            const Item nxt = s_item[(iter + 1) & 1];
+            s_item[iter & 1] = nxt.idx >= 0 ? find_item(cu, n_seqs, H, n_items, nxt.idx + gridDim.x) : nxt;
+        }
         if (tid >= 64) {
             // (row, chunk) pairs of the zero blocks (b, j > b): 96 + 64 + 32
 #pragma unroll
