@@ -82,12 +82,14 @@ def test_status_reads_the_error_word():
     assert L.gdr_prefill_status(None, st) == 1
 
 
-@pytest.mark.parametrize("lengths,heads", [((640, 300, 100), 4),         # one pass (kFull)
-                                           ((3000,), 1)])               # segmented pass
-def test_timed_out_wait_is_reported_and_context_stays_usable(lengths, heads):
+@pytest.mark.parametrize("lengths,heads,d", [((640, 300, 100), 4, 64),     # one pass (kFull)
+                                             ((3000,), 1, 64),              # segmented pass
+                                             ((640, 300, 100), 4, 128),    # d 128: records in two parts
+                                             ((3000,), 1, 128)])
+def test_timed_out_wait_is_reported_and_context_stays_usable(lengths, heads, d):
     gdr = _gdr()
     LW = _wait_test_lib(gdr)
-    inp, dev = _case(lengths, heads)
+    inp, dev = _case(lengths, heads, d)
     o, fin, ws = _buffers(gdr, dev)
     st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     wsp = ctypes.c_void_p(ws.data_ptr())
