@@ -180,6 +180,21 @@ template <> struct Vec8<float> {
 
 __device__ __forceinline__ void load8f(const float* p, float (&x)[8]) { Vec8<float>::load(p, x); }
 
+// The conv taps of the raw path keep channel c in column g_col(c) of their
+// rows: the 16-byte words of a row are swizzled, word w at w ^ bit 3 of w (an
+// involution), so that the eight lanes of a quarter-warp reading a thread's
+// two words (channels 8 cg .. 8 cg + 7) hit each bank group once.
+__device__ __forceinline__ int swz_word(int w) { return w ^ ((w >> 3) & 1); }
+__device__ __forceinline__ int g_col(int c) { return 4 * swz_word(c >> 2) + (c & 3); }
+
+// Channels c0 .. c0 + 7 (c0 a multiple of 8) of a swizzled row.
+__device__ __forceinline__ void load8g(const float* row, int c0, float (&x)[8]) {
+    const int w = c0 >> 2;
+    const float4 a = *reinterpret_cast<const float4*>(row + 4 * swz_word(w));
+    const float4 b = *reinterpret_cast<const float4*>(row + 4 * swz_word(w + 1));
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+
 __device__ __forceinline__ uint4 pack8(const float (&x)[8]) {
     uint4 u;
     u.x = pack_bf16(x[0], x[1]); u.y = pack_bf16(x[2], x[3]);
@@ -652,7 +667,10 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
             cp_async_wait_all();                       // the halo rows
 #pragma unroll
             for (int u = 0; u < kTapsPer; ++u)         // the taps, tap-major
-                if (tid + u * NT < 3 * 4 * D) reinterpret_cast<float*>(sm + L::Taps)[tid + u * NT] = taps[u];
+                if (tid + u * NT < 3 * 4 * D) {
+                    const int i = tid + u * NT;     // (tensor, tap) row i / D, channel i % D
+                    reinterpret_cast<float*>(sm + L::Taps)[i - i % D + g_col(i % D)] = taps[u];
+                }
         }
         failed = __syncthreads_or(!ok);
         if (failed) {
@@ -674,24 +692,33 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
 #pragma unroll
         for (int tsr = 0; tsr < 3; ++tsr) {
             const InT* stg = reinterpret_cast<const InT*>(sm + (tsr == 0 ? L::sQ : (tsr == 1 ? L::sK : L::sV)));
-            const float* wsm = reinterpret_cast<const float*>(sm + L::Taps) + (size_t)tsr * 4 * D + c0;
+            const float* wsm = reinterpret_cast<const float*>(sm + L::Taps) + (size_t)tsr * 4 * D;
             float w[8][4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 float t8[8];
-                load8f(wsm + (size_t)j * D, t8);
+                load8g(wsm + (size_t)j * D, c0, t8);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) w[e][j] = t8[e];
             }
+            // the RPT + 3 raw rows r0 - 3 .. r0 + RPT - 1 this thread's rows read,
+            // each loaded once
+            const InT* hal = reinterpret_cast<const InT*>(sm + L::Halo) + (size_t)tsr * 3 * D;
+            uint4 xr[RPT + 3];                    // as stored (bf16): raw projections are bf16
+#pragma unroll
+            for (int i = 0; i < RPT + 3; ++i) {
+                const int rr = r0 - 3 + i;
+                xr[i] = *reinterpret_cast<const uint4*>(rr >= 0 ? stg + (size_t)rr * D + c0 : hal + (size_t)(rr + 3) * D + c0);
+            }
 #pragma unroll
             for (int u = 0; u < RPT; ++u) {
-                const int r = r0 + u;
-                float x[4][8];                    // x[j]: raw row r - 3 + j
+                float x[4][8];                    // x[j]: raw row r0 + u - 3 + j
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    const int rr = r - 3 + j;
-                    const InT* hal = reinterpret_cast<const InT*>(sm + L::Halo) + (size_t)tsr * 3 * D;
-                    Vec8<InT>::load(rr >= 0 ? stg + (size_t)rr * D + c0 : hal + (size_t)(rr + 3) * D + c0, x[j]);
+                    const uint4 q4 = xr[u + j];
+                    const float2 a = unpack_bf16(q4.x), b = unpack_bf16(q4.y), c = unpack_bf16(q4.z), d = unpack_bf16(q4.w);
+                    x[j][0] = a.x; x[j][1] = a.y; x[j][2] = b.x; x[j][3] = b.y;
+                    x[j][4] = c.x; x[j][5] = c.y; x[j][6] = d.x; x[j][7] = d.y;
                 }
                 float yy[8];
 #pragma unroll
