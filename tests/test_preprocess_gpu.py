@@ -99,12 +99,20 @@ def test_preprocess_no_tokens_is_noop():
     assert out["q"].shape == (0, 2, 64)
 
 
-def _fused_vs_chain(w, lengths, snap=0, init=False):
+def _fused_vs_chain(w, lengths, snap=0, init=False, steep=None):
     """The fused prefill from raw projections against (a) the oracle's prefill
     of the oracle's activations (cast to bf16) at the prefill bound 2e-2 max
-    |ref|, and (b) the two-kernel chain preprocess -> prefill."""
+    |ref|, and (b) the two-kernel chain preprocess -> prefill.  ``steep``:
+    (tokens, channels) whose a_raw is set to -40 (log a near -35)."""
     gdr = _gdr()
     inp = wl.make_preprocess_inputs(w, lengths=lengths)
+    if steep is not None:
+        toks, chans = steep
+        for t in toks:
+            if w.scalar_decay:
+                inp["a_raw"][t, :] = -40.0
+            else:
+                inp["a_raw"][t, :, chans] = -40.0
     d = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in inp.items()}
     H, dd = w.n_heads, w.d_k
     n = len(inp["lengths"])
@@ -148,3 +156,16 @@ def test_fused_prefill_from_projections(d, scalar):
 def test_fused_prefill_graft_layer_shape():
     """The graft layer's shape (8192 tokens x 14 heads x 64), one sequence."""
     _fused_vs_chain(wl.PREPROCESS, None)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("scalar", [False, True])
+def test_fused_prefill_steep_decay(d, scalar):
+    """Decays below the factored range (log a < -10) inside the fused path,
+    on enough chunks (6 heads x 64 chunks) that most CTAs take a second item,
+    whose decay is scanned during the first item's solve: chunk j holds one
+    steep row at position 3, 25 or 47 (j % 4 = 0, 1, 2; none for j % 4 = 3),
+    so that each row range of that scan meets one, next to chunks without."""
+    w = wl.shrink(wl.PREPROCESS, n_heads=6, d_k=d, d_v=d, scalar_decay=scalar, seed=1111)
+    toks = [64 * j + (3, 25, 47)[j % 4] for j in range(64) if j % 4 != 3]
+    _fused_vs_chain(w, [4096], steep=(toks, [1, d // 2 + 3, d - 1]))
