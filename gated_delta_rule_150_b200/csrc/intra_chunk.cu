@@ -693,13 +693,13 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         for (int tsr = 0; tsr < 3; ++tsr) {
             const InT* stg = reinterpret_cast<const InT*>(sm + (tsr == 0 ? L::sQ : (tsr == 1 ? L::sK : L::sV)));
             const float* wsm = reinterpret_cast<const float*>(sm + L::Taps) + (size_t)tsr * 4 * D;
-            float w[8][4];
+            float2 w[4][4];                       // [tap][channel pair]
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 float t8[8];
                 load8g(wsm + (size_t)j * D, c0, t8);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) w[e][j] = t8[e];
+                for (int p = 0; p < 4; ++p) w[j][p] = make_float2(t8[2 * p], t8[2 * p + 1]);
             }
             // the RPT + 3 raw rows r0 - 3 .. r0 + RPT - 1 this thread's rows read,
             // each loaded once
@@ -712,35 +712,32 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
             }
 #pragma unroll
             for (int u = 0; u < RPT; ++u) {
-                float x[4][8];                    // x[j]: raw row r0 + u - 3 + j
+                // x of tap j: raw row r0 + u - 3 + j, as channel pairs, on
+                // packed fp32 FMAs (__ffma2_rn: two fmaf per instruction)
+                float2 acc[4];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
+                for (int j = 3; j >= 0; --j) {
                     const uint4 q4 = xr[u + j];
-                    const float2 a = unpack_bf16(q4.x), b = unpack_bf16(q4.y), c = unpack_bf16(q4.z), d = unpack_bf16(q4.w);
-                    x[j][0] = a.x; x[j][1] = a.y; x[j][2] = b.x; x[j][3] = b.y;
-                    x[j][4] = c.x; x[j][5] = c.y; x[j][6] = d.x; x[j][7] = d.y;
-                }
-                float yy[8];
+                    const float2 x2[4] = {unpack_bf16(q4.x), unpack_bf16(q4.y), unpack_bf16(q4.z), unpack_bf16(q4.w)};
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    float acc = w[e][3] * x[3][e];
-                    acc = fmaf(w[e][2], x[2][e], acc);
-                    acc = fmaf(w[e][1], x[1][e], acc);
-                    acc = fmaf(w[e][0], x[0][e], acc);
-                    yy[e] = acc;
+                    for (int p = 0; p < 4; ++p)
+                        acc[p] = (j == 3) ? __fmul2_rn(w[3][p], x2[p]) : __ffma2_rn(w[j][p], x2[p], acc[p]);
                 }
                 if (tsr < 2) {
                     // L2 norm over the row's D channels: CG consecutive lanes
-                    float ss = 0.f;
+                    float2 s2 = __fmul2_rn(acc[0], acc[0]);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) ss = fmaf(yy[e], yy[e], ss);
+                    for (int p = 1; p < 4; ++p) s2 = __ffma2_rn(acc[p], acc[p], s2);
+                    float ss = s2.x + s2.y;
 #pragma unroll
                     for (int m = 1; m < CG; m <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
                     const float inv = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
+                    const float2 inv2 = make_float2(inv, inv);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) yy[e] *= inv;
+                    for (int p = 0; p < 4; ++p) acc[p] = __fmul2_rn(acc[p], inv2);
                 }
-                y[tsr][u] = pack8(yy);
+                y[tsr][u] = make_uint4(pack_bf16(acc[0].x, acc[0].y), pack_bf16(acc[1].x, acc[1].y),
+                                       pack_bf16(acc[2].x, acc[2].y), pack_bf16(acc[3].x, acc[3].y));
             }
         }
         __syncthreads();                      // every raw row has been read
@@ -798,16 +795,26 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
         }
         float xq[8], xk[8], kk0[8], b1[8], qg[8], kd[8];
         if (!SCALAR && !bad_chunk) {
+            // channel pairs on sm_100's packed fp32 multiply (__fmul2_rn, each
+            // lane rounded like fmul: the same values as scalar code, 2.4 %
+            // less intra time at d 128)
+            const float2 sc2 = make_float2(scale, scale), br2 = make_float2(br, br);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float d = gr[e] - mj[e];
-                const float F = __expf(d), Fi = __expf(-d);
-                xq[e] = scale * qv[e] * F;
-                xk[e] = kv[e] * F;
-                kk0[e] = kv[e] * Fi;
-                b1[e] = br * xk[e] * em[e];
-                qg[e] = xq[e] * em[e];
-                kd[e] = kk0[e] * eld[e];
+            for (int p = 0; p < 4; ++p) {
+                const int e = 2 * p;
+                const float d0 = gr[e] - mj[e], d1 = gr[e + 1] - mj[e + 1];
+                const float2 F = make_float2(__expf(d0), __expf(d1)), Fi = make_float2(__expf(-d0), __expf(-d1));
+                const float2 q2 = make_float2(qv[e], qv[e + 1]), k2 = make_float2(kv[e], kv[e + 1]);
+                const float2 em2 = make_float2(em[e], em[e + 1]), eld2 = make_float2(eld[e], eld[e + 1]);
+                const float2 xq2 = __fmul2_rn(__fmul2_rn(sc2, q2), F);
+                const float2 xk2 = __fmul2_rn(k2, F);
+                const float2 kk2 = __fmul2_rn(k2, Fi);
+                const float2 b12 = __fmul2_rn(__fmul2_rn(br2, xk2), em2);
+                const float2 qg2 = __fmul2_rn(xq2, em2);
+                const float2 kd2 = __fmul2_rn(kk2, eld2);
+                xq[e] = xq2.x; xq[e + 1] = xq2.y; xk[e] = xk2.x; xk[e + 1] = xk2.y;
+                kk0[e] = kk2.x; kk0[e + 1] = kk2.y; b1[e] = b12.x; b1[e + 1] = b12.y;
+                qg[e] = qg2.x; qg[e + 1] = qg2.y; kd[e] = kd2.x; kd[e + 1] = kd2.y;
             }
         } else if (SCALAR) {
             const float G = __expf(gr[0]), Ed = __expf(gl[0] - gr[0]);   // one gate per row
@@ -842,7 +849,12 @@ intra_chunk_kernel(const int32_t* __restrict__ cu, int n_seqs, int H,
                 if (b < jb) continue;
                 float kb[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) kb[e] = (b == jb) ? kk0[e] : kk0[e] * ecross[b][e];
+                for (int p = 0; p < 4; ++p) {
+                    const float2 r2 = (b == jb) ? make_float2(kk0[2 * p], kk0[2 * p + 1])
+                                                : __fmul2_rn(make_float2(kk0[2 * p], kk0[2 * p + 1]),
+                                                             make_float2(ecross[b][2 * p], ecross[b][2 * p + 1]));
+                    kb[2 * p] = r2.x; kb[2 * p + 1] = r2.y;
+                }
                 *reinterpret_cast<uint4*>(sm + L::kt_off(b) + sw128_chunk(16 * (b + 1), r, cg)) = pack8(kb);
             }
         }

@@ -148,24 +148,31 @@ decode_draft_kernel(int H, int K, const T* __restrict__ q, const T* __restrict__
 #pragma unroll
         for (int p = 0; p < PASSES; ++p) {
             const int row = row0 + kRowsPerPass * p;
-            float pk = 0.f, pq = 0.f;
+            // column pairs on packed fp32 (__fmul2_rn, __ffma2_rn; the k and q
+            // dot products summed as two interleaved halves): 1 % faster
+            float2 pk2 = make_float2(0.f, 0.f), pq2 = make_float2(0.f, 0.f);
+            float2 xl[NV], xh[NV];
 #pragma unroll
             for (int i = 0; i < NV; ++i) {
-                float4& x = s[p][i];
-                x.x *= aa[i].x; x.y *= aa[i].y; x.z *= aa[i].z; x.w *= aa[i].w;
-                pk += x.x * cur.k[i].x + x.y * cur.k[i].y + x.z * cur.k[i].z + x.w * cur.k[i].w;
-                pq += x.x * qq[i].x + x.y * qq[i].y + x.z * qq[i].z + x.w * qq[i].w;
+                const float4 x = s[p][i];
+                xl[i] = __fmul2_rn(make_float2(x.x, x.y), make_float2(aa[i].x, aa[i].y));
+                xh[i] = __fmul2_rn(make_float2(x.z, x.w), make_float2(aa[i].z, aa[i].w));
+                pk2 = __ffma2_rn(xl[i], make_float2(cur.k[i].x, cur.k[i].y), pk2);
+                pk2 = __ffma2_rn(xh[i], make_float2(cur.k[i].z, cur.k[i].w), pk2);
+                pq2 = __ffma2_rn(xl[i], make_float2(qq[i].x, qq[i].y), pq2);
+                pq2 = __ffma2_rn(xh[i], make_float2(qq[i].z, qq[i].w), pq2);
             }
-            pk = sum16(pk);
-            pq = sum16(pq);
+            const float pk = sum16(pk2.x + pk2.y);
+            const float pq = sum16(pq2.x + pq2.y);
             const float d = cur.beta * (cur.v[p] - pk);
+            const float2 d2 = make_float2(d, d);
 #pragma unroll
             for (int i = 0; i < NV; ++i) {
-                float4& x = s[p][i];
-                x.x += d * cur.k[i].x; x.y += d * cur.k[i].y;
-                x.z += d * cur.k[i].z; x.w += d * cur.k[i].w;
+                const float2 lo = __ffma2_rn(d2, make_float2(cur.k[i].x, cur.k[i].y), xl[i]);
+                const float2 hi = __ffma2_rn(d2, make_float2(cur.k[i].z, cur.k[i].w), xh[i]);
+                s[p][i] = make_float4(lo.x, lo.y, hi.x, hi.y);
                 // kept states are written once and mostly never read again
-                __stcs(reinterpret_cast<float4*>(St + (size_t)row * DK + 4 * (lane16 + kTPR * i)), x);
+                __stcs(reinterpret_cast<float4*>(St + (size_t)row * DK + 4 * (lane16 + kTPR * i)), s[p][i]);
             }
             if (lane16 == 0) o[tok * DV + row] = pq + d * kq;
         }
