@@ -36,15 +36,6 @@ __device__ __forceinline__ float to_f<float>(float x) { return x; }
 template <>
 __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
 
-// Four consecutive elements starting at p (16-byte aligned for fp32, 8 for bf16).
-__device__ __forceinline__ float4 load4(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
-__device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
-    const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
-    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
-    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
-    return make_float4(a.x, a.y, b.x, b.y);
-}
-
 __device__ __forceinline__ float sum16(float x) {
 #pragma unroll
     for (int m = 8; m >= 1; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
@@ -61,72 +52,109 @@ struct DecodeGate {
     float eps;
 };
 
-// One CTA per (sequence, head).  Thread t handles row group t / 16 and the
-// float4 columns {t % 16 + 16 i}.  DK/64 float4 per thread per row.
-template <typename T, int DK, int DV, bool SCALAR, bool GATED>
-__global__ void __launch_bounds__(kThreads)
-decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
-                   const float* __restrict__ beta, const float* __restrict__ log_a, float scale,
-                   float* __restrict__ state, float* __restrict__ o, const DecodeGate<T> og) {
-    constexpr int NV = DK / (4 * kTPR);        // float4 per thread per row: 1 or 2
-    constexpr int PASSES = DV / kRowsPerPass;  // 4 or 8
-    pdl_launch_dependents();
-    pdl_wait();                                // the previous kernel's writes are visible
-    const int bh = blockIdx.x;
-    const int lane16 = threadIdx.x % kTPR;
-    const int rgrp = threadIdx.x / kTPR;
+// Four consecutive elements as loaded (16-byte aligned for fp32, 8 for
+// bf16), converted only where they are used, so that every load of a step is
+// issued before the first of them is waited for.
+template <typename T> struct Raw4;
+template <> struct Raw4<float> {
+    float4 u;
+    __device__ __forceinline__ void load(const float* p) { u = __ldg(reinterpret_cast<const float4*>(p)); }
+    __device__ __forceinline__ float4 get() const { return u; }
+};
+template <> struct Raw4<__nv_bfloat16> {
+    uint2 u;
+    __device__ __forceinline__ void load(const __nv_bfloat16* p) { u = __ldg(reinterpret_cast<const uint2*>(p)); }
+    __device__ __forceinline__ float4 get() const {
+        const float2 a = unpack_bf16(u.x), b = unpack_bf16(u.y);
+        return make_float4(a.x, a.y, b.x, b.y);
+    }
+};
 
+// Everything one thread reads for one (sequence, head): its state rows
+// (row group rgrp, float4 columns lane16 + 16 i) and the token's inputs,
+// all requested at once (the state rows no longer wait behind the inputs'
+// round trip and the decay's exponentials: 2.5 % more state bandwidth at
+// d 128, the same at d 64).
+template <typename T, int DK, int DV, bool SCALAR>
+struct StepLoads {
+    static constexpr int NV = DK / (4 * kTPR);        // float4 per thread per row: 1 or 2
+    static constexpr int PASSES = DV / kRowsPerPass;  // 4 or 8
+    Raw4<T> k[NV], q[NV];
+    float4 la[NV];                                    // log a (scalar gate: la[0].x)
+    T v[PASSES];
+    float beta;
+    float4 s[PASSES][NV];
+    __device__ __forceinline__ void issue(int bh, const T* __restrict__ q_, const T* __restrict__ k_,
+                                          const T* __restrict__ v_, const float* __restrict__ beta_,
+                                          const float* __restrict__ log_a_, const float* state,
+                                          int lane16, int rgrp) {
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            const int c = 4 * (lane16 + kTPR * i);
+            k[i].load(k_ + (size_t)bh * DK + c);
+            q[i].load(q_ + (size_t)bh * DK + c);
+            if (!SCALAR) la[i] = __ldg(reinterpret_cast<const float4*>(log_a_ + (size_t)bh * DK + c));
+        }
+        if (SCALAR) la[0].x = __ldg(log_a_ + bh);
+        beta = __ldg(beta_ + bh);
+        const float* S = state + (size_t)bh * DV * DK;
+#pragma unroll
+        for (int p = 0; p < PASSES; ++p)
+#pragma unroll
+            for (int i = 0; i < NV; ++i)
+                s[p][i] = *reinterpret_cast<const float4*>(S + (size_t)(rgrp + kRowsPerPass * p) * DK +
+                                                           4 * (lane16 + kTPR * i));
+#pragma unroll
+        for (int p = 0; p < PASSES; ++p) v[p] = v_[(size_t)bh * DV + rgrp + kRowsPerPass * p];
+    }
+};
+
+// The step of one (sequence, head) from its loads: state rows updated and
+// written back, outputs (with the gate epilogue) stored.
+template <typename T, int DK, int DV, bool SCALAR, bool GATED>
+__device__ __forceinline__ void step_one(const StepLoads<T, DK, DV, SCALAR>& in, int bh, float scale,
+                                         float* __restrict__ state, float* __restrict__ o,
+                                         const DecodeGate<T>& og, int lane16, int rgrp) {
+    constexpr int NV = StepLoads<T, DK, DV, SCALAR>::NV;
+    constexpr int PASSES = StepLoads<T, DK, DV, SCALAR>::PASSES;
     float4 kk[NV], qq[NV], aa[NV];
     float kq_part = 0.f;
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
-        const int c = 4 * (lane16 + kTPR * i);
-        kk[i] = load4(k + (size_t)bh * DK + c);
-        float4 qv = load4(q + (size_t)bh * DK + c);
+        kk[i] = in.k[i].get();
+        const float4 qv = in.q[i].get();
         qq[i] = make_float4(qv.x * scale, qv.y * scale, qv.z * scale, qv.w * scale);
         if (SCALAR) {
-            const float a = expf(__ldg(log_a + bh));
+            const float a = expf(in.la[0].x);
             aa[i] = make_float4(a, a, a, a);
         } else {
-            const float4 la = load4(log_a + (size_t)bh * DK + c);
+            const float4 la = in.la[i];
             aa[i] = make_float4(expf(la.x), expf(la.y), expf(la.z), expf(la.w));
         }
         kq_part += kk[i].x * qq[i].x + kk[i].y * qq[i].y + kk[i].z * qq[i].z + kk[i].w * qq[i].w;
     }
     const float kq = sum16(kq_part);
-    const float b = __ldg(beta + bh);
-
     float* S = state + (size_t)bh * DV * DK;
-    // Issue every load of this thread's rows first (memory-level parallelism).
-    float4 s[PASSES][NV];
-#pragma unroll
-    for (int p = 0; p < PASSES; ++p)
-#pragma unroll
-        for (int i = 0; i < NV; ++i)
-            s[p][i] = *reinterpret_cast<const float4*>(S + (size_t)(rgrp + kRowsPerPass * p) * DK +
-                                                       4 * (lane16 + kTPR * i));
-    float vv[PASSES];
-#pragma unroll
-    for (int p = 0; p < PASSES; ++p) vv[p] = to_f<T>(v[(size_t)bh * DV + rgrp + kRowsPerPass * p]);
-
     float ov[PASSES];                          // this row group's outputs (epilogue)
 #pragma unroll
     for (int p = 0; p < PASSES; ++p) {
         const int row = rgrp + kRowsPerPass * p;
         float pk = 0.f, pq = 0.f;
+        float4 s[NV];
 #pragma unroll
         for (int i = 0; i < NV; ++i) {
-            float4& x = s[p][i];
+            float4 x = in.s[p][i];
             x.x *= aa[i].x; x.y *= aa[i].y; x.z *= aa[i].z; x.w *= aa[i].w;
             pk += x.x * kk[i].x + x.y * kk[i].y + x.z * kk[i].z + x.w * kk[i].w;
             pq += x.x * qq[i].x + x.y * qq[i].y + x.z * qq[i].z + x.w * qq[i].w;
+            s[i] = x;
         }
         pk = sum16(pk);
         pq = sum16(pq);
-        const float d = b * (vv[p] - pk);
+        const float d = in.beta * (to_f<T>(in.v[p]) - pk);
 #pragma unroll
         for (int i = 0; i < NV; ++i) {
-            float4& x = s[p][i];
+            float4& x = s[i];
             x.x += d * kk[i].x; x.y += d * kk[i].y; x.z += d * kk[i].z; x.w += d * kk[i].w;
             *reinterpret_cast<float4*>(S + (size_t)row * DK + 4 * (lane16 + kTPR * i)) = x;
         }
@@ -154,6 +182,22 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
             o[(size_t)bh * DV + row] = ov[p] * rstd * __ldg(og.weight + row) * sig;
         }
     }
+}
+
+// One CTA per (sequence, head).
+template <typename T, int DK, int DV, bool SCALAR, bool GATED>
+__global__ void __launch_bounds__(kThreads)
+decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+                   const float* __restrict__ beta, const float* __restrict__ log_a, float scale,
+                   float* __restrict__ state, float* __restrict__ o, const DecodeGate<T> og) {
+    pdl_launch_dependents();
+    pdl_wait();                                // the previous kernel's writes are visible
+    const int lane16 = threadIdx.x % kTPR;
+    const int rgrp = threadIdx.x / kTPR;
+    const int bh = blockIdx.x;
+    StepLoads<T, DK, DV, SCALAR> in;
+    in.issue(bh, q, k, v, beta, log_a, state, lane16, rgrp);
+    step_one<T, DK, DV, SCALAR, GATED>(in, bh, scale, state, o, og, lane16, rgrp);
 }
 
 template <typename T, int DK, int DV, bool GATED>
