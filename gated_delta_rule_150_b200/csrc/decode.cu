@@ -184,9 +184,13 @@ __device__ __forceinline__ void step_one(const StepLoads<T, DK, DV, SCALAR>& in,
     }
 }
 
-// One CTA per (sequence, head).
+// One CTA per (sequence, head).  The explicit minimum of one CTA per SM
+// leaves the register allocation free to keep every load in flight (128
+// registers at d 128, 53 at d 64; measured 2.5 % faster at d 128 than the
+// tighter default allocation of 114, and no slower at d 64 with 4 CTAs per SM
+// instead of 6).
 template <typename T, int DK, int DV, bool SCALAR, bool GATED>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 1)
 decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                    const float* __restrict__ beta, const float* __restrict__ log_a, float scale,
                    float* __restrict__ state, float* __restrict__ o, const DecodeGate<T> og) {

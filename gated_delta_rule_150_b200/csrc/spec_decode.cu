@@ -35,29 +35,45 @@ __device__ __forceinline__ float to_f<float>(float x) { return x; }
 template <>
 __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
 
-__device__ __forceinline__ float4 load4(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
-__device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
-    const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
-    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
-    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
-    return make_float4(a.x, a.y, b.x, b.y);
-}
-
 __device__ __forceinline__ float sum16(float x) {
 #pragma unroll
     for (int m = 8; m >= 1; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
     return x;
 }
 
-// One token's inputs as seen by one thread: its float4 columns of k, q and
-// log a, the v entries of its rows (PASSES rows from row0, 16 apart),
-// and beta.
+// Four consecutive elements as loaded (16-byte aligned for fp32, 8 for
+// bf16), converted where they are used: the next token's loads are issued
+// before this token is computed, and a conversion right after a load would
+// wait for it there (5 % faster draft than converting at the load).
+template <typename T> struct Raw4;
+template <> struct Raw4<float> {
+    float4 u;
+    __device__ __forceinline__ void load(const float* p) { u = __ldg(reinterpret_cast<const float4*>(p)); }
+    __device__ __forceinline__ float4 get() const { return u; }
+};
+template <> struct Raw4<__nv_bfloat16> {
+    uint2 u;
+    __device__ __forceinline__ void load(const __nv_bfloat16* p) { u = __ldg(reinterpret_cast<const uint2*>(p)); }
+    __device__ __forceinline__ float4 get() const {
+        const float2 a = unpack_bf16(u.x), b = unpack_bf16(u.y);
+        return make_float4(a.x, a.y, b.x, b.y);
+    }
+};
+
+// One token's inputs as seen by one thread, as loaded: its float4 columns of
+// k, q and log a (a scalar gate: la[0].x), the v entries of its rows (PASSES
+// rows from row0, 16 apart), and beta.
 template <typename T, int DK, int DV, int PASSES, bool SCALAR>
 struct TokenIn {
     static constexpr int NV = DK / (4 * kTPR);
-    float4 k[NV], q[NV], la[NV];
-    float v[PASSES];
+    Raw4<T> k[NV], q[NV];
+    float4 la[NV];
+    T v[PASSES];
     float beta;
+    __device__ __forceinline__ float4 decay(int i) const {
+        const float4 x = SCALAR ? make_float4(la[0].x, la[0].x, la[0].x, la[0].x) : la[i];
+        return make_float4(expf(x.x), expf(x.y), expf(x.z), expf(x.w));
+    }
 
     __device__ __forceinline__ void load(const T* __restrict__ q_, const T* __restrict__ k_,
                                          const T* __restrict__ v_, const float* __restrict__ beta_,
@@ -66,17 +82,13 @@ struct TokenIn {
 #pragma unroll
         for (int i = 0; i < NV; ++i) {
             const int c = 4 * (lane16 + kTPR * i);
-            k[i] = load4(k_ + tok * DK + c);
-            q[i] = load4(q_ + tok * DK + c);
-            if (SCALAR) {
-                const float x = __ldg(log_a_ + tok);
-                la[i] = make_float4(x, x, x, x);
-            } else {
-                la[i] = load4(log_a_ + tok * DK + c);
-            }
+            k[i].load(k_ + tok * DK + c);
+            q[i].load(q_ + tok * DK + c);
+            if (!SCALAR) la[i] = __ldg(reinterpret_cast<const float4*>(log_a_ + tok * DK + c));
         }
+        if (SCALAR) la[0].x = __ldg(log_a_ + tok);
 #pragma unroll
-        for (int p = 0; p < PASSES; ++p) v[p] = to_f<T>(v_[tok * DV + row0 + kRowsPerPass * p]);
+        for (int p = 0; p < PASSES; ++p) v[p] = v_[tok * DV + row0 + kRowsPerPass * p];
         beta = __ldg(beta_ + tok);
     }
 };
@@ -88,8 +100,8 @@ struct TokenIn {
 // (b K + t) H + h of q, k, v, beta, log a, o and token_states; the next
 // token's inputs are loaded while this one computes.
 // At d 64 the kernel is capped at 64 registers so that four CTAs fit on an SM
-// (7 % faster on B200 than three CTAs at 78 registers, despite a 24-byte
-// spill in the bf16 per-channel case); wider states keep their registers.
+// (7 % faster on B200 than three CTAs at 78 registers; the fp32 per-channel
+// case spills 68 bytes); wider states keep their registers.
 template <int DK, int DV>
 constexpr int draft_min_ctas() { return (DK == 64 && DV == 64) ? 4 : 1; }
 
@@ -131,16 +143,15 @@ decode_draft_kernel(int H, int K, const T* __restrict__ q, const T* __restrict__
         const size_t tok = tok0 + (size_t)t * H;
         if (t + 1 < K) nxt.load(q, k, v, beta, log_a, tok + H, lane16, row0);
 
-        float4 aa[NV], qq[NV];
+        float4 aa[NV], qq[NV], kk[NV];
         float kq_part = 0.f;
 #pragma unroll
         for (int i = 0; i < NV; ++i) {
-            aa[i] = make_float4(expf(cur.la[i].x), expf(cur.la[i].y), expf(cur.la[i].z),
-                                expf(cur.la[i].w));
-            qq[i] = make_float4(cur.q[i].x * scale, cur.q[i].y * scale, cur.q[i].z * scale,
-                                cur.q[i].w * scale);
-            kq_part += cur.k[i].x * qq[i].x + cur.k[i].y * qq[i].y + cur.k[i].z * qq[i].z +
-                       cur.k[i].w * qq[i].w;
+            aa[i] = cur.decay(i);
+            const float4 qv = cur.q[i].get();
+            kk[i] = cur.k[i].get();
+            qq[i] = make_float4(qv.x * scale, qv.y * scale, qv.z * scale, qv.w * scale);
+            kq_part += kk[i].x * qq[i].x + kk[i].y * qq[i].y + kk[i].z * qq[i].z + kk[i].w * qq[i].w;
         }
         const float kq = sum16(kq_part);
 
@@ -157,19 +168,19 @@ decode_draft_kernel(int H, int K, const T* __restrict__ q, const T* __restrict__
                 const float4 x = s[p][i];
                 xl[i] = __fmul2_rn(make_float2(x.x, x.y), make_float2(aa[i].x, aa[i].y));
                 xh[i] = __fmul2_rn(make_float2(x.z, x.w), make_float2(aa[i].z, aa[i].w));
-                pk2 = __ffma2_rn(xl[i], make_float2(cur.k[i].x, cur.k[i].y), pk2);
-                pk2 = __ffma2_rn(xh[i], make_float2(cur.k[i].z, cur.k[i].w), pk2);
+                pk2 = __ffma2_rn(xl[i], make_float2(kk[i].x, kk[i].y), pk2);
+                pk2 = __ffma2_rn(xh[i], make_float2(kk[i].z, kk[i].w), pk2);
                 pq2 = __ffma2_rn(xl[i], make_float2(qq[i].x, qq[i].y), pq2);
                 pq2 = __ffma2_rn(xh[i], make_float2(qq[i].z, qq[i].w), pq2);
             }
             const float pk = sum16(pk2.x + pk2.y);
             const float pq = sum16(pq2.x + pq2.y);
-            const float d = cur.beta * (cur.v[p] - pk);
+            const float d = cur.beta * (to_f<T>(cur.v[p]) - pk);
             const float2 d2 = make_float2(d, d);
 #pragma unroll
             for (int i = 0; i < NV; ++i) {
-                const float2 lo = __ffma2_rn(d2, make_float2(cur.k[i].x, cur.k[i].y), xl[i]);
-                const float2 hi = __ffma2_rn(d2, make_float2(cur.k[i].z, cur.k[i].w), xh[i]);
+                const float2 lo = __ffma2_rn(d2, make_float2(kk[i].x, kk[i].y), xl[i]);
+                const float2 hi = __ffma2_rn(d2, make_float2(kk[i].z, kk[i].w), xh[i]);
                 s[p][i] = make_float4(lo.x, lo.y, hi.x, hi.y);
                 // kept states are written once and mostly never read again
                 __stcs(reinterpret_cast<float4*>(St + (size_t)row * DK + 4 * (lane16 + kTPR * i)), s[p][i]);
