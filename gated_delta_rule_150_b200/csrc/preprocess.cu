@@ -20,8 +20,9 @@
 // conv), the block's a_raw rows, beta_raw and the head's conv taps and gate
 // bias: about 45 KB per CTA at d 64, all in flight at once, so the kernel
 // keeps enough bytes moving to stream at HBM speed.  Then D / 8 threads own
-// a token (eight channels each) and compute its outputs from shared memory;
-// a tap that reaches before the token's sequence start is skipped.  L2 norms
+// a token (eight channels each; at d 128 two consecutive tokens) and compute
+// its outputs from shared memory, one tensor after another; a tap that
+// reaches before the token's sequence start is skipped.  L2 norms
 // are shuffle sums over the token's D / 8 lanes.  Outputs go straight to
 // global memory, each token row written by D / 8 neighbouring threads.  HBM
 // traffic: x_q, x_k, x_v, beta_raw and a_raw read (plus a three-row halo per
@@ -36,6 +37,12 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kTok = 32;            // tokens per CTA (32 measured faster than 64)
+// Consecutive tokens per thread: at d 128 a thread takes two, so each staged
+// raw row is unpacked for both (1.34 against 1.39 ms on 8 varlen sequences x
+// 32 heads); at d 64 one (two tokens per thread took twice the registers
+// there for no gain).
+template <int D>
+__host__ __device__ constexpr int run_for() { return D == 128 ? 2 : 1; }
 
 template <typename T, int D, bool SCALAR>
 struct PreLayout {
@@ -129,7 +136,8 @@ preprocess_kernel(int n_seqs, int H, int64_t T_tot, const int32_t* __restrict__ 
                   float* __restrict__ beta, float* __restrict__ log_a) {
     using L = PreLayout<T, D, SCALAR>;
     constexpr int G = D / 8;                       // threads per token
-    constexpr int TPP = kThreads / G;              // tokens per pass
+    constexpr int kRun = run_for<D>();
+    constexpr int TPP = kThreads / G * kRun;       // tokens per pass
     constexpr int kPer = D * (int)sizeof(T) / 16;  // 16-byte pieces per raw row
     extern __shared__ __align__(16) uint8_t sm[];
     const int tid = threadIdx.x;
@@ -181,7 +189,7 @@ preprocess_kernel(int n_seqs, int H, int64_t T_tot, const int32_t* __restrict__ 
     cp_async_wait_all();
     __syncthreads();
 
-    // ---- outputs: thread (token r, channels c0 .. c0 + 7) -----------------------------
+    // ---- outputs: thread (tokens r0 .. r0 + kRun - 1, channels c0 .. c0 + 7) ----------
     const int cg = tid % G, c0 = 8 * cg;
     const T* X = reinterpret_cast<const T*>(sm + L::X);
     const float* Wt = reinterpret_cast<const float*>(sm + L::W);
@@ -189,62 +197,87 @@ preprocess_kernel(int n_seqs, int H, int64_t T_tot, const int32_t* __restrict__ 
     const float* Bv = reinterpret_cast<const float*>(sm + L::B);
     const float* Bias = reinterpret_cast<const float*>(sm + L::Bias);
 #pragma unroll 1
-    for (int r = tid / G; r < kTok; r += TPP) {
-        if (r >= ntok) break;                      // uniform over the token's lanes
-        const int64_t t = t0 + r;
-        // first token of t's sequence: cu[n] for the largest n with cu[n] <= t
+    for (int r0 = (tid / G) * kRun; r0 < kTok; r0 += TPP) {
+        if (r0 >= ntok) break;                     // uniform over the run's lanes
+        const int64_t t = t0 + r0;
+        // first token of t's sequence: cu[n] for the largest n with cu[n] <= t;
+        // a later token of the run starts a new sequence where cu[n + 1] is it
         int lo = 0, hi = n_seqs - 1, n = 0;
         while (lo <= hi) {
             const int mid = (lo + hi) >> 1;
             if ((int64_t)__ldg(cu + mid) <= t) { n = mid; lo = mid + 1; } else { hi = mid - 1; }
         }
-        const int64_t s = __ldg(cu + n);
-        float2 y[3][4];
+        int64_t su[kRun];
+        su[0] = __ldg(cu + n);
+        {
+            const int64_t nxt = __ldg(cu + n + 1);
+#pragma unroll
+            for (int u = 1; u < kRun; ++u) su[u] = nxt <= t + u ? nxt : su[u - 1];
+        }
+        // one tensor at a time: conv of the run's tokens, L2 norm (q, k), store
+        // (kRun rows of accumulators live, not 3 kRun; each tensor's rows go
+        // out before the next tensor is computed: 7 % faster at d 64 than
+        // storing all three at the end)
 #pragma unroll
         for (int tsr = 0; tsr < 3; ++tsr) {
+            float2 y[kRun][4];
+            // the run's raw rows, each unpacked once: staged row r0 + i is token t - 3 + i
+            float2 x[kRun + 3][4];
 #pragma unroll
-            for (int p = 0; p < 4; ++p) y[tsr][p] = make_float2(0.f, 0.f);
-            // taps 3 .. 0 on rows t, t - 1, t - 2, t - 3 (staged row r + j is token t - 3 + j)
+            for (int i = 0; i < kRun + 3; ++i)
+                Vec8<T>::load2(X + ((size_t)(tsr * (kTok + 3) + r0 + i)) * D + c0, x[i]);
+            // taps 3 .. 0 on rows t + u, ..., t + u - 3
 #pragma unroll
             for (int j = 3; j >= 0; --j) {
-                if (t - 3 + j < s) continue;
-                float2 x[4], w[4];
-                Vec8<T>::load2(X + ((size_t)(tsr * (kTok + 3) + r + j)) * D + c0, x);
+                float2 w[4];
                 load8_swz2(Wt + (size_t)(tsr * 4 + j) * D, cg, w);
 #pragma unroll
-                for (int p = 0; p < 4; ++p)
-                    y[tsr][p] = (j == 3) ? __fmul2_rn(w[p], x[p]) : __ffma2_rn(w[p], x[p], y[tsr][p]);
+                for (int u = 0; u < kRun; ++u) {
+                    if (j < 3 && t + u - 3 + j < su[u]) continue;
+#pragma unroll
+                    for (int p = 0; p < 4; ++p)
+                        y[u][p] = (j == 3) ? __fmul2_rn(w[p], x[u + j][p])
+                                           : __ffma2_rn(w[p], x[u + j][p], y[u][p]);
+                }
             }
-        }
+            if (tsr < 2) {
 #pragma unroll
-        for (int tsr = 0; tsr < 2; ++tsr) {
-            float2 s2 = __fmul2_rn(y[tsr][0], y[tsr][0]);
+                for (int u = 0; u < kRun; ++u) {
+                    float2 s2 = __fmul2_rn(y[u][0], y[u][0]);
 #pragma unroll
-            for (int p = 1; p < 4; ++p) s2 = __ffma2_rn(y[tsr][p], y[tsr][p], s2);
-            const float ss = group_sum<G>(s2.x + s2.y);
-            const float inv = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
-            const float2 inv2 = make_float2(inv, inv);
+                    for (int p = 1; p < 4; ++p) s2 = __ffma2_rn(y[u][p], y[u][p], s2);
+                    const float ss = group_sum<G>(s2.x + s2.y);
+                    const float inv = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
+                    const float2 inv2 = make_float2(inv, inv);
 #pragma unroll
-            for (int p = 0; p < 4; ++p) y[tsr][p] = __fmul2_rn(y[tsr][p], inv2);
-        }
-        const size_t row = ((size_t)t * H + h) * D + c0;
-        Vec8<T>::store2(q + row, y[0]);
-        Vec8<T>::store2(k + row, y[1]);
-        Vec8<T>::store2(v + row, y[2]);
-        if (SCALAR) {
-            if (cg == 0) log_a[(size_t)t * H + h] = log_sigmoid(Av[r] + Bias[0]);
-        } else {
-            float2 z[4], bz[4];
-            load8_swz2(Av + (size_t)r * D, cg, z);
-            load8_swz2(Bias, cg, bz);
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                const float2 zb = __fadd2_rn(z[p], bz[p]);
-                z[p] = make_float2(log_sigmoid(zb.x), log_sigmoid(zb.y));
+                    for (int p = 0; p < 4; ++p) y[u][p] = __fmul2_rn(y[u][p], inv2);
+                }
             }
-            Vec8<float>::store2(log_a + row, z);
+            T* dst = tsr == 0 ? q : (tsr == 1 ? k : v);
+#pragma unroll
+            for (int u = 0; u < kRun; ++u)
+                if (r0 + u < ntok) Vec8<T>::store2(dst + ((size_t)(t + u) * H + h) * D + c0, y[u]);
         }
-        if (cg == 0) beta[(size_t)t * H + h] = sigmoid(Bv[r]);
+#pragma unroll
+        for (int u = 0; u < kRun; ++u) {
+            const int r = r0 + u;
+            if (r >= ntok) break;
+            const size_t row = ((size_t)(t + u) * H + h) * D + c0;
+            if (SCALAR) {
+                if (cg == 0) log_a[(size_t)(t + u) * H + h] = log_sigmoid(Av[r] + Bias[0]);
+            } else {
+                float2 z[4], bz[4];
+                load8_swz2(Av + (size_t)r * D, cg, z);
+                load8_swz2(Bias, cg, bz);
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    const float2 zb = __fadd2_rn(z[p], bz[p]);
+                    z[p] = make_float2(log_sigmoid(zb.x), log_sigmoid(zb.y));
+                }
+                Vec8<float>::store2(log_a + row, z);
+            }
+            if (cg == 0) beta[(size_t)(t + u) * H + h] = sigmoid(Bv[r]);
+        }
     }
 }
 
