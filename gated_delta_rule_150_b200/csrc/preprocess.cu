@@ -18,8 +18,10 @@
 // stages, by 16-byte cp.async from every thread, the raw rows of x_q, x_k and
 // x_v for tokens [t0 - 3, t0 + kTok) (the three before the block for the
 // conv), the block's a_raw rows, beta_raw and the head's conv taps and gate
-// bias: about 45 KB per CTA at d 64, all in flight at once, so the kernel
-// keeps enough bytes moving to stream at HBM speed.  Then D / 8 threads own
+// bias: about 25 KB per CTA at d 64, all in flight at once, so the kernel
+// keeps enough bytes moving to stream at HBM speed, in four commit groups
+// (x_q, x_k, x_v, the gates) so that each tensor is computed as soon as its
+// rows have landed (11 % faster at d 128, 2 % at d 64).  Then D / 8 threads own
 // a token (eight channels each; at d 128 two consecutive tokens) and compute
 // its outputs from shared memory, one tensor after another; a tap that
 // reaches before the token's sequence start is skipped.  L2 norms
@@ -147,17 +149,34 @@ preprocess_kernel(int n_seqs, int H, int64_t T_tot, const int32_t* __restrict__ 
     const int64_t t0 = (int64_t)(blockIdx.x / (unsigned)H) * kTok;
     const int ntok = (int)(T_tot - t0 < kTok ? T_tot - t0 : kTok);
 
-    // ---- stage everything the block reads -----------------------------------------
-    for (int i = tid; i < 3 * (kTok + 3) * kPer; i += kThreads) {
-        const int tsr = i / ((kTok + 3) * kPer), rem = i % ((kTok + 3) * kPer);
-        const int row = rem / kPer, piece = rem % kPer;
-        const int64_t tok = t0 - 3 + row;
-        const bool in = tok >= 0 && tok < T_tot;
+    // ---- stage everything the block reads, in four commit groups -----------------
+    // (x_q with the taps, x_k, x_v, then a_raw, beta_raw and the bias), so
+    // that q is computed while x_k, x_v and the gates are still arriving
+    auto stage_x = [&](int tsr) {
         const T* x = tsr == 0 ? xq : (tsr == 1 ? xk : xv);
-        const T* src = x + ((in ? tok : 0) * H + h) * (int64_t)D;
-        cp_async16(sm + L::X + ((size_t)(tsr * (kTok + 3) + row) * D) * sizeof(T) + 16 * piece,
-                   reinterpret_cast<const uint8_t*>(src) + 16 * piece, in ? 16u : 0u);
+        for (int i = tid; i < (kTok + 3) * kPer; i += kThreads) {
+            const int row = i / kPer, piece = i % kPer;
+            const int64_t tok = t0 - 3 + row;
+            const bool in = tok >= 0 && tok < T_tot;
+            const T* src = x + ((in ? tok : 0) * H + h) * (int64_t)D;
+            cp_async16(sm + L::X + ((size_t)(tsr * (kTok + 3) + row) * D) * sizeof(T) + 16 * piece,
+                       reinterpret_cast<const uint8_t*>(src) + 16 * piece, in ? 16u : 0u);
+        }
+    };
+    stage_x(0);
+    // taps transposed to [tensor][tap][channel] (16-byte words swizzled as
+    // above), so that a thread's eight channels of one tap are two 16-byte words
+    for (int i = tid; i < 3 * 4 * D; i += kThreads) {
+        const int tsr = i / (4 * D), j = (i / D) % 4, c = i % D;
+        const float* w = tsr == 0 ? wq : (tsr == 1 ? wk : wv);
+        reinterpret_cast<float*>(sm + L::W)[(tsr * 4 + j) * D + 4 * swz_word(c / 4) + c % 4] =
+            __ldg(w + ((size_t)h * D + c) * 4 + j);
     }
+    cp_async_commit();
+    stage_x(1);
+    cp_async_commit();
+    stage_x(2);
+    cp_async_commit();
     if (SCALAR) {
         for (int i = tid; i < kTok; i += kThreads)
             cp_async4(sm + L::A + 4 * i, a_raw + ((i < ntok ? t0 + i : 0) * H + h), i < ntok ? 4u : 0u);
@@ -171,14 +190,6 @@ preprocess_kernel(int n_seqs, int H, int64_t T_tot, const int32_t* __restrict__ 
     }
     for (int i = tid; i < kTok; i += kThreads)
         cp_async4(sm + L::B + 4 * i, beta_raw + ((i < ntok ? t0 + i : 0) * H + h), i < ntok ? 4u : 0u);
-    // taps transposed to [tensor][tap][channel] (16-byte words swizzled as
-    // above), so that a thread's eight channels of one tap are two 16-byte words
-    for (int i = tid; i < 3 * 4 * D; i += kThreads) {
-        const int tsr = i / (4 * D), j = (i / D) % 4, c = i % D;
-        const float* w = tsr == 0 ? wq : (tsr == 1 ? wk : wv);
-        reinterpret_cast<float*>(sm + L::W)[(tsr * 4 + j) * D + 4 * swz_word(c / 4) + c % 4] =
-            __ldg(w + ((size_t)h * D + c) * 4 + j);
-    }
     if (SCALAR) {
         if (tid == 0) cp_async4(sm + L::Bias, a_bias + h, 4u);
     } else {
@@ -186,20 +197,20 @@ preprocess_kernel(int n_seqs, int H, int64_t T_tot, const int32_t* __restrict__ 
             cp_async16(sm + L::Bias + 16 * swz_word(i), a_bias + (size_t)h * D + 4 * i, 16u);
     }
     cp_async_commit();
-    cp_async_wait_all();
-    __syncthreads();
 
     // ---- outputs: thread (tokens r0 .. r0 + kRun - 1, channels c0 .. c0 + 7) ----------
+    static_assert(TPP == kTok, "one pass over the block's tokens");
     const int cg = tid % G, c0 = 8 * cg;
     const T* X = reinterpret_cast<const T*>(sm + L::X);
     const float* Wt = reinterpret_cast<const float*>(sm + L::W);
     const float* Av = reinterpret_cast<const float*>(sm + L::A);
     const float* Bv = reinterpret_cast<const float*>(sm + L::B);
     const float* Bias = reinterpret_cast<const float*>(sm + L::Bias);
-#pragma unroll 1
-    for (int r0 = (tid / G) * kRun; r0 < kTok; r0 += TPP) {
-        if (r0 >= ntok) break;                     // uniform over the run's lanes
-        const int64_t t = t0 + r0;
+    const int r0 = (tid / G) * kRun;
+    const bool act = r0 < ntok;                    // uniform over the run's lanes
+    const int64_t t = t0 + r0;
+    int64_t su[kRun];
+    if (act) {
         // first token of t's sequence: cu[n] for the largest n with cu[n] <= t;
         // a later token of the run starts a new sequence where cu[n + 1] is it
         int lo = 0, hi = n_seqs - 1, n = 0;
@@ -207,77 +218,80 @@ preprocess_kernel(int n_seqs, int H, int64_t T_tot, const int32_t* __restrict__ 
             const int mid = (lo + hi) >> 1;
             if ((int64_t)__ldg(cu + mid) <= t) { n = mid; lo = mid + 1; } else { hi = mid - 1; }
         }
-        int64_t su[kRun];
         su[0] = __ldg(cu + n);
-        {
-            const int64_t nxt = __ldg(cu + n + 1);
+        const int64_t nxt = __ldg(cu + n + 1);
 #pragma unroll
-            for (int u = 1; u < kRun; ++u) su[u] = nxt <= t + u ? nxt : su[u - 1];
-        }
-        // one tensor at a time: conv of the run's tokens, L2 norm (q, k), store
-        // (kRun rows of accumulators live, not 3 kRun; each tensor's rows go
-        // out before the next tensor is computed: 7 % faster at d 64 than
-        // storing all three at the end)
+        for (int u = 1; u < kRun; ++u) su[u] = nxt <= t + u ? nxt : su[u - 1];
+    }
+    // one tensor at a time, each as soon as its rows have landed: conv of the
+    // run's tokens, L2 norm (q, k), store
 #pragma unroll
-        for (int tsr = 0; tsr < 3; ++tsr) {
-            float2 y[kRun][4];
-            // the run's raw rows, each unpacked once: staged row r0 + i is token t - 3 + i
-            float2 x[kRun + 3][4];
+    for (int tsr = 0; tsr < 3; ++tsr) {
+        if (tsr == 0) cp_async_wait_group<3>();
+        else if (tsr == 1) cp_async_wait_group<2>();
+        else cp_async_wait_group<1>();
+        __syncthreads();
+        if (!act) continue;
+        float2 y[kRun][4];
+        // the run's raw rows, each unpacked once: staged row r0 + i is token t - 3 + i
+        float2 x[kRun + 3][4];
 #pragma unroll
-            for (int i = 0; i < kRun + 3; ++i)
-                Vec8<T>::load2(X + ((size_t)(tsr * (kTok + 3) + r0 + i)) * D + c0, x[i]);
-            // taps 3 .. 0 on rows t + u, ..., t + u - 3
+        for (int i = 0; i < kRun + 3; ++i)
+            Vec8<T>::load2(X + ((size_t)(tsr * (kTok + 3) + r0 + i)) * D + c0, x[i]);
+        // taps 3 .. 0 on rows t + u, ..., t + u - 3
 #pragma unroll
-            for (int j = 3; j >= 0; --j) {
-                float2 w[4];
-                load8_swz2(Wt + (size_t)(tsr * 4 + j) * D, cg, w);
+        for (int j = 3; j >= 0; --j) {
+            float2 w[4];
+            load8_swz2(Wt + (size_t)(tsr * 4 + j) * D, cg, w);
 #pragma unroll
-                for (int u = 0; u < kRun; ++u) {
-                    if (j < 3 && t + u - 3 + j < su[u]) continue;
+            for (int u = 0; u < kRun; ++u) {
+                if (j < 3 && t + u - 3 + j < su[u]) continue;
 #pragma unroll
-                    for (int p = 0; p < 4; ++p)
-                        y[u][p] = (j == 3) ? __fmul2_rn(w[p], x[u + j][p])
-                                           : __ffma2_rn(w[p], x[u + j][p], y[u][p]);
-                }
+                for (int p = 0; p < 4; ++p)
+                    y[u][p] = (j == 3) ? __fmul2_rn(w[p], x[u + j][p])
+                                       : __ffma2_rn(w[p], x[u + j][p], y[u][p]);
             }
-            if (tsr < 2) {
-#pragma unroll
-                for (int u = 0; u < kRun; ++u) {
-                    float2 s2 = __fmul2_rn(y[u][0], y[u][0]);
-#pragma unroll
-                    for (int p = 1; p < 4; ++p) s2 = __ffma2_rn(y[u][p], y[u][p], s2);
-                    const float ss = group_sum<G>(s2.x + s2.y);
-                    const float inv = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
-                    const float2 inv2 = make_float2(inv, inv);
-#pragma unroll
-                    for (int p = 0; p < 4; ++p) y[u][p] = __fmul2_rn(y[u][p], inv2);
-                }
-            }
-            T* dst = tsr == 0 ? q : (tsr == 1 ? k : v);
-#pragma unroll
-            for (int u = 0; u < kRun; ++u)
-                if (r0 + u < ntok) Vec8<T>::store2(dst + ((size_t)(t + u) * H + h) * D + c0, y[u]);
         }
+        if (tsr < 2) {
 #pragma unroll
-        for (int u = 0; u < kRun; ++u) {
-            const int r = r0 + u;
-            if (r >= ntok) break;
-            const size_t row = ((size_t)(t + u) * H + h) * D + c0;
-            if (SCALAR) {
-                if (cg == 0) log_a[(size_t)(t + u) * H + h] = log_sigmoid(Av[r] + Bias[0]);
-            } else {
-                float2 z[4], bz[4];
-                load8_swz2(Av + (size_t)r * D, cg, z);
-                load8_swz2(Bias, cg, bz);
+            for (int u = 0; u < kRun; ++u) {
+                float2 s2 = __fmul2_rn(y[u][0], y[u][0]);
 #pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    const float2 zb = __fadd2_rn(z[p], bz[p]);
-                    z[p] = make_float2(log_sigmoid(zb.x), log_sigmoid(zb.y));
-                }
-                Vec8<float>::store2(log_a + row, z);
+                for (int p = 1; p < 4; ++p) s2 = __ffma2_rn(y[u][p], y[u][p], s2);
+                const float ss = group_sum<G>(s2.x + s2.y);
+                const float inv = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
+                const float2 inv2 = make_float2(inv, inv);
+#pragma unroll
+                for (int p = 0; p < 4; ++p) y[u][p] = __fmul2_rn(y[u][p], inv2);
             }
-            if (cg == 0) beta[(size_t)(t + u) * H + h] = sigmoid(Bv[r]);
         }
+        T* dst = tsr == 0 ? q : (tsr == 1 ? k : v);
+#pragma unroll
+        for (int u = 0; u < kRun; ++u)
+            if (r0 + u < ntok) Vec8<T>::store2(dst + ((size_t)(t + u) * H + h) * D + c0, y[u]);
+    }
+    cp_async_wait_group<0>();
+    __syncthreads();
+    if (!act) return;
+#pragma unroll
+    for (int u = 0; u < kRun; ++u) {
+        const int r = r0 + u;
+        if (r >= ntok) break;
+        const size_t row = ((size_t)(t + u) * H + h) * D + c0;
+        if (SCALAR) {
+            if (cg == 0) log_a[(size_t)(t + u) * H + h] = log_sigmoid(Av[r] + Bias[0]);
+        } else {
+            float2 z[4], bz[4];
+            load8_swz2(Av + (size_t)r * D, cg, z);
+            load8_swz2(Bias, cg, bz);
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                const float2 zb = __fadd2_rn(z[p], bz[p]);
+                z[p] = make_float2(log_sigmoid(zb.x), log_sigmoid(zb.y));
+            }
+            Vec8<float>::store2(log_a + row, z);
+        }
+        if (cg == 0) beta[(size_t)(t + u) * H + h] = sigmoid(Bv[r]);
     }
 }
 
