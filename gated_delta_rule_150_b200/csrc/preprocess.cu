@@ -165,12 +165,14 @@ preprocess_kernel(int n_seqs, int H, int64_t T_tot, const int32_t* __restrict__ 
     };
     stage_x(0);
     // taps transposed to [tensor][tap][channel] (16-byte words swizzled as
-    // above), so that a thread's eight channels of one tap are two 16-byte words
+    // above), so that a thread's eight channels of one tap are two 16-byte
+    // words; copied element by element by 4-byte cp.async, in flight with the
+    // rows (5 % faster at d 64 than loading them into registers and storing)
     for (int i = tid; i < 3 * 4 * D; i += kThreads) {
         const int tsr = i / (4 * D), j = (i / D) % 4, c = i % D;
         const float* w = tsr == 0 ? wq : (tsr == 1 ? wk : wv);
-        reinterpret_cast<float*>(sm + L::W)[(tsr * 4 + j) * D + 4 * swz_word(c / 4) + c % 4] =
-            __ldg(w + ((size_t)h * D + c) * 4 + j);
+        cp_async4(sm + L::W + 4 * ((tsr * 4 + j) * D + 4 * swz_word(c / 4) + c % 4),
+                  w + ((size_t)h * D + c) * 4 + j, 4u);
     }
     cp_async_commit();
     stage_x(1);
