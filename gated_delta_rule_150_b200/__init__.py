@@ -22,6 +22,7 @@ import torch
 __all__ = ["PrefillArgs", "PreparedPrefill", "prefill", "kernel_count", "decode_step",
            "decode_draft", "decode_accept", "PreprocessArgs", "preprocess", "Projections",
            "prefill_from_projections", "cumdecay", "chunk_factors", "workspace_size",
+           "projections_workspace_size",
            "snapshot_count", "snapshot_offsets", "snapshot_offload", "prefill_status", "lib", "GdrError", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_build", "libgdr.so")
@@ -97,6 +98,8 @@ def lib():
             L.gdr_version.restype = i
             L.gdr_prefill_workspace_size.restype = ctypes.c_size_t
             L.gdr_prefill_workspace_size.argtypes = [i, i, i, i, i64, i]
+            L.gdr_prefill_from_projections_workspace_size.restype = ctypes.c_size_t
+            L.gdr_prefill_from_projections_workspace_size.argtypes = [i, i, i, i64, i]
             L.gdr_prefill_kernel_count.restype = i
             L.gdr_prefill_kernel_count.argtypes = [i, i, i, i, i64, i]
             L.gdr_snapshot_count.restype = i64
@@ -248,6 +251,14 @@ def _host_cu(cu_seqlens, cu_seqlens_host):
 def workspace_size(n_seqs, n_heads, d_k, d_v, total_tokens, scalar_decay=False) -> int:
     return int(lib().gdr_prefill_workspace_size(n_seqs, n_heads, d_k, d_v, total_tokens,
                                                 int(bool(scalar_decay))))
+
+
+def projections_workspace_size(n_seqs, n_heads, d, total_tokens, scalar_decay=False) -> int:
+    """Workspace of ``prefill_from_projections`` with room for the staged
+    activations (larger than ``workspace_size`` only at d 128 with a
+    per-channel gate)."""
+    return int(lib().gdr_prefill_from_projections_workspace_size(n_seqs, n_heads, d, total_tokens,
+                                                                 int(bool(scalar_decay))))
 
 
 def kernel_count(n_seqs, n_heads, d_k, d_v, total_tokens, scalar_decay=False) -> int:
@@ -616,9 +627,11 @@ def prefill_from_projections(xq, xk, xv, conv_q, conv_k, conv_v, beta_raw, a_raw
                              norm_eps=1e-6):
     """``preprocess`` and ``prefill`` in one: the input activations (conv-4, L2
     norm of q and k, beta and log-decay gates) are applied inside the
-    prefill's first kernel.  Raw projections as for ``preprocess`` (bf16);
-    the other arguments and the result (o, final_state, snapshots) as for
-    ``prefill``."""
+    prefill's first kernel, or, at d 128 with a per-channel gate and a
+    workspace of ``projections_workspace_size`` bytes (the default), by their
+    own kernel into the workspace (faster there).  Raw projections as for
+    ``preprocess`` (bf16); the other arguments and the result (o,
+    final_state, snapshots) as for ``prefill``."""
     if xq.dtype != torch.bfloat16 or xk.dtype != xq.dtype or xv.dtype != xq.dtype:
         raise TypeError("the fused path takes bf16 projections")
     _expect_dim(xq, 3, "xq")
@@ -648,8 +661,8 @@ def prefill_from_projections(xq, xk, xv, conv_q, conv_k, conv_v, beta_raw, a_raw
         ns = snapshot_count(_host_cu(cu_seqlens, cu_seqlens_host), snap_interval)
         snapshots = torch.empty(max(ns, 1), H, d, d, dtype=torch.float32, device=dev)[:ns]
     if workspace is None:
-        workspace = torch.empty(workspace_size(n, H, d, d, T, scalar_decay), dtype=torch.uint8,
-                                device=dev)
+        workspace = torch.empty(projections_workspace_size(n, H, d, T, scalar_decay),
+                                dtype=torch.uint8, device=dev)
     snap_arg = snapshots if (snap_interval and snapshots is not None and snapshots.numel()) else None
     if snap_interval and snap_arg is None:
         snap_arg = final_state

@@ -156,6 +156,30 @@ gdr_status gdr_snapshot_offsets(const int32_t* host_cu, int n_seqs, int snap_int
     return GDR_OK;
 }
 
+namespace {
+
+// The activations gdr_prefill_from_projections stages in the workspace when
+// it runs them as their own kernel: only at d 128 with a per-channel gate,
+// where that chain measured faster than the fused first stage.
+bool staged_activations(int d, int scalar_decay) { return d == 128 && !scalar_decay; }
+
+size_t align256(size_t x) { return (x + 255u) & ~(size_t)255u; }
+
+// [q | k | v] bf16, beta fp32, log a fp32, each 256-byte aligned
+size_t activation_bytes(int n_heads, int d, int64_t total_tokens) {
+    const size_t th = (size_t)total_tokens * (size_t)n_heads;
+    return 3 * align256(th * d * 2) + align256(th * 4) + align256(th * d * 4);
+}
+
+}  // namespace
+
+size_t gdr_prefill_from_projections_workspace_size(int n_seqs, int n_heads, int d,
+                                                   int64_t total_tokens, int scalar_decay) {
+    const size_t base = gdr_prefill_workspace_size(n_seqs, n_heads, d, d, total_tokens, scalar_decay);
+    if (base == 0 || !staged_activations(d, scalar_decay)) return base;
+    return align256(base) + activation_bytes(n_heads, d, total_tokens);
+}
+
 gdr_status gdr_prefill_from_projections(const gdr_prefill_args* a, const gdr_projections* p,
                                         void* stream) {
     if (!a || !p) return GDR_ERR_INVALID_ARG;
@@ -182,6 +206,47 @@ gdr_status gdr_prefill_from_projections(const gdr_prefill_args* a, const gdr_pro
     s = check_workspace(&r, &lay);
     if (s != GDR_OK) return s;
     if (r.n_seqs == 0) return GDR_OK;
+    // with room for the activations (d 128, per-channel gate): gdr_preprocess
+    // into the workspace's tail, then gdr_prefill from there
+    if (staged_activations(r.d_k, r.scalar_decay) && r.total_tokens > 0 &&
+        r.workspace_bytes >= gdr_prefill_from_projections_workspace_size(
+                                 r.n_seqs, r.n_heads, r.d_k, r.total_tokens, r.scalar_decay)) {
+        const size_t th = (size_t)r.total_tokens * (size_t)r.n_heads;
+        uint8_t* act = static_cast<uint8_t*>(r.workspace) + align256(lay.total);
+        gdr_preprocess_args pa;
+        memset(&pa, 0, sizeof(pa));
+        pa.n_seqs = r.n_seqs;
+        pa.n_heads = r.n_heads;
+        pa.d = r.d_k;
+        pa.total_tokens = r.total_tokens;
+        pa.cu_seqlens = r.cu_seqlens;
+        pa.io_dtype = GDR_BF16;
+        pa.xq = p->xq;
+        pa.xk = p->xk;
+        pa.xv = p->xv;
+        pa.conv_q = p->conv_q;
+        pa.conv_k = p->conv_k;
+        pa.conv_v = p->conv_v;
+        pa.beta_raw = p->beta_raw;
+        pa.a_raw = p->a_raw;
+        pa.a_bias = p->a_bias;
+        pa.scalar_decay = r.scalar_decay;
+        const size_t qkv = align256(th * r.d_k * 2);
+        pa.q = act;
+        pa.k = act + qkv;
+        pa.v = act + 2 * qkv;
+        pa.beta = reinterpret_cast<float*>(act + 3 * qkv);
+        pa.log_a = reinterpret_cast<float*>(act + 3 * qkv + align256(th * 4));
+        s = gdr_preprocess(&pa, stream);
+        if (s != GDR_OK) return s;
+        gdr_prefill_args c = *a;
+        c.q = pa.q;
+        c.k = pa.k;
+        c.v = pa.v;
+        c.beta = pa.beta;
+        c.log_a = pa.log_a;
+        return gdr_prefill(&c, stream);
+    }
     if (r.snap_interval > 0) {
         s = kernel_address(a->snapshots, reinterpret_cast<void**>(&r.snapshots));
         if (s != GDR_OK) return s;

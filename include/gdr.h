@@ -418,16 +418,30 @@ typedef struct {
  * gdr_prefill, with its q, k, v, beta and log_a ignored (may be NULL);
  * qkv_dtype must be GDR_BF16 and d_k == d_v (64 or 128), else
  * GDR_ERR_UNSUPPORTED.  xq, xk, xv, the conv taps and (per-channel gate)
- * a_raw and a_bias must be 16-byte aligned.  Outputs, workspace (same size as
- * gdr_prefill's) and errors as for gdr_prefill.
- * Speed: at d 64 this call is faster than gdr_preprocess followed by
- * gdr_prefill (about 8 % on a B200); at d 128, where the prefill's first
- * stage is bound by its per-chunk latency, the two calls are about 12 %
- * faster and this one saves the activations' memory (1284 bytes per token
- * and head).
+ * a_raw and a_bias must be 16-byte aligned.  Outputs and errors as for
+ * gdr_prefill.  Workspace: at least gdr_prefill_workspace_size(...) bytes,
+ * with which the activations are applied inside the prefill's first kernel.
+ * At d 128 with a per-channel gate that first stage is bound by its
+ * per-chunk latency and the activations lengthen it more than an HBM round
+ * trip of them costs: given gdr_prefill_from_projections_workspace_size(...)
+ * bytes, the call runs gdr_preprocess into the workspace's tail and then
+ * gdr_prefill (about 12 % faster on a B200; 1284 more bytes of workspace
+ * per token and head).  At d 64, or with a scalar gate, both sizes are the
+ * same and the fused first stage runs (about 8 % faster than the two calls
+ * at d 64).
  */
 gdr_status gdr_prefill_from_projections(const gdr_prefill_args* args, const gdr_projections* proj,
                                         void* stream);
+
+/*
+ * Workspace bytes with which gdr_prefill_from_projections stages the
+ * activations (see above): gdr_prefill_workspace_size(n_seqs, n_heads, d, d,
+ * total_tokens, scalar_decay), plus, at d == 128 with scalar_decay == 0,
+ * room for q, k, v (bf16), beta and log a (fp32) of every token and head.
+ * 0 for invalid sizes, as gdr_prefill_workspace_size.
+ */
+size_t gdr_prefill_from_projections_workspace_size(int n_seqs, int n_heads, int d,
+                                                   int64_t total_tokens, int scalar_decay);
 
 /* ------------------------------------------------------------------------
  * Speculative decoding with rollback ("Modele hybrydowe", section "Co stan

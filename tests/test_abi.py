@@ -164,6 +164,21 @@ def test_workspace_size_grows_with_tokens(L):
     assert gdr.kernel_count(32, 32, 128, 64, 278000) == 2 + 1
 
 
+def test_projections_workspace_size(L):
+    """The staged-activation workspace: larger only at d 128 with a per-channel
+    gate, by q, k, v (bf16), beta and log a (fp32) of every token-head, each
+    part rounded up to 256 bytes."""
+    for d, scalar in ((64, False), (64, True), (128, True)):
+        assert gdr.projections_workspace_size(1, 14, d, 8192, scalar) == \
+            gdr.workspace_size(1, 14, d, d, 8192, scalar)
+    base = gdr.workspace_size(2, 14, 128, 128, 8191)
+    up = lambda x: (x + 255) // 256 * 256
+    th = 8191 * 14
+    assert gdr.projections_workspace_size(2, 14, 128, 8191) == \
+        up(base) + 3 * up(th * 128 * 2) + up(th * 4) + up(th * 128 * 4)
+    assert gdr.projections_workspace_size(1, 14, 96, 8192) == 0
+
+
 def test_snapshot_count_matches_oracle(L):
     import oracle
     for lengths, iv in (([4096, 100, 8192, 0, 4095], 4096), ([64, 128, 1], 64), ([5, 7], 0)):

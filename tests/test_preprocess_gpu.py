@@ -99,7 +99,7 @@ def test_preprocess_no_tokens_is_noop():
     assert out["q"].shape == (0, 2, 64)
 
 
-def _fused_vs_chain(w, lengths, snap=0, init=False, steep=None):
+def _fused_vs_chain(w, lengths, snap=0, init=False, steep=None, minimal_ws=False):
     """The fused prefill from raw projections against (a) the oracle's prefill
     of the oracle's activations (cast to bf16) at the prefill bound 2e-2 max
     |ref|, and (b) the two-kernel chain preprocess -> prefill.  ``steep``:
@@ -121,7 +121,12 @@ def _fused_vs_chain(w, lengths, snap=0, init=False, steep=None):
     ini = None if init_state is None else init_state.cuda()
     kw = dict(scalar_decay=w.scalar_decay, init_state=ini, snap_interval=snap,
               cu_seqlens_host=inp["cu_seqlens"])
-    o, fin, snaps = gdr.prefill_from_projections(*(d[a] for a in ARGS), **kw)
+    ws = None
+    if minimal_ws:
+        # gdr_prefill's workspace: the fused first stage, also at d 128
+        ws = torch.empty(gdr.workspace_size(n, H, dd, dd, inp["xq"].shape[0], w.scalar_decay),
+                         dtype=torch.uint8, device="cuda")
+    o, fin, snaps = gdr.prefill_from_projections(*(d[a] for a in ARGS), workspace=ws, **kw)
     act = gdr.preprocess(*(d[a] for a in ARGS), scalar_decay=w.scalar_decay)
     o2, fin2, snaps2 = gdr.prefill(act["q"], act["k"], act["v"], act["beta"], act["log_a"],
                                    d["cu_seqlens"], **kw)
@@ -143,14 +148,16 @@ def _fused_vs_chain(w, lengths, snap=0, init=False, steep=None):
         assert err <= 2e-2, f"fused vs chain {name}: {err:.3e}"
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d,minimal_ws", [(64, False), (128, False), (128, True)])
 @pytest.mark.parametrize("scalar", [False, True])
-def test_fused_prefill_from_projections(d, scalar):
+def test_fused_prefill_from_projections(d, minimal_ws, scalar):
     """Ragged sequences (1, 2, 3 tokens, empty, chunk-crossing lengths),
     initial states and snapshots: the conv's history restarts at each
-    sequence start, including inside a chunk, and crosses chunk boundaries."""
+    sequence start, including inside a chunk, and crosses chunk boundaries.
+    At d 128 with a per-channel gate both the staged activations (default
+    workspace) and the fused first stage (gdr_prefill's workspace)."""
     w = wl.shrink(wl.PREPROCESS, n_heads=3, d_k=d, d_v=d, scalar_decay=scalar, seed=1110)
-    _fused_vs_chain(w, [1, 2, 3, 0, 130, 64, 200, 5], snap=64, init=True)
+    _fused_vs_chain(w, [1, 2, 3, 0, 130, 64, 200, 5], snap=64, init=True, minimal_ws=minimal_ws)
 
 
 def test_fused_prefill_graft_layer_shape():
@@ -158,9 +165,9 @@ def test_fused_prefill_graft_layer_shape():
     _fused_vs_chain(wl.PREPROCESS, None)
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d,minimal_ws", [(64, False), (128, False), (128, True)])
 @pytest.mark.parametrize("scalar", [False, True])
-def test_fused_prefill_steep_decay(d, scalar):
+def test_fused_prefill_steep_decay(d, minimal_ws, scalar):
     """Decays below the factored range (log a < -10) inside the fused path,
     on enough chunks (6 heads x 64 chunks) that most CTAs take a second item,
     whose decay is scanned during the first item's solve: chunk j holds one
@@ -168,4 +175,4 @@ def test_fused_prefill_steep_decay(d, scalar):
     so that each row range of that scan meets one, next to chunks without."""
     w = wl.shrink(wl.PREPROCESS, n_heads=6, d_k=d, d_v=d, scalar_decay=scalar, seed=1111)
     toks = [64 * j + (3, 25, 47)[j % 4] for j in range(64) if j % 4 != 3]
-    _fused_vs_chain(w, [4096], steep=(toks, [1, d // 2 + 3, d - 1]))
+    _fused_vs_chain(w, [4096], steep=(toks, [1, d // 2 + 3, d - 1]), minimal_ws=minimal_ws)
