@@ -176,3 +176,36 @@ def test_fused_prefill_steep_decay(d, minimal_ws, scalar):
     w = wl.shrink(wl.PREPROCESS, n_heads=6, d_k=d, d_v=d, scalar_decay=scalar, seed=1111)
     toks = [64 * j + (3, 25, 47)[j % 4] for j in range(64) if j % 4 != 3]
     _fused_vs_chain(w, [4096], steep=(toks, [1, d // 2 + 3, d - 1]), minimal_ws=minimal_ws)
+
+
+@pytest.mark.parametrize("d,minimal_ws", [(64, False), (128, False), (128, True)])
+def test_prefill_from_projections_output_epilogue(d, minimal_ws):
+    """The output epilogue (RMSNorm and sigmoid gate) through the raw-projection
+    path, fused first stage and staged activations alike, against the oracle's
+    epilogue of the oracle's prefill of the oracle's activations."""
+    gdr = _gdr()
+    w = wl.shrink(wl.PREPROCESS, n_heads=3, d_k=d, d_v=d, seed=1112)
+    inp = wl.make_preprocess_inputs(w, lengths=[300, 0, 77, 130])
+    dd = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in inp.items()}
+    T, H = inp["xq"].shape[0], w.n_heads
+    n = len(inp["lengths"])
+    g = wl.make_output_gate(T, H, d, torch.bfloat16, seed=91 + d)
+    ws = None
+    if minimal_ws:
+        ws = torch.empty(gdr.workspace_size(n, H, d, d, T), dtype=torch.uint8, device="cuda")
+    y = torch.full((T, H, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    y, fin, _ = gdr.prefill_from_projections(*(dd[a] for a in ARGS), cu_seqlens_host=inp["cu_seqlens"],
+                                             out=y, workspace=ws, gate_raw=g["gate_raw"].cuda(),
+                                             norm_weight=g["norm_weight"].cuda(), norm_eps=1e-6)
+    torch.cuda.synchronize()
+    assert not torch.isnan(y).any()
+    ref_act = oracle.preprocess(*(inp[a] for a in ARGS))
+    cast = {m: torch.from_numpy(ref_act[m]).to(torch.bfloat16) for m in ("q", "k", "v")}
+    ref = oracle.prefill(cast["q"], cast["k"], cast["v"], ref_act["beta"], ref_act["log_a"],
+                         inp["cu_seqlens"])
+    y_ref = oracle.output_epilogue(ref["o"], g["gate_raw"], g["norm_weight"], 1e-6)
+    y_ref = np.asarray(y_ref, dtype=np.float64)
+    err = np.abs(y.double().cpu().numpy() - y_ref).max() / np.abs(y_ref).max()
+    assert err <= 2e-2, f"gated o: {err:.3e}"
+    err = np.abs(fin.double().cpu().numpy() - ref["final_state"]).max() / np.abs(ref["final_state"]).max()
+    assert err <= 2e-2, f"final state: {err:.3e}"
