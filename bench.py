@@ -635,6 +635,8 @@ def bench_prefill_workload(gdr, w, stream, pk, rank, args):
            "roofline": dominant_roofline(ps, st, pk),
            "path_roofline": roofline_obj(ps.bytes, ps.flops, ms, pk), "tokens": ps.T,
            "sequences": ps.n, "l2": ps.l2, "steps": n}
+    if w is wl.GRAFT_LAYER or w is wl.TINY_KDA:
+        res["graph_replay"] = bench_graph(ps, stream, ms, n)
     if w is wl.GRAFT_LAYER:
         res["output_epilogue"] = bench_epilogue(gdr, ps, stream, ms, n)
     if w.snap_interval:
@@ -642,6 +644,29 @@ def bench_prefill_workload(gdr, w, stream, pk, rank, args):
     del ps
     torch.cuda.empty_cache()
     return res
+
+
+def bench_graph(ps, stream, ms_eager, n):
+    """The same steps replayed from CUDA graphs (one captured per input set:
+    the prefill's launches and their programmatic-launch edges recorded once,
+    so a step costs one graph launch on the host)."""
+    try:
+        graphs = []
+        for i in range(len(ps.sets)):
+            ps.step(i)                                  # outside capture first
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                ps.step(i)
+            graphs.append(g)
+        for i in range(2):
+            graphs[i % len(graphs)].replay()
+        ms = timed(lambda i: graphs[i % len(graphs)].replay(), n, stream)
+        del graphs
+        return {"ms_per_step": round(ms, 4), "eager_ms_per_step": round(ms_eager, 4),
+                "graphs": len(ps.sets)}
+    except Exception as e:                              # reported, not fatal
+        return {"error": str(e)[:200]}
 
 
 def bench_epilogue(gdr, ps, stream, ms_plain, n):
